@@ -1,0 +1,376 @@
+"""Pins of the fp64 oracle against facts fixed by the pages and by mathematics (CPU only).
+
+Each test pins one part of the oracle to something other than itself: a closed form, a special
+case that reduces to a library routine (torch's fp64 softmax attention, numpy's sort), brute-force
+enumeration, an invariant of the definition, or the counts the pages print.  A plausible slip in the
+oracle (a dropped term, a wrong window offset or sign, a transposed operand, a wrong tie-break)
+breaks at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+SEED = 77
+
+
+def bf(seed, tensor, seq, rows, cols, scale=1.0):
+    return synth.bf16_normal(seed, tensor, seq, cols, 0, rows, scale=scale)
+
+
+def f64(u16):
+    return synth.bf16_to_f64(u16)
+
+
+ONE_BF16 = np.uint16(0x3F80)
+
+
+# ---------------------------------------------------------------- compressor (a1 / a2)
+
+@pytest.mark.parametrize("m,win", [(4, 8), (16, 16), (128, 128), (4, 4)])
+def test_equal_logits_give_window_mean(m, win):
+    """Equal logits and an offset-independent bias make the softmax uniform: entry = window mean."""
+    d, L = 16, 8 * m + 3
+    x = bf(SEED, synth.X, 0, L, d)
+    logit = np.full((L, d), np.uint16(0x4040), dtype=np.uint16)  # 3.0 everywhere
+    colbias = synth.f32_normal(SEED, synth.BIAS_C, 0, d, 0, 1)
+    bias = np.repeat(colbias, win, axis=0)  # same bias at every offset of a channel
+    js = np.arange(L // m)
+    E, _ = oracle.compress(x, logit, bias, None, L, m, win, js)
+    xf = f64(x)
+    for j in js:
+        t0, t1 = max(0, m * j - (win - m)), m * j + m
+        np.testing.assert_allclose(E[j], xf[t0:t1].mean(axis=0), rtol=1e-14, atol=1e-15)
+
+
+def test_clipped_first_window_is_four_token_mean():
+    """Entry 0 of the overlapping CSA window keeps only its 4 existing tokens [0, 4)."""
+    d, L = 8, 16
+    x = bf(SEED, synth.X, 1, L, d)
+    logit = np.zeros((L, d), dtype=np.uint16)
+    bias = np.zeros((8, d), dtype=np.float32)
+    E, _ = oracle.compress(x, logit, bias, None, L, 4, 8, [0, 1])
+    np.testing.assert_allclose(E[0], f64(x)[0:4].mean(0), rtol=1e-15)
+    np.testing.assert_allclose(E[1], f64(x)[0:8].mean(0), rtol=1e-15)
+
+
+@pytest.mark.parametrize("m,win", [(4, 8), (128, 128)])
+def test_weights_sum_to_one_per_channel(m, win):
+    d, L = 32, 3 * m + 1
+    logit = bf(SEED, synth.A, 0, L, d)
+    bias = synth.f32_normal(SEED, synth.BIAS_C, 0, d, 0, win, scale=0.5)
+    js = np.arange(L // m)
+    Wt = oracle.compress_weights(logit, bias, L, m, win, js)
+    eps = win * np.finfo(np.float64).eps  # n-term summation bound
+    np.testing.assert_allclose(Wt.sum(axis=1), 1.0, rtol=0, atol=eps)
+    assert (Wt >= 0).all()
+    # all-ones latent: the weighted sum reproduces the weight total, 1
+    ones = np.full((L, d), ONE_BF16, dtype=np.uint16)
+    E, KI = oracle.compress(ones, logit, bias, ones[:, :8], L, m, win, js)
+    np.testing.assert_allclose(E, 1.0, rtol=0, atol=2 * eps)
+    np.testing.assert_allclose(KI, 1.0, rtol=0, atol=2 * eps)
+
+
+def test_two_token_window_is_logistic():
+    """m=1 with an overlapping window of 2: weights are the logistic function of the logit gap."""
+    d, L = 4, 6
+    x = bf(SEED, synth.X, 2, L, d)
+    logit = bf(SEED, synth.A, 2, L, d)
+    bias = synth.f32_normal(SEED, synth.BIAS_C, 2, d, 0, 2, scale=0.5)
+    E, _ = oracle.compress(x, logit, bias, None, L, 1, 2, np.arange(L))
+    xf, lf, bb = f64(x), f64(logit), bias.astype(np.float64)
+    for j in range(1, L):
+        za = lf[j - 1] + bb[0]
+        zb = lf[j] + bb[1]
+        wb = np.array([1.0 / (1.0 + math.exp(float(a - b))) for a, b in zip(za, zb)])
+        np.testing.assert_allclose(E[j], wb * xf[j] + (1 - wb) * xf[j - 1], rtol=1e-14, atol=1e-15)
+    np.testing.assert_array_equal(E[0], xf[0])  # clipped: only token 0 exists
+
+
+def test_identity_at_m1():
+    d, L = 16, 20
+    x = bf(SEED, synth.X, 3, L, d)
+    logit = bf(SEED, synth.A, 3, L, d)
+    kI = bf(SEED, synth.KI, 3, L, 8)
+    bias = synth.f32_normal(SEED, synth.BIAS_C, 3, d, 0, 1)
+    E, KI = oracle.compress(x, logit, bias, kI, L, 1, 1, np.arange(L))
+    np.testing.assert_array_equal(E, f64(x))
+    np.testing.assert_array_equal(KI, f64(kI))
+
+
+@pytest.mark.parametrize("offset", range(8))
+def test_bias_offset_counts_from_unclipped_start(offset):
+    """A dominant bias at one window offset selects token start_j + offset (start_j = 4j - 4)."""
+    d, L = 8, 24
+    x = bf(SEED, synth.X, 4, L, d)
+    logit = np.zeros((L, d), dtype=np.uint16)
+    bias = np.zeros((8, d), dtype=np.float32)
+    bias[offset, :] = 200.0
+    E, _ = oracle.compress(x, logit, bias, None, L, 4, 8, np.arange(L // 4))
+    xf = f64(x)
+    for j in range(L // 4):
+        t = 4 * j - 4 + offset
+        if t >= 0:
+            np.testing.assert_allclose(E[j], xf[t], rtol=1e-15, atol=1e-60)
+        else:  # the dominant token does not exist: the rest are equal-weighted
+            np.testing.assert_allclose(E[j], xf[0:4].mean(0), rtol=1e-15)
+
+
+@pytest.mark.parametrize("m,win", [(4, 8), (16, 16)])
+def test_locality(m, win):
+    """Changing token t changes only the entries whose window holds t."""
+    d, L = 8, 12 * m
+    x = bf(SEED, synth.X, 5, L, d)
+    logit = bf(SEED, synth.A, 5, L, d)
+    bias = synth.f32_normal(SEED, synth.BIAS_C, 5, d, 0, win, scale=0.5)
+    js = np.arange(L // m)
+    E0, _ = oracle.compress(x, logit, bias, None, L, m, win, js)
+    t = 5 * m + 1
+    x2, l2 = x.copy(), logit.copy()
+    x2[t] ^= np.uint16(0x8000)  # flip signs of token t's latent
+    l2[t] = np.uint16(0x4100)   # and change its logits
+    E1, _ = oracle.compress(x2, l2, bias, None, L, m, win, js)
+    changed = set(np.nonzero(np.any(E0 != E1, axis=1))[0].tolist())
+    expect = {t // m, t // m + 1} if win == 2 * m else {t // m}
+    assert changed == expect
+
+
+def test_entry_existence_rule():
+    x = np.zeros((10, 4), dtype=np.uint16)
+    b = np.zeros((8, 4), dtype=np.float32)
+    oracle.compress(x, x, b, None, 8, 4, 8, [1])
+    with pytest.raises(ValueError):
+        oracle.compress(x, x, b, None, 7, 4, 8, [1])  # entry 1 needs tokens up to 7
+
+
+# ---------------------------------------------------------------- indexer (a3) and top-k (a4)
+
+def test_index_score_one_hot():
+    d_I, n = 16, 50
+    KI = bf(SEED, synth.KI, 6, n, d_I)
+    for h, c in [(0, 3), (2, 15), (3, 0)]:
+        qI = np.zeros((4, d_I), dtype=np.uint16)
+        qI[h, c] = ONE_BF16
+        w = np.zeros(4, dtype=np.float32)
+        w[h] = 0.75
+        s = oracle.index_scores(qI, w, KI)
+        np.testing.assert_array_equal(s, 0.75 * np.maximum(f64(KI)[:, c], 0.0))
+
+
+def test_index_score_relu_split_matches_matmul():
+    """relu(x) - relu(-x) = x: one head's score at q minus at -q is the plain dot product."""
+    d_I, n = 64, 300
+    KI = bf(SEED, synth.KI, 7, n, d_I)
+    q = bf(SEED, synth.QI, 7, 1, d_I)
+    qn = q ^ np.uint16(0x8000)
+    qI = np.zeros((4, d_I), dtype=np.uint16)
+    qI[1] = q[0]
+    qIn = np.zeros((4, d_I), dtype=np.uint16)
+    qIn[1] = qn[0]
+    w = np.array([0, 1, 0, 0], dtype=np.float32)
+    diff = oracle.index_scores(qI, w, KI) - oracle.index_scores(qIn, w, KI)
+    ref = torch.from_numpy(f64(KI)) @ torch.from_numpy(f64(q)[0])
+    np.testing.assert_allclose(diff, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_index_score_heads_add():
+    d_I, n = 32, 100
+    KI = bf(SEED, synth.KI, 8, n, d_I)
+    qI = bf(SEED, synth.QI, 8, 4, d_I)
+    w = synth.f32_uniform(SEED, synth.W, 8, 4, 0, 1)[0]
+    total = oracle.index_scores(qI, w, KI)
+    parts = 0
+    for h in range(4):
+        wh = np.zeros(4, np.float32)
+        wh[h] = w[h]
+        parts = parts + oracle.index_scores(qI, wh, KI)
+    np.testing.assert_allclose(total, parts, rtol=1e-14)
+
+
+def brute_topk(s, k):
+    n = len(s)
+    keep = min(n, k)
+    for S in itertools.combinations(range(n), keep):
+        Sset = set(S)
+        ok = all((s[i] > s[j]) or (s[i] == s[j] and i < j) for i in S for j in range(n) if j not in Sset)
+        if ok:
+            return list(S) + [-1] * (k - keep)
+    raise AssertionError("no valid selection")
+
+
+@pytest.mark.parametrize("trial", range(30))
+def test_topk_brute_force(trial):
+    rng = np.random.default_rng(trial)
+    n = int(rng.integers(0, 10))
+    k = int(rng.integers(1, 6))
+    s = rng.integers(0, 4, size=n).astype(np.float64)  # many ties on purpose
+    assert oracle.topk(s, k).tolist() == brute_topk(s.tolist(), k)
+
+
+def test_topk_matches_library_sort():
+    rng = np.random.default_rng(5)
+    s = np.round(rng.standard_normal(20000), 2)  # ties
+    k = 1024
+    order = np.lexsort((np.arange(len(s)), -s))  # score desc, index asc
+    np.testing.assert_array_equal(oracle.topk(s, k), np.sort(order[:k]))
+    short = s[:100]
+    out = oracle.topk(short, k)
+    assert (out[:100] == np.arange(100)).all() and (out[100:] == -1).all()
+
+
+# ---------------------------------------------------------------- attention (a5 / a6 / a7)
+
+def sdpa64(qf, kf, scale, causal_rows=None):
+    """torch fp64 softmax attention; qf [H,d] for one query, kf [n,d] keys=values."""
+    q = torch.from_numpy(qf)[None, :, None, :]          # [1,H,1,d]
+    k = torch.from_numpy(kf)[None, None, :, :].expand(1, qf.shape[0], -1, -1)
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, k, scale=scale)
+    lse = torch.logsumexp(scale * (torch.from_numpy(qf) @ torch.from_numpy(kf).T), dim=-1)
+    return o[0, :, 0, :].numpy(), lse.numpy()
+
+
+def test_csa_dense_special_case_matches_library():
+    """m=1, k >= L, W=0: the CSA partial is dense softmax attention over all L tokens."""
+    H, d, L = 4, 32, 57
+    x = bf(SEED, synth.X, 9, L, d)
+    q = bf(SEED, synth.Q, 9, H, d)
+    idx = np.arange(L, dtype=np.int32)
+    O, lse = oracle.csa_attn(q, x, idx, 1, x, L, 0, 1 / math.sqrt(d))
+    Oref, lref = sdpa64(f64(q), f64(x), 1 / math.sqrt(d))
+    np.testing.assert_allclose(O, Oref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lref, rtol=1e-13)
+
+
+def test_full_pipeline_m1_is_dense_causal_attention():
+    """Compressor at m=1 (identity), k >= N, W=0 for CSA, and HCA at m'=1 each reduce to dense
+    causal attention; checked for every query position against torch's causal fp64 softmax."""
+    H, d, N, d_I = 2, 16, 24, 8
+    x = bf(SEED, synth.X, 10, N, d)
+    logit = bf(SEED, synth.A, 10, N, d)
+    kI = bf(SEED, synth.KI, 10, N, d_I)
+    bias = np.zeros((1, d), np.float32)
+    E, KI = oracle.compress(x, logit, bias, kI, N, 1, 1, np.arange(N))
+    Eb, KIb = oracle.round_bf16(E), oracle.round_bf16(KI)
+    qs = bf(SEED, synth.Q, 10, N * H, d).reshape(N, H, d)
+    qI = bf(SEED, synth.QI, 10, N * 4, d_I).reshape(N, 4, d_I)
+    w = synth.f32_uniform(SEED, synth.W, 10, 4, 0, N)
+    scale = 1 / math.sqrt(d)
+    qt = torch.from_numpy(f64(qs)).permute(1, 0, 2)[None]          # [1,H,N,d]
+    kt = torch.from_numpy(f64(x))[None, None].expand(1, H, N, d)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, kt, is_causal=True, scale=scale)[0]
+    for i in range(N):
+        L = i + 1
+        s = oracle.index_scores(qI[i], w[i], KIb[:L])
+        idx = oracle.topk(s, N + 5)
+        O_c, _ = oracle.csa_attn(qs[i], Eb, idx, 1, x, L, 0, scale)
+        O_h, _ = oracle.hca_attn(qs[i], Eb, 1, x, L, 0, scale)
+        np.testing.assert_allclose(O_c, ref[:, i, :].numpy(), rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(O_h, ref[:, i, :].numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_single_key_returns_it():
+    H, d = 3, 16
+    x = bf(SEED, synth.X, 11, 8, d)
+    q = bf(SEED, synth.Q, 11, H, d)
+    O, lse = oracle.csa_attn(q, x, np.array([-1, -1], np.int32), 4, x, 1, 1, 0.25)  # window = token 0
+    np.testing.assert_array_equal(O, np.repeat(f64(x)[0:1], H, axis=0))
+    np.testing.assert_allclose(lse, 0.25 * f64(q) @ f64(x)[0], rtol=1e-14)
+
+
+def test_key_permutation_invariance():
+    H, d, n = 4, 32, 40
+    E = bf(SEED, synth.X, 12, n, d)
+    q = bf(SEED, synth.Q, 12, H, d)
+    idx = np.arange(0, n, 2, dtype=np.int32)
+    perm = np.random.default_rng(1).permutation(idx).astype(np.int32)
+    O1, l1 = oracle.csa_attn(q, E, idx, 1, E, n, 5, 0.2)
+    O2, l2 = oracle.csa_attn(q, E, perm, 1, E, n, 5, 0.2)
+    np.testing.assert_allclose(O1, O2, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(l1, l2, rtol=1e-14)
+
+
+def test_lse_merge_of_a_partition_equals_one_softmax():
+    H, d, n = 4, 32, 64
+    E = bf(SEED, synth.X, 13, n, d)
+    q = bf(SEED, synth.Q, 13, H, d, scale=3.0)
+    rng = np.random.default_rng(3)
+    mask = rng.random(n) < 0.4
+    A = np.nonzero(mask)[0].astype(np.int32)
+    Bp = np.nonzero(~mask)[0].astype(np.int32)
+    Oa, la = oracle.csa_attn(q, E, A, 1, E, n, 0, 0.2)
+    Ob, lb = oracle.csa_attn(q, E, Bp, 1, E, n, 0, 0.2)
+    Oall, lall = oracle.csa_attn(q, E, np.arange(n, dtype=np.int32), 1, E, n, 0, 0.2)
+    O, l = oracle.lse_merge(Oa, la, Ob, lb)
+    np.testing.assert_allclose(O, Oall, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(l, lall, rtol=1e-13)
+    Oe, le = oracle.csa_attn(q, E, np.array([-1], np.int32), 1, E, n, 0, 0.2)   # empty partial
+    assert np.isneginf(le).all() and (Oe == 0).all()
+    O2, l2 = oracle.lse_merge(Oall, lall, Oe, le)
+    np.testing.assert_array_equal(O2, Oall)
+
+
+def test_noncausal_index_rejected():
+    E = np.zeros((8, 4), np.uint16)
+    q = np.zeros((1, 4), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.csa_attn(q, E, np.array([2], np.int32), 4, E, 8, 0, 1.0)  # L=8 -> entries 0,1 only
+
+
+# ---------------------------------------------------------------- the pages' printed counts
+
+def test_page_counts_one_million_tokens():
+    """1M tokens: 250,000 CSA entries, ~7,800 HCA entries, ~1,100 attended positions (~900x).
+
+    The attended-position count is read off the oracle itself: with q = 0 every logit is 0, so the
+    softmax is uniform and lse = log(number of keys)."""
+    g = json.load(open(os.path.join(GOLDEN, "page_counts.json")))
+    N, m, mh, k, W = g["tokens"], g["m"], g["m_hca"], g["k"], g["W"]
+    d = 4
+    tol = g["approx_rel_tol"]
+    assert N // m == g["csa_entries"]
+    assert abs(N // mh - g["hca_entries_approx"]) <= tol * g["hca_entries_approx"]
+    raw = np.zeros((N, d), np.uint16)
+    entries = np.zeros((N // m, d), np.uint16)
+    s = np.random.default_rng(0).random(N // m)
+    idx = oracle.topk(s, k)
+    q = np.zeros((1, d), np.uint16)
+    _, lse = oracle.csa_attn(q, entries, idx, m, raw, N, W, 0.5)
+    n_keys = round(math.exp(lse[0]))
+    assert n_keys == k + W
+    assert abs(n_keys - g["positions_approx"]) <= tol * g["positions_approx"]
+    assert abs(N / n_keys - g["reduction_approx"]) <= tol * g["reduction_approx"]
+    hca = np.zeros((N // mh, d), np.uint16)
+    _, lse_h = oracle.hca_attn(q, hca, mh, raw, N, 0, 0.5)
+    assert round(math.exp(lse_h[0])) == N // mh
+
+
+def test_two_pow_20_counts():
+    assert (1 << 20) // 4 == 262144 and (1 << 20) // 128 == 8192
+
+
+# ---------------------------------------------------------------- bf16 rounding of stored caches
+
+def test_oracle_bf16_rounding_matches_library_on_float32_values():
+    rng = np.random.default_rng(11)
+    v = np.concatenate([rng.standard_normal(200000) * 10.0 ** rng.integers(-30, 30, 200000),
+                        [1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 0.0, -0.0, 3.0e38]])
+    v32 = v.astype(np.float32)
+    ref = torch.from_numpy(v32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.round_bf16(v32.astype(np.float64)), ref)
+
+
+def test_oracle_bf16_rounding_matches_generator_on_doubles():
+    """Two independent direct double->bf16 roundings (the oracle's and the input generator's)."""
+    rng = np.random.default_rng(12)
+    v = rng.standard_normal(20000) * 10.0 ** rng.integers(-20, 20, 20000)
+    lib = synth.host_lib()
+    gen = np.array([lib.synth_bf16_host(float(a)) for a in v], dtype=np.uint16)
+    np.testing.assert_array_equal(oracle.round_bf16(v), gen)
