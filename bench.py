@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid compressed attention decode step (CSA + HCA) on B200.
+
+Default workload: 1M-context decode, B=4 sequences of N=2^20 raw tokens (262,144 CSA entries and
+8,192 HCA entries each), production widths (d=512 latent, 64 heads, indexer 4 x 64, top-k 1024,
+window 128, m'=128).  A step = one decode step of all B sequences through ``hybrid_attn_decode``:
+append one token per sequence (compressing the entries it completes), indexer scan + exact top-k,
+sparse attention over the selected entries + window, dense HCA attention, log-sum-exp merge.
+
+Prints one JSON line (rank 0).  Inputs are synthetic (seeded counter-based generator), resident in
+HBM before the timed region; the per-step working set (about 172 MB) exceeds the 126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config ctx1m|...]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA+HCA decode queries/s at 1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="ctx1m", choices=["ctx1m", "long", "ragged", "tiny"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops", 1590.0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Polls NVML (SM clock, max SM clock, clock-event reasons) every 2 ms in a thread."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _reasons(self):
+        try:
+            return self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                self.samples.append((t, mhz, int(self._reasons())))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.th.join()
+
+    def summary(self, t0, t1):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        use = inside if inside else self.samples[-5:]
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = sorted(s[1] for s in use)
+        bits = 0
+        for s in use:
+            bits |= s[2]
+        names = sorted(n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle")
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(inside), "window": "timed region" if inside else "right after the timed region"}
+
+
+# ------------------------------------------------------------------------------------ workloads
+
+def workload(name):
+    from synth import workloads
+    return {"ctx1m": workloads.ctx1m_decode, "long": workloads.long_decode, "ragged": workloads.ragged_decode,
+            "tiny": workloads.tiny}[name]()
+
+
+def dims_of(wd):
+    import compressed_sparse_kv_overlapped_b200 as csa
+    return csa.make_dims(d=wd.d, H=wd.H, d_I=wd.d_I, H_I=wd.H_I, m=wd.m, m_hca=wd.m_hca, k=wd.k, W=wd.W)
+
+
+def step_bytes(wd, lens):
+    """Algorithmic HBM bytes of one decode step: indexer-key scan, gathered top-k entries, raw window,
+    HCA entries (queries and outputs not counted)."""
+    idx = sum((L // wd.m) * wd.d_I * 2 for L in lens)
+    gather = sum(min(wd.k, L // wd.m) * wd.d * 2 for L in lens)
+    window = sum(min(wd.W, L) * wd.d * 2 for L in lens)
+    hca = sum((L // wd.m_hca) * wd.d * 2 for L in lens)
+    return idx, gather, window, hca
+
+
+# ------------------------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world):
+    import torch
+
+    import compressed_sparse_kv_overlapped_b200 as csa
+    from synth import device as sdev
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = workload(args.config)
+    wd = wl.dims
+    B = wl.B
+    K, W = args.steps, args.warmup
+    extra = W + K + (0 if args.no_e2e else K) + 1
+    layer = csa.HybridLayer(dims_of(wd), [n + extra for n in wl.n0], device=dev)
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths(list(wl.n0))
+    layer.compress()
+    steps_total = W + K
+    q_all = torch.empty(steps_total, B, wd.H, wd.d, dtype=torch.bfloat16, device=dev)
+    qi_all = torch.empty(steps_total, B, wd.H_I, wd.d_I, dtype=torch.bfloat16, device=dev)
+    w_all = torch.empty(steps_total, B, wd.H_I, dtype=torch.float32, device=dev)
+    for b in range(B):
+        sdev.fill_queries(wl, b, 0, steps_total, q_all[:, b], qi_all[:, b], w_all[:, b])
+    out = torch.empty(B, wd.H, wd.d, dtype=torch.float32, device=dev)
+    max_len = max(layer.capacity)
+    ws = layer.decode_workspace(max_len)
+    torch.cuda.synchronize()
+
+    def args_for(s):
+        return layer.decode_args(q_all[s], qi_all[s], w_all[s], out, max_len=max_len)
+
+    # warm-up (eager)
+    for s in range(W):
+        layer.decode(args_for(s), ws)
+    st = csa.csa_sync_status()
+    if st != csa.CSA_OK:
+        raise RuntimeError(f"device status {st} during warm-up")
+
+    # capture the K timed steps (with per-stage events) in one CUDA graph
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(csa.CSA_DECODE_MARKS * K)]
+    for e in marks:  # torch creates the CUDA event on first record
+        e.record()
+    torch.cuda.synchronize()
+    lens_before = list(layer.lens)
+    stream = torch.cuda.Stream(device=dev)
+    graph = torch.cuda.CUDAGraph()
+    csa.csa_set_stage_events(marks)
+    with torch.cuda.graph(graph, stream=stream):
+        for s in range(K):
+            csa.hybrid_attn_decode(args_for(W + s), ws, torch.cuda.current_stream())
+    csa.csa_set_stage_events(None)
+    layer.lens = [n + K for n in lens_before]
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.05)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        e0.record()
+        graph.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.stop()
+    st = csa.csa_sync_status()
+    if st != csa.CSA_OK:
+        raise RuntimeError(f"device status {st} in the timed region")
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # per-stage durations inside the timed region
+    M = csa.CSA_DECODE_MARKS
+    stage = {"append": 0.0, "index_scan": 0.0, "topk_select": 0.0, "attention": 0.0}
+    for s in range(K):
+        ev = marks[M * s:M * (s + 1)]
+        stage["append"] += ev[0].elapsed_time(ev[1])
+        stage["index_scan"] += ev[1].elapsed_time(ev[2])
+        stage["topk_select"] += ev[2].elapsed_time(ev[3])
+        stage["attention"] += ev[3].elapsed_time(ev[4])
+    stage = {k: v / K for k, v in stage.items()}
+
+    # algorithmic bytes per step (lengths after each step's append)
+    tot = [0, 0, 0, 0]
+    for s in range(K):
+        lens = [n + s + 1 for n in lens_before]
+        for i, v in enumerate(step_bytes(wd, lens)):
+            tot[i] += v
+    per_step = [v / K for v in tot]
+    bytes_step = sum(per_step)
+    hbm_peak, tf_peak, peak_src = peaks()
+    ms_step = ms / K
+    achieved_step_gbs = bytes_step / (ms_step * 1e-3) / 1e9
+    scan_ms = stage["index_scan"]
+    scan_gbs = per_step[0] / (scan_ms * 1e-3) / 1e9 if scan_ms > 0 else None
+    result = {
+        "metric": METRIC, "value": B * world * K / (ms * 1e-3), "unit": "queries/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
+        "config": {"workload": wl.name, "B": B, "N": wl.n0[0] if len(set(wl.n0)) == 1 else "ragged",
+                   "d": wd.d, "heads": wd.H, "d_I": wd.d_I, "H_I": wd.H_I, "k": wd.k, "W": wd.W, "m": wd.m,
+                   "m_hca": wd.m_hca, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "per-step working set larger than L2 (no flush)"},
+        "hbm": {"algorithmic_bytes_per_step": int(bytes_step),
+                "breakdown_bytes": {"index_keys": int(per_step[0]), "gathered_entries": int(per_step[1]),
+                                    "window": int(per_step[2]), "hca_entries": int(per_step[3])},
+                "achieved_gbs": achieved_step_gbs, "peak_gbs": hbm_peak, "frac": achieved_step_gbs / hbm_peak,
+                "peak_source": peak_src},
+        "stages_ms": stage,
+        "roofline": {"kernel": "index_scan_kernel", "bound": "hbm", "achieved": scan_gbs, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": (scan_gbs / hbm_peak) if scan_gbs else None, "traffic": None,
+                     "bytes_per_launch": int(per_step[0]), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
+        "clocks": clocks.summary(t0, t1),
+    }
+    # attention launches a merge kernel when a query's keys are split over several CTAs
+    result["gpu_launches"] = K * (4 + (1 if _attn_items(wd, B, max_len) > 1 else 0))
+
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(layer, wl, K, W, max_len, ws, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, samples=4)
+    return result
+
+
+def _attn_items(wd, B, max_len):
+    per_q = wd.k + wd.W + max_len // wd.m_hca
+    kpi = int(os.environ.get("CSA_KEYS_PER_ITEM", "0")) or max(128, min(2048, ((per_q * B + 127) // 128 + 63) // 64 * 64))
+    kpi = (kpi + 63) // 64 * 64
+    return (per_q + kpi - 1) // kpi
+
+
+def run_e2e(layer, wl, K, W, max_len, ws, dev, world):
+    """The same decode steps through the C ABI with the step's inputs in pinned HOST memory: every
+    step copies its query tensors and the appended token's raw rows host->device and reads the
+    output back device->host, all inside the timed region."""
+    import numpy as np
+    import torch
+
+    import compressed_sparse_kv_overlapped_b200 as csa
+    from synth import workloads
+
+    wd = wl.dims
+    B = wl.B
+    base = W + K  # query rows already used
+    hq = torch.empty(K, B, wd.H, wd.d, dtype=torch.bfloat16).pin_memory()
+    hqi = torch.empty(K, B, wd.H_I, wd.d_I, dtype=torch.bfloat16).pin_memory()
+    hw = torch.empty(K, B, wd.H_I, dtype=torch.float32).pin_memory()
+    lens0 = list(layer.lens)
+    rows = {}
+    for name, width in (("x", wd.d), ("a", wd.d), ("b", wd.d), ("kI", wd.d_I)):
+        rows[name] = torch.empty(K, B, width, dtype=torch.bfloat16).pin_memory()
+    for b in range(B):
+        q, qi, w = workloads.queries(wl, b, base, base + K)
+        hq[:, b] = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16)
+        hqi[:, b] = torch.from_numpy(qi.view(np.int16)).view(torch.bfloat16)
+        hw[:, b] = torch.from_numpy(w)
+        for name in rows:
+            t = workloads.raw_tokens(wl, b, lens0[b], lens0[b] + K, name)
+            rows[name][:, b] = torch.from_numpy(t.view(np.int16)).view(torch.bfloat16)
+    dq = torch.empty(B, wd.H, wd.d, dtype=torch.bfloat16, device=dev)
+    dqi = torch.empty(B, wd.H_I, wd.d_I, dtype=torch.bfloat16, device=dev)
+    dw = torch.empty(B, wd.H_I, dtype=torch.float32, device=dev)
+    out = torch.empty(B, wd.H, wd.d, dtype=torch.float32, device=dev)
+    hout = torch.empty(K, B, wd.H, wd.d, dtype=torch.float32).pin_memory()
+    targets = {"x": layer.x, "a": layer.logit_c, "b": layer.logit_h, "kI": layer.idx_key}
+    args = layer.decode_args(dq, dqi, dw, out, max_len=max_len)
+    h2d = (hq[0].numel() * 2 + hqi[0].numel() * 2 + hw[0].numel() * 4 +
+           sum(r[0].numel() * 2 for r in rows.values()))
+    d2h = out.numel() * 4
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(K):
+        dq.copy_(hq[s], non_blocking=True)
+        dqi.copy_(hqi[s], non_blocking=True)
+        dw.copy_(hw[s], non_blocking=True)
+        for b in range(B):
+            r = layer.tok_off[b] + lens0[b] + s
+            for name, t in targets.items():
+                t[r].copy_(rows[name][s, b], non_blocking=True)
+        csa.hybrid_attn_decode(args, ws, stream)
+        hout[s].copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    layer.lens = [n + K for n in lens0]
+    st = csa.csa_sync_status()
+    if st != csa.CSA_OK:
+        raise RuntimeError(f"device status {st} in the e2e region")
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": B * world * K / (ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms / K,
+            "how": "eager hybrid_attn_decode calls; per-step H2D of queries + appended token rows from pinned "
+                   "memory and D2H of the output, on one stream"}
+
+
+# ------------------------------------------------------------------------------------ oracle arm
+
+class OracleDecode:
+    """The fp64 oracle's decode query at the workload's geometry, for one prepared sequence: caches
+    (indexer keys, HCA entries) are built untimed; CSA entries are built for the entries each sample
+    query selects (also untimed).  A timed query runs the oracle's indexer scores, top-k, sparse
+    attention with the window, HCA attention and LSE merge."""
+
+    def __init__(self, wl, b=0, rows=(0,)):
+        import numpy as np
+
+        import oracle
+        from synth import workloads
+        self.wl, self.b = wl, b
+        wd = wl.dims
+        L = wl.n0[b] + 1
+        self.L = L
+        self.shape = oracle.Shape(d=wd.d, H=wd.H, d_I=wd.d_I, H_I=wd.H_I, m=wd.m, m_hca=wd.m_hca, k=wd.k, W=wd.W)
+        x = workloads.raw_tokens(wl, b, 0, L, "x")
+        a_idx = workloads.raw_tokens_cols(wl, b, 0, L, "a", 0, wd.d_I)
+        kI = workloads.raw_tokens(wl, b, 0, L, "kI")
+        bias_c = workloads.bias_c(wl)
+        n_c, n_h = L // wd.m, L // wd.m_hca
+        # indexer keys: the compressor on channels 0..d_I-1 with the raw indexer keys as values
+        KI, _ = oracle.compress_parallel(kI, a_idx, np.ascontiguousarray(bias_c[:, :wd.d_I]), None, L, wd.m,
+                                         2 * wd.m, np.arange(n_c))
+        self.KI = oracle.round_bf16(KI)
+        del a_idx, kI
+        bl = workloads.raw_tokens(wl, b, 0, L, "b")
+        H, _ = oracle.compress_parallel(x, bl, workloads.bias_h(wl), None, L, wd.m_hca, wd.m_hca, np.arange(n_h))
+        self.H = oracle.round_bf16(H)
+        del bl
+        self.x = x
+        self.E = np.zeros((n_c, wd.d), np.uint16)
+        self.queries = []
+        a = None
+        for r in rows:
+            q, qi, w = workloads.queries(wl, b, r, r + 1)
+            idx = oracle.topk(oracle.index_scores(qi[0], w[0], self.KI), wd.k)
+            need = idx[idx >= 0]
+            if a is None:
+                a = workloads.raw_tokens(wl, b, 0, L, "a")
+            E, _ = oracle.compress_parallel(x, a, bias_c, None, L, wd.m, 2 * wd.m, need)
+            self.E[need] = oracle.round_bf16(E)
+            self.queries.append((q[0], qi[0], w[0]))
+
+    def run(self, i):
+        import oracle
+        q, qi, w = self.queries[i]
+        return oracle.hybrid_query(self.shape, self.L, q, qi, w, self.x, self.E, self.KI, self.H)
+
+
+def cpu_baseline(wl, samples=4):
+    from concurrent.futures import ThreadPoolExecutor
+    threads = min(samples, os.cpu_count() or 1)
+    od = OracleDecode(wl, 0, rows=tuple(range(samples)))
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(od.run, range(samples)))
+    dt = time.perf_counter() - t0
+    return {"value": samples / dt, "unit": "queries/s", "cores": threads, "kind": "oracle",
+            "sample": f"{samples} decode queries of one sequence at L={od.L} (the workload's geometry), caches "
+                      f"prepared untimed, one query per thread"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, on the host cores, on this arm's config / metric / unit.  A step is one
+    decode query per sequence slot (B of them), evaluated on one prepared sequence in parallel."""
+    if rank != 0:
+        return None
+    from concurrent.futures import ThreadPoolExecutor
+    wl = workload(args.config)
+    B = wl.B
+    K, W = args.steps, args.warmup
+    od = OracleDecode(wl, 0, rows=tuple(range(B)))
+    threads = min(B, os.cpu_count() or 1)
+    with ThreadPoolExecutor(threads) as ex:
+        for _ in range(W):
+            list(ex.map(od.run, range(B)))
+        t0 = time.perf_counter()
+        for _ in range(K):
+            list(ex.map(od.run, range(B)))
+        dt = time.perf_counter() - t0
+    v = B * K / dt
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "queries/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": dt * 1e3 / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded counter-based generator)",
+            "config": {"workload": wl.name, "B": B},
+            "cpu_baseline": {"value": v, "unit": "queries/s", "cores": threads, "kind": "oracle",
+                             "sample": f"each step: {B} decode queries at L={od.L} on one prepared sequence"},
+            "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_ours(args, rank, world)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,596 @@
+// capi.cu -- the extern "C" boundary of libcsa (declared in include/csa.h): host-side argument
+// validation, workspace layout, and the orchestration of the decode and prefill hot paths.
+// No call allocates device memory or synchronizes the host.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <string>
+
+#include "compress_dev.cuh"
+#include "kernels.h"
+
+namespace csa {
+
+__device__ int g_status;
+
+namespace {
+
+thread_local std::string g_err;
+
+// optional stage events of hybrid_attn_decode (csa_set_stage_events)
+thread_local cudaEvent_t* g_events = nullptr;
+thread_local int g_event_count = 0;
+thread_local int g_event_cursor = 0;
+
+cudaEvent_t next_mark() {
+    if (!g_events) return nullptr;
+    cudaEvent_t e = g_events[g_event_cursor];
+    g_event_cursor = (g_event_cursor + 1) % g_event_count;
+    return e;
+}
+
+cudaError_t mark(cudaEvent_t e, cudaStream_t stream) { return e ? cudaEventRecord(e, stream) : cudaSuccess; }
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+    return fail(CSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+int check_dims(const csa_dims* d) {
+    if (!d) return fail(CSA_ERR_ARG, "dims is NULL");
+    if (d->d != 128 && d->d != 512) return fail(CSA_ERR_UNSUPPORTED, "d = %d (supported: 128, 512)", d->d);
+    if (d->H < 1 || d->H > 64) return fail(CSA_ERR_UNSUPPORTED, "H = %d (supported: 1..64)", d->H);
+    if (d->d_I != 32 && d->d_I != 64) return fail(CSA_ERR_UNSUPPORTED, "d_I = %d (supported: 32, 64)", d->d_I);
+    if (d->d_I > d->d) return fail(CSA_ERR_UNSUPPORTED, "d_I > d");
+    if (d->H_I < 1 || d->H_I > 8) return fail(CSA_ERR_UNSUPPORTED, "H_I = %d (supported: 1..8)", d->H_I);
+    if (d->m != 1 && d->m != 2 && d->m != 4 && d->m != 8) return fail(CSA_ERR_UNSUPPORTED, "m = %d", d->m);
+    if (d->m_hca < 1 || d->m_hca > 1024) return fail(CSA_ERR_UNSUPPORTED, "m_hca = %d", d->m_hca);
+    if (d->k < 1 || d->k > kMaxK) return fail(CSA_ERR_UNSUPPORTED, "k = %d (supported: 1..%d)", d->k, kMaxK);
+    if (d->W < 0 || d->W > 4096) return fail(CSA_ERR_UNSUPPORTED, "W = %d (supported: 0..4096)", d->W);
+    return CSA_OK;
+}
+
+int env_int(const char* name, int dflt) {
+    const char* v = getenv(name);
+    return v ? atoi(v) : dflt;
+}
+
+// Keys per attention item: about 128 items over all queries, a multiple of 64 (one tile).
+int pick_keys_per_item(int64_t total_keys) {
+    const int forced = env_int("CSA_KEYS_PER_ITEM", 0);
+    if (forced > 0) return ((forced + 63) / 64) * 64;
+    int64_t kpi = (total_keys + 127) / 128;
+    kpi = ((kpi + 63) / 64) * 64;
+    if (kpi < 128) kpi = 128;
+    if (kpi > 2048) kpi = 2048;
+    return (int)kpi;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Decode append: one CTA per sequence.  len += 1 (if appending), compress the CSA / HCA entry the
+// new token completes, publish the query table, clear this query's index scratch words.
+// ---------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+    const int b = blockIdx.x;
+    __shared__ int64_t s_len;
+    if (threadIdx.x == 0) {
+        const int64_t len = p.seqs[b].len + (p.append ? 1 : 0);
+        s_len = len;
+        p.queries[b].seq = b;
+        p.queries[b].reserved = 0;
+        p.queries[b].len = len;
+    }
+    if (p.zero_words) {
+        const int64_t per = (p.n_zero_words + p.B - 1) / p.B;
+        const int64_t z0 = (int64_t)b * per, z1 = min(p.n_zero_words, z0 + per);
+        for (int64_t i = z0 + threadIdx.x; i < z1; i += blockDim.x) p.zero_words[i] = 0u;
+    }
+    __syncthreads();
+    const int64_t len = s_len;
+    if (len < 1) {
+        if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
+        return;
+    }
+    const csa_seq sq = p.seqs[b];
+    if (p.append) {
+        const int tpe = p.d >> 3;
+        if (len % p.m == 0 && threadIdx.x < tpe) {
+            const int64_t j = len / p.m - 1;
+            compress_entry8(j, p.m, 2 * p.m, p.d, p.d_I, threadIdx.x * 8, p.x, p.logit_c, p.bias_c, p.idx_key,
+                            sq.tok_off, p.entries + (sq.csa_off + j) * p.d, p.entry_keys + (sq.csa_off + j) * p.d_I);
+        }
+        if (len % p.m_hca == 0 && threadIdx.x >= 128 && threadIdx.x < 128 + tpe) {
+            const int64_t j = len / p.m_hca - 1;
+            compress_entry8(j, p.m_hca, p.m_hca, p.d, p.d_I, (threadIdx.x - 128) * 8, p.x, p.logit_h, p.bias_h,
+                            nullptr, sq.tok_off, p.hca_entries + (sq.hca_off + j) * p.d, nullptr);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) p.seqs[b].len = len;
+    }
+}
+
+__global__ void prefill_queries_kernel(csa_query* q, int64_t p0, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        q[i].seq = 0;
+        q[i].reserved = 0;
+        q[i].len = p0 + i + 1;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Workspace layouts
+// ---------------------------------------------------------------------------------------------
+struct DecodePlan {
+    int64_t max_e;        // max CSA entries
+    int64_t max_eh;       // max HCA entries
+    int64_t e_stride;
+    int kpi, n_items;
+    size_t off_queries, off_idx, off_index, off_attn, total;
+};
+
+DecodePlan plan_decode(const csa_dims& d, int B, int64_t max_len) {
+    DecodePlan pl{};
+    pl.max_e = max_len / d.m;
+    pl.max_eh = max_len / d.m_hca;
+    pl.e_stride = ((pl.max_e + 3) / 4) * 4;
+    if (pl.e_stride < 4) pl.e_stride = 4;
+    const int64_t per_q = (int64_t)d.k + d.W + pl.max_eh;
+    pl.kpi = pick_keys_per_item(per_q * B);
+    pl.n_items = (int)((per_q + pl.kpi - 1) / pl.kpi);
+    size_t off = 0;
+    pl.off_queries = off;
+    off += align256((size_t)B * sizeof(csa_query));
+    pl.off_idx = off;
+    off += align256((size_t)B * d.k * 4);
+    pl.off_index = off;
+    off += index_ws_bytes(B, pl.e_stride);
+    pl.off_attn = off;
+    off += attn_ws_bytes(B, pl.n_items, d.d);
+    pl.total = off;
+    return pl;
+}
+
+struct PrefillPlan {
+    int64_t qc;           // queries per chunk
+    int64_t e_stride;
+    int kpi;
+    size_t off_queries, off_idx, off_index, total;
+};
+
+PrefillPlan plan_prefill(const csa_dims& d, int64_t q_end) {
+    PrefillPlan pl{};
+    const int64_t max_e = q_end / d.m;
+    pl.e_stride = ((max_e + 3) / 4) * 4;
+    if (pl.e_stride < 4) pl.e_stride = 4;
+    pl.qc = env_int("CSA_PREFILL_CHUNK", 2048);
+    if (pl.qc < 1) pl.qc = 1;
+    const int64_t keys = (int64_t)d.k + d.W + q_end / d.m_hca;
+    pl.kpi = (int)(((keys + 63) / 64) * 64);
+    size_t off = 0;
+    pl.off_queries = off;
+    off += align256((size_t)pl.qc * sizeof(csa_query));
+    pl.off_idx = off;
+    off += align256((size_t)pl.qc * d.k * 4);
+    pl.off_index = off;
+    off += index_ws_bytes((int)pl.qc, pl.e_stride);
+    pl.total = off;
+    return pl;
+}
+
+int status_ptr(int** out) {
+    static int* ptrs[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(CSA_ERR_CUDA, "device ordinal %d", dev);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_status);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        ptrs[dev] = static_cast<int*>(p);
+    }
+    *out = ptrs[dev];
+    return CSA_OK;
+}
+
+int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_e,
+              int64_t e_stride, const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
+              float* score_out, void* ws_index, bool zero_ws, int* status, cudaStream_t stream,
+              cudaEvent_t mid = nullptr) {
+    IndexParams ip{};
+    ip.seqs = seqs;
+    ip.queries = queries;
+    ip.Q = Q;
+    ip.H_I = d.H_I;
+    ip.d_I = d.d_I;
+    ip.m = d.m;
+    ip.k = d.k;
+    ip.q_idx = q_idx;
+    ip.w = w;
+    ip.entry_keys = entry_keys;
+    ip.max_entries = max_e;
+    ip.idx_out = idx_out;
+    ip.score_out = score_out;
+    ip.status = status;
+    index_ws_carve(ip, ws_index, Q, e_stride);
+    cudaError_t e = launch_index_topk(ip, max_e, stream, zero_ws, mid);
+    if (e != cudaSuccess) return cuda_fail(e, "index_topk launch");
+    return CSA_OK;
+}
+
+}  // namespace
+
+int* device_status() {
+    int* p = nullptr;
+    status_ptr(&p);
+    return p;
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+int csa_version(void) { return 100; }
+
+int csa_set_stage_events(void* const* events, int count) {
+    if (!events || count == 0) {
+        g_events = nullptr;
+        g_event_count = 0;
+        g_event_cursor = 0;
+        return CSA_OK;
+    }
+    if (count < 0 || count % CSA_DECODE_MARKS) return fail(CSA_ERR_ARG, "count = %d", count);
+    g_events = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events));
+    g_event_count = count;
+    g_event_cursor = 0;
+    return CSA_OK;
+}
+
+const char* csa_last_error(void) { return g_err.c_str(); }
+
+int csa_sync_status(csa_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int* sp = nullptr;
+    int rc = status_ptr(&sp);
+    if (rc != CSA_OK) return rc;
+    int v = 0;
+    e = cudaMemcpy(&v, sp, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "read status");
+    if (v != 0) {
+        int zero = 0;
+        e = cudaMemcpy(sp, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "clear status");
+    }
+    return v;
+}
+
+int csa_compress(const csa_dims* dims, int which, const csa_seq* seqs, const int64_t* ranges, int B,
+                 int64_t max_entries, const csa_bf16* x, const csa_bf16* logit, const float* bias,
+                 const csa_bf16* idx_key, csa_bf16* entries, csa_bf16* entry_keys, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (which != 0 && which != 1) return fail(CSA_ERR_ARG, "which = %d (0 CSA, 1 HCA)", which);
+    if (!seqs || !ranges || !x || !logit || !bias || !entries) return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (B < 1 || max_entries < 0) return fail(CSA_ERR_ARG, "B = %d, max_entries = %lld", B, (long long)max_entries);
+    if (which == 1 && (idx_key || entry_keys)) return fail(CSA_ERR_ARG, "HCA has no indexer keys");
+    if ((idx_key == nullptr) != (entry_keys == nullptr)) return fail(CSA_ERR_ARG, "idx_key and entry_keys go together");
+    if (!aligned16(x) || !aligned16(logit) || !aligned16(bias) || !aligned16(entries) ||
+        (idx_key && (!aligned16(idx_key) || !aligned16(entry_keys))))
+        return fail(CSA_ERR_ARG, "tensors must be 16-byte aligned");
+    if (max_entries == 0) return CSA_OK;
+    int* st = nullptr;
+    if ((rc = status_ptr(&st))) return rc;
+    CompressParams p{};
+    p.seqs = seqs;
+    p.ranges = ranges;
+    p.B = B;
+    p.which = which;
+    p.d = dims->d;
+    p.d_I = dims->d_I;
+    p.m = which ? dims->m_hca : dims->m;
+    p.win = which ? dims->m_hca : 2 * dims->m;
+    p.x = x;
+    p.logit = logit;
+    p.bias = bias;
+    p.idx_key = idx_key;
+    p.entries = entries;
+    p.entry_keys = entry_keys;
+    p.status = st;
+    cudaError_t e = launch_compress(p, max_entries, stream);
+    return e == cudaSuccess ? CSA_OK : cuda_fail(e, "compress launch");
+}
+
+size_t csa_workspace_size(int op, const void* args) {
+    if (!args) return 0;
+    if (op == CSA_OP_INDEX_TOPK || op == CSA_OP_SPARSE_ATTN || op == CSA_OP_HCA_ATTN) {
+        const csa_ws_query* a = static_cast<const csa_ws_query*>(args);
+        if (check_dims(&a->dims) || a->Q < 1 || a->max_len < 0) return 0;
+        if (op == CSA_OP_INDEX_TOPK) {
+            int64_t es = ((a->max_len / a->dims.m + 3) / 4) * 4;
+            if (es < 4) es = 4;
+            return index_ws_bytes(a->Q, es) + 256;
+        }
+        const int64_t keys = op == CSA_OP_SPARSE_ATTN ? (int64_t)a->dims.k + a->dims.W
+                                                      : a->max_len / a->dims.m_hca + a->dims.W;
+        const int kpi = pick_keys_per_item(keys * a->Q);
+        const int items = (int)((keys + kpi - 1) / kpi);
+        return attn_ws_bytes(a->Q, items < 1 ? 1 : items, a->dims.d) + 256;
+    }
+    if (op == CSA_OP_DECODE) {
+        const csa_decode_args* a = static_cast<const csa_decode_args*>(args);
+        if (check_dims(&a->dims) || a->B < 1 || a->max_len < 1) return 0;
+        return plan_decode(a->dims, a->B, a->max_len).total;
+    }
+    if (op == CSA_OP_PREFILL) {
+        const csa_prefill_args* a = static_cast<const csa_prefill_args*>(args);
+        if (check_dims(&a->dims) || a->q_end < 1) return 0;
+        return plan_prefill(a->dims, a->q_end).total;
+    }
+    return 0;
+}
+
+int csa_index_topk(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
+                   const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
+                   float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !queries || !q_idx || !w || !entry_keys || !idx_out) return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (Q < 1 || max_len < 1) return fail(CSA_ERR_ARG, "Q = %d, max_len = %lld", Q, (long long)max_len);
+    if (!aligned16(q_idx) || !aligned16(entry_keys)) return fail(CSA_ERR_ARG, "q_idx / entry_keys must be 16-byte aligned");
+    csa_ws_query wq{*dims, Q, 0, max_len};
+    const size_t need = csa_workspace_size(CSA_OP_INDEX_TOPK, &wq);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", need);
+    int* st = nullptr;
+    if ((rc = status_ptr(&st))) return rc;
+    const int64_t max_e = max_len / dims->m;
+    int64_t es = ((max_e + 3) / 4) * 4;
+    if (es < 4) es = 4;
+    return run_index(*dims, seqs, queries, Q, max_e, es, q_idx, w, entry_keys, idx_out, score_out, ws, true, st,
+                     stream);
+}
+
+static int run_attention(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q,
+                         const csa_bf16* q, const csa_bf16* entries, const int32_t* idx, int k_slots, const csa_bf16* x,
+                         int W, const csa_bf16* hca, float scale, float* out, float* lse, void* ws, int kpi,
+                         int n_items, cudaStream_t stream) {
+    int* st = nullptr;
+    int rc = status_ptr(&st);
+    if (rc) return rc;
+    AttnParams p{};
+    p.seqs = seqs;
+    p.queries = queries;
+    p.Q = Q;
+    p.H = dims->H;
+    p.d = dims->d;
+    p.q = q;
+    p.entries = entries;
+    p.idx = idx;
+    p.k_slots = k_slots;
+    p.m = dims->m;
+    p.raw = x;
+    p.W = W;
+    p.hca = hca;
+    p.m_hca = dims->m_hca;
+    p.use_hca = hca != nullptr;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.keys_per_item = kpi;
+    p.n_items = n_items;
+    p.out = out;
+    p.lse = lse;
+    p.status = st;
+    if (n_items < 1 || n_items > 256) return fail(CSA_ERR_UNSUPPORTED, "%d attention items per query (1..256)", n_items);
+    cudaError_t e = launch_attention(p, ws, stream);
+    return e == cudaSuccess ? CSA_OK : cuda_fail(e, "attention launch");
+}
+
+int csa_sparse_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, const csa_bf16* q,
+                    const csa_bf16* entries, const int32_t* idx, const csa_bf16* x, float scale, float* out,
+                    float* lse, void* ws, size_t ws_bytes, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !queries || !q || !entries || !idx || !x || !out) return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (Q < 1) return fail(CSA_ERR_ARG, "Q = %d", Q);
+    if (!aligned16(q) || !aligned16(entries) || !aligned16(x) || !aligned16(out))
+        return fail(CSA_ERR_ARG, "q / entries / x / out must be 16-byte aligned");
+    csa_ws_query wq{*dims, Q, 0, 1};
+    const size_t need = csa_workspace_size(CSA_OP_SPARSE_ATTN, &wq);
+    if (need > 256 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+        return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", need);
+    const int64_t keys = (int64_t)dims->k + dims->W;
+    const int kpi = pick_keys_per_item(keys * Q);
+    const int items = (int)((keys + kpi - 1) / kpi);
+    return run_attention(dims, seqs, queries, Q, q, entries, idx, dims->k, x, dims->W, nullptr, scale, out, lse, ws,
+                         kpi, items, stream);
+}
+
+int hca_dense_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
+                   const csa_bf16* q, const csa_bf16* hca_entries, const csa_bf16* x, int W, float scale, float* out,
+                   float* lse, void* ws, size_t ws_bytes, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !queries || !q || !hca_entries || !x || !out) return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (Q < 1 || max_len < 1 || W < 0 || W > 4096) return fail(CSA_ERR_ARG, "Q = %d, max_len, W = %d", Q, W);
+    if (!aligned16(q) || !aligned16(hca_entries) || !aligned16(x) || !aligned16(out))
+        return fail(CSA_ERR_ARG, "q / hca_entries / x / out must be 16-byte aligned");
+    csa_dims d2 = *dims;
+    d2.W = W;
+    csa_ws_query wq{d2, Q, 0, max_len};
+    const size_t need = csa_workspace_size(CSA_OP_HCA_ATTN, &wq);
+    if (need > 256 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+        return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", need);
+    // key list: [raw window | HCA entries] (no CSA slots)
+    const int64_t keys = max_len / dims->m_hca + W;
+    const int kpi = pick_keys_per_item(keys * Q);
+    int items = (int)((keys + kpi - 1) / kpi);
+    if (items < 1) items = 1;
+    return run_attention(&d2, seqs, queries, Q, q, nullptr, nullptr, 0, x, W, hca_entries, scale, out, lse, ws, kpi,
+                         items, stream);
+}
+
+int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
+    if (!a) return fail(CSA_ERR_ARG, "args is NULL");
+    int rc = check_dims(&a->dims);
+    if (rc) return rc;
+    const csa_dims& d = a->dims;
+    if (a->B < 1 || a->max_len < 1) return fail(CSA_ERR_ARG, "B = %d, max_len = %lld", a->B, (long long)a->max_len);
+    if (!a->seqs || !a->x || !a->logit_c || !a->logit_h || !a->idx_key || !a->bias_c || !a->bias_h || !a->entries ||
+        !a->entry_keys || !a->hca_entries || !a->q || !a->q_idx || !a->w || !a->out)
+        return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (!aligned16(a->x) || !aligned16(a->logit_c) || !aligned16(a->logit_h) || !aligned16(a->idx_key) ||
+        !aligned16(a->bias_c) || !aligned16(a->bias_h) || !aligned16(a->entries) || !aligned16(a->entry_keys) ||
+        !aligned16(a->hca_entries) || !aligned16(a->q) || !aligned16(a->q_idx) || !aligned16(a->out))
+        return fail(CSA_ERR_ARG, "tensors must be 16-byte aligned");
+    const DecodePlan pl = plan_decode(d, a->B, a->max_len);
+    if (!ws || ws_bytes < pl.total || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", pl.total);
+    int* st = nullptr;
+    if ((rc = status_ptr(&st))) return rc;
+    char* w = static_cast<char*>(ws);
+    csa_query* queries = reinterpret_cast<csa_query*>(w + pl.off_queries);
+    int32_t* idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t*>(w + pl.off_idx);
+    void* ws_index = w + pl.off_index;
+
+    AppendParams ap{};
+    ap.seqs = a->seqs;
+    ap.B = a->B;
+    ap.append = a->append ? 1 : 0;
+    ap.d = d.d;
+    ap.d_I = d.d_I;
+    ap.m = d.m;
+    ap.m_hca = d.m_hca;
+    ap.x = a->x;
+    ap.logit_c = a->logit_c;
+    ap.logit_h = a->logit_h;
+    ap.idx_key = a->idx_key;
+    ap.bias_c = a->bias_c;
+    ap.bias_h = a->bias_h;
+    ap.entries = a->entries;
+    ap.entry_keys = a->entry_keys;
+    ap.hca_entries = a->hca_entries;
+    ap.queries = queries;
+    ap.zero_words = static_cast<uint32_t*>(ws_index);  // histograms + counters of the index scratch
+    ap.n_zero_words = (int64_t)(index_zero_bytes(a->B) / 4);
+    ap.status = st;
+    cudaEvent_t ev[CSA_DECODE_MARKS] = {};
+    for (int i = 0; i < CSA_DECODE_MARKS; ++i) ev[i] = next_mark();
+    cudaError_t e = mark(ev[0], stream);
+    if (e == cudaSuccess) e = launch_append(ap, stream);
+    if (e == cudaSuccess) e = mark(ev[1], stream);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
+                   ws_index, false, st, stream, ev[2]);
+    if (rc) return rc;
+    if ((e = mark(ev[3], stream)) != cudaSuccess) return cuda_fail(e, "event record");
+    rc = run_attention(&d, a->seqs, queries, a->B, a->q, a->entries, idx, d.k, a->x, d.W, a->hca_entries, a->scale,
+                       a->out, a->lse, w + pl.off_attn, pl.kpi, pl.n_items, stream);
+    if (rc) return rc;
+    if ((e = mark(ev[4], stream)) != cudaSuccess) return cuda_fail(e, "event record");
+    return CSA_OK;
+}
+
+int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
+    if (!a) return fail(CSA_ERR_ARG, "args is NULL");
+    int rc = check_dims(&a->dims);
+    if (rc) return rc;
+    const csa_dims& d = a->dims;
+    if (a->q_begin < 0 || a->q_end <= a->q_begin || a->q_end > a->len)
+        return fail(CSA_ERR_ARG, "query range [%lld, %lld) of len %lld", (long long)a->q_begin, (long long)a->q_end,
+                    (long long)a->len);
+    if (!a->seq || !a->x || !a->logit_c || !a->logit_h || !a->idx_key || !a->bias_c || !a->bias_h || !a->entries ||
+        !a->entry_keys || !a->hca_entries || !a->q || !a->q_idx || !a->w || !a->out)
+        return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (!aligned16(a->x) || !aligned16(a->logit_c) || !aligned16(a->logit_h) || !aligned16(a->idx_key) ||
+        !aligned16(a->bias_c) || !aligned16(a->bias_h) || !aligned16(a->entries) || !aligned16(a->entry_keys) ||
+        !aligned16(a->hca_entries) || !aligned16(a->q) || !aligned16(a->q_idx) || !aligned16(a->out))
+        return fail(CSA_ERR_ARG, "tensors must be 16-byte aligned");
+    const PrefillPlan pl = plan_prefill(d, a->q_end);
+    if (!ws || ws_bytes < pl.total || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", pl.total);
+    int* st = nullptr;
+    if ((rc = status_ptr(&st))) return rc;
+    cudaError_t e;
+    if (a->compress) {
+        CompressParams cp{};
+        cp.seqs = a->seq;
+        cp.ranges = nullptr;
+        cp.B = 1;
+        cp.d = d.d;
+        cp.d_I = d.d_I;
+        cp.x = a->x;
+        cp.status = st;
+        cp.which = 0;
+        cp.m = d.m;
+        cp.win = 2 * d.m;
+        cp.range_begin = 0;
+        cp.range_end = a->q_end / d.m;
+        cp.logit = a->logit_c;
+        cp.bias = a->bias_c;
+        cp.idx_key = a->idx_key;
+        cp.entries = a->entries;
+        cp.entry_keys = a->entry_keys;
+        if ((e = launch_compress(cp, cp.range_end, stream)) != cudaSuccess) return cuda_fail(e, "compress launch");
+        cp.which = 1;
+        cp.m = d.m_hca;
+        cp.win = d.m_hca;
+        cp.range_end = a->q_end / d.m_hca;
+        cp.logit = a->logit_h;
+        cp.bias = a->bias_h;
+        cp.idx_key = nullptr;
+        cp.entries = a->hca_entries;
+        cp.entry_keys = nullptr;
+        if (cp.range_end > 0 && (e = launch_compress(cp, cp.range_end, stream)) != cudaSuccess)
+            return cuda_fail(e, "compress launch");
+    }
+    char* w = static_cast<char*>(ws);
+    csa_query* queries = reinterpret_cast<csa_query*>(w + pl.off_queries);
+    const int64_t max_e = a->q_end / d.m;
+    for (int64_t p0 = a->q_begin; p0 < a->q_end; p0 += pl.qc) {
+        const int64_t n = a->q_end - p0 < pl.qc ? a->q_end - p0 : pl.qc;
+        const int64_t r0 = p0 - a->q_begin;
+        if ((e = launch_prefill_queries(queries, p0, n, stream)) != cudaSuccess) return cuda_fail(e, "query table");
+        int32_t* idx = a->idx_out ? a->idx_out + r0 * d.k : reinterpret_cast<int32_t*>(w + pl.off_idx);
+        rc = run_index(d, a->seq, queries, (int)n, max_e, pl.e_stride, a->q_idx + r0 * d.H_I * d.d_I,
+                       a->w + r0 * d.H_I, a->entry_keys, idx, nullptr, w + pl.off_index, true, st, stream);
+        if (rc) return rc;
+        rc = run_attention(&d, a->seq, queries, (int)n, a->q + r0 * d.H * d.d, a->entries, idx, d.k, a->x, d.W,
+                           a->hca_entries, a->scale, a->out + r0 * d.H * d.d, a->lse ? a->lse + r0 * d.H : nullptr,
+                           nullptr, pl.kpi, 1, stream);
+        if (rc) return rc;
+    }
+    return CSA_OK;
+}
+
+}  // extern "C"
+
+namespace csa {
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
+    append_kernel<<<p.B, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_queries(csa_query* queries, int64_t p0, int64_t n, cudaStream_t stream) {
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 1024) blocks = 1024;
+    prefill_queries_kernel<<<(unsigned)blocks, 256, 0, stream>>>(queries, p0, n);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

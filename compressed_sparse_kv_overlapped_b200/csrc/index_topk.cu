@@ -1,0 +1,496 @@
+// index_topk.cu -- a3/a4: Lightning-Indexer scores and exact top-k.
+//
+// "Frontier Techniques: NTK RoPE, CSA+HCA, QAT, MTP", 2.1 (the Lightning Indexer scores the
+// compressed entries; each query keeps the top-1024); "DeepSeek V4 comprimeix el context: aixi
+// funcionen CSA i HCA", "CSA: buscar primer i atendre despres" (a light indexer scores every
+// compressed entry and only the best are attended).  Score (reading R3):
+//     s_j = sum_h w_h * relu(q^I_h . K^I_j),   j < floor(L / m);
+// top-k by (score desc, index asc), written in ascending index order, -1 past the end.
+//
+// Two kernels:
+//  scan   -- grid (chunks, queries).  Streams the indexer-key cache with coalesced 16-byte loads
+//            and computes the [16 entries x d_I] . [d_I x H_I] products on the tensor cores
+//            (mma.sync m16n8k16, K permuted so that every thread's operand is one contiguous
+//            16-byte load), applies relu / head weights in registers, writes the fp32 score and
+//            accumulates a coarse histogram of the top 11 bits of the order-preserving score key.
+//  select -- grid (filter CTAs, queries).  Every CTA finds the threshold bin from the histogram,
+//            sends its entries above it to the result list and those inside it to a candidate
+//            list; the last CTA of a query (ticket, no spinning) radix-selects the exact winners
+//            among the candidates on the 64-bit key (score key << 32 | ~index), which makes
+//            every key unique and breaks ties to the lower index, sorts the k indices and writes
+//            them.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+
+namespace {
+
+constexpr int kScanThreads = 256;
+constexpr int kSelectThreads = 512;
+constexpr int kCandSmem = 8192;  // candidates the last CTA keeps in shared memory
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// Streaming 16-byte load: not kept in L1, first to be evicted from L2.
+__device__ __forceinline__ uint4 ld_stream(const void* p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+// Scores of 16 consecutive entries (rows r0 .. r0+15 of the key cache) for one warp.
+// KV = number of 16-byte vectors per key row (d_I / 8 / 4 per thread group): d_I = 64 -> 2, 32 -> 1.
+template <int KV>
+__device__ __forceinline__ void score16(const uint16_t* keys, int64_t r0, int64_t nrows, int g, int c,
+                                        const uint32_t (&bq)[2 * KV][2], const float (&wv)[2], uint64_t pol,
+                                        float& s_lo, float& s_hi) {
+    // thread (g, c) loads rows g and g+8, vectors [32*v + 8c, 32*v + 8c + 8) for v < KV
+    uint4 lo[KV], hi[KV];
+    const int64_t rl = r0 + g, rh = r0 + g + 8;
+#pragma unroll
+    for (int v = 0; v < KV; ++v) {
+        lo[v] = rl < nrows ? ld_stream(keys + rl * (KV * 32) + v * 32 + c * 8, pol) : make_uint4(0, 0, 0, 0);
+        hi[v] = rh < nrows ? ld_stream(keys + rh * (KV * 32) + v * 32 + c * 8, pol) : make_uint4(0, 0, 0, 0);
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int v = 0; v < KV; ++v) {
+        // k-step 2v uses (x, y), k-step 2v+1 uses (z, w) of the thread's vector
+        uint32_t a0[4] = {lo[v].x, hi[v].x, lo[v].y, hi[v].y};
+        uint32_t a1[4] = {lo[v].z, hi[v].z, lo[v].w, hi[v].w};
+        mma_bf16_16816(acc, a0, bq[2 * v]);
+        mma_bf16_16816(acc, a1, bq[2 * v + 1]);
+    }
+    // acc[0], acc[1]: row g, heads 2c, 2c+1; acc[2], acc[3]: row g+8
+    float pl = wv[0] * fmaxf(acc[0], 0.f) + wv[1] * fmaxf(acc[1], 0.f);
+    float ph = wv[0] * fmaxf(acc[2], 0.f) + wv[1] * fmaxf(acc[3], 0.f);
+    pl += __shfl_xor_sync(0xffffffffu, pl, 1);
+    ph += __shfl_xor_sync(0xffffffffu, ph, 1);
+    pl += __shfl_xor_sync(0xffffffffu, pl, 2);
+    ph += __shfl_xor_sync(0xffffffffu, ph, 2);
+    s_lo = pl;
+    s_hi = ph;
+}
+
+template <int KV>
+__global__ void __launch_bounds__(kScanThreads) index_scan_kernel(IndexParams p) {
+    __shared__ uint32_t hist[kHistBins];
+    __shared__ float sc[kScanThreads / 32][4][16];
+    const int qi = blockIdx.y;
+    const csa_query qr = p.queries[qi];
+    const csa_seq sq = p.seqs[qr.seq];
+    if (qr.len < 1 || qr.len > sq.len) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, CSA_ERR_INDEX);
+        return;
+    }
+    const int64_t E = qr.len / p.m;
+    if (E <= p.k) return;  // everything is selected; the select kernel handles it alone
+    if (E > p.max_entries) {  // longer than the grid was sized for: the select kernel reports it
+        return;
+    }
+    const int64_t c0 = (int64_t)blockIdx.x * p.chunk;
+    if (c0 >= E) return;
+    const int64_t c1 = min(E, c0 + p.chunk);
+    for (int i = threadIdx.x; i < kHistBins; i += kScanThreads) hist[i] = 0u;
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, c = lane & 3;
+    // B fragments (query, permuted exactly like the key loads) and head weights
+    uint32_t bq[2 * KV][2];
+    float wv[2];
+    {
+        const uint16_t* qrow = p.q_idx + ((int64_t)qi * p.H_I + g) * p.d_I;
+        const bool hv = g < p.H_I;
+#pragma unroll
+        for (int v = 0; v < KV; ++v) {
+            uint4 t = hv ? *reinterpret_cast<const uint4*>(qrow + v * 32 + c * 8) : make_uint4(0, 0, 0, 0);
+            bq[2 * v][0] = t.x; bq[2 * v][1] = t.y;
+            bq[2 * v + 1][0] = t.z; bq[2 * v + 1][1] = t.w;
+        }
+        const int h0 = 2 * c, h1 = 2 * c + 1;
+        wv[0] = h0 < p.H_I ? p.w[(int64_t)qi * p.H_I + h0] : 0.f;
+        wv[1] = h1 < p.H_I ? p.w[(int64_t)qi * p.H_I + h1] : 0.f;
+    }
+    __syncthreads();
+
+    const uint16_t* keys = p.entry_keys + sq.csa_off * p.d_I;
+    float* srow = p.scores + (int64_t)qi * p.e_stride;
+    const uint64_t pol = policy_evict_first();
+    constexpr int kRowsPerPass = kScanThreads / 32 * 16 * 4;  // 512 entries: 4 groups of 16 per warp
+    for (int64_t base = c0; base < c1; base += kRowsPerPass) {
+        float s[4][2];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t r0 = base + (int64_t)(u * (kScanThreads / 32) + warp) * 16;
+            score16<KV>(keys, r0, c1, g, c, bq, wv, pol, s[u][0], s[u][1]);
+        }
+        // stage in shared memory, then coalesced store + histogram
+        if (c == 0) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) { sc[warp][u][g] = s[u][0]; sc[warp][u][g + 8] = s[u][1]; }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (lane < 16) {
+                const int64_t r = base + (int64_t)(u * (kScanThreads / 32) + warp) * 16 + lane;
+                if (r < c1) {
+                    const float v = sc[warp][u][lane];
+                    srow[r] = v;
+                    atomicAdd(&hist[float_key(v) >> 21], 1u);
+                }
+            }
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
+    for (int i = threadIdx.x; i < kHistBins; i += kScanThreads)
+        if (hist[i]) atomicAdd(&gh[i], hist[i]);
+}
+
+// ---- select ----------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t composite(uint32_t key, int64_t j) {
+    return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+}
+
+// Block-wide inclusive suffix sum over kHistBins bins held in shared memory: after the call,
+// suf[b] = sum of hist[b' >= b].  Uses kSelectThreads threads, 4 bins each.
+__device__ void suffix_counts(const uint32_t* hist, uint32_t* suf, uint32_t* warp_tot) {
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    // thread t owns bins [4*(511-t), 4*(511-t)+4) so that a forward scan over threads is a
+    // suffix scan over bins
+    const int b0 = 4 * (kSelectThreads - 1 - t);
+    uint32_t v[4];
+    uint32_t s = 0;
+#pragma unroll
+    for (int i = 3; i >= 0; --i) { s += hist[b0 + i]; v[i] = s; }
+    uint32_t incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t x = lane < kSelectThreads / 32 ? warp_tot[lane] : 0u;
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane < kSelectThreads / 32) warp_tot[lane] = x;
+    }
+    __syncthreads();
+    const uint32_t before = (warp > 0 ? warp_tot[warp - 1] : 0u) + (incl - s);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) suf[b0 + i] = before + v[i];
+    __syncthreads();
+}
+
+// Exact selection of the `need` largest composite keys among n candidates (all distinct, all
+// sharing the top 11 bits `top11`).  Returns the key T of the need-th largest: exactly `need`
+// candidates satisfy key >= T.  Radix passes of 8 bits over bits 52..0; the digit of each pass is
+// found by one warp with a suffix scan over the 256 digit counts.
+__device__ uint64_t radix_threshold(const uint64_t* cand, bool in_global, uint32_t n, uint32_t need,
+                                    uint32_t top11, uint32_t* cnt256, uint32_t* misc) {
+    uint64_t prefix = (uint64_t)top11 << 53;
+    uint64_t mask = (uint64_t)0x7FF << 53;
+    uint32_t remaining = need;
+    for (int shift = 45; shift >= -3; shift -= 8) {
+        const int sh = shift < 0 ? 0 : shift;
+        const int bits = shift < 0 ? 8 + shift : 8;  // the last pass covers bits 4..0
+        const uint32_t dmask = (1u << bits) - 1u;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) cnt256[i] = 0;
+        __syncthreads();
+        for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint64_t v = in_global ? __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i) : cand[i];
+            if ((v & mask) == prefix) atomicAdd(&cnt256[(uint32_t)(v >> sh) & dmask], 1u);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            // lane l owns digits [8*(31-l), 8*(31-l)+8): a forward scan over lanes is a suffix
+            // scan over digits
+            const int lane = threadIdx.x;
+            const int d0 = 8 * (31 - lane);
+            uint32_t loc[8];
+            uint32_t s = 0;
+#pragma unroll
+            for (int i = 7; i >= 0; --i) { s += cnt256[d0 + i]; loc[i] = s; }
+            uint32_t incl = s;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const uint32_t before = incl - s;  // count of digits above this lane's range
+            // digit dg with suffix(dg) >= remaining > suffix(dg + 1); suffix is monotone
+            int found = -1;
+            uint32_t above_dg = 0;
+#pragma unroll
+            for (int i = 7; i >= 0; --i) {
+                const uint32_t suf_i = before + loc[i];
+                const uint32_t suf_next = i < 7 ? before + loc[i + 1] : before;
+                if (found < 0 && suf_i >= remaining && suf_next < remaining) { found = d0 + i; above_dg = suf_next; }
+            }
+            const uint32_t hit = __ballot_sync(0xffffffffu, found >= 0);
+            const int src = __ffs(hit) - 1;
+            const int dg = __shfl_sync(0xffffffffu, found, src);
+            const uint32_t ab = __shfl_sync(0xffffffffu, above_dg, src);
+            if (lane == 0) { misc[0] = (uint32_t)dg; misc[1] = remaining - ab; }
+        }
+        __syncthreads();
+        const uint64_t dg = misc[0];
+        remaining = misc[1];
+        prefix |= dg << sh;
+        mask |= (uint64_t)dmask << sh;
+        __syncthreads();
+    }
+    return prefix;
+}
+
+__global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParams p) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);          // kHistBins
+    uint32_t* suf = hist + kHistBins;                                  // kHistBins
+    uint32_t* misc = suf + kHistBins;                                  // 64
+    uint64_t* cand_s = reinterpret_cast<uint64_t*>(misc + 64);         // kCandSmem
+    int32_t* list = reinterpret_cast<int32_t*>(cand_s + kCandSmem);    // kMaxK (sort buffer)
+    __shared__ uint32_t s_last;
+
+    const int qi = blockIdx.y;
+    const csa_query qr = p.queries[qi];
+    const csa_seq sq = p.seqs[qr.seq];
+    const bool valid = qr.len >= 1 && qr.len <= sq.len;
+    int64_t E = valid ? qr.len / p.m : 0;
+    if (E > p.max_entries) {  // the grid was sized for fewer entries: refuse rather than guess
+        if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, CSA_ERR_INDEX);
+        E = 0;
+    }
+    int32_t* out = p.idx_out + (int64_t)qi * p.k;
+    float* sout = p.score_out ? p.score_out + (int64_t)qi * p.k : nullptr;
+    const float* srow = p.scores + (int64_t)qi * p.e_stride;
+
+    if (E <= p.k) {  // select everything: no scores were computed
+        if (blockIdx.x != 0) return;
+        for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
+            out[i] = i < E ? i : -1;
+            if (sout) sout[i] = __int_as_float(0x7FC00000);
+        }
+        if (sout && E > 0) {
+            // scores of the selected entries (recomputed here; E <= k is small)
+            for (int64_t j = threadIdx.x; j < E; j += blockDim.x) {
+                const uint16_t* kr = p.entry_keys + (sq.csa_off + j) * p.d_I;
+                float s = 0.f;
+                for (int h = 0; h < p.H_I; ++h) {
+                    const uint16_t* qh = p.q_idx + ((int64_t)qi * p.H_I + h) * p.d_I;
+                    float dot = 0.f;
+                    for (int cc = 0; cc < p.d_I; ++cc)
+                        dot = fmaf(__uint_as_float((uint32_t)qh[cc] << 16), __uint_as_float((uint32_t)kr[cc] << 16), dot);
+                    s += p.w[(int64_t)qi * p.H_I + h] * fmaxf(dot, 0.f);
+                }
+                sout[j] = s;
+            }
+        }
+        return;
+    }
+
+    // 1. threshold bin
+    const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = gh[i];
+    __syncthreads();
+    suffix_counts(hist, suf, misc);
+    if (threadIdx.x == 0) {
+        int b1 = kHistBins - 1;
+        while (b1 > 0 && suf[b1] < (uint32_t)p.k) --b1;
+        misc[32] = (uint32_t)b1;
+        misc[33] = b1 + 1 < kHistBins ? suf[b1 + 1] : 0u;  // strictly above
+    }
+    __syncthreads();
+    const uint32_t b1 = misc[32];
+    const uint32_t above = misc[33];
+    const uint32_t need = (uint32_t)p.k - above;
+
+    // 2. filter this CTA's slice
+    uint32_t* ctr = p.counters + (int64_t)qi * 4;
+    int32_t* sel = p.sel + (int64_t)qi * kMaxK;
+    uint64_t* cand = p.cand + (int64_t)qi * p.e_stride;
+    const int64_t per = (E + gridDim.x - 1) / gridDim.x;
+    const int64_t lo = (int64_t)blockIdx.x * per, hi = min(E, lo + per);
+    const int lane = threadIdx.x & 31;
+    for (int64_t j0 = lo; j0 < hi; j0 += blockDim.x) {
+        const int64_t j = j0 + threadIdx.x;
+        uint32_t key = 0, bin = 0;
+        if (j < hi) { key = float_key(srow[j]); bin = key >> 21; }
+        const bool is_sel = j < hi && bin > b1;
+        const bool is_cand = j < hi && bin == b1;
+        const uint32_t ms = __ballot_sync(0xffffffffu, is_sel);
+        const uint32_t mc = __ballot_sync(0xffffffffu, is_cand);
+        uint32_t bs = 0, bc = 0;
+        if (lane == 0) {
+            if (ms) bs = atomicAdd(&ctr[0], __popc(ms));
+            if (mc) bc = atomicAdd(&ctr[1], __popc(mc));
+        }
+        bs = __shfl_sync(0xffffffffu, bs, 0);
+        bc = __shfl_sync(0xffffffffu, bc, 0);
+        const uint32_t below = (1u << lane) - 1u;
+        if (is_sel) {
+            const uint32_t pos = bs + __popc(ms & below);
+            if (pos < (uint32_t)kMaxK) sel[pos] = (int32_t)j;
+        }
+        if (is_cand) cand[bc + __popc(mc & below)] = composite(key, j);
+    }
+
+    // 3. the last CTA of this query finishes the selection
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(&ctr[2], 1u) == gridDim.x - 1) ? 1u : 0u;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    const uint32_t n_above = *((volatile uint32_t*)&ctr[0]);
+    const uint32_t n_cand = *((volatile uint32_t*)&ctr[1]);
+    if (n_above != above || n_cand < need) {  // histogram and filter disagree: cannot happen
+        if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
+        return;
+    }
+    const uint64_t* cs = cand;
+    if (n_cand <= (uint32_t)kCandSmem) {
+        for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x)
+            cand_s[i] = __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i);
+        __syncthreads();
+        cs = cand_s;
+    }
+    const bool cand_global = cs == cand;
+    const uint64_t T = radix_threshold(cs, cand_global, n_cand, need, b1, hist, misc);
+    // gather the final list: entries above + candidates >= T
+    if (threadIdx.x == 0) misc[40] = above;
+    for (uint32_t i = threadIdx.x; i < above; i += blockDim.x) list[i] = __ldcg(sel + i);
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
+        const uint64_t v = cand_global ? __ldcg(reinterpret_cast<const unsigned long long*>(cs) + i) : cs[i];
+        if (v >= T) {
+            const uint32_t pos = atomicAdd(&misc[40], 1u);
+            if (pos < (uint32_t)p.k) list[pos] = (int32_t)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
+        }
+    }
+    __syncthreads();
+    // bitonic sort of the k indices (padded to a power of two with INT_MAX)
+    int npow = 1;
+    while (npow < p.k) npow <<= 1;
+    for (int i = p.k + threadIdx.x; i < npow; i += blockDim.x) list[i] = 0x7FFFFFFF;
+    __syncthreads();
+    for (int size = 2; size <= npow; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = threadIdx.x; t < npow / 2; t += blockDim.x) {
+                const int i = 2 * t - (t & (stride - 1));
+                const int jx = i + stride;
+                const bool up = (i & size) == 0;
+                const int32_t a = list[i], b = list[jx];
+                if ((a > b) == up) { list[i] = b; list[jx] = a; }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
+        const int32_t j = list[i];
+        out[i] = j;
+        if (sout) sout[i] = srow[j];
+    }
+    // leave the per-query counters and histogram clean for the next call
+    __syncthreads();
+    uint32_t* ghw = p.hist + (int64_t)qi * kHistBins;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ghw[i] = 0u;
+    if (threadIdx.x < 4) ctr[threadIdx.x] = 0u;
+}
+
+constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+}  // namespace
+
+size_t index_ws_bytes(int Q, int64_t e_stride) {
+    size_t s = 0;
+    s += align256((size_t)Q * kHistBins * 4);
+    s += align256((size_t)Q * 4 * 4);
+    s += align256((size_t)Q * kMaxK * 4);
+    s += align256((size_t)Q * e_stride * 4);
+    s += align256((size_t)Q * e_stride * 8);
+    return s;
+}
+
+size_t index_zero_bytes(int Q) { return align256((size_t)Q * kHistBins * 4) + align256((size_t)Q * 4 * 4); }
+
+void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
+    char* b = static_cast<char*>(ws);
+    p.hist = reinterpret_cast<uint32_t*>(b);
+    b += align256((size_t)Q * kHistBins * 4);
+    p.counters = reinterpret_cast<uint32_t*>(b);
+    b += align256((size_t)Q * 4 * 4);
+    p.sel = reinterpret_cast<int32_t*>(b);
+    b += align256((size_t)Q * kMaxK * 4);
+    p.scores = reinterpret_cast<float*>(b);
+    b += align256((size_t)Q * e_stride * 4);
+    p.cand = reinterpret_cast<uint64_t*>(b);
+    p.e_stride = e_stride;
+}
+
+cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
+                              cudaEvent_t mid) {
+    if (zero_ws) {
+        // histogram + counters are contiguous at the start of the workspace
+        const size_t nz = reinterpret_cast<char*>(p.sel) - reinterpret_cast<char*>(p.hist);
+        cudaError_t e = cudaMemsetAsync(p.hist, 0, nz, stream);
+        if (e != cudaSuccess) return e;
+    }
+    if (max_entries > p.k) {
+        const int64_t total = max_entries * (int64_t)p.Q;
+        // aim for ~4 scan CTAs per SM over all queries, chunks of 512..16384 entries
+        int64_t chunk = (total + 148 * 4 - 1) / (148 * 4);
+        chunk = ((chunk + 511) / 512) * 512;
+        if (chunk < 512) chunk = 512;
+        if (chunk > 16384) chunk = 16384;
+        p.chunk = chunk;
+        const int64_t gx = (max_entries + chunk - 1) / chunk;
+        if (p.d_I == 64)
+            index_scan_kernel<2><<<dim3((unsigned)gx, (unsigned)p.Q), kScanThreads, 0, stream>>>(p);
+        else
+            index_scan_kernel<1><<<dim3((unsigned)gx, (unsigned)p.Q), kScanThreads, 0, stream>>>(p);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (mid) {
+        cudaError_t e = cudaEventRecord(mid, stream);
+        if (e != cudaSuccess) return e;
+    }
+    int f = (int)((max_entries + 16383) / 16384);
+    if (f < 1) f = 1;
+    if (f > 64) f = 64;
+    p.filter_ctas = f;
+    const size_t smem = (size_t)kHistBins * 8 + 64 * 4 + (size_t)kCandSmem * 8 + (size_t)kMaxK * 4;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        attr_set = true;
+    }
+    index_select_kernel<<<dim3((unsigned)f, (unsigned)p.Q), kSelectThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

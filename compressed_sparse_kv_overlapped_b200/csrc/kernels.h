@@ -1,0 +1,115 @@
+// kernels.h -- internal launch interface between the C ABI (capi.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+struct CompressParams {
+    const csa_seq* seqs;
+    const int64_t* ranges;   // [B][2], or nullptr: every sequence uses [range_begin, range_end)
+    int64_t range_begin, range_end;
+    int B;
+    int which;               // 0 CSA, 1 HCA
+    int d, d_I, m, win;
+    const uint16_t* x;
+    const uint16_t* logit;
+    const float* bias;
+    const uint16_t* idx_key; // nullable
+    uint16_t* entries;
+    uint16_t* entry_keys;    // nullable
+    int* status;
+};
+cudaError_t launch_compress(const CompressParams& p, int64_t max_entries, cudaStream_t stream);
+
+// Indexer score scan + top-k select.
+constexpr int kHistBins = 2048;  // coarse histogram over the top 11 bits of the score key
+constexpr int kMaxK = 2048;
+
+struct IndexParams {
+    const csa_seq* seqs;
+    const csa_query* queries;
+    int Q, H_I, d_I, m, k;
+    const uint16_t* q_idx;    // [Q, H_I, d_I]
+    const float* w;           // [Q, H_I]
+    const uint16_t* entry_keys;
+    int64_t chunk;            // entries per scan CTA
+    int64_t max_entries;      // host bound of floor(L/m) over all queries (grid sizing)
+    int64_t e_stride;         // row stride of the score buffer
+    int filter_ctas;          // CTAs per query in the select kernel
+    // workspace
+    float* scores;            // [Q, e_stride]
+    uint32_t* hist;           // [Q, kHistBins]
+    uint32_t* counters;       // [Q, 4]: selected, candidates, done-ticket, spare
+    int32_t* sel;             // [Q, kMaxK] indices above the threshold bin
+    uint64_t* cand;           // [Q, e_stride] candidates in the threshold bin (composite keys)
+    // outputs
+    int32_t* idx_out;         // [Q, k]
+    float* score_out;         // [Q, k] nullable
+    int* status;
+};
+size_t index_ws_bytes(int Q, int64_t e_stride);
+size_t index_zero_bytes(int Q);  // leading bytes of the index workspace that must start at zero
+void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride);
+// `mid` (nullable): event recorded between the scan and the select kernels.
+cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
+                              cudaEvent_t mid = nullptr);
+
+// Attention over a per-query key list = [selected CSA entries | raw window | HCA entries].
+struct AttnParams {
+    const csa_seq* seqs;
+    const csa_query* queries;
+    int Q, H, d;
+    const uint16_t* q;          // [Q, H, d]
+    const uint16_t* entries;    // CSA entry cache (nullable when k_slots == 0)
+    const int32_t* idx;         // [Q, k_slots] (nullable when k_slots == 0)
+    int k_slots;
+    int m;                      // CSA ratio (bounds check of idx)
+    const uint16_t* raw;        // raw latents (window)
+    int W;
+    const uint16_t* hca;        // HCA cache (nullable when use_hca == 0)
+    int m_hca;
+    int use_hca;
+    float scale_log2;           // scale * log2(e)
+    int keys_per_item;          // multiple of 64
+    int n_items;                // items per query: ceil((k_slots + W + max HCA entries) / keys_per_item)
+    // outputs: direct when n_items == 1, else partials + combine
+    float* out;                 // [Q, H, d]
+    float* lse;                 // [Q, H] nullable
+    float* part_o;              // [Q, items, 64, d]
+    float* part_lse;            // [Q, items, 64]
+    int* status;
+};
+size_t attn_ws_bytes(int Q, int items, int d);
+cudaError_t launch_attention(AttnParams& p, void* ws, cudaStream_t stream);
+
+// Decode helper: append one token per sequence, compress completed entries, build the query table.
+struct AppendParams {
+    csa_seq* seqs;
+    int B, append;
+    int d, d_I, m, m_hca;
+    const uint16_t* x;
+    const uint16_t* logit_c;
+    const uint16_t* logit_h;
+    const uint16_t* idx_key;
+    const float* bias_c;
+    const float* bias_h;
+    uint16_t* entries;
+    uint16_t* entry_keys;
+    uint16_t* hca_entries;
+    csa_query* queries;      // [B] out
+    uint32_t* zero_words;    // index workspace words to clear (nullable)
+    int64_t n_zero_words;
+    int* status;
+};
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+
+// Prefill helper: query table for positions [p0, p0 + n) of one sequence.
+cudaError_t launch_prefill_queries(csa_query* queries, int64_t p0, int64_t n, cudaStream_t stream);
+
+int* device_status();  // address of the device status word on the current device
+
+}  // namespace csa

@@ -1,0 +1,136 @@
+"""Device-resident state of one hybrid attention layer: ragged, packed per-sequence caches.
+
+Memory layout in HBM (row-major, every tensor 256-byte aligned by the allocator):
+
+  raw tokens   x, logit_c, logit_h : [sum_b cap_b, d]   bf16   (sequence b at rows tok_off[b]..)
+               idx_key             : [sum_b cap_b, d_I] bf16
+  CSA cache    entries             : [sum_b cap_b // m, d]   bf16   (rows csa_off[b]..)
+               entry_keys          : [sum_b cap_b // m, d_I] bf16
+  HCA cache    hca_entries         : [sum_b cap_b // m', d]  bf16   (rows hca_off[b]..)
+  parameters   bias_c [2m, d], bias_h [m', d] fp32
+  table        seqs                : [B, 4] int64 = (tok_off, csa_off, hca_off, len) = csa_seq
+
+The caller fills the raw-token rows (and the parameters); ``compress`` builds the caches and
+``decode`` runs one step through ``hybrid_attn_decode``.  Torch is used for allocation only.
+"""
+from __future__ import annotations
+
+from . import (CSA_OP_DECODE, CSA_OP_PREFILL, csa_compress, csa_decode_args, csa_prefill_args, csa_workspace_size,
+               hybrid_attn_decode, hybrid_attn_prefill)
+
+
+class HybridLayer:
+    def __init__(self, dims, capacity, device="cuda"):
+        import torch
+
+        self.dims = dims
+        self.B = len(capacity)
+        self.capacity = [int(c) for c in capacity]
+        d, dI, m, mh = dims.d, dims.d_I, dims.m, dims.m_hca
+        tok, csa, hca = [], [], []
+        t = c = h = 0
+        for cap in self.capacity:
+            tok.append(t)
+            csa.append(c)
+            hca.append(h)
+            t += cap
+            c += cap // m
+            h += cap // mh
+        self.tok_off, self.csa_off, self.hca_off = tok, csa, hca
+        bf = torch.bfloat16
+        self.x = torch.empty(max(t, 1), d, dtype=bf, device=device)
+        self.logit_c = torch.empty(max(t, 1), d, dtype=bf, device=device)
+        self.logit_h = torch.empty(max(t, 1), d, dtype=bf, device=device)
+        self.idx_key = torch.empty(max(t, 1), dI, dtype=bf, device=device)
+        self.entries = torch.zeros(max(c, 1), d, dtype=bf, device=device)
+        self.entry_keys = torch.zeros(max(c, 1), dI, dtype=bf, device=device)
+        self.hca_entries = torch.zeros(max(h, 1), d, dtype=bf, device=device)
+        self.bias_c = torch.zeros(2 * m, d, dtype=torch.float32, device=device)
+        self.bias_h = torch.zeros(mh, d, dtype=torch.float32, device=device)
+        self.seqs = torch.tensor([[tok[b], csa[b], hca[b], 0] for b in range(self.B)], dtype=torch.int64,
+                                 device=device)
+        self.lens = [0] * self.B
+        self.device = device
+
+    # ---- lengths ------------------------------------------------------------------------------
+    def set_lengths(self, lens) -> None:
+        import torch
+        assert len(lens) == self.B and all(0 <= n <= c for n, c in zip(lens, self.capacity))
+        self.lens = [int(n) for n in lens]
+        self.seqs[:, 3] = torch.tensor(self.lens, dtype=torch.int64, device=self.device)
+
+    # ---- compressor full pass -----------------------------------------------------------------
+    def compress(self, stream=None) -> None:
+        """(Re)build every complete CSA and HCA entry of every sequence from the raw tokens."""
+        import torch
+        d = self.dims
+        rc = torch.tensor([[0, n // d.m] for n in self.lens], dtype=torch.int64, device=self.device)
+        rh = torch.tensor([[0, n // d.m_hca] for n in self.lens], dtype=torch.int64, device=self.device)
+        csa_compress(d, 0, self.seqs, rc, self.B, max(n // d.m for n in self.lens), self.x, self.logit_c,
+                     self.bias_c, self.idx_key, self.entries, self.entry_keys, stream)
+        if max(n // d.m_hca for n in self.lens) > 0:
+            csa_compress(d, 1, self.seqs, rh, self.B, max(n // d.m_hca for n in self.lens), self.x, self.logit_h,
+                         self.bias_h, None, self.hca_entries, None, stream)
+        self._keep = (rc, rh)  # the kernels read the range tables asynchronously
+
+    # ---- decode -------------------------------------------------------------------------------
+    def decode_args(self, q, q_idx, w, out, append=True, lse=None, idx_out=None, max_len=None,
+                    scale=None) -> csa_decode_args:
+        d = self.dims
+        a = csa_decode_args()
+        a.dims = d
+        a.B = self.B
+        a.append = 1 if append else 0
+        a.max_len = int(max_len if max_len is not None else max(self.capacity))
+        a.scale = float(scale if scale is not None else d.d ** -0.5)
+        for name, t in (("seqs", self.seqs), ("x", self.x), ("logit_c", self.logit_c), ("logit_h", self.logit_h),
+                        ("idx_key", self.idx_key), ("bias_c", self.bias_c), ("bias_h", self.bias_h),
+                        ("entries", self.entries), ("entry_keys", self.entry_keys),
+                        ("hca_entries", self.hca_entries), ("q", q), ("q_idx", q_idx), ("w", w), ("out", out),
+                        ("lse", lse), ("idx_out", idx_out)):
+            setattr(a, name, None if t is None else t.data_ptr())
+        return a
+
+    def decode_workspace(self, max_len=None):
+        import torch
+        a = csa_decode_args()
+        a.dims = self.dims
+        a.B = self.B
+        a.max_len = int(max_len if max_len is not None else max(self.capacity))
+        n = csa_workspace_size(CSA_OP_DECODE, a)
+        return torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+
+    def decode(self, args: csa_decode_args, ws, stream=None) -> None:
+        hybrid_attn_decode(args, ws, stream)
+        if args.append:
+            self.lens = [n + 1 for n in self.lens]
+
+    # ---- prefill (sequence 0) -----------------------------------------------------------------
+    def prefill_args(self, q, q_idx, w, out, q_begin, q_end, compress=True, lse=None, idx_out=None,
+                     scale=None) -> csa_prefill_args:
+        d = self.dims
+        a = csa_prefill_args()
+        a.dims = d
+        a.compress = 1 if compress else 0
+        a.len = int(self.lens[0])
+        a.q_begin, a.q_end = int(q_begin), int(q_end)
+        a.scale = float(scale if scale is not None else d.d ** -0.5)
+        a.seq = self.seqs.data_ptr()
+        for name, t in (("x", self.x), ("logit_c", self.logit_c), ("logit_h", self.logit_h),
+                        ("idx_key", self.idx_key), ("bias_c", self.bias_c), ("bias_h", self.bias_h),
+                        ("entries", self.entries), ("entry_keys", self.entry_keys),
+                        ("hca_entries", self.hca_entries), ("q", q), ("q_idx", q_idx), ("w", w), ("out", out),
+                        ("lse", lse), ("idx_out", idx_out)):
+            setattr(a, name, None if t is None else t.data_ptr())
+        return a
+
+    def prefill_workspace(self, q_end):
+        import torch
+        a = csa_prefill_args()
+        a.dims = self.dims
+        a.q_end = int(q_end)
+        n = csa_workspace_size(CSA_OP_PREFILL, a)
+        return torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+
+    def prefill(self, args: csa_prefill_args, ws, stream=None) -> None:
+        hybrid_attn_prefill(args, ws, stream)

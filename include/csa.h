@@ -1,0 +1,246 @@
+/*
+ * csa.h -- C ABI of libcsa: hybrid compressed attention (CSA + HCA) on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources are web pages, cited by title and section):
+ *  - "Frontier Techniques: NTK RoPE, CSA+HCA, QAT, MTP", section 2 "CSA + HCA -- sparse attention
+ *    at 1M tokens": CSA compresses every m = 4 tokens into one entry, a Lightning Indexer keeps the
+ *    top-1024 entries per query, and attention also covers a 128-token raw sliding window (2.1);
+ *    HCA compresses every m' = 128 tokens and attends all of its entries densely (2.2).
+ *  - "DeepSeek V4 comprimeix el context: aixi funcionen CSA i HCA": one 512-wide KV latent shared
+ *    by all heads (MQA) ("DeepSeek comprimeix la dimensio temporal"); an entry is a softmax-
+ *    weighted sum of its tokens with a separate weight per channel (same section); windows
+ *    overlap and weights are recomputed per window ("Finestres solapades per evitar fronteres
+ *    artificials"); a light indexer scores compressed entries and attention runs over the chosen
+ *    ones plus the local window ("CSA: buscar primer i atendre despres"); HCA attends every
+ *    128-token summary ("HCA: un resum global 128 vegades mes curt").
+ *
+ * Readings adopted where the pages are silent (the same readings as the fp64 test oracle):
+ *  R1 CSA entry j covers tokens [m*j - m, m*j + m) clipped at 0 (window 2m, overlap m); HCA entry j
+ *     covers [m'*j, m'*j + m').  Entry j exists once m*(j+1) <= L.
+ *  R2 z_t[c] = logit_t[c] + bias[t - start_j][c], start_j the unclipped window start; weights are a
+ *     softmax over the window per channel; entry = sum_t w_t * x_t; indexer key (channels
+ *     c < d_I) = sum_t w_t * idx_key_t[c] with the same weights.
+ *  R3 indexer score s_j = sum_h w_h * relu(q^I_h . K^I_j) (no scale); top-k by score descending,
+ *     ties to the lower entry index; fewer than k causal entries selects all and pads with -1.
+ *  R4 a query at visible length L sees raw tokens [0, L): CSA entries j < floor(L/m), HCA entries
+ *     j < floor(L/m'), and the raw window [max(0, L-W), L).
+ *  R5 K = V = the stored bf16 vector; logits scaled by `scale` (1/sqrt(d)); the CSA partial
+ *     (selected entries + window) and the HCA partial are merged by log-sum-exp; the window is
+ *     counted once (in the CSA partial).
+ *
+ * Conventions shared by every call:
+ *  - bf16 data is passed as csa_bf16 (the raw 16-bit pattern); all tensors are dense row-major.
+ *  - Every pointer argument is DEVICE memory owned by the caller, except `dims` and `args`
+ *    structs, which are read on the host during the call.  The library never allocates device
+ *    memory: scratch space is the caller's `ws` buffer of at least csa_workspace_size() bytes
+ *    (256-byte aligned).  The workspace holds no state between calls.
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream) and never synchronize
+ *    the host.  They may be captured in CUDA graphs.
+ *  - Return codes: CSA_OK, or a negative CSA_ERR_* when host-side validation or the launch fails
+ *    (then nothing, or only part of the work, was enqueued; csa_last_error() has the reason).
+ *    Data-dependent errors found on the device (an out-of-range entry index, a wait that timed
+ *    out) set a device status word instead, which csa_sync_status() returns; the affected
+ *    element is skipped, never read out of bounds.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t csa_bf16;
+typedef struct CUstream_st* csa_stream_t;
+
+#define CSA_OK 0
+#define CSA_ERR_ARG (-1)         /* invalid argument (null pointer, bad size, misalignment) */
+#define CSA_ERR_UNSUPPORTED (-2) /* a size outside what the kernels implement */
+#define CSA_ERR_CUDA (-3)        /* a CUDA launch or runtime call failed */
+#define CSA_ERR_TIMEOUT (-4)     /* device: a bounded wait inside a kernel ran out */
+#define CSA_ERR_INDEX (-5)       /* device: an entry index or length was out of range */
+
+/* Widths of one hybrid attention layer.  Supported: d in {128, 512}; 1 <= H <= 64;
+ * d_I in {32, 64}; 1 <= H_I <= 8; m in {1, 2, 4, 8}; m_hca in {1..1024}; 1 <= k <= 2048;
+ * 0 <= W <= 4096. */
+typedef struct csa_dims {
+    int32_t d;     /* KV latent width (keys = values = latent) */
+    int32_t H;     /* query heads sharing the latent (MQA) */
+    int32_t d_I;   /* indexer key width */
+    int32_t H_I;   /* indexer heads */
+    int32_t m;     /* CSA compression ratio (window 2m, overlapping) */
+    int32_t m_hca; /* HCA compression ratio (window m', non-overlapping) */
+    int32_t k;     /* CSA entries selected per query */
+    int32_t W;     /* raw sliding window, in tokens */
+} csa_dims;
+
+/* Where one sequence lives inside the (ragged, packed) caches.  Device memory. */
+typedef struct csa_seq {
+    int64_t tok_off; /* row of token 0 in the raw arrays x, logit_c, logit_h ([*, d]), idx_key ([*, d_I]) */
+    int64_t csa_off; /* row of CSA entry 0 in entries ([*, d]) and entry_keys ([*, d_I]) */
+    int64_t hca_off; /* row of HCA entry 0 in hca_entries ([*, d]) */
+    int64_t len;     /* raw tokens currently held, L */
+} csa_seq;
+
+/* One query: its sequence and its visible length L (the query sees raw tokens [0, L)).
+ * Device memory. */
+typedef struct csa_query {
+    int32_t seq;      /* index into the csa_seq table */
+    int32_t reserved; /* must be 0 */
+    int64_t len;      /* visible length L, 1 <= L <= seqs[seq].len */
+} csa_query;
+
+/* a1/a2 -- token-axis compressor ("DeepSeek V4 comprimeix el context", sections "DeepSeek
+ * comprimeix la dimensio temporal" and "Finestres solapades per evitar fronteres artificials";
+ * "Frontier Techniques", 2.1 and 2.2).
+ *  which = 0: CSA (ratio dims->m, window 2m, rows at seqs[b].csa_off, also writes entry_keys if
+ *             non-NULL from idx_key); which = 1: HCA (ratio dims->m_hca, window m', rows at
+ *             seqs[b].hca_off; idx_key/entry_keys must be NULL).
+ *  ranges: device int64 [B][2]; sequence b recomputes entries [ranges[b][0], ranges[b][1]).
+ *          Entries must be complete: m*ranges[b][1] <= seqs[b].len (else CSA_ERR_INDEX on device).
+ *  max_entries: host-side upper bound of ranges[b][1] - ranges[b][0] (sizes the grid).
+ *  x, logit: [*, d] bf16 rows addressed by seqs[b].tok_off; bias: fp32 [win, d].
+ *  Outputs entries/entry_keys are bf16 (round-to-nearest-even of fp32 accumulations). */
+int csa_compress(const csa_dims* dims, int which, const csa_seq* seqs, const int64_t* ranges, int B,
+                 int64_t max_entries, const csa_bf16* x, const csa_bf16* logit, const float* bias,
+                 const csa_bf16* idx_key, csa_bf16* entries, csa_bf16* entry_keys, csa_stream_t stream);
+
+/* a3/a4 -- Lightning-Indexer scores and top-k ("Frontier Techniques", 2.1; "DeepSeek V4
+ * comprimeix el context", "CSA: buscar primer i atendre despres").  For query i at length L:
+ * s_j = sum_h w[i][h] * relu(q_idx[i][h] . entry_keys[csa_off + j]) over j < floor(L/m); the k
+ * best by (score desc, index asc) are written to idx_out[i][0..k) in ascending index order, -1 past
+ * the end.  score_out (nullable): the fp32 score of each written index (NaN past the end).
+ *  q_idx: bf16 [Q, H_I, d_I]; w: fp32 [Q, H_I]; max_len: host bound of every query's L. */
+int csa_index_topk(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
+                   const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
+                   float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* a5 -- sparse MQA attention over the selected CSA entries plus the raw window ("DeepSeek V4
+ * comprimeix el context", "CSA: buscar primer i atendre despres"; "Frontier Techniques", 2.1).
+ * Keys (= values): entries[csa_off + idx[i][s]] for every s with idx[i][s] >= 0, then
+ * x[tok_off + t] for t in [max(0, L-W), L).  For every head h:
+ *   out[i][h] = softmax_keys(scale * q[i][h] . key) @ keys,  lse[i][h] = logsumexp(scale * q . key).
+ * An index >= floor(L/m) is skipped and reported as CSA_ERR_INDEX.
+ *  q: bf16 [Q, H, d]; idx: int32 [Q, k]; out: fp32 [Q, H, d]; lse: fp32 [Q, H] (nullable). */
+int csa_sparse_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, const csa_bf16* q,
+                    const csa_bf16* entries, const int32_t* idx, const csa_bf16* x, float scale, float* out,
+                    float* lse, void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* a6 -- dense MQA attention over every visible HCA entry ("Frontier Techniques", 2.2; "DeepSeek V4
+ * comprimeix el context", "HCA: un resum global 128 vegades mes curt").  Keys: hca_entries[hca_off
+ * + j] for j < floor(L/m_hca), then (when W > 0) the raw window [max(0, L-W), L).  An empty key set
+ * gives lse = -inf and out = 0.  max_len: host bound of every query's L. */
+int hca_dense_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
+                   const csa_bf16* q, const csa_bf16* hca_entries, const csa_bf16* x, int W, float scale,
+                   float* out, float* lse, void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* Arguments of one decode step of B sequences (all pointers device memory). */
+typedef struct csa_decode_args {
+    csa_dims dims;
+    int32_t B;
+    int32_t append;      /* 1: every sequence first takes one new token (its rows at tok_off + len
+                            must already be written in x/logit_c/logit_h/idx_key); len += 1 and
+                            the entries that this token completes are compressed */
+    int64_t max_len;     /* host bound of every sequence's len after the append (sizes grids) */
+    float scale;         /* logit scale, normally 1/sqrt(d) */
+    csa_seq* seqs;       /* [B]; len is updated in place when append = 1 */
+    const csa_bf16* x;       /* raw latents [*, d] */
+    const csa_bf16* logit_c; /* CSA compressor logits [*, d] */
+    const csa_bf16* logit_h; /* HCA compressor logits [*, d] */
+    const csa_bf16* idx_key; /* raw indexer keys [*, d_I] */
+    const float* bias_c;     /* [2m, d] */
+    const float* bias_h;     /* [m_hca, d] */
+    csa_bf16* entries;       /* CSA entry cache [*, d] */
+    csa_bf16* entry_keys;    /* CSA indexer-key cache [*, d_I] */
+    csa_bf16* hca_entries;   /* HCA entry cache [*, d] */
+    const csa_bf16* q;       /* [B, H, d] */
+    const csa_bf16* q_idx;   /* [B, H_I, d_I] */
+    const float* w;          /* [B, H_I] */
+    float* out;              /* [B, H, d] merged output */
+    float* lse;              /* [B, H] merged log-sum-exp (nullable) */
+    int32_t* idx_out;        /* [B, k] selected entries (nullable) */
+} csa_decode_args;
+
+/* a8 + a3..a7 -- one decode step: optional append (and the compressor updates it triggers), then
+ * for every sequence one query at L = len: indexer top-k, sparse CSA attention with the window,
+ * dense HCA attention (window excluded), merged by log-sum-exp. */
+int hybrid_attn_decode(const csa_decode_args* args, void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* Arguments of a causal prefill of one sequence (all pointers device memory). */
+typedef struct csa_prefill_args {
+    csa_dims dims;
+    int32_t compress;        /* 1: first compress every CSA and HCA entry complete in [0, q_end) */
+    int32_t reserved;
+    int64_t len;             /* host copy of seq->len (>= q_end) */
+    int64_t q_begin, q_end;  /* query positions to compute; position p sees L = p + 1 tokens */
+    float scale;
+    const csa_seq* seq;      /* [1] */
+    const csa_bf16* x;
+    const csa_bf16* logit_c;
+    const csa_bf16* logit_h;
+    const csa_bf16* idx_key;
+    const float* bias_c;
+    const float* bias_h;
+    csa_bf16* entries;
+    csa_bf16* entry_keys;
+    csa_bf16* hca_entries;
+    const csa_bf16* q;       /* [q_end - q_begin, H, d] */
+    const csa_bf16* q_idx;   /* [q_end - q_begin, H_I, d_I] */
+    const float* w;          /* [q_end - q_begin, H_I] */
+    float* out;              /* [q_end - q_begin, H, d] */
+    float* lse;              /* [q_end - q_begin, H] (nullable) */
+    int32_t* idx_out;        /* [q_end - q_begin, k] (nullable) */
+} csa_prefill_args;
+
+/* a1, a2 full pass + a3..a7 for every query position in [q_begin, q_end) of one sequence. */
+int hybrid_attn_prefill(const csa_prefill_args* args, void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* Workspace sizes.  `op` selects the call and `args` points to the arguments it describes:
+ *   CSA_OP_INDEX_TOPK:  csa_ws_query {dims, Q, max_len}
+ *   CSA_OP_SPARSE_ATTN: csa_ws_query {dims, Q, max_len}
+ *   CSA_OP_HCA_ATTN:    csa_ws_query {dims, Q, max_len}
+ *   CSA_OP_DECODE:      csa_decode_args
+ *   CSA_OP_PREFILL:     csa_prefill_args
+ * Returns 0 for an unknown op or invalid arguments. */
+#define CSA_OP_INDEX_TOPK 1
+#define CSA_OP_SPARSE_ATTN 2
+#define CSA_OP_HCA_ATTN 3
+#define CSA_OP_DECODE 4
+#define CSA_OP_PREFILL 5
+
+typedef struct csa_ws_query {
+    csa_dims dims;
+    int32_t Q;
+    int32_t reserved;
+    int64_t max_len;
+} csa_ws_query;
+
+size_t csa_workspace_size(int op, const void* args);
+
+/* Message of the last error returned on the calling host thread ("" if none). */
+const char* csa_last_error(void);
+
+/* Synchronizes `stream`, then returns and clears the device status word of the current device
+ * (CSA_OK, CSA_ERR_INDEX or CSA_ERR_TIMEOUT), or CSA_ERR_CUDA if synchronization failed. */
+int csa_sync_status(csa_stream_t stream);
+
+/* Per-stage timing of hybrid_attn_decode (a profiling aid; off by default).  With a non-NULL
+ * array of `count` cudaEvent_t handles (created by the caller, owned by the caller), every later
+ * hybrid_attn_decode call on this host thread records CSA_DECODE_MARKS consecutive events of the
+ * array, cyclically from index 0, on its stream: before the append kernel, after it, after the
+ * indexer score scan, after the top-k select, after attention (and its merge).  Inside a stream
+ * capture the records become graph nodes.  NULL / 0 turns it off.  Returns CSA_OK or CSA_ERR_ARG
+ * (count not a positive multiple of CSA_DECODE_MARKS). */
+#define CSA_DECODE_MARKS 5
+int csa_set_stage_events(void* const* events, int count);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int csa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H */

@@ -1,0 +1,298 @@
+"""GPU parity: every stage of the CUDA path, called through the C ABI, against the fp64 oracle on
+the same seeded inputs.  Stage tests feed both sides identical input bytes (the oracle's caches);
+end-to-end tests let each side build its own caches from the raw tokens."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import compressed_sparse_kv_overlapped_b200 as csa
+import oracle
+import synth
+from synth import device as sdev
+from synth import workloads
+from tests import gpu_harness as gh
+
+pytestmark = pytest.mark.gpu
+
+SMALL_PROD = workloads.Dims()  # production widths, used with short sequences
+
+
+def wl_small(n0, steps=3, B=1, seed=2001, dims=SMALL_PROD, mode="decode"):
+    return workloads.Workload(f"small_{n0}", seed, dims, tuple(n0) if isinstance(n0, (list, tuple)) else (n0,) * B,
+                              steps, mode=mode)
+
+
+# --------------------------------------------------------------------------------- generator
+
+def test_device_generator_matches_host():
+    for tensor, ncols, r0, r1 in [(synth.X, 512, 5, 300), (synth.KI, 64, 0, 1000), (synth.Q, 64 * 512, 2, 4),
+                                  (synth.QI, 4 * 64, 0, 37)]:
+        host = synth.bf16_normal(1234, tensor, 2, ncols, r0, r1)
+        dev = torch.empty(r1 - r0, ncols, dtype=torch.int16, device="cuda")
+        synth.dev_fill("bf16_normal", 1234, tensor, 2, ncols, r0, r1, dev.data_ptr())
+        np.testing.assert_array_equal(dev.cpu().numpy().view(np.uint16), host)
+    host = synth.f32_normal(9, synth.BIAS_C, 0, 512, 0, 8, scale=0.5)
+    dev = torch.empty(8, 512, dtype=torch.float32, device="cuda")
+    synth.dev_fill("f32_normal", 9, synth.BIAS_C, 0, 512, 0, 8, dev.data_ptr(), scale=0.5)
+    np.testing.assert_array_equal(dev.cpu().numpy(), host)
+    host = synth.f32_uniform(9, synth.W, 3, 4, 0, 100)
+    dev = torch.empty(100, 4, dtype=torch.float32, device="cuda")
+    synth.dev_fill("f32_uniform", 9, synth.W, 3, 4, 0, 100, dev.data_ptr())
+    np.testing.assert_array_equal(dev.cpu().numpy(), host)
+
+
+# --------------------------------------------------------------------------------- a1/a2
+
+@pytest.mark.parametrize("wl", [workloads.tiny(), wl_small(5003), wl_small([700, 2600, 130], B=3)],
+                         ids=["tiny", "prod5003", "ragged3"])
+def test_compressor_within_one_ulp(wl):
+    layer = gh.new_layer(wl)
+    d = wl.dims
+    for b in range(wl.B):
+        n = wl.n0[b]
+        ref = gh.OracleSeq(wl, b, n)
+        n_c, n_h = n // d.m, n // d.m_hca
+        E = gh.u16(layer.entries[layer.csa_off[b]:layer.csa_off[b] + n_c])
+        K = gh.u16(layer.entry_keys[layer.csa_off[b]:layer.csa_off[b] + n_c])
+        for got, want, name in ((E, ref.E64, "entries"), (K, ref.KI64, "entry_keys")):
+            far, diff = gh.ulp_compare(got, want)
+            assert far == 0, f"{name}: {far} elements beyond one bf16 ulp"
+            assert diff <= max(2, 2e-3 * want.size), f"{name}: {diff} of {want.size} rounded differently"
+        if n_h:
+            Hh = gh.u16(layer.hca_entries[layer.hca_off[b]:layer.hca_off[b] + n_h])
+            far, diff = gh.ulp_compare(Hh, ref.H64)
+            assert far == 0 and diff <= max(2, 2e-3 * ref.H64.size), (far, diff)
+
+
+def test_incremental_append_equals_full_pass():
+    """Decode appends (compressor called per completed 4- and 128-token block) leave the caches
+    bit-identical to one full compressor pass over the same tokens."""
+    wl = wl_small([1000, 515], steps=260, B=2)
+    layer = gh.new_layer(wl)
+    d = wl.dims
+    q = torch.empty(wl.B, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(wl.B, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(wl.B, d.H_I, dtype=torch.float32, device="cuda")
+    out = torch.empty(wl.B, d.H, d.d, dtype=torch.float32, device="cuda")
+    ws = layer.decode_workspace()
+    for s in range(wl.steps):
+        for b in range(wl.B):
+            sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
+        layer.decode(layer.decode_args(q, qi, w, out), ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    full = gh.new_layer(wl, lens=[n + wl.steps for n in wl.n0])
+    for name in ("entries", "entry_keys", "hca_entries"):
+        assert torch.equal(getattr(layer, name).view(torch.int16), getattr(full, name).view(torch.int16)), name
+    assert layer.seqs[:, 3].tolist() == [n + wl.steps for n in wl.n0]
+
+
+# --------------------------------------------------------------------------------- a3/a4 (stage)
+
+def _index_case(E_list, k, d_I=64, H_I=4, seed=3001, quantize=False, zero_w=False):
+    dims = csa.make_dims(d=512, H=64, d_I=d_I, H_I=H_I, m=4, m_hca=128, k=k, W=128)
+    Q = len(E_list)
+    KIs = []
+    for qi_, E in enumerate(E_list):
+        K = synth.bf16_normal(seed, synth.KI, qi_, d_I, 0, max(E, 1))
+        if quantize:  # few distinct key values -> many exactly equal scores
+            K = oracle.round_bf16(np.round(synth.bf16_to_f64(K) * 2) / 2)
+        KIs.append(K)
+    offs = np.cumsum([0] + [max(E, 1) for E in E_list])
+    keys = gh.to_dev_bf16(np.concatenate(KIs))
+    seqs = torch.tensor([[0, offs[i], 0, 4 * E + 3] for i, E in enumerate(E_list)], dtype=torch.int64,
+                        device="cuda")
+    qt = gh.query_table([(i, 4 * E + 3) for i, E in enumerate(E_list)])
+    qI = synth.bf16_normal(seed, synth.QI, 99, H_I * d_I, 0, Q).reshape(Q, H_I, d_I)
+    w = synth.f32_uniform(seed, synth.W, 99, H_I, 0, Q)
+    if zero_w:
+        w[:] = 0
+    idx = torch.full((Q, k), -7, dtype=torch.int32, device="cuda")
+    sc = torch.empty(Q, k, dtype=torch.float32, device="cuda")
+    max_len = 4 * max(E_list) + 3
+    wq = csa.csa_ws_query()
+    wq.dims, wq.Q, wq.max_len = dims, Q, max_len
+    ws = torch.empty(csa.csa_workspace_size(csa.CSA_OP_INDEX_TOPK, wq), dtype=torch.uint8, device="cuda")
+    csa.csa_index_topk(dims, seqs, qt, Q, max_len, gh.to_dev_bf16(qI), torch.from_numpy(w).cuda(), keys, idx, sc, ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    idx_h, sc_h = idx.cpu().numpy(), sc.cpu().numpy()
+    for i, E in enumerate(E_list):
+        s = oracle.index_scores(qI[i], w[i], KIs[i][:E])
+        ref = oracle.topk(s, k)
+        gh.sets_match(idx_h[i], ref, s, k)
+        valid = idx_h[i][idx_h[i] >= 0]
+        assert (np.diff(valid) > 0).all(), "indices not ascending"
+        assert (idx_h[i][len(valid):] == -1).all() and len(valid) == min(E, k)
+        np.testing.assert_allclose(sc_h[i][:len(valid)], s[valid], rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("E_list,k,d_I", [([5000], 1024, 64), ([300], 32, 32), ([1024], 1024, 64),
+                                          ([600], 1024, 64), ([1025, 70000, 4097, 1], 1024, 64),
+                                          ([262144], 1024, 64), ([40000, 33000], 2048, 64)],
+                         ids=["E5000", "tiny", "E=k", "E<k", "ragged4", "E262144", "k2048"])
+def test_index_topk_stage(E_list, k, d_I):
+    _index_case(E_list, k, d_I)
+
+
+def test_index_topk_ties_and_zero_scores():
+    _index_case([20000, 3000], 1024, quantize=True)   # heavy exact ties: lower index wins
+    _index_case([5000], 1024, zero_w=True)             # every score 0: indices 0..k-1
+
+
+# --------------------------------------------------------------------------------- a5/a6 (stage)
+
+def _stage_layer(wl):
+    """A layer whose caches hold the ORACLE's bf16 entries (identical input bytes on both sides)."""
+    layer = csa.HybridLayer(gh.dims_of(wl.dims), [wl.capacity(b) for b in range(wl.B)])
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths(list(wl.n0))
+    refs = []
+    for b in range(wl.B):
+        r = gh.OracleSeq(wl, b, wl.n0[b])
+        n_c, n_h = len(r.E), wl.n0[b] // wl.dims.m_hca
+        layer.entries[layer.csa_off[b]:layer.csa_off[b] + n_c] = gh.to_dev_bf16(r.E)
+        layer.entry_keys[layer.csa_off[b]:layer.csa_off[b] + n_c] = gh.to_dev_bf16(r.KI)
+        if n_h:
+            layer.hca_entries[layer.hca_off[b]:layer.hca_off[b] + n_h] = gh.to_dev_bf16(r.H[:n_h])
+        refs.append(r)
+    return layer, refs
+
+
+@pytest.mark.parametrize("wl,lens", [(workloads.tiny(), [1023, 17, 5]),
+                                     (wl_small(5000, B=1), [5000, 4096, 130, 1]),
+                                     (wl_small([3000, 1300], B=2), [3000, 1299])],
+                         ids=["tiny", "prod", "prod_ragged"])
+def test_sparse_and_hca_attention_stage(wl, lens):
+    layer, refs = _stage_layer(wl)
+    d = wl.dims
+    sh = gh.oshape(d)
+    pairs = [(i % wl.B, L) for i, L in enumerate(lens)]
+    pairs = [(b, min(L, wl.n0[b])) for b, L in pairs]
+    Q = len(pairs)
+    qs = np.stack([workloads.queries(wl, b, i, i + 1)[0][0] for i, (b, _) in enumerate(pairs)])
+    idxs = []
+    for i, (b, L) in enumerate(pairs):
+        _, qi_, w_ = workloads.queries(wl, b, i, i + 1)
+        s = oracle.index_scores(qi_[0], w_[0], refs[b].KI[:L // d.m])
+        idxs.append(oracle.topk(s, d.k))
+    qt = gh.query_table(pairs)
+    q_d = gh.to_dev_bf16(qs)
+    idx_d = torch.from_numpy(np.stack(idxs)).cuda()
+    out = torch.empty(Q, d.H, d.d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(Q, d.H, dtype=torch.float32, device="cuda")
+    dims = gh.dims_of(d)
+    wq = csa.csa_ws_query()
+    wq.dims, wq.Q, wq.max_len = dims, Q, max(wl.n0)
+    ws = torch.empty(max(csa.csa_workspace_size(csa.CSA_OP_SPARSE_ATTN, wq),
+                         csa.csa_workspace_size(csa.CSA_OP_HCA_ATTN, wq)) + 256, dtype=torch.uint8, device="cuda")
+    csa.csa_sparse_attn(dims, layer.seqs, qt, Q, q_d, layer.entries, idx_d, layer.x, sh.scale, out, lse, ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    for i, (b, L) in enumerate(pairs):
+        O, l = oracle.csa_attn(qs[i], refs[b].E, idxs[i], d.m, refs[b].x, L, d.W, sh.scale)
+        gh.check_close(out[i].cpu().numpy(), O, f"csa q{i} L={L}")
+        gh.check_close(lse[i].cpu().numpy(), l, f"csa lse q{i}")
+    for W in (0, d.W):
+        out.fill_(float("nan"))
+        csa.hca_dense_attn(dims, layer.seqs, qt, Q, max(wl.n0), q_d, layer.hca_entries, layer.x, W, sh.scale, out,
+                           lse, ws)
+        assert csa.csa_sync_status() == csa.CSA_OK
+        for i, (b, L) in enumerate(pairs):
+            O, l = oracle.hca_attn(qs[i], refs[b].H, d.m_hca, refs[b].x, L, W, sh.scale)
+            if np.isneginf(l).all():  # no key at all: zero output, lse = -inf
+                assert np.isneginf(lse[i].cpu().numpy()).all() and (out[i] == 0).all()
+                continue
+            gh.check_close(out[i].cpu().numpy(), O, f"hca q{i} L={L} W={W}")
+            gh.check_close(lse[i].cpu().numpy(), l, f"hca lse q{i}")
+
+
+def test_bad_index_is_reported_not_read():
+    wl = workloads.tiny()
+    layer, refs = _stage_layer(wl)
+    d = wl.dims
+    dims = gh.dims_of(d)
+    qt = gh.query_table([(0, 64)])  # 16 causal entries
+    q = gh.to_dev_bf16(workloads.queries(wl, 0, 0, 1)[0])
+    idx = torch.full((1, d.k), -1, dtype=torch.int32, device="cuda")
+    idx[0, 0], idx[0, 1] = 3, 200  # 200 is not causal at L = 64
+    out = torch.empty(1, d.H, d.d, dtype=torch.float32, device="cuda")
+    ws = torch.empty(1 << 22, dtype=torch.uint8, device="cuda")
+    csa.csa_sparse_attn(dims, layer.seqs, qt, 1, q, layer.entries, idx, layer.x, 0.1, out, None, ws)
+    assert csa.csa_sync_status() == csa.CSA_ERR_INDEX
+    assert csa.csa_sync_status() == csa.CSA_OK  # cleared
+    idx_ok = idx.clone()
+    idx_ok[0, 1] = -1
+    out2 = torch.empty_like(out)
+    csa.csa_sparse_attn(dims, layer.seqs, qt, 1, q, layer.entries, idx_ok, layer.x, 0.1, out2, None, ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    assert torch.equal(out, out2)  # the bad slot was skipped, nothing else changed
+
+
+# --------------------------------------------------------------------------------- end to end
+
+def _decode_e2e(wl, steps, check_every=1):
+    layer = gh.new_layer(wl)
+    d = wl.dims
+    B = wl.B
+    q = torch.empty(B, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(B, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(B, d.H_I, dtype=torch.float32, device="cuda")
+    out = torch.empty(B, d.H, d.d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(B, d.H, dtype=torch.float32, device="cuda")
+    idx = torch.empty(B, d.k, dtype=torch.int32, device="cuda")
+    ws = layer.decode_workspace()
+    refs = [gh.OracleSeq(wl, b, wl.n0[b] + steps) for b in range(B)]
+    n_diff = 0
+    for s in range(steps):
+        for b in range(B):
+            sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
+        layer.decode(layer.decode_args(q, qi, w, out, lse=lse, idx_out=idx), ws)
+        assert csa.csa_sync_status() == csa.CSA_OK
+        if s % check_every and s != steps - 1:
+            continue
+        for b in range(B):
+            L = wl.n0[b] + s + 1
+            qh, qih, wh = workloads.queries(wl, b, s, s + 1)
+            r = refs[b].query(L, qh[0], qih[0], wh[0])
+            slack = gh.score_slack(qih[0], wh[0], refs[b].KI[:L // d.m])
+            n_diff += gh.sets_explained(idx[b].cpu().numpy(), r["idx"], r["scores"], slack)
+            gh.check_close(out[b].cpu().numpy(), r["O"], f"decode step {s} seq {b} L={L}")
+            gh.check_close(lse[b].cpu().numpy(), r["lse"], f"decode lse step {s} seq {b}")
+    return n_diff
+
+
+@pytest.mark.parametrize("wl,steps", [(workloads.tiny(), 1), (wl_small(6000), 3),
+                                      (wl_small([700, 3000, 9001], B=3), 2)],
+                         ids=["tiny", "prod6000", "ragged3"])
+def test_decode_end_to_end(wl, steps):
+    _decode_e2e(wl, steps)
+
+
+@pytest.mark.parametrize("N,rows,dims", [
+    (1024, list(range(0, 1024, 7)) + [1023], workloads.TINY_DIMS),
+    (3000, [0, 1, 2, 3, 4, 5, 127, 128, 129, 1023, 1024, 2047, 2048, 2999], SMALL_PROD)],
+    ids=["tiny1024", "prod3000"])
+def test_prefill_end_to_end(N, rows, dims):
+    wl = workloads.Workload(f"prefill{N}", 4004, dims, (N,), 0, mode="prefill")
+    layer = csa.HybridLayer(gh.dims_of(dims), [N])
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths([N])
+    d = dims
+    q = torch.empty(N, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(N, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(N, d.H_I, dtype=torch.float32, device="cuda")
+    sdev.fill_queries(wl, 0, 0, N, q, qi, w)
+    out = torch.empty(N, d.H, d.d, dtype=torch.float32, device="cuda")
+    idx = torch.empty(N, d.k, dtype=torch.int32, device="cuda")
+    ws = layer.prefill_workspace(N)
+    layer.prefill(layer.prefill_args(q, qi, w, out, 0, N, compress=True, idx_out=idx), ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    ref = gh.OracleSeq(wl, 0, N)
+    qh, qih, wh = workloads.queries(wl, 0, 0, N)
+    out_h, idx_h = out.cpu().numpy(), idx.cpu().numpy()
+    for i in rows:
+        L = i + 1
+        r = ref.query(L, qh[i], qih[i], wh[i])
+        slack = gh.score_slack(qih[i], wh[i], ref.KI[:L // d.m])
+        gh.sets_explained(idx_h[i], r["idx"], r["scores"], slack)
+        gh.check_close(out_h[i], r["O"], f"prefill row {i}")
