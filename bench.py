@@ -37,6 +37,8 @@ def parse():
     ap.add_argument("--config", default="ctx1m", choices=["ctx1m", "long", "ragged", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--stage", default=None, choices=["index"],
+                    help="time one stage alone on a compact case of the workload's geometry (profiling aid)")
     return ap.parse_args()
 
 
@@ -439,8 +441,59 @@ def run_reference(args, rank, world):
             "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_stage_index(args):
+    """csa_index_topk alone at the workload's indexer geometry (B queries over B sequences of
+    floor(N/4) entries of d_I-wide keys, keys N(0, 0.5^2)); no raw-token arrays, so the device holds
+    only the key cache (128 MiB at ctx1m) and the scratch.  Times K launches with CUDA events."""
+    import torch
+
+    import compressed_sparse_kv_overlapped_b200 as csa
+    import synth
+    wl = workload(args.config)
+    wd = wl.dims
+    B = wl.B
+    E = [n // wd.m for n in wl.n0]
+    keys = torch.empty(sum(E), wd.d_I, dtype=torch.bfloat16, device="cuda")
+    off = 0
+    rows = []
+    for b in range(B):
+        synth.dev_fill("bf16_normal", wl.seed, synth.KI, b, wd.d_I, 0, E[b], keys[off].data_ptr(), scale=0.5)
+        rows.append([0, off, 0, wl.n0[b]])
+        off += E[b]
+    seqs = torch.tensor(rows, dtype=torch.int64, device="cuda")
+    qt = torch.tensor([[b, wl.n0[b]] for b in range(B)], dtype=torch.int64, device="cuda")
+    qi = torch.empty(B, wd.H_I, wd.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(B, wd.H_I, dtype=torch.float32, device="cuda")
+    for b in range(B):
+        synth.dev_fill("bf16_normal", wl.seed, synth.QI, b, wd.H_I * wd.d_I, 0, 1, qi[b].data_ptr())
+        synth.dev_fill("f32_uniform", wl.seed, synth.W, b, wd.H_I, 0, 1, w[b].data_ptr())
+    idx = torch.empty(B, wd.k, dtype=torch.int32, device="cuda")
+    dims = dims_of(wd)
+    wq = csa.csa_ws_query()
+    wq.dims, wq.Q, wq.max_len = dims, B, max(wl.n0)
+    ws = torch.empty(csa.csa_workspace_size(csa.CSA_OP_INDEX_TOPK, wq), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        csa.csa_index_topk(dims, seqs, qt, B, max(wl.n0), qi, w, keys, idx, None, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        csa.csa_index_topk(dims, seqs, qt, B, max(wl.n0), qi, w, keys, idx, None, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    nbytes = sum(E) * wd.d_I * 2
+    hbm, _, src = peaks()
+    assert csa.csa_sync_status() == csa.CSA_OK
+    return {"stage": "index_topk (memset + scan + select)", "workload": wl.name, "ms_per_call": ms,
+            "key_bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "peak_gbs": hbm, "peak_source": src}
+
+
 def main():
     args = parse()
+    if args.stage == "index":
+        print(json.dumps(run_stage_index(args)), flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":

@@ -29,7 +29,10 @@ cudaEvent_t next_mark() {
     return e;
 }
 
-cudaError_t mark(cudaEvent_t e, cudaStream_t stream) { return e ? cudaEventRecord(e, stream) : cudaSuccess; }
+// External records become event nodes (with timestamps) when the stream is being captured.
+cudaError_t mark(cudaEvent_t e, cudaStream_t stream) {
+    return e ? cudaEventRecordWithFlags(e, stream, cudaEventRecordExternal) : cudaSuccess;
+}
 
 int fail(int code, const char* fmt, ...) {
     char buf[512];

@@ -476,7 +476,7 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
         if (e != cudaSuccess) return e;
     }
     if (mid) {
-        cudaError_t e = cudaEventRecord(mid, stream);
+        cudaError_t e = cudaEventRecordWithFlags(mid, stream, cudaEventRecordExternal);
         if (e != cudaSuccess) return e;
     }
     int f = (int)((max_entries + 16383) / 16384);

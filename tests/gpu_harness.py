@@ -114,7 +114,7 @@ def sets_explained(gpu_idx, oracle_idx, scores, slack):
 class OracleSeq:
     """The oracle's view of one sequence of a workload: host inputs and oracle-built caches."""
 
-    def __init__(self, wl: workloads.Workload, b: int, T: int):
+    def __init__(self, wl: workloads.Workload, b: int, T: int, with_mass: bool = False):
         self.wl, self.b, self.T = wl, b, T
         d = wl.dims
         self.x = workloads.raw_tokens(wl, b, 0, T, "x")
@@ -128,24 +128,40 @@ class OracleSeq:
         self.E = oracle.round_bf16(E)
         self.KI = oracle.round_bf16(KI)
         self.E64, self.KI64 = E, KI
+        if with_mass:  # sum_t w_t |x_t|: the scale of the fp32 accumulation error of each element
+            ax = oracle.round_bf16(np.abs(synth.bf16_to_f64(self.x)))
+            akI = oracle.round_bf16(np.abs(synth.bf16_to_f64(self.kI)))
+            self.E_mass, self.KI_mass = oracle.compress_parallel(ax, self.a, self.bias_c, akI, T, d.m, 2 * d.m,
+                                                                 np.arange(n_c))
         if n_h:
             H, _ = oracle.compress_parallel(self.x, self.bl, self.bias_h, None, T, d.m_hca, d.m_hca, np.arange(n_h))
             self.H = oracle.round_bf16(H)
             self.H64 = H
+            if with_mass:
+                self.H_mass, _ = oracle.compress_parallel(ax, self.bl, self.bias_h, None, T, d.m_hca, d.m_hca,
+                                                          np.arange(n_h))
         else:
             self.H = np.zeros((1, d.d), np.uint16)
             self.H64 = np.zeros((0, d.d))
+            self.H_mass = np.zeros((0, d.d))
 
     def query(self, L, q, qI, w):
         return oracle.hybrid_query(oshape(self.wl.dims), L, q, qI, w, self.x, self.E, self.KI, self.H)
 
 
-def ulp_compare(gpu_u16: np.ndarray, ref64: np.ndarray):
+def ulp_compare(gpu_u16: np.ndarray, ref64: np.ndarray, abs_mass: np.ndarray | None = None):
     """Compare bf16 GPU values with fp64 reference values: returns (#elements off by more than one
-    bf16 ulp of the reference, #elements that differ from the reference's own rounding)."""
+    bf16 ulp of the reference plus the fp32 accumulation bound, #elements that differ from the
+    reference's own rounding).
+
+    abs_mass = sum_t w_t |x_t| per element (the oracle's compressor applied to |x|).  A weighted sum
+    accumulated in fp32 carries an absolute error of a few fp32 ulps of that mass; where terms
+    cancel, this exceeds one bf16 ulp of the (small) result.  2^-18 is 32 fp32 ulps."""
     g = synth.bf16_to_f64(gpu_u16)
     r_round = synth.bf16_to_f64(oracle.round_bf16(ref64))
     ulp = np.maximum(np.abs(r_round) * 2.0 ** -7, 2.0 ** -133)
+    if abs_mass is not None:
+        ulp = ulp + abs_mass * 2.0 ** -18
     far = int((np.abs(g - ref64) > ulp).sum())
     diff = int((gpu_u16 != oracle.round_bf16(ref64)).sum())
     return far, diff
@@ -153,3 +169,39 @@ def ulp_compare(gpu_u16: np.ndarray, ref64: np.ndarray):
 
 def scale_of(wd) -> float:
     return 1.0 / math.sqrt(wd.d)
+
+
+class OracleSeqLazy:
+    """The oracle's view of one long sequence (e.g. 2^20 tokens) for sampled queries: indexer keys and
+    HCA entries are built for the whole sequence, CSA entries only where a sampled query needs them."""
+
+    def __init__(self, wl: workloads.Workload, b: int, T: int):
+        self.wl, self.b, self.T = wl, b, T
+        d = wl.dims
+        self.x = workloads.raw_tokens(wl, b, 0, T, "x")
+        self.a = workloads.raw_tokens(wl, b, 0, T, "a")
+        kI = workloads.raw_tokens(wl, b, 0, T, "kI")
+        self.bias_c = workloads.bias_c(wl)
+        n_c, n_h = T // d.m, T // d.m_hca
+        # indexer keys = the compressor on channels 0..d_I-1 with the raw indexer keys as values
+        KI, _ = oracle.compress_parallel(kI, np.ascontiguousarray(self.a[:, :d.d_I]),
+                                         np.ascontiguousarray(self.bias_c[:, :d.d_I]), None, T, d.m, 2 * d.m,
+                                         np.arange(n_c))
+        self.KI = oracle.round_bf16(KI)
+        bl = workloads.raw_tokens(wl, b, 0, T, "b")
+        H, _ = oracle.compress_parallel(self.x, bl, workloads.bias_h(wl), None, T, d.m_hca, d.m_hca, np.arange(n_h))
+        self.H = oracle.round_bf16(H)
+        self.E = np.zeros((max(n_c, 1), d.d), np.uint16)
+        self.have = np.zeros(max(n_c, 1), bool)
+
+    def query(self, L, q, qI, w):
+        d = self.wl.dims
+        n_c = L // d.m
+        s = oracle.index_scores(qI, w, self.KI[:n_c])
+        idx = oracle.topk(s, d.k)
+        need = np.array([j for j in idx if j >= 0 and not self.have[j]], dtype=np.int64)
+        if len(need):
+            E, _ = oracle.compress_parallel(self.x, self.a, self.bias_c, None, self.T, d.m, 2 * d.m, need)
+            self.E[need] = oracle.round_bf16(E)
+            self.have[need] = True
+        return oracle.hybrid_query(oshape(d), L, q, qI, w, self.x, self.E, self.KI, self.H)
