@@ -159,8 +159,15 @@ def run_ours(args, rank, world):
     q_all = torch.empty(steps_total, B, wd.H, wd.d, dtype=torch.bfloat16, device=dev)
     qi_all = torch.empty(steps_total, B, wd.H_I, wd.d_I, dtype=torch.bfloat16, device=dev)
     w_all = torch.empty(steps_total, B, wd.H_I, dtype=torch.float32, device=dev)
-    for b in range(B):
-        sdev.fill_queries(wl, b, 0, steps_total, q_all[:, b], qi_all[:, b], w_all[:, b])
+    tq = torch.empty(steps_total, wd.H, wd.d, dtype=torch.bfloat16, device=dev)
+    tqi = torch.empty(steps_total, wd.H_I, wd.d_I, dtype=torch.bfloat16, device=dev)
+    tw = torch.empty(steps_total, wd.H_I, dtype=torch.float32, device=dev)
+    for b in range(B):  # generate each sequence's rows contiguously, then scatter into [step, b]
+        sdev.fill_queries(wl, b, 0, steps_total, tq, tqi, tw)
+        q_all[:, b].copy_(tq)
+        qi_all[:, b].copy_(tqi)
+        w_all[:, b].copy_(tw)
+    del tq, tqi, tw
     out = torch.empty(B, wd.H, wd.d, dtype=torch.float32, device=dev)
     max_len = max(layer.capacity)
     ws = layer.decode_workspace(max_len)

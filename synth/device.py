@@ -25,6 +25,9 @@ def fill_layer_inputs(layer, wl, stream_ptr: int = 0) -> None:
 def fill_queries(wl, b: int, r0: int, r1: int, q, q_idx, w, stream_ptr: int = 0) -> None:
     """Rows [r0, r1) of sequence b's query tensors into q [n,H,d], q_idx [n,H_I,d_I], w [n,H_I]."""
     d = wl.dims
+    for t in (q, q_idx, w):  # the fill writes rows back to back from data_ptr()
+        if not t.is_contiguous():
+            raise ValueError("fill_queries needs contiguous tensors")
     dev_fill("bf16_normal", wl.seed, Q, b, d.H * d.d, r0, r1, q.data_ptr(), stream_ptr)
     dev_fill("bf16_normal", wl.seed, QI, b, d.H_I * d.d_I, r0, r1, q_idx.data_ptr(), stream_ptr)
     dev_fill("f32_uniform", wl.seed, W, b, d.H_I, r0, r1, w.data_ptr(), stream_ptr)
