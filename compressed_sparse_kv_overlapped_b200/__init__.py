@@ -30,7 +30,7 @@ CSA_OP_PREFILL = 5
 
 EXPORTS = ("csa_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
            "hybrid_attn_prefill", "csa_workspace_size", "csa_last_error", "csa_sync_status", "csa_version",
-           "csa_set_stage_events")
+           "csa_set_stage_events", "csa_index_topk_noalloc")
 CSA_DECODE_MARKS = 5
 
 _i32, _i64, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
@@ -86,8 +86,10 @@ def lib() -> ctypes.CDLL:
         L.csa_last_error.restype = ctypes.c_char_p
         L.csa_sync_status.argtypes = [_vp]
         L.csa_set_stage_events.argtypes = [_vp, ctypes.c_int]
+        L.csa_index_topk_noalloc.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
         for n in ("csa_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
-                  "hybrid_attn_prefill", "csa_sync_status", "csa_version", "csa_set_stage_events"):
+                  "hybrid_attn_prefill", "csa_sync_status", "csa_version", "csa_set_stage_events",
+                  "csa_index_topk_noalloc"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -164,6 +166,15 @@ def csa_index_topk(dims, seqs, queries, Q, max_len, q_idx, w, entry_keys, idx_ou
                               _ptr(entry_keys), _ptr(idx_out), _ptr(score_out), _ptr(ws),
                               0 if ws is None else ws.numel() * ws.element_size(), _vp(_stream(stream)))
     _check(rc, "csa_index_topk")
+
+
+def csa_index_topk_noalloc(dims, seqs, queries, Q, max_len, q_idx, w, entry_keys, idx_out, score_out,
+                           stream=None):
+    """csa_index_topk with the library's built-in scratch instead of a workspace (see csa.h)."""
+    rc = lib().csa_index_topk_noalloc(ctypes.byref(dims), _ptr(seqs), _ptr(queries), Q, max_len, _ptr(q_idx),
+                                      _ptr(w), _ptr(entry_keys), _ptr(idx_out), _ptr(score_out),
+                                      _vp(_stream(stream)))
+    _check(rc, "csa_index_topk_noalloc")
 
 
 def csa_sparse_attn(dims, seqs, queries, Q, q, entries, idx, x, scale, out, lse, ws, stream=None):

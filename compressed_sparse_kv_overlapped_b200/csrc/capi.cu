@@ -242,6 +242,18 @@ int* device_status() {
     return p;
 }
 
+int validate_dims(const csa_dims* d) { return check_dims(d); }
+
+int set_error(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
 }  // namespace csa
 
 using namespace csa;

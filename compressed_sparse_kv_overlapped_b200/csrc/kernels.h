@@ -112,4 +112,8 @@ cudaError_t launch_prefill_queries(csa_query* queries, int64_t p0, int64_t n, cu
 
 int* device_status();  // address of the device status word on the current device
 
+// Error reporting shared by entry points defined outside capi.cu.
+int validate_dims(const csa_dims* d);             // CSA_OK or the error code (message set)
+int set_error(int code, const char* fmt, ...);    // records the message for csa_last_error()
+
 }  // namespace csa

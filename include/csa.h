@@ -236,6 +236,22 @@ int csa_sync_status(csa_stream_t stream);
 #define CSA_DECODE_MARKS 5
 int csa_set_stage_events(void* const* events, int count);
 
+/* csa_index_topk without a workspace argument (no counterpart in the pages: it only changes where
+ * the scratch lives).  For callers that cannot provide device memory at call time -- code under a
+ * framework whose allocator owns all device buffers, loops that must not allocate once running, or
+ * bindings that only see input and output pointers.  The scratch is a fixed array inside the
+ * library, about 12.3 MiB on every device that loads it, held until the process exits.
+ * Limits: Q <= 16 and Q * ceil4(floor(max_len / m)) <= 1,048,576; larger calls return
+ * CSA_ERR_UNSUPPORTED with a message and enqueue nothing.  It never allocates or frees memory.
+ * The first call on a device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture.  All calls on a device share
+ * the one array, so calls whose kernels overlap on the GPU (different streams, or concurrent
+ * graph replays) race: serialize them.  Each call clears the parts that must start at zero.
+ * Arguments, results and device-side errors are those of csa_index_topk. */
+int csa_index_topk_noalloc(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q,
+                           int64_t max_len, const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys,
+                           int32_t* idx_out, float* score_out, csa_stream_t stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int csa_version(void);
 
