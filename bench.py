@@ -37,7 +37,7 @@ def parse():
     ap.add_argument("--config", default="ctx1m", choices=["ctx1m", "long", "ragged", "tiny"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--stage", default=None, choices=["index"],
+    ap.add_argument("--stage", default=None, choices=["index", "attn"],
                     help="time one stage alone on a compact case of the workload's geometry (profiling aid)")
     return ap.parse_args()
 
@@ -183,7 +183,9 @@ def run_ours(args, rank, world):
     if st != csa.CSA_OK:
         raise RuntimeError(f"device status {st} during warm-up")
 
-    # capture the K timed steps (with per-stage events) in one CUDA graph
+    # Two graphs of K decode steps each: the timed one (the product path as a caller runs it) and
+    # an identical one with per-stage CUDA events recorded between the kernels (events between
+    # kernels disable programmatic dependent launch there, so it is timed separately).
     marks = [torch.cuda.Event(enable_timing=True) for _ in range(csa.CSA_DECODE_MARKS * K)]
     for e in marks:  # torch creates the CUDA event on first record
         e.record()
@@ -191,13 +193,21 @@ def run_ours(args, rank, world):
     lens_before = list(layer.lens)
     stream = torch.cuda.Stream(device=dev)
     graph = torch.cuda.CUDAGraph()
-    csa.csa_set_stage_events(marks)
     with torch.cuda.graph(graph, stream=stream):
         for s in range(K):
             csa.hybrid_attn_decode(args_for(W + s), ws, torch.cuda.current_stream())
+    graph_ev = torch.cuda.CUDAGraph()
+    csa.csa_set_stage_events(marks)
+    with torch.cuda.graph(graph_ev, stream=stream):
+        for s in range(K):
+            csa.hybrid_attn_decode(args_for(W + s), ws, torch.cuda.current_stream())
     csa.csa_set_stage_events(None)
-    layer.lens = [n + K for n in lens_before]
 
+    def reset_lengths():
+        layer.set_lengths(lens_before)
+        torch.cuda.synchronize()
+
+    reset_lengths()
     clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.05)
@@ -223,6 +233,15 @@ def run_ours(args, rank, world):
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
+    # the same K steps again, with the stage events
+    reset_lengths()
+    with torch.cuda.stream(stream):
+        graph_ev.replay()
+    torch.cuda.synchronize()
+    st = csa.csa_sync_status()
+    if st != csa.CSA_OK:
+        raise RuntimeError(f"device status {st} in the stage-timed region")
+    layer.lens = [n + K for n in lens_before]
 
     # per-stage durations inside the timed region
     M = csa.CSA_DECODE_MARKS
@@ -262,6 +281,7 @@ def run_ours(args, rank, world):
                 "achieved_gbs": achieved_step_gbs, "peak_gbs": hbm_peak, "frac": achieved_step_gbs / hbm_peak,
                 "peak_source": peak_src},
         "stages_ms": stage,
+        "stages_note": "per-stage CUDA events recorded on the decode stream in a second, identical K-step graph",
         "roofline": {"kernel": "index_scan_kernel", "bound": "hbm", "achieved": scan_gbs, "peak": hbm_peak,
                      "unit": "GB/s", "frac": (scan_gbs / hbm_peak) if scan_gbs else None, "traffic": None,
                      "bytes_per_launch": int(per_step[0]), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
@@ -496,8 +516,78 @@ def run_stage_index(args):
             "key_bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "peak_gbs": hbm, "peak_source": src}
 
 
+def run_stage_attn(args):
+    """The decode attention alone at the workload's geometry: for each of the B queries, the sparse
+    CSA part (k selected entries + W window tokens) through csa_sparse_attn and the HCA part
+    (floor(N/m') entries) through hca_dense_attn, on caches filled directly with N(0, 0.5^2) values
+    (no raw-token arrays beyond the window rows).  Times K launches of each with CUDA events."""
+    import numpy as np
+    import torch
+
+    import compressed_sparse_kv_overlapped_b200 as csa
+    import synth
+    wl = workload(args.config)
+    wd = wl.dims
+    B = wl.B
+    n_c = [n // wd.m for n in wl.n0]
+    n_h = [n // wd.m_hca for n in wl.n0]
+    ent = torch.empty(sum(n_c), wd.d, dtype=torch.bfloat16, device="cuda")
+    hca = torch.empty(sum(n_h), wd.d, dtype=torch.bfloat16, device="cuda")
+    raw = torch.empty(B * wd.W, wd.d, dtype=torch.bfloat16, device="cuda")
+    rows = []
+    oc = oh = 0
+    for b in range(B):
+        synth.dev_fill("bf16_normal", wl.seed, synth.X, b, wd.d, 0, n_c[b], ent[oc].data_ptr(), scale=0.5)
+        synth.dev_fill("bf16_normal", wl.seed, synth.B, b, wd.d, 0, n_h[b], hca[oh].data_ptr(), scale=0.5)
+        synth.dev_fill("bf16_normal", wl.seed, synth.A, b, wd.d, 0, wd.W, raw[b * wd.W].data_ptr())
+        # raw rows of sequence b are stored so that its last W tokens land at raw[b*W : (b+1)*W]
+        rows.append([b * wd.W - (wl.n0[b] - wd.W), oc, oh, wl.n0[b]])
+        oc += n_c[b]
+        oh += n_h[b]
+    seqs = torch.tensor(rows, dtype=torch.int64, device="cuda")
+    qt = torch.tensor([[b, wl.n0[b]] for b in range(B)], dtype=torch.int64, device="cuda")
+    q = torch.empty(B, wd.H, wd.d, dtype=torch.bfloat16, device="cuda")
+    synth.dev_fill("bf16_normal", wl.seed, synth.Q, 0, wd.H * wd.d, 0, B, q.data_ptr())
+    rng = np.random.default_rng(0)
+    idx = np.stack([np.sort(rng.choice(n_c[b], size=min(wd.k, n_c[b]), replace=False)) for b in range(B)])
+    idx = torch.from_numpy(idx.astype(np.int32)).cuda()
+    out = torch.empty(B, wd.H, wd.d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(B, wd.H, dtype=torch.float32, device="cuda")
+    dims = dims_of(wd)
+    wq = csa.csa_ws_query()
+    wq.dims, wq.Q, wq.max_len = dims, B, max(wl.n0)
+    wq0 = csa.csa_ws_query()  # the HCA call below runs without the window
+    wq0.dims, wq0.Q, wq0.max_len = dims_of(wd), B, max(wl.n0)
+    wq0.dims.W = 0
+    ws = torch.empty(max(csa.csa_workspace_size(csa.CSA_OP_SPARSE_ATTN, wq),
+                         csa.csa_workspace_size(csa.CSA_OP_HCA_ATTN, wq0)), dtype=torch.uint8, device="cuda")
+    scale = wd.d ** -0.5
+    res = {"stage": "attention", "workload": wl.name}
+    for name, fn, nbytes in (
+            ("sparse", lambda: csa.csa_sparse_attn(dims, seqs, qt, B, q, ent, idx, raw, scale, out, lse, ws),
+             B * (wd.k + wd.W) * wd.d * 2),
+            ("hca", lambda: csa.hca_dense_attn(dims, seqs, qt, B, max(wl.n0), q, hca, raw, 0, scale, out, lse, ws),
+             sum(n_h) * wd.d * 2)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        res[name] = {"ms_per_call": ms, "key_bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9}
+    assert csa.csa_sync_status() == csa.CSA_OK
+    return res
+
+
 def main():
     args = parse()
+    if args.stage == "attn":
+        print(json.dumps(run_stage_attn(args)), flush=True)
+        return
     if args.stage == "index":
         print(json.dumps(run_stage_index(args)), flush=True)
         return

@@ -8,7 +8,8 @@
 // Techniques: NTK RoPE, CSA+HCA, QAT, MTP", 2.1 (top-1024 + 128-token window) and 2.2.
 //
 // The key list of query i is [CSA slots idx[i][0..k) | raw window | HCA entries 0..floor(L/m')).
-// It is cut into items of `keys_per_item` keys; one CTA computes one (query, item) pair:
+// It is cut into items (the front part and the HCA part separately, so the HCA items do not depend
+// on the top-k and can run while it is computed); one CTA computes one (query, item) pair:
 //     S   = Q . K^T           (64 heads x 64 keys,  contraction over d)   tcgen05, M=64 N=64
 //     P   = exp2(S*scale*log2e - m)  (online softmax, one row per thread)
 //     O  += P . V             (64 heads x d, contraction over 64 keys)    tcgen05, M=64 N=256/128
@@ -44,8 +45,9 @@ struct Smem {
     static constexpr int kQ = 0;
     static constexpr int kK0 = kQ + NKB * kBlock;
     static constexpr int kK1 = kK0 + NKB * kBlock;
-    static constexpr int kP = kK1 + NKB * kBlock;
-    static constexpr int kBar = kP + kBlock;           // mbarriers
+    static constexpr int kP0 = kK1 + NKB * kBlock;     // P, double-buffered
+    static constexpr int kP1 = kP0 + kBlock;
+    static constexpr int kBar = kP1 + kBlock;          // mbarriers
     static constexpr int kMisc = kBar + 16 * 8;        // tmem base, abort flag, masks
     static constexpr int kRowPtr = kMisc + 64;         // per loader warp: 16 row pointers
     static constexpr int kTotal = kRowPtr + 4 * 16 * 8;
@@ -53,58 +55,81 @@ struct Smem {
 };
 
 struct Bars {
-    uint64_t full[2];   // loaders -> MMA / softmax: stage holds tile t
-    uint64_t empty[2];  // MMA commit after P.V of the tile in the stage
-    uint64_t s_full;    // MMA commit after Q.K^T
-    uint64_t s_free;    // softmax finished reading S
-    uint64_t p_full;    // softmax wrote P (and rescaled O)
-    uint64_t o_done;    // MMA commit after P.V
-    uint64_t fin;       // MMA commit before teardown
+    uint64_t full[2];    // loaders -> MMA / softmax: key stage holds tile t
+    uint64_t empty[2];   // MMA commit after P.V of the tile in the stage
+    uint64_t s_full;     // MMA commit after Q.K^T
+    uint64_t s_free;     // softmax finished reading S
+    uint64_t p_full[2];  // softmax wrote P buffer t&1 (and rescaled O if needed)
+    uint64_t o_done[2];  // MMA commit after the P.V that read P buffer t&1
+    uint64_t fin;        // MMA commit before teardown
 };
 
-// Resolve slot `s` of query (qr, sq)'s key list [CSA slots | raw window | HCA entries] into a row
-// pointer (nullptr = masked slot).
-__device__ __forceinline__ const uint16_t* key_row(const AttnParams& p, int D, int qi, const csa_query& qr,
-                                                   const csa_seq& sq, int64_t s) {
+// Per-CTA constants of the key list [CSA slots | raw window | HCA entries] of one query.
+struct KeyList {
+    const int32_t* idx;      // this query's k slots
+    int64_t n_causal;        // floor(L / m)
+    int64_t n_hca;           // floor(L / m') (0 without HCA)
+    int64_t win_row0;        // raw row of the first window token
+    int64_t nw;              // window tokens present
+    int64_t csa_row0, hca_row0;
+};
+
+// Row pointer of slot `s` (nullptr = masked slot).
+__device__ __forceinline__ const uint16_t* key_row(const AttnParams& p, int D, const KeyList& kl, int64_t s) {
     if (s < p.k_slots) {
-        const int32_t j = p.idx[(int64_t)qi * p.k_slots + s];
+        const int32_t j = kl.idx[s];
         if (j < 0) return nullptr;
-        if ((int64_t)j >= qr.len / p.m) {
+        if ((int64_t)j >= kl.n_causal) {
             report(p.status, CSA_ERR_INDEX);
             return nullptr;
         }
-        return p.entries + (sq.csa_off + j) * D;
+        return p.entries + (kl.csa_row0 + j) * D;
     }
     s -= p.k_slots;
-    if (s < p.W) {
-        const int64_t nw = qr.len < p.W ? qr.len : p.W;
-        if (s >= nw) return nullptr;
-        return p.raw + (sq.tok_off + qr.len - nw + s) * D;
-    }
+    if (s < p.W) return s < kl.nw ? p.raw + (kl.win_row0 + s) * D : nullptr;
     s -= p.W;
-    if (p.use_hca && s < qr.len / p.m_hca) return p.hca + (sq.hca_off + s) * D;
-    return nullptr;
+    return s < kl.n_hca ? p.hca + (kl.hca_row0 + s) * D : nullptr;
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_item_base) {
     using L = Smem<D>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     Bars* bars = reinterpret_cast<Bars*>(sm + L::kBar);
-    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);  // [0] tmem base, [1] abort, [2..9] masks
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);  // [0] tmem base, [1] abort, [2..5] masks
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     uint16_t* mask16 = reinterpret_cast<uint16_t*>(misc + 2);     // [stage][4 warps]
     const uint32_t sbase = smem_u32(sm);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qi = blockIdx.y, item = blockIdx.x;
+    const int qi = blockIdx.y, item = blockIdx.x + p_item_base;
+    // The query table and sequence lengths come from kernels at least two launches back, which are
+    // complete once this grid runs (every kernel of the chain waits before it lets the next start).
     const csa_query qr = p.queries[qi];
     const csa_seq sq = p.seqs[qr.seq];
     const bool qvalid = qr.len >= 1 && qr.len <= sq.len;
-    const int64_t n_keys = (int64_t)p.k_slots + p.W + ((p.use_hca && qvalid) ? qr.len / p.m_hca : 0);
-    const int64_t s0 = (int64_t)item * p.keys_per_item;
-    int64_t s1 = min(n_keys, s0 + p.keys_per_item);
+    KeyList kl;
+    kl.idx = p.idx ? p.idx + (int64_t)qi * p.k_slots : nullptr;
+    kl.n_causal = qr.len / p.m;
+    kl.n_hca = (p.use_hca && qvalid) ? qr.len / p.m_hca : 0;
+    kl.nw = qr.len < p.W ? qr.len : p.W;
+    kl.win_row0 = sq.tok_off + qr.len - kl.nw;
+    kl.csa_row0 = sq.csa_off;
+    kl.hca_row0 = sq.hca_off;
+    const int64_t front = (int64_t)p.k_slots + p.W;
+    const int64_t n_keys = front + kl.n_hca;
+    int64_t s0, s1;
+    if (p.n_items == 1) {
+        s0 = 0;
+        s1 = n_keys;
+    } else if (item < p.items_front) {
+        s0 = (int64_t)item * p.kpi_front;
+        s1 = min(front, s0 + p.kpi_front);
+    } else {
+        s0 = front + (int64_t)(item - p.items_front) * p.kpi_hca;
+        s1 = min(n_keys, s0 + p.kpi_hca);
+    }
     if (s1 < s0) s1 = s0;
     if (!qvalid) {
         if (threadIdx.x == 0 && item == 0) report(p.status, CSA_ERR_INDEX);
@@ -123,8 +148,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
         mbar_init(&bars->empty[1], 1);
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->s_free, 128);
-        mbar_init(&bars->p_full, 128);
-        mbar_init(&bars->o_done, 1);
+        mbar_init(&bars->p_full[0], 128);
+        mbar_init(&bars->p_full[1], 128);
+        mbar_init(&bars->o_done[0], 1);
+        mbar_init(&bars->o_done[1], 1);
         mbar_init(&bars->fin, 1);
         misc[1] = 0;
         fence_mbar_init();
@@ -144,24 +171,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
         const uint64_t* rowptr = reinterpret_cast<const uint64_t*>(sm + L::kRowPtr) + lw * 16;
         uint64_t* rowptr_w = reinterpret_cast<uint64_t*>(sm + L::kRowPtr) + lw * 16;
         constexpr int CPR = D / 8;  // 16-byte chunks per row
+        if (T > 0) {
+            // Q: 64 (padded) heads, 16 per loader warp; an input, so it may load before the wait
+            for (int e = lane; e < 16 * CPR; e += 32) {
+                const int h = lw * 16 + e / CPR, ch = e % CPR;
+                const bool ok = h < p.H;
+                const uint16_t* src = ok ? p.q + ((int64_t)qi * p.H + h) * D + ch * 8 : p.q;
+                const uint32_t dst = sbase + L::kQ + (ch >> 3) * L::kBlock + sw128_offset(h, ch & 7);
+                cp_async16(dst, src, ok ? 16u : 0u);
+            }
+        }
+        grid_dep_wait();  // the selected indices come from the previous kernel
         for (int t = 0; t < T; ++t) {
             const int st = t & 1;
             if (t >= 2 && !mbar_wait(&bars->empty[st], ((t >> 1) - 1) & 1, p.status, abort_flag)) break;
-            if (t == 0) {
-                // Q: 64 (padded) heads, 16 per loader warp
-                for (int e = lane; e < 16 * CPR; e += 32) {
-                    const int h = lw * 16 + e / CPR, ch = e % CPR;
-                    const bool ok = h < p.H;
-                    const uint16_t* src = ok ? p.q + ((int64_t)qi * p.H + h) * D + ch * 8 : p.q;
-                    const uint32_t dst = sbase + L::kQ + (ch >> 3) * L::kBlock + sw128_offset(h, ch & 7);
-                    cp_async16(dst, src, ok ? 16u : 0u);
-                }
-            }
             const int64_t tb = s0 + (int64_t)t * kTileKeys;
             bool valid = false;
             if (lane < 16) {
                 const int64_t s = tb + lw * 16 + lane;
-                const uint16_t* r = s < s1 ? key_row(p, D, qi, qr, sq, s) : nullptr;
+                const uint16_t* r = s < s1 ? key_row(p, D, kl, s) : nullptr;
                 rowptr_w[lane] = reinterpret_cast<uint64_t>(r);
                 valid = r != nullptr;
             }
@@ -184,34 +212,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
         cp_async_wait_all();
     } else if (warp == 8) {
         // ------------------------------------------------------------------ MMA issuer
+        grid_dep_wait();
         if (lane == 0 && T > 0) {
             constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
             constexpr int N2 = D >= 256 ? 256 : D;
+            constexpr int HALVES = D >= 256 ? D / 256 : 1;
             constexpr uint32_t id2 = idesc_bf16(64, N2, false, true);
             const uint32_t tS = tmem + kColS;
+            // descriptor bases; the start address field is (address >> 4) in the low bits
+            const uint64_t dQ = sdesc_kmajor(sbase + L::kQ);
+            const uint64_t dK[2] = {sdesc_kmajor(sbase + L::kK0), sdesc_kmajor(sbase + L::kK1)};
+            const uint64_t dV[2] = {sdesc_mnmajor(sbase + L::kK0, L::kBlock), sdesc_mnmajor(sbase + L::kK1, L::kBlock)};
+            const uint64_t dP[2] = {sdesc_kmajor(sbase + L::kP0), sdesc_kmajor(sbase + L::kP1)};
             auto gemm1 = [&](int t) {
-                const uint32_t kb0 = sbase + ((t & 1) ? L::kK1 : L::kK0);
+                const uint64_t kd = dK[t & 1];
 #pragma unroll 1
                 for (int kb = 0; kb < L::NKB; ++kb) {
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t a = sdesc_kmajor(sbase + L::kQ + kb * L::kBlock + ks * 32);
-                        const uint64_t b = sdesc_kmajor(kb0 + kb * L::kBlock + ks * 32);
-                        umma_bf16(tS, a, b, id1, (kb | ks) != 0);
+                        const uint64_t off = (uint64_t)((kb * L::kBlock + ks * 32) >> 4);
+                        umma_bf16(tS, dQ + off, kd + off, id1, (kb | ks) != 0);
                     }
                 }
             };
             auto gemm2 = [&](int t) {
-                const uint32_t kb0 = sbase + ((t & 1) ? L::kK1 : L::kK0);
+                const uint64_t vd = dV[t & 1], pd = dP[t & 1];
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a = sdesc_kmajor(sbase + L::kP + ks * 32);
 #pragma unroll
-                    for (int half = 0; half < (D >= 256 ? D / 256 : 1); ++half) {
+                    for (int half = 0; half < HALVES; ++half) {
                         // V rows ks*16 .. ks*16+15 of the key tile, dims [half*256, half*256 + N2)
-                        const uint64_t b = sdesc_mnmajor(kb0 + half * 4 * L::kBlock + ks * 16 * 128, L::kBlock);
+                        const uint64_t b = vd + (uint64_t)((half * 4 * L::kBlock + ks * 16 * 128) >> 4);
                         const uint32_t tO = tmem + kColO + ((uint32_t)(half * 16) << 16);
-                        umma_bf16(tO, a, b, id2, (t > 0 || ks > 0) ? 1u : 0u);
+                        umma_bf16(tO, pd + (uint64_t)((ks * 32) >> 4), b, id2, (t > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
             };
@@ -230,12 +263,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
                     gemm1(t + 1);
                     umma_commit(&bars->s_full);
                 }
-                ok = mbar_wait(&bars->p_full, t & 1, p.status, abort_flag);
+                ok = mbar_wait(&bars->p_full[t & 1], (t >> 1) & 1, p.status, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 gemm2(t);
                 umma_commit(&bars->empty[t & 1]);
-                umma_commit(&bars->o_done);
+                umma_commit(&bars->o_done[t & 1]);
             }
             umma_commit(&bars->fin);
             mbar_wait(&bars->fin, 0, p.status, nullptr);
@@ -243,10 +276,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ softmax + epilogue
+        grid_dep_wait();
+        grid_dep_launch();
         const int i = lane;
         const bool row_thread = i < 16;
         const int h = warp * 16 + (i & 15);                 // head row handled by this lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        constexpr int OC = D >= 256 ? 256 : D;              // O columns held by each lane
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int t = 0; t < T; ++t) {
@@ -257,14 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
             tc_fence_after();
             float s[64];
             {
-                uint32_t r[16];
+                uint32_t r[4][16];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    tmem_ld16(tmem + lane_base + kColS + q4 * 16, r);
-                    tmem_ld_wait();
+                for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tmem + lane_base + kColS + q4 * 16, r[q4]);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) s[q4 * 16 + j] = __uint_as_float(r[j]);
-                }
+                for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) s[q4 * 16 + j] = __uint_as_float(r[q4][j]);
             }
             tc_fence_before();
             mbar_arrive(&bars->s_free);
@@ -283,32 +319,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
                 m_run = mx;
                 l_run *= alpha;
             }
-            // P buffer and O are free once the previous P.V finished
-            if (t > 0) {
-                ok = mbar_wait(&bars->o_done, (t - 1) & 1, p.status, abort_flag);
+            // O must hold every earlier P.V before it is rescaled (rare)
+            const bool any = __any_sync(0xffffffffu, row_thread && alpha != 1.f);
+            if (t > 0 && any) {
+                ok = mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                // rescale O rows whose reference max moved (warp-collective TMEM access)
-                const float a_lo = __shfl_sync(0xffffffffu, alpha, i & 15);
-                const float a_me = row_thread ? alpha : a_lo;
-                const bool any = __any_sync(0xffffffffu, row_thread && alpha != 1.f);
-                if (any) {
-                    constexpr int OC = D >= 256 ? 256 : D;
+                const float a_me = __shfl_sync(0xffffffffu, alpha, i & 15);
 #pragma unroll 1
-                    for (int c = 0; c < OC; c += 16) {
-                        uint32_t r[16];
-                        tmem_ld16(tmem + lane_base + kColO + c, r);
-                        tmem_ld_wait();
+                for (int c = 0; c < OC; c += 64) {
+                    uint32_t r[4][16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * a_me);
-                        tmem_st16(tmem + lane_base + kColO + c, r);
+                    for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tmem + lane_base + kColO + c + q4 * 16, r[q4]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) r[q4][j] = __float_as_uint(__uint_as_float(r[q4][j]) * a_me);
+                        tmem_st16(tmem + lane_base + kColO + c + q4 * 16, r[q4]);
                     }
-                    tmem_st_wait();
                 }
+                tmem_st_wait();
+            }
+            // P buffer t&1 is free once the P.V of tile t-2 finished
+            if (t >= 2) {
+                ok = mbar_wait(&bars->o_done[st], ((t >> 1) - 1) & 1, p.status, abort_flag);
+                if (!ok) break;
             }
             if (row_thread) {
                 float lsum = 0.f;
-                unsigned char* prow = sm + L::kP;
+                unsigned char* prow = sm + (st ? L::kP1 : L::kP0);
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     uint32_t w4[4];
@@ -325,15 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            mbar_arrive(&bars->p_full[st]);
         }
         // ---- epilogue
-        if (ok && T > 0) ok = mbar_wait(&bars->o_done, (T - 1) & 1, p.status, abort_flag);
+        if (ok && T > 0) ok = mbar_wait(&bars->o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, p.status, abort_flag);
         const float l_row = __shfl_sync(0xffffffffu, l_run, i & 15);
         const float m_row = __shfl_sync(0xffffffffu, m_run, i & 15);
         const bool has = ok && T > 0 && l_row > 0.f;
         const float inv = has ? 1.f / l_row : 0.f;
-        constexpr int OC = D >= 256 ? 256 : D;
         const int dim0 = row_thread ? 0 : 256;
         const bool writes = (row_thread || D >= 512) && h < p.H;
         float* orow = direct ? p.out + ((int64_t)qi * p.H + h) * D
@@ -341,22 +380,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
         if (has) tc_fence_after();
         if (has || direct) {
 #pragma unroll 1
-            for (int c = 0; c < OC; c += 16) {
-                uint32_t r[16];
+            for (int c = 0; c < OC; c += 64) {
+                uint32_t r[4][16];
                 if (has) {
-                    tmem_ld16(tmem + lane_base + kColO + c, r);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tmem + lane_base + kColO + c + q4 * 16, r[q4]);
                     tmem_ld_wait();
                 }
                 if (writes) {
 #pragma unroll
-                    for (int j = 0; j < 16; j += 4) {
-                        float4 v;
-                        v.x = has ? __uint_as_float(r[j]) * inv : 0.f;
-                        v.y = has ? __uint_as_float(r[j + 1]) * inv : 0.f;
-                        v.z = has ? __uint_as_float(r[j + 2]) * inv : 0.f;
-                        v.w = has ? __uint_as_float(r[j + 3]) * inv : 0.f;
-                        *reinterpret_cast<float4*>(orow + dim0 + c + j) = v;
-                    }
+                    for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+                        for (int j = 0; j < 16; j += 4) {
+                            float4 v;
+                            v.x = has ? __uint_as_float(r[q4][j]) * inv : 0.f;
+                            v.y = has ? __uint_as_float(r[q4][j + 1]) * inv : 0.f;
+                            v.z = has ? __uint_as_float(r[q4][j + 2]) * inv : 0.f;
+                            v.w = has ? __uint_as_float(r[q4][j + 3]) * inv : 0.f;
+                            *reinterpret_cast<float4*>(orow + dim0 + c + q4 * 16 + j) = v;
+                        }
                 }
             }
         }
@@ -378,48 +420,67 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p) {
 }
 
 // out[q][h] = sum_items exp(lse_i - lse) * O_i,  lse = logsumexp_i lse_i  (items with lse = -inf
-// contribute nothing and are not read).
+// contribute nothing and are not read).  One CTA per (head, query); warp 0 computes the weights, then
+// every thread accumulates one float4 column of all contributing partials with batched loads.
 template <int D>
 __global__ void combine_kernel(AttnParams p) {
     const int h = blockIdx.x, qi = blockIdx.y;
     const int n_items = p.n_items;
     __shared__ float wts[256];
-    __shared__ float s_lse;
-    if (threadIdx.x == 0) {
+    __shared__ int used[256];
+    __shared__ int n_used;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
         float mx = -INFINITY;
-        for (int it = 0; it < n_items; ++it)
+        for (int it = lane; it < n_items; it += 32)
             mx = fmaxf(mx, p.part_lse[((int64_t)qi * n_items + it) * kHeadsPad + h]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float sum = 0.f;
-        for (int it = 0; it < n_items; ++it) {
+        for (int it = lane; it < n_items; it += 32) {
             const float l = p.part_lse[((int64_t)qi * n_items + it) * kHeadsPad + h];
             const float w = mx == -INFINITY ? 0.f : expf(l - mx);
             wts[it] = w;
             sum += w;
         }
-        const float lse = mx == -INFINITY ? -INFINITY : mx + logf(sum);
-        for (int it = 0; it < n_items; ++it) wts[it] = sum > 0.f ? wts[it] / sum : 0.f;
-        s_lse = lse;
-        if (p.lse) p.lse[(int64_t)qi * p.H + h] = lse;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        __syncwarp();
+        if (lane == 0) {
+            int nu = 0;
+            for (int it = 0; it < n_items; ++it)
+                if (wts[it] > 0.f) { wts[nu] = wts[it] / sum; used[nu] = it; ++nu; }
+            n_used = nu;
+            if (p.lse) p.lse[(int64_t)qi * p.H + h] = mx == -INFINITY ? -INFINITY : mx + logf(sum);
+        }
     }
     __syncthreads();
+    const int nu = n_used;
     for (int c = threadIdx.x * 4; c < D; c += blockDim.x * 4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int it = 0; it < n_items; ++it) {
-            const float w = wts[it];
-            if (w == 0.f) continue;
-            const float4 v = *reinterpret_cast<const float4*>(
-                p.part_o + (((int64_t)qi * n_items + it) * kHeadsPad + h) * D + c);
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
+        for (int b = 0; b < nu; b += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (b + u < nu)
+                    v[u] = __ldcg(reinterpret_cast<const float4*>(
+                        p.part_o + (((int64_t)qi * n_items + used[b + u]) * kHeadsPad + h) * D + c));
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (b + u < nu) {
+                    const float w = wts[b + u];
+                    acc.x = fmaf(w, v[u].x, acc.x);
+                    acc.y = fmaf(w, v[u].y, acc.y);
+                    acc.z = fmaf(w, v[u].z, acc.z);
+                    acc.w = fmaf(w, v[u].w, acc.w);
+                }
         }
         *reinterpret_cast<float4*>(p.out + ((int64_t)qi * p.H + h) * D + c) = acc;
     }
 }
 
 template <int D>
-cudaError_t launch_d(AttnParams& p, cudaStream_t stream) {
+cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, cudaStream_t stream, bool pdl) {
     using L = Smem<D>;
     static bool attr = false;
     if (!attr) {
@@ -427,12 +488,8 @@ cudaError_t launch_d(AttnParams& p, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    const int n_items = p.n_items;
-    attn_kernel<D><<<dim3((unsigned)n_items, (unsigned)p.Q), kThreads, L::kAlloc, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || n_items == 1) return e;
-    combine_kernel<D><<<dim3((unsigned)p.H, (unsigned)p.Q), D / 4, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(attn_kernel<D>, dim3((unsigned)item_count, (unsigned)p.Q), dim3(kThreads), L::kAlloc, stream,
+                         pdl, p, item_begin);
 }
 
 }  // namespace
@@ -444,16 +501,28 @@ size_t attn_ws_bytes(int Q, int items, int d) {
     return ((o + 255) & ~(size_t)255) + ((l + 255) & ~(size_t)255);
 }
 
-cudaError_t launch_attention(AttnParams& p, void* ws, cudaStream_t stream) {
-    const int n_items = p.n_items;
-    if (n_items > 1) {
-        const size_t o = (size_t)p.Q * n_items * kHeadsPad * p.d * 4;
+void attn_ws_carve(AttnParams& p, void* ws) {
+    if (p.n_items > 1) {
+        const size_t o = (size_t)p.Q * p.n_items * kHeadsPad * p.d * 4;
         p.part_o = static_cast<float*>(ws);
         p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + ((o + 255) & ~(size_t)255));
     }
-    if (p.d == 512) return launch_d<512>(p, stream);
-    if (p.d == 128) return launch_d<128>(p, stream);
+}
+
+cudaError_t launch_attention_items(const AttnParams& p, int item_begin, int item_count, cudaStream_t stream,
+                                   bool pdl) {
+    if (item_count <= 0) return cudaSuccess;
+    if (p.d == 512) return launch_items_d<512>(p, item_begin, item_count, stream, pdl);
+    if (p.d == 128) return launch_items_d<128>(p, item_begin, item_count, stream, pdl);
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_combine(const AttnParams& p, cudaStream_t stream) {
+    if (p.n_items <= 1) return cudaSuccess;
+    if (p.d == 512) combine_kernel<512><<<dim3((unsigned)p.H, (unsigned)p.Q), 128, 0, stream>>>(p);
+    else if (p.d == 128) combine_kernel<128><<<dim3((unsigned)p.H, (unsigned)p.Q), 32, 0, stream>>>(p);
+    else return cudaErrorInvalidValue;
+    return cudaGetLastError();
 }
 
 }  // namespace csa

@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <mutex>
 #include <string>
 
 #include "compress_dev.cuh"
@@ -71,15 +72,46 @@ int env_int(const char* name, int dflt) {
     return v ? atoi(v) : dflt;
 }
 
-// Keys per attention item: about 128 items over all queries, a multiple of 64 (one tile).
-int pick_keys_per_item(int64_t total_keys) {
+int round64(int64_t v) { return (int)(((v + 63) / 64) * 64); }
+
+int clamp_kpi(int64_t v, int lo, int hi) {
+    int64_t r = ((v + 63) / 64) * 64;
+    if (r < lo) r = lo;
+    if (r > hi) r = hi;
+    return (int)r;
+}
+
+// How one query's key list [front = CSA slots + window | HCA entries] is cut into attention items.
+struct ItemPlan {
+    int n_items, items_front, kpi_front, kpi_hca;
+};
+
+ItemPlan make_items(int64_t front_keys, int64_t max_hca, int kpi_front, int kpi_hca) {
+    ItemPlan ip{};
+    ip.kpi_front = kpi_front;
+    ip.kpi_hca = kpi_hca;
+    ip.items_front = front_keys > 0 ? (int)((front_keys + kpi_front - 1) / kpi_front) : 0;
+    const int ih = max_hca > 0 ? (int)((max_hca + kpi_hca - 1) / kpi_hca) : 0;
+    ip.n_items = ip.items_front + ih;
+    if (ip.n_items < 1) ip.n_items = 1;  // an empty list: one empty item writing out = 0, lse = -inf
+    return ip;
+}
+
+// Standalone calls: about 128 CTAs over all queries.
+ItemPlan plan_standalone(int64_t front_keys, int64_t max_hca, int Q) {
     const int forced = env_int("CSA_KEYS_PER_ITEM", 0);
-    if (forced > 0) return ((forced + 63) / 64) * 64;
-    int64_t kpi = (total_keys + 127) / 128;
-    kpi = ((kpi + 63) / 64) * 64;
-    if (kpi < 128) kpi = 128;
-    if (kpi > 2048) kpi = 2048;
-    return (int)kpi;
+    const int64_t total = (front_keys + max_hca) * (int64_t)Q;
+    const int kpi = forced > 0 ? round64(forced) : clamp_kpi((total + 127) / 128, 128, 2048);
+    return make_items(front_keys, max_hca, kpi, kpi);
+}
+
+// Decode: small front items (they run after the top-k, on the critical path) and about 40 HCA
+// items over all queries (they run alongside the indexer scan).
+ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh) {
+    const int f = env_int("CSA_KPI_FRONT", 0), h = env_int("CSA_KPI_HCA", 0);
+    const int kpi_front = f > 0 ? round64(f) : 128;
+    const int kpi_hca = h > 0 ? round64(h) : clamp_kpi(((int64_t)B * max_eh + 39) / 40, 128, 4096);
+    return make_items((int64_t)d.k + d.W, max_eh, kpi_front, kpi_hca);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -87,6 +119,7 @@ int pick_keys_per_item(int64_t total_keys) {
 // new token completes, publish the query table, clear this query's index scratch words.
 // ---------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+    grid_dep_launch();  // the scan may start its launch; it waits for this grid before reading
     const int b = blockIdx.x;
     __shared__ int64_t s_len;
     if (threadIdx.x == 0) {
@@ -140,7 +173,7 @@ struct DecodePlan {
     int64_t max_e;        // max CSA entries
     int64_t max_eh;       // max HCA entries
     int64_t e_stride;
-    int kpi, n_items;
+    ItemPlan items;
     size_t off_queries, off_idx, off_index, off_attn, total;
 };
 
@@ -150,9 +183,7 @@ DecodePlan plan_decode(const csa_dims& d, int B, int64_t max_len) {
     pl.max_eh = max_len / d.m_hca;
     pl.e_stride = ((pl.max_e + 3) / 4) * 4;
     if (pl.e_stride < 4) pl.e_stride = 4;
-    const int64_t per_q = (int64_t)d.k + d.W + pl.max_eh;
-    pl.kpi = pick_keys_per_item(per_q * B);
-    pl.n_items = (int)((per_q + pl.kpi - 1) / pl.kpi);
+    pl.items = plan_decode_items(d, B, pl.max_eh);
     size_t off = 0;
     pl.off_queries = off;
     off += align256((size_t)B * sizeof(csa_query));
@@ -161,7 +192,7 @@ DecodePlan plan_decode(const csa_dims& d, int B, int64_t max_len) {
     pl.off_index = off;
     off += index_ws_bytes(B, pl.e_stride);
     pl.off_attn = off;
-    off += attn_ws_bytes(B, pl.n_items, d.d);
+    off += attn_ws_bytes(B, pl.items.n_items, d.d);
     pl.total = off;
     return pl;
 }
@@ -169,7 +200,6 @@ DecodePlan plan_decode(const csa_dims& d, int B, int64_t max_len) {
 struct PrefillPlan {
     int64_t qc;           // queries per chunk
     int64_t e_stride;
-    int kpi;
     size_t off_queries, off_idx, off_index, total;
 };
 
@@ -180,8 +210,6 @@ PrefillPlan plan_prefill(const csa_dims& d, int64_t q_end) {
     if (pl.e_stride < 4) pl.e_stride = 4;
     pl.qc = env_int("CSA_PREFILL_CHUNK", 2048);
     if (pl.qc < 1) pl.qc = 1;
-    const int64_t keys = (int64_t)d.k + d.W + q_end / d.m_hca;
-    pl.kpi = (int)(((keys + 63) / 64) * 64);
     size_t off = 0;
     pl.off_queries = off;
     off += align256((size_t)pl.qc * sizeof(csa_query));
@@ -209,10 +237,36 @@ int status_ptr(int** out) {
     return CSA_OK;
 }
 
+// Helper stream + fork/join events of hybrid_attn_decode, one set per device, created on the first
+// decode call on that device (not device memory).
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+int side_stream(SideStream** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(CSA_ERR_CUDA, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStream& ss = g_side[dev];
+    if (!ss.s) {
+        if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess ||
+            (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "helper stream");
+    }
+    *out = &ss;
+    return CSA_OK;
+}
+
 int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_e,
               int64_t e_stride, const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
               float* score_out, void* ws_index, bool zero_ws, int* status, cudaStream_t stream,
-              cudaEvent_t mid = nullptr) {
+              cudaEvent_t mid = nullptr, bool pdl = false) {
     IndexParams ip{};
     ip.seqs = seqs;
     ip.queries = queries;
@@ -229,7 +283,7 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
     ip.score_out = score_out;
     ip.status = status;
     index_ws_carve(ip, ws_index, Q, e_stride);
-    cudaError_t e = launch_index_topk(ip, max_e, stream, zero_ws, mid);
+    cudaError_t e = launch_index_topk(ip, max_e, stream, zero_ws, mid, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "index_topk launch");
     return CSA_OK;
 }
@@ -341,11 +395,10 @@ size_t csa_workspace_size(int op, const void* args) {
             if (es < 4) es = 4;
             return index_ws_bytes(a->Q, es) + 256;
         }
-        const int64_t keys = op == CSA_OP_SPARSE_ATTN ? (int64_t)a->dims.k + a->dims.W
-                                                      : a->max_len / a->dims.m_hca + a->dims.W;
-        const int kpi = pick_keys_per_item(keys * a->Q);
-        const int items = (int)((keys + kpi - 1) / kpi);
-        return attn_ws_bytes(a->Q, items < 1 ? 1 : items, a->dims.d) + 256;
+        const ItemPlan ip = op == CSA_OP_SPARSE_ATTN
+                                ? plan_standalone((int64_t)a->dims.k + a->dims.W, 0, a->Q)
+                                : plan_standalone(a->dims.W, a->max_len / a->dims.m_hca, a->Q);
+        return attn_ws_bytes(a->Q, ip.n_items, a->dims.d) + 256;
     }
     if (op == CSA_OP_DECODE) {
         const csa_decode_args* a = static_cast<const csa_decode_args*>(args);
@@ -381,14 +434,15 @@ int csa_index_topk(const csa_dims* dims, const csa_seq* seqs, const csa_query* q
                      stream);
 }
 
-static int run_attention(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q,
-                         const csa_bf16* q, const csa_bf16* entries, const int32_t* idx, int k_slots, const csa_bf16* x,
-                         int W, const csa_bf16* hca, float scale, float* out, float* lse, void* ws, int kpi,
-                         int n_items, cudaStream_t stream) {
+static int make_attn(AttnParams& p, const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q,
+                     const csa_bf16* q, const csa_bf16* entries, const int32_t* idx, int k_slots, const csa_bf16* x,
+                     int W, const csa_bf16* hca, float scale, float* out, float* lse, void* ws, const ItemPlan& ip) {
     int* st = nullptr;
     int rc = status_ptr(&st);
     if (rc) return rc;
-    AttnParams p{};
+    if (ip.n_items < 1 || ip.n_items > 256)
+        return fail(CSA_ERR_UNSUPPORTED, "%d attention items per query (1..256)", ip.n_items);
+    p = AttnParams{};
     p.seqs = seqs;
     p.queries = queries;
     p.Q = Q;
@@ -405,13 +459,20 @@ static int run_attention(const csa_dims* dims, const csa_seq* seqs, const csa_qu
     p.m_hca = dims->m_hca;
     p.use_hca = hca != nullptr;
     p.scale_log2 = scale * 1.4426950408889634f;
-    p.keys_per_item = kpi;
-    p.n_items = n_items;
+    p.n_items = ip.n_items;
+    p.items_front = ip.items_front;
+    p.kpi_front = ip.kpi_front;
+    p.kpi_hca = ip.kpi_hca;
     p.out = out;
     p.lse = lse;
     p.status = st;
-    if (n_items < 1 || n_items > 256) return fail(CSA_ERR_UNSUPPORTED, "%d attention items per query (1..256)", n_items);
-    cudaError_t e = launch_attention(p, ws, stream);
+    attn_ws_carve(p, ws);
+    return CSA_OK;
+}
+
+static int run_attention_all(const AttnParams& p, cudaStream_t stream) {
+    cudaError_t e = launch_attention_items(p, 0, p.n_items, stream);
+    if (e == cudaSuccess) e = launch_combine(p, stream);
     return e == cudaSuccess ? CSA_OK : cuda_fail(e, "attention launch");
 }
 
@@ -428,11 +489,11 @@ int csa_sparse_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* 
     const size_t need = csa_workspace_size(CSA_OP_SPARSE_ATTN, &wq);
     if (need > 256 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)))
         return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", need);
-    const int64_t keys = (int64_t)dims->k + dims->W;
-    const int kpi = pick_keys_per_item(keys * Q);
-    const int items = (int)((keys + kpi - 1) / kpi);
-    return run_attention(dims, seqs, queries, Q, q, entries, idx, dims->k, x, dims->W, nullptr, scale, out, lse, ws,
-                         kpi, items, stream);
+    AttnParams p;
+    int rc2 = make_attn(p, dims, seqs, queries, Q, q, entries, idx, dims->k, x, dims->W, nullptr, scale, out, lse, ws,
+                        plan_standalone((int64_t)dims->k + dims->W, 0, Q));
+    if (rc2) return rc2;
+    return run_attention_all(p, stream);
 }
 
 int hca_dense_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
@@ -451,12 +512,11 @@ int hca_dense_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* q
     if (need > 256 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)))
         return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", need);
     // key list: [raw window | HCA entries] (no CSA slots)
-    const int64_t keys = max_len / dims->m_hca + W;
-    const int kpi = pick_keys_per_item(keys * Q);
-    int items = (int)((keys + kpi - 1) / kpi);
-    if (items < 1) items = 1;
-    return run_attention(&d2, seqs, queries, Q, q, nullptr, nullptr, 0, x, W, hca_entries, scale, out, lse, ws, kpi,
-                         items, stream);
+    AttnParams p;
+    int rc2 = make_attn(p, &d2, seqs, queries, Q, q, nullptr, nullptr, 0, x, W, hca_entries, scale, out, lse, ws,
+                        plan_standalone(W, max_len / dims->m_hca, Q));
+    if (rc2) return rc2;
+    return run_attention_all(p, stream);
 }
 
 int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
@@ -509,13 +569,42 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     if (e == cudaSuccess) e = launch_append(ap, stream);
     if (e == cudaSuccess) e = mark(ev[1], stream);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    AttnParams ap2;
+    rc = make_attn(ap2, &d, a->seqs, queries, a->B, a->q, a->entries, idx, d.k, a->x, d.W, a->hca_entries, a->scale,
+                   a->out, a->lse, w + pl.off_attn, pl.items);
+    if (rc) return rc;
+    const int n_front = pl.items.n_items == 1 ? 1 : pl.items.items_front;
+    const int n_hca = pl.items.n_items - n_front;
+    // The HCA items do not depend on the top-k: they run on a helper stream while the indexer
+    // scans, joined back before the merge.
+    SideStream* side = nullptr;
+    if (n_hca > 0 && (rc = side_stream(&side))) return rc;
+    std::unique_lock<std::mutex> lock(g_side_mu, std::defer_lock);
+    if (side) {
+        lock.lock();
+        if ((e = cudaEventRecord(side->fork, stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess ||
+            (e = launch_attention_items(ap2, n_front, n_hca, side->s)) != cudaSuccess ||
+            (e = cudaEventRecord(side->join, side->s)) != cudaSuccess)
+            return cuda_fail(e, "HCA attention launch");
+    }
+    // programmatic dependent launch chains append -> scan -> select -> attention unless stage
+    // events are being recorded between them
+    const bool pdl = ev[0] == nullptr && env_int("CSA_NO_PDL", 0) == 0;
     rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
-                   ws_index, false, st, stream, ev[2]);
-    if (rc) return rc;
+                   ws_index, false, st, stream, ev[2], pdl && !side);
+    if (rc) {
+        if (side) cudaStreamWaitEvent(stream, side->join, 0);  // keep the capture / stream joined
+        return rc;
+    }
     if ((e = mark(ev[3], stream)) != cudaSuccess) return cuda_fail(e, "event record");
-    rc = run_attention(&d, a->seqs, queries, a->B, a->q, a->entries, idx, d.k, a->x, d.W, a->hca_entries, a->scale,
-                       a->out, a->lse, w + pl.off_attn, pl.kpi, pl.n_items, stream);
-    if (rc) return rc;
+    e = launch_attention_items(ap2, 0, n_front, stream, pdl);
+    if (side) {
+        cudaError_t e2 = cudaStreamWaitEvent(stream, side->join, 0);
+        if (e == cudaSuccess) e = e2;
+    }
+    if (e == cudaSuccess) e = launch_combine(ap2, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     if ((e = mark(ev[4], stream)) != cudaSuccess) return cuda_fail(e, "event record");
     return CSA_OK;
 }
@@ -584,10 +673,13 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
         rc = run_index(d, a->seq, queries, (int)n, max_e, pl.e_stride, a->q_idx + r0 * d.H_I * d.d_I,
                        a->w + r0 * d.H_I, a->entry_keys, idx, nullptr, w + pl.off_index, true, st, stream);
         if (rc) return rc;
-        rc = run_attention(&d, a->seq, queries, (int)n, a->q + r0 * d.H * d.d, a->entries, idx, d.k, a->x, d.W,
-                           a->hca_entries, a->scale, a->out + r0 * d.H * d.d, a->lse ? a->lse + r0 * d.H : nullptr,
-                           nullptr, pl.kpi, 1, stream);
+        AttnParams pp;
+        ItemPlan one{1, 0, 64, 64};
+        rc = make_attn(pp, &d, a->seq, queries, (int)n, a->q + r0 * d.H * d.d, a->entries, idx, d.k, a->x, d.W,
+                       a->hca_entries, a->scale, a->out + r0 * d.H * d.d, a->lse ? a->lse + r0 * d.H : nullptr, nullptr,
+                       one);
         if (rc) return rc;
+        if ((rc = run_attention_all(pp, stream))) return rc;
     }
     return CSA_OK;
 }

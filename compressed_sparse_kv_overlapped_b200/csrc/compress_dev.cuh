@@ -21,11 +21,13 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 
 // Channels [c0, c0+8) of entry j of one sequence (token rows start at tok0), written as bf16 to
 // out_row (+ c0) and, when key_row != nullptr, the indexer key channels to key_row (+ c0).
-// An online softmax over the window in fp32: one pass, one 16-byte load per operand per token.
+// An online softmax over the window in fp32.  Tokens are taken 4 at a time: the loads of a batch
+// are all issued before its softmax updates, so a 128-token window costs 32 memory round trips.
 __device__ __forceinline__ void compress_entry8(int64_t j, int m, int win, int d, int d_I, int c0,
                                                 const uint16_t* x, const uint16_t* logit, const float* bias,
                                                 const uint16_t* idx_key, int64_t tok0, uint16_t* out_row,
                                                 uint16_t* key_row) {
+    constexpr int kBatch = 4;
     const int64_t start = (int64_t)m * j - (win - m);
     const int64_t t0 = start < 0 ? 0 : start;
     const int64_t t1 = (int64_t)m * j + m;
@@ -33,34 +35,43 @@ __device__ __forceinline__ void compress_entry8(int64_t j, int m, int win, int d
     float mx[8], den[8], acc[8], acck[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) { mx[i] = -INFINITY; den[i] = 0.f; acc[i] = 0.f; acck[i] = 0.f; }
-    for (int64_t t = t0; t < t1; ++t) {
-        const int64_t row = tok0 + t;
-        const uint4 lv = __ldg(reinterpret_cast<const uint4*>(logit + row * d + c0));
-        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + row * d + c0));
-        const float4* bp = reinterpret_cast<const float4*>(bias + (t - start) * d + c0);
-        const float4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
-        float z[8], xf[8], kf[8];
-        unpack8(lv, z);
-        unpack8(xv, xf);
-        z[0] += b0.x; z[1] += b0.y; z[2] += b0.z; z[3] += b0.w;
-        z[4] += b1.x; z[5] += b1.y; z[6] += b1.z; z[7] += b1.w;
-        if (want_key) {
-            const uint4 kv = __ldg(reinterpret_cast<const uint4*>(idx_key + row * d_I + c0));
-            unpack8(kv, kf);
+    for (int64_t tb = t0; tb < t1; tb += kBatch) {
+        uint4 lv[kBatch], xv[kBatch], kv[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int64_t t = tb + u;
+            if (t < t1) {
+                const int64_t row = tok0 + t;
+                lv[u] = __ldg(reinterpret_cast<const uint4*>(logit + row * d + c0));
+                xv[u] = __ldg(reinterpret_cast<const uint4*>(x + row * d + c0));
+                if (want_key) kv[u] = __ldg(reinterpret_cast<const uint4*>(idx_key + row * d_I + c0));
+            }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (z[i] > mx[i]) {
-                const float r = expf(mx[i] - z[i]);  // 0 on the first token (mx = -inf)
-                den[i] = den[i] * r + 1.f;
-                acc[i] = acc[i] * r + xf[i];
-                if (want_key) acck[i] = acck[i] * r + kf[i];
-                mx[i] = z[i];
-            } else {
-                const float e = expf(z[i] - mx[i]);
-                den[i] += e;
-                acc[i] = fmaf(e, xf[i], acc[i]);
-                if (want_key) acck[i] = fmaf(e, kf[i], acck[i]);
+        for (int u = 0; u < kBatch; ++u) {
+            if (tb + u >= t1) break;
+            float z[8], xf[8], kf[8];
+            unpack8(lv[u], z);
+            unpack8(xv[u], xf);
+            const float4* bp = reinterpret_cast<const float4*>(bias + (tb + u - start) * d + c0);
+            const float4 b0v = __ldg(bp), b1v = __ldg(bp + 1);  // parameters: L1/L2 resident
+            z[0] += b0v.x; z[1] += b0v.y; z[2] += b0v.z; z[3] += b0v.w;
+            z[4] += b1v.x; z[5] += b1v.y; z[6] += b1v.z; z[7] += b1v.w;
+            if (want_key) unpack8(kv[u], kf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (z[i] > mx[i]) {
+                    const float r = expf(mx[i] - z[i]);  // 0 on the first token (mx = -inf)
+                    den[i] = den[i] * r + 1.f;
+                    acc[i] = acc[i] * r + xf[i];
+                    if (want_key) acck[i] = acck[i] * r + kf[i];
+                    mx[i] = z[i];
+                } else {
+                    const float e = expf(z[i] - mx[i]);
+                    den[i] += e;
+                    acc[i] = fmaf(e, xf[i], acc[i]);
+                    if (want_key) acck[i] = fmaf(e, kf[i], acck[i]);
+                }
             }
         }
     }

@@ -91,6 +91,8 @@ template <int KV>
 __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(IndexParams p) {
     __shared__ uint32_t hist[kHistBins];
     __shared__ float sc[kScanThreads / 32][4][16];
+    grid_dep_wait();  // the query table may come from the previous kernel
+    grid_dep_launch();
     const int qi = blockIdx.y;
     const csa_query qr = p.queries[qi];
     const csa_seq sq = p.seqs[qr.seq];
@@ -166,16 +168,20 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(IndexParams p)
 
 // ---- select ----------------------------------------------------------------------------------
 
+constexpr int kSelPerThread = 8;                                   // scores per thread in the filter
+constexpr int kSelPerCta = kSelectThreads * kSelPerThread;          // 4096 entries per filter CTA
+
 __device__ __forceinline__ uint64_t composite(uint32_t key, int64_t j) {
     return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
 }
 
-// Block-wide inclusive suffix sum over kHistBins bins held in shared memory: after the call,
-// suf[b] = sum of hist[b' >= b].  Uses kSelectThreads threads, 4 bins each.
-__device__ void suffix_counts(const uint32_t* hist, uint32_t* suf, uint32_t* warp_tot) {
+// Block-wide suffix sums over kHistBins bins: suf[b] = sum of hist[b' >= b].  Thread t owns bins
+// [4*(511-t), 4*(511-t)+4), so a forward scan over threads is a suffix scan over bins.  Also finds
+// the unique bin b with suf[b] >= target > suf[b+1] (target >= 1); writes it to out[0] and
+// suf[b+1] to out[1] (out[0] = 0xFFFFFFFF if no bin qualifies).  Uses kSelectThreads threads.
+__device__ void suffix_find(const uint32_t* hist, uint32_t* suf, uint32_t* warp_tot, uint32_t target,
+                            uint32_t* out) {
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    // thread t owns bins [4*(511-t), 4*(511-t)+4) so that a forward scan over threads is a
-    // suffix scan over bins
     const int b0 = 4 * (kSelectThreads - 1 - t);
     uint32_t v[4];
     uint32_t s = 0;
@@ -184,85 +190,76 @@ __device__ void suffix_counts(const uint32_t* hist, uint32_t* suf, uint32_t* war
     uint32_t incl = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
     }
     if (lane == 31) warp_tot[warp] = incl;
+    if (t == 0) out[0] = 0xFFFFFFFFu;
     __syncthreads();
     if (warp == 0) {
         uint32_t x = lane < kSelectThreads / 32 ? warp_tot[lane] : 0u;
+#pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
         if (lane < kSelectThreads / 32) warp_tot[lane] = x;
     }
     __syncthreads();
-    const uint32_t before = (warp > 0 ? warp_tot[warp - 1] : 0u) + (incl - s);
+    const uint32_t before = (warp > 0 ? warp_tot[warp - 1] : 0u) + (incl - s);  // bins above b0+3
 #pragma unroll
-    for (int i = 0; i < 4; ++i) suf[b0 + i] = before + v[i];
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t here = before + v[i];
+        const uint32_t above = i < 3 ? before + v[i + 1] : before;
+        suf[b0 + i] = here;
+        if (here >= target && above < target) { out[0] = (uint32_t)(b0 + i); out[1] = above; }
+    }
     __syncthreads();
 }
 
-// Exact selection of the `need` largest composite keys among n candidates (all distinct, all
-// sharing the top 11 bits `top11`).  Returns the key T of the need-th largest: exactly `need`
-// candidates satisfy key >= T.  Radix passes of 8 bits over bits 52..0; the digit of each pass is
-// found by one warp with a suffix scan over the 256 digit counts.
+// Exact selection of the `need` largest composite keys among n distinct candidates that share the
+// top 11 bits `top11`.  Returns T with exactly `need` candidates >= T.  Radix passes of 11 bits over
+// bits 52..0 (counted with warp-aggregated shared-memory atomics, so equal digits do not
+// serialize); stops as soon as the chosen digit holds exactly the remaining count.
 __device__ uint64_t radix_threshold(const uint64_t* cand, bool in_global, uint32_t n, uint32_t need,
-                                    uint32_t top11, uint32_t* cnt256, uint32_t* misc) {
+                                    uint32_t top11, uint32_t* cnt, uint32_t* suf, uint32_t* misc) {
     uint64_t prefix = (uint64_t)top11 << 53;
     uint64_t mask = (uint64_t)0x7FF << 53;
     uint32_t remaining = need;
-    for (int shift = 45; shift >= -3; shift -= 8) {
+    const int lane = threadIdx.x & 31;
+    for (int shift = 42;; shift -= 11) {
         const int sh = shift < 0 ? 0 : shift;
-        const int bits = shift < 0 ? 8 + shift : 8;  // the last pass covers bits 4..0
+        const int bits = shift < 0 ? 11 + shift : 11;
         const uint32_t dmask = (1u << bits) - 1u;
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) cnt256[i] = 0;
+        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) cnt[i] = 0;
         __syncthreads();
-        for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
-            const uint64_t v = in_global ? __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i) : cand[i];
-            if ((v & mask) == prefix) atomicAdd(&cnt256[(uint32_t)(v >> sh) & dmask], 1u);
+        const uint32_t n_round = (n + 31u) & ~31u;
+        for (uint32_t i = threadIdx.x; i < n_round; i += blockDim.x) {
+            bool match = false;
+            uint32_t dg = 0;
+            if (i < n) {
+                const uint64_t v =
+                    in_global ? __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i) : cand[i];
+                match = (v & mask) == prefix;
+                dg = (uint32_t)(v >> sh) & dmask;
+            }
+            const uint32_t active = __ballot_sync(0xffffffffu, match);
+            if (match) {
+                const uint32_t peers = __match_any_sync(active, dg);
+                if (lane == __ffs(peers) - 1) atomicAdd(&cnt[dg], (uint32_t)__popc(peers));
+            }
         }
         __syncthreads();
-        if (threadIdx.x < 32) {
-            // lane l owns digits [8*(31-l), 8*(31-l)+8): a forward scan over lanes is a suffix
-            // scan over digits
-            const int lane = threadIdx.x;
-            const int d0 = 8 * (31 - lane);
-            uint32_t loc[8];
-            uint32_t s = 0;
-#pragma unroll
-            for (int i = 7; i >= 0; --i) { s += cnt256[d0 + i]; loc[i] = s; }
-            uint32_t incl = s;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const uint32_t before = incl - s;  // count of digits above this lane's range
-            // digit dg with suffix(dg) >= remaining > suffix(dg + 1); suffix is monotone
-            int found = -1;
-            uint32_t above_dg = 0;
-#pragma unroll
-            for (int i = 7; i >= 0; --i) {
-                const uint32_t suf_i = before + loc[i];
-                const uint32_t suf_next = i < 7 ? before + loc[i + 1] : before;
-                if (found < 0 && suf_i >= remaining && suf_next < remaining) { found = d0 + i; above_dg = suf_next; }
-            }
-            const uint32_t hit = __ballot_sync(0xffffffffu, found >= 0);
-            const int src = __ffs(hit) - 1;
-            const int dg = __shfl_sync(0xffffffffu, found, src);
-            const uint32_t ab = __shfl_sync(0xffffffffu, above_dg, src);
-            if (lane == 0) { misc[0] = (uint32_t)dg; misc[1] = remaining - ab; }
-        }
+        suffix_find(cnt, suf, misc, remaining, misc + 48);  // misc[0..15]: warp totals
+        const uint32_t dg = misc[48];
+        const uint32_t above = misc[49];
+        const uint32_t in_digit = cnt[dg];
         __syncthreads();
-        const uint64_t dg = misc[0];
-        remaining = misc[1];
-        prefix |= dg << sh;
+        remaining -= above;
+        prefix |= (uint64_t)dg << sh;
         mask |= (uint64_t)dmask << sh;
-        __syncthreads();
+        if (in_digit == remaining || sh == 0) return prefix;  // lower bits left at zero
     }
-    return prefix;
 }
 
 __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParams p) {
@@ -272,7 +269,10 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     uint32_t* misc = suf + kHistBins;                                  // 64
     uint64_t* cand_s = reinterpret_cast<uint64_t*>(misc + 64);         // kCandSmem
     int32_t* list = reinterpret_cast<int32_t*>(cand_s + kCandSmem);    // kMaxK (sort buffer)
-    __shared__ uint32_t s_last;
+    __shared__ uint32_t s_last, s_base[2];
+    __shared__ uint32_t s_wsum[kSelectThreads / 32];
+    grid_dep_wait();  // scores and histogram come from the scan kernel
+    grid_dep_launch();
 
     const int qi = blockIdx.y;
     const csa_query qr = p.queries[qi];
@@ -311,50 +311,78 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
         return;
     }
 
-    // 1. threshold bin
+    // 1. threshold bin (every CTA of the query finds the same one)
     const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = gh[i];
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = __ldcg(gh + i);
     __syncthreads();
-    suffix_counts(hist, suf, misc);
-    if (threadIdx.x == 0) {
-        int b1 = kHistBins - 1;
-        while (b1 > 0 && suf[b1] < (uint32_t)p.k) --b1;
-        misc[32] = (uint32_t)b1;
-        misc[33] = b1 + 1 < kHistBins ? suf[b1 + 1] : 0u;  // strictly above
-    }
-    __syncthreads();
+    suffix_find(hist, suf, misc, (uint32_t)p.k, misc + 32);
     const uint32_t b1 = misc[32];
     const uint32_t above = misc[33];
+    if (b1 == 0xFFFFFFFFu) {  // histogram holds fewer than k scores: cannot happen
+        if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
+        return;
+    }
     const uint32_t need = (uint32_t)p.k - above;
 
-    // 2. filter this CTA's slice
+    // 2. filter this CTA's 4096 scores (two 16-byte loads per thread), one atomic per list per CTA
     uint32_t* ctr = p.counters + (int64_t)qi * 4;
     int32_t* sel = p.sel + (int64_t)qi * kMaxK;
     uint64_t* cand = p.cand + (int64_t)qi * p.e_stride;
-    const int64_t per = (E + gridDim.x - 1) / gridDim.x;
-    const int64_t lo = (int64_t)blockIdx.x * per, hi = min(E, lo + per);
-    const int lane = threadIdx.x & 31;
-    for (int64_t j0 = lo; j0 < hi; j0 += blockDim.x) {
-        const int64_t j = j0 + threadIdx.x;
-        uint32_t key = 0, bin = 0;
-        if (j < hi) { key = float_key(srow[j]); bin = key >> 21; }
-        const bool is_sel = j < hi && bin > b1;
-        const bool is_cand = j < hi && bin == b1;
-        const uint32_t ms = __ballot_sync(0xffffffffu, is_sel);
-        const uint32_t mc = __ballot_sync(0xffffffffu, is_cand);
-        uint32_t bs = 0, bc = 0;
-        if (lane == 0) {
-            if (ms) bs = atomicAdd(&ctr[0], __popc(ms));
-            if (mc) bc = atomicAdd(&ctr[1], __popc(mc));
+    const int64_t j0 = (int64_t)blockIdx.x * kSelPerCta + (int64_t)threadIdx.x * kSelPerThread;
+    float sv[kSelPerThread];
+    if (j0 + kSelPerThread <= E) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(srow + j0));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(srow + j0 + 4));
+        sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w; sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
+    } else {
+#pragma unroll
+        for (int u = 0; u < kSelPerThread; ++u) sv[u] = j0 + u < E ? __ldcg(srow + j0 + u) : 0.f;
+    }
+    uint32_t ns = 0, nc = 0, flags = 0;  // flags: 2 bits per score (1 = above, 2 = in threshold bin)
+#pragma unroll
+    for (int u = 0; u < kSelPerThread; ++u) {
+        if (j0 + u < E) {
+            const uint32_t bin = float_key(sv[u]) >> 21;
+            if (bin > b1) { ++ns; flags |= 1u << (2 * u); }
+            else if (bin == b1) { ++nc; flags |= 2u << (2 * u); }
         }
-        bs = __shfl_sync(0xffffffffu, bs, 0);
-        bc = __shfl_sync(0xffffffffu, bc, 0);
-        const uint32_t below = (1u << lane) - 1u;
-        if (is_sel) {
-            const uint32_t pos = bs + __popc(ms & below);
-            if (pos < (uint32_t)kMaxK) sel[pos] = (int32_t)j;
+    }
+    // block exclusive scan of (ns << 16 | nc)
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t packed = (ns << 16) | nc;
+    uint32_t incl = packed;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t x = lane < kSelectThreads / 32 ? s_wsum[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
         }
-        if (is_cand) cand[bc + __popc(mc & below)] = composite(key, j);
+        if (lane < kSelectThreads / 32) s_wsum[lane] = x;
+        if (lane == kSelectThreads / 32 - 1) {
+            s_base[0] = (x >> 16) ? atomicAdd(&ctr[0], x >> 16) : 0u;
+            s_base[1] = (x & 0xFFFFu) ? atomicAdd(&ctr[1], x & 0xFFFFu) : 0u;
+        }
+    }
+    __syncthreads();
+    const uint32_t excl = (warp > 0 ? s_wsum[warp - 1] : 0u) + incl - packed;
+    uint32_t ps = s_base[0] + (excl >> 16), pc = s_base[1] + (excl & 0xFFFFu);
+#pragma unroll
+    for (int u = 0; u < kSelPerThread; ++u) {
+        const uint32_t f = (flags >> (2 * u)) & 3u;
+        if (f == 1u) {
+            if (ps < (uint32_t)kMaxK) sel[ps] = (int32_t)(j0 + u);
+            ++ps;
+        } else if (f == 2u) {
+            cand[pc++] = composite(float_key(sv[u]), j0 + u);
+        }
     }
 
     // 3. the last CTA of this query finishes the selection
@@ -365,21 +393,22 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     if (!s_last) return;
     __threadfence();
 
-    const uint32_t n_above = *((volatile uint32_t*)&ctr[0]);
-    const uint32_t n_cand = *((volatile uint32_t*)&ctr[1]);
+    const uint32_t n_above = __ldcg(&ctr[0]);
+    const uint32_t n_cand = __ldcg(&ctr[1]);
     if (n_above != above || n_cand < need) {  // histogram and filter disagree: cannot happen
         if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
         return;
     }
     const uint64_t* cs = cand;
+    bool cand_global = true;
     if (n_cand <= (uint32_t)kCandSmem) {
         for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x)
             cand_s[i] = __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i);
         __syncthreads();
         cs = cand_s;
+        cand_global = false;
     }
-    const bool cand_global = cs == cand;
-    const uint64_t T = radix_threshold(cs, cand_global, n_cand, need, b1, hist, misc);
+    const uint64_t T = need == n_cand ? 0ull : radix_threshold(cs, cand_global, n_cand, need, b1, hist, suf, misc);
     // gather the final list: entries above + candidates >= T
     if (threadIdx.x == 0) misc[40] = above;
     for (uint32_t i = threadIdx.x; i < above; i += blockDim.x) list[i] = __ldcg(sel + i);
@@ -392,21 +421,70 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
         }
     }
     __syncthreads();
-    // bitonic sort of the k indices (padded to a power of two with INT_MAX)
-    int npow = 1;
-    while (npow < p.k) npow <<= 1;
-    for (int i = p.k + threadIdx.x; i < npow; i += blockDim.x) list[i] = 0x7FFFFFFF;
-    __syncthreads();
-    for (int size = 2; size <= npow; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = threadIdx.x; t < npow / 2; t += blockDim.x) {
-                const int i = 2 * t - (t & (stride - 1));
-                const int jx = i + stride;
-                const bool up = (i & size) == 0;
-                const int32_t a = list[i], b = list[jx];
-                if ((a > b) == up) { list[i] = b; list[jx] = a; }
+    if (E <= (int64_t)kCandSmem * 64) {
+        // ascending order by compaction: mark the k winners in a bitmap over [0, E) (the candidate
+        // buffer is free now), then popcounts + one block scan give every winner its rank
+        uint32_t* bits = reinterpret_cast<uint32_t*>(cand_s);
+        const int nwords = (int)((E + 31) / 32);
+        for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0u;
+        __syncthreads();
+        for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
+            const int32_t j = list[i];
+            atomicOr(&bits[j >> 5], 1u << (j & 31));
+        }
+        __syncthreads();
+        const int per = (nwords + blockDim.x - 1) / blockDim.x;
+        const int w0 = threadIdx.x * per, w1 = min(nwords, w0 + per);
+        uint32_t cnt = 0;
+        for (int i = w0; i < w1; ++i) cnt += __popc(bits[i]);
+        // block exclusive scan of cnt
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t x = lane < kSelectThreads / 32 ? s_wsum[lane] : 0u;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
             }
-            __syncthreads();
+            if (lane < kSelectThreads / 32) s_wsum[lane] = x;
+        }
+        __syncthreads();
+        uint32_t pos = (warp > 0 ? s_wsum[warp - 1] : 0u) + incl - cnt;
+        __syncthreads();  // list[] is rewritten below
+        for (int i = w0; i < w1; ++i) {
+            uint32_t b = bits[i];
+            while (b) {
+                const int t = __ffs(b) - 1;
+                b &= b - 1u;
+                if (pos < (uint32_t)p.k) list[pos] = i * 32 + t;
+                ++pos;
+            }
+        }
+        __syncthreads();
+    } else {
+        // bitonic sort of the k indices (padded to a power of two with INT_MAX)
+        int npow = 1;
+        while (npow < p.k) npow <<= 1;
+        for (int i = p.k + threadIdx.x; i < npow; i += blockDim.x) list[i] = 0x7FFFFFFF;
+        __syncthreads();
+        for (int size = 2; size <= npow; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int t = threadIdx.x; t < npow / 2; t += blockDim.x) {
+                    const int i = 2 * t - (t & (stride - 1));
+                    const int jx = i + stride;
+                    const bool up = (i & size) == 0;
+                    const int32_t a = list[i], b = list[jx];
+                    if ((a > b) == up) { list[i] = b; list[jx] = a; }
+                }
+                __syncthreads();
+            }
         }
     }
     for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
@@ -452,7 +530,7 @@ void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
 }
 
 cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
-                              cudaEvent_t mid) {
+                              cudaEvent_t mid, bool pdl) {
     if (zero_ws) {
         // histogram + counters are contiguous at the start of the workspace
         const size_t nz = reinterpret_cast<char*>(p.sel) - reinterpret_cast<char*>(p.hist);
@@ -468,29 +546,29 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
         if (chunk > 16384) chunk = 16384;
         p.chunk = chunk;
         const int64_t gx = (max_entries + chunk - 1) / chunk;
-        if (p.d_I == 64)
-            index_scan_kernel<2><<<dim3((unsigned)gx, (unsigned)p.Q), kScanThreads, 0, stream>>>(p);
-        else
-            index_scan_kernel<1><<<dim3((unsigned)gx, (unsigned)p.Q), kScanThreads, 0, stream>>>(p);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = p.d_I == 64
+                            ? launch_kernel(index_scan_kernel<2>, dim3((unsigned)gx, (unsigned)p.Q), dim3(kScanThreads), 0,
+                                            stream, pdl && !zero_ws, p)
+                            : launch_kernel(index_scan_kernel<1>, dim3((unsigned)gx, (unsigned)p.Q), dim3(kScanThreads), 0,
+                                            stream, pdl && !zero_ws, p);
         if (e != cudaSuccess) return e;
     }
     if (mid) {
         cudaError_t e = cudaEventRecordWithFlags(mid, stream, cudaEventRecordExternal);
         if (e != cudaSuccess) return e;
     }
-    int f = (int)((max_entries + 16383) / 16384);
+    int64_t f = (max_entries + kSelPerCta - 1) / kSelPerCta;
     if (f < 1) f = 1;
-    if (f > 64) f = 64;
-    p.filter_ctas = f;
+    p.filter_ctas = (int)f;
     const size_t smem = (size_t)kHistBins * 8 + 64 * 4 + (size_t)kCandSmem * 8 + (size_t)kMaxK * 4;
     static bool attr_set = false;
     if (!attr_set) {
         cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         attr_set = true;
     }
-    index_select_kernel<<<dim3((unsigned)f, (unsigned)p.Q), kSelectThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    // after an event record the select follows the scan without overlap
+    return launch_kernel(index_select_kernel, dim3((unsigned)f, (unsigned)p.Q), dim3(kSelectThreads), smem, stream,
+                         pdl && mid == nullptr, p);
 }
 
 }  // namespace csa

@@ -56,7 +56,7 @@ size_t index_zero_bytes(int Q);  // leading bytes of the index workspace that mu
 void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride);
 // `mid` (nullable): event recorded between the scan and the select kernels.
 cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
-                              cudaEvent_t mid = nullptr);
+                              cudaEvent_t mid = nullptr, bool pdl = false);
 
 // Attention over a per-query key list = [selected CSA entries | raw window | HCA entries].
 struct AttnParams {
@@ -74,9 +74,15 @@ struct AttnParams {
     int m_hca;
     int use_hca;
     float scale_log2;           // scale * log2(e)
-    int keys_per_item;          // multiple of 64
-    int n_items;                // items per query: ceil((k_slots + W + max HCA entries) / keys_per_item)
-    // outputs: direct when n_items == 1, else partials + combine
+    // Items.  n_items == 1: one item covers the whole list (direct output, no merge).  Otherwise
+    // items [0, items_front) cut the front part [0, k_slots + W) into chunks of kpi_front keys and
+    // items [items_front, n_items) cut the HCA part into chunks of kpi_hca keys; every item writes
+    // a partial and combine_kernel merges them.  Chunk sizes are multiples of 64 (one key tile).
+    int n_items;
+    int items_front;
+    int kpi_front;
+    int kpi_hca;
+    // outputs
     float* out;                 // [Q, H, d]
     float* lse;                 // [Q, H] nullable
     float* part_o;              // [Q, items, 64, d]
@@ -84,7 +90,13 @@ struct AttnParams {
     int* status;
 };
 size_t attn_ws_bytes(int Q, int items, int d);
-cudaError_t launch_attention(AttnParams& p, void* ws, cudaStream_t stream);
+// Point the partial buffers of `p` into `ws` (when n_items > 1).
+void attn_ws_carve(AttnParams& p, void* ws);
+// Items [item_begin, item_begin + item_count) of every query.
+cudaError_t launch_attention_items(const AttnParams& p, int item_begin, int item_count, cudaStream_t stream,
+                                   bool pdl = false);
+// The log-sum-exp merge of all items' partials (only when n_items > 1).
+cudaError_t launch_combine(const AttnParams& p, cudaStream_t stream);
 
 // Decode helper: append one token per sequence, compress completed entries, build the query table.
 struct AppendParams {
