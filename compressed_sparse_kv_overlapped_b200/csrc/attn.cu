@@ -171,14 +171,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
         const uint64_t* rowptr = reinterpret_cast<const uint64_t*>(sm + L::kRowPtr) + lw * 16;
         uint64_t* rowptr_w = reinterpret_cast<uint64_t*>(sm + L::kRowPtr) + lw * 16;
         constexpr int CPR = D / 8;  // 16-byte chunks per row
+        // Lane l copies 16-byte chunks l, l+32, ... of each 64-chunk (1 KiB) row: chunk c lands in
+        // block c/8 at swizzled position (c%8) ^ (row%8), and c%8 = l%8 for every chunk of a lane.
+        constexpr int CPL = CPR / 32 > 0 ? CPR / 32 : 1;  // chunks per lane per row (2 at D = 512)
+        const uint32_t lane_blk = (uint32_t)(lane >> 3) * L::kBlock;  // block of chunk `lane`
+        const uint32_t lane_c7 = (uint32_t)(lane & 7);
         if (T > 0) {
             // Q: 64 (padded) heads, 16 per loader warp; an input, so it may load before the wait
-            for (int e = lane; e < 16 * CPR; e += 32) {
-                const int h = lw * 16 + e / CPR, ch = e % CPR;
+            for (int r = 0; r < 16; ++r) {
+                const int h = lw * 16 + r;
                 const bool ok = h < p.H;
-                const uint16_t* src = ok ? p.q + ((int64_t)qi * p.H + h) * D + ch * 8 : p.q;
-                const uint32_t dst = sbase + L::kQ + (ch >> 3) * L::kBlock + sw128_offset(h, ch & 7);
-                cp_async16(dst, src, ok ? 16u : 0u);
+                const uint16_t* src = p.q + ((int64_t)qi * p.H + (ok ? h : 0)) * D;
+                const uint32_t dst = sbase + L::kQ + lane_blk + (uint32_t)h * 128u + ((lane_c7 ^ (h & 7)) << 4);
+                if (CPR >= 32) {
+#pragma unroll
+                    for (int u = 0; u < CPL; ++u)
+                        cp_async16(dst + u * 4 * L::kBlock, src + (lane + 32 * u) * 8, ok ? 16u : 0u);
+                } else if (lane < CPR) {
+                    cp_async16(dst, src + lane * 8, ok ? 16u : 0u);
+                }
             }
         }
         grid_dep_wait();  // the selected indices come from the previous kernel
@@ -195,13 +206,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
             }
             const uint32_t vm = __ballot_sync(0xffffffffu, valid) & 0xFFFFu;
             __syncwarp();
-            const uint32_t kbase = sbase + (st ? L::kK1 : L::kK0);
-            for (int e = lane; e < 16 * CPR; e += 32) {
-                const int r = e / CPR, ch = e % CPR;
+            const uint32_t kbase = sbase + (st ? L::kK1 : L::kK0) + lane_blk;
+#pragma unroll 4
+            for (int r = 0; r < 16; ++r) {
                 const uint16_t* row = reinterpret_cast<const uint16_t*>(rowptr[r]);
                 const int key = lw * 16 + r;
-                const uint32_t dst = kbase + (ch >> 3) * L::kBlock + sw128_offset(key, ch & 7);
-                cp_async16(dst, row ? row + ch * 8 : p.q, row ? 16u : 0u);
+                const uint32_t dst = kbase + (uint32_t)key * 128u + ((lane_c7 ^ (key & 7)) << 4);
+                const uint32_t nb = row ? 16u : 0u;
+                const uint16_t* src = row ? row : p.q;
+                if (CPR >= 32) {
+#pragma unroll
+                    for (int u = 0; u < CPL; ++u) cp_async16(dst + u * 4 * L::kBlock, src + (lane + 32 * u) * 8, nb);
+                } else if (lane < CPR) {
+                    cp_async16(dst, src + lane * 8, nb);
+                }
             }
             cp_async_wait_all();
             fence_proxy_async_smem();
@@ -307,10 +325,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
             const uint64_t vmask = (uint64_t)mask16[st * 4 + 0] | ((uint64_t)mask16[st * 4 + 1] << 16) |
                                    ((uint64_t)mask16[st * 4 + 2] << 32) | ((uint64_t)mask16[st * 4 + 3] << 48);
             float mx = -INFINITY;
+            const float sc = p.scale_log2;
+            if (vmask == ~0ull) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                s[j] = ((vmask >> j) & 1ull) ? s[j] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[j]);
+                for (int j = 0; j < 64; ++j) {
+                    s[j] *= sc;
+                    mx = fmaxf(mx, s[j]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    s[j] = ((vmask >> j) & 1ull) ? s[j] * sc : -INFINITY;
+                    mx = fmaxf(mx, s[j]);
+                }
             }
             // lazy rescaling: move the reference max only when it grows by more than 2^8
             float alpha = 1.f;
@@ -347,19 +374,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
                 if (!ok) break;
             }
             if (row_thread) {
+                // masked slots hold -inf: 2^(-inf - m) = 0; while the row has seen no key, m_use = 0
+                const float m_use = m_run == -INFINITY ? 0.f : m_run;
                 float lsum = 0.f;
-                unsigned char* prow = sm + (st ? L::kP1 : L::kP0);
+                const uint32_t prow = sbase + (st ? L::kP1 : L::kP0);
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     uint32_t w4[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const float p0 = m_run == -INFINITY ? 0.f : exp2f(s[c8 * 8 + 2 * u] - m_run);
-                        const float p1 = m_run == -INFINITY ? 0.f : exp2f(s[c8 * 8 + 2 * u + 1] - m_run);
+                        const float p0 = fast_exp2(s[c8 * 8 + 2 * u] - m_use);
+                        const float p1 = fast_exp2(s[c8 * 8 + 2 * u + 1] - m_use);
+                        lsum += p0 + p1;
                         w4[u] = pack_bf16x2(p0, p1);
-                        lsum += bf16lo(w4[u]) + bf16hi(w4[u]);
                     }
-                    *reinterpret_cast<uint4*>(prow + sw128_offset(h, c8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_offset(h, c8)),
+                                 "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
+                                 : "memory");
                 }
                 l_run += lsum;
             }
@@ -367,39 +398,62 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
             tc_fence_before();
             mbar_arrive(&bars->p_full[st]);
         }
-        // ---- epilogue
+        // ---- epilogue: TMEM -> shared memory (Q and the key stages are free now) -> coalesced stores
         if (ok && T > 0) ok = mbar_wait(&bars->o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, p.status, abort_flag);
         const float l_row = __shfl_sync(0xffffffffu, l_run, i & 15);
         const float m_row = __shfl_sync(0xffffffffu, m_run, i & 15);
         const bool has = ok && T > 0 && l_row > 0.f;
         const float inv = has ? 1.f / l_row : 0.f;
         const int dim0 = row_thread ? 0 : 256;
-        const bool writes = (row_thread || D >= 512) && h < p.H;
-        float* orow = direct ? p.out + ((int64_t)qi * p.H + h) * D
-                             : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + h) * D;
-        if (has) tc_fence_after();
-        if (has || direct) {
+        const bool mine = row_thread || D >= 512;  // lanes 16-31 hold dims 256-511 when D = 512
+        // staging rows of D floats, padded by 4 floats so 16-byte row-strided writes spread banks
+        constexpr int kStride = D + 4;
+        float* stage = reinterpret_cast<float*>(sm + L::kQ);  // Q and both key stages are free now
+        static_assert(64 * (D + 4) * 4 <= 3 * L::NKB * L::kBlock, "epilogue staging exceeds Q + key stages");
+        if (has) {
+            tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < OC; c += 64) {
                 uint32_t r[4][16];
-                if (has) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tmem + lane_base + kColO + c + q4 * 16, r[q4]);
-                    tmem_ld_wait();
-                }
-                if (writes) {
+                for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tmem + lane_base + kColO + c + q4 * 16, r[q4]);
+                tmem_ld_wait();
+                if (mine) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
                         for (int j = 0; j < 16; j += 4) {
                             float4 v;
-                            v.x = has ? __uint_as_float(r[q4][j]) * inv : 0.f;
-                            v.y = has ? __uint_as_float(r[q4][j + 1]) * inv : 0.f;
-                            v.z = has ? __uint_as_float(r[q4][j + 2]) * inv : 0.f;
-                            v.w = has ? __uint_as_float(r[q4][j + 3]) * inv : 0.f;
-                            *reinterpret_cast<float4*>(orow + dim0 + c + q4 * 16 + j) = v;
+                            v.x = __uint_as_float(r[q4][j]) * inv;
+                            v.y = __uint_as_float(r[q4][j + 1]) * inv;
+                            v.z = __uint_as_float(r[q4][j + 2]) * inv;
+                            v.w = __uint_as_float(r[q4][j + 3]) * inv;
+                            *reinterpret_cast<float4*>(stage + h * kStride + dim0 + c + q4 * 16 + j) = v;
                         }
                 }
+            }
+        }
+        // staged rows become visible to the bulk-copy engine (async proxy) after this fence + barrier
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps (128 threads)
+        const int rows = p.H < kHeadsPad ? p.H : kHeadsPad;
+        if (has) {
+            // one lane per warp hands 16 staged rows to the bulk-copy engine
+            if (i == 0) {
+                for (int hh = warp * 16; hh < warp * 16 + 16 && hh < rows; ++hh) {
+                    float* dst = direct ? p.out + ((int64_t)qi * p.H + hh) * D
+                                        : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + hh) * D;
+                    bulk_store(dst, smem_u32(stage + hh * kStride), D * 4);
+                }
+                bulk_commit();
+                bulk_wait_all();
+            }
+        } else if (direct) {
+            const int tid = threadIdx.x;  // 0..127
+            for (int e = tid; e < rows * (D / 4); e += 128) {
+                const int hh = e / (D / 4), c4 = e % (D / 4);
+                *reinterpret_cast<float4*>(p.out + ((int64_t)qi * p.H + hh) * D + c4 * 4) =
+                    make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
         if (row_thread && h < p.H) {
@@ -424,59 +478,69 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
 // every thread accumulates one float4 column of all contributing partials with batched loads.
 template <int D>
 __global__ void combine_kernel(AttnParams p) {
+    constexpr int kMaxBatch = 24;  // partial rows held in registers per pass
     const int h = blockIdx.x, qi = blockIdx.y;
     const int n_items = p.n_items;
-    __shared__ float wts[256];
-    __shared__ int used[256];
-    __shared__ int n_used;
+    const int lane = threadIdx.x & 31;
+    __shared__ float s_lse[256];
+    __shared__ float s_w[256];
+    __shared__ float s_res[2];
+    // every thread owns one float4 column of the output row (D/4 threads)
+    const int c = threadIdx.x * 4;
+    const float* base = p.part_o + ((int64_t)qi * n_items * kHeadsPad + h) * D + c;
+    const int64_t item_stride = (int64_t)kHeadsPad * D;
+    for (int it = threadIdx.x; it < n_items; it += blockDim.x)
+        s_lse[it] = __ldcg(p.part_lse + ((int64_t)qi * n_items + it) * kHeadsPad + h);
+    // the partial rows do not depend on the weights: issue their loads first
+    float4 v[kMaxBatch];
+    const int nb0 = n_items < kMaxBatch ? n_items : kMaxBatch;
+#pragma unroll
+    for (int u = 0; u < kMaxBatch; ++u)
+        if (u < nb0) v[u] = __ldcg(reinterpret_cast<const float4*>(base + u * item_stride));
+    __syncthreads();
     if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
         float mx = -INFINITY;
-        for (int it = lane; it < n_items; it += 32)
-            mx = fmaxf(mx, p.part_lse[((int64_t)qi * n_items + it) * kHeadsPad + h]);
+        for (int it = lane; it < n_items; it += 32) mx = fmaxf(mx, s_lse[it]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float sum = 0.f;
         for (int it = lane; it < n_items; it += 32) {
-            const float l = p.part_lse[((int64_t)qi * n_items + it) * kHeadsPad + h];
-            const float w = mx == -INFINITY ? 0.f : expf(l - mx);
-            wts[it] = w;
+            const float w = mx == -INFINITY ? 0.f : expf(s_lse[it] - mx);
+            s_w[it] = w;
             sum += w;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        __syncwarp();
         if (lane == 0) {
-            int nu = 0;
-            for (int it = 0; it < n_items; ++it)
-                if (wts[it] > 0.f) { wts[nu] = wts[it] / sum; used[nu] = it; ++nu; }
-            n_used = nu;
-            if (p.lse) p.lse[(int64_t)qi * p.H + h] = mx == -INFINITY ? -INFINITY : mx + logf(sum);
+            s_res[0] = sum > 0.f ? 1.f / sum : 0.f;
+            s_res[1] = mx == -INFINITY ? -INFINITY : mx + logf(sum);
         }
     }
     __syncthreads();
-    const int nu = n_used;
-    for (int c = threadIdx.x * 4; c < D; c += blockDim.x * 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int b = 0; b < nu; b += 8) {
-            float4 v[8];
+    const float inv = s_res[0];
+    if (threadIdx.x == 0 && p.lse) p.lse[(int64_t)qi * p.H + h] = s_res[1];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int b = 0; b < n_items; b += kMaxBatch) {
+        const int nb = n_items - b < kMaxBatch ? n_items - b : kMaxBatch;
+        if (b > 0) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (b + u < nu)
-                    v[u] = __ldcg(reinterpret_cast<const float4*>(
-                        p.part_o + (((int64_t)qi * n_items + used[b + u]) * kHeadsPad + h) * D + c));
+            for (int u = 0; u < kMaxBatch; ++u)
+                if (u < nb) v[u] = __ldcg(reinterpret_cast<const float4*>(base + (b + u) * item_stride));
+        }
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (b + u < nu) {
-                    const float w = wts[b + u];
+        for (int u = 0; u < kMaxBatch; ++u) {
+            if (u < nb) {
+                const float w = s_w[b + u] * inv;
+                if (w > 0.f) {  // an empty item (lse = -inf) has weight 0 and unwritten rows
                     acc.x = fmaf(w, v[u].x, acc.x);
                     acc.y = fmaf(w, v[u].y, acc.y);
                     acc.z = fmaf(w, v[u].z, acc.z);
                     acc.w = fmaf(w, v[u].w, acc.w);
                 }
+            }
         }
-        *reinterpret_cast<float4*>(p.out + ((int64_t)qi * p.H + h) * D + c) = acc;
     }
+    *reinterpret_cast<float4*>(p.out + ((int64_t)qi * p.H + h) * D + c) = acc;
 }
 
 template <int D>

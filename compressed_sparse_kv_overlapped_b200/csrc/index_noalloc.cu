@@ -5,7 +5,7 @@
 // whose caching allocator owns every device buffer and forbids direct cudaMalloc, real-time
 // serving loops that must not allocate after start-up, or thin foreign-language bindings that see
 // only the caller's input and output pointers.  For them this entry point keeps its scratch in a
-// fixed array compiled into the library (kScratchBytes, about 12.3 MiB per device), so a call
+// fixed array compiled into the library (kScratchBytes, about 12.9 MiB per device), so a call
 // needs nothing but inputs, outputs and a stream.  The array occupies device memory on every GPU
 // that loads the library until the process exits.
 //
@@ -21,9 +21,12 @@ namespace {
 constexpr int kNoAllocMaxQ = 16;
 constexpr int64_t kNoAllocMaxSlots = int64_t(1) << 20;  // Q * score-row stride
 // Upper bound of index_ws_bytes(Q, e_stride) under the two limits above: histograms, counters,
-// above-threshold lists, fp32 scores and 64-bit candidates.
-constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * kHistBins * 4 + 256 + size_t(kNoAllocMaxQ) * kMaxK * 4 +
-                                 size_t(kNoAllocMaxSlots) * 4 + 256 + size_t(kNoAllocMaxSlots) * 8 + 256;
+// per-CTA segment counts, fp32 scores and the 64-bit kept-entry segments (each query's row rounded
+// up to whole kSelPerCta segments).
+constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * kHistBins * 4 + 256 + 256 +
+                                 size_t(kNoAllocMaxSlots / kSelPerCta + kNoAllocMaxQ) * 4 + 256 +
+                                 size_t(kNoAllocMaxSlots) * 4 + 256 +
+                                 size_t(kNoAllocMaxSlots + kNoAllocMaxQ * kSelPerCta) * 8 + 256;
 
 __device__ __align__(256) unsigned char g_index_scratch[kScratchBytes];
 

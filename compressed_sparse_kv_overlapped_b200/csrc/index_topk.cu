@@ -28,7 +28,6 @@ namespace {
 
 constexpr int kScanThreads = 256;
 constexpr int kSelectThreads = 512;
-constexpr int kCandSmem = 8192;  // candidates the last CTA keeps in shared memory
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
     asm volatile(
@@ -168,8 +167,8 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(IndexParams p)
 
 // ---- select ----------------------------------------------------------------------------------
 
-constexpr int kSelPerThread = 8;                                   // scores per thread in the filter
-constexpr int kSelPerCta = kSelectThreads * kSelPerThread;          // 4096 entries per filter CTA
+constexpr int kSelPerThread = kSelPerCta / kSelectThreads;          // 8 scores per thread
+constexpr int kListSmem = 8192;                                     // kept entries the last CTA holds
 
 __device__ __forceinline__ uint64_t composite(uint32_t key, int64_t j) {
     return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
@@ -217,12 +216,59 @@ __device__ void suffix_find(const uint32_t* hist, uint32_t* suf, uint32_t* warp_
     __syncthreads();
 }
 
-// Exact selection of the `need` largest composite keys among n distinct candidates that share the
-// top 11 bits `top11`.  Returns T with exactly `need` candidates >= T.  Radix passes of 11 bits over
-// bits 52..0 (counted with warp-aggregated shared-memory atomics, so equal digits do not
-// serialize); stops as soon as the chosen digit holds exactly the remaining count.
-__device__ uint64_t radix_threshold(const uint64_t* cand, bool in_global, uint32_t n, uint32_t need,
-                                    uint32_t top11, uint32_t* cnt, uint32_t* suf, uint32_t* misc) {
+// Block-wide exclusive scan of one value per thread; returns this thread's exclusive prefix and
+// writes the total to *total.  `wsum` holds kSelectThreads/32 words.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t x = lane < kSelectThreads / 32 ? wsum[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane < kSelectThreads / 32) wsum[lane] = x;
+    }
+    __syncthreads();
+    const uint32_t excl = (warp > 0 ? wsum[warp - 1] : 0u) + incl - v;
+    *total = wsum[kSelectThreads / 32 - 1];
+    __syncthreads();
+    return excl;
+}
+
+// The kept list of one query: the filter CTAs' segments concatenated in CTA order (so in index
+// order).  Entry i lives in segment c = the last with off[c] <= i.
+struct KeptList {
+    const uint64_t* seg;     // [F][kSelPerCta]
+    const uint32_t* off;     // [F + 1] exclusive prefix of the segment counts (shared memory)
+    int F;
+    const uint64_t* cache;   // the whole list in shared memory, or nullptr
+    __device__ __forceinline__ uint64_t get(uint32_t i) const {
+        if (cache) return cache[i];
+        int lo = 0, hi = F - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (off[mid] <= i) lo = mid; else hi = mid - 1;
+        }
+        return __ldcg(reinterpret_cast<const unsigned long long*>(seg) + (int64_t)lo * kSelPerCta + (i - off[lo]));
+    }
+};
+
+// Exact selection of the `need` largest keys among the list entries whose top 11 bits equal top11
+// (the threshold-bin members; entries of higher bins are kept regardless).  Returns T with exactly
+// `need` of those members >= T.  Radix passes of 11 bits over bits 52..0 (counted with
+// warp-aggregated shared-memory atomics, so equal digits do not serialize); stops as soon as the
+// chosen digit holds exactly the remaining count.
+__device__ uint64_t radix_threshold(const KeptList& L, uint32_t n, uint32_t need, uint32_t top11, uint32_t* cnt,
+                                    uint32_t* suf, uint32_t* misc) {
     uint64_t prefix = (uint64_t)top11 << 53;
     uint64_t mask = (uint64_t)0x7FF << 53;
     uint32_t remaining = need;
@@ -238,8 +284,7 @@ __device__ uint64_t radix_threshold(const uint64_t* cand, bool in_global, uint32
             bool match = false;
             uint32_t dg = 0;
             if (i < n) {
-                const uint64_t v =
-                    in_global ? __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i) : cand[i];
+                const uint64_t v = L.get(i);
                 match = (v & mask) == prefix;
                 dg = (uint32_t)(v >> sh) & dmask;
             }
@@ -267,9 +312,9 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);          // kHistBins
     uint32_t* suf = hist + kHistBins;                                  // kHistBins
     uint32_t* misc = suf + kHistBins;                                  // 64
-    uint64_t* cand_s = reinterpret_cast<uint64_t*>(misc + 64);         // kCandSmem
-    int32_t* list = reinterpret_cast<int32_t*>(cand_s + kCandSmem);    // kMaxK (sort buffer)
-    __shared__ uint32_t s_last, s_base[2];
+    uint64_t* lst = reinterpret_cast<uint64_t*>(misc + 64);            // kListSmem
+    uint32_t* offs = reinterpret_cast<uint32_t*>(lst + kListSmem);    // filter CTAs + 1
+    __shared__ uint32_t s_last;
     __shared__ uint32_t s_wsum[kSelectThreads / 32];
     grid_dep_wait();  // scores and histogram come from the scan kernel
     grid_dep_launch();
@@ -323,11 +368,9 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
         return;
     }
     const uint32_t need = (uint32_t)p.k - above;
+    const uint32_t n_bin = hist[b1];  // members of the threshold bin (over all CTAs)
 
-    // 2. filter this CTA's 4096 scores (two 16-byte loads per thread), one atomic per list per CTA
-    uint32_t* ctr = p.counters + (int64_t)qi * 4;
-    int32_t* sel = p.sel + (int64_t)qi * kMaxK;
-    uint64_t* cand = p.cand + (int64_t)qi * p.e_stride;
+    // 2. keep this CTA's entries of bin >= b1, in index order, in its own segment
     const int64_t j0 = (int64_t)blockIdx.x * kSelPerCta + (int64_t)threadIdx.x * kSelPerThread;
     float sv[kSelPerThread];
     if (j0 + kSelPerThread <= E) {
@@ -338,162 +381,80 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
 #pragma unroll
         for (int u = 0; u < kSelPerThread; ++u) sv[u] = j0 + u < E ? __ldcg(srow + j0 + u) : 0.f;
     }
-    uint32_t ns = 0, nc = 0, flags = 0;  // flags: 2 bits per score (1 = above, 2 = in threshold bin)
+    uint32_t nk = 0, kf = 0;
 #pragma unroll
     for (int u = 0; u < kSelPerThread; ++u) {
-        if (j0 + u < E) {
-            const uint32_t bin = float_key(sv[u]) >> 21;
-            if (bin > b1) { ++ns; flags |= 1u << (2 * u); }
-            else if (bin == b1) { ++nc; flags |= 2u << (2 * u); }
-        }
+        if (j0 + u < E && (float_key(sv[u]) >> 21) >= b1) { ++nk; kf |= 1u << u; }
     }
-    // block exclusive scan of (ns << 16 | nc)
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t packed = (ns << 16) | nc;
-    uint32_t incl = packed;
+    uint32_t cta_total;
+    uint32_t pos = block_excl_scan(nk, s_wsum, &cta_total);
+    uint64_t* myseg = p.seg + (int64_t)qi * p.e_seg + (int64_t)blockIdx.x * kSelPerCta;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t x = lane < kSelectThreads / 32 ? s_wsum[lane] : 0u;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane < kSelectThreads / 32) s_wsum[lane] = x;
-        if (lane == kSelectThreads / 32 - 1) {
-            s_base[0] = (x >> 16) ? atomicAdd(&ctr[0], x >> 16) : 0u;
-            s_base[1] = (x & 0xFFFFu) ? atomicAdd(&ctr[1], x & 0xFFFFu) : 0u;
-        }
-    }
-    __syncthreads();
-    const uint32_t excl = (warp > 0 ? s_wsum[warp - 1] : 0u) + incl - packed;
-    uint32_t ps = s_base[0] + (excl >> 16), pc = s_base[1] + (excl & 0xFFFFu);
-#pragma unroll
-    for (int u = 0; u < kSelPerThread; ++u) {
-        const uint32_t f = (flags >> (2 * u)) & 3u;
-        if (f == 1u) {
-            if (ps < (uint32_t)kMaxK) sel[ps] = (int32_t)(j0 + u);
-            ++ps;
-        } else if (f == 2u) {
-            cand[pc++] = composite(float_key(sv[u]), j0 + u);
-        }
-    }
+    for (int u = 0; u < kSelPerThread; ++u)
+        if (kf & (1u << u)) myseg[pos++] = composite(float_key(sv[u]), j0 + u);
+    if (threadIdx.x == 0) p.seg_count[(int64_t)qi * (p.e_seg / kSelPerCta) + blockIdx.x] = cta_total;
 
     // 3. the last CTA of this query finishes the selection
+    uint32_t* ctr = p.counters + (int64_t)qi * 4;
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(&ctr[2], 1u) == gridDim.x - 1) ? 1u : 0u;
+    if (threadIdx.x == 0) s_last = (atomicAdd(&ctr[0], 1u) == gridDim.x - 1) ? 1u : 0u;
     __syncthreads();
     if (!s_last) return;
     __threadfence();
 
-    const uint32_t n_above = __ldcg(&ctr[0]);
-    const uint32_t n_cand = __ldcg(&ctr[1]);
-    if (n_above != above || n_cand < need) {  // histogram and filter disagree: cannot happen
+    const int F = gridDim.x;
+    // exclusive prefix of the segment counts (8 per thread)
+    {
+        const uint32_t* gc = p.seg_count + (int64_t)qi * (p.e_seg / kSelPerCta);
+        uint32_t c8[8], tot = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int c = threadIdx.x * 8 + u;
+            c8[u] = c < F ? __ldcg(gc + c) : 0u;
+            tot += c8[u];
+        }
+        uint32_t all;
+        uint32_t run = block_excl_scan(tot, s_wsum, &all);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int c = threadIdx.x * 8 + u;
+            if (c <= F) offs[c] = run;
+            run += c8[u];
+        }
+        __syncthreads();
+    }
+    const uint32_t n_tot = offs[F];
+    if (n_tot != above + n_bin) {  // histogram and filter disagree: cannot happen
         if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
         return;
     }
-    const uint64_t* cs = cand;
-    bool cand_global = true;
-    if (n_cand <= (uint32_t)kCandSmem) {
-        for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x)
-            cand_s[i] = __ldcg(reinterpret_cast<const unsigned long long*>(cand) + i);
+    KeptList kl{p.seg + (int64_t)qi * p.e_seg, offs, F, nullptr};
+    if (n_tot <= (uint32_t)kListSmem) {
+        for (uint32_t i = threadIdx.x; i < n_tot; i += blockDim.x) lst[i] = kl.get(i);
         __syncthreads();
-        cs = cand_s;
-        cand_global = false;
+        kl.cache = lst;
     }
-    const uint64_t T = need == n_cand ? 0ull : radix_threshold(cs, cand_global, n_cand, need, b1, hist, suf, misc);
-    // gather the final list: entries above + candidates >= T
-    if (threadIdx.x == 0) misc[40] = above;
-    for (uint32_t i = threadIdx.x; i < above; i += blockDim.x) list[i] = __ldcg(sel + i);
-    __syncthreads();
-    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
-        const uint64_t v = cand_global ? __ldcg(reinterpret_cast<const unsigned long long*>(cs) + i) : cs[i];
+    const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53) : radix_threshold(kl, n_tot, need, b1, hist, suf, misc);
+    // 4. compaction in index order: keep every entry >= T (exactly k of them)
+    const uint32_t per = (n_tot + blockDim.x - 1) / blockDim.x;
+    const uint32_t i0 = threadIdx.x * per, i1 = min(n_tot, i0 + per);
+    uint32_t mine = 0;
+    for (uint32_t i = i0; i < i1; ++i) mine += kl.get(i) >= T ? 1u : 0u;
+    uint32_t kept_total;
+    uint32_t o = block_excl_scan(mine, s_wsum, &kept_total);
+    for (uint32_t i = i0; i < i1; ++i) {
+        const uint64_t v = kl.get(i);
         if (v >= T) {
-            const uint32_t pos = atomicAdd(&misc[40], 1u);
-            if (pos < (uint32_t)p.k) list[pos] = (int32_t)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
+            if (o < (uint32_t)p.k) {
+                out[o] = (int32_t)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
+                if (sout) sout[o] = key_float((uint32_t)(v >> 32));
+            }
+            ++o;
         }
     }
-    __syncthreads();
-    if (E <= (int64_t)kCandSmem * 64) {
-        // ascending order by compaction: mark the k winners in a bitmap over [0, E) (the candidate
-        // buffer is free now), then popcounts + one block scan give every winner its rank
-        uint32_t* bits = reinterpret_cast<uint32_t*>(cand_s);
-        const int nwords = (int)((E + 31) / 32);
-        for (int i = threadIdx.x; i < nwords; i += blockDim.x) bits[i] = 0u;
-        __syncthreads();
-        for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
-            const int32_t j = list[i];
-            atomicOr(&bits[j >> 5], 1u << (j & 31));
-        }
-        __syncthreads();
-        const int per = (nwords + blockDim.x - 1) / blockDim.x;
-        const int w0 = threadIdx.x * per, w1 = min(nwords, w0 + per);
-        uint32_t cnt = 0;
-        for (int i = w0; i < w1; ++i) cnt += __popc(bits[i]);
-        // block exclusive scan of cnt
-        uint32_t incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (lane == 31) s_wsum[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            uint32_t x = lane < kSelectThreads / 32 ? s_wsum[lane] : 0u;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            if (lane < kSelectThreads / 32) s_wsum[lane] = x;
-        }
-        __syncthreads();
-        uint32_t pos = (warp > 0 ? s_wsum[warp - 1] : 0u) + incl - cnt;
-        __syncthreads();  // list[] is rewritten below
-        for (int i = w0; i < w1; ++i) {
-            uint32_t b = bits[i];
-            while (b) {
-                const int t = __ffs(b) - 1;
-                b &= b - 1u;
-                if (pos < (uint32_t)p.k) list[pos] = i * 32 + t;
-                ++pos;
-            }
-        }
-        __syncthreads();
-    } else {
-        // bitonic sort of the k indices (padded to a power of two with INT_MAX)
-        int npow = 1;
-        while (npow < p.k) npow <<= 1;
-        for (int i = p.k + threadIdx.x; i < npow; i += blockDim.x) list[i] = 0x7FFFFFFF;
-        __syncthreads();
-        for (int size = 2; size <= npow; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                for (int t = threadIdx.x; t < npow / 2; t += blockDim.x) {
-                    const int i = 2 * t - (t & (stride - 1));
-                    const int jx = i + stride;
-                    const bool up = (i & size) == 0;
-                    const int32_t a = list[i], b = list[jx];
-                    if ((a > b) == up) { list[i] = b; list[jx] = a; }
-                }
-                __syncthreads();
-            }
-        }
-    }
-    for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
-        const int32_t j = list[i];
-        out[i] = j;
-        if (sout) sout[i] = srow[j];
-    }
-    // leave the per-query counters and histogram clean for the next call
-    __syncthreads();
+    if (threadIdx.x == 0 && kept_total != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
+    // leave the per-query histogram and ticket clean for the next call
     uint32_t* ghw = p.hist + (int64_t)qi * kHistBins;
     for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ghw[i] = 0u;
     if (threadIdx.x < 4) ctr[threadIdx.x] = 0u;
@@ -503,38 +464,42 @@ constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 }  // namespace
 
+int64_t seg_stride(int64_t e_stride) { return ((e_stride + kSelPerCta - 1) / kSelPerCta) * kSelPerCta; }
+
 size_t index_ws_bytes(int Q, int64_t e_stride) {
+    const int64_t es = seg_stride(e_stride);
     size_t s = 0;
     s += align256((size_t)Q * kHistBins * 4);
     s += align256((size_t)Q * 4 * 4);
-    s += align256((size_t)Q * kMaxK * 4);
+    s += align256((size_t)Q * (es / kSelPerCta) * 4);
     s += align256((size_t)Q * e_stride * 4);
-    s += align256((size_t)Q * e_stride * 8);
+    s += align256((size_t)Q * es * 8);
     return s;
 }
 
 size_t index_zero_bytes(int Q) { return align256((size_t)Q * kHistBins * 4) + align256((size_t)Q * 4 * 4); }
 
 void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
+    const int64_t es = seg_stride(e_stride);
     char* b = static_cast<char*>(ws);
     p.hist = reinterpret_cast<uint32_t*>(b);
     b += align256((size_t)Q * kHistBins * 4);
     p.counters = reinterpret_cast<uint32_t*>(b);
     b += align256((size_t)Q * 4 * 4);
-    p.sel = reinterpret_cast<int32_t*>(b);
-    b += align256((size_t)Q * kMaxK * 4);
+    p.seg_count = reinterpret_cast<uint32_t*>(b);
+    b += align256((size_t)Q * (es / kSelPerCta) * 4);
     p.scores = reinterpret_cast<float*>(b);
     b += align256((size_t)Q * e_stride * 4);
-    p.cand = reinterpret_cast<uint64_t*>(b);
+    p.seg = reinterpret_cast<uint64_t*>(b);
     p.e_stride = e_stride;
+    p.e_seg = es;
 }
 
 cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
                               cudaEvent_t mid, bool pdl) {
     if (zero_ws) {
         // histogram + counters are contiguous at the start of the workspace
-        const size_t nz = reinterpret_cast<char*>(p.sel) - reinterpret_cast<char*>(p.hist);
-        cudaError_t e = cudaMemsetAsync(p.hist, 0, nz, stream);
+        cudaError_t e = cudaMemsetAsync(p.hist, 0, index_zero_bytes(p.Q), stream);
         if (e != cudaSuccess) return e;
     }
     if (max_entries > p.k) {
@@ -560,10 +525,12 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
     int64_t f = (max_entries + kSelPerCta - 1) / kSelPerCta;
     if (f < 1) f = 1;
     p.filter_ctas = (int)f;
-    const size_t smem = (size_t)kHistBins * 8 + 64 * 4 + (size_t)kCandSmem * 8 + (size_t)kMaxK * 4;
+    if (f > (int64_t)kSelectThreads * 8 - 1) return cudaErrorInvalidValue;  // > 16M entries per query
+    const size_t smem = (size_t)kHistBins * 8 + 64 * 4 + (size_t)kListSmem * 8 + ((size_t)f + 1) * 4;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const int max_smem = kHistBins * 8 + 64 * 4 + kListSmem * 8 + kSelectThreads * 8 * 4;
+        cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
         attr_set = true;
     }
     // after an event record the select follows the scan without overlap

@@ -28,6 +28,7 @@ cudaError_t launch_compress(const CompressParams& p, int64_t max_entries, cudaSt
 // Indexer score scan + top-k select.
 constexpr int kHistBins = 2048;  // coarse histogram over the top 11 bits of the score key
 constexpr int kMaxK = 2048;
+constexpr int kSelPerCta = 4096;  // scores per select (filter) CTA
 
 struct IndexParams {
     const csa_seq* seqs;
@@ -39,13 +40,14 @@ struct IndexParams {
     int64_t chunk;            // entries per scan CTA
     int64_t max_entries;      // host bound of floor(L/m) over all queries (grid sizing)
     int64_t e_stride;         // row stride of the score buffer
+    int64_t e_seg;            // row stride of the segment buffer (e_stride rounded up to kSelPerCta)
     int filter_ctas;          // CTAs per query in the select kernel
     // workspace
     float* scores;            // [Q, e_stride]
     uint32_t* hist;           // [Q, kHistBins]
-    uint32_t* counters;       // [Q, 4]: selected, candidates, done-ticket, spare
-    int32_t* sel;             // [Q, kMaxK] indices above the threshold bin
-    uint64_t* cand;           // [Q, e_stride] candidates in the threshold bin (composite keys)
+    uint32_t* counters;       // [Q, 4]: [0] done-ticket
+    uint32_t* seg_count;      // [Q, e_seg / kSelPerCta] entries each filter CTA kept
+    uint64_t* seg;            // [Q, e_seg] kept entries (64-bit keys), one kSelPerCta segment per filter CTA
     // outputs
     int32_t* idx_out;         // [Q, k]
     float* score_out;         // [Q, k] nullable
