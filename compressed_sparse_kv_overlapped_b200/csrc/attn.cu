@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
     const int T = s1 > s0 ? (int)((s1 - s0 + kTileKeys - 1) / kTileKeys) : 0;
     const int n_items = p.n_items;
     const bool direct = n_items == 1;
+    const bool dep_wait = !(p.hca_nowait && !direct && item >= p.items_front);
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->full[0], 128);
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
                 }
             }
         }
-        grid_dep_wait();  // the selected indices come from the previous kernel
+        if (dep_wait) grid_dep_wait();  // the selected indices come from the previous kernel
         for (int t = 0; t < T; ++t) {
             const int st = t & 1;
             if (t >= 2 && !mbar_wait(&bars->empty[st], ((t >> 1) - 1) & 1, p.status, abort_flag)) break;
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
         cp_async_wait_all();
     } else if (warp == 8) {
         // ------------------------------------------------------------------ MMA issuer
-        grid_dep_wait();
+        if (dep_wait) grid_dep_wait();
         if (lane == 0 && T > 0) {
             constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
             constexpr int N2 = D >= 256 ? 256 : D;
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ softmax + epilogue
-        grid_dep_wait();
+        if (dep_wait) grid_dep_wait();
         grid_dep_launch();
         const int i = lane;
         const bool row_thread = i < 16;
@@ -479,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
 template <int D>
 __global__ void combine_kernel(AttnParams p) {
     constexpr int kMaxBatch = 24;  // partial rows held in registers per pass
+    grid_dep_wait();  // the partials come from the attention grid
     const int h = blockIdx.x, qi = blockIdx.y;
     const int n_items = p.n_items;
     const int lane = threadIdx.x & 31;
@@ -581,12 +583,12 @@ cudaError_t launch_attention_items(const AttnParams& p, int item_begin, int item
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_combine(const AttnParams& p, cudaStream_t stream) {
+cudaError_t launch_combine(const AttnParams& p, cudaStream_t stream, bool pdl) {
     if (p.n_items <= 1) return cudaSuccess;
-    if (p.d == 512) combine_kernel<512><<<dim3((unsigned)p.H, (unsigned)p.Q), 128, 0, stream>>>(p);
-    else if (p.d == 128) combine_kernel<128><<<dim3((unsigned)p.H, (unsigned)p.Q), 32, 0, stream>>>(p);
-    else return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    const dim3 grid((unsigned)p.H, (unsigned)p.Q);
+    if (p.d == 512) return launch_kernel(combine_kernel<512>, grid, dim3(128), 0, stream, pdl, p);
+    if (p.d == 128) return launch_kernel(combine_kernel<128>, grid, dim3(32), 0, stream, pdl, p);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace csa

@@ -84,6 +84,10 @@ struct AttnParams {
     int items_front;
     int kpi_front;
     int kpi_hca;
+    // 1: HCA items do not wait for the preceding launch (griddepcontrol.wait): their inputs (query
+    // table, HCA entries) were written two or more launches earlier, which are complete by the time
+    // this grid may start.  Only the decode chain sets it.
+    int hca_nowait;
     // outputs
     float* out;                 // [Q, H, d]
     float* lse;                 // [Q, H] nullable
@@ -98,7 +102,7 @@ void attn_ws_carve(AttnParams& p, void* ws);
 cudaError_t launch_attention_items(const AttnParams& p, int item_begin, int item_count, cudaStream_t stream,
                                    bool pdl = false);
 // The log-sum-exp merge of all items' partials (only when n_items > 1).
-cudaError_t launch_combine(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_combine(const AttnParams& p, cudaStream_t stream, bool pdl = false);
 
 // Decode helper: append one token per sequence, compress completed entries, build the query table.
 struct AppendParams {
