@@ -22,7 +22,7 @@
 // the two 16-lane halves of every sub-partition, the interleaved M=64 accumulator layout).
 //
 // Warp roles: warps 0-3 softmax + epilogue, warps 4-7 cp.async loaders (gathered rows, manual
-// swizzle, zero-fill for masked slots), warp 8 TMEM allocator + single-thread MMA issuer.  Two
+// swizzle, zero-fill for masked slots), warp 8 TMEM allocator + Q.K^T issuer, warp 9 P.V issuer.  Two
 // key stages; every wait is bounded (kWaitLimitNs) and winds the CTA down on timeout.
 #include "common.cuh"
 #include "kernels.h"
@@ -33,35 +33,42 @@ namespace {
 
 constexpr int kHeadsPad = 64;  // M of every MMA (heads beyond H are zero rows)
 constexpr int kTileKeys = 64;
-constexpr int kThreads = 288;
+constexpr int kStages = 3;     // key tiles in flight
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;
-constexpr uint32_t kColO = 256;
+// TMEM map.  With M = 64 a head row lives in one half (16 lanes) of its warp's 32-lane
+// sub-partition; the Q.K^T operands that share lanes 0-15 and the O accumulator in lanes 16-31
+// together fill all 512 columns:
+//   lanes 0-15:  Q (the A operand of Q.K^T, 2 bf16 per column) in columns [0, D/2),
+//                S buffers b = 0, 1 in columns kColS + 64 b
+//   lanes 16-31: O, dims [0, D) in columns [0, D)
+constexpr uint32_t kColS = 256;
+constexpr uint32_t kLaneO = 16;
 
 template <int D>
 struct Smem {
     static constexpr int NKB = D / 64;                 // 64-wide blocks along d
     static constexpr int kBlock = 64 * 128;            // one block: 64 rows x 128 bytes
-    static constexpr int kQ = 0;
-    static constexpr int kK0 = kQ + NKB * kBlock;
-    static constexpr int kK1 = kK0 + NKB * kBlock;
-    static constexpr int kP0 = kK1 + NKB * kBlock;     // P, double-buffered
+    static constexpr int kStage = NKB * kBlock;        // one key tile
+    static constexpr int kK = 0;                       // kStages key tiles
+    static constexpr int kP0 = kK + kStages * kStage;  // P, double-buffered
     static constexpr int kP1 = kP0 + kBlock;
     static constexpr int kBar = kP1 + kBlock;          // mbarriers
-    static constexpr int kMisc = kBar + 16 * 8;        // tmem base, abort flag, masks
+    static constexpr int kMisc = kBar + 32 * 8;        // tmem base, abort flag, masks
     static constexpr int kRowPtr = kMisc + 64;         // per loader warp: 16 row pointers
     static constexpr int kTotal = kRowPtr + 4 * 16 * 8;
     static constexpr int kAlloc = kTotal + 1024;       // slack for 1024-byte alignment
 };
 
 struct Bars {
-    uint64_t full[2];    // loaders -> MMA / softmax: key stage holds tile t
-    uint64_t empty[2];   // MMA commit after P.V of the tile in the stage
-    uint64_t s_full;     // MMA commit after Q.K^T
-    uint64_t s_free;     // softmax finished reading S
-    uint64_t p_full[2];  // softmax wrote P buffer t&1 (and rescaled O if needed)
-    uint64_t o_done[2];  // MMA commit after the P.V that read P buffer t&1
-    uint64_t fin;        // MMA commit before teardown
+    uint64_t full[kStages];   // loaders -> MMA / softmax: key stage holds tile t
+    uint64_t empty[kStages];  // MMA commit after P.V of the tile in the stage
+    uint64_t s_full[2];       // MMA commit after Q.K^T of tile t into S buffer t&1
+    uint64_t s_free[2];       // softmax finished reading S buffer t&1
+    uint64_t p_full[2];       // softmax wrote P buffer t&1 (and rescaled O if needed)
+    uint64_t o_done[2];       // MMA commit after the P.V that read P buffer t&1
+    uint64_t q_full;          // softmax warps stored Q in TMEM
+    uint64_t fin;             // both MMA issuers committed before teardown
 };
 
 // Per-CTA constants of the key list [CSA slots | raw window | HCA entries] of one query.
@@ -97,13 +104,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     Bars* bars = reinterpret_cast<Bars*>(sm + L::kBar);
-    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);  // [0] tmem base, [1] abort, [2..5] masks
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::kMisc);  // [0] tmem base, [1] abort, [2..7] masks
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     uint16_t* mask16 = reinterpret_cast<uint16_t*>(misc + 2);     // [stage][4 warps]
     const uint32_t sbase = smem_u32(sm);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qi = blockIdx.y, item = blockIdx.x + p_item_base;
+    int qi = blockIdx.y, item = blockIdx.x + p_item_base;
+    if (p.hca_first) {
+        const int n_hca = p.n_items - p.items_front;
+        const int lin = blockIdx.x;
+        if (lin < p.Q * n_hca) {
+            qi = lin / n_hca;
+            item = p.items_front + lin % n_hca;
+        } else {
+            qi = (lin - p.Q * n_hca) / p.items_front;
+            item = (lin - p.Q * n_hca) % p.items_front;
+        }
+    }
     // The query table and sequence lengths come from kernels at least two launches back, which are
     // complete once this grid runs (every kernel of the chain waits before it lets the next start).
     const csa_query qr = p.queries[qi];
@@ -143,17 +161,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
     const bool dep_wait = !(p.hca_nowait && !direct && item >= p.items_front);
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars->full[0], 128);
-        mbar_init(&bars->full[1], 128);
-        mbar_init(&bars->empty[0], 1);
-        mbar_init(&bars->empty[1], 1);
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->s_free, 128);
-        mbar_init(&bars->p_full[0], 128);
-        mbar_init(&bars->p_full[1], 128);
-        mbar_init(&bars->o_done[0], 1);
-        mbar_init(&bars->o_done[1], 1);
-        mbar_init(&bars->fin, 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&bars->full[i], 128);
+            mbar_init(&bars->empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->s_free[i], 128);
+            mbar_init(&bars->p_full[i], 128);
+            mbar_init(&bars->o_done[i], 1);
+        }
+        mbar_init(&bars->q_full, 128);
+        mbar_init(&bars->fin, 2);
         misc[1] = 0;
         fence_mbar_init();
     }
@@ -177,26 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
         constexpr int CPL = CPR / 32 > 0 ? CPR / 32 : 1;  // chunks per lane per row (2 at D = 512)
         const uint32_t lane_blk = (uint32_t)(lane >> 3) * L::kBlock;  // block of chunk `lane`
         const uint32_t lane_c7 = (uint32_t)(lane & 7);
-        if (T > 0) {
-            // Q: 64 (padded) heads, 16 per loader warp; an input, so it may load before the wait
-            for (int r = 0; r < 16; ++r) {
-                const int h = lw * 16 + r;
-                const bool ok = h < p.H;
-                const uint16_t* src = p.q + ((int64_t)qi * p.H + (ok ? h : 0)) * D;
-                const uint32_t dst = sbase + L::kQ + lane_blk + (uint32_t)h * 128u + ((lane_c7 ^ (h & 7)) << 4);
-                if (CPR >= 32) {
-#pragma unroll
-                    for (int u = 0; u < CPL; ++u)
-                        cp_async16(dst + u * 4 * L::kBlock, src + (lane + 32 * u) * 8, ok ? 16u : 0u);
-                } else if (lane < CPR) {
-                    cp_async16(dst, src + lane * 8, ok ? 16u : 0u);
-                }
-            }
-        }
         if (dep_wait) grid_dep_wait();  // the selected indices come from the previous kernel
         for (int t = 0; t < T; ++t) {
-            const int st = t & 1;
-            if (t >= 2 && !mbar_wait(&bars->empty[st], ((t >> 1) - 1) & 1, p.status, abort_flag)) break;
+            const int st = t % kStages;
+            if (t >= kStages && !mbar_wait(&bars->empty[st], ((t / kStages) - 1) & 1, p.status, abort_flag)) break;
             const int64_t tb = s0 + (int64_t)t * kTileKeys;
             bool valid = false;
             if (lane < 16) {
@@ -207,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
             }
             const uint32_t vm = __ballot_sync(0xffffffffu, valid) & 0xFFFFu;
             __syncwarp();
-            const uint32_t kbase = sbase + (st ? L::kK1 : L::kK0) + lane_blk;
+            const uint32_t kbase = sbase + L::kK + (uint32_t)st * L::kStage + lane_blk;
 #pragma unroll 4
             for (int r = 0; r < 16; ++r) {
                 const uint16_t* row = reinterpret_cast<const uint16_t*>(rowptr[r]);
@@ -229,65 +232,58 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
             mbar_arrive(&bars->full[st]);
         }
         cp_async_wait_all();
-    } else if (warp == 8) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------------ MMA issuers
+        // warp 8 issues Q.K^T of every tile (A = Q from TMEM), warp 9 issues P.V (A = P, B = the key
+        // tile read MN-major as V): the two products of neighbouring tiles reach the tensor pipe
+        // independently, so a P.V never waits behind the issue of the next Q.K^T (each issue blocks
+        // its thread for about the product's duration).
         if (dep_wait) grid_dep_wait();
         if (lane == 0 && T > 0) {
-            constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
-            constexpr int N2 = D >= 256 ? 256 : D;
-            constexpr int HALVES = D >= 256 ? D / 256 : 1;
-            constexpr uint32_t id2 = idesc_bf16(64, N2, false, true);
-            const uint32_t tS = tmem + kColS;
-            // descriptor bases; the start address field is (address >> 4) in the low bits
-            const uint64_t dQ = sdesc_kmajor(sbase + L::kQ);
-            const uint64_t dK[2] = {sdesc_kmajor(sbase + L::kK0), sdesc_kmajor(sbase + L::kK1)};
-            const uint64_t dV[2] = {sdesc_mnmajor(sbase + L::kK0, L::kBlock), sdesc_mnmajor(sbase + L::kK1, L::kBlock)};
-            const uint64_t dP[2] = {sdesc_kmajor(sbase + L::kP0), sdesc_kmajor(sbase + L::kP1)};
-            auto gemm1 = [&](int t) {
-                const uint64_t kd = dK[t & 1];
+            if (warp == 8) {
+                constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
+                bool ok = mbar_wait(&bars->q_full, 0, p.status, abort_flag);
+                for (int g1 = 0; ok && g1 < T; ++g1) {
+                    const int st = g1 % kStages;
+                    if (!mbar_wait(&bars->full[st], (g1 / kStages) & 1, p.status, abort_flag)) break;
+                    if (g1 >= 2 && !mbar_wait(&bars->s_free[g1 & 1], ((g1 >> 1) - 1) & 1, p.status, abort_flag)) break;
+                    tc_fence_after();
+                    const uint64_t kd = sdesc_kmajor(sbase + L::kK + (uint32_t)st * L::kStage);
+                    const uint32_t tS = tmem + kColS + (uint32_t)(g1 & 1) * 64u;
 #pragma unroll 1
-                for (int kb = 0; kb < L::NKB; ++kb) {
+                    for (int kb = 0; kb < L::NKB; ++kb) {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            // K elements [64 kb + 16 ks, +16): columns 32 kb + 8 ks of Q, bytes of the tile block
+                            umma_bf16_ts(tS, tmem + (uint32_t)(kb * 32 + ks * 8),
+                                         kd + (uint64_t)((kb * L::kBlock + ks * 32) >> 4), id1, (kb | ks) != 0);
+                        }
+                    }
+                    umma_commit(&bars->s_full[g1 & 1]);
+                }
+            } else {
+                constexpr int N2 = D >= 256 ? 256 : D;
+                constexpr int HALVES = D >= 256 ? D / 256 : 1;
+                constexpr uint32_t id2 = idesc_bf16(64, N2, false, true);
+                for (int g2 = 0; g2 < T; ++g2) {
+                    if (!mbar_wait(&bars->p_full[g2 & 1], (g2 >> 1) & 1, p.status, abort_flag)) break;
+                    tc_fence_after();
+                    const int st = g2 % kStages;
+                    const uint64_t vd = sdesc_mnmajor(sbase + L::kK + (uint32_t)st * L::kStage, L::kBlock);
+                    const uint64_t pd = sdesc_kmajor(sbase + ((g2 & 1) ? L::kP1 : L::kP0));
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t off = (uint64_t)((kb * L::kBlock + ks * 32) >> 4);
-                        umma_bf16(tS, dQ + off, kd + off, id1, (kb | ks) != 0);
-                    }
-                }
-            };
-            auto gemm2 = [&](int t) {
-                const uint64_t vd = dV[t & 1], pd = dP[t & 1];
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-                    for (int half = 0; half < HALVES; ++half) {
-                        // V rows ks*16 .. ks*16+15 of the key tile, dims [half*256, half*256 + N2)
-                        const uint64_t b = vd + (uint64_t)((half * 4 * L::kBlock + ks * 16 * 128) >> 4);
-                        const uint32_t tO = tmem + kColO + ((uint32_t)(half * 16) << 16);
-                        umma_bf16(tO, pd + (uint64_t)((ks * 32) >> 4), b, id2, (t > 0 || ks > 0) ? 1u : 0u);
+                        for (int half = 0; half < HALVES; ++half) {
+                            // V rows ks*16 .. ks*16+15 of the key tile, dims [half*256, half*256 + N2)
+                            const uint64_t b = vd + (uint64_t)((half * 4 * L::kBlock + ks * 16 * 128) >> 4);
+                            const uint32_t tO = tmem + (kLaneO << 16) + (uint32_t)(half * 256);
+                            umma_bf16(tO, pd + (uint64_t)((ks * 32) >> 4), b, id2, (g2 > 0 || ks > 0) ? 1u : 0u);
+                        }
                     }
+                    umma_commit(&bars->empty[st]);
+                    umma_commit(&bars->o_done[g2 & 1]);
                 }
-            };
-            bool ok = mbar_wait(&bars->full[0], 0, p.status, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                gemm1(0);
-                umma_commit(&bars->s_full);
-            }
-            for (int t = 0; ok && t < T; ++t) {
-                if (t + 1 < T) {
-                    ok = mbar_wait(&bars->full[(t + 1) & 1], ((t + 1) >> 1) & 1, p.status, abort_flag) &&
-                         mbar_wait(&bars->s_free, t & 1, p.status, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    gemm1(t + 1);
-                    umma_commit(&bars->s_full);
-                }
-                ok = mbar_wait(&bars->p_full[t & 1], (t >> 1) & 1, p.status, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                gemm2(t);
-                umma_commit(&bars->empty[t & 1]);
-                umma_commit(&bars->o_done[t & 1]);
             }
             umma_commit(&bars->fin);
             mbar_wait(&bars->fin, 0, p.status, nullptr);
@@ -295,142 +291,180 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ softmax + epilogue
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t o_base = tmem + lane_base + (kLaneO << 16);
+        if (T > 0) {
+            // Q (an input, so before the wait) in the A layout of Q.K^T: head row 16w + r in lane r
+            // of warp w's sub-partition, dims 2c and 2c + 1 in column c.  Written with the 16x256b
+            // shape, so every lane takes part: lane i writes rows i/4 and i/4 + 8 at columns
+            // 8k + 2(i%4) and 8k + 2(i%4) + 1, i.e. 8 bytes of each of those rows per 8 columns.
+            const int qa = lane >> 2, qc = (lane & 3) * 2;
+            const int h0 = warp * 16 + qa, h1 = h0 + 8;
+            const uint2* q0 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h0 < p.H ? h0 : 0)) * D);
+            const uint2* q1 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h1 < p.H ? h1 : 0)) * D);
+#pragma unroll 1
+            for (int cb = 0; cb < D / 2; cb += 128) {
+                uint32_t r[2][32];
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int col = cb + g * 64 + 8 * k + qc;  // a column holds 2 dims: uint2 index col / 2
+                        const bool in = cb + g * 64 < D / 2;
+                        const uint2 v0 = (in && h0 < p.H) ? q0[col / 2] : make_uint2(0, 0);
+                        const uint2 v1 = (in && h1 < p.H) ? q1[col / 2] : make_uint2(0, 0);
+                        r[g][4 * k] = v0.x; r[g][4 * k + 1] = v0.y; r[g][4 * k + 2] = v1.x; r[g][4 * k + 3] = v1.y;
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < 2; ++g)
+                    if (cb + g * 64 < D / 2) tmem_st_16x256_x8(tmem + lane_base + (uint32_t)(cb + g * 64), r[g]);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars->q_full);
+        }
         if (dep_wait) grid_dep_wait();
         grid_dep_launch();
         const int i = lane;
-        const bool row_thread = i < 16;
-        const int h = warp * 16 + (i & 15);                 // head row handled by this lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        constexpr int OC = D >= 256 ? 256 : D;              // O columns held by each lane
-        float m_run = -INFINITY, l_run = 0.f;
+        // S and O are read with the 16x256b shape, so all 32 lanes work: lane i holds rows ra = i/4
+        // and ra + 8 of the warp's 16, at columns 8k + cq and 8k + cq + 1 of every 64-column group;
+        // the four lanes of a quad share a row and combine their partial max / sum by shuffles.
+        const int ra = i >> 2, cq = (i & 3) * 2;
+        const int hr[2] = {warp * 16 + ra, warp * 16 + ra + 8};
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
         bool ok = true;
         for (int t = 0; t < T; ++t) {
-            const int st = t & 1;
-            ok = mbar_wait(&bars->s_full, t & 1, p.status, abort_flag) &&
-                 mbar_wait(&bars->full[st], (t >> 1) & 1, p.status, abort_flag);
+            const int sb = t & 1, st = t % kStages;
+            ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, p.status, abort_flag) &&
+                 mbar_wait(&bars->full[st], (t / kStages) & 1, p.status, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            float s[64];
+            float s[2][16];  // [row ra / ra+8][2k + e] = column 8k + cq + e
             {
-                uint32_t r[4][16];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tmem + lane_base + kColS + q4 * 16, r[q4]);
+                uint32_t r[32];
+                tmem_ld_16x256_x8(tmem + lane_base + kColS + (uint32_t)sb * 64u, r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) s[q4 * 16 + j] = __uint_as_float(r[q4][j]);
+                for (int k = 0; k < 8; ++k) {
+                    s[0][2 * k] = __uint_as_float(r[4 * k]);
+                    s[0][2 * k + 1] = __uint_as_float(r[4 * k + 1]);
+                    s[1][2 * k] = __uint_as_float(r[4 * k + 2]);
+                    s[1][2 * k + 1] = __uint_as_float(r[4 * k + 3]);
+                }
             }
             tc_fence_before();
-            mbar_arrive(&bars->s_free);
+            mbar_arrive(&bars->s_free[sb]);
             const uint64_t vmask = (uint64_t)mask16[st * 4 + 0] | ((uint64_t)mask16[st * 4 + 1] << 16) |
                                    ((uint64_t)mask16[st * 4 + 2] << 32) | ((uint64_t)mask16[st * 4 + 3] << 48);
-            float mx = -INFINITY;
             const float sc = p.scale_log2;
-            if (vmask == ~0ull) {
+            float mx[2] = {-INFINITY, -INFINITY};
+            const uint64_t lm = vmask >> cq;  // bit 8k + e: column 8k + cq + e valid
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    s[j] *= sc;
-                    mx = fmaxf(mx, s[j]);
-                }
-            } else {
+            for (int k = 0; k < 8; ++k) {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    s[j] = ((vmask >> j) & 1ull) ? s[j] * sc : -INFINITY;
-                    mx = fmaxf(mx, s[j]);
+                for (int e = 0; e < 2; ++e) {
+                    const bool v = (lm >> (8 * k + e)) & 1ull;
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        s[rr][2 * k + e] = v ? s[rr][2 * k + e] * sc : -INFINITY;
+                        mx[rr] = fmaxf(mx[rr], s[rr][2 * k + e]);
+                    }
                 }
             }
-            // lazy rescaling: move the reference max only when it grows by more than 2^8
-            float alpha = 1.f;
-            if (mx > m_run + 8.f) {
-                alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - mx);
-                m_run = mx;
-                l_run *= alpha;
+            float alpha[2] = {1.f, 1.f};
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+                // lazy rescaling: move the reference max only when it grows by more than 2^8
+                if (mx[rr] > m_run[rr] + 8.f) {
+                    alpha[rr] = (m_run[rr] == -INFINITY) ? 0.f : exp2f(m_run[rr] - mx[rr]);
+                    m_run[rr] = mx[rr];
+                    l_run[rr] *= alpha[rr];
+                }
             }
-            // O must hold every earlier P.V before it is rescaled (rare)
-            const bool any = __any_sync(0xffffffffu, row_thread && alpha != 1.f);
+            // O must hold every earlier P.V before it is rescaled (rare); O lives in lanes 16-31,
+            // in the same row / column layout as S
+            const bool any = __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f);
             if (t > 0 && any) {
                 ok = mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const float a_me = __shfl_sync(0xffffffffu, alpha, i & 15);
 #pragma unroll 1
-                for (int c = 0; c < OC; c += 64) {
-                    uint32_t r[4][16];
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tmem + lane_base + kColO + c + q4 * 16, r[q4]);
+                for (int c = 0; c < D; c += 64) {
+                    uint32_t r[32];
+                    tmem_ld_16x256_x8(o_base + (uint32_t)c, r);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) r[q4][j] = __float_as_uint(__uint_as_float(r[q4][j]) * a_me);
-                        tmem_st16(tmem + lane_base + kColO + c + q4 * 16, r[q4]);
+                    for (int k = 0; k < 8; ++k) {
+                        r[4 * k] = __float_as_uint(__uint_as_float(r[4 * k]) * alpha[0]);
+                        r[4 * k + 1] = __float_as_uint(__uint_as_float(r[4 * k + 1]) * alpha[0]);
+                        r[4 * k + 2] = __float_as_uint(__uint_as_float(r[4 * k + 2]) * alpha[1]);
+                        r[4 * k + 3] = __float_as_uint(__uint_as_float(r[4 * k + 3]) * alpha[1]);
                     }
+                    tmem_st_16x256_x8(o_base + (uint32_t)c, r);
                 }
                 tmem_st_wait();
             }
             // P buffer t&1 is free once the P.V of tile t-2 finished
             if (t >= 2) {
-                ok = mbar_wait(&bars->o_done[st], ((t >> 1) - 1) & 1, p.status, abort_flag);
+                ok = mbar_wait(&bars->o_done[sb], ((t >> 1) - 1) & 1, p.status, abort_flag);
                 if (!ok) break;
             }
-            if (row_thread) {
-                // masked slots hold -inf: 2^(-inf - m) = 0; while the row has seen no key, m_use = 0
-                const float m_use = m_run == -INFINITY ? 0.f : m_run;
-                float lsum = 0.f;
-                const uint32_t prow = sbase + (st ? L::kP1 : L::kP0);
+            {
+                // masked slots hold -inf: 2^(-inf - m) = 0; while a row has seen no key, m_use = 0
+                const uint32_t prow = sbase + (sb ? L::kP1 : L::kP0) + (uint32_t)(i & 3) * 4u;
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    uint32_t w4[4];
+                for (int rr = 0; rr < 2; ++rr) {
+                    const float m_use = m_run[rr] == -INFINITY ? 0.f : m_run[rr];
+                    float lsum = 0.f;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float p0 = fast_exp2(s[c8 * 8 + 2 * u] - m_use);
-                        const float p1 = fast_exp2(s[c8 * 8 + 2 * u + 1] - m_use);
+                    for (int k = 0; k < 8; ++k) {
+                        const float p0 = fast_exp2(s[rr][2 * k] - m_use);
+                        const float p1 = fast_exp2(s[rr][2 * k + 1] - m_use);
                         lsum += p0 + p1;
-                        w4[u] = pack_bf16x2(p0, p1);
+                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(prow + sw128_offset(hr[rr], k)),
+                                     "r"(pack_bf16x2(p0, p1))
+                                     : "memory");
                     }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_offset(h, c8)),
-                                 "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
-                                 : "memory");
+                    l_run[rr] += lsum;  // this lane's part of the row sum; the quad adds them up at the end
                 }
-                l_run += lsum;
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->p_full[st]);
+            mbar_arrive(&bars->p_full[sb]);
         }
-        // ---- epilogue: TMEM -> shared memory (Q and the key stages are free now) -> coalesced stores
+        // ---- epilogue: TMEM -> shared memory (the key stages are free now) -> bulk stores
         if (ok && T > 0) ok = mbar_wait(&bars->o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, p.status, abort_flag);
-        const float l_row = __shfl_sync(0xffffffffu, l_run, i & 15);
-        const float m_row = __shfl_sync(0xffffffffu, m_run, i & 15);
-        const bool has = ok && T > 0 && l_row > 0.f;
-        const float inv = has ? 1.f / l_row : 0.f;
-        const int dim0 = row_thread ? 0 : 256;
-        const bool mine = row_thread || D >= 512;  // lanes 16-31 hold dims 256-511 when D = 512
-        // staging rows of D floats, padded by 4 floats so 16-byte row-strided writes spread banks
+        float inv[2];
+        bool has[2];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
+            l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
+            has[rr] = ok && T > 0 && l_run[rr] > 0.f;
+            inv[rr] = has[rr] ? 1.f / l_run[rr] : 0.f;
+        }
+        // staging rows of D floats, padded by 4 floats so row-strided writes spread over the banks
         constexpr int kStride = D + 4;
-        float* stage = reinterpret_cast<float*>(sm + L::kQ);  // Q and both key stages are free now
-        static_assert(64 * (D + 4) * 4 <= 3 * L::NKB * L::kBlock, "epilogue staging exceeds Q + key stages");
-        if (has) {
+        float* stage = reinterpret_cast<float*>(sm + L::kK);
+        static_assert(64 * (D + 4) * 4 <= kStages * Smem<D>::kStage, "epilogue staging exceeds the key stages");
+        const bool write_o = ok && T > 0;
+        if (write_o) {
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < OC; c += 64) {
-                uint32_t r[4][16];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tmem + lane_base + kColO + c + q4 * 16, r[q4]);
+            for (int c = 0; c < D; c += 64) {
+                uint32_t r[32];
+                tmem_ld_16x256_x8(o_base + (uint32_t)c, r);
                 tmem_ld_wait();
-                if (mine) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-                        for (int j = 0; j < 16; j += 4) {
-                            float4 v;
-                            v.x = __uint_as_float(r[q4][j]) * inv;
-                            v.y = __uint_as_float(r[q4][j + 1]) * inv;
-                            v.z = __uint_as_float(r[q4][j + 2]) * inv;
-                            v.w = __uint_as_float(r[q4][j + 3]) * inv;
-                            *reinterpret_cast<float4*>(stage + h * kStride + dim0 + c + q4 * 16 + j) = v;
-                        }
+                for (int k = 0; k < 8; ++k) {
+                    const int col = c + 8 * k + cq;
+                    *reinterpret_cast<float2*>(stage + hr[0] * kStride + col) =
+                        make_float2(__uint_as_float(r[4 * k]) * inv[0], __uint_as_float(r[4 * k + 1]) * inv[0]);
+                    *reinterpret_cast<float2*>(stage + hr[1] * kStride + col) =
+                        make_float2(__uint_as_float(r[4 * k + 2]) * inv[1], __uint_as_float(r[4 * k + 3]) * inv[1]);
                 }
             }
         }
@@ -438,8 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
         fence_proxy_async_smem();
         asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps (128 threads)
         const int rows = p.H < kHeadsPad ? p.H : kHeadsPad;
-        if (has) {
-            // one lane per warp hands 16 staged rows to the bulk-copy engine
+        if (write_o) {
+            // one lane per warp hands the warp's 16 staged rows to the bulk-copy engine
             if (i == 0) {
                 for (int hh = warp * 16; hh < warp * 16 + 16 && hh < rows; ++hh) {
                     float* dst = direct ? p.out + ((int64_t)qi * p.H + hh) * D
@@ -457,12 +491,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
                     make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
-        if (row_thread && h < p.H) {
-            const float lse_v = has ? (m_row + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
-            if (direct) {
-                if (p.lse) p.lse[(int64_t)qi * p.H + h] = lse_v;
-            } else {
-                p.part_lse[((int64_t)qi * n_items + item) * kHeadsPad + h] = lse_v;
+        if ((i & 3) == 0) {
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int h = hr[rr];
+                if (h >= p.H) continue;
+                const float lse_v = has[rr] ? (m_run[rr] + log2f(l_run[rr])) * 0.69314718055994531f : -INFINITY;
+                if (direct) {
+                    if (p.lse) p.lse[(int64_t)qi * p.H + h] = lse_v;
+                } else {
+                    p.part_lse[((int64_t)qi * n_items + item) * kHeadsPad + h] = lse_v;
+                }
             }
         }
     }
@@ -554,8 +593,8 @@ cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, 
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    return launch_kernel(attn_kernel<D>, dim3((unsigned)item_count, (unsigned)p.Q), dim3(kThreads), L::kAlloc, stream,
-                         pdl, p, item_begin);
+    const dim3 grid = p.hca_first ? dim3((unsigned)(p.n_items * p.Q)) : dim3((unsigned)item_count, (unsigned)p.Q);
+    return launch_kernel(attn_kernel<D>, grid, dim3(kThreads), L::kAlloc, stream, pdl, p, item_begin);
 }
 
 }  // namespace

@@ -603,6 +603,7 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
         // every item in one launch after the top-k; the HCA items need no top-k and start as soon
         // as the select kernel frees SMs
         ap2.hca_nowait = pdl ? 1 : 0;
+        ap2.hca_first = (pl.items.n_items > 1 && pl.items.items_front > 0) ? 1 : 0;
         rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
                        ws_index, false, st, stream, ev[2], pdl);
         if (rc) return rc;

@@ -5,7 +5,7 @@
 // whose caching allocator owns every device buffer and forbids direct cudaMalloc, real-time
 // serving loops that must not allocate after start-up, or thin foreign-language bindings that see
 // only the caller's input and output pointers.  For them this entry point keeps its scratch in a
-// fixed array compiled into the library (kScratchBytes, about 12.9 MiB per device), so a call
+// fixed array compiled into the library (kScratchBytes, about 12.1 MiB per device), so a call
 // needs nothing but inputs, outputs and a stream.  The array occupies device memory on every GPU
 // that loads the library until the process exits.
 //
@@ -20,13 +20,10 @@ namespace {
 
 constexpr int kNoAllocMaxQ = 16;
 constexpr int64_t kNoAllocMaxSlots = int64_t(1) << 20;  // Q * score-row stride
-// Upper bound of index_ws_bytes(Q, e_stride) under the two limits above: histograms, counters,
-// per-CTA segment counts, fp32 scores and the 64-bit kept-entry segments (each query's row rounded
-// up to whole kSelPerCta segments).
-constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * kHistBins * 4 + 256 + 256 +
-                                 size_t(kNoAllocMaxSlots / kSelPerCta + kNoAllocMaxQ) * 4 + 256 +
-                                 size_t(kNoAllocMaxSlots) * 4 + 256 +
-                                 size_t(kNoAllocMaxSlots + kNoAllocMaxQ * kSelPerCta) * 8 + 256;
+// Upper bound of index_ws_bytes(Q, e_stride) under the two limits above: histograms, fp32 scores
+// and the 64-bit kept-entry segments (each query's score row plus 128 entries).
+constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * kHistBins * 4 + 256 + size_t(kNoAllocMaxSlots) * 4 + 256 +
+                                 size_t(kNoAllocMaxSlots + kNoAllocMaxQ * 8 * kSelClusterMax) * 8 + 256;
 
 __device__ __align__(256) unsigned char g_index_scratch[kScratchBytes];
 
@@ -95,7 +92,7 @@ extern "C" int csa_index_topk_noalloc(const csa_dims* dims, const csa_seq* seqs,
     ip.score_out = score_out;
     ip.status = device_status();
     index_ws_carve(ip, scratch, Q, es);
-    // the histogram and counters must start at zero; the previous call's contents are still there
+    // the histogram must start at zero; clear it in case an earlier call was cut short
     e = launch_index_topk(ip, max_e, stream, /*zero_ws=*/true);
     if (e != cudaSuccess) return set_error(CSA_ERR_CUDA, "csa_index_topk_noalloc: launch: %s", cudaGetErrorString(e));
     return CSA_OK;

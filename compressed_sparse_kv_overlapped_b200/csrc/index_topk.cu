@@ -166,12 +166,56 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(IndexParams p)
 }
 
 // ---- select ----------------------------------------------------------------------------------
+//
+// One thread-block cluster of F = sel_cluster CTAs per query (1..kSelClusterMax).  CTA c filters the scores of entries
+// [c*span, (c+1)*span): every CTA derives the threshold bin from the scan's histogram and keeps the
+// entries of that bin and above, as 64-bit keys in index order, in its own shared memory; it then
+// publishes its count in the leader CTA (rank 0).  After a cluster barrier every CTA knows its
+// offset and pushes its keys into the leader's list through distributed shared memory; after a
+// second barrier the leader radix-selects the exact threshold among the bin's members and
+// compacts the k indices, ascending.  A list longer than shared memory holds goes through the
+// global segment buffer instead, in the same order.
 
-constexpr int kSelPerThread = kSelPerCta / kSelectThreads;          // 8 scores per thread
-constexpr int kListSmem = 8192;                                     // kept entries the last CTA holds
+constexpr int kSelPerMax = 64;                           // scores per thread per round
+constexpr int kSelBufMax = kSelPerMax * kSelectThreads;  // scores a CTA stages in shared memory per round
+constexpr int kStageSmem = 4096;  // kept keys a CTA stages in its own shared memory
+constexpr int kListSmem = 8192;   // kept keys the leader holds (in its score buffer, once filtered)
 
 __device__ __forceinline__ uint64_t composite(uint32_t key, int64_t j) {
     return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every thread of every CTA of the cluster; orders all earlier memory accesses (shared, distributed
+// shared and global) before all later ones at cluster scope.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address in the shared::cluster window of the location `p` (this CTA's shared memory) in CTA `rank`.
+__device__ __forceinline__ uint32_t map_rank(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u64(uint32_t addr, uint64_t v) {
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
 }
 
 // Block-wide suffix sums over kHistBins bins: suf[b] = sum of hist[b' >= b].  Thread t owns bins
@@ -244,55 +288,41 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
     return excl;
 }
 
-// The kept list of one query: the filter CTAs' segments concatenated in CTA order (so in index
-// order).  Entry i lives in segment c = the last with off[c] <= i.
+// The kept list of one query: the cluster CTAs' key runs concatenated in rank order (so in index
+// order), either gathered in the leader's shared memory (`cache`) or left in the global segment
+// buffer, where run c starts at seg + c*span and entry i lives in the last run c with off[c] <= i.
 struct KeptList {
-    const uint64_t* seg;     // [F][kSelPerCta]
-    const uint32_t* off;     // [F + 1] exclusive prefix of the segment counts (shared memory)
-    int F;
-    const uint64_t* cache;   // the whole list in shared memory, or nullptr
+    const uint64_t* seg;
+    const uint32_t* off;     // [F + 1] exclusive prefix of the run lengths
+    int F;                   // CTAs in the cluster
+    int64_t span;
+    const uint64_t* cache;
     __device__ __forceinline__ uint64_t get(uint32_t i) const {
         if (cache) return cache[i];
-        int lo = 0, hi = F - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (off[mid] <= i) lo = mid; else hi = mid - 1;
-        }
-        return __ldcg(reinterpret_cast<const unsigned long long*>(seg) + (int64_t)lo * kSelPerCta + (i - off[lo]));
+        int c = 0;
+        for (int r = 1; r < F; ++r) c += off[r] <= i ? 1 : 0;
+        return __ldcg(reinterpret_cast<const unsigned long long*>(seg) + (int64_t)c * span + (i - off[c]));
     }
 };
 
 // Exact selection of the `need` largest keys among the list entries whose top 11 bits equal top11
 // (the threshold-bin members; entries of higher bins are kept regardless).  Returns T with exactly
-// `need` of those members >= T.  Radix passes of 11 bits over bits 52..0 (counted with
-// warp-aggregated shared-memory atomics, so equal digits do not serialize); stops as soon as the
-// chosen digit holds exactly the remaining count.
+// `need` of those members >= T.  Radix passes of 11 bits over bits 52..0, counted with
+// shared-memory atomics; stops as soon as the chosen digit holds exactly the remaining count.
 __device__ uint64_t radix_threshold(const KeptList& L, uint32_t n, uint32_t need, uint32_t top11, uint32_t* cnt,
                                     uint32_t* suf, uint32_t* misc) {
     uint64_t prefix = (uint64_t)top11 << 53;
     uint64_t mask = (uint64_t)0x7FF << 53;
     uint32_t remaining = need;
-    const int lane = threadIdx.x & 31;
     for (int shift = 42;; shift -= 11) {
         const int sh = shift < 0 ? 0 : shift;
         const int bits = shift < 0 ? 11 + shift : 11;
         const uint32_t dmask = (1u << bits) - 1u;
         for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) cnt[i] = 0;
         __syncthreads();
-        const uint32_t n_round = (n + 31u) & ~31u;
-        for (uint32_t i = threadIdx.x; i < n_round; i += blockDim.x) {
-            bool match = false;
-            uint32_t dg = 0;
-            if (i < n) {
-                const uint64_t v = L.get(i);
-                match = (v & mask) == prefix;
-                dg = (uint32_t)(v >> sh) & dmask;
-            }
-            const uint32_t active = __ballot_sync(0xffffffffu, match);
-            if (match) {
-                const uint32_t peers = __match_any_sync(active, dg);
-                if (lane == __ffs(peers) - 1) atomicAdd(&cnt[dg], (uint32_t)__popc(peers));
-            }
+        for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint64_t v = L.get(i);
+            if ((v & mask) == prefix) atomicAdd(&cnt[(uint32_t)(v >> sh) & dmask], 1u);
         }
         __syncthreads();
         suffix_find(cnt, suf, misc, remaining, misc + 48);  // misc[0..15]: warp totals
@@ -307,25 +337,47 @@ __device__ uint64_t radix_threshold(const KeptList& L, uint32_t n, uint32_t need
     }
 }
 
+// Dynamic shared memory of the select kernel.
+struct SelSmem {
+    static constexpr int kHist = 0;                          // u32[kHistBins]
+    static constexpr int kSuf = kHist + kHistBins * 4;       // u32[kHistBins]
+    static constexpr int kMisc = kSuf + kHistBins * 4;       // u32[64]
+    static constexpr int kXcnt = kMisc + 64 * 4;             // u32[32]: the leader's run lengths (| overflow bit)
+    static constexpr int kOffs = kXcnt + 32 * 4;             // u32[32]: exclusive prefix, F + 1 used
+    static constexpr int kStage = kOffs + 32 * 4;            // u64[kStageSmem]: this CTA's run
+    static constexpr int kBuf = kStage + kStageSmem * 8;     // f32[sel_buf] scores; the leader's list
+                                                             // (u64[kListSmem]) once it has filtered
+    // dynamic shared memory of a launch staging `buf` scores per round
+    static constexpr size_t bytes(int64_t buf) {
+        return (size_t)kBuf + (buf * 4 > (int64_t)kListSmem * 8 ? (size_t)buf * 4 : (size_t)kListSmem * 8);
+    }
+};
+
 __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);          // kHistBins
-    uint32_t* suf = hist + kHistBins;                                  // kHistBins
-    uint32_t* misc = suf + kHistBins;                                  // 64
-    uint64_t* lst = reinterpret_cast<uint64_t*>(misc + 64);            // kListSmem
-    uint32_t* offs = reinterpret_cast<uint32_t*>(lst + kListSmem);    // filter CTAs + 1
-    __shared__ uint32_t s_last;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kHist);
+    uint32_t* suf = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kSuf);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kMisc);
+    uint32_t* xcnt = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kXcnt);
+    uint32_t* offs = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kOffs);
+    uint64_t* stage = reinterpret_cast<uint64_t*>(smem_raw + SelSmem::kStage);
+    uint64_t* lst = reinterpret_cast<uint64_t*>(smem_raw + SelSmem::kBuf);
     __shared__ uint32_t s_wsum[kSelectThreads / 32];
+    __shared__ uint64_t s_bar;
+    __shared__ int s_abort;
     grid_dep_wait();  // scores and histogram come from the scan kernel
     grid_dep_launch();
 
+    // Every branch below that returns before the cluster barriers depends only on the query, so all
+    // CTAs of a cluster take it together.
     const int qi = blockIdx.y;
+    const uint32_t rank = cluster_rank();
     const csa_query qr = p.queries[qi];
     const csa_seq sq = p.seqs[qr.seq];
     const bool valid = qr.len >= 1 && qr.len <= sq.len;
     int64_t E = valid ? qr.len / p.m : 0;
-    if (E > p.max_entries) {  // the grid was sized for fewer entries: refuse rather than guess
-        if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, CSA_ERR_INDEX);
+    if (E > p.max_entries) {  // the launch was sized for fewer entries: refuse rather than guess
+        if (threadIdx.x == 0 && rank == 0) report(p.status, CSA_ERR_INDEX);
         E = 0;
     }
     int32_t* out = p.idx_out + (int64_t)qi * p.k;
@@ -333,7 +385,7 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     const float* srow = p.scores + (int64_t)qi * p.e_stride;
 
     if (E <= p.k) {  // select everything: no scores were computed
-        if (blockIdx.x != 0) return;
+        if (rank != 0) return;
         for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
             out[i] = i < E ? i : -1;
             if (sout) sout[i] = __int_as_float(0x7FC00000);
@@ -356,6 +408,37 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
         return;
     }
 
+    const int F = p.sel_cluster;
+    const int64_t c0 = (int64_t)rank * p.sel_span;
+    const int64_t c1 = min(E, c0 + p.sel_span);
+    // Rounds of sel_buf scores are staged in shared memory by bulk copies (the first round's copy
+    // goes out before the histogram loads).
+    float* sbuf = reinterpret_cast<float*>(smem_raw + SelSmem::kBuf);
+    const uint32_t sbuf_addr = smem_u32(sbuf);
+    const int lane = threadIdx.x & 31;
+    const int L = p.sel_per;  // entries per thread per round: a power of two, 4..kSelPerMax
+    const int G = L / 4;
+    if (threadIdx.x == 0) {
+        mbar_init(&s_bar, 1);
+        fence_mbar_init();
+        s_abort = 0;
+    }
+    __syncthreads();
+    // thread 0: copy the 16-byte-multiple part of round [rb, rb + n) into sbuf
+    auto issue_round = [&](int64_t rb) {
+        const int64_t n = min((int64_t)p.sel_buf, c1 - rb);
+        const uint32_t bytes = (uint32_t)(n & ~(int64_t)3) * 4u;
+        fence_proxy_async_smem();  // earlier generic accesses to sbuf come first
+        if (bytes == 0) {
+            mbar_arrive(&s_bar);
+            return;
+        }
+        mbar_arrive_expect_tx(&s_bar, bytes);
+        for (uint32_t off = 0; off < bytes; off += 65536u)
+            bulk_load(sbuf_addr + off, srow + rb + off / 4u, min(65536u, bytes - off), &s_bar);
+    };
+    if (threadIdx.x == 0 && c0 < c1) issue_round(c0);
+
     // 1. threshold bin (every CTA of the query finds the same one)
     const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
     for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = __ldcg(gh + i);
@@ -363,82 +446,113 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     suffix_find(hist, suf, misc, (uint32_t)p.k, misc + 32);
     const uint32_t b1 = misc[32];
     const uint32_t above = misc[33];
-    if (b1 == 0xFFFFFFFFu) {  // histogram holds fewer than k scores: cannot happen
-        if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
-        return;
-    }
     const uint32_t need = (uint32_t)p.k - above;
-    const uint32_t n_bin = hist[b1];  // members of the threshold bin (over all CTAs)
+    const uint32_t n_bin = b1 == 0xFFFFFFFFu ? 0u : hist[b1];  // members of the threshold bin
+    const float thr = key_float(b1 << 21);                     // the smallest float of bin b1
+    bool failed = b1 == 0xFFFFFFFFu;  // histogram holds fewer than k scores: cannot happen
 
-    // 2. keep this CTA's entries of bin >= b1, in index order, in its own segment
-    const int64_t j0 = (int64_t)blockIdx.x * kSelPerCta + (int64_t)threadIdx.x * kSelPerThread;
-    float sv[kSelPerThread];
-    if (j0 + kSelPerThread <= E) {
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(srow + j0));
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(srow + j0 + 4));
-        sv[0] = a.x; sv[1] = a.y; sv[2] = a.z; sv[3] = a.w; sv[4] = b.x; sv[5] = b.y; sv[6] = b.z; sv[7] = b.w;
-    } else {
-#pragma unroll
-        for (int u = 0; u < kSelPerThread; ++u) sv[u] = j0 + u < E ? __ldcg(srow + j0 + u) : 0.f;
-    }
-    uint32_t nk = 0, kf = 0;
-#pragma unroll
-    for (int u = 0; u < kSelPerThread; ++u) {
-        if (j0 + u < E && (float_key(sv[u]) >> 21) >= b1) { ++nk; kf |= 1u << u; }
-    }
-    uint32_t cta_total;
-    uint32_t pos = block_excl_scan(nk, s_wsum, &cta_total);
-    uint64_t* myseg = p.seg + (int64_t)qi * p.e_seg + (int64_t)blockIdx.x * kSelPerCta;
-#pragma unroll
-    for (int u = 0; u < kSelPerThread; ++u)
-        if (kf & (1u << u)) myseg[pos++] = composite(float_key(sv[u]), j0 + u);
-    if (threadIdx.x == 0) p.seg_count[(int64_t)qi * (p.e_seg / kSelPerCta) + blockIdx.x] = cta_total;
-
-    // 3. the last CTA of this query finishes the selection
-    uint32_t* ctr = p.counters + (int64_t)qi * 4;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(&ctr[0], 1u) == gridDim.x - 1) ? 1u : 0u;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-
-    const int F = gridDim.x;
-    // exclusive prefix of the segment counts (8 per thread)
-    {
-        const uint32_t* gc = p.seg_count + (int64_t)qi * (p.e_seg / kSelPerCta);
-        uint32_t c8[8], tot = 0;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int c = threadIdx.x * 8 + u;
-            c8[u] = c < F ? __ldcg(gc + c) : 0u;
-            tot += c8[u];
-        }
-        uint32_t all;
-        uint32_t run = block_excl_scan(tot, s_wsum, &all);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int c = threadIdx.x * 8 + u;
-            if (c <= F) offs[c] = run;
-            run += c8[u];
-        }
+    // 2. keep this CTA's entries of bin >= b1, in index order
+    uint64_t* gseg = p.seg + (int64_t)qi * p.e_seg + (int64_t)rank * p.sel_span;
+    uint32_t n_mine = 0;
+    bool spilled = false;  // the run lives in gseg instead of `stage`
+    uint32_t phase = 0;
+    for (int64_t rb = c0; rb < c1; rb += p.sel_buf) {
+        const int64_t n = min((int64_t)p.sel_buf, c1 - rb);
+        const int64_t n16 = n & ~(int64_t)3;
+        if (threadIdx.x < n - n16) sbuf[n16 + threadIdx.x] = __ldg(srow + rb + n16 + threadIdx.x);
+        // a wait that runs out leaves this CTA's run empty (and the status word set); the CTA still
+        // takes both cluster barriers below
+        if (!mbar_wait(&s_bar, phase, p.status, &s_abort)) failed = true;
+        phase ^= 1u;
         __syncthreads();
+        // thread t filters entries [t*L, t*L + L) of the round (L a power of two), reading its float4
+        // groups in an order rotated by the lane so a warp's reads spread over all banks; bit
+        // 4*g + e of m64 flags entry 4*g + e of the thread's range
+        const int64_t tb = (int64_t)threadIdx.x * L;
+        const int64_t valid = n - tb < 0 ? 0 : (n - tb > L ? L : n - tb);
+        uint64_t m64 = 0;
+        if (!failed && valid > 0) {
+            const float4* s4 = reinterpret_cast<const float4*>(sbuf + tb);
+#pragma unroll 4
+            for (int g = 0; g < G; ++g) {
+                const int gg = (g + lane) & (G - 1);
+                const float4 v = s4[gg];
+                // a float compare against the bin's lower edge passes every kept entry (the key is
+                // monotone in the float order); passes are confirmed on the exact key below, which
+                // also drops -0.0 below a +0.0 edge
+                const uint32_t m = (v.x >= thr ? 1u : 0u) | (v.y >= thr ? 2u : 0u) | (v.z >= thr ? 4u : 0u) |
+                                   (v.w >= thr ? 8u : 0u);
+                m64 |= (uint64_t)m << (4 * gg);
+            }
+            if (valid < 64) m64 &= (1ull << valid) - 1ull;
+            for (uint64_t c = m64; c; c &= c - 1ull) {
+                const int bit = __ffsll((long long)c) - 1;
+                if ((float_key(sbuf[tb + bit]) >> 21) < b1) m64 &= ~(1ull << bit);
+            }
+        }
+        uint32_t tot;
+        uint32_t pos = block_excl_scan((uint32_t)__popcll(m64), s_wsum, &tot);
+        if (!spilled && n_mine + tot > (uint32_t)kStageSmem) {
+            for (uint32_t i = threadIdx.x; i < n_mine; i += blockDim.x) gseg[i] = stage[i];
+            spilled = true;
+            __syncthreads();
+        }
+        pos += n_mine;
+        for (; m64; m64 &= m64 - 1ull) {
+            const int bit = __ffsll((long long)m64) - 1;
+            const uint64_t key = composite(float_key(sbuf[tb + bit]), rb + tb + bit);
+            if (spilled) gseg[pos] = key;
+            else stage[pos] = key;
+            ++pos;
+        }
+        n_mine += tot;
+        __syncthreads();  // sbuf is free again
+        if (threadIdx.x == 0 && rb + p.sel_buf < c1) issue_round(rb + p.sel_buf);
     }
-    const uint32_t n_tot = offs[F];
-    if (n_tot != above + n_bin) {  // histogram and filter disagree: cannot happen
+    if (failed) n_mine = 0;
+
+    // 3. run lengths to the leader, then every CTA learns its offset
+    if (threadIdx.x == 0) st_cluster_u32(map_rank(&xcnt[rank], 0), n_mine | (spilled ? 0x80000000u : 0u));
+    cluster_sync();
+    if (threadIdx.x < F) suf[threadIdx.x] = ld_cluster_u32(map_rank(&xcnt[threadIdx.x], 0));
+    __syncthreads();
+    uint32_t off_me = 0, total = 0;
+    bool any_spill = false;
+    for (int c = 0; c < F; ++c) {
+        const uint32_t v = suf[c];
+        if ((uint32_t)c < rank) off_me += v & 0x7FFFFFFFu;
+        if (threadIdx.x == 0) offs[c] = total;
+        total += v & 0x7FFFFFFFu;
+        any_spill |= (v >> 31) != 0u;
+    }
+    if (threadIdx.x == 0) offs[F] = total;
+    // every CTA has read the histogram: clear it for the next call, one share per CTA
+    {
+        uint32_t* ghw = p.hist + (int64_t)qi * kHistBins;
+        const int share = kHistBins / F;
+        for (int i = threadIdx.x; i < share; i += blockDim.x) ghw[rank * share + i] = 0u;
+    }
+    const bool in_smem = !any_spill && total <= (uint32_t)kListSmem;
+    if (in_smem) {
+        // the leader's score buffer is free (its filter is done, no copy in flight): it becomes the list
+        const uint32_t dst = map_rank(lst + off_me, 0);
+        for (uint32_t i = threadIdx.x; i < n_mine; i += blockDim.x) st_cluster_u64(dst + i * 8u, stage[i]);
+    } else if (!spilled) {
+        for (uint32_t i = threadIdx.x; i < n_mine; i += blockDim.x) gseg[i] = stage[i];
+    }
+    cluster_sync();
+    if (rank != 0) return;
+
+    // 4. the leader: exact threshold, then compaction in index order
+    const uint32_t n_tot = total;
+    if (b1 == 0xFFFFFFFFu || n_tot != above + n_bin) {  // histogram and filter disagree: cannot happen
         if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
         return;
     }
-    KeptList kl{p.seg + (int64_t)qi * p.e_seg, offs, F, nullptr};
-    if (n_tot <= (uint32_t)kListSmem) {
-        for (uint32_t i = threadIdx.x; i < n_tot; i += blockDim.x) lst[i] = kl.get(i);
-        __syncthreads();
-        kl.cache = lst;
-    }
+    const KeptList kl{p.seg + (int64_t)qi * p.e_seg, offs, F, p.sel_span, in_smem ? lst : nullptr};
     const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53) : radix_threshold(kl, n_tot, need, b1, hist, suf, misc);
-    // 4. compaction in index order: keep every entry >= T (exactly k of them)
-    const uint32_t per = (n_tot + blockDim.x - 1) / blockDim.x;
-    const uint32_t i0 = threadIdx.x * per, i1 = min(n_tot, i0 + per);
+    const uint32_t per_t = (n_tot + blockDim.x - 1) / blockDim.x;
+    const uint32_t i0 = threadIdx.x * per_t, i1 = min(n_tot, i0 + per_t);
     uint32_t mine = 0;
     for (uint32_t i = i0; i < i1; ++i) mine += kl.get(i) >= T ? 1u : 0u;
     uint32_t kept_total;
@@ -454,51 +568,37 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
         }
     }
     if (threadIdx.x == 0 && kept_total != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
-    // leave the per-query histogram and ticket clean for the next call
-    uint32_t* ghw = p.hist + (int64_t)qi * kHistBins;
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ghw[i] = 0u;
-    if (threadIdx.x < 4) ctr[threadIdx.x] = 0u;
 }
 
 constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 }  // namespace
 
-int64_t seg_stride(int64_t e_stride) { return ((e_stride + kSelPerCta - 1) / kSelPerCta) * kSelPerCta; }
-
 size_t index_ws_bytes(int Q, int64_t e_stride) {
-    const int64_t es = seg_stride(e_stride);
     size_t s = 0;
     s += align256((size_t)Q * kHistBins * 4);
-    s += align256((size_t)Q * 4 * 4);
-    s += align256((size_t)Q * (es / kSelPerCta) * 4);
     s += align256((size_t)Q * e_stride * 4);
-    s += align256((size_t)Q * es * 8);
+    s += align256((size_t)Q * (e_stride + 8 * kSelClusterMax) * 8);
     return s;
 }
 
-size_t index_zero_bytes(int Q) { return align256((size_t)Q * kHistBins * 4) + align256((size_t)Q * 4 * 4); }
+size_t index_zero_bytes(int Q) { return align256((size_t)Q * kHistBins * 4); }
 
 void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
-    const int64_t es = seg_stride(e_stride);
     char* b = static_cast<char*>(ws);
     p.hist = reinterpret_cast<uint32_t*>(b);
     b += align256((size_t)Q * kHistBins * 4);
-    p.counters = reinterpret_cast<uint32_t*>(b);
-    b += align256((size_t)Q * 4 * 4);
-    p.seg_count = reinterpret_cast<uint32_t*>(b);
-    b += align256((size_t)Q * (es / kSelPerCta) * 4);
     p.scores = reinterpret_cast<float*>(b);
     b += align256((size_t)Q * e_stride * 4);
     p.seg = reinterpret_cast<uint64_t*>(b);
     p.e_stride = e_stride;
-    p.e_seg = es;
+    p.e_seg = e_stride + 8 * kSelClusterMax;
 }
 
 cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
                               cudaEvent_t mid, bool pdl) {
     if (zero_ws) {
-        // histogram + counters are contiguous at the start of the workspace
+        // the histogram sits at the start of the workspace
         cudaError_t e = cudaMemsetAsync(p.hist, 0, index_zero_bytes(p.Q), stream);
         if (e != cudaSuccess) return e;
     }
@@ -522,20 +622,31 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
         cudaError_t e = cudaEventRecordWithFlags(mid, stream, cudaEventRecordExternal);
         if (e != cudaSuccess) return e;
     }
-    int64_t f = (max_entries + kSelPerCta - 1) / kSelPerCta;
-    if (f < 1) f = 1;
-    p.filter_ctas = (int)f;
-    if (f > (int64_t)kSelectThreads * 8 - 1) return cudaErrorInvalidValue;  // > 16M entries per query
-    const size_t smem = (size_t)kHistBins * 8 + 64 * 4 + (size_t)kListSmem * 8 + ((size_t)f + 1) * 4;
+    // cluster size: about two select CTAs per SM over all queries, 1..kSelClusterMax CTAs per query
+    int F = 1;
+    while (F < kSelClusterMax && (int64_t)p.Q * F * 2 <= 2 * 148) F *= 2;
+    p.sel_cluster = F;
+    p.sel_span = (((p.e_stride + F - 1) / F + 7) / 8) * 8;  // F * span <= e_stride + 8F <= e_seg
+    // scores per thread per round: the smallest power of two that covers the CTA's span in one
+    // round, 4..kSelPerMax; the round buffer holds that many per thread
+    int per = 4;
+    while (per < kSelPerMax && (int64_t)per * kSelectThreads < p.sel_span) per *= 2;
+    p.sel_per = per;
+    p.sel_buf = per * kSelectThreads;
+    const int64_t buf = p.sel_buf;
+    const size_t smem = SelSmem::bytes(buf);
     static bool attr_set = false;
     if (!attr_set) {
-        const int max_smem = kHistBins * 8 + 64 * 4 + kListSmem * 8 + kSelectThreads * 8 * 4;
-        cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+        cudaError_t e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SelSmem::bytes(kSelBufMax));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
         attr_set = true;
     }
     // after an event record the select follows the scan without overlap
-    return launch_kernel(index_select_kernel, dim3((unsigned)f, (unsigned)p.Q), dim3(kSelectThreads), smem, stream,
-                         pdl && mid == nullptr, p);
+    return launch_kernel_cluster(index_select_kernel, dim3((unsigned)F, (unsigned)p.Q), dim3(kSelectThreads), smem,
+                                 stream, pdl && mid == nullptr, dim3((unsigned)F, 1, 1), p);
 }
 
 }  // namespace csa

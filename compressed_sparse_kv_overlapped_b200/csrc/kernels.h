@@ -28,7 +28,7 @@ cudaError_t launch_compress(const CompressParams& p, int64_t max_entries, cudaSt
 // Indexer score scan + top-k select.
 constexpr int kHistBins = 2048;  // coarse histogram over the top 11 bits of the score key
 constexpr int kMaxK = 2048;
-constexpr int kSelPerCta = 4096;  // scores per select (filter) CTA
+constexpr int kSelClusterMax = 16;  // most CTAs (one thread-block cluster) per query in the select kernel
 
 struct IndexParams {
     const csa_seq* seqs;
@@ -40,14 +40,15 @@ struct IndexParams {
     int64_t chunk;            // entries per scan CTA
     int64_t max_entries;      // host bound of floor(L/m) over all queries (grid sizing)
     int64_t e_stride;         // row stride of the score buffer
-    int64_t e_seg;            // row stride of the segment buffer (e_stride rounded up to kSelPerCta)
-    int filter_ctas;          // CTAs per query in the select kernel
+    int64_t sel_span;         // entries per select CTA (multiple of 8)
+    int64_t e_seg;            // row stride of the segment buffer (e_stride + 8 * kSelClusterMax)
+    int sel_cluster;          // select CTAs per query (a power of two, at most kSelClusterMax)
+    int sel_per;              // scores per select thread per round (a power of two)
+    int sel_buf;              // scores a select CTA stages in shared memory per round
     // workspace
     float* scores;            // [Q, e_stride]
-    uint32_t* hist;           // [Q, kHistBins]
-    uint32_t* counters;       // [Q, 4]: [0] done-ticket
-    uint32_t* seg_count;      // [Q, e_seg / kSelPerCta] entries each filter CTA kept
-    uint64_t* seg;            // [Q, e_seg] kept entries (64-bit keys), one kSelPerCta segment per filter CTA
+    uint32_t* hist;           // [Q, kHistBins]; zero between calls (the select kernel clears it)
+    uint64_t* seg;            // [Q, e_seg] kept entries (64-bit keys) when they exceed shared memory
     // outputs
     int32_t* idx_out;         // [Q, k]
     float* score_out;         // [Q, k] nullable
@@ -88,6 +89,10 @@ struct AttnParams {
     // table, HCA entries) were written two or more launches earlier, which are complete by the time
     // this grid may start.  Only the decode chain sets it.
     int hca_nowait;
+    // 1: one-dimensional grid over all (query, item) pairs with every query's HCA items first, so
+    // they take the free SMs before the front items (which wait for the top-k) do.  Launches all
+    // items of all queries.
+    int hca_first;
     // outputs
     float* out;                 // [Q, H, d]
     float* lse;                 // [Q, H] nullable

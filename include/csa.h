@@ -240,7 +240,7 @@ int csa_set_stage_events(void* const* events, int count);
  * the scratch lives).  For callers that cannot provide device memory at call time -- code under a
  * framework whose allocator owns all device buffers, loops that must not allocate once running, or
  * bindings that only see input and output pointers.  The scratch is a fixed array inside the
- * library, about 12.9 MiB on every device that loads it, held until the process exits.
+ * library, about 12.1 MiB on every device that loads it, held until the process exits.
  * Limits: Q <= 16 and Q * ceil4(floor(max_len / m)) <= 1,048,576; larger calls return
  * CSA_ERR_UNSUPPORTED with a message and enqueue nothing.  It never allocates or frees memory.
  * The first call on a device looks up the array's device address (once per device, with that
