@@ -695,13 +695,13 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
     }
     char* w = static_cast<char*>(ws);
     csa_query* queries = reinterpret_cast<csa_query*>(w + pl.off_queries);
-    const int64_t max_e = a->q_end / d.m;
     for (int64_t p0 = a->q_begin; p0 < a->q_end; p0 += pl.qc) {
         const int64_t n = a->q_end - p0 < pl.qc ? a->q_end - p0 : pl.qc;
         const int64_t r0 = p0 - a->q_begin;
         if ((e = launch_prefill_queries(queries, p0, n, stream)) != cudaSuccess) return cuda_fail(e, "query table");
         int32_t* idx = a->idx_out ? a->idx_out + r0 * d.k : reinterpret_cast<int32_t*>(w + pl.off_idx);
-        rc = run_index(d, a->seq, queries, (int)n, max_e, pl.e_stride, a->q_idx + r0 * d.H_I * d.d_I,
+        // the chunk's queries see at most p0 + n tokens: size the scan for that, not for q_end
+        rc = run_index(d, a->seq, queries, (int)n, (p0 + n) / d.m, pl.e_stride, a->q_idx + r0 * d.H_I * d.d_I,
                        a->w + r0 * d.H_I, a->entry_keys, idx, nullptr, w + pl.off_index, true, st, stream);
         if (rc) return rc;
         AttnParams pp;
