@@ -586,28 +586,6 @@ def run_prefill(args, rank, world):
         raise RuntimeError("device status in the timed region")
     ms_comp = ev[0].elapsed_time(ev[1]) / K
     ms = ev[2].elapsed_time(ev[3]) / K
-    # the indexer + top-k alone, in the same query chunks as hybrid_attn_prefill (outside the timed
-    # steps): the attention is the difference
-    qc = int(os.environ.get("CSA_PREFILL_CHUNK", 2048))
-    pos = torch.arange(N, dtype=torch.int64, device=dev)
-    qtab = torch.stack([torch.zeros_like(pos), pos + 1], dim=1).contiguous()
-    idx = torch.empty(qc, wd.k, dtype=torch.int32, device=dev)
-    wq = csa.csa_ws_query()
-    wq.dims, wq.Q, wq.max_len = dims_of(wd), qc, N
-    ws_i = torch.empty(csa.csa_workspace_size(csa.CSA_OP_INDEX_TOPK, wq), dtype=torch.uint8, device=dev)
-
-    def index_all():
-        for p0 in range(0, N, qc):
-            n = min(qc, N - p0)
-            csa.csa_index_topk(dims_of(wd), layer.seqs, qtab[p0:p0 + n], n, p0 + n, qi[p0:p0 + n], w[p0:p0 + n],
-                               layer.entry_keys, idx[:n], None, ws_i)
-    index_all()
-    torch.cuda.synchronize()
-    ev[0].record()
-    index_all()
-    ev[1].record()
-    torch.cuda.synchronize()
-    ms_index = ev[0].elapsed_time(ev[1])
     if world > 1:
         t = torch.tensor([ms, ms_comp], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -628,8 +606,6 @@ def run_prefill(args, rank, world):
         "roofline": {"kernel": "whole prefill (index + select + attention)", "bound": "tensor", "achieved": tflops,
                      "peak": tf_peak, "unit": "TFLOP/s", "frac": tflops / tf_peak, "traffic": None,
                      "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops_sustained)"},
-        "stages_ms": {"index_topk": ms_index, "attention": ms - ms_index,
-                      "note": "index_topk timed alone in the same chunks; attention = step - index_topk"},
         "compress": {"ms": ms_comp, "bytes": comp_bytes, "achieved_gbs": comp_bytes / (ms_comp * 1e-3) / 1e9,
                      "peak_gbs": hbm, "note": "csa_compress for the CSA and HCA caches over all N tokens"},
         "clocks": clocks.summary(t0, t1),

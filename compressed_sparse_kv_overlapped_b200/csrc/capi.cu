@@ -695,15 +695,62 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
     }
     char* w = static_cast<char*>(ws);
     csa_query* queries = reinterpret_cast<csa_query*>(w + pl.off_queries);
+    // the indexer runs as a tensor-core GEMM when its shape allows (d_I = 64, H_I <= 4, rows that fit
+    // the select's shared memory); CSA_PREFILL_SCAN=1 forces the per-query scan
+    const bool gemm_index = d.d_I == 64 && d.H_I <= 4 && a->q_end / d.m <= kSelRowMax &&
+                            env_int("CSA_PREFILL_SCAN", 0) == 0;
     for (int64_t p0 = a->q_begin; p0 < a->q_end; p0 += pl.qc) {
         const int64_t n = a->q_end - p0 < pl.qc ? a->q_end - p0 : pl.qc;
         const int64_t r0 = p0 - a->q_begin;
         if ((e = launch_prefill_queries(queries, p0, n, stream)) != cudaSuccess) return cuda_fail(e, "query table");
         int32_t* idx = a->idx_out ? a->idx_out + r0 * d.k : reinterpret_cast<int32_t*>(w + pl.off_idx);
-        // the chunk's queries see at most p0 + n tokens: size the scan for that, not for q_end
-        rc = run_index(d, a->seq, queries, (int)n, (p0 + n) / d.m, pl.e_stride, a->q_idx + r0 * d.H_I * d.d_I,
-                       a->w + r0 * d.H_I, a->entry_keys, idx, nullptr, w + pl.off_index, true, st, stream);
-        if (rc) return rc;
+        // the chunk's queries see at most p0 + n tokens: size the indexer for that, not for q_end
+        const int64_t max_e_chunk = (p0 + n) / d.m;
+        if (gemm_index) {
+            // scores of the whole chunk as one tensor-core GEMM, then a sampled-threshold select
+            IndexParams ip{};
+            ip.seqs = a->seq;
+            ip.queries = queries;
+            ip.Q = (int)n;
+            ip.H_I = d.H_I;
+            ip.d_I = d.d_I;
+            ip.m = d.m;
+            ip.k = d.k;
+            ip.q_idx = a->q_idx + r0 * d.H_I * d.d_I;
+            ip.w = a->w + r0 * d.H_I;
+            ip.entry_keys = a->entry_keys;
+            ip.max_entries = max_e_chunk;
+            ip.idx_out = idx;
+            ip.score_out = nullptr;
+            ip.status = st;
+            index_ws_carve(ip, w + pl.off_index, (int)n, pl.e_stride);
+            if (max_e_chunk > d.k) {
+                PrefillScoreParams sp{};
+                sp.seq = a->seq;
+                sp.q_idx = ip.q_idx;
+                sp.w = ip.w;
+                sp.entry_keys = a->entry_keys;
+                sp.H_I = d.H_I;
+                sp.m_shift = d.m == 1 ? 0 : d.m == 2 ? 1 : d.m == 4 ? 2 : 3;  // m is 1, 2, 4 or 8
+                sp.Qn = (int)n;
+                sp.pos0 = p0;
+                const int64_t gy = (n + 127) / 128;
+                int64_t ent = (max_e_chunk * gy + 2 * 148 - 1) / (2 * 148);
+                ent = ((ent + 63) / 64) * 64;
+                sp.ent_per_cta = ent < 64 ? 64 : ent;
+                sp.scores = ip.scores;
+                sp.e_stride = ip.e_stride;
+                sp.status = st;
+                if ((e = launch_prefill_scores(sp, max_e_chunk, stream)) != cudaSuccess)
+                    return cuda_fail(e, "prefill score launch");
+            }
+            if ((e = launch_index_topk(ip, max_e_chunk, stream, false, nullptr, false, true)) != cudaSuccess)
+                return cuda_fail(e, "select launch");
+        } else {
+            rc = run_index(d, a->seq, queries, (int)n, max_e_chunk, pl.e_stride, a->q_idx + r0 * d.H_I * d.d_I,
+                           a->w + r0 * d.H_I, a->entry_keys, idx, nullptr, w + pl.off_index, true, st, stream);
+            if (rc) return rc;
+        }
         AttnParams pp;
         ItemPlan one{1, 0, 64, 64};
         rc = make_attn(pp, &d, a->seq, queries, (int)n, a->q + r0 * d.H * d.d, a->entries, idx, d.k, a->x, d.W,

@@ -439,35 +439,17 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     };
     if (threadIdx.x == 0 && c0 < c1) issue_round(c0);
 
-    // 1. threshold bin (every CTA of the query finds the same one)
-    const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = __ldcg(gh + i);
-    __syncthreads();
-    suffix_find(hist, suf, misc, (uint32_t)p.k, misc + 32);
-    const uint32_t b1 = misc[32];
-    const uint32_t above = misc[33];
-    const uint32_t need = (uint32_t)p.k - above;
-    const uint32_t n_bin = b1 == 0xFFFFFFFFu ? 0u : hist[b1];  // members of the threshold bin
-    const float thr = key_float(b1 << 21);                     // the smallest float of bin b1
-    bool failed = b1 == 0xFFFFFFFFu;  // histogram holds fewer than k scores: cannot happen
-
-    // 2. keep this CTA's entries of bin >= b1, in index order
     uint64_t* gseg = p.seg + (int64_t)qi * p.e_seg + (int64_t)rank * p.sel_span;
     uint32_t n_mine = 0;
     bool spilled = false;  // the run lives in gseg instead of `stage`
-    uint32_t phase = 0;
-    for (int64_t rb = c0; rb < c1; rb += p.sel_buf) {
-        const int64_t n = min((int64_t)p.sel_buf, c1 - rb);
-        const int64_t n16 = n & ~(int64_t)3;
-        if (threadIdx.x < n - n16) sbuf[n16 + threadIdx.x] = __ldg(srow + rb + n16 + threadIdx.x);
-        // a wait that runs out leaves this CTA's run empty (and the status word set); the CTA still
-        // takes both cluster barriers below
-        if (!mbar_wait(&s_bar, phase, p.status, &s_abort)) failed = true;
-        phase ^= 1u;
-        __syncthreads();
-        // thread t filters entries [t*L, t*L + L) of the round (L a power of two), reading its float4
-        // groups in an order rotated by the lane so a warp's reads spread over all banks; bit
-        // 4*g + e of m64 flags entry 4*g + e of the thread's range
+    bool failed = false;
+    // Keep the entries of [rb, rb + n) (staged in sbuf) whose bin is >= b_lo, appending them in
+    // index order to the run.  Thread t filters entries [t*L, t*L + L), reading its float4 groups in
+    // an order rotated by the lane so a warp's reads spread over all banks; bit 4*g + e of m64 flags
+    // entry 4*g + e of the thread's range.
+    auto filter_round = [&](int64_t rb, int64_t n, uint32_t b_lo) {
+        const float thr = key_float(b_lo << 21);  // the smallest float of bin b_lo (b_lo = 0: keep all)
+        const bool keep_all = b_lo == 0u;
         const int64_t tb = (int64_t)threadIdx.x * L;
         const int64_t valid = n - tb < 0 ? 0 : (n - tb > L ? L : n - tb);
         uint64_t m64 = 0;
@@ -480,14 +462,15 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
                 // a float compare against the bin's lower edge passes every kept entry (the key is
                 // monotone in the float order); passes are confirmed on the exact key below, which
                 // also drops -0.0 below a +0.0 edge
-                const uint32_t m = (v.x >= thr ? 1u : 0u) | (v.y >= thr ? 2u : 0u) | (v.z >= thr ? 4u : 0u) |
-                                   (v.w >= thr ? 8u : 0u);
+                const uint32_t m = keep_all ? 0xFu
+                                            : (v.x >= thr ? 1u : 0u) | (v.y >= thr ? 2u : 0u) |
+                                                  (v.z >= thr ? 4u : 0u) | (v.w >= thr ? 8u : 0u);
                 m64 |= (uint64_t)m << (4 * gg);
             }
             if (valid < 64) m64 &= (1ull << valid) - 1ull;
             for (uint64_t c = m64; c; c &= c - 1ull) {
                 const int bit = __ffsll((long long)c) - 1;
-                if ((float_key(sbuf[tb + bit]) >> 21) < b1) m64 &= ~(1ull << bit);
+                if ((float_key(sbuf[tb + bit]) >> 21) < b_lo) m64 &= ~(1ull << bit);
             }
         }
         uint32_t tot;
@@ -506,8 +489,74 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
             ++pos;
         }
         n_mine += tot;
-        __syncthreads();  // sbuf is free again
-        if (threadIdx.x == 0 && rb + p.sel_buf < c1) issue_round(rb + p.sel_buf);
+        __syncthreads();
+    };
+
+    uint32_t b1, above, need, n_bin;
+    if (!p.sampled) {
+        // 1. threshold bin from the scan's histogram (every CTA of the query finds the same one)
+        const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
+        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = __ldcg(gh + i);
+        __syncthreads();
+        suffix_find(hist, suf, misc, (uint32_t)p.k, misc + 32);
+        b1 = misc[32];
+        above = misc[33];
+        need = (uint32_t)p.k - above;
+        n_bin = b1 == 0xFFFFFFFFu ? 0u : hist[b1];  // members of the threshold bin
+        failed = b1 == 0xFFFFFFFFu;                 // histogram holds fewer than k scores: cannot happen
+
+        // 2. keep this CTA's entries of bin >= b1, in index order, round by round
+        uint32_t phase = 0;
+        for (int64_t rb = c0; rb < c1; rb += p.sel_buf) {
+            const int64_t n = min((int64_t)p.sel_buf, c1 - rb);
+            const int64_t n16 = n & ~(int64_t)3;
+            if (threadIdx.x < n - n16) sbuf[n16 + threadIdx.x] = __ldg(srow + rb + n16 + threadIdx.x);
+            // a wait that runs out leaves this CTA's run empty (and the status word set); the CTA
+            // still takes both cluster barriers below
+            if (!mbar_wait(&s_bar, phase, p.status, &s_abort)) failed = true;
+            phase ^= 1u;
+            __syncthreads();
+            filter_round(rb, n, b1);  // ends with a barrier: sbuf is free again
+            if (threadIdx.x == 0 && rb + p.sel_buf < c1) issue_round(rb + p.sel_buf);
+        }
+    } else {
+        // No histogram (prefill GEMM scores; one CTA holds the query's whole row in one round).
+        // 1'. estimate a bin from a sample: the bin below which about 2k / n of the sample lies is
+        //     low enough that at least k entries pass it with overwhelming probability
+        const int64_t n = c1 - c0;
+        const int64_t n16 = n & ~(int64_t)3;
+        if (threadIdx.x < n - n16) sbuf[n16 + threadIdx.x] = __ldg(srow + c0 + n16 + threadIdx.x);
+        if (n > 0 && !mbar_wait(&s_bar, 0, p.status, &s_abort)) failed = true;
+        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0u;
+        __syncthreads();
+        const int64_t S = n < 4096 ? n : 4096;
+        for (int64_t i = threadIdx.x; i < S; i += blockDim.x)
+            atomicAdd(&hist[float_key(sbuf[(i * n) / S]) >> 21], 1u);
+        __syncthreads();
+        const int64_t want = (2 * (int64_t)p.k * S + n - 1) / (n > 0 ? n : 1);
+        suffix_find(hist, suf, misc, (uint32_t)(want < S ? want : S + 1), misc + 32);
+        uint32_t b_est = misc[32] == 0xFFFFFFFFu ? 0u : misc[32];  // no bin qualifies: keep everything
+        // 2'. candidates: every entry of bin >= b_est, in index order
+        filter_round(c0, n, b_est);
+        if (n_mine < (uint32_t)p.k && b_est > 0) {  // the estimate was too high (rare): keep everything
+            n_mine = 0;
+            spilled = false;
+            filter_round(c0, n, 0u);
+        }
+        // 3'. the exact threshold bin from the candidates' own histogram
+        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0u;
+        __syncthreads();
+        for (uint32_t i = threadIdx.x; i < n_mine; i += blockDim.x) {
+            const uint64_t key = spilled ? __ldcg(reinterpret_cast<const unsigned long long*>(gseg) + i) : stage[i];
+            atomicAdd(&hist[(uint32_t)(key >> 53)], 1u);
+        }
+        __syncthreads();
+        suffix_find(hist, suf, misc, (uint32_t)p.k, misc + 32);
+        b1 = misc[32];
+        above = misc[33];
+        need = (uint32_t)p.k - above;
+        n_bin = b1 == 0xFFFFFFFFu ? 0u : hist[b1];
+        if (b1 == 0xFFFFFFFFu) failed = true;
     }
     if (failed) n_mine = 0;
 
@@ -545,7 +594,8 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
 
     // 4. the leader: exact threshold, then compaction in index order
     const uint32_t n_tot = total;
-    if (b1 == 0xFFFFFFFFu || n_tot != above + n_bin) {  // histogram and filter disagree: cannot happen
+    // without sampling the kept list is exactly the entries of bins >= b1; with it, a superset
+    if (b1 == 0xFFFFFFFFu || (p.sampled ? n_tot < above + n_bin : n_tot != above + n_bin)) {
         if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
         return;
     }
@@ -574,6 +624,19 @@ constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 }  // namespace
 
+cudaError_t select_attrs() {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SelSmem::bytes(kSelBufMax));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    return cudaSuccess;
+}
+
 size_t index_ws_bytes(int Q, int64_t e_stride) {
     size_t s = 0;
     s += align256((size_t)Q * kHistBins * 4);
@@ -596,7 +659,24 @@ void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
 }
 
 cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
-                              cudaEvent_t mid, bool pdl) {
+                              cudaEvent_t mid, bool pdl, bool sampled) {
+    p.sampled = sampled ? 1 : 0;
+    if (sampled) {
+        // scores are already in p.scores; one select CTA per query holds its whole row
+        if (max_entries > kSelBufMax) return cudaErrorInvalidValue;
+        p.sel_cluster = 1;
+        p.sel_span = ((max_entries + 7) / 8) * 8;
+        if (p.sel_span < 8) p.sel_span = 8;
+        int per = 4;
+        while (per < kSelPerMax && (int64_t)per * kSelectThreads < p.sel_span) per *= 2;
+        p.sel_per = per;
+        p.sel_buf = per * kSelectThreads;
+        const size_t smem = SelSmem::bytes(p.sel_buf);
+        cudaError_t e = select_attrs();
+        if (e != cudaSuccess) return e;
+        return launch_kernel_cluster(index_select_kernel, dim3(1, (unsigned)p.Q), dim3(kSelectThreads), smem, stream,
+                                     pdl, dim3(1, 1, 1), p);
+    }
     if (zero_ws) {
         // the histogram sits at the start of the workspace
         cudaError_t e = cudaMemsetAsync(p.hist, 0, index_zero_bytes(p.Q), stream);
@@ -635,15 +715,8 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
     p.sel_buf = per * kSelectThreads;
     const int64_t buf = p.sel_buf;
     const size_t smem = SelSmem::bytes(buf);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SelSmem::bytes(kSelBufMax));
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t ea = select_attrs();
+    if (ea != cudaSuccess) return ea;
     // after an event record the select follows the scan without overlap
     return launch_kernel_cluster(index_select_kernel, dim3((unsigned)F, (unsigned)p.Q), dim3(kSelectThreads), smem,
                                  stream, pdl && mid == nullptr, dim3((unsigned)F, 1, 1), p);

@@ -45,6 +45,8 @@ struct IndexParams {
     int sel_cluster;          // select CTAs per query (a power of two, at most kSelClusterMax)
     int sel_per;              // scores per select thread per round (a power of two)
     int sel_buf;              // scores a select CTA stages in shared memory per round
+    int sampled;              // 1: no scan histogram; one select CTA per query estimates its threshold
+                              // bin from a sample of its scores (requires a row to fit one round)
     // workspace
     float* scores;            // [Q, e_stride]
     uint32_t* hist;           // [Q, kHistBins]; zero between calls (the select kernel clears it)
@@ -57,9 +59,30 @@ struct IndexParams {
 size_t index_ws_bytes(int Q, int64_t e_stride);
 size_t index_zero_bytes(int Q);  // leading bytes of the index workspace that must start at zero
 void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride);
+// Prefill indexer scores as a tensor-core GEMM (d_I = 64, H_I <= 4): chunk rows [0, Qn) are the
+// consecutive positions pos0, pos0 + 1, ... of one sequence; row r's causal entries (j < (pos0 + r +
+// 1) / m) get scores[r * e_stride + j].
+struct PrefillScoreParams {
+    const csa_seq* seq;
+    const uint16_t* q_idx;   // [Qn, H_I, 64]
+    const float* w;          // [Qn, H_I]
+    const uint16_t* entry_keys;
+    int H_I, m_shift, Qn;     // m = 1 << m_shift
+    int64_t pos0;
+    int64_t ent_per_cta;     // multiple of 64
+    float* scores;
+    int64_t e_stride;
+    int* status;
+};
+cudaError_t launch_prefill_scores(const PrefillScoreParams& p, int64_t max_entries, cudaStream_t stream,
+                                  bool pdl = false);
+
 // `mid` (nullable): event recorded between the scan and the select kernels.
+// `sampled`: p.scores already holds the scores (prefill GEMM), no scan and no histogram; every row
+// must hold at most kSelRowMax entries.
+constexpr int64_t kSelRowMax = 32768;
 cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
-                              cudaEvent_t mid = nullptr, bool pdl = false);
+                              cudaEvent_t mid = nullptr, bool pdl = false, bool sampled = false);
 
 // Attention over a per-query key list = [selected CSA entries | raw window | HCA entries].
 struct AttnParams {
