@@ -514,9 +514,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
 }
 
 // out[q][h] = sum_items exp(lse_i - lse) * O_i,  lse = logsumexp_i lse_i  (items with lse = -inf
-// contribute nothing and are not read).  One CTA per (head, query); warp 0 computes the weights, then
-// every thread accumulates one float4 column of all contributing partials with batched loads.
-template <int D>
+// contribute nothing and are not read).  One CTA per (head, query, 1/SPLIT of the dims); warp 0
+// computes the weights, then every thread accumulates one float4 column of all contributing
+// partials with batched loads.
+template <int D, int SPLIT>
 __global__ void combine_kernel(AttnParams p) {
     constexpr int kMaxBatch = 24;  // partial rows held in registers per pass
     grid_dep_wait();  // the partials come from the attention grid
@@ -526,8 +527,8 @@ __global__ void combine_kernel(AttnParams p) {
     __shared__ float s_lse[256];
     __shared__ float s_w[256];
     __shared__ float s_res[2];
-    // every thread owns one float4 column of the output row (D/4 threads)
-    const int c = threadIdx.x * 4;
+    // every thread owns one float4 column of the output row (D / 4 / SPLIT threads)
+    const int c = (int)blockIdx.z * (D / SPLIT) + threadIdx.x * 4;
     const float* base = p.part_o + ((int64_t)qi * n_items * kHeadsPad + h) * D + c;
     const int64_t item_stride = (int64_t)kHeadsPad * D;
     for (int it = threadIdx.x; it < n_items; it += blockDim.x)
@@ -559,7 +560,7 @@ __global__ void combine_kernel(AttnParams p) {
     }
     __syncthreads();
     const float inv = s_res[0];
-    if (threadIdx.x == 0 && p.lse) p.lse[(int64_t)qi * p.H + h] = s_res[1];
+    if (threadIdx.x == 0 && blockIdx.z == 0 && p.lse) p.lse[(int64_t)qi * p.H + h] = s_res[1];
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int b = 0; b < n_items; b += kMaxBatch) {
         const int nb = n_items - b < kMaxBatch ? n_items - b : kMaxBatch;
@@ -624,9 +625,11 @@ cudaError_t launch_attention_items(const AttnParams& p, int item_begin, int item
 
 cudaError_t launch_combine(const AttnParams& p, cudaStream_t stream, bool pdl) {
     if (p.n_items <= 1) return cudaSuccess;
-    const dim3 grid((unsigned)p.H, (unsigned)p.Q);
-    if (p.d == 512) return launch_kernel(combine_kernel<512>, grid, dim3(128), 0, stream, pdl, p);
-    if (p.d == 128) return launch_kernel(combine_kernel<128>, grid, dim3(32), 0, stream, pdl, p);
+    // 512 dims: two CTAs of 64 threads per (head, query), so the merge spreads over more SMs
+    if (p.d == 512)
+        return launch_kernel(combine_kernel<512, 2>, dim3((unsigned)p.H, (unsigned)p.Q, 2), dim3(64), 0, stream, pdl, p);
+    if (p.d == 128)
+        return launch_kernel(combine_kernel<128, 1>, dim3((unsigned)p.H, (unsigned)p.Q, 1), dim3(32), 0, stream, pdl, p);
     return cudaErrorInvalidValue;
 }
 
