@@ -49,7 +49,8 @@ class csa_decode_args(ctypes.Structure):
     _fields_ = [("dims", csa_dims), ("B", _i32), ("append", _i32), ("max_len", _i64), ("scale", _f32),
                 ("seqs", _vp), ("x", _vp), ("logit_c", _vp), ("logit_h", _vp), ("idx_key", _vp),
                 ("bias_c", _vp), ("bias_h", _vp), ("entries", _vp), ("entry_keys", _vp), ("hca_entries", _vp),
-                ("q", _vp), ("q_idx", _vp), ("w", _vp), ("out", _vp), ("lse", _vp), ("idx_out", _vp)]
+                ("q", _vp), ("q_idx", _vp), ("w", _vp), ("out", _vp), ("lse", _vp), ("idx_out", _vp),
+                ("new_rows", _vp)]
 
 
 class csa_prefill_args(ctypes.Structure):

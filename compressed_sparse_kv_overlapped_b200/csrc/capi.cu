@@ -67,9 +67,24 @@ int check_dims(const csa_dims* d) {
     return CSA_OK;
 }
 
+// Tuning switches from the environment, read once per process (getenv scans the whole
+// environment, and the decode call sits on a per-step path).
 int env_int(const char* name, int dflt) {
+    static std::mutex mu;
+    static const char* names[16];
+    static int values[16];
+    static int n = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (names[i] == name) return values[i];
     const char* v = getenv(name);
-    return v ? atoi(v) : dflt;
+    const int r = v ? atoi(v) : dflt;
+    if (n < 16) {
+        names[n] = name;
+        values[n] = r;
+        ++n;
+    }
+    return r;
 }
 
 int round64(int64_t v) { return (int)(((v + 63) / 64) * 64); }
@@ -160,6 +175,20 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     }
     const csa_seq sq = p.seqs[b];
     if (p.append) {
+        if (p.new_rows) {
+            // the appended token's rows (x | a | b | k^I) go into the caches at row tok_off + len - 1
+            const int64_t r = sq.tok_off + len - 1;
+            const int wd = p.d >> 3, wi = p.d_I >> 3;  // 16-byte chunks per row
+            const uint4* src = reinterpret_cast<const uint4*>(p.new_rows + (int64_t)b * (3 * p.d + p.d_I));
+            for (int i = threadIdx.x; i < 3 * wd + wi; i += blockDim.x) {
+                const uint4 v = src[i];
+                if (i < wd) reinterpret_cast<uint4*>(p.x + r * p.d)[i] = v;
+                else if (i < 2 * wd) reinterpret_cast<uint4*>(p.logit_c + r * p.d)[i - wd] = v;
+                else if (i < 3 * wd) reinterpret_cast<uint4*>(p.logit_h + r * p.d)[i - 2 * wd] = v;
+                else reinterpret_cast<uint4*>(p.idx_key + r * p.d_I)[i - 3 * wd] = v;
+            }
+            __syncthreads();  // the compressor below reads these rows
+        }
         const int tpe = p.d >> 3;
         if (len % p.m == 0 && threadIdx.x < tpe) {
             const int64_t j = len / p.m - 1;
@@ -551,8 +580,10 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
         return fail(CSA_ERR_ARG, "NULL pointer argument");
     if (!aligned16(a->x) || !aligned16(a->logit_c) || !aligned16(a->logit_h) || !aligned16(a->idx_key) ||
         !aligned16(a->bias_c) || !aligned16(a->bias_h) || !aligned16(a->entries) || !aligned16(a->entry_keys) ||
-        !aligned16(a->hca_entries) || !aligned16(a->q) || !aligned16(a->q_idx) || !aligned16(a->out))
+        !aligned16(a->hca_entries) || !aligned16(a->q) || !aligned16(a->q_idx) || !aligned16(a->out) ||
+        !aligned16(a->new_rows))
         return fail(CSA_ERR_ARG, "tensors must be 16-byte aligned");
+    if (a->new_rows && !a->append) return fail(CSA_ERR_ARG, "new_rows without append");
     const DecodePlan pl = plan_decode(d, a->B, a->max_len);
     if (!ws || ws_bytes < pl.total || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", pl.total);
@@ -575,6 +606,7 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     ap.logit_c = a->logit_c;
     ap.logit_h = a->logit_h;
     ap.idx_key = a->idx_key;
+    ap.new_rows = a->new_rows;
     ap.bias_c = a->bias_c;
     ap.bias_h = a->bias_h;
     ap.entries = a->entries;

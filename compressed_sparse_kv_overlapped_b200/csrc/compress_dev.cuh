@@ -42,9 +42,11 @@ __device__ __forceinline__ void compress_entry8(int64_t j, int m, int win, int d
             const int64_t t = tb + u;
             if (t < t1) {
                 const int64_t row = tok0 + t;
-                lv[u] = __ldg(reinterpret_cast<const uint4*>(logit + row * d + c0));
-                xv[u] = __ldg(reinterpret_cast<const uint4*>(x + row * d + c0));
-                if (want_key) kv[u] = __ldg(reinterpret_cast<const uint4*>(idx_key + row * d_I + c0));
+                // coherent (L2) loads: at decode the newest token's rows may have been written by
+                // this same kernel just before (csa_decode_args.new_rows)
+                lv[u] = __ldcg(reinterpret_cast<const uint4*>(logit + row * d + c0));
+                xv[u] = __ldcg(reinterpret_cast<const uint4*>(x + row * d + c0));
+                if (want_key) kv[u] = __ldcg(reinterpret_cast<const uint4*>(idx_key + row * d_I + c0));
             }
         }
 #pragma unroll

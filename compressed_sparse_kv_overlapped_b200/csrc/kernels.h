@@ -137,10 +137,11 @@ struct AppendParams {
     csa_seq* seqs;
     int B, append;
     int d, d_I, m, m_hca;
-    const uint16_t* x;
-    const uint16_t* logit_c;
-    const uint16_t* logit_h;
-    const uint16_t* idx_key;
+    uint16_t* x;
+    uint16_t* logit_c;
+    uint16_t* logit_h;
+    uint16_t* idx_key;
+    const uint16_t* new_rows;  // [B, 3d + d_I] appended token rows to copy into the caches (nullable)
     const float* bias_c;
     const float* bias_h;
     uint16_t* entries;

@@ -75,7 +75,10 @@ class HybridLayer:
 
     # ---- decode -------------------------------------------------------------------------------
     def decode_args(self, q, q_idx, w, out, append=True, lse=None, idx_out=None, max_len=None,
-                    scale=None) -> csa_decode_args:
+                    scale=None, new_rows=None) -> csa_decode_args:
+        """Arguments of one decode step.  With append, the new token's raw rows either are already in
+        the caches at row tok_off + len (new_rows None) or come as new_rows [B, 3d + d_I] bf16
+        (x | logit_c | logit_h | idx_key per sequence) and the call writes them there."""
         d = self.dims
         a = csa_decode_args()
         a.dims = d
@@ -87,7 +90,7 @@ class HybridLayer:
                         ("idx_key", self.idx_key), ("bias_c", self.bias_c), ("bias_h", self.bias_h),
                         ("entries", self.entries), ("entry_keys", self.entry_keys),
                         ("hca_entries", self.hca_entries), ("q", q), ("q_idx", q_idx), ("w", w), ("out", out),
-                        ("lse", lse), ("idx_out", idx_out)):
+                        ("lse", lse), ("idx_out", idx_out), ("new_rows", new_rows)):
             setattr(a, name, None if t is None else t.data_ptr())
         return a
 

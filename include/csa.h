@@ -140,16 +140,17 @@ int hca_dense_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* q
 typedef struct csa_decode_args {
     csa_dims dims;
     int32_t B;
-    int32_t append;      /* 1: every sequence first takes one new token (its rows at tok_off + len
-                            must already be written in x/logit_c/logit_h/idx_key); len += 1 and
-                            the entries that this token completes are compressed */
+    int32_t append;      /* 1: every sequence first takes one new token; len += 1 and the entries
+                            that this token completes are compressed.  The token's rows at
+                            tok_off + len are either already written in x/logit_c/logit_h/idx_key by
+                            the caller (new_rows = NULL) or copied there from new_rows */
     int64_t max_len;     /* host bound of every sequence's len after the append (sizes grids) */
     float scale;         /* logit scale, normally 1/sqrt(d) */
     csa_seq* seqs;       /* [B]; len is updated in place when append = 1 */
-    const csa_bf16* x;       /* raw latents [*, d] */
-    const csa_bf16* logit_c; /* CSA compressor logits [*, d] */
-    const csa_bf16* logit_h; /* HCA compressor logits [*, d] */
-    const csa_bf16* idx_key; /* raw indexer keys [*, d_I] */
+    csa_bf16* x;             /* raw latents [*, d] (written only when new_rows is given) */
+    csa_bf16* logit_c;       /* CSA compressor logits [*, d] (idem) */
+    csa_bf16* logit_h;       /* HCA compressor logits [*, d] (idem) */
+    csa_bf16* idx_key;       /* raw indexer keys [*, d_I] (idem) */
     const float* bias_c;     /* [2m, d] */
     const float* bias_h;     /* [m_hca, d] */
     csa_bf16* entries;       /* CSA entry cache [*, d] */
@@ -161,6 +162,9 @@ typedef struct csa_decode_args {
     float* out;              /* [B, H, d] merged output */
     float* lse;              /* [B, H] merged log-sum-exp (nullable) */
     int32_t* idx_out;        /* [B, k] selected entries (nullable) */
+    const csa_bf16* new_rows; /* [B, 3d + d_I]: x | logit_c | logit_h | idx_key of each sequence's
+                                 appended token, copied into the caches by the call (append = 1;
+                                 16-byte aligned rows), or NULL */
 } csa_decode_args;
 
 /* a8 + a3..a7 -- one decode step: optional append (and the compressor updates it triggers), then

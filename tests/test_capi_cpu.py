@@ -42,15 +42,17 @@ def test_struct_layouts_match_header(tmp_path):
     prog = tmp_path / "sizes.c"
     prog.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "csa.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(csa_dims), sizeof(csa_seq),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(csa_dims), sizeof(csa_seq),"
         " sizeof(csa_query), sizeof(csa_ws_query), sizeof(csa_decode_args), sizeof(csa_prefill_args),"
-        " offsetof(csa_decode_args, out), offsetof(csa_prefill_args, idx_out));return 0;}\n")
+        " offsetof(csa_decode_args, out), offsetof(csa_prefill_args, idx_out),"
+        " offsetof(csa_decode_args, new_rows));return 0;}\n")
     exe = tmp_path / "sizes"
     subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
     assert got == [ctypes.sizeof(csa.csa_dims), 32, 16, ctypes.sizeof(csa.csa_ws_query),
                    ctypes.sizeof(csa.csa_decode_args), ctypes.sizeof(csa.csa_prefill_args),
-                   csa.csa_decode_args.out.offset, csa.csa_prefill_args.idx_out.offset]
+                   csa.csa_decode_args.out.offset, csa.csa_prefill_args.idx_out.offset,
+                   csa.csa_decode_args.new_rows.offset]
 
 
 def test_version_and_error_string(lib):

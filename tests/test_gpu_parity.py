@@ -231,7 +231,22 @@ def test_bad_index_is_reported_not_read():
 
 # --------------------------------------------------------------------------------- end to end
 
-def _decode_e2e(wl, steps, check_every=1):
+def _new_rows(wl, layer, s):
+    """The appended token's raw rows of step s for every sequence as new_rows [B, 3d + d_I], after
+    zeroing those rows in the layer's caches (so only the call's own copy can put them back)."""
+    d = wl.dims
+    rows = []
+    for b in range(wl.B):
+        t = wl.n0[b] + s
+        parts = [workloads.raw_tokens(wl, b, t, t + 1, name)[0] for name in ("x", "a", "b", "kI")]
+        rows.append(np.concatenate(parts))
+        r = layer.tok_off[b] + t
+        for cache in (layer.x, layer.logit_c, layer.logit_h, layer.idx_key):
+            cache[r].zero_()
+    return torch.from_numpy(np.stack(rows).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _decode_e2e(wl, steps, check_every=1, via_new_rows=False):
     layer = gh.new_layer(wl)
     d = wl.dims
     B = wl.B
@@ -247,7 +262,8 @@ def _decode_e2e(wl, steps, check_every=1):
     for s in range(steps):
         for b in range(B):
             sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
-        layer.decode(layer.decode_args(q, qi, w, out, lse=lse, idx_out=idx), ws)
+        nr = _new_rows(wl, layer, s) if via_new_rows else None
+        layer.decode(layer.decode_args(q, qi, w, out, lse=lse, idx_out=idx, new_rows=nr), ws)
         assert csa.csa_sync_status() == csa.CSA_OK
         if s % check_every and s != steps - 1:
             continue
@@ -267,6 +283,15 @@ def _decode_e2e(wl, steps, check_every=1):
                          ids=["tiny", "prod6000", "ragged3"])
 def test_decode_end_to_end(wl, steps):
     _decode_e2e(wl, steps)
+
+
+@pytest.mark.parametrize("wl,steps", [(workloads.tiny(), 1), (wl_small([700, 3000, 9001], B=3), 3)],
+                         ids=["tiny", "ragged3"])
+def test_decode_appended_rows_from_new_rows(wl, steps):
+    """The appended token's rows handed over as new_rows (the caches hold zeros there) give the same
+    results as the oracle: the append kernel copies them in before it compresses (the tiny step and
+    the third ragged step of sequence 2, at L = 1024 and 9004, each complete a CSA entry)."""
+    _decode_e2e(wl, steps, via_new_rows=True)
 
 
 @pytest.mark.parametrize("N,rows,dims", [
