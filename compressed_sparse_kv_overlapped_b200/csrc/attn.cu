@@ -24,8 +24,11 @@
 // Warp roles: warps 0-3 softmax + epilogue, warps 4-7 cp.async loaders (gathered rows, manual
 // swizzle, zero-fill for masked slots), warp 8 TMEM allocator + Q.K^T issuer, warp 9 P.V issuer.  Two
 // key stages; every wait is bounded (kWaitLimitNs) and winds the CTA down on timeout.
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tma.h"
 
 namespace csa {
 
@@ -71,6 +74,12 @@ struct Bars {
     uint64_t fin;             // both MMA issuers committed before teardown
 };
 
+// Tensor maps of the HCA cache and of the raw latents (boxes of 64 rows x 64 bf16, 128-byte swizzle).
+struct AttnMaps {
+    CUtensorMap hca;
+    CUtensorMap x;
+};
+
 // Per-CTA constants of the key list [CSA slots | raw window | HCA entries] of one query.
 struct KeyList {
     const int32_t* idx;      // this query's k slots
@@ -99,7 +108,8 @@ __device__ __forceinline__ const uint16_t* key_row(const AttnParams& p, int D, c
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_item_base) {
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnMaps maps, AttnParams p,
+                                                           int p_item_base) {
     using L = Smem<D>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -197,10 +207,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(AttnParams p, int p_i
         const uint32_t lane_blk = (uint32_t)(lane >> 3) * L::kBlock;  // block of chunk `lane`
         const uint32_t lane_c7 = (uint32_t)(lane & 7);
         if (dep_wait) grid_dep_wait();  // the selected indices come from the previous kernel
+        if (lw == 0 && lane == 0) {
+            if (p.tma_hca) tma_prefetch_map(&maps.hca);
+            if (p.tma_x) tma_prefetch_map(&maps.x);
+        }
         for (int t = 0; t < T; ++t) {
             const int st = t % kStages;
             if (t >= kStages && !mbar_wait(&bars->empty[st], ((t / kStages) - 1) & 1, p.status, abort_flag)) break;
             const int64_t tb = s0 + (int64_t)t * kTileKeys;
+            // A full tile of consecutive cache rows (HCA entries, or raw window tokens) goes by TMA:
+            // one thread issues the boxes, the tile's bytes complete the full barrier, and the
+            // loaders move on without waiting for the data.
+            const CUtensorMap* map = nullptr;
+            int64_t row = 0;
+            if (tb + kTileKeys <= s1) {
+                if (p.tma_hca && tb >= front && tb - front + kTileKeys <= kl.n_hca) {
+                    map = &maps.hca;
+                    row = kl.hca_row0 + (tb - front);
+                } else if (p.tma_x && tb >= p.k_slots && tb - p.k_slots + kTileKeys <= kl.nw) {
+                    map = &maps.x;
+                    row = kl.win_row0 + (tb - p.k_slots);
+                }
+                if (row < 0 || row > 0x7FFFFFFF - kTileKeys) map = nullptr;
+            }
+            if (map) {
+                if (lw == 0 && lane == 0) {
+                    for (int w4 = 0; w4 < 4; ++w4) mask16[st * 4 + w4] = 0xFFFFu;
+                    mbar_arrive_expect_tx(&bars->full[st], (uint32_t)(kTileKeys * D * 2));
+                    const uint32_t kdst = sbase + L::kK + (uint32_t)st * L::kStage;
+#pragma unroll
+                    for (int kb = 0; kb < L::NKB; ++kb)
+                        tma_load_2d(kdst + (uint32_t)kb * L::kBlock, map, kb * 64, (int)row, &bars->full[st]);
+                } else {
+                    mbar_arrive(&bars->full[st]);
+                }
+                continue;
+            }
             bool valid = false;
             if (lane < 16) {
                 const int64_t s = tb + lw * 16 + lane;
@@ -595,7 +637,17 @@ cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, 
         attr = true;
     }
     const dim3 grid = p.hca_first ? dim3((unsigned)(p.n_items * p.Q)) : dim3((unsigned)item_count, (unsigned)p.Q);
-    return launch_kernel(attn_kernel<D>, grid, dim3(kThreads), L::kAlloc, stream, pdl, p, item_begin);
+    // tensor maps over the HCA cache and the raw latents; the kernel only issues boxes that lie
+    // inside one sequence's valid rows, so the row extent is left open
+    AttnMaps maps;
+    AttnParams q = p;
+    q.tma_hca = p.use_hca && p.hca &&
+                tensor_map_2d_bf16(&maps.hca, p.hca, D, 0x7FFFFFFFull, (uint64_t)D * 2, 64, kTileKeys) == cudaSuccess;
+    q.tma_x = p.raw && p.W >= kTileKeys &&
+              tensor_map_2d_bf16(&maps.x, p.raw, D, 0x7FFFFFFFull, (uint64_t)D * 2, 64, kTileKeys) == cudaSuccess;
+    if (!q.tma_hca) std::memset(&maps.hca, 0, sizeof(maps.hca));
+    if (!q.tma_x) std::memset(&maps.x, 0, sizeof(maps.x));
+    return launch_kernel(attn_kernel<D>, grid, dim3(kThreads), L::kAlloc, stream, pdl, maps, q, item_begin);
 }
 
 }  // namespace

@@ -116,6 +116,9 @@ struct AttnParams {
     // they take the free SMs before the front items (which wait for the top-k) do.  Launches all
     // items of all queries.
     int hca_first;
+    // 1: full key tiles that are contiguous rows of the HCA cache / of the raw window are loaded by
+    // TMA (set by the launcher when the tensor maps could be encoded)
+    int tma_hca, tma_x;
     // outputs
     float* out;                 // [Q, H, d]
     float* lse;                 // [Q, H] nullable
