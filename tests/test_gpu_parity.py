@@ -420,3 +420,53 @@ def test_prefill_full_size_sampled():
         slack = gh.score_slack(qih, wh, ref.KI[:L // d.m])
         gh.sets_explained(idx_h[r_i], r["idx"], r["scores"], slack)
         gh.check_close(out_h[r_i], r["O"], f"prefill row {i}")
+
+
+@pytest.mark.slow
+def test_prefill_select_when_the_sample_overestimates():
+    """The prefill select estimates its threshold bin from a strided sample of each row (every 8th
+    score at 32,768 entries).  Here only 300 entries score high and all of them sit at sampled
+    positions, so the sample's estimate keeps fewer than k entries; the select must notice and keep
+    the whole row, and still return the exact top-k.  Indexer keys are written directly into the
+    cache (prefill with compress = 0) so that query q^I = e_0 on head 0 (weight 1, other heads 0)
+    scores entry j as relu(K_j[0])."""
+    N = 131072
+    d = SMALL_PROD
+    wl = workloads.Workload("prefill_sample_check", 4010, d, (N,), 0, mode="prefill")
+    layer = csa.HybridLayer(gh.dims_of(d), [N])
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths([N])
+    layer.compress()
+    E = N // d.m
+    rng = np.random.default_rng(7)
+    col0 = rng.permutation(E).astype(np.float64) / E * 0.5 + 0.25  # distinct values in [0.25, 0.75)
+    high = np.arange(0, 8 * 300, 8)                                  # 300 sampled positions
+    col0[high] = 10.0 + np.arange(300) / 300.0
+    keys = np.zeros((E, d.d_I), dtype=np.float32)
+    keys[:, 0] = col0
+    keys_bf16 = torch.from_numpy(keys).to(torch.bfloat16)
+    layer.entry_keys.copy_(keys_bf16.cuda())
+    q0 = N - 4
+    nq = 4
+    q = torch.zeros(nq, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.zeros(nq, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    qi[:, 0, 0] = 1.0
+    w = torch.zeros(nq, d.H_I, dtype=torch.float32, device="cuda")
+    w[:, 0] = 1.0
+    out = torch.empty(nq, d.H, d.d, dtype=torch.float32, device="cuda")
+    idx = torch.empty(nq, d.k, dtype=torch.int32, device="cuda")
+    ws = layer.prefill_workspace(N)
+    # the call's query rows are positions q0 .. q0 + 3 (row r of q / qi / w is position q0 + r)
+    layer.prefill(layer.prefill_args(q, qi, w, out, q0, N, compress=False, idx_out=idx), ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    kb = keys_bf16.view(torch.int16).numpy().view(np.uint16)
+    qih = np.zeros((d.H_I, d.d_I), dtype=np.uint16)
+    qih[0, 0] = 0x3F80  # bf16 1.0
+    wh = np.array([1.0, 0.0, 0.0, 0.0], dtype=np.float32)
+    got = idx.cpu().numpy()
+    for r in range(nq):
+        L = q0 + r + 1
+        s = oracle.index_scores(qih, wh, kb[:L // d.m])
+        want = oracle.topk(s, d.k)
+        assert set(got[r].tolist()) == set(want.tolist()), f"row {r}"
+        assert set(high.tolist()) <= set(got[r].tolist())
