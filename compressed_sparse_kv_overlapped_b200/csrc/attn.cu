@@ -11,19 +11,21 @@
 // It is cut into items (the front part and the HCA part separately, so the HCA items do not depend
 // on the top-k and can run while it is computed); one CTA computes one (query, item) pair:
 //     S   = Q . K^T           (64 heads x 64 keys,  contraction over d)   tcgen05, M=64 N=64
-//     P   = exp2(S*scale*log2e - m)  (online softmax, one row per thread)
+//     P   = exp2(S*scale*log2e - m)  (online softmax; four lanes share two rows)
 //     O  += P . V             (64 heads x d, contraction over 64 keys)    tcgen05, M=64 N=256/128
 // and writes either the final normalized output (single item) or a partial (O / l, lse) that
 // combine_kernel merges by log-sum-exp.  The CSA/HCA merge of the method is exactly that merge.
 //
-// Layout: Q [64 x d] and each key tile [64 x d] live in shared memory as 128-byte-swizzled
-// K-major blocks of 64 rows x 64 bf16; the key tile doubles as the MN-major B operand of the P.V
-// product, so every key is loaded once.  TMEM holds S (64 columns) and O (d columns split over
-// the two 16-lane halves of every sub-partition, the interleaved M=64 accumulator layout).
+// Layout: with M = 64 a head row lives in one 16-lane half of its warp's TMEM sub-partition.
+// Lanes 0-15 hold Q (the A operand of Q.K^T, two bf16 per column) and two S buffers; lanes 16-31
+// hold the fp32 O accumulator over all d columns.  Each key tile [64 x d] lives in shared memory
+// as 128-byte-swizzled K-major blocks of 64 rows x 64 bf16 and doubles as the MN-major B operand
+// of the P.V product, so every key is loaded once.  P is double-buffered in shared memory.
 //
-// Warp roles: warps 0-3 softmax + epilogue, warps 4-7 cp.async loaders (gathered rows, manual
-// swizzle, zero-fill for masked slots), warp 8 TMEM allocator + Q.K^T issuer, warp 9 P.V issuer.  Two
-// key stages; every wait is bounded (kWaitLimitNs) and winds the CTA down on timeout.
+// Warp roles: warps 0-3 softmax + epilogue (O from TMEM straight to global memory), warps 4-7
+// loaders (cp.async for gathered rows with manual swizzle and zero-fill of masked slots; TMA for
+// full tiles of consecutive cache rows), warp 8 TMEM allocator + Q.K^T issuer, warp 9 P.V issuer.
+// Three key stages; every wait is bounded (kWaitLimitNs) and winds the CTA down on timeout.
 #include <cstring>
 
 #include "common.cuh"
@@ -477,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             tc_fence_before();
             mbar_arrive(&bars->p_full[sb]);
         }
-        // ---- epilogue: TMEM -> shared memory (the key stages are free now) -> bulk stores
+        // ---- epilogue: TMEM -> registers -> global memory
         if (ok && T > 0) ok = mbar_wait(&bars->o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, p.status, abort_flag);
         float inv[2];
         bool has[2];
@@ -488,12 +490,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             has[rr] = ok && T > 0 && l_run[rr] > 0.f;
             inv[rr] = has[rr] ? 1.f / l_run[rr] : 0.f;
         }
-        // staging rows of D floats, padded by 4 floats so row-strided writes spread over the banks
-        constexpr int kStride = D + 4;
-        float* stage = reinterpret_cast<float*>(sm + L::kK);
-        static_assert(64 * (D + 4) * 4 <= kStages * Smem<D>::kStage, "epilogue staging exceeds the key stages");
         const bool write_o = ok && T > 0;
+        const int rows = p.H < kHeadsPad ? p.H : kHeadsPad;
         if (write_o) {
+            // straight from the registers: per row, the four lanes of a quad write 32 consecutive
+            // bytes (one full sector) per instruction
+            float* dst[2];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr)
+                dst[rr] = direct ? p.out + ((int64_t)qi * p.H + hr[rr]) * D
+                                 : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + hr[rr]) * D;
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < D; c += 64) {
@@ -503,27 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int col = c + 8 * k + cq;
-                    *reinterpret_cast<float2*>(stage + hr[0] * kStride + col) =
-                        make_float2(__uint_as_float(r[4 * k]) * inv[0], __uint_as_float(r[4 * k + 1]) * inv[0]);
-                    *reinterpret_cast<float2*>(stage + hr[1] * kStride + col) =
-                        make_float2(__uint_as_float(r[4 * k + 2]) * inv[1], __uint_as_float(r[4 * k + 3]) * inv[1]);
+                    if (hr[0] < rows)
+                        *reinterpret_cast<float2*>(dst[0] + col) =
+                            make_float2(__uint_as_float(r[4 * k]) * inv[0], __uint_as_float(r[4 * k + 1]) * inv[0]);
+                    if (hr[1] < rows)
+                        *reinterpret_cast<float2*>(dst[1] + col) = make_float2(__uint_as_float(r[4 * k + 2]) * inv[1],
+                                                                             __uint_as_float(r[4 * k + 3]) * inv[1]);
                 }
-            }
-        }
-        // staged rows become visible to the bulk-copy engine (async proxy) after this fence + barrier
-        fence_proxy_async_smem();
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps (128 threads)
-        const int rows = p.H < kHeadsPad ? p.H : kHeadsPad;
-        if (write_o) {
-            // one lane per warp hands the warp's 16 staged rows to the bulk-copy engine
-            if (i == 0) {
-                for (int hh = warp * 16; hh < warp * 16 + 16 && hh < rows; ++hh) {
-                    float* dst = direct ? p.out + ((int64_t)qi * p.H + hh) * D
-                                        : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + hh) * D;
-                    bulk_store(dst, smem_u32(stage + hh * kStride), D * 4);
-                }
-                bulk_commit();
-                bulk_wait_all();
             }
         } else if (direct) {
             const int tid = threadIdx.x;  // 0..127

@@ -123,14 +123,9 @@ ItemPlan plan_standalone(int64_t front_keys, int64_t max_hca, int Q) {
 // SMs of the part the decode plan is sized for (B200); another count only changes the balance.
 constexpr int kPlanSMs = 148;
 
-// HCA attention placement at decode: 0 = in the same launch as the front items, after the top-k
-// (default); 1 = on a helper stream alongside the indexer scan.
-bool hca_on_side_stream() { return env_int("CSA_HCA_SIDE", 0) != 0; }
-
-// Decode: small front items (they run after the top-k, on the critical path).  HCA items: with the
-// front items, enough of them to fill the SMs the front items leave free (one wave when it fits);
-// on the helper stream, about 40 over all queries.
-ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh, bool side) {
+// Decode: small front items (they run after the top-k, on the critical path); HCA items enough to
+// fill the SMs the front items leave free (one wave when it fits).
+ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh) {
     const int f = env_int("CSA_KPI_FRONT", 0), h = env_int("CSA_KPI_HCA", 0);
     const int kpi_front = f > 0 ? round64(f) : 128;
     const int64_t front = (int64_t)d.k + d.W;
@@ -138,8 +133,6 @@ ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh, bool side) 
     int kpi_hca;
     if (h > 0) {
         kpi_hca = round64(h);
-    } else if (side) {
-        kpi_hca = clamp_kpi(((int64_t)B * max_eh + 39) / 40, 128, 4096);
     } else {
         const int64_t hca_ctas = front_ctas < kPlanSMs - B ? kPlanSMs - front_ctas : kPlanSMs;
         kpi_hca = clamp_kpi(((int64_t)B * max_eh + hca_ctas - 1) / hca_ctas, 128, 4096);
@@ -230,7 +223,7 @@ DecodePlan plan_decode(const csa_dims& d, int B, int64_t max_len) {
     pl.max_eh = max_len / d.m_hca;
     pl.e_stride = ((pl.max_e + 3) / 4) * 4;
     if (pl.e_stride < 4) pl.e_stride = 4;
-    pl.items = plan_decode_items(d, B, pl.max_eh, hca_on_side_stream());
+    pl.items = plan_decode_items(d, B, pl.max_eh);
     size_t off = 0;
     pl.off_queries = off;
     off += align256((size_t)B * sizeof(csa_query));
@@ -239,10 +232,7 @@ DecodePlan plan_decode(const csa_dims& d, int B, int64_t max_len) {
     pl.off_index = off;
     off += index_ws_bytes(B, pl.e_stride);
     pl.off_attn = off;
-    // sized for either HCA placement, so the size does not depend on the environment
-    const size_t a0 = attn_ws_bytes(B, plan_decode_items(d, B, pl.max_eh, false).n_items, d.d);
-    const size_t a1 = attn_ws_bytes(B, plan_decode_items(d, B, pl.max_eh, true).n_items, d.d);
-    off += a0 > a1 ? a0 : a1;
+    off += attn_ws_bytes(B, pl.items.n_items, d.d);
     pl.total = off;
     return pl;
 }
@@ -284,32 +274,6 @@ int status_ptr(int** out) {
         ptrs[dev] = static_cast<int*>(p);
     }
     *out = ptrs[dev];
-    return CSA_OK;
-}
-
-// Helper stream + fork/join events of hybrid_attn_decode, one set per device, created on the first
-// decode call on that device (not device memory).
-struct SideStream {
-    cudaStream_t s = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-};
-std::mutex g_side_mu;
-SideStream g_side[64];
-
-int side_stream(SideStream** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= 64) return fail(CSA_ERR_CUDA, "device ordinal %d", dev);
-    std::lock_guard<std::mutex> lock(g_side_mu);
-    SideStream& ss = g_side[dev];
-    if (!ss.s) {
-        if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess ||
-            (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess ||
-            (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess)
-            return cuda_fail(e, "helper stream");
-    }
-    *out = &ss;
     return CSA_OK;
 }
 
@@ -626,47 +590,19 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     rc = make_attn(ap2, &d, a->seqs, queries, a->B, a->q, a->entries, idx, d.k, a->x, d.W, a->hca_entries, a->scale,
                    a->out, a->lse, w + pl.off_attn, pl.items);
     if (rc) return rc;
-    const int n_front = pl.items.n_items == 1 ? 1 : pl.items.items_front;
-    const int n_hca = pl.items.n_items - n_front;
     // programmatic dependent launch chains append -> scan -> select -> attention -> merge unless
     // stage events are being recorded between them
     const bool pdl = ev[0] == nullptr && env_int("CSA_NO_PDL", 0) == 0;
-    if (!hca_on_side_stream() || n_hca == 0) {
-        // every item in one launch after the top-k; the HCA items need no top-k and start as soon
-        // as the select kernel frees SMs
-        ap2.hca_nowait = pdl ? 1 : 0;
-        ap2.hca_first = (pl.items.n_items > 1 && pl.items.items_front > 0) ? 1 : 0;
-        rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
-                       ws_index, false, st, stream, ev[2], pdl);
-        if (rc) return rc;
-        if ((e = mark(ev[3], stream)) != cudaSuccess) return cuda_fail(e, "event record");
-        e = launch_attention_items(ap2, 0, pl.items.n_items, stream, pdl);
-        if (e == cudaSuccess) e = launch_combine(ap2, stream, pdl);
-        if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-        if ((e = mark(ev[4], stream)) != cudaSuccess) return cuda_fail(e, "event record");
-        return CSA_OK;
-    }
-    // The HCA items do not depend on the top-k: they run on a helper stream while the indexer
-    // scans, joined back before the merge.
-    SideStream* side = nullptr;
-    if ((rc = side_stream(&side))) return rc;
-    std::unique_lock<std::mutex> lock(g_side_mu);
-    if ((e = cudaEventRecord(side->fork, stream)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess ||
-        (e = launch_attention_items(ap2, n_front, n_hca, side->s)) != cudaSuccess ||
-        (e = cudaEventRecord(side->join, side->s)) != cudaSuccess)
-        return cuda_fail(e, "HCA attention launch");
+    // every item in one launch after the top-k; the HCA items need no top-k and start as soon as the
+    // select kernel frees SMs
+    ap2.hca_nowait = pdl ? 1 : 0;
+    ap2.hca_first = (pl.items.n_items > 1 && pl.items.items_front > 0) ? 1 : 0;
     rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
-                   ws_index, false, st, stream, ev[2], false);
-    if (rc) {
-        cudaStreamWaitEvent(stream, side->join, 0);  // keep the capture / stream joined
-        return rc;
-    }
+                   ws_index, false, st, stream, ev[2], pdl);
+    if (rc) return rc;
     if ((e = mark(ev[3], stream)) != cudaSuccess) return cuda_fail(e, "event record");
-    e = launch_attention_items(ap2, 0, n_front, stream, pdl);
-    cudaError_t e2 = cudaStreamWaitEvent(stream, side->join, 0);
-    if (e == cudaSuccess) e = e2;
-    if (e == cudaSuccess) e = launch_combine(ap2, stream);
+    e = launch_attention_items(ap2, 0, pl.items.n_items, stream, pdl);
+    if (e == cudaSuccess) e = launch_combine(ap2, stream, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     if ((e = mark(ev[4], stream)) != cudaSuccess) return cuda_fail(e, "event record");
     return CSA_OK;
