@@ -280,21 +280,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // ------------------------------------------------------------------ MMA issuers
         // warp 8 issues Q.K^T of every tile (A = Q from TMEM), warp 9 issues P.V (A = P, B = the key
         // tile read MN-major as V): the two products of neighbouring tiles reach the tensor pipe
-        // independently, so a P.V never waits behind the issue of the next Q.K^T (each issue blocks
-        // its thread for about the product's duration).
+        // independently, so a P.V never waits behind the issue of the next Q.K^T.  Each warp runs
+        // its loop with all lanes (warp-uniform waits and operands; one elected lane issues).
         if (dep_wait) grid_dep_wait();
-        if (lane == 0 && T > 0) {
+        if (T > 0) {
             if (warp == 8) {
                 constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
-                bool ok = mbar_wait(&bars->q_full, 0, p.status, abort_flag);
+                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0, p.status, abort_flag));
                 for (int g1 = 0; ok && g1 < T; ++g1) {
                     const int st = g1 % kStages;
-                    if (!mbar_wait(&bars->full[st], (g1 / kStages) & 1, p.status, abort_flag)) break;
-                    if (g1 >= 2 && !mbar_wait(&bars->s_free[g1 & 1], ((g1 >> 1) - 1) & 1, p.status, abort_flag)) break;
+                    bool w = mbar_wait(&bars->full[st], (g1 / kStages) & 1, p.status, abort_flag);
+                    if (w && g1 >= 2) w = mbar_wait(&bars->s_free[g1 & 1], ((g1 >> 1) - 1) & 1, p.status, abort_flag);
+                    if (!__all_sync(0xffffffffu, w)) break;
                     tc_fence_after();
                     const uint64_t kd = sdesc_kmajor(sbase + L::kK + (uint32_t)st * L::kStage);
                     const uint32_t tS = tmem + kColS + (uint32_t)(g1 & 1) * 64u;
-#pragma unroll 1
+#pragma unroll
                     for (int kb = 0; kb < L::NKB; ++kb) {
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks) {
@@ -310,7 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 constexpr int HALVES = D >= 256 ? D / 256 : 1;
                 constexpr uint32_t id2 = idesc_bf16(64, N2, false, true);
                 for (int g2 = 0; g2 < T; ++g2) {
-                    if (!mbar_wait(&bars->p_full[g2 & 1], (g2 >> 1) & 1, p.status, abort_flag)) break;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->p_full[g2 & 1], (g2 >> 1) & 1, p.status, abort_flag)))
+                        break;
                     tc_fence_after();
                     const int st = g2 % kStages;
                     const uint64_t vd = sdesc_mnmajor(sbase + L::kK + (uint32_t)st * L::kStage, L::kBlock);

@@ -118,13 +118,15 @@ __global__ void __launch_bounds__(kPsThreads, 1) prefill_score_kernel(PrefillSco
         cp_async_wait_all();
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // the whole warp runs the loop (warp-uniform waits and operands); one elected lane issues
+        {
             constexpr uint32_t id = idesc_bf16(kPsRows, kPsTile, false, false);
-            bool ok = mbar_wait(&bars->a_full, 0, p.status, abort_flag);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->a_full, 0, p.status, abort_flag));
             for (int t = 0; ok && t < T; ++t) {
                 const int st = t % kPsStages, ab = t & 1;
-                if (!mbar_wait(&bars->full[st], (t / kPsStages) & 1, p.status, abort_flag)) break;
-                if (t >= 2 && !mbar_wait(&bars->acc_empty[ab], ((t >> 1) - 1) & 1, p.status, abort_flag)) break;
+                bool w = mbar_wait(&bars->full[st], (t / kPsStages) & 1, p.status, abort_flag);
+                if (w && t >= 2) w = mbar_wait(&bars->acc_empty[ab], ((t >> 1) - 1) & 1, p.status, abort_flag);
+                if (!__all_sync(0xffffffffu, w)) break;
                 tc_fence_after();
                 const uint64_t bd = sdesc_kmajor(sbase + PsSmem::kB + st * kPsTile * 128);
 #pragma unroll
