@@ -123,8 +123,11 @@ ItemPlan plan_standalone(int64_t front_keys, int64_t max_hca, int Q) {
 // SMs of the part the decode plan is sized for (B200); another count only changes the balance.
 constexpr int kPlanSMs = 148;
 
-// Decode: small front items (they run after the top-k, on the critical path); HCA items enough to
-// fill the SMs the front items leave free (one wave when it fits).
+// Decode: small front items (they run after the top-k, on the critical path); HCA items of at
+// least kHcaMinKeys keys, as many as fill the SMs the front items leave free (one wave when it
+// fits).  The HCA items start when the scan frees SMs and finish by the time the front items do;
+// fewer, longer ones leave fewer partials to merge (measured at ctx1m: 8 tiles per item beat 5).
+constexpr int kHcaMinKeys = 512;
 ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh) {
     const int f = env_int("CSA_KPI_FRONT", 0), h = env_int("CSA_KPI_HCA", 0);
     const int kpi_front = f > 0 ? round64(f) : 128;
@@ -135,7 +138,8 @@ ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh) {
         kpi_hca = round64(h);
     } else {
         const int64_t hca_ctas = front_ctas < kPlanSMs - B ? kPlanSMs - front_ctas : kPlanSMs;
-        kpi_hca = clamp_kpi(((int64_t)B * max_eh + hca_ctas - 1) / hca_ctas, 128, 4096);
+        const int64_t per = ((int64_t)B * max_eh + hca_ctas - 1) / hca_ctas;
+        kpi_hca = clamp_kpi(per > kHcaMinKeys ? per : kHcaMinKeys, 128, 4096);
     }
     return make_items(front, max_eh, kpi_front, kpi_hca);
 }
