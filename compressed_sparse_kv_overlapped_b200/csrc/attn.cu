@@ -503,11 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 dst[rr] = direct ? p.out + ((int64_t)qi * p.H + hr[rr]) * D
                                  : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + hr[rr]) * D;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < D; c += 64) {
-                uint32_t r[32];
-                tmem_ld_16x256_x8(o_base + (uint32_t)c, r);
-                tmem_ld_wait();
+            // two register buffers: the TMEM load of the next 64 columns is in flight while the
+            // current ones are stored
+            auto store64 = [&](const uint32_t (&r)[32], int c) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int col = c + 8 * k + cq;
@@ -518,6 +516,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                         *reinterpret_cast<float2*>(dst[1] + col) = make_float2(__uint_as_float(r[4 * k + 2]) * inv[1],
                                                                              __uint_as_float(r[4 * k + 3]) * inv[1]);
                 }
+            };
+            static_assert(D % 128 == 0, "column chunks come in pairs");
+            uint32_t ra[32], rb[32];
+            tmem_ld_16x256_x8(o_base, ra);
+            tmem_ld_wait();
+#pragma unroll 1
+            for (int c = 0; c < D; c += 128) {
+                tmem_ld_16x256_x8(o_base + (uint32_t)(c + 64), rb);
+                store64(ra, c);
+                tmem_ld_wait();
+                if (c + 128 < D) tmem_ld_16x256_x8(o_base + (uint32_t)(c + 128), ra);
+                store64(rb, c + 64);
+                tmem_ld_wait();
             }
         } else if (direct) {
             const int tid = threadIdx.x;  // 0..127
