@@ -88,6 +88,14 @@ def test_host_validation_rejects_bad_arguments(lib):
         setattr(a, f, 256)
     rc = lib.hybrid_attn_decode(ctypes.byref(a), 256, 16, None)
     assert rc == csa.CSA_ERR_ARG and "workspace" in csa.csa_last_error()
+    # decode: appended rows handed over without an append, or misaligned
+    a.append, a.new_rows = 0, 256
+    rc = lib.hybrid_attn_decode(ctypes.byref(a), 256, 1 << 30, None)
+    assert rc == csa.CSA_ERR_ARG and "new_rows without append" in csa.csa_last_error()
+    a.append, a.new_rows = 1, 264
+    rc = lib.hybrid_attn_decode(ctypes.byref(a), 256, 1 << 30, None)
+    assert rc == csa.CSA_ERR_ARG and "aligned" in csa.csa_last_error()
+    a.new_rows = None
     # prefill: bad query range
     pa = csa.csa_prefill_args()
     pa.dims = dims
