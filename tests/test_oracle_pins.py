@@ -143,6 +143,25 @@ def test_locality(m, win):
     assert changed == expect
 
 
+@pytest.mark.parametrize("m,win", [(4, 8), (16, 16)])
+def test_entry_at_completion_equals_full_pass(m, win):
+    """An entry compressed the moment it completes, with only the tokens seen so far in existence
+    (the decode append), equals the same entry of a pass over the whole sequence (the prefill)."""
+    d, d_I, N = 8, 4, 9 * m
+    x = bf(SEED, synth.X, 13, N, d)
+    logit = bf(SEED, synth.A, 13, N, d)
+    kI = bf(SEED, synth.KI, 13, N, d_I) if win == 2 * m else None
+    bias = synth.f32_normal(SEED, synth.BIAS_C, 13, d, 0, win, scale=0.5)
+    Ef, Kf = oracle.compress(x, logit, bias, kI, N, m, win, np.arange(N // m))
+    for j in range(N // m):
+        L = m * (j + 1)
+        Ej, Kj = oracle.compress(x[:L].copy(), logit[:L].copy(), bias, None if kI is None else kI[:L].copy(), L, m,
+                                 win, [j])
+        np.testing.assert_array_equal(Ej[0], Ef[j])
+        if kI is not None:
+            np.testing.assert_array_equal(Kj[0], Kf[j])
+
+
 def test_entry_existence_rule():
     x = np.zeros((10, 4), dtype=np.uint16)
     b = np.zeros((8, 4), dtype=np.float32)
@@ -193,6 +212,16 @@ def test_index_score_heads_add():
         wh[h] = w[h]
         parts = parts + oracle.index_scores(qI, wh, KI)
     np.testing.assert_allclose(total, parts, rtol=1e-14)
+
+
+def test_index_score_follows_entry_permutation():
+    """Each entry's score depends on that entry's key alone: permuting the keys permutes the scores."""
+    d_I, n = 32, 77
+    KI = bf(SEED, synth.KI, 14, n, d_I)
+    qI = bf(SEED, synth.QI, 14, 4, d_I)
+    w = synth.f32_uniform(SEED, synth.W, 14, 4, 0, 1)[0]
+    perm = np.random.default_rng(3).permutation(n)
+    np.testing.assert_array_equal(oracle.index_scores(qI, w, KI[perm].copy()), oracle.index_scores(qI, w, KI)[perm])
 
 
 def brute_topk(s, k):
