@@ -28,6 +28,17 @@ sys.path.insert(0, ROOT)
 METRIC = "CSA+HCA decode queries/s at 1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
 
 
+def max_over_ranks(values, dev, world):
+    """Element-wise maximum of `values` over the ranks (the slowest rank sets the job's time);
+    the values themselves on one rank."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -231,11 +242,7 @@ def run_ours(args, rank, world):
     st = csa.csa_sync_status()
     if st != csa.CSA_OK:
         raise RuntimeError(f"device status {st} in the timed region")
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, = max_over_ranks([e0.elapsed_time(e1)], dev, world)
     # the same K steps again, with the stage events
     reset_lengths()
     with torch.cuda.stream(stream):
@@ -404,10 +411,7 @@ def run_e2e(layer, wl, K, W, max_len, ws, dev, world):
     st = csa.csa_sync_status()
     if st != csa.CSA_OK:
         raise RuntimeError(f"device status {st} in the e2e region")
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, = max_over_ranks([ms], dev, world)
     return {"value": B * world * K / (ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms / K,
             "how": "eager hybrid_attn_decode calls; per step one H2D copy of a packed pinned buffer (q, q_idx, "
@@ -623,10 +627,7 @@ def run_prefill(args, rank, world):
         raise RuntimeError("device status in the timed region")
     ms_comp = ev[0].elapsed_time(ev[1]) / K
     ms = ev[2].elapsed_time(ev[3]) / K
-    if world > 1:
-        t = torch.tensor([ms, ms_comp], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, ms_comp = (float(v) for v in t.tolist())
+    ms, ms_comp = max_over_ranks([ms, ms_comp], dev, world)
     f_index, f_attn = prefill_flops(wd, N)
     hbm, tf_peak, src = peaks(sustained=True)
     tflops = (f_index + f_attn) / (ms * 1e-3) / 1e12
@@ -731,18 +732,13 @@ def main():
         if res is not None:
             print(json.dumps(res), flush=True)
         return
-    if args.config == "prefill":
-        res = run_prefill(args, rank, world) if args.impl == "ours" else None
-        if res is not None and rank == 0:
-            print(json.dumps(res), flush=True)
-        return
     if world > 1:
         import datetime
 
         import torch
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    res = run_ours(args, rank, world)
+    res = run_prefill(args, rank, world) if args.config == "prefill" else run_ours(args, rank, world)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
