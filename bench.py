@@ -27,6 +27,11 @@ sys.path.insert(0, ROOT)
 
 METRIC = "CSA+HCA decode queries/s at 1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
 
+# DRAM bytes (read + write) of one ctx1m index_scan_kernel launch in an ncu capture of the same kernel
+# and launch shape (profiles/index_scan_ctx1m.md: 134.24 MB read, 4.13 MB of scores written).  Set it
+# to None whenever the scan kernel or its launch shape changes, until it is captured again.
+SCAN_TRAFFIC_BYTES = 138_370_000
+
 
 def max_over_ranks(values, dev, world):
     """Element-wise maximum of `values` over the ranks (the slowest rank sets the job's time);
@@ -302,7 +307,9 @@ def run_ours(args, rank, world):
                                 "note": "per-step durations in the stage-event graph (no launch overlap inside a "
                                         "step), not the timed graph"},
         "roofline": {"kernel": "index_scan_kernel", "bound": "hbm", "achieved": scan_gbs, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": (scan_gbs / hbm_peak) if scan_gbs else None, "traffic": None,
+                     "unit": "GB/s", "frac": (scan_gbs / hbm_peak) if scan_gbs else None,
+                     "traffic": SCAN_TRAFFIC_BYTES if wl.name.startswith("ctx1m") else None,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, profiles/index_scan_ctx1m.md",
                      "bytes_per_launch": int(per_step[0]), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
         "clocks": clocks.summary(t0, t1),
     }
