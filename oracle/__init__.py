@@ -9,10 +9,13 @@ Every stage cites its source passage in ``oracle.c``.  Parity status of each rou
 
 * compress, index_scores, topk, csa_attn, hca_attn, lse_merge: pinned by the invariant and
   special-case tests in ``tests/test_oracle_pins.py`` (window mean, weights summing to one,
-  locality, identity at m=1, brute-force selection, dense attention against a library softmax,
-  partition invariance of the merge).
-* hybrid_query (the composition): parity unpinned beyond those invariants -- the pages print no
-  worked numeric example of the composed method.
+  locality, identity at m=1, each indexer-key channel weighted by its own channel's softmax,
+  brute-force selection, dense attention against a library softmax, partition invariance of the
+  merge).
+* hybrid_query (the composition): pinned at q = 0, q^I = 0, where the merged softmax is uniform
+  over exactly the keys the method attends (lse = log of their count, O = their mean), at lengths
+  below and above the window and the HCA ratio.  Beyond that the pages print no worked numeric
+  example of the composed method.
 """
 from __future__ import annotations
 

@@ -162,6 +162,35 @@ def test_entry_at_completion_equals_full_pass(m, win):
             np.testing.assert_array_equal(Kj[0], Kf[j])
 
 
+@pytest.mark.parametrize("m,win,d_I,c,o", [(4, 8, 16, 0, 5), (4, 8, 16, 1, 2), (4, 8, 16, 9, 7),
+                                            (4, 8, 16, 15, 4), (2, 4, 8, 7, 3), (4, 8, 8, 3, 6)])
+def test_indexer_key_uses_its_own_channel_weights(m, win, d_I, c, o):
+    """Indexer-key channel c is weighted by channel c's own softmax (channels 0..d_I-1 of the
+    compressor).  Only channel c gets a dominant bias, at window offset o, so only channel c's weights
+    pick one token (start_j + o) and every other channel's weights are uniform.  Then KI[j, c] must be
+    that token's indexer key and every other key channel the window mean: a key channel weighted with
+    another channel's weights (a shifted, reversed or tail-aligned channel index) gives a mean where a
+    picked token belongs, or the reverse."""
+    d, L = 24, 10 * m
+    x = bf(SEED, synth.X, 15, L, d)
+    kI = bf(SEED, synth.KI, 15, L, d_I)
+    logit = np.zeros((L, d), dtype=np.uint16)
+    bias = np.zeros((win, d), dtype=np.float32)
+    bias[o, c] = 300.0
+    E, KI = oracle.compress(x, logit, bias, kI, L, m, win, np.arange(L // m))
+    xf, kf = f64(x), f64(kI)
+    for j in range(1, L // m):  # j >= 1: the whole window exists
+        start = m * j - (win - m)
+        t = start + o
+        mean_x, mean_k = xf[start:start + win].mean(0), kf[start:start + win].mean(0)
+        for cc in range(d):
+            want = xf[t, cc] if cc == c else mean_x[cc]
+            np.testing.assert_allclose(E[j, cc], want, rtol=1e-14, atol=1e-15)
+        for cc in range(d_I):
+            want = kf[t, cc] if cc == c else mean_k[cc]
+            np.testing.assert_allclose(KI[j, cc], want, rtol=1e-14, atol=1e-15, err_msg=f"entry {j} key channel {cc}")
+
+
 def test_entry_existence_rule():
     x = np.zeros((10, 4), dtype=np.uint16)
     b = np.zeros((8, 4), dtype=np.float32)
@@ -351,6 +380,33 @@ def test_noncausal_index_rejected():
     q = np.zeros((1, 4), np.uint16)
     with pytest.raises(ValueError):
         oracle.csa_attn(q, E, np.array([2], np.int32), 4, E, 8, 0, 1.0)  # L=8 -> entries 0,1 only
+
+
+@pytest.mark.parametrize("L", [1, 3, 9, 15, 16, 17, 40, 63, 64, 200, 777])
+def test_hybrid_query_composition_at_zero_query(L):
+    """The composed query at q = 0 and q^I = 0: every logit and every indexer score is 0, so the
+    top-k keeps entries 0..min(k, L/m)-1 (ties to the lower index) and the merged softmax is
+    uniform over exactly those entries, the raw window counted once and every visible HCA entry:
+    lse = log(min(k, floor(L/m)) + min(W, L) + floor(L/m')) and O is the plain mean of those keys.
+    A window counted twice, an HCA partial taken with the window, or a wrong visibility rule
+    changes the count."""
+    sh = oracle.Shape(d=16, H=2, d_I=8, H_I=4, m=4, m_hca=16, k=5, W=8)
+    raw = bf(SEED, synth.X, 16, L, sh.d)
+    n_c, n_h = L // sh.m, L // sh.m_hca
+    entries = bf(SEED, synth.A, 16, max(n_c, 1), sh.d)
+    KI = bf(SEED, synth.KI, 16, max(n_c, 1), sh.d_I)
+    hca = bf(SEED, synth.B, 16, max(n_h, 1), sh.d)
+    q = np.zeros((sh.H, sh.d), np.uint16)
+    qI = np.zeros((sh.H_I, sh.d_I), np.uint16)
+    w = np.full(sh.H_I, 0.5, np.float32)
+    r = oracle.hybrid_query(sh, L, q, qI, w, raw, entries, KI, hca)
+    n_sel, n_win = min(sh.k, n_c), min(sh.W, L)
+    count = n_sel + n_win + n_h
+    np.testing.assert_allclose(r["lse"], math.log(count), rtol=1e-14)
+    assert r["idx"][:n_sel].tolist() == list(range(n_sel))
+    assert (r["idx"][n_sel:] == -1).all()
+    keys = np.concatenate([f64(entries)[:n_sel], f64(raw)[L - n_win:L], f64(hca)[:n_h]])
+    np.testing.assert_allclose(r["O"], np.repeat(keys.mean(0)[None], sh.H, axis=0), rtol=1e-12, atol=1e-14)
 
 
 # ---------------------------------------------------------------- the pages' printed counts
