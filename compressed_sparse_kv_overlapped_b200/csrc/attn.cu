@@ -137,8 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // The query table and sequence lengths come from kernels at least two launches back, which are
     // complete once this grid runs (every kernel of the chain waits before it lets the next start).
     const csa_query qr = p.queries[qi];
-    const csa_seq sq = p.seqs[qr.seq];
-    const bool qvalid = qr.len >= 1 && qr.len <= sq.len;
+    const bool seq_ok = qr.seq >= 0 && qr.reserved == 0;
+    const csa_seq sq = seq_ok ? p.seqs[qr.seq] : csa_seq{0, 0, 0, 0};
+    const bool qvalid = seq_ok && qr.len >= 1 && qr.len <= sq.len;
     KeyList kl;
     kl.idx = p.idx ? p.idx + (int64_t)qi * p.k_slots : nullptr;
     kl.n_causal = qr.len / p.m;
@@ -635,12 +636,10 @@ __global__ void combine_kernel(AttnParams p) {
 template <int D>
 cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, cudaStream_t stream, bool pdl) {
     using L = Smem<D>;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static PerDeviceOnce attr;
+    cudaError_t ea = attr.run(
+        [] { return cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc); });
+    if (ea != cudaSuccess) return ea;
     const dim3 grid = p.hca_first ? dim3((unsigned)(p.n_items * p.Q)) : dim3((unsigned)item_count, (unsigned)p.Q);
     // tensor maps over the HCA cache and the raw latents; the kernel only issues boxes that lie
     // inside one sequence's valid rows, so the row extent is left open

@@ -265,12 +265,16 @@ PrefillPlan plan_prefill(const csa_dims& d, int64_t q_end) {
     return pl;
 }
 
+// Device address of g_status on the current device, looked up once per device (in host code the
+// name g_status is a host-side stand-in, not a device address).
 int status_ptr(int** out) {
+    static std::mutex mu;
     static int* ptrs[64] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= 64) return fail(CSA_ERR_CUDA, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(mu);
     if (!ptrs[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_status);
@@ -308,11 +312,7 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
 
 }  // namespace
 
-int* device_status() {
-    int* p = nullptr;
-    status_ptr(&p);
-    return p;
-}
+int device_status(int** out) { return status_ptr(out); }
 
 int validate_dims(const csa_dims* d) { return check_dims(d); }
 

@@ -10,6 +10,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/csa.h"
 
 namespace csa {
@@ -289,6 +292,32 @@ __device__ __forceinline__ float key_float(uint32_t k) {
     uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
     return __uint_as_float(u);
 }
+
+// Host side: run a set-up step (function attributes such as the dynamic shared-memory opt-in)
+// once per device, with that device current.  Function attributes belong to a device, so a
+// process that launches on several devices needs the step on each; concurrent first calls on one
+// device are serialized, and a step that fails is retried by the next call.
+class PerDeviceOnce {
+   public:
+    template <typename F>
+    cudaError_t run(F&& step) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        e = step();
+        if (e == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+        return e;
+    }
+
+   private:
+    static constexpr int kMaxDevices = 64;
+    std::mutex mu_;
+    std::atomic<bool> done_[kMaxDevices] = {};
+};
 
 // Launch `kernel` with an optional programmatic-dependent-launch attribute: the grid may start
 // while the previous kernel in the stream finishes; it must call grid_dep_wait() before it reads

@@ -90,7 +90,7 @@ extern "C" int csa_index_topk_noalloc(const csa_dims* dims, const csa_seq* seqs,
     ip.max_entries = max_e;
     ip.idx_out = idx_out;
     ip.score_out = score_out;
-    ip.status = device_status();
+    if ((rc = device_status(&ip.status)) != CSA_OK) return rc;
     index_ws_carve(ip, scratch, Q, es);
     // the histogram must start at zero; clear it in case an earlier call was cut short
     e = launch_index_topk(ip, max_e, stream, /*zero_ws=*/true);

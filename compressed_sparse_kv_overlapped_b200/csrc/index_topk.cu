@@ -94,6 +94,10 @@ __global__ void __launch_bounds__(kScanThreads) index_scan_kernel(IndexParams p)
     grid_dep_launch();
     const int qi = blockIdx.y;
     const csa_query qr = p.queries[qi];
+    if (qr.seq < 0 || qr.reserved != 0) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, CSA_ERR_INDEX);
+        return;
+    }
     const csa_seq sq = p.seqs[qr.seq];
     if (qr.len < 1 || qr.len > sq.len) {
         if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, CSA_ERR_INDEX);
@@ -373,10 +377,11 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     const int qi = blockIdx.y;
     const uint32_t rank = cluster_rank();
     const csa_query qr = p.queries[qi];
-    const csa_seq sq = p.seqs[qr.seq];
-    const bool valid = qr.len >= 1 && qr.len <= sq.len;
+    const bool seq_ok = qr.seq >= 0 && qr.reserved == 0;
+    const csa_seq sq = seq_ok ? p.seqs[qr.seq] : csa_seq{0, 0, 0, 0};
+    const bool valid = seq_ok && qr.len >= 1 && qr.len <= sq.len;
     int64_t E = valid ? qr.len / p.m : 0;
-    if (E > p.max_entries) {  // the launch was sized for fewer entries: refuse rather than guess
+    if (E > p.max_entries || !seq_ok) {  // the launch was sized for fewer entries: refuse rather than guess
         if (threadIdx.x == 0 && rank == 0) report(p.status, CSA_ERR_INDEX);
         E = 0;
     }
@@ -625,16 +630,13 @@ constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 }  // namespace
 
 cudaError_t select_attrs() {
-    static bool attr_set = false;
-    if (!attr_set) {
+    static PerDeviceOnce attr;
+    return attr.run([] {
         cudaError_t e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)SelSmem::bytes(kSelBufMax));
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    return cudaSuccess;
+        return cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    });
 }
 
 size_t index_ws_bytes(int Q, int64_t e_stride) {

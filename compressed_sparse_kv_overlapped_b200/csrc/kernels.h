@@ -160,7 +160,9 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 // Prefill helper: query table for positions [p0, p0 + n) of one sequence.
 cudaError_t launch_prefill_queries(csa_query* queries, int64_t p0, int64_t n, cudaStream_t stream);
 
-int* device_status();  // address of the device status word on the current device
+// Address of the device status word on the current device: CSA_OK, or an error code (with the
+// message recorded for csa_last_error) when it cannot be looked up.
+int device_status(int** out);
 
 // Error reporting shared by entry points defined outside capi.cu.
 int validate_dims(const csa_dims* d);             // CSA_OK or the error code (message set)

@@ -207,13 +207,11 @@ __global__ void __launch_bounds__(kPsThreads, 1) prefill_score_kernel(PrefillSco
 
 cudaError_t launch_prefill_scores(const PrefillScoreParams& p, int64_t max_entries, cudaStream_t stream, bool pdl) {
     if (p.Qn <= 0 || max_entries <= 0) return cudaSuccess;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             PsSmem::kAlloc);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    static PerDeviceOnce attr;
+    cudaError_t ea = attr.run([] {
+        return cudaFuncSetAttribute(prefill_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PsSmem::kAlloc);
+    });
+    if (ea != cudaSuccess) return ea;
     const int64_t gx = (max_entries + p.ent_per_cta - 1) / p.ent_per_cta;
     const int64_t gy = (p.Qn + kPsRows - 1) / kPsRows;
     return launch_kernel(prefill_score_kernel, dim3((unsigned)gx, (unsigned)gy), dim3(kPsThreads), PsSmem::kAlloc,

@@ -2,8 +2,8 @@
 // driver entry point, no link against libcuda) and the device-side tiled load into shared memory.
 //
 // Every tiled load used here starts at an innermost element offset that is a multiple of 64 bf16
-// (128 bytes), so the 16-byte rule for the innermost coordinate always holds, and no load uses
-// cluster multicast.
+// (128 bytes), so the 16-byte rule for the innermost coordinate always holds, and each load fills
+// only the issuing CTA's own shared memory.
 #pragma once
 
 #include <cuda.h>

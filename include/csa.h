@@ -85,9 +85,11 @@ typedef struct csa_seq {
 } csa_seq;
 
 /* One query: its sequence and its visible length L (the query sees raw tokens [0, L)).
- * Device memory. */
+ * Device memory.  Precondition: seq indexes an entry of the csa_seq table passed with it.  The
+ * calls are not given the table's length, so they cannot check the upper bound; a negative seq or a
+ * non-zero `reserved` is reported as CSA_ERR_INDEX and the query is skipped. */
 typedef struct csa_query {
-    int32_t seq;      /* index into the csa_seq table */
+    int32_t seq;      /* index into the csa_seq table, 0 <= seq < number of sequences */
     int32_t reserved; /* must be 0 */
     int64_t len;      /* visible length L, 1 <= L <= seqs[seq].len */
 } csa_query;
