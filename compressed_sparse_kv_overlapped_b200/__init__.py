@@ -28,7 +28,7 @@ CSA_OP_HCA_ATTN = 3
 CSA_OP_DECODE = 4
 CSA_OP_PREFILL = 5
 
-EXPORTS = ("csa_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
+EXPORTS = ("csa_compress", "csa_compress_all", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
            "hybrid_attn_prefill", "csa_workspace_size", "csa_last_error", "csa_sync_status", "csa_version",
            "csa_set_stage_events", "csa_index_topk_noalloc")
 CSA_DECODE_MARKS = 5
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         P = ctypes.POINTER
         L.csa_compress.argtypes = [P(csa_dims), ctypes.c_int, _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp]
+        L.csa_compress_all.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _vp, _vp, _vp]
         L.csa_index_topk.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                      _vp]
         L.csa_sparse_attn.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp,
@@ -88,7 +90,7 @@ def lib() -> ctypes.CDLL:
         L.csa_sync_status.argtypes = [_vp]
         L.csa_set_stage_events.argtypes = [_vp, ctypes.c_int]
         L.csa_index_topk_noalloc.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
-        for n in ("csa_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
+        for n in ("csa_compress", "csa_compress_all", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
                   "hybrid_attn_prefill", "csa_sync_status", "csa_version", "csa_set_stage_events",
                   "csa_index_topk_noalloc"):
             getattr(L, n).restype = ctypes.c_int
@@ -160,6 +162,14 @@ def csa_compress(dims, which, seqs, ranges, B, max_entries, x, logit, bias, idx_
                             _ptr(logit), _ptr(bias), _ptr(idx_key), _ptr(entries), _ptr(entry_keys),
                             _vp(_stream(stream)))
     _check(rc, "csa_compress")
+
+
+def csa_compress_all(dims, seqs, tok_ranges, B, max_tokens, x, logit_c, logit_h, bias_c, bias_h, idx_key, entries,
+                     entry_keys, hca_entries, stream=None) -> None:
+    rc = lib().csa_compress_all(ctypes.byref(dims), _ptr(seqs), _ptr(tok_ranges), B, max_tokens, _ptr(x),
+                                _ptr(logit_c), _ptr(logit_h), _ptr(bias_c), _ptr(bias_h), _ptr(idx_key),
+                                _ptr(entries), _ptr(entry_keys), _ptr(hca_entries), _vp(_stream(stream)))
+    _check(rc, "csa_compress_all")
 
 
 def csa_index_topk(dims, seqs, queries, Q, max_len, q_idx, w, entry_keys, idx_out, score_out, ws, stream=None):

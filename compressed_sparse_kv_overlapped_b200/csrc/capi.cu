@@ -145,61 +145,99 @@ ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// Decode append: one CTA per sequence.  len += 1 (if appending), compress the CSA / HCA entry the
-// new token completes, publish the query table, clear this query's index scratch words.
+// Decode append: one thread-block cluster of d/64 CTAs per sequence, CTA s owning channels
+// [64s, 64s + 64).  len += 1 (if appending); the new token's rows (new_rows) are copied into the
+// caches slice by slice; the CSA / HCA entries the token completes are compressed, each CTA its
+// channel slice, with the same arithmetic as the full pass (the block-partial form of
+// compress_dev.cuh where the shape allows, else the per-entry serial form); CTA 0 publishes the
+// query table row; the index scratch words are cleared.  seqs[b].len is written by CTA 0 after a
+// cluster barrier, once every CTA of the sequence has read the old value.
 // ---------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     grid_dep_launch();  // the scan may start its launch; it waits for this grid before reading
-    const int b = blockIdx.x;
-    __shared__ int64_t s_len;
-    if (threadIdx.x == 0) {
-        const int64_t len = p.seqs[b].len + (p.append ? 1 : 0);
-        s_len = len;
+    __shared__ float xs[8 * 8 * 24];
+    const int s = blockIdx.x, b = blockIdx.y, ns = gridDim.x;
+    const int tid = threadIdx.x;
+    const csa_seq sq = p.seqs[b];
+    const int64_t len = sq.len + (p.append ? 1 : 0);
+    if (s == 0 && tid == 0) {
         p.queries[b].seq = b;
         p.queries[b].reserved = 0;
         p.queries[b].len = len;
     }
     if (p.zero_words) {
-        const int64_t per = (p.n_zero_words + p.B - 1) / p.B;
-        const int64_t z0 = (int64_t)b * per, z1 = min(p.n_zero_words, z0 + per);
-        for (int64_t i = z0 + threadIdx.x; i < z1; i += blockDim.x) p.zero_words[i] = 0u;
+        const int64_t nc = (int64_t)p.B * ns, ci = (int64_t)b * ns + s;
+        const int64_t per = (p.n_zero_words + nc - 1) / nc;
+        const int64_t z0 = ci * per, z1 = min(p.n_zero_words, z0 + per);
+        for (int64_t i = z0 + tid; i < z1; i += blockDim.x) p.zero_words[i] = 0u;
     }
-    __syncthreads();
-    const int64_t len = s_len;
-    if (len < 1) {
-        if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
-        return;
-    }
-    const csa_seq sq = p.seqs[b];
-    if (p.append) {
+    const bool ok = len >= 1;
+    if (!ok && s == 0 && tid == 0) report(p.status, CSA_ERR_INDEX);
+    const int d = p.d, c0s = s * 64;
+    if (ok && p.append) {
         if (p.new_rows) {
-            // the appended token's rows (x | a | b | k^I) go into the caches at row tok_off + len - 1
+            // the appended token's rows (x | logit_c | logit_h | idx_key), this CTA's channels
             const int64_t r = sq.tok_off + len - 1;
-            const int wd = p.d >> 3, wi = p.d_I >> 3;  // 16-byte chunks per row
-            const uint4* src = reinterpret_cast<const uint4*>(p.new_rows + (int64_t)b * (3 * p.d + p.d_I));
-            for (int i = threadIdx.x; i < 3 * wd + wi; i += blockDim.x) {
-                const uint4 v = src[i];
-                if (i < wd) reinterpret_cast<uint4*>(p.x + r * p.d)[i] = v;
-                else if (i < 2 * wd) reinterpret_cast<uint4*>(p.logit_c + r * p.d)[i - wd] = v;
-                else if (i < 3 * wd) reinterpret_cast<uint4*>(p.logit_h + r * p.d)[i - 2 * wd] = v;
-                else reinterpret_cast<uint4*>(p.idx_key + r * p.d_I)[i - 3 * wd] = v;
+            const uint16_t* src = p.new_rows + (int64_t)b * (3 * d + p.d_I);
+            const int part = tid >> 3, ch = c0s + 8 * (tid & 7);
+            if (part < 3) {
+                uint16_t* dst = part == 0 ? p.x : part == 1 ? p.logit_c : p.logit_h;
+                *reinterpret_cast<uint4*>(dst + r * d + ch) = *reinterpret_cast<const uint4*>(src + part * d + ch);
+            } else if (part == 3 && ch < p.d_I) {
+                *reinterpret_cast<uint4*>(p.idx_key + r * p.d_I + ch) =
+                    *reinterpret_cast<const uint4*>(src + 3 * d + ch);
             }
-            __syncthreads();  // the compressor below reads these rows
+            __syncthreads();  // the compressor below reads these rows (coherent loads)
         }
-        const int tpe = p.d >> 3;
-        if (len % p.m == 0 && threadIdx.x < tpe) {
+        if (len % p.m == 0 && tid < 8) {
             const int64_t j = len / p.m - 1;
-            compress_entry8(j, p.m, 2 * p.m, p.d, p.d_I, threadIdx.x * 8, p.x, p.logit_c, p.bias_c, p.idx_key,
-                            sq.tok_off, p.entries + (sq.csa_off + j) * p.d, p.entry_keys + (sq.csa_off + j) * p.d_I);
+            const int c0 = c0s + 8 * tid;
+            uint16_t* orow = p.entries + (sq.csa_off + j) * d + c0;
+            if (csa_block_shape(p.m)) {
+                const int64_t t0 = sq.tok_off + 4 * j - 4;  // row of window position 0
+                auto fetch = [&](int tensor, int pos) -> uint4 {
+                    const int64_t row = t0 + pos;
+                    if (tensor == 2) return __ldcg(reinterpret_cast<const uint4*>(p.idx_key + row * p.d_I + c0));
+                    const uint16_t* base = tensor == 0 ? p.logit_c : p.x;
+                    return __ldcg(reinterpret_cast<const uint4*>(base + row * d + c0));
+                };
+                if (c0 < p.d_I)
+                    csa_entry_block4<true>(j, d, p.bias_c + c0, fetch, orow,
+                                           p.entry_keys + (sq.csa_off + j) * p.d_I + c0);
+                else
+                    csa_entry_block4<false>(j, d, p.bias_c + c0, fetch, orow, nullptr);
+            } else {
+                compress_entry8(j, p.m, 2 * p.m, d, p.d_I, c0, p.x, p.logit_c, p.bias_c, p.idx_key, sq.tok_off,
+                                p.entries + (sq.csa_off + j) * d, p.entry_keys + (sq.csa_off + j) * p.d_I);
+            }
         }
-        if (len % p.m_hca == 0 && threadIdx.x >= 128 && threadIdx.x < 128 + tpe) {
-            const int64_t j = len / p.m_hca - 1;
-            compress_entry8(j, p.m_hca, p.m_hca, p.d, p.d_I, (threadIdx.x - 128) * 8, p.x, p.logit_h, p.bias_h,
-                            nullptr, sq.tok_off, p.hca_entries + (sq.hca_off + j) * p.d, nullptr);
+        if (len % p.m_hca == 0) {  // uniform over the CTA (the block form has barriers)
+            const int64_t h = len / p.m_hca - 1;
+            if (hca_block_shape(p.m_hca)) {
+                const int nb = p.m_hca / 4, u = tid >> 3, g = tid & 7, ub = u & (nb - 1);
+                const int c0 = c0s + 8 * g;
+                const int64_t row0 = sq.tok_off + (int64_t)p.m_hca * h + 4 * ub;
+                uint4 lg[4], xv[4], kv[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    lg[t] = __ldcg(reinterpret_cast<const uint4*>(p.logit_h + (row0 + t) * d + c0));
+                    xv[t] = __ldcg(reinterpret_cast<const uint4*>(p.x + (row0 + t) * d + c0));
+                    kv[t] = make_uint4(0, 0, 0, 0);
+                }
+                Part8 P;
+                part4<false>(lg, xv, kv, p.bias_h + (int64_t)(4 * ub) * d + c0, d, P);
+                hca_tree(P, nb, xs);
+                if (tid < 8)
+                    *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) = finish8(P.acc, P.den);
+            } else if (tid >= 128 && tid < 136) {
+                compress_entry8(h, p.m_hca, p.m_hca, d, p.d_I, c0s + 8 * (tid - 128), p.x, p.logit_h, p.bias_h,
+                                nullptr, sq.tok_off, p.hca_entries + (sq.hca_off + h) * d, nullptr);
+            }
         }
-        __syncthreads();
-        if (threadIdx.x == 0) p.seqs[b].len = len;
     }
+    // every CTA of the sequence has read seqs[b].len: CTA 0 may now write the new length
+    cluster_barrier();
+    if (ok && p.append && s == 0 && tid == 0) p.seqs[b].len = len;
 }
 
 __global__ void prefill_queries_kernel(csa_query* q, int64_t p0, int64_t n) {
@@ -383,24 +421,130 @@ int csa_compress(const csa_dims* dims, int which, const csa_seq* seqs, const int
     if (max_entries == 0) return CSA_OK;
     int* st = nullptr;
     if ((rc = status_ptr(&st))) return rc;
-    CompressParams p{};
-    p.seqs = seqs;
-    p.ranges = ranges;
-    p.B = B;
-    p.which = which;
-    p.d = dims->d;
-    p.d_I = dims->d_I;
-    p.m = which ? dims->m_hca : dims->m;
-    p.win = which ? dims->m_hca : 2 * dims->m;
-    p.x = x;
-    p.logit = logit;
-    p.bias = bias;
-    p.idx_key = idx_key;
-    p.entries = entries;
-    p.entry_keys = entry_keys;
-    p.status = st;
-    cudaError_t e = launch_compress(p, max_entries, stream);
+    cudaError_t e;
+    if (which == 0 ? csa_block_shape(dims->m) : hca_block_shape(dims->m_hca)) {
+        TileCompressParams tp{};
+        tp.seqs = seqs;
+        tp.ranges = ranges;
+        tp.range_kind = which;
+        tp.B = B;
+        tp.d = dims->d;
+        tp.d_I = dims->d_I;
+        tp.m_hca = dims->m_hca;
+        tp.do_csa = which == 0;
+        tp.do_hca = which == 1;
+        tp.do_keys = idx_key != nullptr;
+        tp.x = x;
+        tp.logit_c = which == 0 ? logit : nullptr;
+        tp.logit_h = which == 1 ? logit : nullptr;
+        tp.idx_key = idx_key;
+        tp.bias_c = which == 0 ? bias : nullptr;
+        tp.bias_h = which == 1 ? bias : nullptr;
+        tp.entries = which == 0 ? entries : nullptr;
+        tp.entry_keys = entry_keys;
+        tp.hca_entries = which == 1 ? entries : nullptr;
+        tp.status = st;
+        e = launch_compress_tiles(tp, max_entries, stream);
+    } else {
+        CompressParams p{};
+        p.seqs = seqs;
+        p.ranges = ranges;
+        p.B = B;
+        p.which = which;
+        p.d = dims->d;
+        p.d_I = dims->d_I;
+        p.m = which ? dims->m_hca : dims->m;
+        p.win = which ? dims->m_hca : 2 * dims->m;
+        p.x = x;
+        p.logit = logit;
+        p.bias = bias;
+        p.idx_key = idx_key;
+        p.entries = entries;
+        p.entry_keys = entry_keys;
+        p.status = st;
+        e = launch_compress(p, max_entries, stream);
+    }
     return e == cudaSuccess ? CSA_OK : cuda_fail(e, "compress launch");
+}
+
+// Both caches for token ranges (one pass over the raw rows when both ratios have the block form).
+static int compress_all(const csa_dims& d, const csa_seq* seqs, const int64_t* tok_ranges, int64_t t0, int64_t t1,
+                        int B, int64_t max_tokens, const csa_bf16* x, const csa_bf16* logit_c,
+                        const csa_bf16* logit_h, const float* bias_c, const float* bias_h, const csa_bf16* idx_key,
+                        csa_bf16* entries, csa_bf16* entry_keys, csa_bf16* hca_entries, int* st,
+                        cudaStream_t stream) {
+    const bool csa_blk = csa_block_shape(d.m), hca_blk = hca_block_shape(d.m_hca);
+    TileCompressParams tp{};
+    tp.seqs = seqs;
+    tp.ranges = tok_ranges;
+    tp.range_begin = t0;
+    tp.range_end = t1;
+    tp.range_kind = 2;
+    tp.B = B;
+    tp.d = d.d;
+    tp.d_I = d.d_I;
+    tp.m_hca = d.m_hca;
+    tp.do_csa = csa_blk;
+    tp.do_hca = hca_blk;
+    tp.do_keys = 1;
+    tp.x = x;
+    tp.logit_c = logit_c;
+    tp.logit_h = logit_h;
+    tp.idx_key = idx_key;
+    tp.bias_c = bias_c;
+    tp.bias_h = bias_h;
+    tp.entries = entries;
+    tp.entry_keys = entry_keys;
+    tp.hca_entries = hca_entries;
+    tp.status = st;
+    cudaError_t e = launch_compress_tiles(tp, max_tokens, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "compress launch");
+    for (int which = 0; which < 2; ++which) {
+        if (which == 0 ? csa_blk : hca_blk) continue;
+        const int m = which ? d.m_hca : d.m;
+        if (max_tokens / m + 1 <= 0) continue;
+        CompressParams p{};
+        p.seqs = seqs;
+        p.ranges = tok_ranges;
+        p.range_begin = t0;
+        p.range_end = t1;
+        p.token_ranges = 1;
+        p.B = B;
+        p.which = which;
+        p.d = d.d;
+        p.d_I = d.d_I;
+        p.m = m;
+        p.win = which ? d.m_hca : 2 * d.m;
+        p.x = x;
+        p.logit = which ? logit_h : logit_c;
+        p.bias = which ? bias_h : bias_c;
+        p.idx_key = which ? nullptr : idx_key;
+        p.entries = which ? hca_entries : entries;
+        p.entry_keys = which ? nullptr : entry_keys;
+        p.status = st;
+        if ((e = launch_compress(p, max_tokens / m + 1, stream)) != cudaSuccess) return cuda_fail(e, "compress launch");
+    }
+    return CSA_OK;
+}
+
+int csa_compress_all(const csa_dims* dims, const csa_seq* seqs, const int64_t* tok_ranges, int B, int64_t max_tokens,
+                     const csa_bf16* x, const csa_bf16* logit_c, const csa_bf16* logit_h, const float* bias_c,
+                     const float* bias_h, const csa_bf16* idx_key, csa_bf16* entries, csa_bf16* entry_keys,
+                     csa_bf16* hca_entries, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !tok_ranges || !x || !logit_c || !logit_h || !bias_c || !bias_h || !idx_key || !entries ||
+        !entry_keys || !hca_entries)
+        return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (B < 1 || max_tokens < 0) return fail(CSA_ERR_ARG, "B = %d, max_tokens = %lld", B, (long long)max_tokens);
+    if (!aligned16(x) || !aligned16(logit_c) || !aligned16(logit_h) || !aligned16(bias_c) || !aligned16(bias_h) ||
+        !aligned16(idx_key) || !aligned16(entries) || !aligned16(entry_keys) || !aligned16(hca_entries))
+        return fail(CSA_ERR_ARG, "tensors must be 16-byte aligned");
+    if (max_tokens == 0) return CSA_OK;
+    int* st = nullptr;
+    if ((rc = status_ptr(&st))) return rc;
+    return compress_all(*dims, seqs, tok_ranges, 0, 0, B, max_tokens, x, logit_c, logit_h, bias_c, bias_h, idx_key,
+                        entries, entry_keys, hca_entries, st, stream);
 }
 
 size_t csa_workspace_size(int op, const void* args) {
@@ -634,36 +778,10 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
     if ((rc = status_ptr(&st))) return rc;
     cudaError_t e;
     if (a->compress) {
-        CompressParams cp{};
-        cp.seqs = a->seq;
-        cp.ranges = nullptr;
-        cp.B = 1;
-        cp.d = d.d;
-        cp.d_I = d.d_I;
-        cp.x = a->x;
-        cp.status = st;
-        cp.which = 0;
-        cp.m = d.m;
-        cp.win = 2 * d.m;
-        cp.range_begin = 0;
-        cp.range_end = a->q_end / d.m;
-        cp.logit = a->logit_c;
-        cp.bias = a->bias_c;
-        cp.idx_key = a->idx_key;
-        cp.entries = a->entries;
-        cp.entry_keys = a->entry_keys;
-        if ((e = launch_compress(cp, cp.range_end, stream)) != cudaSuccess) return cuda_fail(e, "compress launch");
-        cp.which = 1;
-        cp.m = d.m_hca;
-        cp.win = d.m_hca;
-        cp.range_end = a->q_end / d.m_hca;
-        cp.logit = a->logit_h;
-        cp.bias = a->bias_h;
-        cp.idx_key = nullptr;
-        cp.entries = a->hca_entries;
-        cp.entry_keys = nullptr;
-        if (cp.range_end > 0 && (e = launch_compress(cp, cp.range_end, stream)) != cudaSuccess)
-            return cuda_fail(e, "compress launch");
+        // every CSA and HCA entry complete in [0, q_end): one pass over the raw rows
+        rc = compress_all(d, a->seq, nullptr, 0, a->q_end, 1, a->q_end, a->x, a->logit_c, a->logit_h, a->bias_c,
+                          a->bias_h, a->idx_key, a->entries, a->entry_keys, a->hca_entries, st, stream);
+        if (rc) return rc;
     }
     char* w = static_cast<char*>(ws);
     csa_query* queries = reinterpret_cast<csa_query*>(w + pl.off_queries);
@@ -739,8 +857,8 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
 namespace csa {
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
-    append_kernel<<<p.B, 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    const unsigned ns = (unsigned)(p.d / 64);
+    return launch_kernel_cluster(append_kernel, dim3(ns, (unsigned)p.B), dim3(256), 0, stream, false, dim3(ns, 1, 1), p);
 }
 
 cudaError_t launch_prefill_queries(csa_query* queries, int64_t p0, int64_t n, cudaStream_t stream) {

@@ -102,6 +102,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void* src, ui
         : "memory");
 }
 
+// Barrier of every thread of every CTA in the thread-block cluster; orders all earlier memory
+// accesses (shared, distributed shared and global) before all later ones at cluster scope.
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------------------------
 // cp.async (16-byte, L2-only); src_bytes = 0 writes zeros without reading.
 // ---------------------------------------------------------------------------------------------

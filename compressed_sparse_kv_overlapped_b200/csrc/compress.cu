@@ -1,4 +1,4 @@
-// compress.cu -- a1/a2: the token-axis softmax compressor, full-pass kernel.
+// compress.cu -- a1/a2: the token-axis softmax compressor, full-pass kernels.
 //
 // "DeepSeek V4 comprimeix el context: aixi funcionen CSA i HCA", sections "DeepSeek comprimeix la
 // dimensio temporal" (an entry is a softmax-weighted sum of the tokens it summarises, with a
@@ -6,12 +6,22 @@
 // (overlapping windows, weights recomputed per window); "Frontier Techniques: NTK RoPE, CSA+HCA,
 // QAT, MTP", 2.1 (m = 4) and 2.2 (m' = 128).
 //
-// HBM-bound streaming: every thread owns 8 consecutive channels (one 16-byte vector) of one entry
-// and runs an online softmax over the window in fp32 (compress_dev.cuh), so each token row is
-// read with coalesced 16-byte loads and the overlapping CSA windows re-read their shared rows from
-// L1/L2.
+// compress_tile_kernel (CSA ratio 4, HCA ratio a power of two up to 128): one CTA per (128-token
+// tile, sequence, 64-channel slice).  One thread issues four TMA boxes of 132 rows (the tile plus
+// the 4-token halo the first CSA window reaches back to) of the latent, both logit arrays and the
+// indexer keys into shared memory, so every token row is read from HBM once for both caches.
+// Thread (u, g) (u = 4-token block 0..31, g = 8-channel group 0..7) then builds CSA entry 32*tile + u
+// from the two 4-token softmax partials of its window and the partial of block u for HCA, whose
+// entries are merged by the block tree of compress_dev.cuh.  Entries are stored as bf16 with 16-byte
+// stores.  The window arithmetic is shared with the decode append (identical entries).
+//
+// compress_kernel (other ratios): one thread per 8 channels of one entry, an online softmax over
+// the window read with coalesced 16-byte loads.
+#include <cstring>
+
 #include "compress_dev.cuh"
 #include "kernels.h"
+#include "tma.h"
 
 namespace csa {
 
@@ -20,9 +30,10 @@ namespace {
 __global__ void __launch_bounds__(256) compress_kernel(CompressParams p) {
     const int b = blockIdx.y;
     const csa_seq sq = p.seqs[b];
-    const int64_t e0 = p.ranges ? p.ranges[2 * b] : p.range_begin;
-    const int64_t e1 = p.ranges ? p.ranges[2 * b + 1] : p.range_end;
-    if (e0 < 0 || e1 < e0 || (int64_t)p.m * e1 > sq.len) {
+    const int64_t r0 = p.ranges ? p.ranges[2 * b] : p.range_begin;
+    const int64_t r1 = p.ranges ? p.ranges[2 * b + 1] : p.range_end;
+    const int64_t e0 = p.token_ranges ? r0 / p.m : r0, e1 = p.token_ranges ? r1 / p.m : r1;
+    if (r0 < 0 || r1 < r0 || (int64_t)p.m * e1 > sq.len || (p.token_ranges && r1 > sq.len)) {
         if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, CSA_ERR_INDEX);
         return;
     }
@@ -38,6 +49,134 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressParams p) {
     }
 }
 
+constexpr int kTileTok = 128;                  // tokens per tile: one 128-token HCA block, 32 CSA entries
+static_assert(hca_block_shape(kTileTok) && !hca_block_shape(2 * kTileTok), "HCA blocks divide a tile");
+constexpr int kHalo = 4;                       // the previous CSA block (window of the tile's first entry)
+constexpr int kBoxRows = kTileTok + kHalo;     // rows of every TMA box
+constexpr int kSlice = 64;                     // channels per CTA
+constexpr int kBoxBytes = kBoxRows * kSlice * 2;
+
+struct TileMaps {
+    CUtensorMap x, lc, lh, ki;
+};
+
+struct TileSmem {
+    static constexpr int kX = 0;
+    static constexpr int kLc = kX + kBoxBytes;
+    static constexpr int kLh = kLc + kBoxBytes;
+    static constexpr int kKi = kLh + kBoxBytes;       // d_I * 2 bytes per row (at most 128)
+    static constexpr int kXs = kKi + kBoxBytes;       // HCA tree exchange: 8 warps x 8 groups x 24 floats
+    static constexpr int kBar = kXs + 8 * 8 * 24 * 4;
+    static constexpr int kTotal = kBar + 16;
+    static constexpr int kAlloc = kTotal + 128;       // slack for 128-byte alignment
+};
+
+__global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_constant__ TileMaps maps,
+                                                                TileCompressParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + TileSmem::kBar);
+    float* xs = reinterpret_cast<float*>(sm + TileSmem::kXs);
+    const int b = blockIdx.y, slice = blockIdx.z;
+    const int tid = threadIdx.x, u = tid >> 3, g = tid & 7;
+    const csa_seq sq = p.seqs[b];
+    const int64_t r0 = p.ranges ? p.ranges[2 * b] : p.range_begin;
+    const int64_t r1 = p.ranges ? p.ranges[2 * b + 1] : p.range_end;
+    // the entries this call writes for sequence b: CSA [cj0, cj1), HCA [hh0, hh1)
+    int64_t cj0 = 0, cj1 = 0, hh0 = 0, hh1 = 0, t_first;
+    const int mh = p.m_hca;
+    if (p.range_kind == 0) {
+        cj0 = r0; cj1 = r1; t_first = 4 * r0;
+    } else if (p.range_kind == 1) {
+        hh0 = r0; hh1 = r1; t_first = mh * r0;
+    } else {
+        if (p.do_csa) { cj0 = r0 / 4; cj1 = r1 / 4; }
+        if (p.do_hca) { hh0 = r0 / mh; hh1 = r1 / mh; }
+        t_first = r0;
+    }
+    if (r0 < 0 || r1 < r0 || 4 * cj1 > sq.len || (int64_t)mh * hh1 > sq.len || (p.range_kind == 2 && r1 > sq.len) ||
+        sq.tok_off + t_first + (int64_t)kTileTok * gridDim.x + kBoxRows > 0x7FFFFFFF) {
+        if (tid == 0 && blockIdx.x == 0 && slice == 0) report(p.status, CSA_ERR_INDEX);
+        return;
+    }
+    const int64_t tile = t_first / kTileTok + blockIdx.x;
+    const int64_t tt0 = tile * kTileTok;  // first token of the tile
+    // this tile's share
+    const int64_t c_lo = max(cj0, tt0 / 4), c_hi = min(cj1, (tt0 + kTileTok) / 4);
+    const int64_t h_lo = max(hh0, tt0 / mh), h_hi = min(hh1, (tt0 + kTileTok) / mh);
+    const bool csa = p.do_csa && c_lo < c_hi;
+    const bool hca = p.do_hca && h_lo < h_hi;
+    if (!csa && !hca) return;
+    // rows [box0, box0 + kBoxRows) of the sequence cover every token the tile's entries use and end at
+    // the last token used, so no row past the sequence's valid rows is read (negative rows read 0)
+    const int64_t t_hi = max(csa ? 4 * c_hi : 0, hca ? (int64_t)mh * h_hi : 0);
+    int64_t box0 = tt0 - kHalo;
+    if (box0 + kBoxRows > t_hi) box0 = t_hi - kBoxRows;
+    const bool keys = csa && p.do_keys && slice * kSlice < p.d_I;
+    const int d = p.d;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        const uint32_t bytes = (uint32_t)kBoxBytes * (1u + (csa ? 1u : 0u) + (hca ? 1u : 0u)) +
+                               (keys ? (uint32_t)(kBoxRows * p.d_I * 2) : 0u);
+        mbar_arrive_expect_tx(bar, bytes);
+        const int y = (int)(sq.tok_off + box0);
+        const uint32_t s0 = smem_u32(sm);
+        tma_load_2d(s0 + TileSmem::kX, &maps.x, slice * kSlice, y, bar);
+        if (csa) tma_load_2d(s0 + TileSmem::kLc, &maps.lc, slice * kSlice, y, bar);
+        if (hca) tma_load_2d(s0 + TileSmem::kLh, &maps.lh, slice * kSlice, y, bar);
+        if (keys) tma_load_2d(s0 + TileSmem::kKi, &maps.ki, 0, y, bar);
+    }
+    __syncthreads();
+    // the outcome is made CTA-uniform, so a timeout (recorded; nothing is written) never leaves some
+    // threads at a barrier below without the others
+    if (!__syncthreads_and(mbar_wait(bar, 0, p.status, nullptr) ? 1 : 0)) return;
+
+    const uint16_t* sx = reinterpret_cast<const uint16_t*>(sm + TileSmem::kX);
+    const uint16_t* slc = reinterpret_cast<const uint16_t*>(sm + TileSmem::kLc);
+    const uint16_t* slh = reinterpret_cast<const uint16_t*>(sm + TileSmem::kLh);
+    const uint16_t* ski = reinterpret_cast<const uint16_t*>(sm + TileSmem::kKi);
+    const int c0 = slice * kSlice + g * 8;  // this thread's first channel
+
+    if (csa) {
+        const int64_t j = tt0 / 4 + u;
+        if (j >= c_lo && j < c_hi) {
+            const int rbase = (int)(4 * j - 4 - box0);  // smem row of window position 0
+            auto fetch = [&](int tensor, int pos) -> uint4 {
+                const int r = rbase + pos;
+                const uint16_t* base = tensor == 0 ? slc : tensor == 1 ? sx : ski;
+                const int stride = tensor == 2 ? p.d_I : kSlice;
+                return *reinterpret_cast<const uint4*>(base + r * stride + g * 8);
+            };
+            uint16_t* orow = p.entries + (sq.csa_off + j) * d + c0;
+            if (keys && c0 < p.d_I)
+                csa_entry_block4<true>(j, d, p.bias_c + c0, fetch, orow, p.entry_keys + (sq.csa_off + j) * p.d_I + c0);
+            else
+                csa_entry_block4<false>(j, d, p.bias_c + c0, fetch, orow, nullptr);
+        }
+    }
+    if (hca) {
+        const int nb = mh / 4;  // blocks per HCA entry
+        // block u's 4 tokens; blocks past the loaded rows belong to no entry this tile writes
+        int r = (int)(tt0 + 4 * u - box0);
+        if (r < 0 || r + 4 > kBoxRows) r = 0;
+        uint4 lg[4], xv[4], kv[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            lg[t] = *reinterpret_cast<const uint4*>(slh + (r + t) * kSlice + g * 8);
+            xv[t] = *reinterpret_cast<const uint4*>(sx + (r + t) * kSlice + g * 8);
+            kv[t] = make_uint4(0, 0, 0, 0);
+        }
+        Part8 P;
+        part4<false>(lg, xv, kv, p.bias_h + (int64_t)((4 * u) & (mh - 1)) * d + c0, d, P);
+        hca_tree(P, nb, xs);
+        const int64_t h = (tt0 + 4 * u) / mh;
+        const bool holder = (u & (nb - 1)) == 0 && (nb < 8 || (tid & 31) < 8);
+        if (holder && h >= h_lo && h < h_hi)
+            *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) = finish8(P.acc, P.den);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_compress(const CompressParams& p, int64_t max_entries, cudaStream_t stream) {
@@ -48,6 +187,37 @@ cudaError_t launch_compress(const CompressParams& p, int64_t max_entries, cudaSt
     if (gx > 8192) gx = 8192;
     compress_kernel<<<dim3((unsigned)gx, (unsigned)p.B), 256, 0, stream>>>(p);
     return cudaGetLastError();
+}
+
+cudaError_t launch_compress_tiles(const TileCompressParams& p, int64_t max_span, cudaStream_t stream) {
+    if (max_span <= 0 || (!p.do_csa && !p.do_hca)) return cudaSuccess;
+    if (p.d % kSlice != 0 || (p.d_I != 32 && p.d_I != 64) || (p.do_hca && !hca_block_shape(p.m_hca)))
+        return cudaErrorInvalidValue;
+    static PerDeviceOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(compress_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    TileSmem::kAlloc);
+    });
+    if (e != cudaSuccess) return e;
+    // tensor maps over the raw arrays; boxes of 132 rows x 64 channels (the indexer keys: all d_I
+    // channels), no swizzle.  The row extent is left open: the kernel starts every box inside the
+    // sequence's valid rows or before row 0, where the box reads zeros.
+    TileMaps maps;
+    std::memset(&maps, 0, sizeof maps);
+    const uint64_t rows = 0x7FFFFFFFull;
+    e = tensor_map_2d_bf16(&maps.x, p.x, p.d, rows, (uint64_t)p.d * 2, kSlice, kBoxRows, false);
+    if (e == cudaSuccess && p.do_csa)
+        e = tensor_map_2d_bf16(&maps.lc, p.logit_c, p.d, rows, (uint64_t)p.d * 2, kSlice, kBoxRows, false);
+    if (e == cudaSuccess && p.do_hca)
+        e = tensor_map_2d_bf16(&maps.lh, p.logit_h, p.d, rows, (uint64_t)p.d * 2, kSlice, kBoxRows, false);
+    if (e == cudaSuccess && p.do_csa && p.do_keys)
+        e = tensor_map_2d_bf16(&maps.ki, p.idx_key, p.d_I, rows, (uint64_t)p.d_I * 2, p.d_I, kBoxRows, false);
+    if (e != cudaSuccess) return e;
+    int64_t span_tok = p.range_kind == 0 ? 4 * max_span : p.range_kind == 1 ? (int64_t)p.m_hca * max_span : max_span;
+    const int64_t tiles = (span_tok + kTileTok - 1) / kTileTok + 1;  // the range may start inside a tile
+    if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    return launch_kernel(compress_tile_kernel, dim3((unsigned)tiles, (unsigned)p.B, (unsigned)(p.d / kSlice)),
+                         dim3(256), TileSmem::kAlloc, stream, false, maps, p);
 }
 
 }  // namespace csa

@@ -93,4 +93,154 @@ __device__ __forceinline__ void compress_entry8(int64_t j, int m, int win, int d
     }
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// Block-partial form (CSA ratio m = 4, HCA ratio m' a power of two from 4 to 128).  Per channel
+// the softmax over a window is built from 4-token partials (M = max of the block's logits, den =
+// sum exp(z - M), acc = sum exp(z - M) * x), merged pairwise:
+//   CSA entry j = merge(P(tokens 4j-4..4j-1, bias rows 0..3), P(tokens 4j..4j+3, bias rows 4..7)),
+//                 entry 0 = P(tokens 0..3, bias rows 4..7) alone (its window is clipped at 0);
+//   HCA entry h = the balanced binary merge tree over its m'/4 blocks, in block order.
+// Every step uses explicitly rounded fp32 operations (no contraction the compiler may choose
+// differently in another kernel), and a merge is symmetric in its operands, so the full-pass kernel
+// and the decode append produce bit-identical entries.
+// ---------------------------------------------------------------------------------------------
+struct Part8 {
+    float M[8], den[8], acc[8], acck[8];
+};
+
+// Partial of 4 tokens: lg / xv / kv the tokens' logit / latent / indexer-key vectors (channels
+// c0..c0+7), brow the 4 bias rows (fp32, channels c0..c0+7, row stride d).  valid[t] = false drops a
+// token.  With KEYS the indexer key is accumulated with the same weights.
+template <bool KEYS>
+__device__ __forceinline__ void part4(const uint4 (&lg)[4], const uint4 (&xv)[4], const uint4 (&kv)[4],
+                                      const float* brow, int d, Part8& P) {
+    float z[4][8];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float f[8];
+        unpack8(lg[t], f);
+        const float4 b0 = __ldg(reinterpret_cast<const float4*>(brow + t * d));
+        const float4 b1 = __ldg(reinterpret_cast<const float4*>(brow + t * d) + 1);
+        z[t][0] = __fadd_rn(f[0], b0.x); z[t][1] = __fadd_rn(f[1], b0.y);
+        z[t][2] = __fadd_rn(f[2], b0.z); z[t][3] = __fadd_rn(f[3], b0.w);
+        z[t][4] = __fadd_rn(f[4], b1.x); z[t][5] = __fadd_rn(f[5], b1.y);
+        z[t][6] = __fadd_rn(f[6], b1.z); z[t][7] = __fadd_rn(f[7], b1.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) P.M[i] = fmaxf(fmaxf(z[0][i], z[1][i]), fmaxf(z[2][i], z[3][i]));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { P.den[i] = 0.f; P.acc[i] = 0.f; P.acck[i] = 0.f; }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float xf[8], kf[8];
+        unpack8(xv[t], xf);
+        if (KEYS) unpack8(kv[t], kf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float e = expf(__fsub_rn(z[t][i], P.M[i]));
+            P.den[i] = __fadd_rn(P.den[i], e);
+            P.acc[i] = __fmaf_rn(e, xf[i], P.acc[i]);
+            if (KEYS) P.acck[i] = __fmaf_rn(e, kf[i], P.acck[i]);
+        }
+    }
+}
+
+// A <- merge(A, B); symmetric in A and B bit for bit.
+template <bool KEYS>
+__device__ __forceinline__ void merge8(Part8& A, const Part8& B) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float M = fmaxf(A.M[i], B.M[i]);
+        const float fa = expf(__fsub_rn(A.M[i], M));
+        const float fb = expf(__fsub_rn(B.M[i], M));
+        A.den[i] = __fadd_rn(__fmul_rn(fa, A.den[i]), __fmul_rn(fb, B.den[i]));
+        A.acc[i] = __fadd_rn(__fmul_rn(fa, A.acc[i]), __fmul_rn(fb, B.acc[i]));
+        if (KEYS) A.acck[i] = __fadd_rn(__fmul_rn(fa, A.acck[i]), __fmul_rn(fb, B.acck[i]));
+        A.M[i] = M;
+    }
+}
+
+// acc / den, rounded to bf16 (and the key accumulator with KEYS).
+__device__ __forceinline__ uint4 finish8(const float (&acc)[8], const float (&den)[8]) {
+    uint4 o;
+    o.x = pack_bf16x2(__fdiv_rn(acc[0], den[0]), __fdiv_rn(acc[1], den[1]));
+    o.y = pack_bf16x2(__fdiv_rn(acc[2], den[2]), __fdiv_rn(acc[3], den[3]));
+    o.z = pack_bf16x2(__fdiv_rn(acc[4], den[4]), __fdiv_rn(acc[5], den[5]));
+    o.w = pack_bf16x2(__fdiv_rn(acc[6], den[6]), __fdiv_rn(acc[7], den[7]));
+    return o;
+}
+
+// Shuffle a partial from lane (lane ^ mask).
+__device__ __forceinline__ void shfl_xor8(const Part8& A, Part8& B, int mask) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        B.M[i] = __shfl_xor_sync(0xffffffffu, A.M[i], mask);
+        B.den[i] = __shfl_xor_sync(0xffffffffu, A.den[i], mask);
+        B.acc[i] = __shfl_xor_sync(0xffffffffu, A.acc[i], mask);
+    }
+}
+
+// CSA entry j (channels c0..c0+7) from the 8 rows of its window, rows fetched by fetch(tensor, t)
+// for window position t in 0..7 (tensor 0: logit, 1: latent, 2: indexer key).  j = 0 uses positions
+// 4..7 only.  Writes the entry (and, with keys, the indexer key) as bf16.
+template <bool KEYS, typename Fetch>
+__device__ __forceinline__ void csa_entry_block4(int64_t j, int d, const float* bias_c0, Fetch fetch,
+                                                 uint16_t* out_row, uint16_t* key_row) {
+    uint4 lg[4], xv[4], kv[4];
+    Part8 cur;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        lg[t] = fetch(0, 4 + t);
+        xv[t] = fetch(1, 4 + t);
+        kv[t] = KEYS ? fetch(2, 4 + t) : make_uint4(0, 0, 0, 0);
+    }
+    part4<KEYS>(lg, xv, kv, bias_c0 + 4 * d, d, cur);
+    if (j > 0) {
+        Part8 prev;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            lg[t] = fetch(0, t);
+            xv[t] = fetch(1, t);
+            kv[t] = KEYS ? fetch(2, t) : make_uint4(0, 0, 0, 0);
+        }
+        part4<KEYS>(lg, xv, kv, bias_c0, d, prev);
+        merge8<KEYS>(cur, prev);
+    }
+    *reinterpret_cast<uint4*>(out_row) = finish8(cur.acc, cur.den);
+    if (KEYS) *reinterpret_cast<uint4*>(key_row) = finish8(cur.acck, cur.den);
+}
+
+// HCA entries of one 128-token tile, channels c0..c0+7: thread (u = tid / 8, g = tid % 8) of a
+// 256-thread CTA holds the partial of tile block u (tokens 4u..4u+3) in P; the blocks of each entry
+// (nb = m'/4 of them, a power of two up to 32) are merged by the binary tree in block order: lane
+// shuffles for the two levels inside a warp (4 blocks per warp: u ^ 1 is lane ^ 8, u ^ 2 is
+// lane ^ 16), then shared memory `xs` ([8 warps][8 g][24 floats]) for the levels across warps, one
+// level per barrier.  Every thread of the CTA must call it (it contains barriers when nb >= 8).  On
+// return lanes 0..7 of the first warp of each entry hold the merged partial in P.
+__device__ __forceinline__ void hca_tree(Part8& P, int nb, float* xs) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    Part8 Q;
+    if (nb >= 2) { shfl_xor8(P, Q, 8); merge8<false>(P, Q); }
+    if (nb >= 4) { shfl_xor8(P, Q, 16); merge8<false>(P, Q); }
+    if (nb < 8) return;
+    const int wpe = nb / 4;  // warps per entry: 2, 4 or 8
+    float* mine = xs + (warp * 8 + (lane & 7)) * 24;
+    if (lane < 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { mine[i] = P.M[i]; mine[8 + i] = P.den[i]; mine[16 + i] = P.acc[i]; }
+    }
+    for (int step = 1; step < wpe; step *= 2) {
+        __syncthreads();
+        if (lane < 8 && (warp & (2 * step - 1)) == 0) {
+            const float* other = xs + ((warp + step) * 8 + lane) * 24;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { Q.M[i] = other[i]; Q.den[i] = other[8 + i]; Q.acc[i] = other[16 + i]; }
+            merge8<false>(P, Q);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { mine[i] = P.M[i]; mine[8 + i] = P.den[i]; mine[16 + i] = P.acc[i]; }
+        }
+    }
+}
+
 }  // namespace csa

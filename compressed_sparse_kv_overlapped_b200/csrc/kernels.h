@@ -12,6 +12,7 @@ struct CompressParams {
     const csa_seq* seqs;
     const int64_t* ranges;   // [B][2], or nullptr: every sequence uses [range_begin, range_end)
     int64_t range_begin, range_end;
+    int token_ranges;        // 1: the ranges are token ranges [t0, t1): entries [t0/m, t1/m)
     int B;
     int which;               // 0 CSA, 1 HCA
     int d, d_I, m, win;
@@ -24,6 +25,36 @@ struct CompressParams {
     int* status;
 };
 cudaError_t launch_compress(const CompressParams& p, int64_t max_entries, cudaStream_t stream);
+
+// Block-partial compressor (compress_dev.cuh) over 128-token tiles staged by TMA: one CTA per
+// (tile, sequence, 64-channel slice) computes the tile's CSA entries (with indexer keys) and HCA
+// entries from one read of each token row.  Shapes: CSA ratio 4; HCA ratio a power of two from 4 to
+// 128; d a multiple of 64; d_I 32 or 64.  The decode append uses the same arithmetic for the same
+// shapes, so both produce identical entries.
+__host__ __device__ constexpr bool csa_block_shape(int m) { return m == 4; }  // CSA by the block-partial form
+__host__ __device__ constexpr bool hca_block_shape(int m_hca) {             // HCA by the block-partial form
+    return m_hca >= 4 && m_hca <= 128 && (m_hca & (m_hca - 1)) == 0;
+}
+struct TileCompressParams {
+    const csa_seq* seqs;
+    const int64_t* ranges;    // [B][2] or nullptr: every sequence uses [range_begin, range_end)
+    int64_t range_begin, range_end;
+    int range_kind;           // 0: CSA entry range, 1: HCA entry range, 2: token range (both caches)
+    int B, d, d_I, m_hca;
+    int do_csa, do_hca, do_keys;
+    const uint16_t* x;
+    const uint16_t* logit_c;
+    const uint16_t* logit_h;
+    const uint16_t* idx_key;
+    const float* bias_c;
+    const float* bias_h;
+    uint16_t* entries;
+    uint16_t* entry_keys;
+    uint16_t* hca_entries;
+    int* status;
+};
+// max_span: host bound of each sequence's range length, in the range's own units.
+cudaError_t launch_compress_tiles(const TileCompressParams& p, int64_t max_span, cudaStream_t stream);
 
 // Indexer score scan + top-k select.
 constexpr int kHistBins = 2048;  // coarse histogram over the top 11 bits of the score key
@@ -136,6 +167,7 @@ cudaError_t launch_attention_items(const AttnParams& p, int item_begin, int item
 cudaError_t launch_combine(const AttnParams& p, cudaStream_t stream, bool pdl = false);
 
 // Decode helper: append one token per sequence, compress completed entries, build the query table.
+// One thread-block cluster of d/64 CTAs per sequence; CTA s owns channels [64s, 64s + 64).
 struct AppendParams {
     csa_seq* seqs;
     int B, append;

@@ -29,10 +29,10 @@ __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
 }
 
 // A 2-D bf16 tensor map over `rows` rows of `inner` elements (row pitch `pitch_bytes`), box of
-// box_inner x box_rows elements, 128-byte swizzle; cached per (base, inner, rows, pitch, box).
-// Returns cudaSuccess, or an error when the driver entry point is missing or the encoding is
-// rejected (callers then load without TMA).
+// box_inner x box_rows elements, with the 128-byte swizzle (swizzle128) or none; cached per
+// (base, inner, rows, pitch, box, swizzle).  Returns cudaSuccess, or an error when the driver entry
+// point is missing or the encoding is rejected.
 cudaError_t tensor_map_2d_bf16(CUtensorMap* out, const void* base, uint64_t inner, uint64_t rows,
-                               uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows);
+                               uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows, bool swizzle128 = true);
 
 }  // namespace csa

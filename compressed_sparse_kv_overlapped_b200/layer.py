@@ -15,8 +15,8 @@ The caller fills the raw-token rows (and the parameters); ``compress`` builds th
 """
 from __future__ import annotations
 
-from . import (CSA_OP_DECODE, CSA_OP_PREFILL, csa_compress, csa_decode_args, csa_prefill_args, csa_workspace_size,
-               hybrid_attn_decode, hybrid_attn_prefill)
+from . import (CSA_OP_DECODE, CSA_OP_PREFILL, csa_compress, csa_compress_all, csa_decode_args, csa_prefill_args,
+               csa_workspace_size, hybrid_attn_decode, hybrid_attn_prefill)
 
 
 class HybridLayer:
@@ -61,7 +61,18 @@ class HybridLayer:
 
     # ---- compressor full pass -----------------------------------------------------------------
     def compress(self, stream=None) -> None:
-        """(Re)build every complete CSA and HCA entry of every sequence from the raw tokens."""
+        """(Re)build every complete CSA and HCA entry of every sequence from the raw tokens (one pass
+        over the raw rows for both caches, csa_compress_all)."""
+        import torch
+        rt = torch.tensor([[0, n] for n in self.lens], dtype=torch.int64, device=self.device)
+        if max(self.lens) > 0:
+            csa_compress_all(self.dims, self.seqs, rt, self.B, max(self.lens), self.x, self.logit_c, self.logit_h,
+                             self.bias_c, self.bias_h, self.idx_key, self.entries, self.entry_keys,
+                             self.hca_entries, stream)
+        self._keep = rt  # the kernels read the range table asynchronously
+
+    def compress_separately(self, stream=None) -> None:
+        """The same caches through two csa_compress calls (CSA entries with their keys, then HCA)."""
         import torch
         d = self.dims
         rc = torch.tensor([[0, n // d.m] for n in self.lens], dtype=torch.int64, device=self.device)
@@ -71,7 +82,7 @@ class HybridLayer:
         if max(n // d.m_hca for n in self.lens) > 0:
             csa_compress(d, 1, self.seqs, rh, self.B, max(n // d.m_hca for n in self.lens), self.x, self.logit_h,
                          self.bias_h, None, self.hca_entries, None, stream)
-        self._keep = (rc, rh)  # the kernels read the range tables asynchronously
+        self._keep2 = (rc, rh)
 
     # ---- decode -------------------------------------------------------------------------------
     def decode_args(self, q, q_idx, w, out, append=True, lse=None, idx_out=None, max_len=None,

@@ -109,6 +109,21 @@ int csa_compress(const csa_dims* dims, int which, const csa_seq* seqs, const int
                  int64_t max_entries, const csa_bf16* x, const csa_bf16* logit, const float* bias,
                  const csa_bf16* idx_key, csa_bf16* entries, csa_bf16* entry_keys, csa_stream_t stream);
 
+/* a1 + a2 in one pass -- both caches for token ranges ("DeepSeek V4 comprimeix el context", sections
+ * "DeepSeek comprimeix la dimensio temporal" and "Finestres solapades per evitar fronteres
+ * artificials"; "HCA: un resum global 128 vegades mes curt"; "Frontier Techniques", 2.1 and 2.2).
+ * For sequence b with tok_ranges[b] = [t0, t1) (device int64 [B][2], t1 <= seqs[b].len): every CSA
+ * entry j in [t0/m, t1/m) with its indexer key, and every HCA entry in [t0/m_hca, t1/m_hca), i.e. the
+ * entries whose last token lies in [t0, t1).  With m = 4 and m_hca a power of two from 4 to 128 each
+ * raw row (x, both logit arrays, idx_key) is read once for both caches; other ratios run the two
+ * caches one after the other.  max_tokens: host bound of t1 - t0 over the sequences (sizes the
+ * grid).  Entries equal those of csa_compress and of the decode append bit for bit.  A range outside
+ * [0, seqs[b].len] is reported as CSA_ERR_INDEX on the device. */
+int csa_compress_all(const csa_dims* dims, const csa_seq* seqs, const int64_t* tok_ranges, int B, int64_t max_tokens,
+                     const csa_bf16* x, const csa_bf16* logit_c, const csa_bf16* logit_h, const float* bias_c,
+                     const float* bias_h, const csa_bf16* idx_key, csa_bf16* entries, csa_bf16* entry_keys,
+                     csa_bf16* hca_entries, csa_stream_t stream);
+
 /* a3/a4 -- Lightning-Indexer scores and top-k ("Frontier Techniques", 2.1; "DeepSeek V4
  * comprimeix el context", "CSA: buscar primer i atendre despres").  For query i at length L:
  * s_j = sum_h w[i][h] * relu(q_idx[i][h] . entry_keys[csa_off + j]) over j < floor(L/m); the k

@@ -54,6 +54,11 @@ def lib() -> ctypes.CDLL:
         L.oracle_hca_attn.argtypes = [vp, ci, ci, vp, ci, vp, i64, ci, cd, vp, vp]
         L.oracle_hca_attn.restype = ci
         L.oracle_lse_merge.argtypes = [vp, vp, vp, vp, ci, ci, vp, vp]
+        L.oracle_e4m3_round.argtypes = [vp, i64, vp]
+        L.oracle_e4m3_value.argtypes = [vp, i64, vp]
+        L.oracle_quantize_keys_mx8.argtypes = [vp, i64, ci, vp, vp]
+        L.oracle_quantize_keys_mx8.restype = ci
+        L.oracle_index_scores_mx8.argtypes = [vp, vp, ci, ci, vp, vp, i64, vp]
         _lib = L
     return _lib
 
@@ -139,6 +144,44 @@ def index_scores(qI, w, KI) -> np.ndarray:
     H_I, d_I = qI.shape
     s = np.empty(KI.shape[0], dtype=np.float64)
     lib().oracle_index_scores(_p(qI), _p(w), H_I, d_I, _p(KI), KI.shape[0], _p(s))
+    return s
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Doubles with |v| <= 448 to the nearest FP8 E4M3 value (ties to even), as bit patterns."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_round(_p(v), v.size, _p(out))
+    return out
+
+
+def e4m3_value(b) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    out = np.empty(b.shape, dtype=np.float64)
+    lib().oracle_e4m3_value(_p(b), b.size, _p(out))
+    return out
+
+
+def quantize_keys_mx8(KI):
+    """bf16 key rows [n, d_I] -> (E4M3 bytes [n, d_I], biased power-of-two scales [n, d_I / 32])."""
+    KI = _u16(KI)
+    n, d_I = KI.shape
+    Kq = np.empty((n, d_I), dtype=np.uint8)
+    sc = np.empty((n, d_I // 32), dtype=np.uint8)
+    if lib().oracle_quantize_keys_mx8(_p(KI), n, d_I, _p(Kq), _p(sc)) != 0:
+        raise ValueError("d_I must be a multiple of 32")
+    return Kq, sc
+
+
+def index_scores_mx8(qI, w, Kq, scales) -> np.ndarray:
+    """Indexer scores of the dequantized 8-bit keys (fp64)."""
+    qI = _u16(qI)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    Kq = np.ascontiguousarray(Kq, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    H_I, d_I = qI.shape
+    s = np.empty(Kq.shape[0], dtype=np.float64)
+    lib().oracle_index_scores_mx8(_p(qI), _p(w), H_I, d_I, _p(Kq), _p(scales), Kq.shape[0], _p(s))
     return s
 
 

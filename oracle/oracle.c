@@ -325,3 +325,109 @@ void oracle_lse_merge(const double* O1, const double* lse1, const double* O2, co
         lse[h] = l;
     }
 }
+
+/* ---- f1: 8-bit block-scaled indexer keys --------------------------------- */
+/*
+ * "Frontier Techniques: NTK RoPE, CSA+HCA, QAT, MTP", section 3 (DeepSeek V4 quantizes the
+ * indexer's QK path to a 4-bit block-scaled format) and "Compressed attention . CSA / HCA va hai
+ * truc nen", sections 3 and 4 (quantized caches carry block scales; the scale bytes count).  The
+ * pages fix neither the element format nor the block, so this is a reading in the same family
+ * (MX-style, 8-bit elements): the indexer keys of an entry are cut into blocks of 32 consecutive
+ * channels; a block shares one power-of-two scale 2^e, stored as the byte e + 127; its elements
+ * are FP8 E4M3 numbers (exponent bias 7, largest 448, subnormal step 2^-9).  e is the smallest
+ * integer with amax <= 448 * 2^e (amax = the block's largest magnitude; a zero block takes
+ * e = -127), and each element is x / 2^e rounded to the nearest E4M3 value, ties to even.  Only the
+ * keys are quantized; the indexer queries stay bf16, and the score is the plain score of the
+ * dequantized keys, element = 2^e * E4M3 value.
+ */
+
+/* Round |v| <= 448 to the nearest E4M3 value (ties to even). */
+static double e4m3_round(double v) {
+    double a = fabs(v);
+    if (a == 0.0) return v;
+    double q;
+    if (a < ldexp(1.0, -6)) {               /* subnormal grid: steps of 2^-9 */
+        q = rint(a / ldexp(1.0, -9)) * ldexp(1.0, -9);
+    } else {
+        int y;
+        frexp(a, &y);                        /* a in [2^(y-1), 2^y) */
+        double step = ldexp(1.0, y - 1 - 3); /* 3 mantissa bits */
+        q = rint(a / step) * step;
+    }
+    return v < 0 ? -q : q;
+}
+
+/* The E4M3 bit pattern of a value on the E4M3 grid (|v| <= 448). */
+static uint8_t e4m3_bits(double v) {
+    uint8_t s = signbit(v) ? 0x80 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return s;
+    if (a < ldexp(1.0, -6)) return (uint8_t)(s | (uint8_t)(a / ldexp(1.0, -9)));
+    int y;
+    double g = frexp(a, &y);                 /* a = g 2^y, g in [0.5, 1) */
+    int E = y - 1 + 7;
+    int m = (int)((2.0 * g - 1.0) * 8.0);
+    return (uint8_t)(s | (E << 3) | m);
+}
+
+static double e4m3_value(uint8_t b) {
+    int E = (b >> 3) & 15, m = b & 7;
+    double a = E == 0 ? m * ldexp(1.0, -9) : ldexp(1.0 + m / 8.0, E - 7);
+    return (b & 0x80) ? -a : a;
+}
+
+void oracle_e4m3_round(const double* in, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_bits(e4m3_round(in[i]));
+}
+
+void oracle_e4m3_value(const uint8_t* in, int64_t n, double* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(in[i]);
+}
+
+/* Quantize n bf16 key rows [n, d_I] (d_I a multiple of 32) to Kq [n, d_I] E4M3 bytes and
+ * scales [n, d_I / 32] biased exponents. */
+int oracle_quantize_keys_mx8(const uint16_t* K, int64_t n, int d_I, uint8_t* Kq, uint8_t* scales) {
+    if (d_I % 32) return -2;
+    int nb = d_I / 32;
+    for (int64_t j = 0; j < n; ++j) {
+        for (int b = 0; b < nb; ++b) {
+            const uint16_t* x = K + j * d_I + 32 * b;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs(bf16_to_double(x[i]));
+                if (a > amax) amax = a;
+            }
+            int e = -127;
+            if (amax > 0.0) {
+                int y;
+                frexp(amax, &y);
+                e = y - 9;                                    /* a start near the answer (amax < 2^y) */
+                while (amax > ldexp(448.0, e)) ++e;           /* smallest e with amax <= 448 * 2^e */
+                while (e > -127 && amax <= ldexp(448.0, e - 1)) --e;
+            }
+            scales[j * nb + b] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; ++i)
+                Kq[j * d_I + 32 * b + i] = e4m3_bits(e4m3_round(ldexp(bf16_to_double(x[i]), -e)));
+        }
+    }
+    return 0;
+}
+
+/* a3 with 8-bit keys: s_j = sum_h w_h * relu(qI_h . K_j) with K_j the dequantized key
+ * (element 2^e * E4M3 value), everything in double. */
+void oracle_index_scores_mx8(const uint16_t* qI, const float* w, int H_I, int d_I, const uint8_t* Kq,
+                             const uint8_t* scales, int64_t n_entries, double* s) {
+    int nb = d_I / 32;
+    for (int64_t j = 0; j < n_entries; ++j) {
+        double acc = 0.0;
+        for (int h = 0; h < H_I; ++h) {
+            double dot = 0.0;
+            for (int c = 0; c < d_I; ++c) {
+                double k = ldexp(e4m3_value(Kq[j * d_I + c]), (int)scales[j * nb + c / 32] - 127);
+                dot += bf16_to_double(qI[h * d_I + c]) * k;
+            }
+            acc += (double)w[h] * (dot > 0.0 ? dot : 0.0);
+        }
+        s[j] = acc;
+    }
+}

@@ -89,6 +89,101 @@ def test_incremental_append_equals_full_pass():
     assert layer.seqs[:, 3].tolist() == [n + wl.steps for n in wl.n0]
 
 
+# Ratios on both sides of the block form (CSA m = 4, HCA m' a power of two from 4 to 128) and of the
+# per-entry serial form used otherwise.
+_SHAPES = {
+    "m4_h128": workloads.Dims(d=512, H=64, d_I=64, H_I=4, m=4, m_hca=128, k=64, W=16),
+    "m4_h8_d128": workloads.Dims(d=128, H=8, d_I=32, H_I=4, m=4, m_hca=8, k=32, W=16),
+    "m4_h64_d128": workloads.Dims(d=128, H=8, d_I=64, H_I=4, m=4, m_hca=64, k=32, W=16),
+    "m4_h256": workloads.Dims(d=128, H=8, d_I=32, H_I=4, m=4, m_hca=256, k=32, W=16),
+    "m2_h32": workloads.Dims(d=128, H=8, d_I=32, H_I=4, m=2, m_hca=32, k=32, W=16),
+    "m8_h100": workloads.Dims(d=128, H=8, d_I=32, H_I=4, m=8, m_hca=100, k=32, W=16),
+}
+
+
+@pytest.mark.parametrize("shape", list(_SHAPES))
+def test_compressor_shapes_within_one_ulp(shape):
+    """Both caches through csa_compress_all at every ratio form, ragged lengths that end inside a
+    128-token tile, against the fp64 oracle; the two csa_compress calls give the same bytes."""
+    wl = wl_small([1000, 333, 4], B=3, dims=_SHAPES[shape], seed=2100)
+    layer = gh.new_layer(wl)
+    d = wl.dims
+    for b in range(wl.B):
+        n = wl.n0[b]
+        ref = gh.OracleSeq(wl, b, n, with_mass=True)
+        n_c, n_h = n // d.m, n // d.m_hca
+        checks = [(gh.u16(layer.entries[layer.csa_off[b]:layer.csa_off[b] + n_c]), ref.E64, ref.E_mass, "entries"),
+                  (gh.u16(layer.entry_keys[layer.csa_off[b]:layer.csa_off[b] + n_c]), ref.KI64, ref.KI_mass, "keys")]
+        if n_h:
+            checks.append((gh.u16(layer.hca_entries[layer.hca_off[b]:layer.hca_off[b] + n_h]), ref.H64, ref.H_mass,
+                           "hca_entries"))
+        for got, want, mass, name in checks:
+            far, diff = gh.ulp_compare(got, want, mass)
+            assert far == 0, f"seq {b} {name}: {far} elements beyond one bf16 ulp + fp32 accumulation bound"
+            assert diff <= max(2, 2e-3 * want.size), f"seq {b} {name}: {diff} of {want.size} rounded differently"
+    sep = csa.HybridLayer(gh.dims_of(d), [wl.capacity(b) for b in range(wl.B)])
+    sdev.fill_layer_inputs(sep, wl)
+    sep.set_lengths(list(wl.n0))
+    sep.compress_separately()
+    torch.cuda.synchronize()
+    assert csa.csa_sync_status() == csa.CSA_OK
+    for name in ("entries", "entry_keys", "hca_entries"):
+        assert torch.equal(getattr(layer, name).view(torch.int16), getattr(sep, name).view(torch.int16)), name
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_compress_partial_ranges(which):
+    """csa_compress over per-sequence entry ranges that start and end inside 128-token tiles writes
+    exactly those entries, equal to the full pass, and nothing else."""
+    wl = wl_small([3000, 700], B=2, dims=_SHAPES["m4_h8_d128"], seed=2200)
+    d = wl.dims
+    full = gh.new_layer(wl)
+    part = csa.HybridLayer(gh.dims_of(d), [wl.capacity(b) for b in range(wl.B)])
+    sdev.fill_layer_inputs(part, wl)
+    part.set_lengths(list(wl.n0))
+    m = d.m if which == 0 else d.m_hca
+    ranges = [(37, 300), (0, 700 // m)] if which == 0 else [(3, 301), (1, 700 // m)]
+    rt = torch.tensor(ranges, dtype=torch.int64, device="cuda")
+    if which == 0:
+        csa.csa_compress(gh.dims_of(d), 0, part.seqs, rt, 2, max(e - s for s, e in ranges), part.x, part.logit_c,
+                         part.bias_c, part.idx_key, part.entries, part.entry_keys)
+        tensors = [("entries", part.csa_off), ("entry_keys", part.csa_off)]
+    else:
+        csa.csa_compress(gh.dims_of(d), 1, part.seqs, rt, 2, max(e - s for s, e in ranges), part.x, part.logit_h,
+                         part.bias_h, None, part.hca_entries, None)
+        tensors = [("hca_entries", part.hca_off)]
+    torch.cuda.synchronize()
+    assert csa.csa_sync_status() == csa.CSA_OK
+    for name, offs in tensors:
+        P, F = getattr(part, name).view(torch.int16).cpu(), getattr(full, name).view(torch.int16).cpu()
+        written = torch.zeros(P.shape[0], dtype=torch.bool)
+        for b, (e0, e1) in enumerate(ranges):
+            written[offs[b] + e0:offs[b] + e1] = True
+        assert torch.equal(P[written], F[written]), name
+        assert (P[~written] == 0).all(), f"{name}: rows outside the ranges were written"
+
+
+@pytest.mark.parametrize("shape", ["m4_h8_d128", "m4_h64_d128", "m4_h256", "m2_h32"])
+def test_incremental_append_equals_full_pass_shapes(shape):
+    """The decode append at every ratio form leaves the caches bit-identical to one full pass."""
+    d = _SHAPES[shape]
+    wl = wl_small([2 * d.m_hca - 5, 37], steps=d.m_hca + 12, B=2, dims=d, seed=2300)
+    layer = gh.new_layer(wl)
+    q = torch.empty(wl.B, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(wl.B, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(wl.B, d.H_I, dtype=torch.float32, device="cuda")
+    out = torch.empty(wl.B, d.H, d.d, dtype=torch.float32, device="cuda")
+    ws = layer.decode_workspace()
+    for s in range(wl.steps):
+        for b in range(wl.B):
+            sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
+        layer.decode(layer.decode_args(q, qi, w, out), ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    full = gh.new_layer(wl, lens=[n + wl.steps for n in wl.n0])
+    for name in ("entries", "entry_keys", "hca_entries"):
+        assert torch.equal(getattr(layer, name).view(torch.int16), getattr(full, name).view(torch.int16)), name
+
+
 # --------------------------------------------------------------------------------- a3/a4 (stage)
 
 def _index_case(E_list, k, d_I=64, H_I=4, seed=3001, quantize=False, zero_w=False):

@@ -459,3 +459,62 @@ def test_oracle_bf16_rounding_matches_generator_on_doubles():
     lib = synth.host_lib()
     gen = np.array([lib.synth_bf16_host(float(a)) for a in v], dtype=np.uint16)
     np.testing.assert_array_equal(oracle.round_bf16(v), gen)
+
+
+# ---------------------------------------------------------------- 8-bit block-scaled indexer keys
+
+def test_e4m3_rounding_matches_library():
+    """The oracle's nearest-even rounding onto the FP8 E4M3 grid equals torch's float32 -> float8_e4m3fn
+    conversion on float32 values in [-448, 448], subnormals and exact ties included."""
+    rng = np.random.default_rng(21)
+    v = np.concatenate([rng.uniform(-448, 448, 20000), rng.standard_normal(20000) * 2.0 ** rng.integers(-12, 8, 20000),
+                        np.arange(-64, 65) * 2.0 ** -10,  # ties on the subnormal grid (steps of 2^-9)
+                        [1.0625, 1.1875, -3.125, 448.0, -448.0, 0.0, 2.0 ** -6, 2.0 ** -9]]).astype(np.float32)
+    v = v[np.abs(v) <= 448]
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.e4m3_round(v.astype(np.float64)), ref)
+
+
+def test_e4m3_values_match_library():
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)  # every code but NaN
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.e4m3_value(codes), ref)
+
+
+@pytest.mark.parametrize("scale", [1.0, 2.0 ** -20, 3.0e4])
+def test_mx8_block_scale_is_the_smallest_power_of_two(scale):
+    """Each block's scale 2^e is the smallest power of two with amax <= 448 * 2^e, so the largest
+    magnitude lands in (224, 448]; every element is x / 2^e rounded on the E4M3 grid, so the
+    dequantized key is within half an E4M3 step (relative 2^-4 for normal values) of x."""
+    n, d_I = 300, 64
+    K = oracle.round_bf16(synth.bf16_to_f64(bf(SEED, synth.KI, 17, n, d_I)) * scale)
+    K[5] = 0  # an all-zero entry: scale byte 0, zero elements
+    Kq, sc = oracle.quantize_keys_mx8(K)
+    Kf = synth.bf16_to_f64(K)
+    for j in range(n):
+        for b in range(d_I // 32):
+            x = Kf[j, 32 * b:32 * b + 32]
+            e = int(sc[j, b]) - 127
+            amax = np.abs(x).max()
+            if amax == 0:
+                assert e == -127 and (Kq[j, 32 * b:32 * b + 32] & 0x7F == 0).all()
+                continue
+            assert 224 < amax / 2.0 ** e <= 448
+            np.testing.assert_array_equal(Kq[j, 32 * b:32 * b + 32], oracle.e4m3_round(x / 2.0 ** e))
+            deq = oracle.e4m3_value(Kq[j, 32 * b:32 * b + 32]) * 2.0 ** e
+            bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** (e - 10))
+            assert (np.abs(deq - x) <= bound).all()
+
+
+def test_mx8_scores_are_the_plain_scores_of_the_dequantized_keys():
+    """The 8-bit scorer equals the bf16 scorer applied to the dequantized keys (which bf16 holds
+    exactly: 4 significant bits times a power of two)."""
+    n, d_I = 500, 64
+    K = bf(SEED, synth.KI, 18, n, d_I)
+    qI = bf(SEED, synth.QI, 18, 4, d_I)
+    w = synth.f32_uniform(SEED, synth.W, 18, 4, 0, 1)[0]
+    Kq, sc = oracle.quantize_keys_mx8(K)
+    deq = oracle.e4m3_value(Kq) * np.repeat(2.0 ** (sc.astype(np.float64) - 127), 32, axis=1)
+    Kd = oracle.round_bf16(deq)
+    np.testing.assert_array_equal(synth.bf16_to_f64(Kd), deq)
+    np.testing.assert_array_equal(oracle.index_scores_mx8(qI, w, Kq, sc), oracle.index_scores(qI, w, Kd))
