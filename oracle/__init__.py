@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
         L.oracle_hca_attn.argtypes = [vp, ci, ci, vp, ci, vp, i64, ci, cd, vp, vp]
         L.oracle_hca_attn.restype = ci
         L.oracle_lse_merge.argtypes = [vp, vp, vp, vp, ci, ci, vp, vp]
+        L.oracle_rms_norm.argtypes = [vp, i64, ci, vp, cd, vp]
         L.oracle_e4m3_round.argtypes = [vp, i64, vp]
         L.oracle_e4m3_value.argtypes = [vp, i64, vp]
         L.oracle_quantize_keys_mx8.argtypes = [vp, i64, ci, vp, vp]
@@ -216,6 +217,24 @@ def hca_attn(q, hca, m_hca, raw, L, W, scale):
     return O, lse
 
 
+def rms_norm(x, gain, eps: float) -> np.ndarray:
+    """Rows of x (fp64 [rows, d]) RMS-normalized with gain [d] (fp64 out)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    gain = np.ascontiguousarray(gain, dtype=np.float32)
+    rows, d = x.reshape(-1, x.shape[-1]).shape
+    out = np.empty(x.shape, dtype=np.float64)
+    lib().oracle_rms_norm(_p(x), rows, d, _p(gain), float(eps), _p(out))
+    return out
+
+
+def sink_merge(O, lse, sink):
+    """The attention-sink logit z_h of every head as one more softmax term whose value is zero
+    ("DeepSeek V4 comprimeix el context", "CSA: buscar primer i atendre despres", last paragraph):
+    exactly an LSE merge with a partial of output 0 and log-sum-exp z."""
+    z = np.ascontiguousarray(sink, dtype=np.float64)
+    return lse_merge(O, lse, np.zeros_like(np.asarray(O, dtype=np.float64)), z)
+
+
 def lse_merge(O1, lse1, O2, lse2):
     O1, O2 = np.ascontiguousarray(O1, np.float64), np.ascontiguousarray(O2, np.float64)
     lse1, lse2 = np.ascontiguousarray(lse1, np.float64), np.ascontiguousarray(lse2, np.float64)
@@ -243,19 +262,25 @@ class Shape:
         return 1.0 / float(np.sqrt(self.d))
 
 
-def hybrid_query(shape: Shape, L: int, q, qI, w, raw, entries, KI, hca):
+def hybrid_query(shape: Shape, L: int, q, qI, w, raw, entries, KI, hca, sink=None, q_gain=None, eps=1e-6):
     """One query of the hybrid layer at visible length L, composed from the stages above.
 
     raw: uint16 [>=L, d] raw latents of the sequence; entries: uint16 [>=L//m, d] CSA cache;
     KI: uint16 [>=L//m, d_I] indexer-key cache; hca: uint16 [>=L//m', d] HCA cache.
+    Optional: sink [H] attention-sink logits; q_gain [d]: the query heads are RMS-normalized with
+    this gain (and rounded to bf16, the attention's operand type) before attending.
     Returns a dict with the selected indices, the two partials and the merged output.
     """
     n_c = L // shape.m
     s = index_scores(qI, w, KI[:n_c])
     idx = topk(s, shape.k)
+    if q_gain is not None:
+        q = round_bf16(rms_norm(bf16_to_f64(q), q_gain, eps))
     O_c, lse_c = csa_attn(q, entries, idx, shape.m, raw, L, shape.W, shape.scale)
     O_h, lse_h = hca_attn(q, hca, shape.m_hca, raw, L, 0, shape.scale)
     O, lse = lse_merge(O_c, lse_c, O_h, lse_h)
+    if sink is not None:
+        O, lse = sink_merge(O, lse, sink)
     return {"idx": idx, "scores": s, "O_csa": O_c, "lse_csa": lse_c, "O_hca": O_h, "lse_hca": lse_h,
             "O": O, "lse": lse}
 

@@ -431,3 +431,21 @@ void oracle_index_scores_mx8(const uint16_t* qI, const float* w, int H_I, int d_
         s[j] = acc;
     }
 }
+
+/* ---- f3: query / compressed-entry normalization ---------------------------- */
+/*
+ * "DeepSeek V4 comprimeix el context", section "CSA: buscar primer i atendre despres", last
+ * paragraph: the design normalizes the queries and the compressed entries to stabilize the logits.
+ * Reading (the page names no formula): RMS normalization with a learned gain, applied to each query
+ * head's d-wide vector and to each compressed entry (CSA and HCA) as it is produced:
+ *   out[c] = x[c] / sqrt(mean_c' x[c']^2 + eps) * gain[c].
+ * rows of d doubles in, rows of d doubles out.
+ */
+void oracle_rms_norm(const double* x, int64_t rows, int d, const float* gain, double eps, double* out) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c) ss += x[r * d + c] * x[r * d + c];
+        double inv = 1.0 / sqrt(ss / d + eps);
+        for (int c = 0; c < d; ++c) out[r * d + c] = x[r * d + c] * inv * (double)gain[c];
+    }
+}

@@ -518,3 +518,47 @@ def test_mx8_scores_are_the_plain_scores_of_the_dequantized_keys():
     Kd = oracle.round_bf16(deq)
     np.testing.assert_array_equal(synth.bf16_to_f64(Kd), deq)
     np.testing.assert_array_equal(oracle.index_scores_mx8(qI, w, Kq, sc), oracle.index_scores(qI, w, Kd))
+
+
+# ---------------------------------------------------------------- sinks and normalization
+
+def test_rms_norm_matches_library_and_closed_forms():
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((50, 64)) * rng.uniform(0.01, 100, (50, 1))
+    g = synth.f32_normal(SEED, synth.BIAS_C, 31, 64, 0, 1)[0]
+    eps = 1e-6
+    out = oracle.rms_norm(x, g, eps)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (64,), torch.from_numpy(g.astype(np.float64)), eps)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-13, atol=1e-15)
+    ones = np.ones(64, np.float32)
+    y = oracle.rms_norm(x, ones, 0.0)
+    np.testing.assert_allclose((y ** 2).mean(axis=1), 1.0, rtol=1e-13)           # unit RMS
+    np.testing.assert_allclose(oracle.rms_norm(7.5 * x, ones, 0.0), y, rtol=1e-13)  # scale invariant
+    c = np.full((1, 64), 3.0)
+    np.testing.assert_allclose(oracle.rms_norm(c, g, 0.5), 3.0 / math.sqrt(9.5) * g[None].astype(np.float64),
+                               rtol=1e-14)
+
+
+@pytest.mark.parametrize("L", [9, 40, 200])
+def test_sink_at_zero_query_and_vanishing_sink(L):
+    """The sink is one more softmax term with a zero value: at q = 0 every key has logit 0, so with n
+    keys lse = log(n + e^z) and O = (n / (n + e^z)) * mean of the keys; a sink of -inf changes nothing."""
+    sh = oracle.Shape(d=16, H=2, d_I=8, H_I=4, m=4, m_hca=16, k=5, W=8)
+    raw = bf(SEED, synth.X, 19, L, sh.d)
+    entries = bf(SEED, synth.A, 19, max(L // sh.m, 1), sh.d)
+    KI = bf(SEED, synth.KI, 19, max(L // sh.m, 1), sh.d_I)
+    hca = bf(SEED, synth.B, 19, max(L // sh.m_hca, 1), sh.d)
+    q = np.zeros((sh.H, sh.d), np.uint16)
+    qI = np.zeros((sh.H_I, sh.d_I), np.uint16)
+    w = np.full(sh.H_I, 0.5, np.float32)
+    z = np.array([0.7, -2.0])
+    base = oracle.hybrid_query(sh, L, q, qI, w, raw, entries, KI, hca)
+    r = oracle.hybrid_query(sh, L, q, qI, w, raw, entries, KI, hca, sink=z)
+    n = min(sh.k, L // sh.m) + min(sh.W, L) + L // sh.m_hca
+    np.testing.assert_allclose(r["lse"], np.log(n + np.exp(z)), rtol=1e-14)
+    np.testing.assert_allclose(r["O"], base["O"] * (n / (n + np.exp(z)))[:, None], rtol=1e-13, atol=1e-15)
+    q2 = bf(SEED, synth.Q, 19, sh.H, sh.d)
+    a = oracle.hybrid_query(sh, L, q2, qI, w, raw, entries, KI, hca)
+    b = oracle.hybrid_query(sh, L, q2, qI, w, raw, entries, KI, hca, sink=np.full(sh.H, -np.inf))
+    np.testing.assert_array_equal(a["O"], b["O"])
+    np.testing.assert_array_equal(a["lse"], b["lse"])
