@@ -27,10 +27,46 @@ sys.path.insert(0, ROOT)
 
 METRIC = "CSA+HCA decode queries/s at 1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
 
-# DRAM bytes (read + write) of one ctx1m index_scan_kernel launch in an ncu capture of the same kernel
-# and launch shape (profiles/index_scan_ctx1m.md: 134.24 MB read, 4.13 MB of scores written).  Set it
-# to None whenever the scan kernel or its launch shape changes, until it is captured again.
-SCAN_TRAFFIC_BYTES = 138_370_000
+# DRAM bytes (read + write) of one index_scan_kernel launch at the 1M-context workload (B=4), from
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel source it
+# was taken on: the key is the SHA-256 prefix of csrc/index_topk.cu at that capture.  Any other
+# source reports null traffic until it is captured again.
+SCAN_TRAFFIC = {"source_sha256": None, "bytes": None}
+
+
+def _source_sha(name):
+    import hashlib
+    path = os.path.join(ROOT, "compressed_sparse_kv_overlapped_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def scan_traffic():
+    """The captured DRAM bytes of one scan launch if they belong to the current scan source, else None."""
+    try:
+        if SCAN_TRAFFIC["source_sha256"] and _source_sha("index_topk.cu") == SCAN_TRAFFIC["source_sha256"]:
+            return SCAN_TRAFFIC["bytes"]
+    except OSError:
+        pass
+    return None
+
+
+def graph_kernel_nodes(graph):
+    """Kernel nodes of a captured CUDA graph (torch.cuda.CUDAGraph(keep_graph=True)): the number of
+    kernel launches one replay makes."""
+    from cuda.bindings import runtime as rt
+    err, _, n = rt.cudaGraphGetNodes(graph.raw_cuda_graph(), 0)
+    if err != rt.cudaError_t.cudaSuccess:
+        return None
+    err, nodes, n = rt.cudaGraphGetNodes(graph.raw_cuda_graph(), n)
+    if err != rt.cudaError_t.cudaSuccess:
+        return None
+    count = 0
+    for node in nodes[:n]:
+        err, typ = rt.cudaGraphNodeGetType(node)
+        if err == rt.cudaError_t.cudaSuccess and typ == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+            count += 1
+    return count
 
 
 def max_over_ranks(values, dev, world):
@@ -53,6 +89,8 @@ def parse():
     ap.add_argument("--config", default="ctx1m", choices=["ctx1m", "long", "ragged", "tiny", "prefill"],
                     help="decode workloads (the default ctx1m is the headline), or the causal prefill of "
                          "131,072 queries, reported as tensor-pipe throughput")
+    ap.add_argument("--keys", default="bf16", choices=["bf16", "mx8"],
+                    help="indexer keys of the decode workloads: bf16 (the workload as stated) or 8-bit block-scaled")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--stage", default=None, choices=["index", "attn"],
@@ -145,14 +183,17 @@ def dims_of(wd):
     return csa.make_dims(d=wd.d, H=wd.H, d_I=wd.d_I, H_I=wd.H_I, m=wd.m, m_hca=wd.m_hca, k=wd.k, W=wd.W)
 
 
-def step_bytes(wd, lens):
+def step_bytes(wd, lens, keys="bf16"):
     """Algorithmic HBM bytes of one decode step: indexer-key scan, gathered top-k entries, raw window,
-    HCA entries (queries and outputs not counted)."""
-    idx = sum((L // wd.m) * wd.d_I * 2 for L in lens)
+    HCA entries (queries and outputs not counted), and the block-scale bytes of 8-bit keys (one per
+    32 key channels; 0 for bf16 keys)."""
+    kb = wd.d_I if keys == "mx8" else wd.d_I * 2
+    idx = sum((L // wd.m) * kb for L in lens)
+    scales = sum((L // wd.m) * (wd.d_I // 32) for L in lens) if keys == "mx8" else 0
     gather = sum(min(wd.k, L // wd.m) * wd.d * 2 for L in lens)
     window = sum(min(wd.W, L) * wd.d * 2 for L in lens)
     hca = sum((L // wd.m_hca) * wd.d * 2 for L in lens)
-    return idx, gather, window, hca
+    return idx, gather, window, hca, scales
 
 
 # ------------------------------------------------------------------------------------ our arm
@@ -170,7 +211,7 @@ def run_ours(args, rank, world):
     B = wl.B
     K, W = args.steps, args.warmup
     extra = W + K + (0 if args.no_e2e else K) + 1
-    layer = csa.HybridLayer(dims_of(wd), [n + extra for n in wl.n0], device=dev)
+    layer = csa.HybridLayer(dims_of(wd), [n + extra for n in wl.n0], device=dev, key_format=args.keys)
     sdev.fill_layer_inputs(layer, wl)
     layer.set_lengths(list(wl.n0))
     layer.compress()
@@ -211,10 +252,12 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     lens_before = list(layer.lens)
     stream = torch.cuda.Stream(device=dev)
-    graph = torch.cuda.CUDAGraph()
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
     with torch.cuda.graph(graph, stream=stream):
         for s in range(K):
             csa.hybrid_attn_decode(args_for(W + s), ws, torch.cuda.current_stream())
+    launches = graph_kernel_nodes(graph)
+    graph.instantiate()
     graph_ev = torch.cuda.CUDAGraph()
     csa.csa_set_stage_events(marks)
     with torch.cuda.graph(graph_ev, stream=stream):
@@ -276,10 +319,10 @@ def run_ours(args, rank, world):
         return steps_sorted[min(K - 1, int(round(q * (K - 1))))]
 
     # algorithmic bytes per step (lengths after each step's append)
-    tot = [0, 0, 0, 0]
+    tot = [0, 0, 0, 0, 0]
     for s in range(K):
         lens = [n + s + 1 for n in lens_before]
-        for i, v in enumerate(step_bytes(wd, lens)):
+        for i, v in enumerate(step_bytes(wd, lens, args.keys)):
             tot[i] += v
     per_step = [v / K for v in tot]
     bytes_step = sum(per_step)
@@ -287,18 +330,21 @@ def run_ours(args, rank, world):
     ms_step = ms / K
     achieved_step_gbs = bytes_step / (ms_step * 1e-3) / 1e9
     scan_ms = stage["index_scan"]
-    scan_gbs = per_step[0] / (scan_ms * 1e-3) / 1e9 if scan_ms > 0 else None
+    scan_bytes = per_step[0] + per_step[4]  # keys and, for 8-bit keys, their scale bytes
+    scan_gbs = scan_bytes / (scan_ms * 1e-3) / 1e9 if scan_ms > 0 else None
     result = {
         "metric": METRIC, "value": B * world * K / (ms * 1e-3), "unit": "queries/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
-        "config": {"workload": wl.name, "B": B, "N": wl.n0[0] if len(set(wl.n0)) == 1 else "ragged",
+        "config": {"workload": wl.name + ("_mx8keys" if args.keys == "mx8" else ""), "B": B,
+                   "N": wl.n0[0] if len(set(wl.n0)) == 1 else "ragged", "indexer_keys": args.keys,
                    "d": wd.d, "heads": wd.H, "d_I": wd.d_I, "H_I": wd.H_I, "k": wd.k, "W": wd.W, "m": wd.m,
                    "m_hca": wd.m_hca, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "per-step working set larger than L2 (no flush)"},
         "hbm": {"algorithmic_bytes_per_step": int(bytes_step),
-                "breakdown_bytes": {"index_keys": int(per_step[0]), "gathered_entries": int(per_step[1]),
-                                    "window": int(per_step[2]), "hca_entries": int(per_step[3])},
+                "breakdown_bytes": {"index_keys": int(per_step[0]), "scale_bytes": int(per_step[4]),
+                                    "gathered_entries": int(per_step[1]), "window": int(per_step[2]),
+                                    "hca_entries": int(per_step[3])},
                 "achieved_gbs": achieved_step_gbs, "peak_gbs": hbm_peak, "frac": achieved_step_gbs / hbm_peak,
                 "peak_source": peak_src},
         "stages_ms": stage,
@@ -308,26 +354,20 @@ def run_ours(args, rank, world):
                                         "step), not the timed graph"},
         "roofline": {"kernel": "index_scan_kernel", "bound": "hbm", "achieved": scan_gbs, "peak": hbm_peak,
                      "unit": "GB/s", "frac": (scan_gbs / hbm_peak) if scan_gbs else None,
-                     "traffic": SCAN_TRAFFIC_BYTES if wl.name.startswith("ctx1m") else None,
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, profiles/index_scan_ctx1m.md",
-                     "bytes_per_launch": int(per_step[0]), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
+                     "traffic": scan_traffic() if wl.name.startswith("ctx1m") and args.keys == "bf16" else None,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch, "
+                                       "taken on the current scan source (null otherwise)",
+                     "bytes_per_launch": int(scan_bytes), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
         "clocks": clocks.summary(t0, t1),
     }
-    # attention launches a merge kernel when a query's keys are split over several CTAs
-    result["gpu_launches"] = K * (4 + (1 if _attn_items(wd, B, max_len) > 1 else 0))
+    # kernel nodes of the timed graph (all of them this library's kernels)
+    result["gpu_launches"] = launches
 
     if not args.no_e2e:
         result["e2e"] = run_e2e(layer, wl, K, W, max_len, ws, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(wl, samples=4)
+        result["cpu_baseline"] = cpu_baseline(wl, keys=args.keys)
     return result
-
-
-def _attn_items(wd, B, max_len):
-    per_q = wd.k + wd.W + max_len // wd.m_hca
-    kpi = int(os.environ.get("CSA_KEYS_PER_ITEM", "0")) or max(128, min(2048, ((per_q * B + 127) // 128 + 63) // 64 * 64))
-    kpi = (kpi + 63) // 64 * 64
-    return (per_q + kpi - 1) // kpi
 
 
 def run_e2e(layer, wl, K, W, max_len, ws, dev, world):
@@ -434,7 +474,7 @@ class OracleDecode:
     query selects (also untimed).  A timed query runs the oracle's indexer scores, top-k, sparse
     attention with the window, HCA attention and LSE merge."""
 
-    def __init__(self, wl, b=0, rows=(0,)):
+    def __init__(self, wl, b=0, rows=(0,), keys="bf16"):
         import numpy as np
 
         import oracle
@@ -453,6 +493,7 @@ class OracleDecode:
         KI, _ = oracle.compress_parallel(kI, a_idx, np.ascontiguousarray(bias_c[:, :wd.d_I]), None, L, wd.m,
                                          2 * wd.m, np.arange(n_c))
         self.KI = oracle.round_bf16(KI)
+        self.keys_mx8 = oracle.quantize_keys_mx8(self.KI) if keys == "mx8" else None
         del a_idx, kI
         bl = workloads.raw_tokens(wl, b, 0, L, "b")
         H, _ = oracle.compress_parallel(x, bl, workloads.bias_h(wl), None, L, wd.m_hca, wd.m_hca, np.arange(n_h))
@@ -460,35 +501,42 @@ class OracleDecode:
         del bl
         self.x = x
         self.E = np.zeros((n_c, wd.d), np.uint16)
-        self.queries = []
-        a = None
-        for r in rows:
-            q, qi, w = workloads.queries(wl, b, r, r + 1)
-            idx = oracle.topk(oracle.index_scores(qi[0], w[0], self.KI), wd.k)
-            need = idx[idx >= 0]
-            if a is None:
-                a = workloads.raw_tokens(wl, b, 0, L, "a")
-            E, _ = oracle.compress_parallel(x, a, bias_c, None, L, wd.m, 2 * wd.m, need)
-            self.E[need] = oracle.round_bf16(E)
-            self.queries.append((q[0], qi[0], w[0]))
+        self.queries = [tuple(t[0] for t in workloads.queries(wl, b, r, r + 1)) for r in rows]
+
+        def selection(qv):  # the entries a sample query selects (untimed preparation)
+            _, qi, w = qv
+            sc = (oracle.index_scores_mx8(qi, w, *self.keys_mx8) if self.keys_mx8 is not None
+                  else oracle.index_scores(qi, w, self.KI))
+            return oracle.topk(sc, wd.k)
+
+        sel = oracle.parallel_map(selection, self.queries)
+        need = np.unique(np.concatenate([i[i >= 0] for i in sel])).astype(np.int64)
+        a = workloads.raw_tokens(wl, b, 0, L, "a")
+        E, _ = oracle.compress_parallel(x, a, bias_c, None, L, wd.m, 2 * wd.m, need)
+        self.E[need] = oracle.round_bf16(E)
 
     def run(self, i):
         import oracle
         q, qi, w = self.queries[i]
-        return oracle.hybrid_query(self.shape, self.L, q, qi, w, self.x, self.E, self.KI, self.H)
+        return oracle.hybrid_query(self.shape, self.L, q, qi, w, self.x, self.E, self.KI, self.H,
+                                   keys_mx8=self.keys_mx8)
 
 
-def cpu_baseline(wl, samples=4):
+def cpu_baseline(wl, samples=None, keys="bf16"):
+    """The oracle on a bounded sample of the workload: one decode query per host core (at least 4) on
+    one prepared sequence, in parallel threads (the oracle's C code releases the GIL)."""
     from concurrent.futures import ThreadPoolExecutor
-    threads = min(samples, os.cpu_count() or 1)
-    od = OracleDecode(wl, 0, rows=tuple(range(samples)))
+    host = os.cpu_count() or 1
+    samples = samples or max(4, host)
+    threads = min(samples, host)
+    od = OracleDecode(wl, 0, rows=tuple(range(samples)), keys=keys)
     t0 = time.perf_counter()
     with ThreadPoolExecutor(threads) as ex:
         list(ex.map(od.run, range(samples)))
     dt = time.perf_counter() - t0
-    return {"value": samples / dt, "unit": "queries/s", "cores": threads, "kind": "oracle",
-            "sample": f"{samples} decode queries of one sequence at L={od.L} (the workload's geometry), caches "
-                      f"prepared untimed, one query per thread"}
+    return {"value": samples / dt, "unit": "queries/s", "cores": threads, "host_cores": host, "kind": "oracle",
+            "sample": f"{samples} decode queries of one sequence at L={od.L} (the workload's geometry, {keys} "
+                      f"indexer keys), caches prepared untimed, one query per thread"}
 
 
 def run_reference(args, rank, world):
@@ -639,7 +687,7 @@ def run_prefill(args, rank, world):
     hbm, tf_peak, src = peaks(sustained=True)
     tflops = (f_index + f_attn) / (ms * 1e-3) / 1e12
     comp_bytes = N * (3 * wd.d + wd.d_I) * 2 + (N // wd.m) * (wd.d + wd.d_I) * 2 + (N // wd.m_hca) * wd.d * 2
-    return {
+    res = {
         "metric": "causal prefill queries/s (indexer + top-k + sparse/HCA attention); tensor TFLOP/s",
         "value": N * world / (ms * 1e-3), "unit": "queries/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -652,9 +700,174 @@ def run_prefill(args, rank, world):
                      "peak": tf_peak, "unit": "TFLOP/s", "frac": tflops / tf_peak, "traffic": None,
                      "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops_sustained)"},
         "compress": {"ms": ms_comp, "bytes": comp_bytes, "achieved_gbs": comp_bytes / (ms_comp * 1e-3) / 1e9,
-                     "peak_gbs": hbm, "note": "csa_compress for the CSA and HCA caches over all N tokens"},
+                     "peak_gbs": hbm, "frac": comp_bytes / (ms_comp * 1e-3) / 1e9 / hbm,
+                     "note": "csa_compress_all: CSA entries, indexer keys and HCA entries over all N tokens, one pass"},
         "clocks": clocks.summary(t0, t1),
     }
+    del q, qi, w, out, ws, args_c
+    torch.cuda.empty_cache()
+    if not args.no_e2e:
+        res["e2e"] = prefill_e2e(layer, wl, K, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = prefill_cpu_baseline(wl)
+    return res
+
+
+def prefill_e2e(layer, wl, K, dev, world, chunk=8192):
+    """The prefill through the public call with every input in pinned HOST memory: per step the raw
+    rows (x, both logit arrays, indexer keys) and all queries go host -> device, the outputs device ->
+    host, inside the timed region.  hybrid_attn_prefill runs over query chunks (compressing in the
+    first), and a copy stream moves chunk i+1's queries in and chunk i-1's outputs out while chunk i
+    computes."""
+    import torch
+
+    import compressed_sparse_kv_overlapped_b200 as csa
+    from synth import device as sdev
+    wd = wl.dims
+    N = wl.n0[0]
+    try:
+        h_raw = [torch.empty_like(t, device="cpu").pin_memory() for t in (layer.x, layer.logit_c, layer.logit_h,
+                                                                          layer.idx_key)]
+        h_q = torch.empty(N, wd.H, wd.d, dtype=torch.bfloat16).pin_memory()
+        h_qi = torch.empty(N, wd.H_I, wd.d_I, dtype=torch.bfloat16).pin_memory()
+        h_w = torch.empty(N, wd.H_I, dtype=torch.float32).pin_memory()
+        h_out = torch.empty(N, wd.H, wd.d, dtype=torch.float32).pin_memory()
+    except RuntimeError as e:
+        return {"unavailable": f"pinned host buffers of {N} queries could not be allocated: {e}"[:200]}
+    for h, t in zip(h_raw, (layer.x, layer.logit_c, layer.logit_h, layer.idx_key)):
+        h.copy_(t)
+    # the queries, generated on the device chunk by chunk and parked in host memory (untimed)
+    tq = torch.empty(chunk, wd.H, wd.d, dtype=torch.bfloat16, device=dev)
+    tqi = torch.empty(chunk, wd.H_I, wd.d_I, dtype=torch.bfloat16, device=dev)
+    tw = torch.empty(chunk, wd.H_I, dtype=torch.float32, device=dev)
+    for c0 in range(0, N, chunk):
+        n = min(chunk, N - c0)
+        sdev.fill_queries(wl, 0, c0, c0 + n, tq[:n], tqi[:n], tw[:n])
+        h_q[c0:c0 + n].copy_(tq[:n])
+        h_qi[c0:c0 + n].copy_(tqi[:n])
+        h_w[c0:c0 + n].copy_(tw[:n])
+    del tq, tqi, tw
+    dq = [torch.empty(chunk, wd.H, wd.d, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dqi = [torch.empty(chunk, wd.H_I, wd.d_I, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dw = [torch.empty(chunk, wd.H_I, dtype=torch.float32, device=dev) for _ in range(2)]
+    do = [torch.empty(chunk, wd.H, wd.d, dtype=torch.float32, device=dev) for _ in range(2)]
+    ws = layer.prefill_workspace(N)
+    stream = torch.cuda.current_stream()
+    cs = torch.cuda.Stream(device=dev)
+    nch = (N + chunk - 1) // chunk
+
+    def one_step():
+        raw_done = torch.cuda.Event()
+        with torch.cuda.stream(cs):
+            for h, t in zip(h_raw, (layer.x, layer.logit_c, layer.logit_h, layer.idx_key)):
+                t.copy_(h, non_blocking=True)
+            raw_done.record(cs)
+        in_done = [torch.cuda.Event() for _ in range(nch)]
+        comp_done = [torch.cuda.Event() for _ in range(nch)]
+        out_done = [torch.cuda.Event() for _ in range(nch)]
+
+        def h2d(i):
+            c0, n, b = i * chunk, min(chunk, N - i * chunk), i % 2
+            with torch.cuda.stream(cs):
+                if i >= 2:
+                    cs.wait_event(comp_done[i - 2])
+                dq[b][:n].copy_(h_q[c0:c0 + n], non_blocking=True)
+                dqi[b][:n].copy_(h_qi[c0:c0 + n], non_blocking=True)
+                dw[b][:n].copy_(h_w[c0:c0 + n], non_blocking=True)
+                in_done[i].record(cs)
+
+        h2d(0)
+        stream.wait_event(raw_done)
+        for i in range(nch):
+            c0, n, b = i * chunk, min(chunk, N - i * chunk), i % 2
+            if i + 1 < nch:
+                h2d(i + 1)
+            stream.wait_event(in_done[i])
+            if i >= 2:
+                stream.wait_event(out_done[i - 2])
+            a = layer.prefill_args(dq[b], dqi[b], dw[b], do[b], c0, c0 + n, compress=(i == 0))
+            csa.hybrid_attn_prefill(a, ws, stream)
+            comp_done[i].record(stream)
+            with torch.cuda.stream(cs):
+                cs.wait_event(comp_done[i])
+                h_out[c0:c0 + n].copy_(do[b][:n], non_blocking=True)
+                out_done[i].record(cs)
+        for i in range(max(0, nch - 2), nch):
+            stream.wait_event(out_done[i])
+
+    one_step()  # warm-up
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    cs.wait_event(e0)
+    for _ in range(K):
+        one_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if csa.csa_sync_status() != csa.CSA_OK:
+        raise RuntimeError("device status in the prefill e2e region")
+    ms, = max_over_ranks([e0.elapsed_time(e1) / K], dev, world)
+    h2d_b = sum(t.numel() * t.element_size() for t in h_raw) + sum(t.numel() * t.element_size()
+                                                                   for t in (h_q, h_qi, h_w))
+    return {"value": N * world / (ms * 1e-3), "unit": "queries/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d_b), "d2h_bytes_per_step": int(h_out.numel() * 4),
+            "how": f"hybrid_attn_prefill over chunks of {chunk} queries (compress in the first); raw rows and "
+                   f"queries from pinned host memory, outputs back to pinned host memory, on a copy stream "
+                   f"double-buffered against the compute stream"}
+
+
+def prefill_cpu_baseline(wl, n_rows=512):
+    """The oracle on 512 seeded query rows of the prefill (positions 0-4, 127, 128, 4095, 4096 and N-1
+    among them), all host cores: caches (indexer keys and HCA entries for the whole sequence, CSA
+    entries where a sampled row selects them) are prepared untimed; a timed row runs the oracle's
+    indexer scores, top-k, sparse attention with the window, HCA attention and LSE merge."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+
+    import oracle
+    from synth import workloads
+    wd = wl.dims
+    N = wl.n0[0]
+    rng = np.random.default_rng(wl.seed)
+    fixed = [0, 1, 2, 3, 4, 127, 128, 4095, 4096, N - 1]
+    rest = [int(r) for r in rng.choice(N, size=4 * n_rows, replace=False) if int(r) not in fixed]
+    rows = sorted(fixed + rest[:n_rows - len(fixed)])
+    shape = oracle.Shape(d=wd.d, H=wd.H, d_I=wd.d_I, H_I=wd.H_I, m=wd.m, m_hca=wd.m_hca, k=wd.k, W=wd.W)
+    x = workloads.raw_tokens(wl, 0, 0, N, "x")
+    a = workloads.raw_tokens(wl, 0, 0, N, "a")
+    kI = workloads.raw_tokens(wl, 0, 0, N, "kI")
+    bias_c = workloads.bias_c(wl)
+    n_c, n_h = N // wd.m, N // wd.m_hca
+    KI, _ = oracle.compress_parallel(kI, np.ascontiguousarray(a[:, :wd.d_I]), np.ascontiguousarray(bias_c[:, :wd.d_I]),
+                                     None, N, wd.m, 2 * wd.m, np.arange(n_c))
+    KI = oracle.round_bf16(KI)
+    bl = workloads.raw_tokens(wl, 0, 0, N, "b")
+    H, _ = oracle.compress_parallel(x, bl, workloads.bias_h(wl), None, N, wd.m_hca, wd.m_hca, np.arange(n_h))
+    H = oracle.round_bf16(H)
+    del bl, kI
+    qs = [workloads.queries(wl, 0, r, r + 1) for r in rows]
+    host = os.cpu_count() or 1
+    with ThreadPoolExecutor(host) as ex:
+        sel = list(ex.map(lambda i: oracle.topk(oracle.index_scores(qs[i][1][0], qs[i][2][0],
+                                                                    KI[:(rows[i] + 1) // wd.m]), wd.k),
+                          range(len(rows))))
+    need = np.unique(np.concatenate([s[s >= 0] for s in sel] + [np.zeros(0, np.int32)]))
+    E = np.zeros((max(n_c, 1), wd.d), np.uint16)
+    if len(need):
+        Ev, _ = oracle.compress_parallel(x, a, bias_c, None, N, wd.m, 2 * wd.m, need.astype(np.int64))
+        E[need] = oracle.round_bf16(Ev)
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(host) as ex:
+        list(ex.map(lambda i: oracle.hybrid_query(shape, rows[i] + 1, qs[i][0][0], qs[i][1][0], qs[i][2][0], x, E, KI,
+                                                  H), range(len(rows))))
+    dt = time.perf_counter() - t0
+    return {"value": len(rows) / dt, "unit": "queries/s", "cores": min(host, len(rows)), "host_cores": host,
+            "kind": "oracle",
+            "sample": f"{len(rows)} seeded query rows of the N={N} prefill (positions 0-4, 127, 128, 4095, 4096, "
+                      f"N-1 among them), caches prepared untimed, one row per thread"}
 
 
 def run_stage_attn(args):

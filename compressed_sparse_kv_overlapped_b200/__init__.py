@@ -30,7 +30,8 @@ CSA_OP_PREFILL = 5
 
 EXPORTS = ("csa_compress", "csa_compress_all", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
            "hybrid_attn_prefill", "csa_workspace_size", "csa_last_error", "csa_sync_status", "csa_version",
-           "csa_set_stage_events", "csa_index_topk_noalloc")
+           "csa_set_stage_events", "csa_index_topk_noalloc", "csa_debug_inject", "csa_quantize_keys",
+           "csa_index_topk_mx8")
 CSA_DECODE_MARKS = 5
 
 _i32, _i64, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
@@ -45,12 +46,18 @@ class csa_ws_query(ctypes.Structure):
     _fields_ = [("dims", csa_dims), ("Q", _i32), ("reserved", _i32), ("max_len", _i64)]
 
 
+class csa_norms(ctypes.Structure):
+    _fields_ = [("q_norm", _vp), ("entry_norm_c", _vp), ("entry_norm_h", _vp), ("sink", _vp), ("eps", _f32),
+                ("reserved", _i32)]
+
+
 class csa_decode_args(ctypes.Structure):
     _fields_ = [("dims", csa_dims), ("B", _i32), ("append", _i32), ("max_len", _i64), ("scale", _f32),
                 ("seqs", _vp), ("x", _vp), ("logit_c", _vp), ("logit_h", _vp), ("idx_key", _vp),
                 ("bias_c", _vp), ("bias_h", _vp), ("entries", _vp), ("entry_keys", _vp), ("hca_entries", _vp),
                 ("q", _vp), ("q_idx", _vp), ("w", _vp), ("out", _vp), ("lse", _vp), ("idx_out", _vp),
-                ("new_rows", _vp)]
+                ("new_rows", _vp), ("keys_q", _vp), ("key_scales", _vp), ("idx_in", _vp),
+                ("norms", ctypes.POINTER(csa_norms))]
 
 
 class csa_prefill_args(ctypes.Structure):
@@ -58,7 +65,7 @@ class csa_prefill_args(ctypes.Structure):
                 ("q_end", _i64), ("scale", _f32), ("seq", _vp), ("x", _vp), ("logit_c", _vp), ("logit_h", _vp),
                 ("idx_key", _vp), ("bias_c", _vp), ("bias_h", _vp), ("entries", _vp), ("entry_keys", _vp),
                 ("hca_entries", _vp), ("q", _vp), ("q_idx", _vp), ("w", _vp), ("out", _vp), ("lse", _vp),
-                ("idx_out", _vp)]
+                ("idx_out", _vp), ("idx_in", _vp), ("norms", ctypes.POINTER(csa_norms))]
 
 
 _lib = None
@@ -75,7 +82,7 @@ def lib() -> ctypes.CDLL:
         L.csa_compress.argtypes = [P(csa_dims), ctypes.c_int, _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp]
         L.csa_compress_all.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
-                                       _vp, _vp, _vp]
+                                       _vp, _vp, P(csa_norms), _vp]
         L.csa_index_topk.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                      _vp]
         L.csa_sparse_attn.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp,
@@ -89,10 +96,14 @@ def lib() -> ctypes.CDLL:
         L.csa_last_error.restype = ctypes.c_char_p
         L.csa_sync_status.argtypes = [_vp]
         L.csa_set_stage_events.argtypes = [_vp, ctypes.c_int]
+        L.csa_debug_inject.argtypes = [ctypes.c_int, _i64]
+        L.csa_quantize_keys.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp]
+        L.csa_index_topk_mx8.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                         _vp, _sz, _vp]
         L.csa_index_topk_noalloc.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
         for n in ("csa_compress", "csa_compress_all", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
                   "hybrid_attn_prefill", "csa_sync_status", "csa_version", "csa_set_stage_events",
-                  "csa_index_topk_noalloc"):
+                  "csa_index_topk_noalloc", "csa_debug_inject", "csa_quantize_keys", "csa_index_topk_mx8"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -164,11 +175,27 @@ def csa_compress(dims, which, seqs, ranges, B, max_entries, x, logit, bias, idx_
     _check(rc, "csa_compress")
 
 
+def csa_debug_inject(fault: int, wait_limit_ns: int = 0) -> None:
+    """Fault injection for the bounded-wait tests (see csa.h); csa_debug_inject(0) turns it off."""
+    _check(lib().csa_debug_inject(fault, wait_limit_ns), "csa_debug_inject")
+
+
+def make_norms(q_norm=None, entry_norm_c=None, entry_norm_h=None, sink=None, eps=1e-6) -> csa_norms:
+    """csa_norms from device tensors (or None for the parts that are off)."""
+    n = csa_norms()
+    n.q_norm, n.entry_norm_c, n.entry_norm_h, n.sink = (_ptr(q_norm), _ptr(entry_norm_c), _ptr(entry_norm_h),
+                                                        _ptr(sink))
+    n.eps = float(eps)
+    n.reserved = 0
+    return n
+
+
 def csa_compress_all(dims, seqs, tok_ranges, B, max_tokens, x, logit_c, logit_h, bias_c, bias_h, idx_key, entries,
-                     entry_keys, hca_entries, stream=None) -> None:
+                     entry_keys, hca_entries, stream=None, norms=None) -> None:
     rc = lib().csa_compress_all(ctypes.byref(dims), _ptr(seqs), _ptr(tok_ranges), B, max_tokens, _ptr(x),
                                 _ptr(logit_c), _ptr(logit_h), _ptr(bias_c), _ptr(bias_h), _ptr(idx_key),
-                                _ptr(entries), _ptr(entry_keys), _ptr(hca_entries), _vp(_stream(stream)))
+                                _ptr(entries), _ptr(entry_keys), _ptr(hca_entries),
+                                None if norms is None else ctypes.byref(norms), _vp(_stream(stream)))
     _check(rc, "csa_compress_all")
 
 
@@ -186,6 +213,20 @@ def csa_index_topk_noalloc(dims, seqs, queries, Q, max_len, q_idx, w, entry_keys
                                       _ptr(w), _ptr(entry_keys), _ptr(idx_out), _ptr(score_out),
                                       _vp(_stream(stream)))
     _check(rc, "csa_index_topk_noalloc")
+
+
+def csa_quantize_keys(dims, seqs, ranges, B, max_entries, entry_keys, keys_q, key_scales, stream=None) -> None:
+    rc = lib().csa_quantize_keys(ctypes.byref(dims), _ptr(seqs), _ptr(ranges), B, max_entries, _ptr(entry_keys),
+                                 _ptr(keys_q), _ptr(key_scales), _vp(_stream(stream)))
+    _check(rc, "csa_quantize_keys")
+
+
+def csa_index_topk_mx8(dims, seqs, queries, Q, max_len, q_idx, w, keys_q, key_scales, idx_out, score_out, ws,
+                       stream=None):
+    rc = lib().csa_index_topk_mx8(ctypes.byref(dims), _ptr(seqs), _ptr(queries), Q, max_len, _ptr(q_idx), _ptr(w),
+                                  _ptr(keys_q), _ptr(key_scales), _ptr(idx_out), _ptr(score_out), _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(), _vp(_stream(stream)))
+    _check(rc, "csa_index_topk_mx8")
 
 
 def csa_sparse_attn(dims, seqs, queries, Q, q, entries, idx, x, scale, out, lse, ws, stream=None):

@@ -37,6 +37,7 @@ namespace csa {
 namespace {
 
 constexpr int kHeadsPad = 64;  // M of every MMA (heads beyond H are zero rows)
+constexpr int kMaxCluster = 8; // CTAs of a decode cluster that merge their results
 constexpr int kTileKeys = 64;
 constexpr int kStages = 3;     // key tiles in flight
 constexpr int kThreads = 320;
@@ -63,6 +64,11 @@ struct Smem {
     static constexpr int kRowPtr = kMisc + 64;         // per loader warp: 16 row pointers
     static constexpr int kTotal = kRowPtr + 4 * 16 * 8;
     static constexpr int kAlloc = kTotal + 1024;       // slack for 1024-byte alignment
+    // cluster merge: the CTA's [64 x D] fp32 result in the freed key stages, rows padded by 16 bytes
+    // so that the eight rows a warp's quads store hit different banks
+    static constexpr int kOStride = D + 4;
+    static_assert(64 * kOStride * 4 <= kStages * kStage, "the result fits in the key stages");
+    static_assert(kBlock >= (64 + 16 * 64 + 64) * 4, "merge weights fit in the P buffers");
 };
 
 struct Bars {
@@ -171,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const int T = s1 > s0 ? (int)((s1 - s0 + kTileKeys - 1) / kTileKeys) : 0;
     const int n_items = p.n_items;
     const bool direct = n_items == 1;
+    const bool clustered = !direct && p.cluster > 1;
     const bool dep_wait = !(p.hca_nowait && !direct && item >= p.items_front);
 
     if (threadIdx.x == 0) {
@@ -214,9 +221,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             if (p.tma_hca) tma_prefetch_map(&maps.hca);
             if (p.tma_x) tma_prefetch_map(&maps.x);
         }
+        // per stage, the full-barrier parity of the last tile this thread loaded by TMA (bit 2 set:
+        // one is pending), so that a CTA that gives up waits for its own copies before it exits
+        uint32_t tma_pend = 0;
         for (int t = 0; t < T; ++t) {
             const int st = t % kStages;
-            if (t >= kStages && !mbar_wait(&bars->empty[st], ((t / kStages) - 1) & 1, p.status, abort_flag)) break;
+            if (t >= kStages && !mbar_wait(&bars->empty[st], ((t / kStages) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
             const int64_t tb = s0 + (int64_t)t * kTileKeys;
             // A full tile of consecutive cache rows (HCA entries, or raw window tokens) goes by TMA:
             // one thread issues the boxes, the tile's bytes complete the full barrier, and the
@@ -233,6 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 }
                 if (row < 0 || row > 0x7FFFFFFF - kTileKeys) map = nullptr;
             }
+            // fault injection (tests of the bounded waits): the first loader warp skips its arrival
+            // on the first tile, which therefore never becomes full
+            const bool skip = p.debug_fault == 1 && t == 0 && lw == 0;
             if (map) {
                 if (lw == 0 && lane == 0) {
                     for (int w4 = 0; w4 < 4; ++w4) mask16[st * 4 + w4] = 0xFFFFu;
@@ -241,7 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
                     for (int kb = 0; kb < L::NKB; ++kb)
                         tma_load_2d(kdst + (uint32_t)kb * L::kBlock, map, kb * 64, (int)row, &bars->full[st]);
-                } else {
+                    tma_pend = (tma_pend & ~(7u << (3 * st))) | ((4u | (uint32_t)((t / kStages) & 1)) << (3 * st));
+                } else if (!skip) {
                     mbar_arrive(&bars->full[st]);
                 }
                 continue;
@@ -274,9 +288,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             fence_proxy_async_smem();
             if (lane == 0) mask16[st * 4 + lw] = (uint16_t)vm;
             __syncwarp();
-            mbar_arrive(&bars->full[st]);
+            if (!skip) mbar_arrive(&bars->full[st]);
         }
         cp_async_wait_all();
+        if (*abort_flag && tma_pend) {
+            // the CTA gave up: its TMA copies may still be landing in shared memory; wait (bounded)
+            // for the tiles whose barrier phase has not completed before the CTA exits
+            for (int st = 0; st < kStages; ++st) {
+                const uint32_t e = (tma_pend >> (3 * st)) & 7u;
+                if (e & 4u) mbar_wait(&bars->full[st], e & 1u, nullptr, nullptr, p.wait_ns);
+            }
+        }
     } else if (warp >= 8) {
         // ------------------------------------------------------------------ MMA issuers
         // warp 8 issues Q.K^T of every tile (A = Q from TMEM), warp 9 issues P.V (A = P, B = the key
@@ -287,11 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         if (T > 0) {
             if (warp == 8) {
                 constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
-                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0, p.status, abort_flag));
+                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0, p.status, abort_flag, p.wait_ns));
                 for (int g1 = 0; ok && g1 < T; ++g1) {
                     const int st = g1 % kStages;
-                    bool w = mbar_wait(&bars->full[st], (g1 / kStages) & 1, p.status, abort_flag);
-                    if (w && g1 >= 2) w = mbar_wait(&bars->s_free[g1 & 1], ((g1 >> 1) - 1) & 1, p.status, abort_flag);
+                    bool w = mbar_wait(&bars->full[st], (g1 / kStages) & 1, p.status, abort_flag, p.wait_ns);
+                    if (w && g1 >= 2) w = mbar_wait(&bars->s_free[g1 & 1], ((g1 >> 1) - 1) & 1, p.status, abort_flag, p.wait_ns);
                     if (!__all_sync(0xffffffffu, w)) break;
                     tc_fence_after();
                     const uint64_t kd = sdesc_kmajor(sbase + L::kK + (uint32_t)st * L::kStage);
@@ -312,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 constexpr int HALVES = D >= 256 ? D / 256 : 1;
                 constexpr uint32_t id2 = idesc_bf16(64, N2, false, true);
                 for (int g2 = 0; g2 < T; ++g2) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->p_full[g2 & 1], (g2 >> 1) & 1, p.status, abort_flag)))
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->p_full[g2 & 1], (g2 >> 1) & 1, p.status, abort_flag, p.wait_ns)))
                         break;
                     tc_fence_after();
                     const int st = g2 % kStages;
@@ -333,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 }
             }
             umma_commit(&bars->fin);
-            mbar_wait(&bars->fin, 0, p.status, nullptr);
+            mbar_wait(&bars->fin, 0, p.status, nullptr, p.wait_ns);
         }
         __syncwarp();
     } else {
@@ -349,6 +371,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             const int h0 = warp * 16 + qa, h1 = h0 + 8;
             const uint2* q0 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h0 < p.H ? h0 : 0)) * D);
             const uint2* q1 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h1 < p.H ? h1 : 0)) * D);
+            // optional RMS normalization of each head's query (gain p.q_norm): the four lanes of a quad
+            // hold a quarter of the row each; a first pass sums the squares, the second scales
+            float inv0 = 1.f, inv1 = 1.f;
+            if (p.q_norm) {
+                float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 4
+                for (int cb = 0; cb < D / 2; cb += 64) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int col = cb + 8 * k + qc;
+                        float f[4];
+                        const uint2 v0 = h0 < p.H ? q0[col / 2] : make_uint2(0, 0);
+                        const uint2 v1 = h1 < p.H ? q1[col / 2] : make_uint2(0, 0);
+                        f[0] = bf16lo(v0.x); f[1] = bf16hi(v0.x); f[2] = bf16lo(v0.y); f[3] = bf16hi(v0.y);
+                        ss0 = fmaf(f[0], f[0], fmaf(f[1], f[1], fmaf(f[2], f[2], fmaf(f[3], f[3], ss0))));
+                        f[0] = bf16lo(v1.x); f[1] = bf16hi(v1.x); f[2] = bf16lo(v1.y); f[3] = bf16hi(v1.y);
+                        ss1 = fmaf(f[0], f[0], fmaf(f[1], f[1], fmaf(f[2], f[2], fmaf(f[3], f[3], ss1))));
+                    }
+                }
+                ss0 += __shfl_xor_sync(0xffffffffu, ss0, 1);
+                ss0 += __shfl_xor_sync(0xffffffffu, ss0, 2);
+                ss1 += __shfl_xor_sync(0xffffffffu, ss1, 1);
+                ss1 += __shfl_xor_sync(0xffffffffu, ss1, 2);
+                inv0 = rsqrtf(ss0 / D + p.norm_eps);
+                inv1 = rsqrtf(ss1 / D + p.norm_eps);
+            }
+            // dims 2col .. 2col + 3 of a row, normalized and rounded back to bf16 when a gain is given
+            auto qload = [&](const uint2* row, bool valid, float inv, int col) -> uint2 {
+                uint2 v = valid ? row[col / 2] : make_uint2(0, 0);
+                if (p.q_norm && valid) {
+                    const float4 gn = *reinterpret_cast<const float4*>(p.q_norm + 2 * col);
+                    v.x = pack_bf16x2(bf16lo(v.x) * inv * gn.x, bf16hi(v.x) * inv * gn.y);
+                    v.y = pack_bf16x2(bf16lo(v.y) * inv * gn.z, bf16hi(v.y) * inv * gn.w);
+                }
+                return v;
+            };
 #pragma unroll 1
             for (int cb = 0; cb < D / 2; cb += 128) {
                 uint32_t r[2][32];
@@ -358,8 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                     for (int k = 0; k < 8; ++k) {
                         const int col = cb + g * 64 + 8 * k + qc;  // a column holds 2 dims: uint2 index col / 2
                         const bool in = cb + g * 64 < D / 2;
-                        const uint2 v0 = (in && h0 < p.H) ? q0[col / 2] : make_uint2(0, 0);
-                        const uint2 v1 = (in && h1 < p.H) ? q1[col / 2] : make_uint2(0, 0);
+                        const uint2 v0 = qload(q0, in && h0 < p.H, inv0, col);
+                        const uint2 v1 = qload(q1, in && h1 < p.H, inv1, col);
                         r[g][4 * k] = v0.x; r[g][4 * k + 1] = v0.y; r[g][4 * k + 2] = v1.x; r[g][4 * k + 3] = v1.y;
                     }
                 }
@@ -383,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         bool ok = true;
         for (int t = 0; t < T; ++t) {
             const int sb = t & 1, st = t % kStages;
-            ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, p.status, abort_flag) &&
-                 mbar_wait(&bars->full[st], (t / kStages) & 1, p.status, abort_flag);
+            ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, p.status, abort_flag, p.wait_ns) &&
+                 mbar_wait(&bars->full[st], (t / kStages) & 1, p.status, abort_flag, p.wait_ns);
             if (!ok) break;
             tc_fence_after();
             float s[2][16];  // [row ra / ra+8][2k + e] = column 8k + cq + e
@@ -435,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             // in the same row / column layout as S
             const bool any = __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f);
             if (t > 0 && any) {
-                ok = mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status, abort_flag);
+                ok = mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status, abort_flag, p.wait_ns);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll 1
@@ -456,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             }
             // P buffer t&1 is free once the P.V of tile t-2 finished
             if (t >= 2) {
-                ok = mbar_wait(&bars->o_done[sb], ((t >> 1) - 1) & 1, p.status, abort_flag);
+                ok = mbar_wait(&bars->o_done[sb], ((t >> 1) - 1) & 1, p.status, abort_flag, p.wait_ns);
                 if (!ok) break;
             }
             {
@@ -483,8 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             mbar_arrive(&bars->p_full[sb]);
         }
         // ---- epilogue: TMEM -> registers -> global memory
-        if (ok && T > 0) ok = mbar_wait(&bars->o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, p.status, abort_flag);
-        float inv[2];
+        if (ok && T > 0) ok = mbar_wait(&bars->o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, p.status, abort_flag, p.wait_ns);
+        float inv[2], lse2[2];  // lse2: log-sum-exp in log2 units
         bool has[2];
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
@@ -492,17 +550,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
             has[rr] = ok && T > 0 && l_run[rr] > 0.f;
             inv[rr] = has[rr] ? 1.f / l_run[rr] : 0.f;
+            lse2[rr] = has[rr] ? m_run[rr] + log2f(l_run[rr]) : -INFINITY;
+            // a single item holds the query's whole softmax: its sink logit (one more term with a zero
+            // value) joins here; with several items it joins in the merge
+            const float z = (direct && p.sink && hr[rr] < p.H) ? p.sink[hr[rr]] * 1.4426950408889634f : -INFINITY;
+            if (z > -INFINITY && (ok || T == 0)) {
+                const float m_eff = has[rr] ? fmaxf(m_run[rr], z) : z;
+                const float a = has[rr] ? exp2f(m_run[rr] - m_eff) : 0.f;
+                const float l_eff = fmaf(l_run[rr], a, exp2f(z - m_eff));
+                inv[rr] = a / l_eff;
+                lse2[rr] = m_eff + log2f(l_eff);
+            }
         }
         const bool write_o = ok && T > 0;
         const int rows = p.H < kHeadsPad ? p.H : kHeadsPad;
+        const bool to_smem = clustered;  // the cluster merges its CTAs' results in shared memory
+        float* o_smem = reinterpret_cast<float*>(sm + L::kK);
         if (write_o) {
             // straight from the registers: per row, the four lanes of a quad write 32 consecutive
             // bytes (one full sector) per instruction
             float* dst[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr)
-                dst[rr] = direct ? p.out + ((int64_t)qi * p.H + hr[rr]) * D
-                                 : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + hr[rr]) * D;
+                dst[rr] = to_smem ? o_smem + hr[rr] * L::kOStride
+                          : direct ? p.out + ((int64_t)qi * p.H + hr[rr]) * D
+                                   : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + hr[rr]) * D;
             tc_fence_after();
             // two register buffers: the TMEM load of the next 64 columns is in flight while the
             // current ones are stored
@@ -544,13 +616,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             for (int rr = 0; rr < 2; ++rr) {
                 const int h = hr[rr];
                 if (h >= p.H) continue;
-                const float lse_v = has[rr] ? (m_run[rr] + log2f(l_run[rr])) * 0.69314718055994531f : -INFINITY;
+                const float lse_v = lse2[rr] * 0.69314718055994531f;
                 if (direct) {
                     if (p.lse) p.lse[(int64_t)qi * p.H + h] = lse_v;
+                } else if (to_smem) {
+                    reinterpret_cast<float*>(sm + L::kP0)[h] = lse_v;
                 } else {
                     p.part_lse[((int64_t)qi * n_items + item) * kHeadsPad + h] = lse_v;
                 }
             }
+            if (to_smem && (i & 3) == 0)  // rows of heads past H: no contribution
+                for (int rr = 0; rr < 2; ++rr)
+                    if (hr[rr] >= p.H) reinterpret_cast<float*>(sm + L::kP0)[hr[rr]] = -INFINITY;
         }
     }
     tc_fence_before();
@@ -558,6 +635,59 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     if (warp == 8 && T > 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+    if (clustered) {
+        // ---- the cluster's merge: CTA `rank` combines columns [rank * D/F, (rank + 1) * D/F) of the
+        // F results (each normalized by its own sum, with its lse) into one partial of the query
+        const int F = p.cluster;
+        const uint32_t rank = cluster_ctarank();
+        const float* o_smem = reinterpret_cast<const float*>(sm + L::kK);  // [64][kOStride] results
+        float* lse_s = reinterpret_cast<float*>(sm + L::kP0);        // [64] this CTA's lse
+        float* wts = lse_s + kHeadsPad;                               // [F][64] merge weights
+        float* mlse = wts + F * kHeadsPad;                            // [64] merged lse
+        // (the softmax warps wrote lse_s for all 64 rows: -inf for rows without a result, so an
+        // empty or failed CTA contributes nothing and its unwritten rows are never read)
+        cluster_barrier();
+        if (threadIdx.x < kHeadsPad) {
+            const int h = threadIdx.x;
+            float l[kMaxCluster];
+            float mx = -INFINITY;
+            for (int c = 0; c < F; ++c) {
+                l[c] = ld_cluster_f32(lse_s + h, (uint32_t)c);
+                mx = fmaxf(mx, l[c]);
+            }
+            float sum = 0.f;
+            for (int c = 0; c < F; ++c) {
+                l[c] = mx == -INFINITY ? 0.f : expf(l[c] - mx);
+                sum += l[c];
+            }
+            for (int c = 0; c < F; ++c) wts[c * kHeadsPad + h] = sum > 0.f ? l[c] / sum : 0.f;
+            mlse[h] = mx == -INFINITY ? -INFINITY : mx + logf(sum);
+        }
+        __syncthreads();
+        const int cols = D / F, n4 = cols / 4;
+        const int part = item / F;
+        const int n_parts = n_items / F;
+        for (int e = threadIdx.x; e < kHeadsPad * n4; e += kThreads) {
+            const int h = e / n4, col = (int)rank * cols + 4 * (e % n4);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int c = 0; c < F; ++c) {
+                const float w = wts[c * kHeadsPad + h];
+                if (w > 0.f) {
+                    const float4 v = ld_cluster_f32x4(o_smem + h * L::kOStride + col, (uint32_t)c);
+                    acc.x = fmaf(w, v.x, acc.x);
+                    acc.y = fmaf(w, v.y, acc.y);
+                    acc.z = fmaf(w, v.z, acc.z);
+                    acc.w = fmaf(w, v.w, acc.w);
+                }
+            }
+            if (h < p.H)
+                *reinterpret_cast<float4*>(p.part_o + (((int64_t)qi * n_parts + part) * kHeadsPad + h) * D + col) = acc;
+        }
+        if (rank == 0)
+            for (int h = threadIdx.x; h < kHeadsPad; h += kThreads)
+                p.part_lse[((int64_t)qi * n_parts + part) * kHeadsPad + h] = mlse[h];
+        cluster_barrier();  // no CTA leaves while another still reads its shared memory
     }
 }
 
@@ -570,7 +700,7 @@ __global__ void combine_kernel(AttnParams p) {
     constexpr int kMaxBatch = 24;  // partial rows held in registers per pass
     grid_dep_wait();  // the partials come from the attention grid
     const int h = blockIdx.x, qi = blockIdx.y;
-    const int n_items = p.n_items;
+    const int n_items = p.cluster > 1 ? p.n_items / p.cluster : p.n_items;  // partials per query
     const int lane = threadIdx.x & 31;
     __shared__ float s_lse[256];
     __shared__ float s_w[256];
@@ -589,7 +719,9 @@ __global__ void combine_kernel(AttnParams p) {
         if (u < nb0) v[u] = __ldcg(reinterpret_cast<const float4*>(base + u * item_stride));
     __syncthreads();
     if (threadIdx.x < 32) {
-        float mx = -INFINITY;
+        // the head's sink logit, if any: one more softmax term whose value is zero
+        const float z = p.sink ? p.sink[h] : -INFINITY;
+        float mx = z;
         for (int it = lane; it < n_items; it += 32) mx = fmaxf(mx, s_lse[it]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -601,6 +733,7 @@ __global__ void combine_kernel(AttnParams p) {
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (z > -INFINITY) sum += expf(z - mx);
         if (lane == 0) {
             s_res[0] = sum > 0.f ? 1.f / sum : 0.f;
             s_res[1] = mx == -INFINITY ? -INFINITY : mx + logf(sum);
@@ -651,6 +784,9 @@ cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, 
               tensor_map_2d_bf16(&maps.x, p.raw, D, 0x7FFFFFFFull, (uint64_t)D * 2, 64, kTileKeys) == cudaSuccess;
     if (!q.tma_hca) std::memset(&maps.hca, 0, sizeof(maps.hca));
     if (!q.tma_x) std::memset(&maps.x, 0, sizeof(maps.x));
+    if (q.cluster > 1 && q.n_items > 1)
+        return launch_kernel_cluster(attn_kernel<D>, grid, dim3(kThreads), L::kAlloc, stream, pdl,
+                                     dim3((unsigned)q.cluster, 1, 1), maps, q, item_begin);
     return launch_kernel(attn_kernel<D>, grid, dim3(kThreads), L::kAlloc, stream, pdl, maps, q, item_begin);
 }
 

@@ -1,6 +1,7 @@
 // capi.cu -- the extern "C" boundary of libcsa (declared in include/csa.h): host-side argument
 // validation, workspace layout, and the orchestration of the decode and prefill hot paths.
 // No call allocates device memory or synchronizes the host.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -87,6 +88,22 @@ int env_int(const char* name, int dflt) {
     return r;
 }
 
+// Host checks of the optional normalization / sink parameters.
+int check_norms(const csa_dims& d, const csa_norms* n) {
+    if (!n) return CSA_OK;
+    if (n->reserved != 0) return fail(CSA_ERR_ARG, "csa_norms.reserved must be 0");
+    if (!aligned16(n->q_norm) || !aligned16(n->entry_norm_c) || !aligned16(n->entry_norm_h) ||
+        (reinterpret_cast<uintptr_t>(n->sink) & 3u))
+        return fail(CSA_ERR_ARG, "norm gains must be 16-byte aligned, sinks 4-byte aligned");
+    if (!(n->eps >= 0.f)) return fail(CSA_ERR_ARG, "eps = %g", (double)n->eps);
+    if (n->entry_norm_c && !csa_block_shape(d.m))
+        return fail(CSA_ERR_UNSUPPORTED, "CSA entry normalization needs m = 4 (m = %d)", d.m);
+    if (n->entry_norm_h && !hca_block_shape(d.m_hca))
+        return fail(CSA_ERR_UNSUPPORTED, "HCA entry normalization needs m_hca a power of two from 4 to 128 (%d)",
+                    d.m_hca);
+    return CSA_OK;
+}
+
 int round64(int64_t v) { return (int)(((v + 63) / 64) * 64); }
 
 int clamp_kpi(int64_t v, int lo, int hi) {
@@ -128,8 +145,14 @@ constexpr int kPlanSMs = 148;
 // fits).  The HCA items start when the scan frees SMs and finish by the time the front items do;
 // fewer, longer ones leave fewer partials to merge (measured at ctx1m: 8 tiles per item beat 5).
 constexpr int kHcaMinKeys = 512;
-ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh) {
+// The CTAs of each group of `cluster` consecutive items of a query merge their results through
+// distributed shared memory (one partial per group reaches the merge kernel); both parts' item
+// counts are rounded up to a multiple of it (the extra items are empty).
+constexpr int kDecodeCluster = 8;
+ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh, int* cluster) {
     const int f = env_int("CSA_KPI_FRONT", 0), h = env_int("CSA_KPI_HCA", 0);
+    const int cl = env_int("CSA_DECODE_CLUSTER", kDecodeCluster);
+    *cluster = cl == 2 || cl == 4 || cl == 8 ? cl : 1;
     const int kpi_front = f > 0 ? round64(f) : 128;
     const int64_t front = (int64_t)d.k + d.W;
     const int64_t front_ctas = (int64_t)B * ((front + kpi_front - 1) / kpi_front);
@@ -141,7 +164,16 @@ ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh) {
         const int64_t per = ((int64_t)B * max_eh + hca_ctas - 1) / hca_ctas;
         kpi_hca = clamp_kpi(per > kHcaMinKeys ? per : kHcaMinKeys, 128, 4096);
     }
-    return make_items(front, max_eh, kpi_front, kpi_hca);
+    ItemPlan ip = make_items(front, max_eh, kpi_front, kpi_hca);
+    if (*cluster > 1 && ip.n_items > 1) {
+        const int c = *cluster;
+        const int n_hca = ip.n_items - ip.items_front;
+        ip.items_front = (ip.items_front + c - 1) / c * c;
+        ip.n_items = ip.items_front + (n_hca + c - 1) / c * c;
+    } else {
+        *cluster = 1;
+    }
+    return ip;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -156,6 +188,7 @@ ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh) {
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     grid_dep_launch();  // the scan may start its launch; it waits for this grid before reading
     __shared__ float xs[8 * 8 * 24];
+    __shared__ float ss[2];  // entry normalization: this slice's sums of squares (CSA, HCA entry)
     const int s = blockIdx.x, b = blockIdx.y, ns = gridDim.x;
     const int tid = threadIdx.x;
     const csa_seq sq = p.seqs[b];
@@ -189,51 +222,88 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
             }
             __syncthreads();  // the compressor below reads these rows (coherent loads)
         }
-        if (len % p.m == 0 && tid < 8) {
-            const int64_t j = len / p.m - 1;
-            const int c0 = c0s + 8 * tid;
-            uint16_t* orow = p.entries + (sq.csa_off + j) * d + c0;
-            if (csa_block_shape(p.m)) {
-                const int64_t t0 = sq.tok_off + 4 * j - 4;  // row of window position 0
-                auto fetch = [&](int tensor, int pos) -> uint4 {
-                    const int64_t row = t0 + pos;
-                    if (tensor == 2) return __ldcg(reinterpret_cast<const uint4*>(p.idx_key + row * p.d_I + c0));
-                    const uint16_t* base = tensor == 0 ? p.logit_c : p.x;
-                    return __ldcg(reinterpret_cast<const uint4*>(base + row * d + c0));
-                };
-                if (c0 < p.d_I)
-                    csa_entry_block4<true>(j, d, p.bias_c + c0, fetch, orow,
-                                           p.entry_keys + (sq.csa_off + j) * p.d_I + c0);
-                else
-                    csa_entry_block4<false>(j, d, p.bias_c + c0, fetch, orow, nullptr);
+    }
+    // the entries this token completes (the same for every CTA of the sequence's cluster)
+    const bool c_do = ok && p.append && len % p.m == 0;
+    const bool h_do = ok && p.append && len % p.m_hca == 0;
+    const int64_t j = len / p.m - 1, h = len / p.m_hca - 1;
+    float cv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (c_do && tid < 8) {
+        const int c0 = c0s + 8 * tid;
+        const int64_t row = sq.csa_off + j;
+        uint4 key = make_uint4(0, 0, 0, 0);
+        if (csa_block_shape(p.m)) {
+            const int64_t t0 = sq.tok_off + 4 * j - 4;  // row of window position 0
+            auto fetch = [&](int tensor, int pos) -> uint4 {
+                const int64_t r = t0 + pos;
+                if (tensor == 2) return __ldcg(reinterpret_cast<const uint4*>(p.idx_key + r * p.d_I + c0));
+                const uint16_t* base = tensor == 0 ? p.logit_c : p.x;
+                return __ldcg(reinterpret_cast<const uint4*>(base + r * d + c0));
+            };
+            if (c0 < p.d_I) {
+                csa_entry_block4<true>(j, d, p.bias_c + c0, fetch, cv, &key);
+                *reinterpret_cast<uint4*>(p.entry_keys + row * p.d_I + c0) = key;
             } else {
-                compress_entry8(j, p.m, 2 * p.m, d, p.d_I, c0, p.x, p.logit_c, p.bias_c, p.idx_key, sq.tok_off,
-                                p.entries + (sq.csa_off + j) * d, p.entry_keys + (sq.csa_off + j) * p.d_I);
+                csa_entry_block4<false>(j, d, p.bias_c + c0, fetch, cv, nullptr);
             }
+        } else {  // the per-entry serial form writes the entry and its key itself (no normalization)
+            compress_entry8(j, p.m, 2 * p.m, d, p.d_I, c0, p.x, p.logit_c, p.bias_c, p.idx_key, sq.tok_off,
+                            p.entries + row * d, p.entry_keys + row * p.d_I);
+            if (c0 < p.d_I) key = *reinterpret_cast<const uint4*>(p.entry_keys + row * p.d_I + c0);
         }
-        if (len % p.m_hca == 0) {  // uniform over the CTA (the block form has barriers)
-            const int64_t h = len / p.m_hca - 1;
-            if (hca_block_shape(p.m_hca)) {
-                const int nb = p.m_hca / 4, u = tid >> 3, g = tid & 7, ub = u & (nb - 1);
-                const int c0 = c0s + 8 * g;
-                const int64_t row0 = sq.tok_off + (int64_t)p.m_hca * h + 4 * ub;
-                uint4 lg[4], xv[4], kv[4];
+        if (p.keys_q && c0 < p.d_I) {
+            // the 8-bit copy of the key (four lanes per 32-channel block)
+            uint32_t sb;
+            const uint2 q8 = quant_mx8(key, 0xFu << (tid & ~3), &sb);
+            *reinterpret_cast<uint2*>(p.keys_q + row * p.d_I + c0) = q8;
+            if ((tid & 3) == 0) p.key_scales[row * (p.d_I / 32) + c0 / 32] = (uint8_t)sb;
+        }
+    }
+    float hv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (h_do) {  // uniform over the CTA (the block form has barriers)
+        if (hca_block_shape(p.m_hca)) {
+            const int nb = p.m_hca / 4, u = tid >> 3, g = tid & 7, ub = u & (nb - 1);
+            const int c0 = c0s + 8 * g;
+            const int64_t row0 = sq.tok_off + (int64_t)p.m_hca * h + 4 * ub;
+            uint4 lg[4], xv[4], kv[4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    lg[t] = __ldcg(reinterpret_cast<const uint4*>(p.logit_h + (row0 + t) * d + c0));
-                    xv[t] = __ldcg(reinterpret_cast<const uint4*>(p.x + (row0 + t) * d + c0));
-                    kv[t] = make_uint4(0, 0, 0, 0);
-                }
-                Part8 P;
-                part4<false>(lg, xv, kv, p.bias_h + (int64_t)(4 * ub) * d + c0, d, P);
-                hca_tree(P, nb, xs);
-                if (tid < 8)
-                    *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) = finish8(P.acc, P.den);
-            } else if (tid >= 128 && tid < 136) {
-                compress_entry8(h, p.m_hca, p.m_hca, d, p.d_I, c0s + 8 * (tid - 128), p.x, p.logit_h, p.bias_h,
-                                nullptr, sq.tok_off, p.hca_entries + (sq.hca_off + h) * d, nullptr);
+            for (int t = 0; t < 4; ++t) {
+                lg[t] = __ldcg(reinterpret_cast<const uint4*>(p.logit_h + (row0 + t) * d + c0));
+                xv[t] = __ldcg(reinterpret_cast<const uint4*>(p.x + (row0 + t) * d + c0));
+                kv[t] = make_uint4(0, 0, 0, 0);
             }
+            Part8 P;
+            part4<false>(lg, xv, kv, p.bias_h + (int64_t)(4 * ub) * d + c0, d, P);
+            hca_tree(P, nb, xs);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) hv[i] = __fdiv_rn(P.acc[i], P.den[i]);
+        } else if (tid >= 128 && tid < 136) {
+            compress_entry8(h, p.m_hca, p.m_hca, d, p.d_I, c0s + 8 * (tid - 128), p.x, p.logit_h, p.bias_h,
+                            nullptr, sq.tok_off, p.hca_entries + (sq.hca_off + h) * d, nullptr);
         }
+    }
+    float inv_c = 1.f, inv_h = 1.f;
+    if ((p.norm_c || p.norm_h) && (c_do || h_do)) {
+        // entry normalization (block forms only): partial sums of squares of this CTA's 64 channels,
+        // then the totals over the cluster's slices, in the same order as the full pass
+        if (tid < 32) {
+            const float sc = sum_lane8(sumsq8(cv)), sh = sum_lane8(sumsq8(hv));
+            if (tid == 0) { ss[0] = sc; ss[1] = sh; }
+        }
+        cluster_barrier();
+        if (tid < 8) {
+            if (c_do && p.norm_c) inv_c = rms_inv(cluster_sum(&ss[0], ns), d, p.eps);
+            if (h_do && p.norm_h) inv_h = rms_inv(cluster_sum(&ss[1], ns), d, p.eps);
+        }
+    }
+    if (tid < 8) {
+        const int c0 = c0s + 8 * tid;
+        if (c_do && csa_block_shape(p.m))
+            *reinterpret_cast<uint4*>(p.entries + (sq.csa_off + j) * d + c0) =
+                entry_bf16(cv, p.norm_c ? p.norm_c + c0 : nullptr, inv_c);
+        if (h_do && hca_block_shape(p.m_hca))
+            *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) =
+                entry_bf16(hv, p.norm_h ? p.norm_h + c0 : nullptr, inv_h);
     }
     // every CTA of the sequence has read seqs[b].len: CTA 0 may now write the new length
     cluster_barrier();
@@ -256,6 +326,7 @@ struct DecodePlan {
     int64_t max_eh;       // max HCA entries
     int64_t e_stride;
     ItemPlan items;
+    int cluster;          // attention items merged per thread-block cluster (1: none)
     size_t off_queries, off_idx, off_index, off_attn, total;
 };
 
@@ -265,7 +336,7 @@ DecodePlan plan_decode(const csa_dims& d, int B, int64_t max_len) {
     pl.max_eh = max_len / d.m_hca;
     pl.e_stride = ((pl.max_e + 3) / 4) * 4;
     if (pl.e_stride < 4) pl.e_stride = 4;
-    pl.items = plan_decode_items(d, B, pl.max_eh);
+    pl.items = plan_decode_items(d, B, pl.max_eh, &pl.cluster);
     size_t off = 0;
     pl.off_queries = off;
     off += align256((size_t)B * sizeof(csa_query));
@@ -326,7 +397,8 @@ int status_ptr(int** out) {
 int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_e,
               int64_t e_stride, const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
               float* score_out, void* ws_index, bool zero_ws, int* status, cudaStream_t stream,
-              cudaEvent_t mid = nullptr, bool pdl = false) {
+              cudaEvent_t mid = nullptr, bool pdl = false, const csa_bf16* prefetch_entries = nullptr,
+              const uint8_t* keys_q = nullptr, const uint8_t* key_scales = nullptr) {
     IndexParams ip{};
     ip.seqs = seqs;
     ip.queries = queries;
@@ -342,6 +414,10 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
     ip.idx_out = idx_out;
     ip.score_out = score_out;
     ip.status = status;
+    ip.keys_q = keys_q;
+    ip.key_scales = key_scales;
+    ip.prefetch_rows = reinterpret_cast<const unsigned char*>(prefetch_entries);
+    ip.prefetch_row_bytes = (int64_t)d.d * 2;
     index_ws_carve(ip, ws_index, Q, e_stride);
     cudaError_t e = launch_index_topk(ip, max_e, stream, zero_ws, mid, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "index_topk launch");
@@ -353,6 +429,17 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
 int device_status(int** out) { return status_ptr(out); }
 
 int validate_dims(const csa_dims* d) { return check_dims(d); }
+
+namespace {
+std::atomic<int> g_debug_fault{0};
+std::atomic<uint64_t> g_debug_wait_ns{0};
+}  // namespace
+
+void debug_fault_state(int* fault, uint64_t* wait_ns) {
+    *fault = g_debug_fault.load(std::memory_order_relaxed);
+    const uint64_t w = g_debug_wait_ns.load(std::memory_order_relaxed);
+    *wait_ns = w ? w : kWaitLimitNs;
+}
 
 int set_error(int code, const char* fmt, ...) {
     char buf[512];
@@ -370,7 +457,15 @@ using namespace csa;
 
 extern "C" {
 
-int csa_version(void) { return 100; }
+int csa_version(void) { return 200; }
+
+int csa_debug_inject(int fault, int64_t wait_limit_ns) {
+    if (fault < 0 || fault > 1) return fail(CSA_ERR_ARG, "fault = %d (0 none, 1 attention tile never full)", fault);
+    if (wait_limit_ns < 0) return fail(CSA_ERR_ARG, "wait_limit_ns = %lld", (long long)wait_limit_ns);
+    g_debug_fault.store(fault, std::memory_order_relaxed);
+    g_debug_wait_ns.store((uint64_t)wait_limit_ns, std::memory_order_relaxed);
+    return CSA_OK;
+}
 
 int csa_set_stage_events(void* const* events, int count) {
     if (!events || count == 0) {
@@ -471,8 +566,8 @@ int csa_compress(const csa_dims* dims, int which, const csa_seq* seqs, const int
 static int compress_all(const csa_dims& d, const csa_seq* seqs, const int64_t* tok_ranges, int64_t t0, int64_t t1,
                         int B, int64_t max_tokens, const csa_bf16* x, const csa_bf16* logit_c,
                         const csa_bf16* logit_h, const float* bias_c, const float* bias_h, const csa_bf16* idx_key,
-                        csa_bf16* entries, csa_bf16* entry_keys, csa_bf16* hca_entries, int* st,
-                        cudaStream_t stream) {
+                        csa_bf16* entries, csa_bf16* entry_keys, csa_bf16* hca_entries, const csa_norms* norms,
+                        int* st, cudaStream_t stream) {
     const bool csa_blk = csa_block_shape(d.m), hca_blk = hca_block_shape(d.m_hca);
     TileCompressParams tp{};
     tp.seqs = seqs;
@@ -496,6 +591,11 @@ static int compress_all(const csa_dims& d, const csa_seq* seqs, const int64_t* t
     tp.entries = entries;
     tp.entry_keys = entry_keys;
     tp.hca_entries = hca_entries;
+    if (norms) {
+        tp.norm_c = norms->entry_norm_c;
+        tp.norm_h = norms->entry_norm_h;
+        tp.eps = norms->eps;
+    }
     tp.status = st;
     cudaError_t e = launch_compress_tiles(tp, max_tokens, stream);
     if (e != cudaSuccess) return cuda_fail(e, "compress launch");
@@ -530,9 +630,10 @@ static int compress_all(const csa_dims& d, const csa_seq* seqs, const int64_t* t
 int csa_compress_all(const csa_dims* dims, const csa_seq* seqs, const int64_t* tok_ranges, int B, int64_t max_tokens,
                      const csa_bf16* x, const csa_bf16* logit_c, const csa_bf16* logit_h, const float* bias_c,
                      const float* bias_h, const csa_bf16* idx_key, csa_bf16* entries, csa_bf16* entry_keys,
-                     csa_bf16* hca_entries, csa_stream_t stream) {
+                     csa_bf16* hca_entries, const csa_norms* norms, csa_stream_t stream) {
     int rc = check_dims(dims);
     if (rc) return rc;
+    if ((rc = check_norms(*dims, norms))) return rc;
     if (!seqs || !tok_ranges || !x || !logit_c || !logit_h || !bias_c || !bias_h || !idx_key || !entries ||
         !entry_keys || !hca_entries)
         return fail(CSA_ERR_ARG, "NULL pointer argument");
@@ -544,7 +645,7 @@ int csa_compress_all(const csa_dims* dims, const csa_seq* seqs, const int64_t* t
     int* st = nullptr;
     if ((rc = status_ptr(&st))) return rc;
     return compress_all(*dims, seqs, tok_ranges, 0, 0, B, max_tokens, x, logit_c, logit_h, bias_c, bias_h, idx_key,
-                        entries, entry_keys, hca_entries, st, stream);
+                        entries, entry_keys, hca_entries, norms, st, stream);
 }
 
 size_t csa_workspace_size(int op, const void* args) {
@@ -596,9 +697,47 @@ int csa_index_topk(const csa_dims* dims, const csa_seq* seqs, const csa_query* q
                      stream);
 }
 
+int csa_quantize_keys(const csa_dims* dims, const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries,
+                      const csa_bf16* entry_keys, uint8_t* keys_q, uint8_t* key_scales, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !ranges || !entry_keys || !keys_q || !key_scales) return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (B < 1 || max_entries < 0) return fail(CSA_ERR_ARG, "B = %d, max_entries = %lld", B, (long long)max_entries);
+    if (!aligned16(entry_keys) || !aligned16(keys_q)) return fail(CSA_ERR_ARG, "entry_keys / keys_q must be 16-byte aligned");
+    int* st = nullptr;
+    if ((rc = status_ptr(&st))) return rc;
+    cudaError_t e = launch_quantize_keys(seqs, ranges, B, max_entries, dims->m, dims->d_I, entry_keys, keys_q,
+                                         key_scales, st, stream);
+    return e == cudaSuccess ? CSA_OK : cuda_fail(e, "quantize launch");
+}
+
+int csa_index_topk_mx8(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
+                       const csa_bf16* q_idx, const float* w, const uint8_t* keys_q, const uint8_t* key_scales,
+                       int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !queries || !q_idx || !w || !keys_q || !key_scales || !idx_out)
+        return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (Q < 1 || max_len < 1) return fail(CSA_ERR_ARG, "Q = %d, max_len = %lld", Q, (long long)max_len);
+    if (!aligned16(q_idx) || !aligned16(keys_q) || (reinterpret_cast<uintptr_t>(key_scales) & 1u))
+        return fail(CSA_ERR_ARG, "q_idx / keys_q must be 16-byte aligned, key_scales 2-byte aligned");
+    csa_ws_query wq{*dims, Q, 0, max_len};
+    const size_t need = csa_workspace_size(CSA_OP_INDEX_TOPK, &wq);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", need);
+    int* st = nullptr;
+    if ((rc = status_ptr(&st))) return rc;
+    const int64_t max_e = max_len / dims->m;
+    int64_t es = ((max_e + 3) / 4) * 4;
+    if (es < 4) es = 4;
+    return run_index(*dims, seqs, queries, Q, max_e, es, q_idx, w, nullptr, idx_out, score_out, ws, true, st, stream,
+                     nullptr, false, nullptr, keys_q, key_scales);
+}
+
 static int make_attn(AttnParams& p, const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q,
                      const csa_bf16* q, const csa_bf16* entries, const int32_t* idx, int k_slots, const csa_bf16* x,
-                     int W, const csa_bf16* hca, float scale, float* out, float* lse, void* ws, const ItemPlan& ip) {
+                     int W, const csa_bf16* hca, float scale, float* out, float* lse, void* ws, const ItemPlan& ip,
+                     const csa_norms* norms = nullptr) {
     int* st = nullptr;
     int rc = status_ptr(&st);
     if (rc) return rc;
@@ -627,7 +766,13 @@ static int make_attn(AttnParams& p, const csa_dims* dims, const csa_seq* seqs, c
     p.kpi_hca = ip.kpi_hca;
     p.out = out;
     p.lse = lse;
+    if (norms) {
+        p.sink = norms->sink;
+        p.q_norm = norms->q_norm;
+        p.norm_eps = norms->eps;
+    }
     p.status = st;
+    debug_fault_state(&p.debug_fault, &p.wait_ns);
     attn_ws_carve(p, ws);
     return CSA_OK;
 }
@@ -687,15 +832,22 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     if (rc) return rc;
     const csa_dims& d = a->dims;
     if (a->B < 1 || a->max_len < 1) return fail(CSA_ERR_ARG, "B = %d, max_len = %lld", a->B, (long long)a->max_len);
+    // with idx_in (a selection reused from another layer) the indexer does not run: no indexer query
+    const bool reuse = a->idx_in != nullptr;
     if (!a->seqs || !a->x || !a->logit_c || !a->logit_h || !a->idx_key || !a->bias_c || !a->bias_h || !a->entries ||
-        !a->entry_keys || !a->hca_entries || !a->q || !a->q_idx || !a->w || !a->out)
+        !a->entry_keys || !a->hca_entries || !a->q || (!reuse && (!a->q_idx || !a->w)) || !a->out)
         return fail(CSA_ERR_ARG, "NULL pointer argument");
     if (!aligned16(a->x) || !aligned16(a->logit_c) || !aligned16(a->logit_h) || !aligned16(a->idx_key) ||
         !aligned16(a->bias_c) || !aligned16(a->bias_h) || !aligned16(a->entries) || !aligned16(a->entry_keys) ||
         !aligned16(a->hca_entries) || !aligned16(a->q) || !aligned16(a->q_idx) || !aligned16(a->out) ||
         !aligned16(a->new_rows))
         return fail(CSA_ERR_ARG, "tensors must be 16-byte aligned");
+    if (reuse && a->idx_out) return fail(CSA_ERR_ARG, "idx_out with idx_in (the selection is the caller's)");
+    if ((rc = check_norms(d, a->norms))) return rc;
     if (a->new_rows && !a->append) return fail(CSA_ERR_ARG, "new_rows without append");
+    if ((a->keys_q == nullptr) != (a->key_scales == nullptr)) return fail(CSA_ERR_ARG, "keys_q and key_scales go together");
+    if (a->keys_q && (!aligned16(a->keys_q) || (reinterpret_cast<uintptr_t>(a->key_scales) & 1u)))
+        return fail(CSA_ERR_ARG, "keys_q must be 16-byte aligned, key_scales 2-byte aligned");
     const DecodePlan pl = plan_decode(d, a->B, a->max_len);
     if (!ws || ws_bytes < pl.total || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", pl.total);
@@ -703,7 +855,8 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     if ((rc = status_ptr(&st))) return rc;
     char* w = static_cast<char*>(ws);
     csa_query* queries = reinterpret_cast<csa_query*>(w + pl.off_queries);
-    int32_t* idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t*>(w + pl.off_idx);
+    int32_t* idx = reuse ? const_cast<int32_t*>(a->idx_in)
+                         : a->idx_out ? a->idx_out : reinterpret_cast<int32_t*>(w + pl.off_idx);
     void* ws_index = w + pl.off_index;
 
     AppendParams ap{};
@@ -724,6 +877,13 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     ap.entries = a->entries;
     ap.entry_keys = a->entry_keys;
     ap.hca_entries = a->hca_entries;
+    ap.keys_q = a->keys_q;
+    ap.key_scales = a->key_scales;
+    if (a->norms) {
+        ap.norm_c = a->norms->entry_norm_c;
+        ap.norm_h = a->norms->entry_norm_h;
+        ap.eps = a->norms->eps;
+    }
     ap.queries = queries;
     ap.zero_words = static_cast<uint32_t*>(ws_index);  // histograms + counters of the index scratch
     ap.n_zero_words = (int64_t)(index_zero_bytes(a->B) / 4);
@@ -736,18 +896,24 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
     AttnParams ap2;
     rc = make_attn(ap2, &d, a->seqs, queries, a->B, a->q, a->entries, idx, d.k, a->x, d.W, a->hca_entries, a->scale,
-                   a->out, a->lse, w + pl.off_attn, pl.items);
+                   a->out, a->lse, w + pl.off_attn, pl.items, a->norms);
     if (rc) return rc;
     // programmatic dependent launch chains append -> scan -> select -> attention -> merge unless
     // stage events are being recorded between them
     const bool pdl = ev[0] == nullptr && env_int("CSA_NO_PDL", 0) == 0;
     // every item in one launch after the top-k; the HCA items need no top-k and start as soon as the
-    // select kernel frees SMs
-    ap2.hca_nowait = pdl ? 1 : 0;
+    // scan frees SMs (their inputs, written by the append, are two launches back; with a reused
+    // selection the append is the launch right before, so they wait like the others)
+    ap2.hca_nowait = (pdl && !reuse) ? 1 : 0;
     ap2.hca_first = (pl.items.n_items > 1 && pl.items.items_front > 0) ? 1 : 0;
-    rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
-                   ws_index, false, st, stream, ev[2], pdl);
-    if (rc) return rc;
+    ap2.cluster = pl.cluster;
+    if (!reuse) {
+        rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
+                       ws_index, false, st, stream, ev[2], pdl, a->entries, a->keys_q, a->key_scales);
+        if (rc) return rc;
+    } else if ((e = mark(ev[2], stream)) != cudaSuccess) {
+        return cuda_fail(e, "event record");
+    }
     if ((e = mark(ev[3], stream)) != cudaSuccess) return cuda_fail(e, "event record");
     e = launch_attention_items(ap2, 0, pl.items.n_items, stream, pdl);
     if (e == cudaSuccess) e = launch_combine(ap2, stream, pdl);
@@ -764,13 +930,16 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
     if (a->q_begin < 0 || a->q_end <= a->q_begin || a->q_end > a->len)
         return fail(CSA_ERR_ARG, "query range [%lld, %lld) of len %lld", (long long)a->q_begin, (long long)a->q_end,
                     (long long)a->len);
+    const bool reuse = a->idx_in != nullptr;  // a selection reused from another layer: no indexer
     if (!a->seq || !a->x || !a->logit_c || !a->logit_h || !a->idx_key || !a->bias_c || !a->bias_h || !a->entries ||
-        !a->entry_keys || !a->hca_entries || !a->q || !a->q_idx || !a->w || !a->out)
+        !a->entry_keys || !a->hca_entries || !a->q || (!reuse && (!a->q_idx || !a->w)) || !a->out)
         return fail(CSA_ERR_ARG, "NULL pointer argument");
     if (!aligned16(a->x) || !aligned16(a->logit_c) || !aligned16(a->logit_h) || !aligned16(a->idx_key) ||
         !aligned16(a->bias_c) || !aligned16(a->bias_h) || !aligned16(a->entries) || !aligned16(a->entry_keys) ||
         !aligned16(a->hca_entries) || !aligned16(a->q) || !aligned16(a->q_idx) || !aligned16(a->out))
         return fail(CSA_ERR_ARG, "tensors must be 16-byte aligned");
+    if (reuse && a->idx_out) return fail(CSA_ERR_ARG, "idx_out with idx_in (the selection is the caller's)");
+    if ((rc = check_norms(d, a->norms))) return rc;
     const PrefillPlan pl = plan_prefill(d, a->q_end);
     if (!ws || ws_bytes < pl.total || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", pl.total);
@@ -780,7 +949,7 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
     if (a->compress) {
         // every CSA and HCA entry complete in [0, q_end): one pass over the raw rows
         rc = compress_all(d, a->seq, nullptr, 0, a->q_end, 1, a->q_end, a->x, a->logit_c, a->logit_h, a->bias_c,
-                          a->bias_h, a->idx_key, a->entries, a->entry_keys, a->hca_entries, st, stream);
+                          a->bias_h, a->idx_key, a->entries, a->entry_keys, a->hca_entries, a->norms, st, stream);
         if (rc) return rc;
     }
     char* w = static_cast<char*>(ws);
@@ -793,10 +962,13 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
         const int64_t n = a->q_end - p0 < pl.qc ? a->q_end - p0 : pl.qc;
         const int64_t r0 = p0 - a->q_begin;
         if ((e = launch_prefill_queries(queries, p0, n, stream)) != cudaSuccess) return cuda_fail(e, "query table");
-        int32_t* idx = a->idx_out ? a->idx_out + r0 * d.k : reinterpret_cast<int32_t*>(w + pl.off_idx);
+        int32_t* idx = reuse ? const_cast<int32_t*>(a->idx_in) + r0 * d.k
+                             : a->idx_out ? a->idx_out + r0 * d.k : reinterpret_cast<int32_t*>(w + pl.off_idx);
         // the chunk's queries see at most p0 + n tokens: size the indexer for that, not for q_end
         const int64_t max_e_chunk = (p0 + n) / d.m;
-        if (gemm_index) {
+        if (reuse) {
+            // the selection is the source layer's
+        } else if (gemm_index) {
             // scores of the whole chunk as one tensor-core GEMM, then a sampled-threshold select
             IndexParams ip{};
             ip.seqs = a->seq;
@@ -845,7 +1017,7 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
         ItemPlan one{1, 0, 64, 64};
         rc = make_attn(pp, &d, a->seq, queries, (int)n, a->q + r0 * d.H * d.d, a->entries, idx, d.k, a->x, d.W,
                        a->hca_entries, a->scale, a->out + r0 * d.H * d.d, a->lse ? a->lse + r0 * d.H : nullptr, nullptr,
-                       one);
+                       one, a->norms);
         if (rc) return rc;
         if ((rc = run_attention_all(pp, stream))) return rc;
     }

@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -70,15 +71,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns false (and records a
-// timeout) if it does not complete within kWaitLimitNs, or if *abort becomes non-zero.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort) {
+// timeout) if it does not complete within `limit_ns` (kWaitLimitNs unless a kernel was given a
+// shorter limit), or if *abort becomes non-zero.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0u) {
             if (abort && *abort) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 report(status, CSA_ERR_TIMEOUT);
                 if (abort) *abort = 1;
                 return false;
@@ -106,6 +109,29 @@ __device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void* src, ui
 // accesses (shared, distributed shared and global) before all later ones at cluster scope.
 __device__ __forceinline__ void cluster_barrier() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Distributed shared memory of the thread-block cluster: this CTA's rank, and loads of the word /
+// 16 bytes at the location `p` (an address in this CTA's shared memory) in the CTA of rank `rank`.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(const void* p, uint32_t rank) {
+    uint32_t a, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("ld.shared::cluster.b32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return __uint_as_float(v);
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(const void* p, uint32_t rank) {
+    uint32_t a;
+    float4 v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(a)
+                 : "memory");
+    return v;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -283,6 +309,46 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Eight bf16 values (one 16-byte vector) to fp32.
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x);
+    f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z);
+    f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+
+// 8-bit block-scaled keys: the 8 bf16 channels `kb` one lane holds of a 32-channel block that four
+// consecutive lanes of `mask` hold together -> 8 E4M3 bytes (the block's elements x / 2^e rounded to
+// nearest even) and, in *scale_byte, e + 127, where 2^e is the smallest power of two with
+// amax <= 448 * 2^e (amax = 0: e = -127).  All four lanes must call it.
+__device__ __forceinline__ uint2 quant_mx8(const uint4& kb, unsigned mask, uint32_t* scale_byte) {
+    float f[8];
+    unpack8(kb, f);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(mask, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(mask, amax, 2));
+    int e = -127;
+    if (amax > 0.f) {
+        int ex;
+        frexpf(amax, &ex);  // amax in [2^(ex-1), 2^ex)
+        e = ex - 9;
+        while (amax > ldexpf(448.f, e)) ++e;
+        while (e > -127 && amax <= ldexpf(448.f, e - 1)) --e;
+    }
+    *scale_byte = (uint32_t)(e + 127);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint16_t two;
+        // the first operand goes to the high byte: element 2i + 1 high, 2i low
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(two) : "f"(ldexpf(f[2 * i + 1], -e)), "f"(ldexpf(f[2 * i], -e)));
+        w[i] = two;
+    }
+    return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -66,7 +66,8 @@ struct TileSmem {
     static constexpr int kLh = kLc + kBoxBytes;
     static constexpr int kKi = kLh + kBoxBytes;       // d_I * 2 bytes per row (at most 128)
     static constexpr int kXs = kKi + kBoxBytes;       // HCA tree exchange: 8 warps x 8 groups x 24 floats
-    static constexpr int kBar = kXs + 8 * 8 * 24 * 4;
+    static constexpr int kSs = kXs + 8 * 8 * 24 * 4;  // per-entry sums of squares (normalization): 64 floats
+    static constexpr int kBar = kSs + 64 * 4;
     static constexpr int kTotal = kBar + 16;
     static constexpr int kAlloc = kTotal + 128;       // slack for 128-byte alignment
 };
@@ -107,6 +108,10 @@ __global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_cons
     const bool csa = p.do_csa && c_lo < c_hi;
     const bool hca = p.do_hca && h_lo < h_hi;
     if (!csa && !hca) return;
+    // once any CTA has given up on a wait, later CTAs do no work (bounded total time on a fault); not
+    // with normalization, where the CTAs of a cluster must all reach its barriers
+    if (!p.norm_c && !p.norm_h && p.status && *reinterpret_cast<volatile int*>(p.status) == CSA_ERR_TIMEOUT)
+        return;
     // rows [box0, box0 + kBoxRows) of the sequence cover every token the tile's entries use and end at
     // the last token used, so no row past the sequence's valid rows is read (negative rows read 0)
     const int64_t t_hi = max(csa ? 4 * c_hi : 0, hca ? (int64_t)mh * h_hi : 0);
@@ -130,31 +135,43 @@ __global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_cons
     __syncthreads();
     // the outcome is made CTA-uniform, so a timeout (recorded; nothing is written) never leaves some
     // threads at a barrier below without the others
-    if (!__syncthreads_and(mbar_wait(bar, 0, p.status, nullptr) ? 1 : 0)) return;
+    const bool norm = p.norm_c || p.norm_h;  // entry normalization: the slices exchange partial sums
+    const bool loaded = __syncthreads_and(mbar_wait(bar, 0, p.status, nullptr) ? 1 : 0) != 0;
+    // a timeout is recorded and nothing is written; with normalization the CTA still takes the
+    // cluster barriers below, which every CTA of the cluster must reach
+    if (!loaded && !norm) return;
 
     const uint16_t* sx = reinterpret_cast<const uint16_t*>(sm + TileSmem::kX);
     const uint16_t* slc = reinterpret_cast<const uint16_t*>(sm + TileSmem::kLc);
     const uint16_t* slh = reinterpret_cast<const uint16_t*>(sm + TileSmem::kLh);
     const uint16_t* ski = reinterpret_cast<const uint16_t*>(sm + TileSmem::kKi);
+    float* ss_c = reinterpret_cast<float*>(sm + TileSmem::kSs);       // [32] CSA entries of the tile
+    float* ss_h = ss_c + 32;                                          // [32] HCA entries of the tile
     const int c0 = slice * kSlice + g * 8;  // this thread's first channel
+    const int lane = tid & 31;
 
-    if (csa) {
-        const int64_t j = tt0 / 4 + u;
-        if (j >= c_lo && j < c_hi) {
-            const int rbase = (int)(4 * j - 4 - box0);  // smem row of window position 0
-            auto fetch = [&](int tensor, int pos) -> uint4 {
-                const int r = rbase + pos;
-                const uint16_t* base = tensor == 0 ? slc : tensor == 1 ? sx : ski;
-                const int stride = tensor == 2 ? p.d_I : kSlice;
-                return *reinterpret_cast<const uint4*>(base + r * stride + g * 8);
-            };
-            uint16_t* orow = p.entries + (sq.csa_off + j) * d + c0;
-            if (keys && c0 < p.d_I)
-                csa_entry_block4<true>(j, d, p.bias_c + c0, fetch, orow, p.entry_keys + (sq.csa_off + j) * p.d_I + c0);
-            else
-                csa_entry_block4<false>(j, d, p.bias_c + c0, fetch, orow, nullptr);
+    const int64_t j = tt0 / 4 + u;
+    const bool c_mine = loaded && csa && j >= c_lo && j < c_hi;
+    float cv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (c_mine) {
+        const int rbase = (int)(4 * j - 4 - box0);  // smem row of window position 0
+        auto fetch = [&](int tensor, int pos) -> uint4 {
+            const int r = rbase + pos;
+            const uint16_t* base = tensor == 0 ? slc : tensor == 1 ? sx : ski;
+            const int stride = tensor == 2 ? p.d_I : kSlice;
+            return *reinterpret_cast<const uint4*>(base + r * stride + g * 8);
+        };
+        if (keys && c0 < p.d_I) {
+            uint4 key;
+            csa_entry_block4<true>(j, d, p.bias_c + c0, fetch, cv, &key);
+            *reinterpret_cast<uint4*>(p.entry_keys + (sq.csa_off + j) * p.d_I + c0) = key;
+        } else {
+            csa_entry_block4<false>(j, d, p.bias_c + c0, fetch, cv, nullptr);
         }
     }
+    float hv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    bool h_mine = false;
+    int64_t h = 0;
     if (hca) {
         const int nb = mh / 4;  // blocks per HCA entry
         // block u's 4 tokens; blocks past the loaded rows belong to no entry this tile writes
@@ -170,11 +187,32 @@ __global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_cons
         Part8 P;
         part4<false>(lg, xv, kv, p.bias_h + (int64_t)((4 * u) & (mh - 1)) * d + c0, d, P);
         hca_tree(P, nb, xs);
-        const int64_t h = (tt0 + 4 * u) / mh;
-        const bool holder = (u & (nb - 1)) == 0 && (nb < 8 || (tid & 31) < 8);
-        if (holder && h >= h_lo && h < h_hi)
-            *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) = finish8(P.acc, P.den);
+        h = (tt0 + 4 * u) / mh;
+        const bool holder = (u & (nb - 1)) == 0 && (nb < 8 || lane < 8);
+        h_mine = loaded && holder && h >= h_lo && h < h_hi;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hv[i] = __fdiv_rn(P.acc[i], P.den[i]);
     }
+    float inv_c = 1.f, inv_h = 1.f;
+    if (norm) {
+        // partial sums of squares over this CTA's 64 channels, one per entry of the tile, then the
+        // totals over the cluster's slices
+        const float sc = sum_lane8(sumsq8(cv));
+        const float sh = sum_lane8(sumsq8(hv));
+        if (g == 0) {
+            ss_c[u] = sc;
+            if (h_mine) ss_h[h - tt0 / mh] = sh;
+        }
+        cluster_barrier();
+        const int ns = (int)gridDim.z;
+        if (c_mine && p.norm_c) inv_c = rms_inv(cluster_sum(ss_c + u, ns), d, p.eps);
+        if (h_mine && p.norm_h) inv_h = rms_inv(cluster_sum(ss_h + (h - tt0 / mh), ns), d, p.eps);
+        cluster_barrier();  // no CTA leaves while another still reads its shared memory
+    }
+    if (c_mine)
+        *reinterpret_cast<uint4*>(p.entries + (sq.csa_off + j) * d + c0) = entry_bf16(cv, p.norm_c ? p.norm_c + c0 : nullptr, inv_c);
+    if (h_mine)
+        *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) = entry_bf16(hv, p.norm_h ? p.norm_h + c0 : nullptr, inv_h);
 }
 
 }  // namespace
@@ -216,8 +254,11 @@ cudaError_t launch_compress_tiles(const TileCompressParams& p, int64_t max_span,
     int64_t span_tok = p.range_kind == 0 ? 4 * max_span : p.range_kind == 1 ? (int64_t)p.m_hca * max_span : max_span;
     const int64_t tiles = (span_tok + kTileTok - 1) / kTileTok + 1;  // the range may start inside a tile
     if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    return launch_kernel(compress_tile_kernel, dim3((unsigned)tiles, (unsigned)p.B, (unsigned)(p.d / kSlice)),
-                         dim3(256), TileSmem::kAlloc, stream, false, maps, p);
+    const dim3 grid((unsigned)tiles, (unsigned)p.B, (unsigned)(p.d / kSlice));
+    if (p.norm_c || p.norm_h)  // the slices of one tile form a cluster and exchange partial sums
+        return launch_kernel_cluster(compress_tile_kernel, grid, dim3(256), TileSmem::kAlloc, stream, false,
+                                     dim3(1, 1, (unsigned)(p.d / kSlice)), maps, p);
+    return launch_kernel(compress_tile_kernel, grid, dim3(256), TileSmem::kAlloc, stream, false, maps, p);
 }
 
 }  // namespace csa

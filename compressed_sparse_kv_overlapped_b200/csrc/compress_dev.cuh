@@ -12,13 +12,6 @@
 
 namespace csa {
 
-__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
-    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x);
-    f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
-    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z);
-    f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
-}
-
 // Channels [c0, c0+8) of entry j of one sequence (token rows start at tok0), written as bf16 to
 // out_row (+ c0) and, when key_row != nullptr, the indexer key channels to key_row (+ c0).
 // An online softmax over the window in fp32.  Tokens are taken 4 at a time: the loads of a batch
@@ -183,10 +176,11 @@ __device__ __forceinline__ void shfl_xor8(const Part8& A, Part8& B, int mask) {
 
 // CSA entry j (channels c0..c0+7) from the 8 rows of its window, rows fetched by fetch(tensor, t)
 // for window position t in 0..7 (tensor 0: logit, 1: latent, 2: indexer key).  j = 0 uses positions
-// 4..7 only.  Writes the entry (and, with keys, the indexer key) as bf16.
+// 4..7 only.  val gets the entry's fp32 values (acc / den, rounded once); with KEYS, *key gets the
+// indexer key as bf16.
 template <bool KEYS, typename Fetch>
-__device__ __forceinline__ void csa_entry_block4(int64_t j, int d, const float* bias_c0, Fetch fetch,
-                                                 uint16_t* out_row, uint16_t* key_row) {
+__device__ __forceinline__ void csa_entry_block4(int64_t j, int d, const float* bias_c0, Fetch fetch, float (&val)[8],
+                                                 uint4* key) {
     uint4 lg[4], xv[4], kv[4];
     Part8 cur;
 #pragma unroll
@@ -207,8 +201,65 @@ __device__ __forceinline__ void csa_entry_block4(int64_t j, int d, const float* 
         part4<KEYS>(lg, xv, kv, bias_c0, d, prev);
         merge8<KEYS>(cur, prev);
     }
-    *reinterpret_cast<uint4*>(out_row) = finish8(cur.acc, cur.den);
-    if (KEYS) *reinterpret_cast<uint4*>(key_row) = finish8(cur.acck, cur.den);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) val[i] = __fdiv_rn(cur.acc[i], cur.den[i]);
+    if (KEYS) *key = finish8(cur.acck, cur.den);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Optional RMS normalization of every compressed entry ("DeepSeek V4 comprimeix el context",
+// "CSA: buscar primer i atendre despres", last paragraph): out[c] = v[c] / sqrt(mean v^2 + eps) *
+// gain[c].  An entry's channels are spread over 8 lanes (8 channels each) of each of the d/64 CTAs
+// of a thread-block cluster; the sum of squares is added in a fixed order (each lane's 8 channels in
+// order, a butterfly over the 8 lanes, the CTAs by rank) by both the full pass and the append.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ float sumsq8(const float (&v)[8]) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s = __fmaf_rn(v[i], v[i], s);
+    return s;
+}
+
+// Sum over the 8 lanes of an aligned lane group (every lane of the warp takes part; each group of 8
+// ends with the same bits in all its lanes).
+__device__ __forceinline__ float sum_lane8(float s) {
+    s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 1));
+    s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 2));
+    s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 4));
+    return s;
+}
+
+__device__ __forceinline__ float rms_inv(float ss, int d, float eps) {
+    return __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)d), eps)));
+}
+
+// 8 entry values to bf16, normalized by inv * gain[c0 .. c0+7] when gain is given.
+__device__ __forceinline__ uint4 entry_bf16(const float (&v)[8], const float* gain_c0, float inv) {
+    float o[8];
+    if (gain_c0) {
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(gain_c0));
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(gain_c0) + 1);
+        const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = __fmul_rn(__fmul_rn(v[i], inv), g[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = v[i];
+    }
+    uint4 r;
+    r.x = pack_bf16x2(o[0], o[1]);
+    r.y = pack_bf16x2(o[2], o[3]);
+    r.z = pack_bf16x2(o[4], o[5]);
+    r.w = pack_bf16x2(o[6], o[7]);
+    return r;
+}
+
+// The total over the cluster's n CTAs of the value each holds at `p` (same offset in every CTA), in
+// rank order.
+__device__ __forceinline__ float cluster_sum(const float* p, int n) {
+    float s = 0.f;
+    for (int r = 0; r < n; ++r) s = __fadd_rn(s, ld_cluster_f32(p, (uint32_t)r));
+    return s;
 }
 
 // HCA entries of one 128-token tile, channels c0..c0+7: thread (u = tid / 8, g = tid % 8) of a

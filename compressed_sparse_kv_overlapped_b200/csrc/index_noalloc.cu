@@ -5,7 +5,7 @@
 // whose caching allocator owns every device buffer and forbids direct cudaMalloc, real-time
 // serving loops that must not allocate after start-up, or thin foreign-language bindings that see
 // only the caller's input and output pointers.  For them this entry point keeps its scratch in a
-// fixed array compiled into the library (kScratchBytes, about 12.1 MiB per device), so a call
+// fixed array compiled into the library (kScratchBytes, about 14.2 MiB per device), so a call
 // needs nothing but inputs, outputs and a stream.  The array occupies device memory on every GPU
 // that loads the library until the process exits.
 //
@@ -20,10 +20,15 @@ namespace {
 
 constexpr int kNoAllocMaxQ = 16;
 constexpr int64_t kNoAllocMaxSlots = int64_t(1) << 20;  // Q * score-row stride
-// Upper bound of index_ws_bytes(Q, e_stride) under the two limits above: histograms, fp32 scores
-// and the 64-bit kept-entry segments (each query's score row plus 128 entries).
-constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * kHistBins * 4 + 256 + size_t(kNoAllocMaxSlots) * 4 + 256 +
-                                 size_t(kNoAllocMaxSlots + kNoAllocMaxQ * 8 * kSelClusterMax) * 8 + 256;
+// Upper bound of index_ws_bytes(Q, e_stride) under the two limits above (each array rounded up to
+// 256 bytes): histograms and tickets; fp32 scores; 64-bit kept-entry segments (each query's score
+// row plus 128 entries); two words per scan chunk (chunks of at least 256 entries, one more per
+// query for a partial chunk); candidate keys (a quarter of the entries plus 256 per query).
+constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * (kHistBins + 1) * 4 + 256 +   // histograms, tickets
+                                 size_t(kNoAllocMaxSlots) * 4 + 256 +                  // scores
+                                 size_t(kNoAllocMaxSlots + kNoAllocMaxQ * kSegPad) * 8 + 256 +
+                                 2 * (size_t(kNoAllocMaxSlots / 256 + kNoAllocMaxQ) * 4 + 256) +
+                                 size_t(kNoAllocMaxSlots / 4 + kNoAllocMaxQ * 256) * 8 + 256;
 
 __device__ __align__(256) unsigned char g_index_scratch[kScratchBytes];
 

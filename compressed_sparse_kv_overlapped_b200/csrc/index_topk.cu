@@ -5,20 +5,20 @@
 // funcionen CSA i HCA", "CSA: buscar primer i atendre despres" (a light indexer scores every
 // compressed entry and only the best are attended).  Score (reading R3):
 //     s_j = sum_h w_h * relu(q^I_h . K^I_j),   j < floor(L / m);
-// top-k by (score desc, index asc), written in ascending index order, -1 past the end.
+// top-k by (score desc, index asc), written in ascending index order, -1 past the end.  Every
+// selection works on the 64-bit key (order-preserving score key << 32 | ~index), which is unique
+// and breaks ties to the lower index.
 //
 // Two kernels:
-//  scan   -- grid (chunks, queries).  Streams the indexer-key cache with coalesced 16-byte loads
-//            and computes the [16 entries x d_I] . [d_I x H_I] products on the tensor cores
-//            (mma.sync m16n8k16, K permuted so that every thread's operand is one contiguous
-//            16-byte load), applies relu / head weights in registers, writes the fp32 score and
-//            accumulates a coarse histogram of the top 11 bits of the order-preserving score key.
-//  select -- grid (filter CTAs, queries).  Every CTA finds the threshold bin from the histogram,
-//            sends its entries above it to the result list and those inside it to a candidate
-//            list; the last CTA of a query (ticket, no spinning) radix-selects the exact winners
-//            among the candidates on the 64-bit key (score key << 32 | ~index), which makes
-//            every key unique and breaks ties to the lower index, sorts the k indices and writes
-//            them.
+//  index_scan_kernel   -- grid (chunks, queries), the decode / standalone path.  Streams the
+//            indexer-key cache with coalesced 16-byte loads and computes the [16 entries x d_I] .
+//            [d_I x H_I] products on the tensor cores (mma.sync m16n8k16, K permuted so that every
+//            thread's operand is one contiguous 16-byte load), applies relu / head weights in
+//            registers, and counts the scores into the query's histogram of the top 11 key bits.
+//            Each chunk keeps its local candidates; the last chunk of a query to finish (atomic
+//            ticket, no spinning) selects the exact top-k from them (see the kernel).
+//  index_select_kernel -- one CTA per query, the prefill path: the top-k of a score row that the
+//            prefill GEMM stored, with a threshold bin estimated from a sample of the row.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -86,187 +86,92 @@ __device__ __forceinline__ void score16(const uint16_t* keys, int64_t r0, int64_
     s_hi = ph;
 }
 
-template <int KV>
-__global__ void __launch_bounds__(kScanThreads) index_scan_kernel(IndexParams p) {
-    __shared__ uint32_t hist[kHistBins];
-    __shared__ float sc[kScanThreads / 32][4][16];
-    grid_dep_wait();  // the query table may come from the previous kernel
-    grid_dep_launch();
-    const int qi = blockIdx.y;
-    const csa_query qr = p.queries[qi];
-    if (qr.seq < 0 || qr.reserved != 0) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, CSA_ERR_INDEX);
-        return;
-    }
-    const csa_seq sq = p.seqs[qr.seq];
-    if (qr.len < 1 || qr.len > sq.len) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, CSA_ERR_INDEX);
-        return;
-    }
-    const int64_t E = qr.len / p.m;
-    if (E <= p.k) return;  // everything is selected; the select kernel handles it alone
-    if (E > p.max_entries) {  // longer than the grid was sized for: the select kernel reports it
-        return;
-    }
-    const int64_t c0 = (int64_t)blockIdx.x * p.chunk;
-    if (c0 >= E) return;
-    const int64_t c1 = min(E, c0 + p.chunk);
-    for (int i = threadIdx.x; i < kHistBins; i += kScanThreads) hist[i] = 0u;
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, c = lane & 3;
-    // B fragments (query, permuted exactly like the key loads) and head weights
-    uint32_t bq[2 * KV][2];
-    float wv[2];
-    {
-        const uint16_t* qrow = p.q_idx + ((int64_t)qi * p.H_I + g) * p.d_I;
-        const bool hv = g < p.H_I;
-#pragma unroll
-        for (int v = 0; v < KV; ++v) {
-            uint4 t = hv ? *reinterpret_cast<const uint4*>(qrow + v * 32 + c * 8) : make_uint4(0, 0, 0, 0);
-            bq[2 * v][0] = t.x; bq[2 * v][1] = t.y;
-            bq[2 * v + 1][0] = t.z; bq[2 * v + 1][1] = t.w;
-        }
-        const int h0 = 2 * c, h1 = 2 * c + 1;
-        wv[0] = h0 < p.H_I ? p.w[(int64_t)qi * p.H_I + h0] : 0.f;
-        wv[1] = h1 < p.H_I ? p.w[(int64_t)qi * p.H_I + h1] : 0.f;
-    }
-    __syncthreads();
-
-    const uint16_t* keys = p.entry_keys + sq.csa_off * p.d_I;
-    float* srow = p.scores + (int64_t)qi * p.e_stride;
-    const uint64_t pol = policy_evict_first();
-    constexpr int kRowsPerPass = kScanThreads / 32 * 16 * 4;  // 512 entries: 4 groups of 16 per warp
-    for (int64_t base = c0; base < c1; base += kRowsPerPass) {
-        float s[4][2];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int64_t r0 = base + (int64_t)(u * (kScanThreads / 32) + warp) * 16;
-            score16<KV>(keys, r0, c1, g, c, bq, wv, pol, s[u][0], s[u][1]);
-        }
-        // stage in shared memory, then coalesced store + histogram
-        if (c == 0) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) { sc[warp][u][g] = s[u][0]; sc[warp][u][g + 8] = s[u][1]; }
-        }
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (lane < 16) {
-                const int64_t r = base + (int64_t)(u * (kScanThreads / 32) + warp) * 16 + lane;
-                if (r < c1) {
-                    const float v = sc[warp][u][lane];
-                    srow[r] = v;
-                    atomicAdd(&hist[float_key(v) >> 21], 1u);
-                }
-            }
-        }
-        __syncwarp();
-    }
-    __syncthreads();
-    uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
-    for (int i = threadIdx.x; i < kHistBins; i += kScanThreads)
-        if (hist[i]) atomicAdd(&gh[i], hist[i]);
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// ---- select ----------------------------------------------------------------------------------
-//
-// One thread-block cluster of F = sel_cluster CTAs per query (1..kSelClusterMax).  CTA c filters the scores of entries
-// [c*span, (c+1)*span): every CTA derives the threshold bin from the scan's histogram and keeps the
-// entries of that bin and above, as 64-bit keys in index order, in its own shared memory; it then
-// publishes its count in the leader CTA (rank 0).  After a cluster barrier every CTA knows its
-// offset and pushes its keys into the leader's list through distributed shared memory; after a
-// second barrier the leader radix-selects the exact threshold among the bin's members and
-// compacts the k indices, ascending.  A list longer than shared memory holds goes through the
-// global segment buffer instead, in the same order.
+// Streaming 8-byte load (see ld_stream).
+__device__ __forceinline__ uint2 ld_stream8(const void* p, uint64_t pol) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.u32 {%0,%1}, [%2], %3;"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p), "l"(pol));
+    return v;
+}
 
-constexpr int kSelPerMax = 64;                           // scores per thread per round
-constexpr int kSelBufMax = kSelPerMax * kSelectThreads;  // scores a CTA stages in shared memory per round
-constexpr int kStageSmem = 4096;  // kept keys a CTA stages in its own shared memory
-constexpr int kListSmem = 8192;   // kept keys the leader holds (in its score buffer, once filtered)
+// Two E4M3 values (low byte first) to two f16 values (exact: every E4M3 value is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "h"((unsigned short)two_bytes));
+    return r;
+}
+
+// Scores of 16 consecutive entries with 8-bit block-scaled keys (blocks of 32 channels, E4M3
+// elements, one power-of-two scale byte per block): thread (g, c) loads 8 bytes of each block for
+// rows g and g + 8, converts them to f16 (exact), and the products with the f16 query (each head
+// pre-scaled by a power of two 2^qsh[.], so it is exact in f16) accumulate per block in fp32; the
+// block scales and the query scale are applied exactly (powers of two) before relu.
+template <int NB>
+__device__ __forceinline__ void score16_mx8(const uint8_t* keys, const uint8_t* scales, int64_t r0, int64_t nrows,
+                                            int g, int c, const uint32_t (&bq)[2 * NB][2], const float (&wv)[2],
+                                            const int (&qsh)[2], uint64_t pol, float& s_lo, float& s_hi) {
+    constexpr int DI = 32 * NB;
+    uint2 lo[NB], hi[NB];
+    uint32_t sl = 0x7F7F7F7Fu, sh = 0x7F7F7F7Fu;  // scale bytes of rows g and g + 8 (2^0 past the end)
+    const int64_t rl = r0 + g, rh = r0 + g + 8;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        lo[b] = rl < nrows ? ld_stream8(keys + rl * DI + b * 32 + c * 8, pol) : make_uint2(0, 0);
+        hi[b] = rh < nrows ? ld_stream8(keys + rh * DI + b * 32 + c * 8, pol) : make_uint2(0, 0);
+    }
+    if (rl < nrows) sl = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rl * NB) : scales[rl];
+    if (rh < nrows) sh = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rh * NB) : scales[rh];
+    float tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const uint32_t l0 = e4m3x2_to_f16x2(lo[b].x), l1 = e4m3x2_to_f16x2(lo[b].x >> 16);
+        const uint32_t l2 = e4m3x2_to_f16x2(lo[b].y), l3 = e4m3x2_to_f16x2(lo[b].y >> 16);
+        const uint32_t h0 = e4m3x2_to_f16x2(hi[b].x), h1 = e4m3x2_to_f16x2(hi[b].x >> 16);
+        const uint32_t h2 = e4m3x2_to_f16x2(hi[b].y), h3 = e4m3x2_to_f16x2(hi[b].y >> 16);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t a0[4] = {l0, h0, l1, h1};
+        const uint32_t a1[4] = {l2, h2, l3, h3};
+        mma_f16_16816(acc, a0, bq[2 * b]);
+        mma_f16_16816(acc, a1, bq[2 * b + 1]);
+        const int el = (int)((sl >> (8 * b)) & 0xFFu) - 127, eh = (int)((sh >> (8 * b)) & 0xFFu) - 127;
+        tot[0] = __fadd_rn(tot[0], ldexpf(acc[0], el - qsh[0]));
+        tot[1] = __fadd_rn(tot[1], ldexpf(acc[1], el - qsh[1]));
+        tot[2] = __fadd_rn(tot[2], ldexpf(acc[2], eh - qsh[0]));
+        tot[3] = __fadd_rn(tot[3], ldexpf(acc[3], eh - qsh[1]));
+    }
+    float pl = wv[0] * fmaxf(tot[0], 0.f) + wv[1] * fmaxf(tot[1], 0.f);
+    float ph = wv[0] * fmaxf(tot[2], 0.f) + wv[1] * fmaxf(tot[3], 0.f);
+    pl += __shfl_xor_sync(0xffffffffu, pl, 1);
+    ph += __shfl_xor_sync(0xffffffffu, ph, 1);
+    pl += __shfl_xor_sync(0xffffffffu, pl, 2);
+    ph += __shfl_xor_sync(0xffffffffu, ph, 2);
+    s_lo = pl;
+    s_hi = ph;
+}
+
+// ---- block-wide helpers ---------------------------------------------------------------------
+
+// Bring `bytes` (a multiple of 16, 16-byte aligned) at `src` into L2 without waiting for them.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 __device__ __forceinline__ uint64_t composite(uint32_t key, int64_t j) {
     return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Every thread of every CTA of the cluster; orders all earlier memory accesses (shared, distributed
-// shared and global) before all later ones at cluster scope.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Address in the shared::cluster window of the location `p` (this CTA's shared memory) in CTA `rank`.
-__device__ __forceinline__ uint32_t map_rank(const void* p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_u64(uint32_t addr, uint64_t v) {
-    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-
-// Block-wide suffix sums over kHistBins bins: suf[b] = sum of hist[b' >= b].  Thread t owns bins
-// [4*(511-t), 4*(511-t)+4), so a forward scan over threads is a suffix scan over bins.  Also finds
-// the unique bin b with suf[b] >= target > suf[b+1] (target >= 1); writes it to out[0] and
-// suf[b+1] to out[1] (out[0] = 0xFFFFFFFF if no bin qualifies).  Uses kSelectThreads threads.
-__device__ void suffix_find(const uint32_t* hist, uint32_t* suf, uint32_t* warp_tot, uint32_t target,
-                            uint32_t* out) {
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int b0 = 4 * (kSelectThreads - 1 - t);
-    uint32_t v[4];
-    uint32_t s = 0;
-#pragma unroll
-    for (int i = 3; i >= 0; --i) { s += hist[b0 + i]; v[i] = s; }
-    uint32_t incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    if (t == 0) out[0] = 0xFFFFFFFFu;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t x = lane < kSelectThreads / 32 ? warp_tot[lane] : 0u;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane < kSelectThreads / 32) warp_tot[lane] = x;
-    }
-    __syncthreads();
-    const uint32_t before = (warp > 0 ? warp_tot[warp - 1] : 0u) + (incl - s);  // bins above b0+3
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t here = before + v[i];
-        const uint32_t above = i < 3 ? before + v[i + 1] : before;
-        suf[b0 + i] = here;
-        if (here >= target && above < target) { out[0] = (uint32_t)(b0 + i); out[1] = above; }
-    }
-    __syncthreads();
-}
-
-// Block-wide exclusive scan of one value per thread; returns this thread's exclusive prefix and
-// writes the total to *total.  `wsum` holds kSelectThreads/32 words.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
+// Exclusive prefix of one value per thread; *total gets the block's sum.  wsum: NT/32 words.
+template <int NT>
+__device__ __forceinline__ uint32_t excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t incl = v;
 #pragma unroll
@@ -277,44 +182,61 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        uint32_t x = lane < kSelectThreads / 32 ? wsum[lane] : 0u;
+        uint32_t x = lane < NT / 32 ? wsum[lane] : 0u;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
-        if (lane < kSelectThreads / 32) wsum[lane] = x;
+        if (lane < NT / 32) wsum[lane] = x;
     }
     __syncthreads();
     const uint32_t excl = (warp > 0 ? wsum[warp - 1] : 0u) + incl - v;
-    *total = wsum[kSelectThreads / 32 - 1];
+    *total = wsum[NT / 32 - 1];
     __syncthreads();
     return excl;
 }
 
-// The kept list of one query: the cluster CTAs' key runs concatenated in rank order (so in index
-// order), either gathered in the leader's shared memory (`cache`) or left in the global segment
-// buffer, where run c starts at seg + c*span and entry i lives in the last run c with off[c] <= i.
-struct KeptList {
-    const uint64_t* seg;
-    const uint32_t* off;     // [F + 1] exclusive prefix of the run lengths
-    int F;                   // CTAs in the cluster
-    int64_t span;
-    const uint64_t* cache;
+// Over kHistBins bins: the unique bin b with suffix(b) >= target > suffix(b + 1), where suffix(b) =
+// sum of hist[b' >= b] (target >= 1).  out[0] = b (0xFFFFFFFF if the total is below target),
+// out[1] = suffix(b + 1), out[2] = suffix(b).  Thread t owns kHistBins/NT consecutive bins counted
+// from the top, so a forward scan over threads is a suffix scan over bins.
+template <int NT>
+__device__ void find_bin(const uint32_t* hist, uint32_t target, uint32_t* wsum, uint32_t* out) {
+    constexpr int PER = kHistBins / NT;
+    const int t = threadIdx.x;
+    const int b0 = PER * (NT - 1 - t);  // bins [b0, b0 + PER)
+    uint32_t part = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) part += hist[b0 + i];
+    if (t == 0) out[0] = 0xFFFFFFFFu;
+    uint32_t total;
+    const uint32_t above_mine = excl_scan<NT>(part, wsum, &total);  // bins above b0 + PER - 1
+    uint32_t above = above_mine;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+        const uint32_t here = above + hist[b0 + i];
+        if (here >= target && above < target) { out[0] = (uint32_t)(b0 + i); out[1] = above; out[2] = here; }
+        above = here;
+    }
+    __syncthreads();
+}
+
+// A list of 64-bit keys, in shared or global memory.
+struct KeyList {
+    const uint64_t* smem;
+    const uint64_t* gmem;
     __device__ __forceinline__ uint64_t get(uint32_t i) const {
-        if (cache) return cache[i];
-        int c = 0;
-        for (int r = 1; r < F; ++r) c += off[r] <= i ? 1 : 0;
-        return __ldcg(reinterpret_cast<const unsigned long long*>(seg) + (int64_t)c * span + (i - off[c]));
+        return smem ? smem[i] : __ldcg(reinterpret_cast<const unsigned long long*>(gmem) + i);
     }
 };
 
-// Exact selection of the `need` largest keys among the list entries whose top 11 bits equal top11
-// (the threshold-bin members; entries of higher bins are kept regardless).  Returns T with exactly
-// `need` of those members >= T.  Radix passes of 11 bits over bits 52..0, counted with
-// shared-memory atomics; stops as soon as the chosen digit holds exactly the remaining count.
-__device__ uint64_t radix_threshold(const KeptList& L, uint32_t n, uint32_t need, uint32_t top11, uint32_t* cnt,
-                                    uint32_t* suf, uint32_t* misc) {
+// The key T with exactly `need` of the list's members of bin top11 (top 11 bits) at or above it:
+// radix passes of 11 bits below the top 11, counted with shared-memory atomics in cnt[kHistBins];
+// stops as soon as the chosen digit holds exactly the remaining count.
+template <int NT>
+__device__ uint64_t radix_select(const KeyList& L, uint32_t n, uint32_t need, uint32_t top11, uint32_t* cnt,
+                                 uint32_t* wsum, uint32_t* res) {
     uint64_t prefix = (uint64_t)top11 << 53;
     uint64_t mask = (uint64_t)0x7FF << 53;
     uint32_t remaining = need;
@@ -322,17 +244,15 @@ __device__ uint64_t radix_threshold(const KeptList& L, uint32_t n, uint32_t need
         const int sh = shift < 0 ? 0 : shift;
         const int bits = shift < 0 ? 11 + shift : 11;
         const uint32_t dmask = (1u << bits) - 1u;
-        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) cnt[i] = 0;
+        for (int i = threadIdx.x; i < kHistBins; i += NT) cnt[i] = 0;
         __syncthreads();
-        for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
+        for (uint32_t i = threadIdx.x; i < n; i += NT) {
             const uint64_t v = L.get(i);
             if ((v & mask) == prefix) atomicAdd(&cnt[(uint32_t)(v >> sh) & dmask], 1u);
         }
         __syncthreads();
-        suffix_find(cnt, suf, misc, remaining, misc + 48);  // misc[0..15]: warp totals
-        const uint32_t dg = misc[48];
-        const uint32_t above = misc[49];
-        const uint32_t in_digit = cnt[dg];
+        find_bin<NT>(cnt, remaining, wsum, res);
+        const uint32_t dg = res[0], above = res[1], in_digit = res[2] - res[1];
         __syncthreads();
         remaining -= above;
         prefix |= (uint64_t)dg << sh;
@@ -341,279 +261,188 @@ __device__ uint64_t radix_threshold(const KeptList& L, uint32_t n, uint32_t need
     }
 }
 
-// Dynamic shared memory of the select kernel.
-struct SelSmem {
-    static constexpr int kHist = 0;                          // u32[kHistBins]
-    static constexpr int kSuf = kHist + kHistBins * 4;       // u32[kHistBins]
-    static constexpr int kMisc = kSuf + kHistBins * 4;       // u32[64]
-    static constexpr int kXcnt = kMisc + 64 * 4;             // u32[32]: the leader's run lengths (| overflow bit)
-    static constexpr int kOffs = kXcnt + 32 * 4;             // u32[32]: exclusive prefix, F + 1 used
-    static constexpr int kStage = kOffs + 32 * 4;            // u64[kStageSmem]: this CTA's run
-    static constexpr int kBuf = kStage + kStageSmem * 8;     // f32[sel_buf] scores; the leader's list
-                                                             // (u64[kListSmem]) once it has filtered
-    // dynamic shared memory of a launch staging `buf` scores per round
-    static constexpr size_t bytes(int64_t buf) {
-        return (size_t)kBuf + (buf * 4 > (int64_t)kListSmem * 8 ? (size_t)buf * 4 : (size_t)kListSmem * 8);
+constexpr int kListKeys = 4096;                  // keys of the final list held in shared memory
+constexpr int kScanDynSmem = kListKeys * 8;      // dynamic shared memory: chunk scores, then the list
+static_assert(kScanDynSmem <= 48 * 1024, "no opt-in needed for the scan's dynamic shared memory");
+constexpr int64_t kScanChunkMax = kScanDynSmem / 4;
+static_assert(kScanChunkMax >= 512, "a chunk holds at least one pass of the scan");
+
+// Scores of the selected entries of a query that selects all of its E <= k entries (recomputed; E is
+// small), written to sout[0..E).
+__device__ void scores_of_all(const IndexParams& p, int qi, int64_t csa_off, int64_t E, float* sout) {
+    for (int64_t j = threadIdx.x; j < E; j += blockDim.x) {
+        float s = 0.f;
+        for (int h = 0; h < p.H_I; ++h) {
+            const uint16_t* qh = p.q_idx + ((int64_t)qi * p.H_I + h) * p.d_I;
+            float dot = 0.f;
+            for (int cc = 0; cc < p.d_I; ++cc) {
+                float k;
+                if (p.keys_q) {  // the dequantized 8-bit key: 2^e times the E4M3 value
+                    const uint32_t two = e4m3x2_to_f16x2(p.keys_q[(csa_off + j) * p.d_I + cc]);
+                    const int e = (int)p.key_scales[(csa_off + j) * (p.d_I / 32) + cc / 32] - 127;
+                    k = ldexpf(__low2float(*reinterpret_cast<const __half2*>(&two)), e);
+                } else {
+                    k = __uint_as_float((uint32_t)p.entry_keys[(csa_off + j) * p.d_I + cc] << 16);
+                }
+                dot = fmaf(__uint_as_float((uint32_t)qh[cc] << 16), k, dot);
+            }
+            s += p.w[(int64_t)qi * p.H_I + h] * fmaxf(dot, 0.f);
+        }
+        sout[j] = s;
     }
+}
+
+// 8-bit block-scaled copies of stored bf16 indexer keys: 8 threads per entry (4 per 32-channel block),
+// entries [r0, r1) of sequence b (ranges as csa_compress).
+__global__ void __launch_bounds__(256) quantize_keys_kernel(const csa_seq* seqs, const int64_t* ranges, int m, int d_I,
+                                                            const uint16_t* keys, uint8_t* keys_q, uint8_t* scales,
+                                                            int* status) {
+    const int b = blockIdx.y;
+    const int tpe = d_I / 8;  // threads per entry: 8 or 4
+    const int64_t e0 = ranges[2 * b], e1 = ranges[2 * b + 1];
+    const csa_seq sq = seqs[b];
+    if (e0 < 0 || e1 < e0 || (int64_t)m * e1 > sq.len) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) report(status, CSA_ERR_INDEX);
+        return;
+    }
+    const int lane = threadIdx.x & 31, sub = threadIdx.x / tpe, g = threadIdx.x % tpe;
+    const unsigned mask = 0xFu << (lane & ~3);
+    for (int64_t j = e0 + (int64_t)blockIdx.x * (256 / tpe) + sub; j < e1; j += (int64_t)gridDim.x * (256 / tpe)) {
+        const int64_t row = sq.csa_off + j;
+        const uint4 kb = *reinterpret_cast<const uint4*>(keys + row * d_I + 8 * g);
+        uint32_t sb;
+        const uint2 q = quant_mx8(kb, mask, &sb);
+        *reinterpret_cast<uint2*>(keys_q + row * d_I + 8 * g) = q;
+        if ((g & 3) == 0) scales[row * (d_I / 32) + g / 4] = (uint8_t)sb;
+    }
+}
+
+// ---- prefill select ---------------------------------------------------------------------------
+//
+// One CTA per query over a stored score row of at most kSelBufMax entries: the row is staged in
+// shared memory by bulk copies; a histogram of a strided sample of 4,096 scores gives a bin above
+// which about 2k/n of the sample lies, low enough that at least k entries pass it with overwhelming
+// probability; every entry of that bin and above is kept, in index order (the whole row instead if
+// fewer than k passed); the candidates' own histogram gives the exact threshold bin, a radix select
+// inside it the threshold, and the k indices are compacted in ascending order.
+
+constexpr int kSelPerMax = 64;                           // scores per thread
+constexpr int kSelBufMax = kSelPerMax * kSelectThreads;  // scores of one row (shared memory)
+constexpr int kSelListMax = 8192;                        // kept keys held in shared memory
+
+struct SelSmem {
+    static constexpr int kHist = 0;                         // u32[kHistBins]
+    static constexpr int kList = kHist + kHistBins * 4;     // u64[kSelListMax]
+    static constexpr int kBuf = kList + kSelListMax * 8;    // f32[buf]
+    static constexpr size_t bytes(int64_t buf) { return (size_t)kBuf + (size_t)buf * 4; }
 };
 
 __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kHist);
-    uint32_t* suf = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kSuf);
-    uint32_t* misc = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kMisc);
-    uint32_t* xcnt = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kXcnt);
-    uint32_t* offs = reinterpret_cast<uint32_t*>(smem_raw + SelSmem::kOffs);
-    uint64_t* stage = reinterpret_cast<uint64_t*>(smem_raw + SelSmem::kStage);
-    uint64_t* lst = reinterpret_cast<uint64_t*>(smem_raw + SelSmem::kBuf);
+    uint64_t* slist = reinterpret_cast<uint64_t*>(smem_raw + SelSmem::kList);
+    float* sbuf = reinterpret_cast<float*>(smem_raw + SelSmem::kBuf);
     __shared__ uint32_t s_wsum[kSelectThreads / 32];
+    __shared__ uint32_t s_res[4];
     __shared__ uint64_t s_bar;
-    __shared__ int s_abort;
-    grid_dep_wait();  // scores and histogram come from the scan kernel
+    grid_dep_wait();  // the scores come from the prefill GEMM
     grid_dep_launch();
-
-    // Every branch below that returns before the cluster barriers depends only on the query, so all
-    // CTAs of a cluster take it together.
-    const int qi = blockIdx.y;
-    const uint32_t rank = cluster_rank();
+    const int qi = blockIdx.x, tid = threadIdx.x;
     const csa_query qr = p.queries[qi];
     const bool seq_ok = qr.seq >= 0 && qr.reserved == 0;
     const csa_seq sq = seq_ok ? p.seqs[qr.seq] : csa_seq{0, 0, 0, 0};
     const bool valid = seq_ok && qr.len >= 1 && qr.len <= sq.len;
-    int64_t E = valid ? qr.len / p.m : 0;
-    if (E > p.max_entries || !seq_ok) {  // the launch was sized for fewer entries: refuse rather than guess
-        if (threadIdx.x == 0 && rank == 0) report(p.status, CSA_ERR_INDEX);
-        E = 0;
-    }
+    const int64_t E = valid ? qr.len / p.m : 0;
     int32_t* out = p.idx_out + (int64_t)qi * p.k;
     float* sout = p.score_out ? p.score_out + (int64_t)qi * p.k : nullptr;
-    const float* srow = p.scores + (int64_t)qi * p.e_stride;
-
-    if (E <= p.k) {  // select everything: no scores were computed
-        if (rank != 0) return;
-        for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
-            out[i] = i < E ? i : -1;
+    if (!valid || E > p.max_entries || E > kSelBufMax || E <= p.k) {
+        const bool bad = !valid || E > p.max_entries || E > kSelBufMax;
+        if (bad && tid == 0) report(p.status, CSA_ERR_INDEX);
+        const int64_t n = bad ? 0 : E;
+        for (int i = tid; i < p.k; i += kSelectThreads) {
+            out[i] = i < n ? i : -1;
             if (sout) sout[i] = __int_as_float(0x7FC00000);
         }
-        if (sout && E > 0) {
-            // scores of the selected entries (recomputed here; E <= k is small)
-            for (int64_t j = threadIdx.x; j < E; j += blockDim.x) {
-                const uint16_t* kr = p.entry_keys + (sq.csa_off + j) * p.d_I;
-                float s = 0.f;
-                for (int h = 0; h < p.H_I; ++h) {
-                    const uint16_t* qh = p.q_idx + ((int64_t)qi * p.H_I + h) * p.d_I;
-                    float dot = 0.f;
-                    for (int cc = 0; cc < p.d_I; ++cc)
-                        dot = fmaf(__uint_as_float((uint32_t)qh[cc] << 16), __uint_as_float((uint32_t)kr[cc] << 16), dot);
-                    s += p.w[(int64_t)qi * p.H_I + h] * fmaxf(dot, 0.f);
-                }
-                sout[j] = s;
-            }
+        if (sout && n > 0) {
+            __syncthreads();
+            scores_of_all(p, qi, sq.csa_off, n, sout);
         }
         return;
     }
-
-    const int F = p.sel_cluster;
-    const int64_t c0 = (int64_t)rank * p.sel_span;
-    const int64_t c1 = min(E, c0 + p.sel_span);
-    // Rounds of sel_buf scores are staged in shared memory by bulk copies (the first round's copy
-    // goes out before the histogram loads).
-    float* sbuf = reinterpret_cast<float*>(smem_raw + SelSmem::kBuf);
-    const uint32_t sbuf_addr = smem_u32(sbuf);
-    const int lane = threadIdx.x & 31;
-    const int L = p.sel_per;  // entries per thread per round: a power of two, 4..kSelPerMax
-    const int G = L / 4;
-    if (threadIdx.x == 0) {
+    const int n = (int)E;
+    const float* srow = p.scores + (int64_t)qi * p.e_stride;
+    // 1. the row into shared memory (bulk copies of the 16-byte-multiple part, then the tail)
+    const int n16 = n & ~3;
+    if (tid == 0) {
         mbar_init(&s_bar, 1);
         fence_mbar_init();
-        s_abort = 0;
-    }
-    __syncthreads();
-    // thread 0: copy the 16-byte-multiple part of round [rb, rb + n) into sbuf
-    auto issue_round = [&](int64_t rb) {
-        const int64_t n = min((int64_t)p.sel_buf, c1 - rb);
-        const uint32_t bytes = (uint32_t)(n & ~(int64_t)3) * 4u;
-        fence_proxy_async_smem();  // earlier generic accesses to sbuf come first
-        if (bytes == 0) {
-            mbar_arrive(&s_bar);
-            return;
-        }
+        const uint32_t bytes = (uint32_t)n16 * 4u;
         mbar_arrive_expect_tx(&s_bar, bytes);
         for (uint32_t off = 0; off < bytes; off += 65536u)
-            bulk_load(sbuf_addr + off, srow + rb + off / 4u, min(65536u, bytes - off), &s_bar);
-    };
-    if (threadIdx.x == 0 && c0 < c1) issue_round(c0);
-
-    uint64_t* gseg = p.seg + (int64_t)qi * p.e_seg + (int64_t)rank * p.sel_span;
-    uint32_t n_mine = 0;
-    bool spilled = false;  // the run lives in gseg instead of `stage`
-    bool failed = false;
-    // Keep the entries of [rb, rb + n) (staged in sbuf) whose bin is >= b_lo, appending them in
-    // index order to the run.  Thread t filters entries [t*L, t*L + L), reading its float4 groups in
-    // an order rotated by the lane so a warp's reads spread over all banks; bit 4*g + e of m64 flags
-    // entry 4*g + e of the thread's range.
-    auto filter_round = [&](int64_t rb, int64_t n, uint32_t b_lo) {
-        const float thr = key_float(b_lo << 21);  // the smallest float of bin b_lo (b_lo = 0: keep all)
-        const bool keep_all = b_lo == 0u;
-        const int64_t tb = (int64_t)threadIdx.x * L;
-        const int64_t valid = n - tb < 0 ? 0 : (n - tb > L ? L : n - tb);
-        uint64_t m64 = 0;
-        if (!failed && valid > 0) {
-            const float4* s4 = reinterpret_cast<const float4*>(sbuf + tb);
-#pragma unroll 4
-            for (int g = 0; g < G; ++g) {
-                const int gg = (g + lane) & (G - 1);
-                const float4 v = s4[gg];
-                // a float compare against the bin's lower edge passes every kept entry (the key is
-                // monotone in the float order); passes are confirmed on the exact key below, which
-                // also drops -0.0 below a +0.0 edge
-                const uint32_t m = keep_all ? 0xFu
-                                            : (v.x >= thr ? 1u : 0u) | (v.y >= thr ? 2u : 0u) |
-                                                  (v.z >= thr ? 4u : 0u) | (v.w >= thr ? 8u : 0u);
-                m64 |= (uint64_t)m << (4 * gg);
-            }
-            if (valid < 64) m64 &= (1ull << valid) - 1ull;
-            for (uint64_t c = m64; c; c &= c - 1ull) {
-                const int bit = __ffsll((long long)c) - 1;
-                if ((float_key(sbuf[tb + bit]) >> 21) < b_lo) m64 &= ~(1ull << bit);
-            }
-        }
-        uint32_t tot;
-        uint32_t pos = block_excl_scan((uint32_t)__popcll(m64), s_wsum, &tot);
-        if (!spilled && n_mine + tot > (uint32_t)kStageSmem) {
-            for (uint32_t i = threadIdx.x; i < n_mine; i += blockDim.x) gseg[i] = stage[i];
-            spilled = true;
-            __syncthreads();
-        }
-        pos += n_mine;
-        for (; m64; m64 &= m64 - 1ull) {
-            const int bit = __ffsll((long long)m64) - 1;
-            const uint64_t key = composite(float_key(sbuf[tb + bit]), rb + tb + bit);
-            if (spilled) gseg[pos] = key;
-            else stage[pos] = key;
-            ++pos;
-        }
-        n_mine += tot;
-        __syncthreads();
-    };
-
-    uint32_t b1, above, need, n_bin;
-    if (!p.sampled) {
-        // 1. threshold bin from the scan's histogram (every CTA of the query finds the same one)
-        const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
-        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = __ldcg(gh + i);
-        __syncthreads();
-        suffix_find(hist, suf, misc, (uint32_t)p.k, misc + 32);
-        b1 = misc[32];
-        above = misc[33];
-        need = (uint32_t)p.k - above;
-        n_bin = b1 == 0xFFFFFFFFu ? 0u : hist[b1];  // members of the threshold bin
-        failed = b1 == 0xFFFFFFFFu;                 // histogram holds fewer than k scores: cannot happen
-
-        // 2. keep this CTA's entries of bin >= b1, in index order, round by round
-        uint32_t phase = 0;
-        for (int64_t rb = c0; rb < c1; rb += p.sel_buf) {
-            const int64_t n = min((int64_t)p.sel_buf, c1 - rb);
-            const int64_t n16 = n & ~(int64_t)3;
-            if (threadIdx.x < n - n16) sbuf[n16 + threadIdx.x] = __ldg(srow + rb + n16 + threadIdx.x);
-            // a wait that runs out leaves this CTA's run empty (and the status word set); the CTA
-            // still takes both cluster barriers below
-            if (!mbar_wait(&s_bar, phase, p.status, &s_abort)) failed = true;
-            phase ^= 1u;
-            __syncthreads();
-            filter_round(rb, n, b1);  // ends with a barrier: sbuf is free again
-            if (threadIdx.x == 0 && rb + p.sel_buf < c1) issue_round(rb + p.sel_buf);
-        }
-    } else {
-        // No histogram (prefill GEMM scores; one CTA holds the query's whole row in one round).
-        // 1'. estimate a bin from a sample: the bin below which about 2k / n of the sample lies is
-        //     low enough that at least k entries pass it with overwhelming probability
-        const int64_t n = c1 - c0;
-        const int64_t n16 = n & ~(int64_t)3;
-        if (threadIdx.x < n - n16) sbuf[n16 + threadIdx.x] = __ldg(srow + c0 + n16 + threadIdx.x);
-        if (n > 0 && !mbar_wait(&s_bar, 0, p.status, &s_abort)) failed = true;
-        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0u;
-        __syncthreads();
-        const int64_t S = n < 4096 ? n : 4096;
-        for (int64_t i = threadIdx.x; i < S; i += blockDim.x)
-            atomicAdd(&hist[float_key(sbuf[(i * n) / S]) >> 21], 1u);
-        __syncthreads();
-        const int64_t want = (2 * (int64_t)p.k * S + n - 1) / (n > 0 ? n : 1);
-        suffix_find(hist, suf, misc, (uint32_t)(want < S ? want : S + 1), misc + 32);
-        uint32_t b_est = misc[32] == 0xFFFFFFFFu ? 0u : misc[32];  // no bin qualifies: keep everything
-        // 2'. candidates: every entry of bin >= b_est, in index order
-        filter_round(c0, n, b_est);
-        if (n_mine < (uint32_t)p.k && b_est > 0) {  // the estimate was too high (rare): keep everything
-            n_mine = 0;
-            spilled = false;
-            filter_round(c0, n, 0u);
-        }
-        // 3'. the exact threshold bin from the candidates' own histogram
-        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0u;
-        __syncthreads();
-        for (uint32_t i = threadIdx.x; i < n_mine; i += blockDim.x) {
-            const uint64_t key = spilled ? __ldcg(reinterpret_cast<const unsigned long long*>(gseg) + i) : stage[i];
-            atomicAdd(&hist[(uint32_t)(key >> 53)], 1u);
-        }
-        __syncthreads();
-        suffix_find(hist, suf, misc, (uint32_t)p.k, misc + 32);
-        b1 = misc[32];
-        above = misc[33];
-        need = (uint32_t)p.k - above;
-        n_bin = b1 == 0xFFFFFFFFu ? 0u : hist[b1];
-        if (b1 == 0xFFFFFFFFu) failed = true;
+            bulk_load(smem_u32(sbuf) + off, srow + off / 4u, min(65536u, bytes - off), &s_bar);
     }
-    if (failed) n_mine = 0;
-
-    // 3. run lengths to the leader, then every CTA learns its offset
-    if (threadIdx.x == 0) st_cluster_u32(map_rank(&xcnt[rank], 0), n_mine | (spilled ? 0x80000000u : 0u));
-    cluster_sync();
-    if (threadIdx.x < F) suf[threadIdx.x] = ld_cluster_u32(map_rank(&xcnt[threadIdx.x], 0));
+    if (tid < n - n16) sbuf[n16 + tid] = __ldg(srow + n16 + tid);
     __syncthreads();
-    uint32_t off_me = 0, total = 0;
-    bool any_spill = false;
-    for (int c = 0; c < F; ++c) {
-        const uint32_t v = suf[c];
-        if ((uint32_t)c < rank) off_me += v & 0x7FFFFFFFu;
-        if (threadIdx.x == 0) offs[c] = total;
-        total += v & 0x7FFFFFFFu;
-        any_spill |= (v >> 31) != 0u;
+    if (!__syncthreads_and(mbar_wait(&s_bar, 0, p.status, nullptr) ? 1 : 0)) return;  // timeout recorded
+    // 2. threshold bin estimated from a sample
+    for (int i = tid; i < kHistBins; i += kSelectThreads) hist[i] = 0u;
+    __syncthreads();
+    const int S = n < 4096 ? n : 4096;
+    for (int i = tid; i < S; i += kSelectThreads) atomicAdd(&hist[float_key(sbuf[((int64_t)i * n) / S]) >> 21], 1u);
+    __syncthreads();
+    const int64_t want = (2 * (int64_t)p.k * S + n - 1) / n;
+    find_bin<kSelectThreads>(hist, (uint32_t)(want < S ? want : S + 1), s_wsum, s_res);
+    uint32_t b_lo = s_res[0] == 0xFFFFFFFFu ? 0u : s_res[0];  // no bin qualifies: keep everything
+    // 3. candidates: the entries of bin >= b_lo in index order, in shared memory or (a long list) in
+    //    the query's global segment
+    const int L = (n + kSelectThreads - 1) / kSelectThreads;  // entries per thread
+    const int i0 = tid * L, i1 = min(n, i0 + L);
+    uint64_t* gseg = p.seg + (int64_t)qi * p.e_seg;
+    uint32_t n_cand = 0;
+    bool in_smem = true;
+    for (int pass = 0; pass < 2; ++pass) {
+        uint32_t mine = 0;
+        for (int i = i0; i < i1; ++i) mine += (float_key(sbuf[i]) >> 21) >= b_lo ? 1u : 0u;
+        uint32_t tot;
+        uint32_t o = excl_scan<kSelectThreads>(mine, s_wsum, &tot);
+        if (tot < (uint32_t)p.k && b_lo > 0) {  // the estimate was too high (rare): keep everything
+            b_lo = 0;
+            continue;
+        }
+        in_smem = tot <= (uint32_t)kSelListMax;
+        uint64_t* dst = in_smem ? slist : gseg;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t key = float_key(sbuf[i]);
+            if ((key >> 21) >= b_lo) dst[o++] = composite(key, i);
+        }
+        n_cand = tot;
+        break;
     }
-    if (threadIdx.x == 0) offs[F] = total;
-    // every CTA has read the histogram: clear it for the next call, one share per CTA
-    {
-        uint32_t* ghw = p.hist + (int64_t)qi * kHistBins;
-        const int share = kHistBins / F;
-        for (int i = threadIdx.x; i < share; i += blockDim.x) ghw[rank * share + i] = 0u;
-    }
-    const bool in_smem = !any_spill && total <= (uint32_t)kListSmem;
-    if (in_smem) {
-        // the leader's score buffer is free (its filter is done, no copy in flight): it becomes the list
-        const uint32_t dst = map_rank(lst + off_me, 0);
-        for (uint32_t i = threadIdx.x; i < n_mine; i += blockDim.x) st_cluster_u64(dst + i * 8u, stage[i]);
-    } else if (!spilled) {
-        for (uint32_t i = threadIdx.x; i < n_mine; i += blockDim.x) gseg[i] = stage[i];
-    }
-    cluster_sync();
-    if (rank != 0) return;
-
-    // 4. the leader: exact threshold, then compaction in index order
-    const uint32_t n_tot = total;
-    // without sampling the kept list is exactly the entries of bins >= b1; with it, a superset
-    if (b1 == 0xFFFFFFFFu || (p.sampled ? n_tot < above + n_bin : n_tot != above + n_bin)) {
-        if (threadIdx.x == 0) report(p.status, CSA_ERR_INDEX);
+    __syncthreads();
+    // 4. the exact threshold bin from the candidates' own histogram, then the radix select
+    const KeyList KL{in_smem ? slist : nullptr, in_smem ? nullptr : gseg};
+    for (int i = tid; i < kHistBins; i += kSelectThreads) hist[i] = 0u;
+    __syncthreads();
+    for (uint32_t i = tid; i < n_cand; i += kSelectThreads) atomicAdd(&hist[(uint32_t)(KL.get(i) >> 53)], 1u);
+    __syncthreads();
+    find_bin<kSelectThreads>(hist, (uint32_t)p.k, s_wsum, s_res);
+    const uint32_t b1 = s_res[0], above = s_res[1], n_bin = s_res[2] - s_res[1];
+    if (b1 == 0xFFFFFFFFu) {  // fewer than k candidates: cannot happen (the whole row was kept)
+        if (tid == 0) report(p.status, CSA_ERR_INDEX);
         return;
     }
-    const KeptList kl{p.seg + (int64_t)qi * p.e_seg, offs, F, p.sel_span, in_smem ? lst : nullptr};
-    const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53) : radix_threshold(kl, n_tot, need, b1, hist, suf, misc);
-    const uint32_t per_t = (n_tot + blockDim.x - 1) / blockDim.x;
-    const uint32_t i0 = threadIdx.x * per_t, i1 = min(n_tot, i0 + per_t);
+    const uint32_t need = (uint32_t)p.k - above;
+    const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53)
+                                     : radix_select<kSelectThreads>(KL, n_cand, need, b1, hist, s_wsum, s_res);
+    // 5. compaction in index order
+    const uint32_t per_t = (n_cand + kSelectThreads - 1) / kSelectThreads;
+    const uint32_t j0 = tid * per_t, j1 = min(n_cand, j0 + per_t);
     uint32_t mine = 0;
-    for (uint32_t i = i0; i < i1; ++i) mine += kl.get(i) >= T ? 1u : 0u;
+    for (uint32_t i = j0; i < j1; ++i) mine += KL.get(i) >= T ? 1u : 0u;
     uint32_t kept_total;
-    uint32_t o = block_excl_scan(mine, s_wsum, &kept_total);
-    for (uint32_t i = i0; i < i1; ++i) {
-        const uint64_t v = kl.get(i);
+    uint32_t o = excl_scan<kSelectThreads>(mine, s_wsum, &kept_total);
+    for (uint32_t i = j0; i < j1; ++i) {
+        const uint64_t v = KL.get(i);
         if (v >= T) {
             if (o < (uint32_t)p.k) {
                 out[o] = (int32_t)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
@@ -622,106 +451,416 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
             ++o;
         }
     }
-    if (threadIdx.x == 0 && kept_total != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
+    if (tid == 0 && kept_total != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
+}
+
+// ---- decode scan ------------------------------------------------------------------------------------
+//
+// Scan CTA (chunk c, query qi): the scores of entries [c*chunk, min(E, (c+1)*chunk)) on the tensor
+// cores, written to the score row and kept in shared memory, counted into the query's histogram of
+// the top 11 bits of the order-preserving score key; then the chunk's candidates -- its entries of
+// bin >= b_c, b_c the highest bin that still leaves at least kloc entries (kloc about twice the
+// chunk's expected share of the top-k) -- go to the candidate buffer in index order, with b_c.
+// The last CTA of the query to finish (atomic ticket; nothing waits) selects the exact top-k:
+// the threshold bin b1 of the query's histogram fixes the members of bins >= b1, which are exactly
+// the entries it must consider; a chunk with b_c <= b1 holds all of its members among its
+// candidates, a chunk with b_c > b1 (more than its share of the top-k) is filtered again from its
+// stored scores.  A radix select inside bin b1 on the 64-bit key (score key << 32 | ~index: unique,
+// ties to the lower index) gives the threshold, and the k indices are compacted in ascending order.
+template <int KV, bool MX8>
+__global__ void __launch_bounds__(kScanThreads, 4) index_scan_kernel(IndexParams p) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ uint32_t hist[kHistBins];
+    __shared__ float sc[kScanThreads / 32][4][16];
+    __shared__ uint32_t s_wsum[kScanThreads / 32];
+    __shared__ uint32_t s_res[4];
+    __shared__ int s_last;
+    float* ssc = reinterpret_cast<float*>(dsm);  // the chunk's scores
+    grid_dep_wait();  // the query table may come from the previous kernel
+    grid_dep_launch();
+    const int qi = blockIdx.y;
+    const int tid = threadIdx.x;
+    const csa_query qr = p.queries[qi];
+    const bool seq_ok = qr.seq >= 0 && qr.reserved == 0;
+    const csa_seq sq = seq_ok ? p.seqs[qr.seq] : csa_seq{0, 0, 0, 0};
+    const bool valid = seq_ok && qr.len >= 1 && qr.len <= sq.len;
+    const int64_t E = valid ? qr.len / p.m : 0;
+    int32_t* out = p.idx_out + (int64_t)qi * p.k;
+    float* sout = p.score_out ? p.score_out + (int64_t)qi * p.k : nullptr;
+    if (!valid || E > p.max_entries || E <= p.k) {
+        // an invalid query (reported, nothing selected) or one that selects everything: chunk 0 alone
+        if (blockIdx.x != 0) return;
+        const bool bad = !valid || E > p.max_entries;
+        if (bad && tid == 0) report(p.status, CSA_ERR_INDEX);
+        const int64_t n = bad ? 0 : E;
+        for (int i = tid; i < p.k; i += kScanThreads) {
+            out[i] = i < n ? i : -1;
+            if (sout) sout[i] = __int_as_float(0x7FC00000);
+        }
+        if (sout && n > 0) {
+            __syncthreads();
+            scores_of_all(p, qi, sq.csa_off, n, sout);
+        }
+        return;
+    }
+    const int64_t chunk = p.chunk;
+    const int nch = (int)((E + chunk - 1) / chunk);
+    const int cidx = blockIdx.x;
+    if (cidx >= nch) return;
+    const int64_t c0 = (int64_t)cidx * chunk;
+    const int64_t c1 = min(E, c0 + chunk);
+    for (int i = tid; i < kHistBins; i += kScanThreads) hist[i] = 0u;
+
+    const int lane = tid & 31, warp = tid >> 5;
+    {
+        const int g = lane >> 2, c = lane & 3;
+        // B fragments (query, permuted exactly like the key loads) and head weights
+        uint32_t bq[2 * KV][2];
+        float wv[2];
+        int qsh[2] = {0, 0};  // 8-bit keys: the power-of-two pre-scale of heads 2c and 2c + 1
+        const uint16_t* qrow = p.q_idx + ((int64_t)qi * p.H_I + g) * p.d_I;
+        const bool hv = g < p.H_I;
+        uint4 qv[KV];
+#pragma unroll
+        for (int v = 0; v < KV; ++v)
+            qv[v] = hv ? *reinterpret_cast<const uint4*>(qrow + v * 32 + c * 8) : make_uint4(0, 0, 0, 0);
+        if (!MX8) {
+#pragma unroll
+            for (int v = 0; v < KV; ++v) {
+                bq[2 * v][0] = qv[v].x; bq[2 * v][1] = qv[v].y;
+                bq[2 * v + 1][0] = qv[v].z; bq[2 * v + 1][1] = qv[v].w;
+            }
+        } else {
+            // head g's query in f16, scaled by 2^s with s chosen so that its largest magnitude lies in
+            // [2^14, 2^15): exact in f16 (down to 2^-31 of that magnitude) and far from overflow
+            float f[KV][8];
+            float amax = 0.f;
+#pragma unroll
+            for (int v = 0; v < KV; ++v) {
+                unpack8(qv[v], f[v]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[v][i]));
+            }
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            int ex = 0;
+            if (amax > 0.f) frexpf(amax, &ex);  // amax in [2^(ex-1), 2^ex)
+            const int sg = amax > 0.f ? 15 - ex : 0;
+#pragma unroll
+            for (int v = 0; v < KV; ++v) {
+                uint32_t h[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __half2 t = __floats2half2_rn(ldexpf(f[v][2 * i], sg), ldexpf(f[v][2 * i + 1], sg));
+                    h[i] = *reinterpret_cast<const uint32_t*>(&t);
+                }
+                bq[2 * v][0] = h[0]; bq[2 * v][1] = h[1];
+                bq[2 * v + 1][0] = h[2]; bq[2 * v + 1][1] = h[3];
+            }
+            // heads 2c and 2c + 1 live in the quads of rows 2c and 2c + 1
+            qsh[0] = __shfl_sync(0xffffffffu, sg, (2 * c) * 4);
+            qsh[1] = __shfl_sync(0xffffffffu, sg, (2 * c + 1) * 4);
+        }
+        const int h0 = 2 * c, h1 = 2 * c + 1;
+        wv[0] = h0 < p.H_I ? p.w[(int64_t)qi * p.H_I + h0] : 0.f;
+        wv[1] = h1 < p.H_I ? p.w[(int64_t)qi * p.H_I + h1] : 0.f;
+        __syncthreads();
+
+        const uint16_t* keys = p.entry_keys + sq.csa_off * p.d_I;
+        float* srow = p.scores + (int64_t)qi * p.e_stride;
+        const uint64_t pol = policy_evict_first();
+        constexpr int kRowsPerPass = kScanThreads / 32 * 16 * 4;  // 512 entries: 4 groups of 16 per warp
+        for (int64_t base = c0; base < c1; base += kRowsPerPass) {
+            float s[4][2];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t r0 = base + (int64_t)(u * (kScanThreads / 32) + warp) * 16;
+                if (MX8)
+                    score16_mx8<KV>(p.keys_q + sq.csa_off * p.d_I, p.key_scales + sq.csa_off * KV, r0, c1, g, c, bq,
+                                    wv, qsh, pol, s[u][0], s[u][1]);
+                else
+                    score16<KV>(keys, r0, c1, g, c, bq, wv, pol, s[u][0], s[u][1]);
+            }
+            // stage in shared memory, then coalesced store + histogram
+            if (c == 0) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) { sc[warp][u][g] = s[u][0]; sc[warp][u][g + 8] = s[u][1]; }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (lane < 16) {
+                    const int64_t r = base + (int64_t)(u * (kScanThreads / 32) + warp) * 16 + lane;
+                    if (r < c1) {
+                        const float v = sc[warp][u][lane];
+                        srow[r] = v;
+                        ssc[r - c0] = v;
+                        atomicAdd(&hist[float_key(v) >> 21], 1u);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    {
+        uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
+        for (int i = tid; i < kHistBins; i += kScanThreads)
+            if (hist[i]) atomicAdd(&gh[i], hist[i]);
+    }
+    // ---- the chunk's candidates
+    const int n = (int)(c1 - c0);
+    const int cap = p.cand_cap;
+    const int64_t kloc64 = (2 * (int64_t)p.k * n + E - 1) / E + 16;
+    const uint32_t kloc = (uint32_t)min((int64_t)cap, min((int64_t)n, kloc64));
+    find_bin<kScanThreads>(hist, kloc, s_wsum, s_res);
+    uint32_t bc = s_res[0] == 0xFFFFFFFFu ? 0u : s_res[0];
+    if (s_res[0] != 0xFFFFFFFFu && s_res[2] > (uint32_t)cap) bc += 1;  // suffix(bc + 1) < kloc <= cap
+    {
+        const int per = (n + kScanThreads - 1) / kScanThreads;
+        const int i0 = tid * per, i1 = min(n, i0 + per);
+        uint32_t mine = 0;
+        for (int i = i0; i < i1; ++i) mine += (float_key(ssc[i]) >> 21) >= bc ? 1u : 0u;
+        uint32_t tot;
+        uint32_t o = excl_scan<kScanThreads>(mine, s_wsum, &tot);
+        uint64_t* cand = p.cand + ((int64_t)qi * p.max_chunks + cidx) * cap;
+        for (int i = i0; i < i1; ++i) {
+            const uint32_t key = float_key(ssc[i]);
+            if ((key >> 21) >= bc) cand[o++] = composite(key, c0 + i);
+        }
+        if (tid == 0) p.meta[(int64_t)qi * p.max_chunks + cidx] = (bc << 16) | tot;
+    }
+    // ---- ticket: the last chunk of the query to finish selects
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&p.ticket[qi], 1u) == (uint32_t)(nch - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // 1. the threshold bin of the whole query
+    {
+        const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
+        for (int i = tid; i < kHistBins; i += kScanThreads) hist[i] = __ldcg(gh + i);
+    }
+    __syncthreads();
+    find_bin<kScanThreads>(hist, (uint32_t)p.k, s_wsum, s_res);
+    const uint32_t b1 = s_res[0], above = s_res[1], at = s_res[2];
+    if (b1 == 0xFFFFFFFFu) {  // the histogram holds fewer than k scores: cannot happen for E > k
+        if (tid == 0) report(p.status, CSA_ERR_INDEX);
+        return;
+    }
+    const uint32_t n_bin = at - above, need = (uint32_t)p.k - above;
+    // 2. members of bins >= b1, chunk by chunk in index order: counts (written over the chunk's meta
+    //    word), then offsets, then the list
+    const uint32_t* meta = p.meta + (int64_t)qi * p.max_chunks;
+    uint32_t* cnt_g = p.coff + (int64_t)qi * p.max_chunks;  // per chunk: count, then offset
+    const float* srow = p.scores + (int64_t)qi * p.e_stride;
+    const uint64_t* cand_q = p.cand + (int64_t)qi * p.max_chunks * cap;
+    auto chunk_items = [&](int c, uint32_t mw, bool count_only, uint32_t off, uint64_t* dst) -> uint32_t {
+        // one warp: the chunk's members of bins >= b1, in index order
+        const uint32_t bcc = mw >> 16, nc = mw & 0xFFFFu;
+        uint32_t found = 0;
+        if (bcc <= b1) {
+            const uint64_t* cd = cand_q + (int64_t)c * cap;
+            for (uint32_t i0 = 0; i0 < nc; i0 += 32) {
+                const uint32_t i = i0 + lane;
+                const uint64_t v = i < nc ? __ldcg(reinterpret_cast<const unsigned long long*>(cd) + i) : 0ull;
+                const bool hit = i < nc && (uint32_t)(v >> 53) >= b1;
+                const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+                if (!count_only && hit) dst[off + found + __popc(bal & ((1u << lane) - 1u))] = v;
+                found += __popc(bal);
+            }
+        } else {
+            const int64_t e0 = (int64_t)c * chunk, e1 = min(E, e0 + chunk);
+            for (int64_t j0 = e0; j0 < e1; j0 += 32) {
+                const int64_t j = j0 + lane;
+                const uint32_t key = j < e1 ? float_key(__ldcg(srow + j)) : 0u;
+                const bool hit = j < e1 && (key >> 21) >= b1;
+                const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+                if (!count_only && hit) dst[off + found + __popc(bal & ((1u << lane) - 1u))] = composite(key, j);
+                found += __popc(bal);
+            }
+        }
+        return found;
+    };
+    // pass A: counts, one warp per chunk
+    __shared__ uint32_t s_tot;
+    for (int c = warp; c < nch; c += kScanThreads / 32) {
+        const uint32_t f = chunk_items(c, __ldcg(meta + c), true, 0, nullptr);
+        if (lane == 0) cnt_g[c] = f;
+    }
+    __threadfence_block();
+    __syncthreads();
+    // offsets: exclusive scan over the chunk counts, kScanThreads chunks at a time (in place)
+    {
+        uint32_t carry = 0;
+        for (int cb = 0; cb < nch; cb += kScanThreads) {
+            const int c = cb + tid;
+            const uint32_t v = c < nch ? __ldcg(cnt_g + c) : 0u;
+            uint32_t tot;
+            const uint32_t ex = excl_scan<kScanThreads>(v, s_wsum, &tot);
+            if (c < nch) cnt_g[c] = carry + ex;
+            carry += tot;
+        }
+        if (tid == 0) s_tot = carry;
+    }
+    __threadfence_block();
+    __syncthreads();
+    const uint32_t n_tot = s_tot;
+    if (n_tot != at) {  // the members must be exactly the histogram's count of bins >= b1
+        if (tid == 0) report(p.status, CSA_ERR_INDEX);
+        return;
+    }
+    const bool in_smem = n_tot <= (uint32_t)kListKeys;
+    uint64_t* lst = in_smem ? reinterpret_cast<uint64_t*>(dsm) : p.seg + (int64_t)qi * p.e_seg;
+    // pass B: the list
+    for (int c = warp; c < nch; c += kScanThreads / 32) chunk_items(c, __ldcg(meta + c), false, __ldcg(cnt_g + c), lst);
+    __threadfence_block();
+    __syncthreads();
+    // 3. the exact threshold inside bin b1, then compaction in index order
+    const KeyList L{in_smem ? lst : nullptr, in_smem ? nullptr : lst};
+    const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53) : radix_select<kScanThreads>(L, n_tot, need, b1, hist,
+                                                                                          s_wsum, s_res);
+    const uint32_t per_t = (n_tot + kScanThreads - 1) / kScanThreads;
+    const uint32_t i0 = tid * per_t, i1 = min(n_tot, i0 + per_t);
+    uint32_t mine = 0;
+    for (uint32_t i = i0; i < i1; ++i) mine += L.get(i) >= T ? 1u : 0u;
+    uint32_t kept_total;
+    uint32_t o = excl_scan<kScanThreads>(mine, s_wsum, &kept_total);
+    for (uint32_t i = i0; i < i1; ++i) {
+        const uint64_t v = L.get(i);
+        if (v >= T) {
+            if (o < (uint32_t)p.k) {
+                const uint32_t j = 0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull);
+                out[o] = (int32_t)j;
+                if (sout) sout[o] = key_float((uint32_t)(v >> 32));
+                // the attention that follows gathers these rows: start bringing them into L2 now
+                if (p.prefetch_rows) prefetch_l2(p.prefetch_rows + (sq.csa_off + j) * p.prefetch_row_bytes,
+                                                 p.prefetch_row_bytes);
+            }
+            ++o;
+        }
+    }
+    if (tid == 0 && kept_total != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
 }
 
 constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 }  // namespace
 
-cudaError_t select_attrs() {
-    static PerDeviceOnce attr;
-    return attr.run([] {
-        cudaError_t e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SelSmem::bytes(kSelBufMax));
-        if (e != cudaSuccess) return e;
-        return cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    });
+namespace {
+
+// Scan chunking of Q queries of up to e_stride entries: chunks of a multiple of 64 entries sized so
+// that all chunks make about one wave of four scan CTAs per SM (so SMs carry equal shares), at least
+// 256 and at most what the chunk's score buffer in shared memory holds.
+struct ScanPlan {
+    int64_t chunk;
+    int max_chunks;
+    int cap;
+};
+
+ScanPlan scan_plan(int Q, int64_t e_stride) {
+    constexpr int64_t kSlots = 148 * 4;
+    ScanPlan sp;
+    int64_t c = (e_stride * Q + kSlots - 1) / kSlots;
+    c = ((c + 63) / 64) * 64;
+    if (c < 256) c = 256;
+    if (c > kScanChunkMax) c = kScanChunkMax;
+    sp.chunk = c;
+    sp.max_chunks = (int)((e_stride + c - 1) / c);
+    sp.cap = (int)(c / 4 < 256 ? c / 4 : 256);
+    return sp;
 }
 
+// Per-chunk words and candidate keys are sized by bounds that hold for every chunk size the plan
+// can choose (chunks of at least 256 entries keeping at most a quarter of their entries, at most
+// 256), so the workspace of Q queries also serves any smaller query count.
+size_t chunk_words(int Q, int64_t e_stride) { return (size_t)Q * (size_t)(e_stride / 256 + 1); }
+size_t cand_keys(int Q, int64_t e_stride) { return (size_t)Q * (size_t)(e_stride / 4 + 256); }
+
+}  // namespace
+
+size_t index_zero_bytes(int Q) { return align256((size_t)Q * (kHistBins + 1) * 4); }
+
 size_t index_ws_bytes(int Q, int64_t e_stride) {
-    size_t s = 0;
-    s += align256((size_t)Q * kHistBins * 4);
+    size_t s = index_zero_bytes(Q);
     s += align256((size_t)Q * e_stride * 4);
-    s += align256((size_t)Q * (e_stride + 8 * kSelClusterMax) * 8);
+    s += align256((size_t)Q * (e_stride + kSegPad) * 8);
+    s += 2 * align256(chunk_words(Q, e_stride) * 4);
+    s += align256(cand_keys(Q, e_stride) * 8);
     return s;
 }
 
-size_t index_zero_bytes(int Q) { return align256((size_t)Q * kHistBins * 4); }
-
 void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
+    const ScanPlan sp = scan_plan(Q, e_stride);
     char* b = static_cast<char*>(ws);
     p.hist = reinterpret_cast<uint32_t*>(b);
-    b += align256((size_t)Q * kHistBins * 4);
+    p.ticket = p.hist + (size_t)Q * kHistBins;
+    b += index_zero_bytes(Q);
     p.scores = reinterpret_cast<float*>(b);
     b += align256((size_t)Q * e_stride * 4);
     p.seg = reinterpret_cast<uint64_t*>(b);
+    b += align256((size_t)Q * (e_stride + kSegPad) * 8);
+    p.meta = reinterpret_cast<uint32_t*>(b);
+    b += align256(chunk_words(Q, e_stride) * 4);
+    p.coff = reinterpret_cast<uint32_t*>(b);
+    b += align256(chunk_words(Q, e_stride) * 4);
+    p.cand = reinterpret_cast<uint64_t*>(b);
     p.e_stride = e_stride;
-    p.e_seg = e_stride + 8 * kSelClusterMax;
+    p.e_seg = e_stride + kSegPad;
+    p.chunk = sp.chunk;
+    p.max_chunks = sp.max_chunks;
+    p.cand_cap = sp.cap;
 }
 
 cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
                               cudaEvent_t mid, bool pdl, bool sampled) {
-    p.sampled = sampled ? 1 : 0;
     if (sampled) {
         // scores are already in p.scores; one select CTA per query holds its whole row
         if (max_entries > kSelBufMax) return cudaErrorInvalidValue;
-        p.sel_cluster = 1;
-        p.sel_span = ((max_entries + 7) / 8) * 8;
-        if (p.sel_span < 8) p.sel_span = 8;
-        int per = 4;
-        while (per < kSelPerMax && (int64_t)per * kSelectThreads < p.sel_span) per *= 2;
-        p.sel_per = per;
-        p.sel_buf = per * kSelectThreads;
-        const size_t smem = SelSmem::bytes(p.sel_buf);
-        cudaError_t e = select_attrs();
+        const int64_t buf = ((max_entries + 3) / 4) * 4;
+        const size_t smem = SelSmem::bytes(buf < 4 ? 4 : buf);
+        static PerDeviceOnce attr;
+        cudaError_t e = attr.run([] {
+            return cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)SelSmem::bytes(kSelBufMax));
+        });
         if (e != cudaSuccess) return e;
-        return launch_kernel_cluster(index_select_kernel, dim3(1, (unsigned)p.Q), dim3(kSelectThreads), smem, stream,
-                                     pdl, dim3(1, 1, 1), p);
+        return launch_kernel(index_select_kernel, dim3((unsigned)p.Q), dim3(kSelectThreads), smem, stream, pdl, p);
     }
     if (zero_ws) {
-        // the histogram sits at the start of the workspace
+        // the histograms and tickets sit at the start of the workspace
         cudaError_t e = cudaMemsetAsync(p.hist, 0, index_zero_bytes(p.Q), stream);
         if (e != cudaSuccess) return e;
     }
-    if (max_entries > p.k) {
-        const int64_t total = max_entries * (int64_t)p.Q;
-        // aim for ~4 scan CTAs per SM over all queries, chunks of 512..16384 entries
-        int64_t chunk = (total + 148 * 4 - 1) / (148 * 4);
-        chunk = ((chunk + 511) / 512) * 512;
-        if (chunk < 512) chunk = 512;
-        if (chunk > 16384) chunk = 16384;
-        p.chunk = chunk;
-        const int64_t gx = (max_entries + chunk - 1) / chunk;
-        cudaError_t e = p.d_I == 64
-                            ? launch_kernel(index_scan_kernel<2>, dim3((unsigned)gx, (unsigned)p.Q), dim3(kScanThreads), 0,
-                                            stream, pdl && !zero_ws, p)
-                            : launch_kernel(index_scan_kernel<1>, dim3((unsigned)gx, (unsigned)p.Q), dim3(kScanThreads), 0,
-                                            stream, pdl && !zero_ws, p);
-        if (e != cudaSuccess) return e;
-    }
-    if (mid) {
-        cudaError_t e = cudaEventRecordWithFlags(mid, stream, cudaEventRecordExternal);
-        if (e != cudaSuccess) return e;
-    }
-    // cluster size: about two select CTAs per SM over all queries, 1..kSelClusterMax CTAs per query
-    int F = 1;
-    while (F < kSelClusterMax && (int64_t)p.Q * F * 2 <= 2 * 148) F *= 2;
-    p.sel_cluster = F;
-    p.sel_span = (((p.e_stride + F - 1) / F + 7) / 8) * 8;  // F * span <= e_stride + 8F <= e_seg
-    // scores per thread per round: the smallest power of two that covers the CTA's span in one
-    // round, 4..kSelPerMax; the round buffer holds that many per thread
-    int per = 4;
-    while (per < kSelPerMax && (int64_t)per * kSelectThreads < p.sel_span) per *= 2;
-    p.sel_per = per;
-    p.sel_buf = per * kSelectThreads;
-    const int64_t buf = p.sel_buf;
-    const size_t smem = SelSmem::bytes(buf);
-    cudaError_t ea = select_attrs();
-    if (ea != cudaSuccess) return ea;
-    // after an event record the select follows the scan without overlap
-    return launch_kernel_cluster(index_select_kernel, dim3((unsigned)F, (unsigned)p.Q), dim3(kSelectThreads), smem,
-                                 stream, pdl && mid == nullptr, dim3((unsigned)F, 1, 1), p);
+    cudaError_t e;
+    // chunk 0 of a query that selects all of its entries writes the result alone
+    const int64_t gx = max_entries > p.k ? (max_entries + p.chunk - 1) / p.chunk : 1;
+    if (gx > p.max_chunks) return cudaErrorInvalidValue;  // the workspace was carved for fewer entries
+    const dim3 grid((unsigned)gx, (unsigned)p.Q);
+    const bool dep = pdl && !zero_ws;
+    if (p.keys_q)
+        e = p.d_I == 64 ? launch_kernel(index_scan_kernel<2, true>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p)
+                        : launch_kernel(index_scan_kernel<1, true>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p);
+    else
+        e = p.d_I == 64 ? launch_kernel(index_scan_kernel<2, false>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p)
+                        : launch_kernel(index_scan_kernel<1, false>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p);
+    if (e != cudaSuccess) return e;
+    if (mid) return cudaEventRecordWithFlags(mid, stream, cudaEventRecordExternal);
+    return cudaSuccess;
+}
+
+cudaError_t launch_quantize_keys(const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries, int m,
+                                 int d_I, const uint16_t* keys, uint8_t* keys_q, uint8_t* scales, int* status,
+                                 cudaStream_t stream) {
+    if (max_entries <= 0) return cudaSuccess;
+    const int per_cta = 256 / (d_I / 8);
+    int64_t gx = (max_entries + per_cta - 1) / per_cta;
+    if (gx > 8192) gx = 8192;
+    quantize_keys_kernel<<<dim3((unsigned)gx, (unsigned)B), 256, 0, stream>>>(seqs, ranges, m, d_I, keys, keys_q,
+                                                                             scales, status);
+    return cudaGetLastError();
 }
 
 }  // namespace csa

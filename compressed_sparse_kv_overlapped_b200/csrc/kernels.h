@@ -51,6 +51,9 @@ struct TileCompressParams {
     uint16_t* entries;
     uint16_t* entry_keys;
     uint16_t* hca_entries;
+    const float* norm_c;      // [d] RMS-normalization gain of the CSA entries (nullable)
+    const float* norm_h;      // [d] the same for the HCA entries (nullable)
+    float eps;
     int* status;
 };
 // max_span: host bound of each sequence's range length, in the range's own units.
@@ -59,7 +62,7 @@ cudaError_t launch_compress_tiles(const TileCompressParams& p, int64_t max_span,
 // Indexer score scan + top-k select.
 constexpr int kHistBins = 2048;  // coarse histogram over the top 11 bits of the score key
 constexpr int kMaxK = 2048;
-constexpr int kSelClusterMax = 16;  // most CTAs (one thread-block cluster) per query in the select kernel
+constexpr int kSegPad = 128;  // keys of slack past each score row in the segment buffer
 
 struct IndexParams {
     const csa_seq* seqs;
@@ -68,20 +71,26 @@ struct IndexParams {
     const uint16_t* q_idx;    // [Q, H_I, d_I]
     const float* w;           // [Q, H_I]
     const uint16_t* entry_keys;
+    const uint8_t* keys_q;      // nullable: 8-bit block-scaled keys [*, d_I] E4M3 (scored instead of entry_keys)
+    const uint8_t* key_scales;  // [*, d_I / 32] biased power-of-two exponents of keys_q
     int64_t chunk;            // entries per scan CTA
     int64_t max_entries;      // host bound of floor(L/m) over all queries (grid sizing)
     int64_t e_stride;         // row stride of the score buffer
-    int64_t sel_span;         // entries per select CTA (multiple of 8)
-    int64_t e_seg;            // row stride of the segment buffer (e_stride + 8 * kSelClusterMax)
-    int sel_cluster;          // select CTAs per query (a power of two, at most kSelClusterMax)
-    int sel_per;              // scores per select thread per round (a power of two)
-    int sel_buf;              // scores a select CTA stages in shared memory per round
-    int sampled;              // 1: no scan histogram; one select CTA per query estimates its threshold
-                              // bin from a sample of its scores (requires a row to fit one round)
+    int64_t e_seg;            // row stride of the segment buffer (e_stride + 128)
+    int max_chunks;           // scan chunks per query the workspace holds (ceil(e_stride / chunk))
+    int cand_cap;             // candidate keys a scan chunk may keep
     // workspace
     float* scores;            // [Q, e_stride]
-    uint32_t* hist;           // [Q, kHistBins]; zero between calls (the select kernel clears it)
+    uint32_t* hist;           // [Q, kHistBins]; zero before the scan
+    uint32_t* ticket;         // [Q] finished scan chunks; zero before the scan
     uint64_t* seg;            // [Q, e_seg] kept entries (64-bit keys) when they exceed shared memory
+    uint32_t* meta;           // [Q, max_chunks] per scan chunk: (threshold bin << 16) | candidate count
+    uint32_t* coff;           // [Q, max_chunks] per scan chunk: member count, then list offset
+    uint64_t* cand;           // [Q, max_chunks, cand_cap] candidate keys of each chunk, in index order
+    // optional: rows of this cache (row stride prefetch_row_bytes, a multiple of 16) at the selected
+    // entries are prefetched into L2 as soon as the selection is known (the attention's gather)
+    const unsigned char* prefetch_rows;
+    int64_t prefetch_row_bytes;
     // outputs
     int32_t* idx_out;         // [Q, k]
     float* score_out;         // [Q, k] nullable
@@ -89,7 +98,14 @@ struct IndexParams {
 };
 size_t index_ws_bytes(int Q, int64_t e_stride);
 size_t index_zero_bytes(int Q);  // leading bytes of the index workspace that must start at zero
+// Points the workspace arrays of `p` into `ws` and sets the scan chunking (chunk, max_chunks,
+// cand_cap), all derived from (Q, e_stride) exactly as index_ws_bytes sizes them.
 void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride);
+// 8-bit block-scaled copies (keys_q [*, d_I] E4M3, scales [*, d_I / 32]) of the stored bf16 indexer
+// keys of entries [ranges[b][0], ranges[b][1]) of every sequence.
+cudaError_t launch_quantize_keys(const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries, int m,
+                                 int d_I, const uint16_t* keys, uint8_t* keys_q, uint8_t* scales, int* status,
+                                 cudaStream_t stream);
 // Prefill indexer scores as a tensor-core GEMM (d_I = 64, H_I <= 4): chunk rows [0, Qn) are the
 // consecutive positions pos0, pos0 + 1, ... of one sequence; row r's causal entries (j < (pos0 + r +
 // 1) / m) get scores[r * e_stride + j].
@@ -108,9 +124,9 @@ struct PrefillScoreParams {
 cudaError_t launch_prefill_scores(const PrefillScoreParams& p, int64_t max_entries, cudaStream_t stream,
                                   bool pdl = false);
 
-// `mid` (nullable): event recorded between the scan and the select kernels.
-// `sampled`: p.scores already holds the scores (prefill GEMM), no scan and no histogram; every row
-// must hold at most kSelRowMax entries.
+// `mid` (nullable): event recorded after the scan kernel (which also selects).
+// `sampled`: p.scores already holds the scores (prefill GEMM): no scan, the select kernel takes each
+// row's top-k with a sampled threshold; every row must hold at most kSelRowMax entries.
 constexpr int64_t kSelRowMax = 32768;
 cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t stream, bool zero_ws,
                               cudaEvent_t mid = nullptr, bool pdl = false, bool sampled = false);
@@ -131,6 +147,10 @@ struct AttnParams {
     int m_hca;
     int use_hca;
     float scale_log2;           // scale * log2(e)
+    const float* sink;          // [H] attention-sink logits (nullable): one more softmax term per head
+                                // with a zero value, joined where the query's softmax is complete
+    const float* q_norm;        // [d] RMS-normalization gain of every query head (nullable)
+    float norm_eps;
     // Items.  n_items == 1: one item covers the whole list (direct output, no merge).  Otherwise
     // items [0, items_front) cut the front part [0, k_slots + W) into chunks of kpi_front keys and
     // items [items_front, n_items) cut the HCA part into chunks of kpi_hca keys; every item writes
@@ -147,9 +167,19 @@ struct AttnParams {
     // they take the free SMs before the front items (which wait for the top-k) do.  Launches all
     // items of all queries.
     int hca_first;
+    // > 1: the launch forms thread-block clusters of `cluster` consecutive items of one query (the
+    // item counts of both parts are multiples of it); the CTAs of a cluster merge their results
+    // through distributed shared memory and store one partial per cluster, so part_o holds
+    // n_items / cluster partials per query
+    int cluster;
     // 1: full key tiles that are contiguous rows of the HCA cache / of the raw window are loaded by
     // TMA (set by the launcher when the tensor maps could be encoded)
     int tma_hca, tma_x;
+    // fault injection for the tests of the bounded waits (csa_debug_inject): 1 = the first loader
+    // warp does not arrive on the first key tile's barrier, so the tile never becomes full; wait_ns =
+    // the limit of every wait in the kernel
+    int debug_fault;
+    uint64_t wait_ns;
     // outputs
     float* out;                 // [Q, H, d]
     float* lse;                 // [Q, H] nullable
@@ -182,6 +212,11 @@ struct AppendParams {
     uint16_t* entries;
     uint16_t* entry_keys;
     uint16_t* hca_entries;
+    uint8_t* keys_q;         // nullable: 8-bit block-scaled copy of each new indexer key
+    uint8_t* key_scales;
+    const float* norm_c;     // [d] RMS-normalization gains of new CSA / HCA entries (nullable)
+    const float* norm_h;
+    float eps;
     csa_query* queries;      // [B] out
     uint32_t* zero_words;    // index workspace words to clear (nullable)
     int64_t n_zero_words;
@@ -195,6 +230,10 @@ cudaError_t launch_prefill_queries(csa_query* queries, int64_t p0, int64_t n, cu
 // Address of the device status word on the current device: CSA_OK, or an error code (with the
 // message recorded for csa_last_error) when it cannot be looked up.
 int device_status(int** out);
+
+// Fault injection state (csa_debug_inject): the fault code and the wait limit in nanoseconds the
+// next attention launches use.
+void debug_fault_state(int* fault, uint64_t* wait_ns);
 
 // Error reporting shared by entry points defined outside capi.cu.
 int validate_dims(const csa_dims* d);             // CSA_OK or the error code (message set)

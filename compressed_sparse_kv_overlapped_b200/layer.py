@@ -15,12 +15,17 @@ The caller fills the raw-token rows (and the parameters); ``compress`` builds th
 """
 from __future__ import annotations
 
-from . import (CSA_OP_DECODE, CSA_OP_PREFILL, csa_compress, csa_compress_all, csa_decode_args, csa_prefill_args,
-               csa_workspace_size, hybrid_attn_decode, hybrid_attn_prefill)
+import ctypes
+
+from . import (CSA_OP_DECODE, CSA_OP_PREFILL, csa_compress, csa_compress_all, csa_decode_args, csa_norms,
+               csa_prefill_args, csa_quantize_keys, csa_workspace_size, hybrid_attn_decode, hybrid_attn_prefill)
 
 
 class HybridLayer:
-    def __init__(self, dims, capacity, device="cuda"):
+    """key_format "mx8" adds 8-bit block-scaled copies of the indexer keys (keys_q [*, d_I] E4M3,
+    key_scales [*, d_I / 32]) that the decode's indexer scores instead of the bf16 keys."""
+
+    def __init__(self, dims, capacity, device="cuda", key_format="bf16"):
         import torch
 
         self.dims = dims
@@ -45,12 +50,28 @@ class HybridLayer:
         self.entries = torch.zeros(max(c, 1), d, dtype=bf, device=device)
         self.entry_keys = torch.zeros(max(c, 1), dI, dtype=bf, device=device)
         self.hca_entries = torch.zeros(max(h, 1), d, dtype=bf, device=device)
+        if key_format not in ("bf16", "mx8"):
+            raise ValueError(f"key_format {key_format!r}")
+        self.key_format = key_format
+        self.keys_q = self.key_scales = None
+        if key_format == "mx8":
+            self.keys_q = torch.zeros(max(c, 1), dI, dtype=torch.uint8, device=device)
+            self.key_scales = torch.zeros(max(c, 1), dI // 32, dtype=torch.uint8, device=device)
         self.bias_c = torch.zeros(2 * m, d, dtype=torch.float32, device=device)
         self.bias_h = torch.zeros(mh, d, dtype=torch.float32, device=device)
         self.seqs = torch.tensor([[tok[b], csa[b], hca[b], 0] for b in range(self.B)], dtype=torch.int64,
                                  device=device)
         self.lens = [0] * self.B
         self.device = device
+        self.norms = None  # optional csa_norms (set_norms)
+
+    # ---- normalization and sinks ----------------------------------------------------------------
+    def set_norms(self, q_norm=None, entry_norm_c=None, entry_norm_h=None, sink=None, eps=1e-6) -> None:
+        """Optional query / entry RMS-normalization gains ([d] fp32) and sink logits ([H] fp32), device
+        tensors kept by the layer; every later compress, decode and prefill uses them."""
+        from . import make_norms
+        self._norm_tensors = (q_norm, entry_norm_c, entry_norm_h, sink)
+        self.norms = make_norms(q_norm, entry_norm_c, entry_norm_h, sink, eps)
 
     # ---- lengths ------------------------------------------------------------------------------
     def set_lengths(self, lens) -> None:
@@ -68,8 +89,20 @@ class HybridLayer:
         if max(self.lens) > 0:
             csa_compress_all(self.dims, self.seqs, rt, self.B, max(self.lens), self.x, self.logit_c, self.logit_h,
                              self.bias_c, self.bias_h, self.idx_key, self.entries, self.entry_keys,
-                             self.hca_entries, stream)
+                             self.hca_entries, stream, norms=self.norms)
+        if self.keys_q is not None:
+            self.quantize_keys(stream)
         self._keep = rt  # the kernels read the range table asynchronously
+
+    def quantize_keys(self, stream=None) -> None:
+        """The 8-bit copies of every complete entry's indexer key (key_format "mx8")."""
+        import torch
+        d = self.dims
+        rq = torch.tensor([[0, n // d.m] for n in self.lens], dtype=torch.int64, device=self.device)
+        if max(n // d.m for n in self.lens) > 0:
+            csa_quantize_keys(d, self.seqs, rq, self.B, max(n // d.m for n in self.lens), self.entry_keys, self.keys_q,
+                              self.key_scales, stream)
+        self._keep_q = rq
 
     def compress_separately(self, stream=None) -> None:
         """The same caches through two csa_compress calls (CSA entries with their keys, then HCA)."""
@@ -86,7 +119,7 @@ class HybridLayer:
 
     # ---- decode -------------------------------------------------------------------------------
     def decode_args(self, q, q_idx, w, out, append=True, lse=None, idx_out=None, max_len=None,
-                    scale=None, new_rows=None) -> csa_decode_args:
+                    scale=None, new_rows=None, idx_in=None) -> csa_decode_args:
         """Arguments of one decode step.  With append, the new token's raw rows either are already in
         the caches at row tok_off + len (new_rows None) or come as new_rows [B, 3d + d_I] bf16
         (x | logit_c | logit_h | idx_key per sequence) and the call writes them there."""
@@ -101,8 +134,11 @@ class HybridLayer:
                         ("idx_key", self.idx_key), ("bias_c", self.bias_c), ("bias_h", self.bias_h),
                         ("entries", self.entries), ("entry_keys", self.entry_keys),
                         ("hca_entries", self.hca_entries), ("q", q), ("q_idx", q_idx), ("w", w), ("out", out),
-                        ("lse", lse), ("idx_out", idx_out), ("new_rows", new_rows)):
+                        ("lse", lse), ("idx_out", idx_out), ("new_rows", new_rows), ("keys_q", self.keys_q),
+                        ("key_scales", self.key_scales), ("idx_in", idx_in)):
             setattr(a, name, None if t is None else t.data_ptr())
+        if self.norms is not None:
+            a.norms = ctypes.pointer(self.norms)
         return a
 
     def decode_workspace(self, max_len=None):
@@ -121,7 +157,7 @@ class HybridLayer:
 
     # ---- prefill (sequence 0) -----------------------------------------------------------------
     def prefill_args(self, q, q_idx, w, out, q_begin, q_end, compress=True, lse=None, idx_out=None,
-                     scale=None) -> csa_prefill_args:
+                     scale=None, idx_in=None) -> csa_prefill_args:
         d = self.dims
         a = csa_prefill_args()
         a.dims = d
@@ -134,8 +170,10 @@ class HybridLayer:
                         ("idx_key", self.idx_key), ("bias_c", self.bias_c), ("bias_h", self.bias_h),
                         ("entries", self.entries), ("entry_keys", self.entry_keys),
                         ("hca_entries", self.hca_entries), ("q", q), ("q_idx", q_idx), ("w", w), ("out", out),
-                        ("lse", lse), ("idx_out", idx_out)):
+                        ("lse", lse), ("idx_out", idx_out), ("idx_in", idx_in)):
             setattr(a, name, None if t is None else t.data_ptr())
+        if self.norms is not None:
+            a.norms = ctypes.pointer(self.norms)
         return a
 
     def prefill_workspace(self, q_end):

@@ -94,6 +94,29 @@ typedef struct csa_query {
     int64_t len;      /* visible length L, 1 <= L <= seqs[seq].len */
 } csa_query;
 
+/* f3 -- optional normalization and sink parameters of a layer ("DeepSeek V4 comprimeix el context",
+ * "CSA: buscar primer i atendre despres", last paragraph: queries and compressed entries are
+ * normalized to stabilize the logits, and learned attention-sink logits absorb excess attention).
+ * Read on the host during a call; every pointer is device memory (fp32, 16-byte aligned) or NULL,
+ * which turns that part off.
+ *  q_norm:       [d] gain of the RMS normalization of each query head, q / sqrt(mean q^2 + eps) *
+ *                gain, applied before the logits (the normalized query is rounded to bf16).
+ *  entry_norm_c: [d] gain of the same normalization of every CSA entry as it is compressed (the
+ *                stored entry, key and value of the attention, is the normalized one); the raw
+ *                window and the indexer keys are not normalized.  Needs m = 4.
+ *  entry_norm_h: [d] the same for the HCA entries.  Needs m_hca a power of two from 4 to 128.
+ *  sink:         [H] the sink logit z_h of each head: one more term of the head's (merged) softmax
+ *                with a zero value, lse' = log(e^lse + e^z), out' = out * e^(lse - lse').
+ *  eps:          the normalization's epsilon. */
+typedef struct csa_norms {
+    const float* q_norm;
+    const float* entry_norm_c;
+    const float* entry_norm_h;
+    const float* sink;
+    float eps;
+    int32_t reserved; /* must be 0 */
+} csa_norms;
+
 /* a1/a2 -- token-axis compressor ("DeepSeek V4 comprimeix el context", sections "DeepSeek
  * comprimeix la dimensio temporal" and "Finestres solapades per evitar fronteres artificials";
  * "Frontier Techniques", 2.1 and 2.2).
@@ -117,12 +140,13 @@ int csa_compress(const csa_dims* dims, int which, const csa_seq* seqs, const int
  * entries whose last token lies in [t0, t1).  With m = 4 and m_hca a power of two from 4 to 128 each
  * raw row (x, both logit arrays, idx_key) is read once for both caches; other ratios run the two
  * caches one after the other.  max_tokens: host bound of t1 - t0 over the sequences (sizes the
- * grid).  Entries equal those of csa_compress and of the decode append bit for bit.  A range outside
- * [0, seqs[b].len] is reported as CSA_ERR_INDEX on the device. */
+ * grid).  Entries equal those of csa_compress and of the decode append bit for bit.  norms (host
+ * struct, nullable): only entry_norm_c / entry_norm_h / eps are used (normalized entries; csa_compress
+ * has no normalization).  A range outside [0, seqs[b].len] is reported as CSA_ERR_INDEX on the device. */
 int csa_compress_all(const csa_dims* dims, const csa_seq* seqs, const int64_t* tok_ranges, int B, int64_t max_tokens,
                      const csa_bf16* x, const csa_bf16* logit_c, const csa_bf16* logit_h, const float* bias_c,
                      const float* bias_h, const csa_bf16* idx_key, csa_bf16* entries, csa_bf16* entry_keys,
-                     csa_bf16* hca_entries, csa_stream_t stream);
+                     csa_bf16* hca_entries, const csa_norms* norms, csa_stream_t stream);
 
 /* a3/a4 -- Lightning-Indexer scores and top-k ("Frontier Techniques", 2.1; "DeepSeek V4
  * comprimeix el context", "CSA: buscar primer i atendre despres").  For query i at length L:
@@ -133,6 +157,26 @@ int csa_compress_all(const csa_dims* dims, const csa_seq* seqs, const int64_t* t
 int csa_index_topk(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
                    const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
                    float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* f1 -- 8-bit block-scaled indexer keys ("Frontier Techniques", section 3: the indexer's QK path is
+ * quantized to a block-scaled format; "Compressed attention", sections 3-4: block scales carry
+ * bytes).  Each 32-channel block of a key shares one power-of-two scale 2^e, stored as the byte
+ * e + 127, where 2^e is the smallest power of two with amax <= 448 * 2^e (a zero block: e = -127);
+ * the block's elements are FP8 E4M3 bytes of x / 2^e rounded to nearest even.  Rows follow the
+ * CSA entry rows (keys_q row csa_off + j holds entry j's d_I bytes, key_scales row csa_off + j its
+ * d_I / 32 scale bytes).  Per entry 64 + 2 bytes instead of 128 at d_I = 64.
+ *
+ * csa_quantize_keys: the 8-bit copies of the stored bf16 keys of entries [ranges[b][0],
+ * ranges[b][1]) of every sequence (ranges and max_entries as csa_compress; the entries must
+ * exist: m * ranges[b][1] <= seqs[b].len, else CSA_ERR_INDEX on the device).
+ * csa_index_topk_mx8: csa_index_topk scoring the dequantized 8-bit keys (queries stay bf16):
+ * s_j = sum_h w_h relu(q_idx_h . K_j), K_j[c] = 2^e * E4M3 value; same outputs, same workspace
+ * size (CSA_OP_INDEX_TOPK). */
+int csa_quantize_keys(const csa_dims* dims, const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries,
+                      const csa_bf16* entry_keys, uint8_t* keys_q, uint8_t* key_scales, csa_stream_t stream);
+int csa_index_topk_mx8(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
+                       const csa_bf16* q_idx, const float* w, const uint8_t* keys_q, const uint8_t* key_scales,
+                       int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* a5 -- sparse MQA attention over the selected CSA entries plus the raw window ("DeepSeek V4
  * comprimeix el context", "CSA: buscar primer i atendre despres"; "Frontier Techniques", 2.1).
@@ -152,6 +196,7 @@ int csa_sparse_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* 
 int hca_dense_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
                    const csa_bf16* q, const csa_bf16* hca_entries, const csa_bf16* x, int W, float scale,
                    float* out, float* lse, void* ws, size_t ws_bytes, csa_stream_t stream);
+
 
 /* Arguments of one decode step of B sequences (all pointers device memory). */
 typedef struct csa_decode_args {
@@ -182,6 +227,21 @@ typedef struct csa_decode_args {
     const csa_bf16* new_rows; /* [B, 3d + d_I]: x | logit_c | logit_h | idx_key of each sequence's
                                  appended token, copied into the caches by the call (append = 1;
                                  16-byte aligned rows), or NULL */
+    uint8_t* keys_q;          /* optional 8-bit block-scaled indexer keys [*, d_I] (see
+                                 csa_quantize_keys; 16-byte aligned), or NULL.  When given, the
+                                 indexer scores these instead of entry_keys, and the append also
+                                 writes the 8-bit copy of every key it completes */
+    uint8_t* key_scales;      /* their block scales [*, d_I / 32] (2-byte aligned), with keys_q */
+    const int32_t* idx_in;    /* optional [B, k]: a selection reused from another layer of the same
+                                 sequences (cross-layer index reuse, "Compressed attention", sections
+                                 1 and 5: consecutive layers may share the selected-position table,
+                                 and the reusing layer must read the source layer's selection).
+                                 When given, this call runs no indexer (q_idx and w may be NULL,
+                                 idx_out must be NULL) and attends these entries of its own CSA
+                                 cache; entries are named by their position j, which is the same in
+                                 every layer of a sequence */
+    const csa_norms* norms;   /* optional (host struct, see csa_norms): query / entry normalization
+                                 and sink logits; NULL: none */
 } csa_decode_args;
 
 /* a8 + a3..a7 -- one decode step: optional append (and the compressor updates it triggers), then
@@ -213,6 +273,11 @@ typedef struct csa_prefill_args {
     float* out;              /* [q_end - q_begin, H, d] */
     float* lse;              /* [q_end - q_begin, H] (nullable) */
     int32_t* idx_out;        /* [q_end - q_begin, k] (nullable) */
+    const int32_t* idx_in;   /* optional [q_end - q_begin, k]: a selection reused from another layer
+                                (as in csa_decode_args): no indexer runs; q_idx / w may be NULL and
+                                idx_out must be NULL */
+    const csa_norms* norms;  /* optional (host struct): as in csa_decode_args; the entry
+                                normalization applies to the compress step (compress = 1) */
 } csa_prefill_args;
 
 /* a1, a2 full pass + a3..a7 for every query position in [q_begin, q_end) of one sequence. */
@@ -251,7 +316,8 @@ int csa_sync_status(csa_stream_t stream);
  * array of `count` cudaEvent_t handles (created by the caller, owned by the caller), every later
  * hybrid_attn_decode call on this host thread records CSA_DECODE_MARKS consecutive events of the
  * array, cyclically from index 0, on its stream: before the append kernel, after it, after the
- * indexer score scan, after the top-k select, after attention (and its merge).  Inside a stream
+ * indexer (the score scan, whose last CTA per query also selects the top-k), again at the same point
+ * (the select has no kernel of its own), after attention (and its merge).  Inside a stream
  * capture the records become graph nodes.  NULL / 0 turns it off.  Returns CSA_OK or CSA_ERR_ARG
  * (count not a positive multiple of CSA_DECODE_MARKS). */
 #define CSA_DECODE_MARKS 5
@@ -261,7 +327,7 @@ int csa_set_stage_events(void* const* events, int count);
  * the scratch lives).  For callers that cannot provide device memory at call time -- code under a
  * framework whose allocator owns all device buffers, loops that must not allocate once running, or
  * bindings that only see input and output pointers.  The scratch is a fixed array inside the
- * library, about 12.1 MiB on every device that loads it, held until the process exits.
+ * library, about 14.2 MiB on every device that loads it, held until the process exits.
  * Limits: Q <= 16 and Q * ceil4(floor(max_len / m)) <= 1,048,576; larger calls return
  * CSA_ERR_UNSUPPORTED with a message and enqueue nothing.  It never allocates or frees memory.
  * The first call on a device looks up the array's device address (once per device, with that
@@ -272,6 +338,17 @@ int csa_set_stage_events(void* const* events, int count);
 int csa_index_topk_noalloc(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q,
                            int64_t max_len, const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys,
                            int32_t* idx_out, float* score_out, csa_stream_t stream);
+
+/* Fault injection for testing the bounded waits (a test aid; off by default; no counterpart in the
+ * pages).  Every wait inside a kernel gives up after a time limit, records CSA_ERR_TIMEOUT in the
+ * device status word and lets the kernel wind down (the CTA waits for its own copies in flight,
+ * frees its tensor memory and exits), so a fault never hangs the device.  fault = 1 makes the
+ * attention kernel's first loader warp skip its arrival on the first key tile of every CTA, so that
+ * tile never becomes full and the waits on it run out; fault = 0 turns injection off.
+ * wait_limit_ns > 0 sets the limit of the attention kernel's waits (0 restores the default of 2 s).
+ * Process-wide; applies to attention launches issued after the call.  Returns CSA_OK or
+ * CSA_ERR_ARG. */
+int csa_debug_inject(int fault, int64_t wait_limit_ns);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int csa_version(void);

@@ -262,17 +262,22 @@ class Shape:
         return 1.0 / float(np.sqrt(self.d))
 
 
-def hybrid_query(shape: Shape, L: int, q, qI, w, raw, entries, KI, hca, sink=None, q_gain=None, eps=1e-6):
+def hybrid_query(shape: Shape, L: int, q, qI, w, raw, entries, KI, hca, sink=None, q_gain=None, eps=1e-6,
+                 keys_mx8=None):
     """One query of the hybrid layer at visible length L, composed from the stages above.
 
     raw: uint16 [>=L, d] raw latents of the sequence; entries: uint16 [>=L//m, d] CSA cache;
     KI: uint16 [>=L//m, d_I] indexer-key cache; hca: uint16 [>=L//m', d] HCA cache.
     Optional: sink [H] attention-sink logits; q_gain [d]: the query heads are RMS-normalized with
-    this gain (and rounded to bf16, the attention's operand type) before attending.
+    this gain (and rounded to bf16, the attention's operand type) before attending; keys_mx8 =
+    (Kq, scales): the indexer scores these 8-bit keys instead of KI.
     Returns a dict with the selected indices, the two partials and the merged output.
     """
     n_c = L // shape.m
-    s = index_scores(qI, w, KI[:n_c])
+    if keys_mx8 is not None:
+        s = index_scores_mx8(qI, w, keys_mx8[0][:n_c], keys_mx8[1][:n_c])
+    else:
+        s = index_scores(qI, w, KI[:n_c])
     idx = topk(s, shape.k)
     if q_gain is not None:
         q = round_bf16(rms_norm(bf16_to_f64(q), q_gain, eps))

@@ -42,21 +42,23 @@ def test_struct_layouts_match_header(tmp_path):
     prog = tmp_path / "sizes.c"
     prog.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "csa.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(csa_dims), sizeof(csa_seq),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(csa_dims), sizeof(csa_seq),"
         " sizeof(csa_query), sizeof(csa_ws_query), sizeof(csa_decode_args), sizeof(csa_prefill_args),"
         " offsetof(csa_decode_args, out), offsetof(csa_prefill_args, idx_out),"
-        " offsetof(csa_decode_args, new_rows));return 0;}\n")
+        " offsetof(csa_decode_args, new_rows), offsetof(csa_decode_args, norms), offsetof(csa_prefill_args, norms),"
+        " sizeof(csa_norms));return 0;}\n")
     exe = tmp_path / "sizes"
     subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
     assert got == [ctypes.sizeof(csa.csa_dims), 32, 16, ctypes.sizeof(csa.csa_ws_query),
                    ctypes.sizeof(csa.csa_decode_args), ctypes.sizeof(csa.csa_prefill_args),
                    csa.csa_decode_args.out.offset, csa.csa_prefill_args.idx_out.offset,
-                   csa.csa_decode_args.new_rows.offset]
+                   csa.csa_decode_args.new_rows.offset, csa.csa_decode_args.norms.offset,
+                   csa.csa_prefill_args.norms.offset, ctypes.sizeof(csa.csa_norms)]
 
 
 def test_version_and_error_string(lib):
-    assert csa.csa_version() == 100
+    assert csa.csa_version() == 200
     assert isinstance(csa.csa_last_error(), str)
 
 
@@ -102,6 +104,35 @@ def test_host_validation_rejects_bad_arguments(lib):
     pa.len, pa.q_begin, pa.q_end = 10, 5, 20
     rc = lib.hybrid_attn_prefill(ctypes.byref(pa), 256, 1 << 20, None)
     assert rc == csa.CSA_ERR_ARG and "query range" in csa.csa_last_error()
+
+
+def test_compress_all_and_fault_injection_validation(lib):
+    dims = csa.make_dims()
+    P = [16] * 11
+    rc = lib.csa_compress_all(ctypes.byref(dims), 16, None, 1, 10, *P[:9], None, None)
+    assert rc == csa.CSA_ERR_ARG and "NULL" in csa.csa_last_error()
+    rc = lib.csa_compress_all(ctypes.byref(dims), 16, 16, 1, 10, 16, 16, 16, 16, 24, 16, 16, 16, 16, None, None)
+    assert rc == csa.CSA_ERR_ARG and "aligned" in csa.csa_last_error()
+    rc = lib.csa_compress_all(ctypes.byref(dims), 16, 16, 0, 10, *P[:9], None, None)
+    assert rc == csa.CSA_ERR_ARG
+    assert lib.csa_compress_all(ctypes.byref(dims), 16, 16, 1, 0, *P[:9], None, None) == csa.CSA_OK  # nothing to do
+    # normalization parameters
+    n = csa.make_norms()
+    n.reserved = 1
+    rc = lib.csa_compress_all(ctypes.byref(dims), 16, 16, 1, 10, *P[:9], ctypes.byref(n), None)
+    assert rc == csa.CSA_ERR_ARG and "reserved" in csa.csa_last_error()
+    n.reserved, n.q_norm = 0, 24
+    rc = lib.csa_compress_all(ctypes.byref(dims), 16, 16, 1, 10, *P[:9], ctypes.byref(n), None)
+    assert rc == csa.CSA_ERR_ARG and "aligned" in csa.csa_last_error()
+    n.q_norm, n.entry_norm_c = None, 16
+    rc = lib.csa_compress_all(ctypes.byref(csa.make_dims(m=2)), 16, 16, 1, 10, *P[:9], ctypes.byref(n), None)
+    assert rc == csa.CSA_ERR_UNSUPPORTED and "m = 4" in csa.csa_last_error()
+    n.entry_norm_c, n.entry_norm_h = None, 16
+    rc = lib.csa_compress_all(ctypes.byref(csa.make_dims(m_hca=256)), 16, 16, 1, 10, *P[:9], ctypes.byref(n), None)
+    assert rc == csa.CSA_ERR_UNSUPPORTED
+    assert lib.csa_debug_inject(2, 0) == csa.CSA_ERR_ARG
+    assert lib.csa_debug_inject(1, -5) == csa.CSA_ERR_ARG
+    assert lib.csa_debug_inject(0, 0) == csa.CSA_OK
 
 
 def test_workspace_sizes(lib):

@@ -236,6 +236,366 @@ def test_index_topk_ties_and_zero_scores():
     _index_case([5000], 1024, zero_w=True)             # every score 0: indices 0..k-1
 
 
+def _ordered_keys(E, pattern, d_I=64):
+    """Keys whose score under q^I = (256, 1, 0, ...) on head 0 is an exact integer rank r_j < 65536:
+    key_j = (r_j // 256, r_j % 256, 0, ...), every value exact in bf16 and every sum exact in fp32."""
+    j = np.arange(E)
+    if pattern == "increasing":
+        r = j
+    elif pattern == "decreasing":
+        r = E - 1 - j
+    elif pattern == "blocks":  # the best ranks sit in a few runs of 1,500 entries far apart
+        run = j // 1500
+        r = np.where(run % 17 == 3, 50000 + (run // 17) * 1500 + j % 1500, j // 7)
+    else:
+        raise ValueError(pattern)
+    K = np.zeros((E, d_I), np.float64)
+    K[:, 0] = r // 256
+    K[:, 1] = r % 256
+    return oracle.round_bf16(K)
+
+
+@pytest.mark.parametrize("pattern", ["increasing", "decreasing", "blocks"])
+def test_index_topk_concentrated_top_entries(pattern):
+    """The top-k concentrated in a few scan chunks (far more than a chunk's share of them): those
+    chunks' candidates do not cover their members of the threshold bin, so the select re-filters
+    them from the stored scores.  The result must still be the exact top-k."""
+    E, k, d_I, H_I = 60000, 1024, 64, 4
+    dims = csa.make_dims(d=512, H=64, d_I=d_I, H_I=H_I, m=4, m_hca=128, k=k, W=128)
+    K = _ordered_keys(E, pattern)
+    qI = np.zeros((1, H_I, d_I), np.float64)
+    qI[0, 0, 0], qI[0, 0, 1] = 256.0, 1.0
+    qI = oracle.round_bf16(qI)
+    w = np.array([[1.0, 0.0, 0.0, 0.0]], np.float32)
+    seqs = torch.tensor([[0, 0, 0, 4 * E]], dtype=torch.int64, device="cuda")
+    qt = gh.query_table([(0, 4 * E)])
+    wq = csa.csa_ws_query()
+    wq.dims, wq.Q, wq.max_len = dims, 1, 4 * E
+    ws = torch.empty(csa.csa_workspace_size(csa.CSA_OP_INDEX_TOPK, wq), dtype=torch.uint8, device="cuda")
+    idx = torch.full((1, k), -7, dtype=torch.int32, device="cuda")
+    sc = torch.empty(1, k, dtype=torch.float32, device="cuda")
+    csa.csa_index_topk(dims, seqs, qt, 1, 4 * E, gh.to_dev_bf16(qI), torch.from_numpy(w).cuda(), gh.to_dev_bf16(K),
+                       idx, sc, ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    s = oracle.index_scores(qI[0], w[0], K)
+    ref = oracle.topk(s, k)
+    np.testing.assert_array_equal(idx.cpu().numpy()[0], ref)
+    np.testing.assert_array_equal(sc.cpu().numpy()[0], s[ref].astype(np.float32))
+
+
+# --------------------------------------------------------------------------------- f1: 8-bit keys
+
+@pytest.mark.parametrize("E_list,d_I,scale", [([5000, 300], 64, 1.0), ([2000], 32, 1.0), ([700], 64, 2.0 ** -30),
+                                              ([900], 64, 7.0e3)], ids=["prod", "d32", "tiny_values", "large"])
+def test_quantize_keys_matches_oracle(E_list, d_I, scale):
+    """csa_quantize_keys writes exactly the oracle's E4M3 bytes and scale bytes (all-zero rows and
+    extreme magnitudes included)."""
+    dims = csa.make_dims(d=512, H=64, d_I=d_I, H_I=4, m=4, m_hca=128, k=1024, W=128)
+    Ks = [oracle.round_bf16(synth.bf16_to_f64(synth.bf16_normal(3101, synth.KI, i, d_I, 0, E)) * scale)
+          for i, E in enumerate(E_list)]
+    Ks[0][3] = 0
+    offs = np.cumsum([0] + list(E_list))
+    keys = gh.to_dev_bf16(np.concatenate(Ks))
+    seqs = torch.tensor([[0, offs[i], 0, 4 * E] for i, E in enumerate(E_list)], dtype=torch.int64, device="cuda")
+    ranges = torch.tensor([[0, E] for E in E_list], dtype=torch.int64, device="cuda")
+    kq = torch.full((offs[-1], d_I), 0xAA, dtype=torch.uint8, device="cuda")
+    ks = torch.full((offs[-1], d_I // 32), 0xAA, dtype=torch.uint8, device="cuda")
+    csa.csa_quantize_keys(dims, seqs, ranges, len(E_list), max(E_list), keys, kq, ks)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    ref_q, ref_s = oracle.quantize_keys_mx8(np.concatenate(Ks))
+    np.testing.assert_array_equal(ks.cpu().numpy(), ref_s)
+    np.testing.assert_array_equal(kq.cpu().numpy(), ref_q)
+
+
+@pytest.mark.parametrize("E_list,k,d_I", [([5000], 1024, 64), ([300], 32, 32), ([600], 1024, 64),
+                                          ([1025, 70000, 4097, 1], 1024, 64), ([262144], 1024, 64),
+                                          ([40000, 33000], 2048, 64)],
+                         ids=["E5000", "tiny", "E<k", "ragged4", "E262144", "k2048"])
+def test_index_topk_mx8_stage(E_list, k, d_I, H_I=4, seed=3201):
+    """The indexer on 8-bit keys selects the oracle's top-k of the dequantized keys' scores (both sides
+    score the same bytes; ties resolved as for bf16 keys), with the scores."""
+    dims = csa.make_dims(d=512, H=64, d_I=d_I, H_I=H_I, m=4, m_hca=128, k=k, W=128)
+    Q = len(E_list)
+    KQ, SC = [], []
+    for i, E in enumerate(E_list):
+        kq, sc = oracle.quantize_keys_mx8(synth.bf16_normal(seed, synth.KI, i, d_I, 0, max(E, 1)))
+        KQ.append(kq)
+        SC.append(sc)
+    offs = np.cumsum([0] + [max(E, 1) for E in E_list])
+    keys_q = torch.from_numpy(np.concatenate(KQ)).cuda()
+    key_scales = torch.from_numpy(np.concatenate(SC)).cuda()
+    seqs = torch.tensor([[0, offs[i], 0, 4 * E + 3] for i, E in enumerate(E_list)], dtype=torch.int64, device="cuda")
+    qt = gh.query_table([(i, 4 * E + 3) for i, E in enumerate(E_list)])
+    qI = synth.bf16_normal(seed, synth.QI, 99, H_I * d_I, 0, Q).reshape(Q, H_I, d_I)
+    w = synth.f32_uniform(seed, synth.W, 99, H_I, 0, Q)
+    idx = torch.full((Q, k), -7, dtype=torch.int32, device="cuda")
+    sc_out = torch.empty(Q, k, dtype=torch.float32, device="cuda")
+    max_len = 4 * max(E_list) + 3
+    wq = csa.csa_ws_query()
+    wq.dims, wq.Q, wq.max_len = dims, Q, max_len
+    ws = torch.empty(csa.csa_workspace_size(csa.CSA_OP_INDEX_TOPK, wq), dtype=torch.uint8, device="cuda")
+    csa.csa_index_topk_mx8(dims, seqs, qt, Q, max_len, gh.to_dev_bf16(qI), torch.from_numpy(w).cuda(), keys_q,
+                           key_scales, idx, sc_out, ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    idx_h, sc_h = idx.cpu().numpy(), sc_out.cpu().numpy()
+    for i, E in enumerate(E_list):
+        s = oracle.index_scores_mx8(qI[i], w[i], KQ[i][:E], SC[i][:E])
+        ref = oracle.topk(s, k)
+        gh.sets_match(idx_h[i], ref, s, k)
+        valid = idx_h[i][idx_h[i] >= 0]
+        assert (np.diff(valid) > 0).all() and len(valid) == min(E, k)
+        np.testing.assert_allclose(sc_h[i][:len(valid)], s[valid], rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("wl,steps", [(workloads.tiny(), 3), (wl_small([3000, 9001], B=2), 5)], ids=["tiny", "prod"])
+def test_decode_with_8bit_keys(wl, steps):
+    """Decode with the indexer on 8-bit keys: the append writes the 8-bit copy of every key it completes
+    (equal to quantizing the stored bf16 key), the selection is the oracle's top-k of the 8-bit keys'
+    scores, and the output is the oracle's attention over the GPU's caches with that selection."""
+    d = wl.dims
+    layer = csa.HybridLayer(gh.dims_of(d), [wl.capacity(b) for b in range(wl.B)], key_format="mx8")
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths(list(wl.n0))
+    layer.compress()
+    B = wl.B
+    q = torch.empty(B, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(B, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(B, d.H_I, dtype=torch.float32, device="cuda")
+    out = torch.empty(B, d.H, d.d, dtype=torch.float32, device="cuda")
+    idx = torch.empty(B, d.k, dtype=torch.int32, device="cuda")
+    ws = layer.decode_workspace()
+    sh = gh.oshape(d)
+    for s in range(steps):
+        for b in range(B):
+            sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
+        layer.decode(layer.decode_args(q, qi, w, out, idx_out=idx), ws)
+        assert csa.csa_sync_status() == csa.CSA_OK
+        keys = gh.u16(layer.entry_keys)
+        kq, ks = layer.keys_q.cpu().numpy(), layer.key_scales.cpu().numpy()
+        ent, hca, x = gh.u16(layer.entries), gh.u16(layer.hca_entries), gh.u16(layer.x)
+        for b in range(B):
+            L = wl.n0[b] + s + 1
+            c0, n_c = layer.csa_off[b], L // d.m
+            rq, rs = oracle.quantize_keys_mx8(keys[c0:c0 + n_c])
+            np.testing.assert_array_equal(kq[c0:c0 + n_c], rq)
+            np.testing.assert_array_equal(ks[c0:c0 + n_c], rs)
+            qh, qih, wh = workloads.queries(wl, b, s, s + 1)
+            sc = oracle.index_scores_mx8(qih[0], wh[0], rq, rs)
+            gh.sets_match(idx[b].cpu().numpy(), oracle.topk(sc, d.k), sc, d.k)
+            t0, h0 = layer.tok_off[b], layer.hca_off[b]
+            O_c, l_c = oracle.csa_attn(qh[0], ent[c0:c0 + max(n_c, 1)], idx[b].cpu().numpy(), d.m,
+                                       x[t0:t0 + L], L, d.W, sh.scale)
+            O_h, l_h = oracle.hca_attn(qh[0], hca[h0:h0 + max(L // d.m_hca, 1)], d.m_hca, x[t0:t0 + L], L, 0, sh.scale)
+            O, _ = oracle.lse_merge(O_c, l_c, O_h, l_h)
+            gh.check_close(out[b].cpu().numpy(), O, f"8-bit keys: step {s} seq {b}")
+
+
+# --------------------------------------------------------------------------------- f2: index reuse
+
+def _oracle_on_gpu_caches(layer, b, L, qh, idx_b, d):
+    """The oracle's merged output for one query of `layer` at length L over the layer's own (GPU)
+    caches with a given selection."""
+    sh = gh.oshape(d)
+    ent, hca, x = gh.u16(layer.entries), gh.u16(layer.hca_entries), gh.u16(layer.x)
+    c0, t0, h0 = layer.csa_off[b], layer.tok_off[b], layer.hca_off[b]
+    O_c, l_c = oracle.csa_attn(qh, ent[c0:c0 + max(L // d.m, 1)], idx_b, d.m, x[t0:t0 + L], L, d.W, sh.scale)
+    O_h, l_h = oracle.hca_attn(qh, hca[h0:h0 + max(L // d.m_hca, 1)], d.m_hca, x[t0:t0 + L], L, 0, sh.scale)
+    return oracle.lse_merge(O_c, l_c, O_h, l_h)[0]
+
+
+@pytest.mark.parametrize("wl", [workloads.tiny(), wl_small([3000, 9001], B=2)], ids=["tiny", "prod"])
+def test_decode_reuses_the_source_layers_selection(wl):
+    """Cross-layer index reuse: layer 2 (its own caches, other inputs) attends the entries layer 1's
+    indexer selected in the same step; its output is the oracle's attention over layer 2's caches
+    with layer 1's selection."""
+    d = wl.dims
+    wl2 = workloads.Workload(wl.name + "_layer2", wl.seed + 77, d, wl.n0, wl.steps)
+    l1, l2 = gh.new_layer(wl), gh.new_layer(wl2)
+    B = wl.B
+    mk = lambda *shape, dt=torch.bfloat16: torch.empty(*shape, dtype=dt, device="cuda")
+    q, qi, w = mk(B, d.H, d.d), mk(B, d.H_I, d.d_I), mk(B, d.H_I, dt=torch.float32)
+    q2 = mk(B, d.H, d.d)
+    out1, out2 = mk(B, d.H, d.d, dt=torch.float32), mk(B, d.H, d.d, dt=torch.float32)
+    idx = mk(B, d.k, dt=torch.int32)
+    ws1, ws2 = l1.decode_workspace(), l2.decode_workspace()
+    for s in range(2):
+        for b in range(B):
+            sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
+            sdev.fill_queries(wl2, b, s, s + 1, q2[b:b + 1], qi[b:b + 1].clone(), w[b:b + 1].clone())
+        l1.decode(l1.decode_args(q, qi, w, out1, idx_out=idx), ws1)
+        l2.decode(l2.decode_args(q2, None, None, out2, idx_in=idx), ws2)
+        assert csa.csa_sync_status() == csa.CSA_OK
+        for b in range(B):
+            L = wl.n0[b] + s + 1
+            qh = workloads.queries(wl2, b, s, s + 1)[0][0]
+            O = _oracle_on_gpu_caches(l2, b, L, qh, idx[b].cpu().numpy(), d)
+            gh.check_close(out2[b].cpu().numpy(), O, f"reuse step {s} seq {b}")
+
+
+def test_prefill_reuses_the_source_layers_selection():
+    d = workloads.TINY_DIMS
+    N = 1024
+    wl1 = workloads.Workload("prefill_l1", 4101, d, (N,), 0, mode="prefill")
+    wl2 = workloads.Workload("prefill_l2", 4102, d, (N,), 0, mode="prefill")
+    layers, qs = [], []
+    for wl in (wl1, wl2):
+        layer = csa.HybridLayer(gh.dims_of(d), [N])
+        sdev.fill_layer_inputs(layer, wl)
+        layer.set_lengths([N])
+        q = torch.empty(N, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+        qi = torch.empty(N, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+        w = torch.empty(N, d.H_I, dtype=torch.float32, device="cuda")
+        sdev.fill_queries(wl, 0, 0, N, q, qi, w)
+        layers.append(layer)
+        qs.append((q, qi, w))
+    idx = torch.empty(N, d.k, dtype=torch.int32, device="cuda")
+    out1 = torch.empty(N, d.H, d.d, dtype=torch.float32, device="cuda")
+    out2 = torch.empty_like(out1)
+    l1, l2 = layers
+    l1.prefill(l1.prefill_args(*qs[0], out1, 0, N, compress=True, idx_out=idx), l1.prefill_workspace(N))
+    l2.prefill(l2.prefill_args(qs[1][0], None, None, out2, 0, N, compress=True, idx_in=idx), l2.prefill_workspace(N))
+    assert csa.csa_sync_status() == csa.CSA_OK
+    qh = workloads.queries(wl2, 0, 0, N)[0]
+    idx_h, o2 = idx.cpu().numpy(), out2.cpu().numpy()
+    for i in list(range(0, N, 61)) + [N - 1]:
+        O = _oracle_on_gpu_caches(l2, 0, i + 1, qh[i], idx_h[i], d)
+        gh.check_close(o2[i], O, f"prefill reuse row {i}")
+
+
+# --------------------------------------------------------------------------------- f3: norms, sinks
+
+def _norm_tensors(wl, seed=5101):
+    d = wl.dims
+    g = lambda t, rows: torch.from_numpy(1.0 + 0.25 * synth.f32_normal(seed, t, 0, d.d, 0, rows)[0]).cuda()
+    q_norm, en_c, en_h = g(synth.Q, 1), g(synth.A, 1), g(synth.B, 1)
+    sink = torch.from_numpy(2.0 * synth.f32_normal(seed, synth.W, 0, d.H, 0, 1)[0]).cuda()
+    return q_norm, en_c, en_h, sink
+
+
+def _normed_layer(wl, lens=None, eps=1e-5):
+    layer = csa.HybridLayer(gh.dims_of(wl.dims), [wl.capacity(b) for b in range(wl.B)])
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths(list(wl.n0) if lens is None else lens)
+    t = _norm_tensors(wl)
+    layer.set_norms(*t, eps=eps)
+    layer.compress()
+    torch.cuda.synchronize()
+    return layer, t
+
+
+@pytest.mark.parametrize("wl", [workloads.tiny(), wl_small([2000, 333], B=2)], ids=["tiny", "prod"])
+def test_normalized_entries_within_one_ulp(wl):
+    """RMS-normalized CSA and HCA entries against the oracle's normalization of its fp64 entries:
+    one bf16 ulp plus the fp32 accumulation bound carried through the normalization."""
+    layer, (q_norm, en_c, en_h, sink) = _normed_layer(wl)
+    d = wl.dims
+    eps = 1e-5
+    for b in range(wl.B):
+        n = wl.n0[b]
+        ref = gh.OracleSeq(wl, b, n, with_mass=True)
+        for name, off, E64, mass, gain, n_e in (("entries", layer.csa_off, ref.E64, ref.E_mass, en_c, n // d.m),
+                                                ("hca_entries", layer.hca_off, getattr(ref, "H64", None),
+                                                 getattr(ref, "H_mass", None), en_h, n // d.m_hca)):
+            if n_e == 0:
+                continue
+            gn = gain.cpu().numpy().astype(np.float64)
+            want = oracle.rms_norm(E64, gn.astype(np.float32), eps)
+            inv = 1.0 / np.sqrt((E64 ** 2).mean(axis=1, keepdims=True) + eps)
+            got = gh.u16(getattr(layer, name)[off[b]:off[b] + n_e])
+            g64 = synth.bf16_to_f64(got)
+            ulp = np.maximum(np.abs(synth.bf16_to_f64(oracle.round_bf16(want))) * 2.0 ** -7, 2.0 ** -133)
+            bound = ulp + mass * 2.0 ** -18 * inv * np.abs(gn) + np.abs(want) * 2.0 ** -20
+            assert (np.abs(g64 - want) <= bound).all(), f"seq {b} {name}: {(np.abs(g64 - want) > bound).sum()} beyond bound"
+
+
+@pytest.mark.parametrize("wl", [workloads.tiny(), wl_small([1000, 515], B=2, steps=130)], ids=["tiny", "prod"])
+def test_normalized_append_equals_full_pass(wl):
+    """With entry normalization the decode append still leaves the caches bit-identical to a full pass."""
+    d = wl.dims
+    layer, t = _normed_layer(wl)
+    q = torch.empty(wl.B, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(wl.B, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(wl.B, d.H_I, dtype=torch.float32, device="cuda")
+    out = torch.empty(wl.B, d.H, d.d, dtype=torch.float32, device="cuda")
+    ws = layer.decode_workspace()
+    for s in range(wl.steps):
+        for b in range(wl.B):
+            sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
+        layer.decode(layer.decode_args(q, qi, w, out), ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    full, _ = _normed_layer(wl, lens=[n + wl.steps for n in wl.n0])
+    for name in ("entries", "entry_keys", "hca_entries"):
+        assert torch.equal(getattr(layer, name).view(torch.int16), getattr(full, name).view(torch.int16)), name
+
+
+def _oracle_normed(layer, b, L, qh, idx_b, d, q_gain, sink, eps):
+    sh = gh.oshape(d)
+    ent, hca, x = gh.u16(layer.entries), gh.u16(layer.hca_entries), gh.u16(layer.x)
+    c0, t0, h0 = layer.csa_off[b], layer.tok_off[b], layer.hca_off[b]
+    qn = oracle.round_bf16(oracle.rms_norm(synth.bf16_to_f64(qh), q_gain, eps))
+    O_c, l_c = oracle.csa_attn(qn, ent[c0:c0 + max(L // d.m, 1)], idx_b, d.m, x[t0:t0 + L], L, d.W, sh.scale)
+    O_h, l_h = oracle.hca_attn(qn, hca[h0:h0 + max(L // d.m_hca, 1)], d.m_hca, x[t0:t0 + L], L, 0, sh.scale)
+    O, lse = oracle.lse_merge(O_c, l_c, O_h, l_h)
+    return oracle.sink_merge(O, lse, sink)
+
+
+@pytest.mark.parametrize("wl,steps", [(workloads.tiny(), 2), (wl_small([3000, 9001], B=2), 2)], ids=["tiny", "prod"])
+def test_decode_with_norms_and_sinks(wl, steps):
+    """Query normalization and sink logits in the decode step (merge kernel), over the GPU's own
+    normalized caches and selection."""
+    d = wl.dims
+    layer, (q_norm, en_c, en_h, sink) = _normed_layer(wl)
+    B = wl.B
+    q = torch.empty(B, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(B, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(B, d.H_I, dtype=torch.float32, device="cuda")
+    out = torch.empty(B, d.H, d.d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(B, d.H, dtype=torch.float32, device="cuda")
+    idx = torch.empty(B, d.k, dtype=torch.int32, device="cuda")
+    ws = layer.decode_workspace()
+    qg, sk = q_norm.cpu().numpy(), sink.cpu().numpy().astype(np.float64)
+    for s in range(steps):
+        for b in range(B):
+            sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
+        layer.decode(layer.decode_args(q, qi, w, out, lse=lse, idx_out=idx), ws)
+        assert csa.csa_sync_status() == csa.CSA_OK
+        for b in range(B):
+            L = wl.n0[b] + s + 1
+            qh = workloads.queries(wl, b, s, s + 1)[0][0]
+            O, l = _oracle_normed(layer, b, L, qh, idx[b].cpu().numpy(), d, qg, sk, 1e-5)
+            gh.check_close(out[b].cpu().numpy(), O, f"norms+sinks step {s} seq {b}")
+            gh.check_close(lse[b].cpu().numpy(), l, f"norms+sinks lse step {s} seq {b}")
+
+
+def test_prefill_with_norms_and_sinks():
+    """The same in the prefill, where one item holds a query's whole softmax (sink in the epilogue)."""
+    d = workloads.TINY_DIMS
+    N = 1024
+    wl = workloads.Workload("prefill_norms", 4201, d, (N,), 0, mode="prefill")
+    layer = csa.HybridLayer(gh.dims_of(d), [N])
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths([N])
+    q_norm, en_c, en_h, sink = _norm_tensors(wl)
+    layer.set_norms(q_norm, en_c, en_h, sink, eps=1e-5)
+    q = torch.empty(N, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(N, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(N, d.H_I, dtype=torch.float32, device="cuda")
+    sdev.fill_queries(wl, 0, 0, N, q, qi, w)
+    out = torch.empty(N, d.H, d.d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(N, d.H, dtype=torch.float32, device="cuda")
+    idx = torch.empty(N, d.k, dtype=torch.int32, device="cuda")
+    layer.prefill(layer.prefill_args(q, qi, w, out, 0, N, compress=True, lse=lse, idx_out=idx),
+                  layer.prefill_workspace(N))
+    assert csa.csa_sync_status() == csa.CSA_OK
+    qh = workloads.queries(wl, 0, 0, N)[0]
+    qg, sk = q_norm.cpu().numpy(), sink.cpu().numpy().astype(np.float64)
+    o, lh, ih = out.cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+    for i in [0, 1, 3, 4, 15, 16, 100, 511, N - 1]:
+        O, l = _oracle_normed(layer, 0, i + 1, qh[i], ih[i], d, qg, sk, 1e-5)
+        gh.check_close(o[i], O, f"prefill norms row {i}")
+        gh.check_close(lh[i], l, f"prefill norms lse row {i}")
+
+
 # --------------------------------------------------------------------------------- a5/a6 (stage)
 
 def _stage_layer(wl):
@@ -322,6 +682,36 @@ def test_bad_index_is_reported_not_read():
     csa.csa_sparse_attn(dims, layer.seqs, qt, 1, q, layer.entries, idx_ok, layer.x, 0.1, out2, None, ws)
     assert csa.csa_sync_status() == csa.CSA_OK
     assert torch.equal(out, out2)  # the bad slot was skipped, nothing else changed
+
+
+def test_wait_that_runs_out_is_reported_and_the_device_recovers():
+    """A bounded wait that runs out (fault injection: one attention loader warp never arrives on the
+    first key tile) is reported as CSA_ERR_TIMEOUT after the short limit, the kernel winds down, and
+    the next call on the same context returns CSA_OK with the right output."""
+    wl = workloads.tiny()
+    layer, refs = _stage_layer(wl)
+    d = wl.dims
+    dims = gh.dims_of(d)
+    sh = gh.oshape(d)
+    L = 1000
+    qt = gh.query_table([(0, L)])
+    qh, qih, wh = workloads.queries(wl, 0, 0, 1)
+    idx_h = oracle.topk(oracle.index_scores(qih[0], wh[0], refs[0].KI[:L // d.m]), d.k)
+    q = gh.to_dev_bf16(qh)
+    idx = torch.from_numpy(idx_h[None].copy()).cuda()
+    out = torch.empty(1, d.H, d.d, dtype=torch.float32, device="cuda")
+    ws = torch.empty(1 << 22, dtype=torch.uint8, device="cuda")
+    try:
+        csa.csa_debug_inject(1, 1_000_000)  # 1 ms limit
+        csa.csa_sparse_attn(dims, layer.seqs, qt, 1, q, layer.entries, idx, layer.x, sh.scale, out, None, ws)
+        assert csa.csa_sync_status() == csa.CSA_ERR_TIMEOUT
+    finally:
+        csa.csa_debug_inject(0, 0)
+    assert csa.csa_sync_status() == csa.CSA_OK  # reading the status cleared it
+    csa.csa_sparse_attn(dims, layer.seqs, qt, 1, q, layer.entries, idx, layer.x, sh.scale, out, None, ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    O, _ = oracle.csa_attn(qh[0], refs[0].E, idx_h, d.m, refs[0].x, L, d.W, sh.scale)
+    gh.check_close(out[0].cpu().numpy(), O, "after the timeout")
 
 
 # --------------------------------------------------------------------------------- end to end
