@@ -140,8 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             item = (lin - p.Q * n_hca) % p.items_front;
         }
     }
-    // The query table and sequence lengths come from kernels at least two launches back, which are
-    // complete once this grid runs (every kernel of the chain waits before it lets the next start).
+    // The query table and sequence lengths: in the decode chain with an indexer they come from the
+    // append two launches back, complete once this grid runs (every kernel of the chain waits before
+    // it lets the next start); otherwise the previous launch may still be writing them.
+    if (!p.queries_early) grid_dep_wait();
     const csa_query qr = p.queries[qi];
     const bool seq_ok = qr.seq >= 0 && qr.reserved == 0;
     const csa_seq sq = seq_ok ? p.seqs[qr.seq] : csa_seq{0, 0, 0, 0};

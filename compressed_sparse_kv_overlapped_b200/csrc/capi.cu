@@ -905,6 +905,7 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     // scan frees SMs (their inputs, written by the append, are two launches back; with a reused
     // selection the append is the launch right before, so they wait like the others)
     ap2.hca_nowait = (pdl && !reuse) ? 1 : 0;
+    ap2.queries_early = reuse ? 0 : 1;  // the append is two launches back only with the indexer between
     ap2.hca_first = (pl.items.n_items > 1 && pl.items.items_front > 0) ? 1 : 0;
     ap2.cluster = pl.cluster;
     if (!reuse) {

@@ -163,6 +163,9 @@ struct AttnParams {
     // table, HCA entries) were written two or more launches earlier, which are complete by the time
     // this grid may start.  Only the decode chain sets it.
     int hca_nowait;
+    // 1: the query table and the sequence table were written two or more launches back (complete
+    // when this grid runs), so they are read before waiting on the previous launch
+    int queries_early;
     // 1: one-dimensional grid over all (query, item) pairs with every query's HCA items first, so
     // they take the free SMs before the front items (which wait for the top-k) do.  Launches all
     // items of all queries.

@@ -1,6 +1,7 @@
 """GPU parity: every stage of the CUDA path, called through the C ABI, against the fp64 oracle on
 the same seeded inputs.  Stage tests feed both sides identical input bytes (the oracle's caches);
 end-to-end tests let each side build its own caches from the raw tokens."""
+import dataclasses
 import math
 
 import numpy as np
@@ -352,6 +353,7 @@ def test_decode_with_8bit_keys(wl, steps):
     """Decode with the indexer on 8-bit keys: the append writes the 8-bit copy of every key it completes
     (equal to quantizing the stored bf16 key), the selection is the oracle's top-k of the 8-bit keys'
     scores, and the output is the oracle's attention over the GPU's caches with that selection."""
+    wl = dataclasses.replace(wl, steps=max(wl.steps, steps))  # room for every appended token
     d = wl.dims
     layer = csa.HybridLayer(gh.dims_of(d), [wl.capacity(b) for b in range(wl.B)], key_format="mx8")
     sdev.fill_layer_inputs(layer, wl)
@@ -408,6 +410,7 @@ def test_decode_reuses_the_source_layers_selection(wl):
     """Cross-layer index reuse: layer 2 (its own caches, other inputs) attends the entries layer 1's
     indexer selected in the same step; its output is the oracle's attention over layer 2's caches
     with layer 1's selection."""
+    wl = dataclasses.replace(wl, steps=max(wl.steps, 2))  # room for both appended tokens
     d = wl.dims
     wl2 = workloads.Workload(wl.name + "_layer2", wl.seed + 77, d, wl.n0, wl.steps)
     l1, l2 = gh.new_layer(wl), gh.new_layer(wl2)
@@ -543,6 +546,7 @@ def _oracle_normed(layer, b, L, qh, idx_b, d, q_gain, sink, eps):
 def test_decode_with_norms_and_sinks(wl, steps):
     """Query normalization and sink logits in the decode step (merge kernel), over the GPU's own
     normalized caches and selection."""
+    wl = dataclasses.replace(wl, steps=max(wl.steps, steps))  # room for every appended token
     d = wl.dims
     layer, (q_norm, en_c, en_h, sink) = _normed_layer(wl)
     B = wl.B
