@@ -653,13 +653,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         if (threadIdx.x < kHeadsPad) {
             const int h = threadIdx.x;
             float l[kMaxCluster];
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) l[c] = c < F ? ld_cluster_f32(lse_s + h, (uint32_t)c) : -INFINITY;
             float mx = -INFINITY;
-            for (int c = 0; c < F; ++c) {
-                l[c] = ld_cluster_f32(lse_s + h, (uint32_t)c);
-                mx = fmaxf(mx, l[c]);
-            }
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) mx = fmaxf(mx, l[c]);
             float sum = 0.f;
-            for (int c = 0; c < F; ++c) {
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) {
                 l[c] = mx == -INFINITY ? 0.f : expf(l[c] - mx);
                 sum += l[c];
             }
@@ -670,18 +671,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const int cols = D / F, n4 = cols / 4;
         const int part = item / F;
         const int n_parts = n_items / F;
+        // every load of an output's F contributions is issued before any of them is used (the
+        // remote shared-memory latency is paid once per output, not once per contribution)
         for (int e = threadIdx.x; e < kHeadsPad * n4; e += kThreads) {
             const int h = e / n4, col = (int)rank * cols + 4 * (e % n4);
+            float4 v[kMaxCluster];
+            float w[kMaxCluster];
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) {
+                w[c] = c < F ? wts[c * kHeadsPad + h] : 0.f;
+                v[c] = w[c] > 0.f ? ld_cluster_f32x4(o_smem + h * L::kOStride + col, (uint32_t)c)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int c = 0; c < F; ++c) {
-                const float w = wts[c * kHeadsPad + h];
-                if (w > 0.f) {
-                    const float4 v = ld_cluster_f32x4(o_smem + h * L::kOStride + col, (uint32_t)c);
-                    acc.x = fmaf(w, v.x, acc.x);
-                    acc.y = fmaf(w, v.y, acc.y);
-                    acc.z = fmaf(w, v.z, acc.z);
-                    acc.w = fmaf(w, v.w, acc.w);
-                }
+#pragma unroll
+            for (int c = 0; c < kMaxCluster; ++c) {
+                acc.x = fmaf(w[c], v[c].x, acc.x);
+                acc.y = fmaf(w[c], v[c].y, acc.y);
+                acc.z = fmaf(w[c], v[c].z, acc.z);
+                acc.w = fmaf(w[c], v[c].w, acc.w);
             }
             if (h < p.H)
                 *reinterpret_cast<float4*>(p.part_o + (((int64_t)qi * n_parts + part) * kHeadsPad + h) * D + col) = acc;

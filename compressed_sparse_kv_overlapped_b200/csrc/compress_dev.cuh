@@ -257,8 +257,13 @@ __device__ __forceinline__ uint4 entry_bf16(const float (&v)[8], const float* ga
 // The total over the cluster's n CTAs of the value each holds at `p` (same offset in every CTA), in
 // rank order.
 __device__ __forceinline__ float cluster_sum(const float* p, int n) {
+    float v[8];  // at most 8 slices (d <= 512); every load is issued before the sum
+#pragma unroll
+    for (int r = 0; r < 8; ++r) v[r] = r < n ? ld_cluster_f32(p, (uint32_t)r) : 0.f;
     float s = 0.f;
-    for (int r = 0; r < n; ++r) s = __fadd_rn(s, ld_cluster_f32(p, (uint32_t)r));
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+        if (r < n) s = __fadd_rn(s, v[r]);
     return s;
 }
 

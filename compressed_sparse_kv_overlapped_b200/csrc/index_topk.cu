@@ -651,71 +651,96 @@ __global__ void __launch_bounds__(kScanThreads, 4) index_scan_kernel(IndexParams
         return;
     }
     const uint32_t n_bin = at - above, need = (uint32_t)p.k - above;
-    // 2. members of bins >= b1, chunk by chunk in index order: counts (written over the chunk's meta
-    //    word), then offsets, then the list
+    // 2. the members of bins >= b1, in index order.  Their source per chunk: its candidates when
+    //    b_c <= b1 (they hold every member), else its stored scores.  All source items are numbered
+    //    densely, chunk after chunk; every thread takes a contiguous range of that numbering, counts
+    //    its members, and after a block scan writes them at its offset -- loads independent of each
+    //    other, so the tail costs a few memory latencies rather than one per chunk.
     const uint32_t* meta = p.meta + (int64_t)qi * p.max_chunks;
-    uint32_t* cnt_g = p.coff + (int64_t)qi * p.max_chunks;  // per chunk: count, then offset
     const float* srow = p.scores + (int64_t)qi * p.e_stride;
     const uint64_t* cand_q = p.cand + (int64_t)qi * p.max_chunks * cap;
-    auto chunk_items = [&](int c, uint32_t mw, bool count_only, uint32_t off, uint64_t* dst) -> uint32_t {
-        // one warp: the chunk's members of bins >= b1, in index order
-        const uint32_t bcc = mw >> 16, nc = mw & 0xFFFFu;
-        uint32_t found = 0;
-        if (bcc <= b1) {
-            const uint64_t* cd = cand_q + (int64_t)c * cap;
-            for (uint32_t i0 = 0; i0 < nc; i0 += 32) {
-                const uint32_t i = i0 + lane;
-                const uint64_t v = i < nc ? __ldcg(reinterpret_cast<const unsigned long long*>(cd) + i) : 0ull;
-                const bool hit = i < nc && (uint32_t)(v >> 53) >= b1;
-                const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-                if (!count_only && hit) dst[off + found + __popc(bal & ((1u << lane) - 1u))] = v;
-                found += __popc(bal);
-            }
-        } else {
-            const int64_t e0 = (int64_t)c * chunk, e1 = min(E, e0 + chunk);
-            for (int64_t j0 = e0; j0 < e1; j0 += 32) {
-                const int64_t j = j0 + lane;
-                const uint32_t key = j < e1 ? float_key(__ldcg(srow + j)) : 0u;
-                const bool hit = j < e1 && (key >> 21) >= b1;
-                const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-                if (!count_only && hit) dst[off + found + __popc(bal & ((1u << lane) - 1u))] = composite(key, j);
-                found += __popc(bal);
-            }
-        }
-        return found;
-    };
-    // pass A: counts, one warp per chunk
+    // src[c] = exclusive prefix of the chunks' source lengths, src[nch] = their total (in shared
+    // memory -- the histogram is not needed again before the radix select clears it -- or, for more
+    // chunks than it holds, in the global per-chunk words)
+    uint32_t* src = nch < kHistBins ? hist : p.coff + (int64_t)qi * p.max_chunks;
     __shared__ uint32_t s_tot;
-    for (int c = warp; c < nch; c += kScanThreads / 32) {
-        const uint32_t f = chunk_items(c, __ldcg(meta + c), true, 0, nullptr);
-        if (lane == 0) cnt_g[c] = f;
-    }
-    __threadfence_block();
-    __syncthreads();
-    // offsets: exclusive scan over the chunk counts, kScanThreads chunks at a time (in place)
     {
         uint32_t carry = 0;
         for (int cb = 0; cb < nch; cb += kScanThreads) {
             const int c = cb + tid;
-            const uint32_t v = c < nch ? __ldcg(cnt_g + c) : 0u;
+            uint32_t len = 0;
+            if (c < nch) {
+                const uint32_t mw = __ldcg(meta + c);
+                len = (mw >> 16) <= b1 ? (mw & 0xFFFFu) : (uint32_t)(min(E, (int64_t)(c + 1) * chunk) - (int64_t)c * chunk);
+            }
             uint32_t tot;
-            const uint32_t ex = excl_scan<kScanThreads>(v, s_wsum, &tot);
-            if (c < nch) cnt_g[c] = carry + ex;
+            const uint32_t ex = excl_scan<kScanThreads>(len, s_wsum, &tot);
+            if (c < nch) src[c] = carry + ex;
             carry += tot;
         }
-        if (tid == 0) s_tot = carry;
+        if (tid == 0) {
+            src[nch] = carry;
+            s_tot = carry;
+        }
     }
     __threadfence_block();
     __syncthreads();
-    const uint32_t n_tot = s_tot;
+    const uint32_t S = s_tot;
+    const uint32_t per = (S + kScanThreads - 1) / kScanThreads;
+    const uint32_t d0 = min(S, tid * per), d1 = min(S, d0 + per);
+    // the chunk holding dense item d0: the last c with src[c] <= d0
+    int c_first = 0;
+    {
+        int lo = 0, hi = nch - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (src[mid] <= d0) lo = mid; else hi = mid - 1;
+        }
+        c_first = lo;
+    }
+    // visit dense items [d0, d1) in batches of 8 (loads issued together), calling f(key) for members
+    auto visit = [&](auto&& f) {
+        int c = c_first;
+        uint32_t c_lo = src[c], c_hi = src[c + 1];
+        bool from_cand = (__ldcg(meta + c) >> 16) <= b1;
+        for (uint32_t i0 = d0; i0 < d1; i0 += 8) {
+            uint64_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t i = i0 + u;
+                v[u] = 0ull;
+                if (i < d1) {
+                    while (i >= c_hi) {  // next chunk with items
+                        ++c;
+                        c_lo = c_hi;
+                        c_hi = src[c + 1];
+                        from_cand = (__ldcg(meta + c) >> 16) <= b1;
+                    }
+                    const uint32_t slot = i - c_lo;
+                    if (from_cand) {
+                        v[u] = __ldcg(reinterpret_cast<const unsigned long long*>(cand_q + (int64_t)c * cap) + slot);
+                    } else {
+                        const int64_t j = (int64_t)c * chunk + slot;
+                        v[u] = composite(float_key(__ldcg(srow + j)), j);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u < d1 && (uint32_t)(v[u] >> 53) >= b1) f(v[u]);
+        }
+    };
+    uint32_t n_mine = 0;
+    visit([&](uint64_t) { ++n_mine; });
+    uint32_t n_tot;
+    uint32_t pos = excl_scan<kScanThreads>(n_mine, s_wsum, &n_tot);
     if (n_tot != at) {  // the members must be exactly the histogram's count of bins >= b1
         if (tid == 0) report(p.status, CSA_ERR_INDEX);
         return;
     }
     const bool in_smem = n_tot <= (uint32_t)kListKeys;
     uint64_t* lst = in_smem ? reinterpret_cast<uint64_t*>(dsm) : p.seg + (int64_t)qi * p.e_seg;
-    // pass B: the list
-    for (int c = warp; c < nch; c += kScanThreads / 32) chunk_items(c, __ldcg(meta + c), false, __ldcg(cnt_g + c), lst);
+    visit([&](uint64_t v) { lst[pos++] = v; });
     __threadfence_block();
     __syncthreads();
     // 3. the exact threshold inside bin b1, then compaction in index order
