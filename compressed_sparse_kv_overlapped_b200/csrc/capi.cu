@@ -145,10 +145,13 @@ constexpr int kPlanSMs = 148;
 // fits).  The HCA items start when the scan frees SMs and finish by the time the front items do;
 // fewer, longer ones leave fewer partials to merge (measured at ctx1m: 8 tiles per item beat 5).
 constexpr int kHcaMinKeys = 512;
-// The CTAs of each group of `cluster` consecutive items of a query merge their results through
-// distributed shared memory (one partial per group reaches the merge kernel); both parts' item
-// counts are rounded up to a multiple of it (the extra items are empty).
-constexpr int kDecodeCluster = 8;
+// With CSA_DECODE_CLUSTER = 2, 4 or 8, the CTAs of each group of that many consecutive items of a
+// query merge their results through distributed shared memory (one partial per group reaches the
+// merge kernel); both parts' item counts are rounded up to a multiple of it (the extra items are
+// empty).  Off by default: at four 1M-token sequences the rounding takes the plan from 132 CTAs to
+// 160, and a cluster has to find all its SMs free in one GPC, so the items no longer fit one wave;
+// the merge kernel it saves costs less than the second wave.
+constexpr int kDecodeCluster = 1;
 ItemPlan plan_decode_items(const csa_dims& d, int B, int64_t max_eh, int* cluster) {
     const int f = env_int("CSA_KPI_FRONT", 0), h = env_int("CSA_KPI_HCA", 0);
     const int cl = env_int("CSA_DECODE_CLUSTER", kDecodeCluster);
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
             part4<false>(lg, xv, kv, p.bias_h + (int64_t)(4 * ub) * d + c0, d, P);
             hca_tree(P, nb, xs);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) hv[i] = __fdiv_rn(P.acc[i], P.den[i]);
+            for (int i = 0; i < 8; ++i) hv[i] = entry_div(P.acc[i], P.den[i]);
         } else if (tid >= 128 && tid < 136) {
             compress_entry8(h, p.m_hca, p.m_hca, d, p.d_I, c0s + 8 * (tid - 128), p.x, p.logit_h, p.bias_h,
                             nullptr, sq.tok_off, p.hca_entries + (sq.hca_off + h) * d, nullptr);

@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_cons
         const bool holder = (u & (nb - 1)) == 0 && (nb < 8 || lane < 8);
         h_mine = loaded && holder && h >= h_lo && h < h_hi;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) hv[i] = __fdiv_rn(P.acc[i], P.den[i]);
+        for (int i = 0; i < 8; ++i) hv[i] = entry_div(P.acc[i], P.den[i]);
     }
     float inv_c = 1.f, inv_h = 1.f;
     if (norm) {

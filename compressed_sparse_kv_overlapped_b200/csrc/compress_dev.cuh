@@ -12,6 +12,12 @@
 
 namespace csa {
 
+// The softmax runs in base 2: a logit z (plus its bias) enters as z * log2(e), and every weight is
+// 2^(difference) from the hardware exp2 approximation (relative error about 2^-22, far below the
+// bf16 rounding of the entries), one subtraction and one special-function op per weight.  Maxima
+// (M) are kept in the same base-2 scale.
+constexpr float kLog2e = 1.4426950408889634f;
+
 // Channels [c0, c0+8) of entry j of one sequence (token rows start at tok0), written as bf16 to
 // out_row (+ c0) and, when key_row != nullptr, the indexer key channels to key_row (+ c0).
 // An online softmax over the window in fp32.  Tokens are taken 4 at a time: the loads of a batch
@@ -52,17 +58,19 @@ __device__ __forceinline__ void compress_entry8(int64_t j, int m, int win, int d
             const float4 b0v = __ldg(bp), b1v = __ldg(bp + 1);  // parameters: L1/L2 resident
             z[0] += b0v.x; z[1] += b0v.y; z[2] += b0v.z; z[3] += b0v.w;
             z[4] += b1v.x; z[5] += b1v.y; z[6] += b1v.z; z[7] += b1v.w;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) z[i] *= kLog2e;
             if (want_key) unpack8(kv[u], kf);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 if (z[i] > mx[i]) {
-                    const float r = expf(mx[i] - z[i]);  // 0 on the first token (mx = -inf)
+                    const float r = fast_exp2(mx[i] - z[i]);  // 0 on the first token (mx = -inf)
                     den[i] = den[i] * r + 1.f;
                     acc[i] = acc[i] * r + xf[i];
                     if (want_key) acck[i] = acck[i] * r + kf[i];
                     mx[i] = z[i];
                 } else {
-                    const float e = expf(z[i] - mx[i]);
+                    const float e = fast_exp2(z[i] - mx[i]);
                     den[i] += e;
                     acc[i] = fmaf(e, xf[i], acc[i]);
                     if (want_key) acck[i] = fmaf(e, kf[i], acck[i]);
@@ -89,8 +97,9 @@ __device__ __forceinline__ void compress_entry8(int64_t j, int m, int win, int d
 
 // ---------------------------------------------------------------------------------------------
 // Block-partial form (CSA ratio m = 4, HCA ratio m' a power of two from 4 to 128).  Per channel
-// the softmax over a window is built from 4-token partials (M = max of the block's logits, den =
-// sum exp(z - M), acc = sum exp(z - M) * x), merged pairwise:
+// the softmax over a window is built from 4-token partials (z = logit + bias, M = max of the
+// block's z in the base-2 scale, den = sum 2^(z log2(e) - M), acc = the same weights times x),
+// merged pairwise:
 //   CSA entry j = merge(P(tokens 4j-4..4j-1, bias rows 0..3), P(tokens 4j..4j+3, bias rows 4..7)),
 //                 entry 0 = P(tokens 0..3, bias rows 4..7) alone (its window is clipped at 0);
 //   HCA entry h = the balanced binary merge tree over its m'/4 blocks, in block order.
@@ -115,13 +124,17 @@ __device__ __forceinline__ void part4(const uint4 (&lg)[4], const uint4 (&xv)[4]
         unpack8(lg[t], f);
         const float4 b0 = __ldg(reinterpret_cast<const float4*>(brow + t * d));
         const float4 b1 = __ldg(reinterpret_cast<const float4*>(brow + t * d) + 1);
-        z[t][0] = __fadd_rn(f[0], b0.x); z[t][1] = __fadd_rn(f[1], b0.y);
-        z[t][2] = __fadd_rn(f[2], b0.z); z[t][3] = __fadd_rn(f[3], b0.w);
-        z[t][4] = __fadd_rn(f[4], b1.x); z[t][5] = __fadd_rn(f[5], b1.y);
-        z[t][6] = __fadd_rn(f[6], b1.z); z[t][7] = __fadd_rn(f[7], b1.w);
-    }
+        const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) P.M[i] = fmaxf(fmaxf(z[0][i], z[1][i]), fmaxf(z[2][i], z[3][i]));
+        for (int i = 0; i < 8; ++i) z[t][i] = __fadd_rn(f[i], b[i]);
+    }
+    // M in the base-2 scale; a weight is 2^(z log2(e) - M), one fused multiply-add and one exp2
+    float nM[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        P.M[i] = __fmul_rn(fmaxf(fmaxf(z[0][i], z[1][i]), fmaxf(z[2][i], z[3][i])), kLog2e);
+        nM[i] = -P.M[i];
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) { P.den[i] = 0.f; P.acc[i] = 0.f; P.acck[i] = 0.f; }
 #pragma unroll
@@ -131,7 +144,7 @@ __device__ __forceinline__ void part4(const uint4 (&lg)[4], const uint4 (&xv)[4]
         if (KEYS) unpack8(kv[t], kf);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float e = expf(__fsub_rn(z[t][i], P.M[i]));
+            const float e = fast_exp2(__fmaf_rn(z[t][i], kLog2e, nM[i]));
             P.den[i] = __fadd_rn(P.den[i], e);
             P.acc[i] = __fmaf_rn(e, xf[i], P.acc[i]);
             if (KEYS) P.acck[i] = __fmaf_rn(e, kf[i], P.acck[i]);
@@ -145,8 +158,8 @@ __device__ __forceinline__ void merge8(Part8& A, const Part8& B) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float M = fmaxf(A.M[i], B.M[i]);
-        const float fa = expf(__fsub_rn(A.M[i], M));
-        const float fb = expf(__fsub_rn(B.M[i], M));
+        const float fa = fast_exp2(__fsub_rn(A.M[i], M));
+        const float fb = fast_exp2(__fsub_rn(B.M[i], M));
         A.den[i] = __fadd_rn(__fmul_rn(fa, A.den[i]), __fmul_rn(fb, B.den[i]));
         A.acc[i] = __fadd_rn(__fmul_rn(fa, A.acc[i]), __fmul_rn(fb, B.acc[i]));
         if (KEYS) A.acck[i] = __fadd_rn(__fmul_rn(fa, A.acck[i]), __fmul_rn(fb, B.acck[i]));
@@ -154,13 +167,18 @@ __device__ __forceinline__ void merge8(Part8& A, const Part8& B) {
     }
 }
 
+// acc / den.  den lies in [1, window] (the largest weight of a window is 2^0), so the fast
+// reciprocal-based division is safe; its error (about 2 ulp in fp32) is far below the bf16
+// rounding of the entries.
+__device__ __forceinline__ float entry_div(float acc, float den) { return __fdividef(acc, den); }
+
 // acc / den, rounded to bf16 (and the key accumulator with KEYS).
 __device__ __forceinline__ uint4 finish8(const float (&acc)[8], const float (&den)[8]) {
     uint4 o;
-    o.x = pack_bf16x2(__fdiv_rn(acc[0], den[0]), __fdiv_rn(acc[1], den[1]));
-    o.y = pack_bf16x2(__fdiv_rn(acc[2], den[2]), __fdiv_rn(acc[3], den[3]));
-    o.z = pack_bf16x2(__fdiv_rn(acc[4], den[4]), __fdiv_rn(acc[5], den[5]));
-    o.w = pack_bf16x2(__fdiv_rn(acc[6], den[6]), __fdiv_rn(acc[7], den[7]));
+    o.x = pack_bf16x2(entry_div(acc[0], den[0]), entry_div(acc[1], den[1]));
+    o.y = pack_bf16x2(entry_div(acc[2], den[2]), entry_div(acc[3], den[3]));
+    o.z = pack_bf16x2(entry_div(acc[4], den[4]), entry_div(acc[5], den[5]));
+    o.w = pack_bf16x2(entry_div(acc[6], den[6]), entry_div(acc[7], den[7]));
     return o;
 }
 
@@ -202,7 +220,7 @@ __device__ __forceinline__ void csa_entry_block4(int64_t j, int d, const float* 
         merge8<KEYS>(cur, prev);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) val[i] = __fdiv_rn(cur.acc[i], cur.den[i]);
+    for (int i = 0; i < 8; ++i) val[i] = entry_div(cur.acc[i], cur.den[i]);
     if (KEYS) *key = finish8(cur.acck, cur.den);
 }
 

@@ -21,13 +21,14 @@ namespace {
 constexpr int kNoAllocMaxQ = 16;
 constexpr int64_t kNoAllocMaxSlots = int64_t(1) << 20;  // Q * score-row stride
 // Upper bound of index_ws_bytes(Q, e_stride) under the two limits above (each array rounded up to
-// 256 bytes): histograms and tickets; fp32 scores; 64-bit kept-entry segments (each query's score
-// row plus 128 entries); two words per scan chunk (chunks of at least 256 entries, one more per
-// query for a partial chunk); candidate keys (a quarter of the entries plus 256 per query).
-constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * (kHistBins + 1) * 4 + 256 +   // histograms, tickets
+// 256 bytes): histograms; fp32 scores; 64-bit kept-entry segments (each query's score
+// row plus 128 entries); two words per scan chunk (chunks of at least 256 entries, nine more per
+// query: a partial chunk and the ends of the final select's per-CTA prefixes); candidate keys (a
+// quarter of the entries plus 256 per query).
+constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * kHistBins * 4 + 256 +         // histograms
                                  size_t(kNoAllocMaxSlots) * 4 + 256 +                  // scores
                                  size_t(kNoAllocMaxSlots + kNoAllocMaxQ * kSegPad) * 8 + 256 +
-                                 2 * (size_t(kNoAllocMaxSlots / 256 + kNoAllocMaxQ) * 4 + 256) +
+                                 2 * (size_t(kNoAllocMaxSlots / 256 + 9 * kNoAllocMaxQ) * 4 + 256) +
                                  size_t(kNoAllocMaxSlots / 4 + kNoAllocMaxQ * 256) * 8 + 256;
 
 __device__ __align__(256) unsigned char g_index_scratch[kScratchBytes];

@@ -9,14 +9,15 @@
 // selection works on the 64-bit key (order-preserving score key << 32 | ~index), which is unique
 // and breaks ties to the lower index.
 //
-// Two kernels:
+// Three kernels:
 //  index_scan_kernel   -- grid (chunks, queries), the decode / standalone path.  Streams the
 //            indexer-key cache with coalesced 16-byte loads and computes the [16 entries x d_I] .
 //            [d_I x H_I] products on the tensor cores (mma.sync m16n8k16, K permuted so that every
 //            thread's operand is one contiguous 16-byte load), applies relu / head weights in
 //            registers, and counts the scores into the query's histogram of the top 11 key bits.
-//            Each chunk keeps its local candidates; the last chunk of a query to finish (atomic
-//            ticket, no spinning) selects the exact top-k from them (see the kernel).
+//            Each chunk keeps its local candidates.
+//  index_final_kernel  -- one thread-block cluster per query after the scan: the exact top-k from
+//            the chunks' candidates (see the kernel).
 //  index_select_kernel -- one CTA per query, the prefill path: the top-k of a score row that the
 //            prefill GEMM stored, with a threshold bin estimated from a sample of the row.
 #include "common.cuh"
@@ -58,13 +59,15 @@ template <int KV>
 __device__ __forceinline__ void score16(const uint16_t* keys, int64_t r0, int64_t nrows, int g, int c,
                                         const uint32_t (&bq)[2 * KV][2], const float (&wv)[2], uint64_t pol,
                                         float& s_lo, float& s_hi) {
-    // thread (g, c) loads rows g and g+8, vectors [32*v + 8c, 32*v + 8c + 8) for v < KV
+    // thread (g, c) loads rows g and g+8, vectors [32*v + 8c, 32*v + 8c + 8) for v < KV.  Rows past
+    // the end (scores the caller drops) load the last row instead: the loads stay unconditional,
+    // so none waits at a branch join before the next is issued.
     uint4 lo[KV], hi[KV];
-    const int64_t rl = r0 + g, rh = r0 + g + 8;
+    const int64_t rl = min(r0 + g, nrows - 1), rh = min(r0 + g + 8, nrows - 1);
 #pragma unroll
     for (int v = 0; v < KV; ++v) {
-        lo[v] = rl < nrows ? ld_stream(keys + rl * (KV * 32) + v * 32 + c * 8, pol) : make_uint4(0, 0, 0, 0);
-        hi[v] = rh < nrows ? ld_stream(keys + rh * (KV * 32) + v * 32 + c * 8, pol) : make_uint4(0, 0, 0, 0);
+        lo[v] = ld_stream(keys + rl * (KV * 32) + v * 32 + c * 8, pol);
+        hi[v] = ld_stream(keys + rh * (KV * 32) + v * 32 + c * 8, pol);
     }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -120,16 +123,17 @@ __device__ __forceinline__ void score16_mx8(const uint8_t* keys, const uint8_t* 
                                             int g, int c, const uint32_t (&bq)[2 * NB][2], const float (&wv)[2],
                                             const int (&qsh)[2], uint64_t pol, float& s_lo, float& s_hi) {
     constexpr int DI = 32 * NB;
+    // rows past the end (scores the caller drops) load the last row: unconditional loads (see score16)
     uint2 lo[NB], hi[NB];
-    uint32_t sl = 0x7F7F7F7Fu, sh = 0x7F7F7F7Fu;  // scale bytes of rows g and g + 8 (2^0 past the end)
-    const int64_t rl = r0 + g, rh = r0 + g + 8;
+    const int64_t rl = min(r0 + g, nrows - 1), rh = min(r0 + g + 8, nrows - 1);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-        lo[b] = rl < nrows ? ld_stream8(keys + rl * DI + b * 32 + c * 8, pol) : make_uint2(0, 0);
-        hi[b] = rh < nrows ? ld_stream8(keys + rh * DI + b * 32 + c * 8, pol) : make_uint2(0, 0);
+        lo[b] = ld_stream8(keys + rl * DI + b * 32 + c * 8, pol);
+        hi[b] = ld_stream8(keys + rh * DI + b * 32 + c * 8, pol);
     }
-    if (rl < nrows) sl = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rl * NB) : scales[rl];
-    if (rh < nrows) sh = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rh * NB) : scales[rh];
+    // scale bytes of rows g and g + 8
+    const uint32_t sl = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rl * NB) : scales[rl];
+    const uint32_t sh = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rh * NB) : scales[rh];
     float tot[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
@@ -170,6 +174,7 @@ __device__ __forceinline__ uint64_t composite(uint32_t key, int64_t j) {
 }
 
 // Exclusive prefix of one value per thread; *total gets the block's sum.  wsum: NT/32 words.
+// Two barriers: the warps' totals are published, then every warp sums the ones before it.
 template <int NT>
 __device__ __forceinline__ uint32_t excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -181,41 +186,44 @@ __device__ __forceinline__ uint32_t excl_scan(uint32_t v, uint32_t* wsum, uint32
     }
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-        uint32_t x = lane < NT / 32 ? wsum[lane] : 0u;
+    uint32_t before = 0, all = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane < NT / 32) wsum[lane] = x;
+    for (int w = 0; w < NT / 32; ++w) {
+        const uint32_t x = wsum[w];
+        before += w < warp ? x : 0u;
+        all += x;
     }
-    __syncthreads();
-    const uint32_t excl = (warp > 0 ? wsum[warp - 1] : 0u) + incl - v;
-    *total = wsum[NT / 32 - 1];
-    __syncthreads();
-    return excl;
+    *total = all;
+    __syncthreads();  // wsum may be written again after the return
+    return before + incl - v;
 }
 
 // Over kHistBins bins: the unique bin b with suffix(b) >= target > suffix(b + 1), where suffix(b) =
 // sum of hist[b' >= b] (target >= 1).  out[0] = b (0xFFFFFFFF if the total is below target),
 // out[1] = suffix(b + 1), out[2] = suffix(b).  Thread t owns kHistBins/NT consecutive bins counted
-// from the top, so a forward scan over threads is a suffix scan over bins.
+// from the top, so a forward scan over threads is a suffix scan over bins; it reads them with
+// 16-byte loads (hist 16-byte aligned; a quarter-warp's loads cover all banks once).
 template <int NT>
 __device__ void find_bin(const uint32_t* hist, uint32_t target, uint32_t* wsum, uint32_t* out) {
     constexpr int PER = kHistBins / NT;
+    static_assert(PER % 4 == 0, "find_bin reads its bins as 16-byte vectors");
     const int t = threadIdx.x;
     const int b0 = PER * (NT - 1 - t);  // bins [b0, b0 + PER)
+    uint32_t h[PER];
+#pragma unroll
+    for (int i = 0; i < PER / 4; ++i) {
+        const uint4 v = reinterpret_cast<const uint4*>(hist + b0)[i];
+        h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
+    }
     uint32_t part = 0;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) part += hist[b0 + i];
+    for (int i = 0; i < PER; ++i) part += h[i];
     if (t == 0) out[0] = 0xFFFFFFFFu;
     uint32_t total;
-    const uint32_t above_mine = excl_scan<NT>(part, wsum, &total);  // bins above b0 + PER - 1
-    uint32_t above = above_mine;
+    uint32_t above = excl_scan<NT>(part, wsum, &total);  // bins above b0 + PER - 1
 #pragma unroll
     for (int i = PER - 1; i >= 0; --i) {
-        const uint32_t here = above + hist[b0 + i];
+        const uint32_t here = above + h[i];
         if (here >= target && above < target) { out[0] = (uint32_t)(b0 + i); out[1] = above; out[2] = here; }
         above = here;
     }
@@ -261,7 +269,55 @@ __device__ uint64_t radix_select(const KeyList& L, uint32_t n, uint32_t need, ui
     }
 }
 
+// Ordered compaction of one round of NT * PER items laid out warp-contiguously: lane l of warp w
+// holds item w * 32 * PER + u * 32 + l of the round as v[u], a member when keep[u].  Every load
+// of such a layout reads 32 consecutive items; the members keep item order through one ballot per
+// u and one block scan over the warps' counts.  write(written + rank, v) is called for each member
+// (rank = its place among the round's members); returns the round's member count (every thread).
+template <int NT, int PER, typename Write>
+__device__ __forceinline__ uint32_t compact_round(const uint64_t (&v)[PER], const bool (&keep)[PER], uint32_t written,
+                                                  Write&& write, uint32_t* wsum) {
+    const int lane = threadIdx.x & 31;
+    uint32_t mask[PER];
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        mask[u] = __ballot_sync(0xffffffffu, keep[u]);
+        cnt += __popc(mask[u]);
+    }
+    uint32_t tot;
+    const uint32_t ex = excl_scan<NT>(lane == 0 ? cnt : 0u, wsum, &tot);
+    uint32_t off = written + __shfl_sync(0xffffffffu, ex, 0);
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        if (keep[u]) write(off + __popc(mask[u] & lt), v[u]);
+        off += __popc(mask[u]);
+    }
+    return tot;
+}
+
+// Distributed shared memory: store 8 bytes / a word at the location `p` (an address in this CTA's
+// shared memory) in the CTA of rank `rank`, and load a word from there.
+__device__ __forceinline__ void st_cluster_u64(const void* p, uint32_t rank, uint64_t v) {
+    uint32_t a;
+    asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(a), "l"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(const void* p, uint32_t rank, uint32_t v) {
+    uint32_t a;
+    asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(const void* p, uint32_t rank) {
+    uint32_t a, v;
+    asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+
 constexpr int kListKeys = 4096;                  // keys of the final list held in shared memory
+constexpr int kTailPer = 8;                      // items per thread and round of an ordered compaction
 constexpr int kScanDynSmem = kListKeys * 8;      // dynamic shared memory: chunk scores, then the list
 static_assert(kScanDynSmem <= 48 * 1024, "no opt-in needed for the scan's dynamic shared memory");
 constexpr int64_t kScanChunkMax = kScanDynSmem / 4;
@@ -461,20 +517,14 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
 // the top 11 bits of the order-preserving score key; then the chunk's candidates -- its entries of
 // bin >= b_c, b_c the highest bin that still leaves at least kloc entries (kloc about twice the
 // chunk's expected share of the top-k) -- go to the candidate buffer in index order, with b_c.
-// The last CTA of the query to finish (atomic ticket; nothing waits) selects the exact top-k:
-// the threshold bin b1 of the query's histogram fixes the members of bins >= b1, which are exactly
-// the entries it must consider; a chunk with b_c <= b1 holds all of its members among its
-// candidates, a chunk with b_c > b1 (more than its share of the top-k) is filtered again from its
-// stored scores.  A radix select inside bin b1 on the 64-bit key (score key << 32 | ~index: unique,
-// ties to the lower index) gives the threshold, and the k indices are compacted in ascending order.
+// index_final_kernel selects the exact top-k from them.
 template <int KV, bool MX8>
-__global__ void __launch_bounds__(kScanThreads, 4) index_scan_kernel(IndexParams p) {
+__global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams p) {
     extern __shared__ __align__(16) unsigned char dsm[];
-    __shared__ uint32_t hist[kHistBins];
+    __shared__ __align__(16) uint32_t hist[kHistBins];
     __shared__ float sc[kScanThreads / 32][4][16];
     __shared__ uint32_t s_wsum[kScanThreads / 32];
     __shared__ uint32_t s_res[4];
-    __shared__ int s_last;
     float* ssc = reinterpret_cast<float*>(dsm);  // the chunk's scores
     grid_dep_wait();  // the query table may come from the previous kernel
     grid_dep_launch();
@@ -617,159 +667,257 @@ __global__ void __launch_bounds__(kScanThreads, 4) index_scan_kernel(IndexParams
     uint32_t bc = s_res[0] == 0xFFFFFFFFu ? 0u : s_res[0];
     if (s_res[0] != 0xFFFFFFFFu && s_res[2] > (uint32_t)cap) bc += 1;  // suffix(bc + 1) < kloc <= cap
     {
-        const int per = (n + kScanThreads - 1) / kScanThreads;
-        const int i0 = tid * per, i1 = min(n, i0 + per);
-        uint32_t mine = 0;
-        for (int i = i0; i < i1; ++i) mine += (float_key(ssc[i]) >> 21) >= bc ? 1u : 0u;
-        uint32_t tot;
-        uint32_t o = excl_scan<kScanThreads>(mine, s_wsum, &tot);
         uint64_t* cand = p.cand + ((int64_t)qi * p.max_chunks + cidx) * cap;
-        for (int i = i0; i < i1; ++i) {
-            const uint32_t key = float_key(ssc[i]);
-            if ((key >> 21) >= bc) cand[o++] = composite(key, c0 + i);
+        uint32_t n_cand = 0;
+        for (int base = 0; base < n; base += kScanThreads * kTailPer) {
+            const int first = base + warp * 32 * kTailPer + lane;
+            uint64_t v[kTailPer];
+            bool keep[kTailPer];
+#pragma unroll
+            for (int u = 0; u < kTailPer; ++u) {
+                const int i = first + u * 32;
+                const uint32_t key = i < n ? float_key(ssc[i]) : 0u;
+                keep[u] = i < n && (key >> 21) >= bc;
+                v[u] = composite(key, c0 + i);
+            }
+            n_cand += compact_round<kScanThreads, kTailPer>(
+                v, keep, n_cand, [&](uint32_t pos, uint64_t x) { if (pos < (uint32_t)cap) cand[pos] = x; }, s_wsum);
         }
-        if (tid == 0) p.meta[(int64_t)qi * p.max_chunks + cidx] = (bc << 16) | tot;
+        if (tid == 0) p.meta[(int64_t)qi * p.max_chunks + cidx] = (bc << 16) | n_cand;
     }
-    // ---- ticket: the last chunk of the query to finish selects
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&p.ticket[qi], 1u) == (uint32_t)(nch - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
+}
 
-    // 1. the threshold bin of the whole query
+// ---- final selection (decode / standalone path) -------------------------------------------------
+//
+// One thread-block cluster of kFinalF CTAs per query, after the scan grid.  Every CTA derives the
+// threshold bin b1 from the query's histogram (the k-th largest key lies in bin b1; the entries of
+// bins >= b1, n_tot of them, are exactly the ones to consider), then gathers those members from
+// its share of the chunks, in index order: from a chunk's candidates when b_c <= b1 (they hold all
+// of its members), else from its stored scores.  It publishes its count in the leader (rank 0);
+// after a cluster barrier each CTA stores its members at its offset of the leader's list
+// (distributed shared memory, or the global segment buffer for a list longer than shared memory
+// holds); after a second barrier the leader radix-selects the exact threshold inside bin b1 (64-bit
+// key: score key << 32 | ~index, unique, ties to the lower index) and compacts the k indices in
+// ascending order.
+constexpr int kFinalF = 8;           // CTAs per query
+constexpr int kFinalThreads = 256;
+constexpr int kFinalDynSmem = kListKeys * 8;  // the members list (also this CTA's chunk words)
+constexpr int kFinalChunks = (kHistBins - 2) / 2;  // chunks per CTA whose words fit the histogram's space
+
+__global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexParams p) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    __shared__ __align__(16) uint32_t hist[kHistBins];
+    __shared__ uint32_t s_wsum[kFinalThreads / 32];
+    __shared__ uint32_t s_res[4];
+    __shared__ uint32_t s_cnt[kFinalF];  // the leader's: members per rank
+    __shared__ uint32_t s_tot;
+    grid_dep_wait();  // the scan's histograms, candidates and scores
+    grid_dep_launch();
+    const int qi = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t rank = cluster_ctarank();
+    const csa_query qr = p.queries[qi];
+    const bool seq_ok = qr.seq >= 0 && qr.reserved == 0;
+    const csa_seq sq = seq_ok ? p.seqs[qr.seq] : csa_seq{0, 0, 0, 0};
+    const bool valid = seq_ok && qr.len >= 1 && qr.len <= sq.len;
+    const int64_t E = valid ? qr.len / p.m : 0;
+    // the scan handled (and reported) these; the outcome is uniform over the cluster
+    if (!valid || E > p.max_entries || E <= p.k) return;
+    const int64_t chunk = p.chunk;
+    const int nch = (int)((E + chunk - 1) / chunk);
+    const int cap = p.cand_cap;
+    const int cb = (int)((int64_t)nch * rank / kFinalF), ce = (int)((int64_t)nch * (rank + 1) / kFinalF);
+    const int nmine = ce - cb;
+    const uint32_t* meta = p.meta + (int64_t)qi * p.max_chunks + cb;
+    const bool words_smem = nmine <= kFinalChunks;
+    // 1. the threshold bin; the histogram and this CTA's chunk words are loaded together
+    uint32_t* mw = reinterpret_cast<uint32_t*>(dsm);
     {
         const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
-        for (int i = tid; i < kHistBins; i += kScanThreads) hist[i] = __ldcg(gh + i);
+        uint32_t hv[kHistBins / kFinalThreads];
+#pragma unroll
+        for (int i = 0; i < kHistBins / kFinalThreads; ++i) hv[i] = __ldcg(gh + tid + i * kFinalThreads);
+        if (words_smem)
+            for (int c = tid; c < nmine; c += kFinalThreads) mw[c] = __ldcg(meta + c);
+#pragma unroll
+        for (int i = 0; i < kHistBins / kFinalThreads; ++i) hist[tid + i * kFinalThreads] = hv[i];
     }
     __syncthreads();
-    find_bin<kScanThreads>(hist, (uint32_t)p.k, s_wsum, s_res);
+    find_bin<kFinalThreads>(hist, (uint32_t)p.k, s_wsum, s_res);
     const uint32_t b1 = s_res[0], above = s_res[1], at = s_res[2];
     if (b1 == 0xFFFFFFFFu) {  // the histogram holds fewer than k scores: cannot happen for E > k
-        if (tid == 0) report(p.status, CSA_ERR_INDEX);
+        if (tid == 0 && rank == 0) report(p.status, CSA_ERR_INDEX);
         return;
     }
-    const uint32_t n_bin = at - above, need = (uint32_t)p.k - above;
-    // 2. the members of bins >= b1, in index order.  Their source per chunk: its candidates when
-    //    b_c <= b1 (they hold every member), else its stored scores.  All source items are numbered
-    //    densely, chunk after chunk; every thread takes a contiguous range of that numbering, counts
-    //    its members, and after a block scan writes them at its offset -- loads independent of each
-    //    other, so the tail costs a few memory latencies rather than one per chunk.
-    const uint32_t* meta = p.meta + (int64_t)qi * p.max_chunks;
-    const float* srow = p.scores + (int64_t)qi * p.e_stride;
-    const uint64_t* cand_q = p.cand + (int64_t)qi * p.max_chunks * cap;
-    // src[c] = exclusive prefix of the chunks' source lengths, src[nch] = their total (in shared
-    // memory -- the histogram is not needed again before the radix select clears it -- or, for more
-    // chunks than it holds, in the global per-chunk words)
-    uint32_t* src = nch < kHistBins ? hist : p.coff + (int64_t)qi * p.max_chunks;
-    __shared__ uint32_t s_tot;
+    const uint32_t n_bin = at - above, need = (uint32_t)p.k - above, n_tot = at;
+    const bool in_smem = n_tot <= (uint32_t)kListKeys;
+    // 2. this CTA's source items, numbered densely chunk after chunk: src[c] = the first number of
+    //    chunk cb + c (src[nmine] = the total), flag[c] = its members come from its candidates; in
+    //    the histogram's space (free until the radix select), or the global chunk words
+    uint32_t* src = words_smem ? hist : p.coff + (int64_t)qi * (p.max_chunks + kFinalF) + cb + rank;
+    uint32_t* flag = hist + kFinalChunks + 1;
     {
         uint32_t carry = 0;
-        for (int cb = 0; cb < nch; cb += kScanThreads) {
-            const int c = cb + tid;
-            uint32_t len = 0;
-            if (c < nch) {
-                const uint32_t mw = __ldcg(meta + c);
-                len = (mw >> 16) <= b1 ? (mw & 0xFFFFu) : (uint32_t)(min(E, (int64_t)(c + 1) * chunk) - (int64_t)c * chunk);
+        for (int c0 = 0; c0 < nmine; c0 += kFinalThreads) {
+            const int c = c0 + tid;
+            uint32_t len = 0, fc = 0;
+            if (c < nmine) {
+                const uint32_t w = words_smem ? mw[c] : __ldcg(meta + c);
+                fc = (w >> 16) <= b1 ? 1u : 0u;
+                const int64_t cc = cb + c;
+                len = fc ? (w & 0xFFFFu) : (uint32_t)(min(E, (cc + 1) * chunk) - cc * chunk);
             }
             uint32_t tot;
-            const uint32_t ex = excl_scan<kScanThreads>(len, s_wsum, &tot);
-            if (c < nch) src[c] = carry + ex;
+            const uint32_t ex = excl_scan<kFinalThreads>(len, s_wsum, &tot);  // synchronizes: mw reads done
+            if (c < nmine) {
+                src[c] = carry + ex;
+                if (words_smem) flag[c] = fc;
+            }
             carry += tot;
         }
         if (tid == 0) {
-            src[nch] = carry;
+            src[nmine] = carry;
             s_tot = carry;
         }
     }
-    __threadfence_block();
+    if (!words_smem) __threadfence_block();
     __syncthreads();
     const uint32_t S = s_tot;
-    const uint32_t per = (S + kScanThreads - 1) / kScanThreads;
-    const uint32_t d0 = min(S, tid * per), d1 = min(S, d0 + per);
-    // the chunk holding dense item d0: the last c with src[c] <= d0
-    int c_first = 0;
-    {
-        int lo = 0, hi = nch - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (src[mid] <= d0) lo = mid; else hi = mid - 1;
-        }
-        c_first = lo;
-    }
-    // visit dense items [d0, d1) in batches of 8 (loads issued together), calling f(key) for members
-    auto visit = [&](auto&& f) {
-        int c = c_first;
-        uint32_t c_lo = src[c], c_hi = src[c + 1];
-        bool from_cand = (__ldcg(meta + c) >> 16) <= b1;
-        for (uint32_t i0 = d0; i0 < d1; i0 += 8) {
-            uint64_t v[8];
+    auto src_at = [&](int c) -> uint32_t { return words_smem ? src[c] : __ldcg(src + c); };
+    auto from_cand = [&](int c) -> bool { return words_smem ? flag[c] != 0u : (__ldcg(meta + c) >> 16) <= b1; };
+    const unsigned long long* cand_q =
+        reinterpret_cast<const unsigned long long*>(p.cand) + ((int64_t)qi * p.max_chunks + cb) * cap;
+    const float* srow_q = p.scores + (int64_t)qi * p.e_stride;
+    uint64_t* lst = reinterpret_cast<uint64_t*>(dsm);  // this CTA's members; the leader's: the whole list
+    uint64_t* gseg = p.seg + (int64_t)qi * p.e_seg;
+    // One pass over the source items in rounds of kTailPer per thread, laid out warp-contiguously
+    // (see compact_round).  All addresses of a round are found first (chunk boundaries from shared
+    // memory), then the loads are issued unconditionally, back to back, so a round costs one memory
+    // latency (a load inside the data-dependent branches would be consumed at their join, one
+    // latency per item).  An item of a stored-score chunk loads the aligned 8-byte word holding its
+    // score (a word reaching 4 bytes past the score rows stays inside the workspace: the segment
+    // buffer follows them).  Members are handed to sink(position among this CTA's members, key).
+    auto gather = [&](auto&& sink) -> uint32_t {
+        uint32_t written = 0;
+        for (uint32_t base = 0; base < S; base += kFinalThreads * kTailPer) {
+            const uint32_t first = base + (uint32_t)(warp * 32 * kTailPer + lane);
+            int c = 0;
+            if (first < S) {  // the chunk holding item `first`: the last c with src[c] <= first
+                int lo = 0, hi = nmine - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (src_at(mid) <= first) lo = mid; else hi = mid - 1;
+                }
+                c = lo;
+            }
+            const unsigned long long* ad[kTailPer];
+            uint32_t jk[kTailPer];  // bit 31: a stored score, bit 30: in the high half of its word; bits 0..29: j
+            uint32_t c_lo = first < S ? src_at(c) : 0u, c_hi = first < S ? src_at(c + 1) : 0u;
+            bool fcand = first < S && from_cand(c);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const uint32_t i = i0 + u;
-                v[u] = 0ull;
-                if (i < d1) {
+            for (int u = 0; u < kTailPer; ++u) {
+                const uint32_t i = first + u * 32;
+                ad[u] = cand_q;  // a valid address for an empty slot
+                jk[u] = 0u;
+                if (i < S) {
                     while (i >= c_hi) {  // next chunk with items
                         ++c;
                         c_lo = c_hi;
-                        c_hi = src[c + 1];
-                        from_cand = (__ldcg(meta + c) >> 16) <= b1;
+                        c_hi = src_at(c + 1);
+                        fcand = from_cand(c);
                     }
                     const uint32_t slot = i - c_lo;
-                    if (from_cand) {
-                        v[u] = __ldcg(reinterpret_cast<const unsigned long long*>(cand_q + (int64_t)c * cap) + slot);
+                    if (fcand) {
+                        ad[u] = cand_q + (int64_t)c * cap + slot;
                     } else {
-                        const int64_t j = (int64_t)c * chunk + slot;
-                        v[u] = composite(float_key(__ldcg(srow + j)), j);
+                        const uint32_t j = (uint32_t)((int64_t)(cb + c) * chunk + slot);
+                        const uintptr_t f = reinterpret_cast<uintptr_t>(srow_q + j);
+                        ad[u] = reinterpret_cast<const unsigned long long*>(f & ~(uintptr_t)7);
+                        jk[u] = 0x80000000u | ((f & 4) ? 0x40000000u : 0u) | j;
                     }
                 }
             }
+            uint64_t v[kTailPer];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (i0 + u < d1 && (uint32_t)(v[u] >> 53) >= b1) f(v[u]);
+            for (int u = 0; u < kTailPer; ++u) v[u] = __ldcg(ad[u]);
+            bool keep[kTailPer];
+#pragma unroll
+            for (int u = 0; u < kTailPer; ++u) {
+                if (jk[u] & 0x80000000u) {
+                    const uint32_t w = (jk[u] & 0x40000000u) ? (uint32_t)(v[u] >> 32) : (uint32_t)v[u];
+                    v[u] = composite(float_key(__uint_as_float(w)), jk[u] & 0x3FFFFFFFu);
+                }
+                keep[u] = first + u * 32 < S && (uint32_t)(v[u] >> 53) >= b1;
+            }
+            written += compact_round<kFinalThreads, kTailPer>(v, keep, written, sink, s_wsum);
         }
+        return written;
     };
-    uint32_t n_mine = 0;
-    visit([&](uint64_t) { ++n_mine; });
-    uint32_t n_tot;
-    uint32_t pos = excl_scan<kScanThreads>(n_mine, s_wsum, &n_tot);
-    if (n_tot != at) {  // the members must be exactly the histogram's count of bins >= b1
-        if (tid == 0) report(p.status, CSA_ERR_INDEX);
+    // 3. members into the list: kept in this CTA's shared memory first (a list that fits), counts to
+    //    the leader, then every CTA stores its members at its offset of the leader's list
+    const uint32_t n_mine = gather([&](uint32_t pos, uint64_t x) {
+        if (in_smem && pos < (uint32_t)kListKeys) lst[pos] = x;
+    });
+    if (tid == 0) st_cluster_u32(&s_cnt[rank], 0, n_mine);
+    cluster_barrier();
+    uint32_t off, total;  // members of the ranks before this one, of all ranks
+    {
+        const uint32_t cr = lane < kFinalF ? ld_cluster_u32(&s_cnt[lane], 0) : 0u;
+        off = (uint32_t)lane < rank ? cr : 0u;
+        total = cr;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            off += __shfl_xor_sync(0xffffffffu, off, o);
+            total += __shfl_xor_sync(0xffffffffu, total, o);
+        }
+    }
+    if (total != n_tot) {  // the members must be exactly the histogram's count of bins >= b1
+        if (tid == 0 && rank == 0) report(p.status, CSA_ERR_INDEX);
+        cluster_barrier();  // every CTA takes the same barriers
         return;
     }
-    const bool in_smem = n_tot <= (uint32_t)kListKeys;
-    uint64_t* lst = in_smem ? reinterpret_cast<uint64_t*>(dsm) : p.seg + (int64_t)qi * p.e_seg;
-    visit([&](uint64_t v) { lst[pos++] = v; });
-    __threadfence_block();
-    __syncthreads();
-    // 3. the exact threshold inside bin b1, then compaction in index order
-    const KeyList L{in_smem ? lst : nullptr, in_smem ? nullptr : lst};
-    const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53) : radix_select<kScanThreads>(L, n_tot, need, b1, hist,
-                                                                                          s_wsum, s_res);
-    const uint32_t per_t = (n_tot + kScanThreads - 1) / kScanThreads;
-    const uint32_t i0 = tid * per_t, i1 = min(n_tot, i0 + per_t);
-    uint32_t mine = 0;
-    for (uint32_t i = i0; i < i1; ++i) mine += L.get(i) >= T ? 1u : 0u;
-    uint32_t kept_total;
-    uint32_t o = excl_scan<kScanThreads>(mine, s_wsum, &kept_total);
-    for (uint32_t i = i0; i < i1; ++i) {
-        const uint64_t v = L.get(i);
-        if (v >= T) {
-            if (o < (uint32_t)p.k) {
-                const uint32_t j = 0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull);
-                out[o] = (int32_t)j;
-                if (sout) sout[o] = key_float((uint32_t)(v >> 32));
-                // the attention that follows gathers these rows: start bringing them into L2 now
-                if (p.prefetch_rows) prefetch_l2(p.prefetch_rows + (sq.csa_off + j) * p.prefetch_row_bytes,
-                                                 p.prefetch_row_bytes);
-            }
-            ++o;
-        }
+    if (in_smem) {
+        if (rank != 0)
+            for (uint32_t i = tid; i < n_mine; i += kFinalThreads) st_cluster_u64(&lst[off + i], 0, lst[i]);
+    } else {
+        gather([&](uint32_t pos, uint64_t x) { gseg[off + pos] = x; });
     }
-    if (tid == 0 && kept_total != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
+    cluster_barrier();  // the leader's list is complete
+    int32_t* out = p.idx_out + (int64_t)qi * p.k;
+    if (rank == 0) {
+        // 4. the exact threshold inside bin b1, then compaction in index order
+        const KeyList L{in_smem ? lst : nullptr, in_smem ? nullptr : gseg};
+        const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53) : radix_select<kFinalThreads>(L, n_tot, need, b1, hist,
+                                                                                               s_wsum, s_res);
+        float* sout = p.score_out ? p.score_out + (int64_t)qi * p.k : nullptr;
+        uint32_t kept = 0;
+        for (uint32_t base = 0; base < n_tot; base += kFinalThreads * kTailPer) {
+            const uint32_t first = base + (uint32_t)(warp * 32 * kTailPer + lane);
+            uint64_t v[kTailPer];
+            bool keep[kTailPer];
+#pragma unroll
+            for (int u = 0; u < kTailPer; ++u) {
+                const uint32_t i = first + u * 32;
+                v[u] = i < n_tot ? L.get(i) : 0ull;
+                keep[u] = i < n_tot && v[u] >= T;
+            }
+            kept += compact_round<kFinalThreads, kTailPer>(v, keep, kept, [&](uint32_t o, uint64_t x) {
+                if (o < (uint32_t)p.k) {
+                    out[o] = (int32_t)(0xFFFFFFFFu - (uint32_t)(x & 0xFFFFFFFFull));
+                    if (sout) sout[o] = key_float((uint32_t)(x >> 32));
+                }
+            }, s_wsum);
+        }
+        if (tid == 0 && kept != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
+    }
+    if (!p.prefetch_rows) return;  // (uniform over the cluster)
+    cluster_barrier();  // the indices are out (the barrier orders global memory at cluster scope)
+    // 5. the attention that follows gathers the selected rows: every CTA of the cluster starts
+    //    bringing its share of them into L2
+    for (int o = (int)rank * kFinalThreads + tid; o < p.k; o += kFinalF * kFinalThreads) {
+        const int32_t j = __ldcg(out + o);
+        if (j >= 0) prefetch_l2(p.prefetch_rows + (sq.csa_off + j) * p.prefetch_row_bytes, p.prefetch_row_bytes);
+    }
 }
-
 constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 }  // namespace
@@ -777,8 +925,10 @@ constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 namespace {
 
 // Scan chunking of Q queries of up to e_stride entries: chunks of a multiple of 64 entries sized so
-// that all chunks make about one wave of four scan CTAs per SM (so SMs carry equal shares), at least
-// 256 and at most what the chunk's score buffer in shared memory holds.
+// that all chunks make about one wave of two scan CTAs per SM (so SMs carry equal shares), at least
+// 256 and at most what the chunk's score buffer in shared memory holds.  Two CTAs, not more: a pass
+// keeps its sixteen 16-byte key loads per thread in registers (up to 128 per thread), and the
+// loads in flight, not the warp count, set the streaming rate.
 struct ScanPlan {
     int64_t chunk;
     int max_chunks;
@@ -786,7 +936,7 @@ struct ScanPlan {
 };
 
 ScanPlan scan_plan(int Q, int64_t e_stride) {
-    constexpr int64_t kSlots = 148 * 4;
+    constexpr int64_t kSlots = 148 * 2;
     ScanPlan sp;
     int64_t c = (e_stride * Q + kSlots - 1) / kSlots;
     c = ((c + 63) / 64) * 64;
@@ -800,13 +950,15 @@ ScanPlan scan_plan(int Q, int64_t e_stride) {
 
 // Per-chunk words and candidate keys are sized by bounds that hold for every chunk size the plan
 // can choose (chunks of at least 256 entries keeping at most a quarter of their entries, at most
-// 256), so the workspace of Q queries also serves any smaller query count.
-size_t chunk_words(int Q, int64_t e_stride) { return (size_t)Q * (size_t)(e_stride / 256 + 1); }
+// 256), so the workspace of Q queries also serves any smaller query count.  A query's chunk words
+// hold max_chunks + kFinalF entries (the final select's prefix over a CTA's chunks has one more,
+// per CTA).
+size_t chunk_words(int Q, int64_t e_stride) { return (size_t)Q * (size_t)(e_stride / 256 + 1 + kFinalF); }
 size_t cand_keys(int Q, int64_t e_stride) { return (size_t)Q * (size_t)(e_stride / 4 + 256); }
 
 }  // namespace
 
-size_t index_zero_bytes(int Q) { return align256((size_t)Q * (kHistBins + 1) * 4); }
+size_t index_zero_bytes(int Q) { return align256((size_t)Q * kHistBins * 4); }
 
 size_t index_ws_bytes(int Q, int64_t e_stride) {
     size_t s = index_zero_bytes(Q);
@@ -821,7 +973,6 @@ void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
     const ScanPlan sp = scan_plan(Q, e_stride);
     char* b = static_cast<char*>(ws);
     p.hist = reinterpret_cast<uint32_t*>(b);
-    p.ticket = p.hist + (size_t)Q * kHistBins;
     b += index_zero_bytes(Q);
     p.scores = reinterpret_cast<float*>(b);
     b += align256((size_t)Q * e_stride * 4);
@@ -855,10 +1006,12 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
         return launch_kernel(index_select_kernel, dim3((unsigned)p.Q), dim3(kSelectThreads), smem, stream, pdl, p);
     }
     if (zero_ws) {
-        // the histograms and tickets sit at the start of the workspace
+        // the histograms sit at the start of the workspace
         cudaError_t e = cudaMemsetAsync(p.hist, 0, index_zero_bytes(p.Q), stream);
         if (e != cudaSuccess) return e;
     }
+    // the scan's final select packs entry indices into 30 bits
+    if (max_entries >= (int64_t(1) << 30)) return cudaErrorInvalidValue;
     cudaError_t e;
     // chunk 0 of a query that selects all of its entries writes the result alone
     const int64_t gx = max_entries > p.k ? (max_entries + p.chunk - 1) / p.chunk : 1;
@@ -872,8 +1025,10 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
         e = p.d_I == 64 ? launch_kernel(index_scan_kernel<2, false>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p)
                         : launch_kernel(index_scan_kernel<1, false>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p);
     if (e != cudaSuccess) return e;
-    if (mid) return cudaEventRecordWithFlags(mid, stream, cudaEventRecordExternal);
-    return cudaSuccess;
+    if (mid && (e = cudaEventRecordWithFlags(mid, stream, cudaEventRecordExternal)) != cudaSuccess) return e;
+    // the exact selection: one cluster of kFinalF CTAs per query
+    return launch_kernel_cluster(index_final_kernel, dim3(kFinalF, (unsigned)p.Q), dim3(kFinalThreads), kFinalDynSmem,
+                                 stream, pdl, dim3(kFinalF, 1, 1), p);
 }
 
 cudaError_t launch_quantize_keys(const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries, int m,

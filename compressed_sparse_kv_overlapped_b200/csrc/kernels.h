@@ -82,10 +82,9 @@ struct IndexParams {
     // workspace
     float* scores;            // [Q, e_stride]
     uint32_t* hist;           // [Q, kHistBins]; zero before the scan
-    uint32_t* ticket;         // [Q] finished scan chunks; zero before the scan
     uint64_t* seg;            // [Q, e_seg] kept entries (64-bit keys) when they exceed shared memory
     uint32_t* meta;           // [Q, max_chunks] per scan chunk: (threshold bin << 16) | candidate count
-    uint32_t* coff;           // [Q, max_chunks] per scan chunk: member count, then list offset
+    uint32_t* coff;           // [Q, max_chunks + 8] the final select's per-CTA prefixes over chunks (many chunks)
     uint64_t* cand;           // [Q, max_chunks, cand_cap] candidate keys of each chunk, in index order
     // optional: rows of this cache (row stride prefetch_row_bytes, a multiple of 16) at the selected
     // entries are prefetched into L2 as soon as the selection is known (the attention's gather)

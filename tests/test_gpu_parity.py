@@ -783,6 +783,22 @@ def test_decode_appended_rows_from_new_rows(wl, steps):
     _decode_e2e(wl, steps, via_new_rows=True)
 
 
+@pytest.mark.parametrize("cluster", [4, 8])
+def test_decode_cluster_merge(cluster):
+    """The optional merge of decode partials across a thread-block cluster (CSA_DECODE_CLUSTER, read
+    once per process, so the decode end-to-end cases rerun in a child process with it set)."""
+    import os
+    import pathlib
+    import subprocess
+    import sys
+    here = pathlib.Path(__file__).resolve()
+    env = dict(os.environ, CSA_DECODE_CLUSTER=str(cluster))
+    cases = [f"{here}::test_decode_end_to_end", f"{here}::test_decode_with_norms_and_sinks"]
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider", *cases],
+                       cwd=here.parents[1], env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+
+
 @pytest.mark.parametrize("N,rows,dims", [
     (1024, list(range(0, 1024, 7)) + [1023], workloads.TINY_DIMS),
     (3000, [0, 1, 2, 3, 4, 5, 127, 128, 129, 1023, 1024, 2047, 2048, 2999], SMALL_PROD)],
