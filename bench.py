@@ -31,7 +31,7 @@ METRIC = "CSA+HCA decode queries/s at 1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel source it
 # was taken on: the key is the SHA-256 prefix of csrc/index_topk.cu at that capture.  Any other
 # source reports null traffic until it is captured again.
-SCAN_TRAFFIC = {"source_sha256": None, "bytes": None}
+SCAN_TRAFFIC = {"source_sha256": "141fca9a179e755c", "bytes": 134262272 + 5982464}
 
 
 def _source_sha(name):
@@ -93,8 +93,11 @@ def parse():
                     help="indexer keys of the decode workloads: bf16 (the workload as stated) or 8-bit block-scaled")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--stage", default=None, choices=["index", "attn"],
-                    help="time one stage alone on a compact case of the workload's geometry (profiling aid)")
+    ap.add_argument("--stage", default=None, choices=["index", "attn", "compress"],
+                    help="time one stage alone on a compact case of the workload's geometry (profiling aid); "
+                         "compress: the full compressor pass at the prefill geometry")
+    ap.add_argument("--prefill-n", type=int, default=None,
+                    help="sequence length of the prefill workload (default 131,072; a smaller one for profiling)")
     return ap.parse_args()
 
 
@@ -634,6 +637,53 @@ def prefill_flops(wd, N):
     return index, attn
 
 
+def prefill_workload(args):
+    import dataclasses
+
+    from synth import workloads
+    wl = workloads.prefill()
+    if args.prefill_n:
+        wl = dataclasses.replace(wl, name=f"prefill_N{args.prefill_n}", n0=(int(args.prefill_n),))
+    return wl
+
+
+def compress_bytes(wd, N):
+    """Algorithmic bytes of the full compressor pass over N tokens: the token rows (x, both logit
+    arrays, raw indexer keys) read once; CSA entries with their indexer keys and HCA entries written."""
+    return N * (3 * wd.d + wd.d_I) * 2 + (N // wd.m) * (wd.d + wd.d_I) * 2 + (N // wd.m_hca) * wd.d * 2
+
+
+def run_stage_compress(args):
+    """csa_compress_all alone (one pass for the CSA entries, their indexer keys and the HCA entries)
+    at the prefill geometry; K calls timed with CUDA events."""
+    import torch
+
+    import compressed_sparse_kv_overlapped_b200 as csa
+    from synth import device as sdev
+    wl = prefill_workload(args)
+    wd = wl.dims
+    N = wl.n0[0]
+    layer = csa.HybridLayer(dims_of(wd), [N])
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths([N])
+    for _ in range(args.warmup):
+        layer.compress()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        layer.compress()
+    e1.record()
+    torch.cuda.synchronize()
+    assert csa.csa_sync_status() == csa.CSA_OK
+    ms = e0.elapsed_time(e1) / args.steps
+    nb = compress_bytes(wd, N)
+    hbm, _, src = peaks()
+    return {"stage": "compress (csa_compress_all, CSA + keys + HCA in one pass)", "workload": wl.name,
+            "us_per_call": ms * 1e3, "bytes": nb, "achieved_gbs": nb / (ms * 1e-3) / 1e9, "peak_gbs": hbm,
+            "frac": nb / (ms * 1e-3) / 1e9 / hbm, "peak_source": src}
+
+
 def run_prefill(args, rank, world):
     """Causal prefill of one sequence (hybrid_attn_prefill over all N queries; the compressor pass
     is timed on its own, then each step runs the indexer, top-k and attention for every query).
@@ -643,7 +693,7 @@ def run_prefill(args, rank, world):
     import compressed_sparse_kv_overlapped_b200 as csa
     from synth import device as sdev
     from synth import workloads
-    wl = workloads.prefill()
+    wl = prefill_workload(args)
     wd = wl.dims
     N = wl.n0[0]
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -692,7 +742,7 @@ def run_prefill(args, rank, world):
     f_index, f_attn = prefill_flops(wd, N)
     hbm, tf_peak, src = peaks(sustained=True)
     tflops = (f_index + f_attn) / (ms * 1e-3) / 1e12
-    comp_bytes = N * (3 * wd.d + wd.d_I) * 2 + (N // wd.m) * (wd.d + wd.d_I) * 2 + (N // wd.m_hca) * wd.d * 2
+    comp_bytes = compress_bytes(wd, N)
     res = {
         "metric": "causal prefill queries/s (indexer + top-k + sparse/HCA attention); tensor TFLOP/s",
         "value": N * world / (ms * 1e-3), "unit": "queries/s", "n_gpus": world, "steps": K, "warmup": W,
@@ -950,6 +1000,9 @@ def main():
         return
     if args.stage == "index":
         print(json.dumps(run_stage_index(args)), flush=True)
+        return
+    if args.stage == "compress":
+        print(json.dumps(run_stage_compress(args)), flush=True)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
