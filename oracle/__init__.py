@@ -12,6 +12,10 @@ Every stage cites its source passage in ``oracle.c``.  Parity status of each rou
   locality, identity at m=1, each indexer-key channel weighted by its own channel's softmax,
   brute-force selection, dense attention against a library softmax, partition invariance of the
   merge).
+* e2m1_code, quantize_entries_mx4, dequantize_entries_mx4 (FP4 entries, R15): pinned by the E2M1
+  grid (every value maps to itself, every midpoint to its even neighbour, saturation), the block
+  scale's definition at its boundary, exact round trips of on-grid rows, and a brute-force nearest
+  search on random rows.
 * hybrid_query (the composition): pinned at q = 0, q^I = 0, where the merged softmax is uniform
   over exactly the keys the method attends (lse = log of their count, O = their mean), at lengths
   below and above the window and the HCA ratio.  Beyond that the pages print no worked numeric
@@ -60,6 +64,10 @@ def lib() -> ctypes.CDLL:
         L.oracle_quantize_keys_mx8.argtypes = [vp, i64, ci, vp, vp]
         L.oracle_quantize_keys_mx8.restype = ci
         L.oracle_index_scores_mx8.argtypes = [vp, vp, ci, ci, vp, vp, i64, vp]
+        L.oracle_e2m1_round.argtypes = [vp, i64, vp]
+        L.oracle_quantize_entries_mx4.argtypes = [vp, i64, ci, vp, vp]
+        L.oracle_quantize_entries_mx4.restype = ci
+        L.oracle_dequantize_entries_mx4.argtypes = [vp, vp, i64, ci, vp]
         _lib = L
     return _lib
 
@@ -174,6 +182,46 @@ def quantize_keys_mx8(KI):
     return Kq, sc
 
 
+def e2m1_code(v) -> np.ndarray:
+    """fp64 values -> the 4-bit E2M1 code of the nearest value (ties to the even code, |v| > 6 -> 6)."""
+    v = np.ascontiguousarray(v, dtype=np.float64).ravel()
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e2m1_round(_p(v), v.size, _p(out))
+    return out
+
+
+def quantize_entries_mx4(E):
+    """bf16 entry rows [n, d] -> (packed E2M1 codes [n, d / 2], biased power-of-two scales [n, d / 32])."""
+    E = _u16(E)
+    n, d = E.shape
+    Eq = np.empty((n, d // 2), dtype=np.uint8)
+    sc = np.empty((n, d // 32), dtype=np.uint8)
+    if lib().oracle_quantize_entries_mx4(_p(E), n, d, _p(Eq), _p(sc)) != 0:
+        raise ValueError("d must be a multiple of 32")
+    return Eq, sc
+
+
+def dequantize_entries_mx4(Eq, scales) -> np.ndarray:
+    """packed E2M1 codes [n, d / 2] + scales [n, d / 32] -> dequantized values [n, d] (fp64)."""
+    Eq = np.ascontiguousarray(Eq, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    n, d = Eq.shape[0], Eq.shape[1] * 2
+    out = np.empty((n, d), dtype=np.float64)
+    lib().oracle_dequantize_entries_mx4(_p(Eq), _p(scales), n, d, _p(out))
+    return out
+
+
+def mx4_entries_as_bf16(E) -> np.ndarray:
+    """The entry rows the attention sees when the cache holds them in FP4 (R15): quantized, then
+    dequantized.  Every dequantized value (at most two significant bits times a power of two) is a
+    bf16 value, so it is returned as bf16 bit patterns for the bf16 attention routines."""
+    Eq, sc = quantize_entries_mx4(E)
+    v = dequantize_entries_mx4(Eq, sc)
+    b = round_bf16(v)
+    assert np.array_equal(bf16_to_f64(b), v), "a dequantized FP4 value is not a bf16 value"
+    return b
+
+
 def index_scores_mx8(qI, w, Kq, scales) -> np.ndarray:
     """Indexer scores of the dequantized 8-bit keys (fp64)."""
     qI = _u16(qI)
@@ -263,16 +311,20 @@ class Shape:
 
 
 def hybrid_query(shape: Shape, L: int, q, qI, w, raw, entries, KI, hca, sink=None, q_gain=None, eps=1e-6,
-                 keys_mx8=None):
+                 keys_mx8=None, entries_mx4=False):
     """One query of the hybrid layer at visible length L, composed from the stages above.
 
     raw: uint16 [>=L, d] raw latents of the sequence; entries: uint16 [>=L//m, d] CSA cache;
     KI: uint16 [>=L//m, d_I] indexer-key cache; hca: uint16 [>=L//m', d] HCA cache.
     Optional: sink [H] attention-sink logits; q_gain [d]: the query heads are RMS-normalized with
     this gain (and rounded to bf16, the attention's operand type) before attending; keys_mx8 =
-    (Kq, scales): the indexer scores these 8-bit keys instead of KI.
+    (Kq, scales): the indexer scores these 8-bit keys instead of KI; entries_mx4: the CSA and HCA
+    caches hold FP4 entries with block scales (R15), so the attention sees their dequantized values.
     Returns a dict with the selected indices, the two partials and the merged output.
     """
+    if entries_mx4:
+        entries = mx4_entries_as_bf16(entries[:L // shape.m]) if L // shape.m > 0 else entries
+        hca = mx4_entries_as_bf16(hca[:L // shape.m_hca]) if L // shape.m_hca > 0 else hca
     n_c = L // shape.m
     if keys_mx8 is not None:
         s = index_scores_mx8(qI, w, keys_mx8[0][:n_c], keys_mx8[1][:n_c])

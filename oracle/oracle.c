@@ -449,3 +449,83 @@ void oracle_rms_norm(const double* x, int64_t rows, int d, const float* gain, do
         for (int c = 0; c < d; ++c) out[r * d + c] = x[r * d + c] * inv * (double)gain[c];
     }
 }
+
+/* ---- f4: FP4 compressed entries with block scales --------------------------- */
+/*
+ * "Compressed attention · CSA / HCA va hai truc nen", section 3 (Giai phap): the V4.1 FP4 KV cache
+ * carries block scales and a packing overhead.  Reading R15 (the page gives no format): the same
+ * block-scaled family as the 8-bit indexer keys (R11), with 4-bit elements: every stored entry row
+ * (CSA and HCA; the raw window tokens stay bf16) is cut into blocks of 32 channels; block scale 2^e
+ * with e the smallest integer such that amax <= 6 * 2^e (e >= -127; a zero block takes e = -127),
+ * stored as the byte e + 127; elements E2M1 (sign, two exponent bits with bias 1, one mantissa
+ * bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), x / 2^e rounded to the nearest magnitude, a tie to
+ * the one whose mantissa bit is 0; two elements per byte, the even channel in the low nibble.  The
+ * attention uses the dequantized entries (code value * 2^e) as keys and values.
+ */
+static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* The 4-bit code of the E2M1 value nearest to v (ties to the even code), magnitudes above 6 to 6;
+   bit 3 is the sign (kept for negative values that round to zero). */
+static uint8_t e2m1_code(double v) {
+    double a = fabs(v);
+    int m = 7;
+    if (a < 6.0) {
+        int i = 0;
+        while (!(a < kE2M1[i + 1])) ++i;             /* kE2M1[i] <= a < kE2M1[i + 1] */
+        double dl = a - kE2M1[i], dh = kE2M1[i + 1] - a;
+        m = dl < dh ? i : dh < dl ? i + 1 : ((i & 1) == 0 ? i : i + 1);
+    }
+    return (uint8_t)(((v < 0.0 || (v == 0.0 && signbit(v))) ? 8 : 0) | m);
+}
+
+static double e2m1_value(uint8_t code) {
+    double a = kE2M1[code & 7];
+    return (code & 8) ? -a : a;
+}
+
+void oracle_e2m1_round(const double* in, int64_t n, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e2m1_code(in[i]);
+}
+
+/* bf16 entry rows [n, d] -> packed codes [n, d / 2] and scale bytes [n, d / 32].  Returns -2 if d is
+   not a multiple of 32. */
+int oracle_quantize_entries_mx4(const uint16_t* E, int64_t n, int d, uint8_t* Eq, uint8_t* scales) {
+    if (d % 32) return -2;
+    int nb = d / 32;
+    for (int64_t j = 0; j < n; ++j) {
+        for (int b = 0; b < nb; ++b) {
+            const uint16_t* x = E + j * d + 32 * b;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs(bf16_to_double(x[i]));
+                if (a > amax) amax = a;
+            }
+            int e = -127;
+            if (amax > 0.0) {
+                int y;
+                frexp(amax, &y);
+                e = y - 3;                                     /* a start near the answer */
+                while (amax > ldexp(6.0, e)) ++e;              /* smallest e with amax <= 6 * 2^e */
+                while (e > -127 && amax <= ldexp(6.0, e - 1)) --e;
+            }
+            scales[j * nb + b] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; i += 2) {
+                uint8_t lo = e2m1_code(ldexp(bf16_to_double(x[i]), -e));
+                uint8_t hi = e2m1_code(ldexp(bf16_to_double(x[i + 1]), -e));
+                Eq[j * (d / 2) + 16 * b + i / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* packed codes + scale bytes -> the dequantized values [n, d] (fp64). */
+void oracle_dequantize_entries_mx4(const uint8_t* Eq, const uint8_t* scales, int64_t n, int d, double* out) {
+    int nb = d / 32;
+    for (int64_t j = 0; j < n; ++j)
+        for (int c = 0; c < d; ++c) {
+            uint8_t byte = Eq[j * (d / 2) + c / 2];
+            uint8_t code = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+            out[j * d + c] = ldexp(e2m1_value(code), (int)scales[j * nb + c / 32] - 127);
+        }
+}

@@ -520,6 +520,76 @@ def test_mx8_scores_are_the_plain_scores_of_the_dequantized_keys():
     np.testing.assert_array_equal(oracle.index_scores_mx8(qI, w, Kq, sc), oracle.index_scores(qI, w, Kd))
 
 
+# ---------------------------------------------------------------- FP4 entries (R15)
+
+E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]  # the magnitudes of codes 0..7 (sign bit 3)
+
+
+def test_e2m1_grid_midpoints_and_saturation():
+    """Every E2M1 value maps to its own code, a midpoint to the neighbour whose mantissa bit (code
+    bit 0) is 0, anything just past a midpoint to the upper neighbour, magnitudes above 6 to 6, and
+    a negative value keeps its sign bit even when it rounds to zero."""
+    vals, want = [], []
+    for c, g in enumerate(E2M1):
+        vals += [g, -g]
+        want += [c, (8 | c) if g > 0 else 8]
+    for i in range(7):
+        lo, hi = E2M1[i], E2M1[i + 1]
+        mid = (lo + hi) / 2
+        vals += [mid, np.nextafter(mid, np.inf), np.nextafter(mid, -np.inf)]
+        want += [i if i % 2 == 0 else i + 1, i + 1, i]
+    vals += [6.5, 7.0, 1e30, -100.0, -0.1, -0.25]
+    want += [7, 7, 7, 15, 8, 8]
+    np.testing.assert_array_equal(oracle.e2m1_code(np.array(vals)), np.array(want, dtype=np.uint8))
+
+
+@pytest.mark.parametrize("scale", [1.0, 2.0 ** -30, 5.0e3])
+def test_mx4_block_scale_and_nearest_value(scale):
+    """Each 32-channel block's scale 2^e is the smallest power of two with amax <= 6 * 2^e (so
+    3 < amax / 2^e <= 6), and every element dequantizes to a nearest point of the grid scaled by
+    2^e (brute force over the 8 magnitudes and both signs)."""
+    n, d = 60, 128
+    E = oracle.round_bf16(synth.bf16_to_f64(bf(SEED, synth.X, 31, n, d)) * scale)
+    E[7] = 0  # an all-zero entry: scale byte 0, zero codes
+    Eq, sc = oracle.quantize_entries_mx4(E)
+    deq = oracle.dequantize_entries_mx4(Eq, sc)
+    Ef = synth.bf16_to_f64(E)
+    grid = np.array(E2M1 + [-g for g in E2M1])
+    for j in range(n):
+        for b in range(d // 32):
+            x = Ef[j, 32 * b:32 * b + 32]
+            e = int(sc[j, b]) - 127
+            amax = np.abs(x).max()
+            if amax == 0:
+                assert e == -127 and not deq[j, 32 * b:32 * b + 32].any()
+                continue
+            assert 3 < amax / 2.0 ** e <= 6
+            dist = np.abs(grid[None, :] * 2.0 ** e - x[:, None]).min(axis=1)
+            np.testing.assert_array_equal(np.abs(deq[j, 32 * b:32 * b + 32] - x), dist)
+
+
+def test_mx4_round_trip_and_nibble_order():
+    """Rows whose blocks hold only grid values times 2^e, with 6 * 2^e present, come back exactly;
+    the even channel sits in the low nibble of each byte."""
+    rng = np.random.default_rng(5)
+    n, d = 8, 64
+    rows = np.empty((n, d))
+    for j in range(n):
+        for b in range(d // 32):
+            e = int(rng.integers(-20, 20))
+            blk = rng.choice(E2M1, size=32) * rng.choice([-1.0, 1.0], size=32)
+            blk[int(rng.integers(0, 32))] = 6.0
+            rows[j, 32 * b:32 * b + 32] = blk * 2.0 ** e
+    E = oracle.round_bf16(rows)
+    assert np.array_equal(synth.bf16_to_f64(E), rows)
+    Eq, sc = oracle.quantize_entries_mx4(E)
+    np.testing.assert_array_equal(oracle.dequantize_entries_mx4(Eq, sc), rows)
+    row = np.zeros((1, 32))
+    row[0, 0], row[0, 1], row[0, 2], row[0, 3] = 0.5, 6.0, -1.5, 0.0
+    Eq, sc = oracle.quantize_entries_mx4(oracle.round_bf16(row))
+    assert sc[0, 0] == 127 and Eq[0, 0] == (1 | (7 << 4)) and Eq[0, 1] == (8 | 3)
+
+
 # ---------------------------------------------------------------- sinks and normalization
 
 def test_rms_norm_matches_library_and_closed_forms():
