@@ -91,6 +91,9 @@ def parse():
                          "131,072 queries, reported as tensor-pipe throughput")
     ap.add_argument("--keys", default="bf16", choices=["bf16", "mx8"],
                     help="indexer keys of the decode workloads: bf16 (the workload as stated) or 8-bit block-scaled")
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp4"],
+                    help="compressed entries the decode attention reads: bf16 (the workload as stated) or FP4 "
+                         "with 32-channel block scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--stage", default=None, choices=["index", "attn", "compress"],
@@ -186,17 +189,20 @@ def dims_of(wd):
     return csa.make_dims(d=wd.d, H=wd.H, d_I=wd.d_I, H_I=wd.H_I, m=wd.m, m_hca=wd.m_hca, k=wd.k, W=wd.W)
 
 
-def step_bytes(wd, lens, keys="bf16"):
+def step_bytes(wd, lens, keys="bf16", kv="bf16"):
     """Algorithmic HBM bytes of one decode step: indexer-key scan, gathered top-k entries, raw window,
-    HCA entries (queries and outputs not counted), and the block-scale bytes of 8-bit keys (one per
-    32 key channels; 0 for bf16 keys)."""
+    HCA entries (queries and outputs not counted), the block-scale bytes of 8-bit keys (one per 32 key
+    channels; 0 for bf16 keys) and of FP4 entries (one per 32 channels of every gathered or HCA entry;
+    0 for bf16 entries, whose rows are then 2 bytes per channel instead of half a byte)."""
     kb = wd.d_I if keys == "mx8" else wd.d_I * 2
+    eb = wd.d // 2 if kv == "fp4" else wd.d * 2
     idx = sum((L // wd.m) * kb for L in lens)
     scales = sum((L // wd.m) * (wd.d_I // 32) for L in lens) if keys == "mx8" else 0
-    gather = sum(min(wd.k, L // wd.m) * wd.d * 2 for L in lens)
+    gather = sum(min(wd.k, L // wd.m) * eb for L in lens)
     window = sum(min(wd.W, L) * wd.d * 2 for L in lens)
-    hca = sum((L // wd.m_hca) * wd.d * 2 for L in lens)
-    return idx, gather, window, hca, scales
+    hca = sum((L // wd.m_hca) * eb for L in lens)
+    escales = sum((min(wd.k, L // wd.m) + L // wd.m_hca) * (wd.d // 32) for L in lens) if kv == "fp4" else 0
+    return idx, gather, window, hca, scales, escales
 
 
 # ------------------------------------------------------------------------------------ our arm
@@ -214,7 +220,8 @@ def run_ours(args, rank, world):
     B = wl.B
     K, W = args.steps, args.warmup
     extra = W + K + (0 if args.no_e2e else K) + 1
-    layer = csa.HybridLayer(dims_of(wd), [n + extra for n in wl.n0], device=dev, key_format=args.keys)
+    layer = csa.HybridLayer(dims_of(wd), [n + extra for n in wl.n0], device=dev, key_format=args.keys,
+                            kv_format=args.kv)
     sdev.fill_layer_inputs(layer, wl)
     layer.set_lengths(list(wl.n0))
     layer.compress()
@@ -328,10 +335,10 @@ def run_ours(args, rank, world):
         return steps_sorted[min(K - 1, int(round(q * (K - 1))))]
 
     # algorithmic bytes per step (lengths after each step's append)
-    tot = [0, 0, 0, 0, 0]
+    tot = [0, 0, 0, 0, 0, 0]
     for s in range(K):
         lens = [n + s + 1 for n in lens_before]
-        for i, v in enumerate(step_bytes(wd, lens, args.keys)):
+        for i, v in enumerate(step_bytes(wd, lens, args.keys, args.kv)):
             tot[i] += v
     per_step = [v / K for v in tot]
     bytes_step = sum(per_step)
@@ -345,15 +352,16 @@ def run_ours(args, rank, world):
         "metric": METRIC, "value": B * world * K / (ms * 1e-3), "unit": "queries/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
-        "config": {"workload": wl.name + ("_mx8keys" if args.keys == "mx8" else ""), "B": B,
-                   "N": wl.n0[0] if len(set(wl.n0)) == 1 else "ragged", "indexer_keys": args.keys,
+        "config": {"workload": wl.name + ("_mx8keys" if args.keys == "mx8" else "") + ("_fp4kv" if args.kv == "fp4" else ""),
+                   "B": B, "N": wl.n0[0] if len(set(wl.n0)) == 1 else "ragged", "indexer_keys": args.keys,
+                   "entries": args.kv,
                    "d": wd.d, "heads": wd.H, "d_I": wd.d_I, "H_I": wd.H_I, "k": wd.k, "W": wd.W, "m": wd.m,
                    "m_hca": wd.m_hca, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "per-step working set larger than L2 (no flush)"},
         "hbm": {"algorithmic_bytes_per_step": int(bytes_step),
                 "breakdown_bytes": {"index_keys": int(per_step[0]), "scale_bytes": int(per_step[4]),
                                     "gathered_entries": int(per_step[1]), "window": int(per_step[2]),
-                                    "hca_entries": int(per_step[3])},
+                                    "hca_entries": int(per_step[3]), "entry_scale_bytes": int(per_step[5])},
                 "achieved_gbs": achieved_step_gbs, "peak_gbs": hbm_peak, "frac": achieved_step_gbs / hbm_peak,
                 "peak_source": peak_src},
         "stages_ms": stage,
@@ -375,7 +383,7 @@ def run_ours(args, rank, world):
     if not args.no_e2e:
         result["e2e"] = run_e2e(layer, wl, K, W, max_len, ws, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(wl, keys=args.keys)
+        result["cpu_baseline"] = cpu_baseline(wl, keys=args.keys, kv=args.kv)
     return result
 
 
@@ -483,7 +491,7 @@ class OracleDecode:
     query selects (also untimed).  A timed query runs the oracle's indexer scores, top-k, sparse
     attention with the window, HCA attention and LSE merge."""
 
-    def __init__(self, wl, b=0, rows=(0,), keys="bf16"):
+    def __init__(self, wl, b=0, rows=(0,), keys="bf16", kv="bf16"):
         import numpy as np
 
         import oracle
@@ -507,6 +515,8 @@ class OracleDecode:
         bl = workloads.raw_tokens(wl, b, 0, L, "b")
         H, _ = oracle.compress_parallel(x, bl, workloads.bias_h(wl), None, L, wd.m_hca, wd.m_hca, np.arange(n_h))
         self.H = oracle.round_bf16(H)
+        if kv == "fp4" and n_h:
+            self.H = oracle.mx4_entries_as_bf16(self.H)
         del bl
         self.x = x
         self.E = np.zeros((n_c, wd.d), np.uint16)
@@ -522,7 +532,7 @@ class OracleDecode:
         need = np.unique(np.concatenate([i[i >= 0] for i in sel])).astype(np.int64)
         a = workloads.raw_tokens(wl, b, 0, L, "a")
         E, _ = oracle.compress_parallel(x, a, bias_c, None, L, wd.m, 2 * wd.m, need)
-        self.E[need] = oracle.round_bf16(E)
+        self.E[need] = oracle.mx4_entries_as_bf16(oracle.round_bf16(E)) if kv == "fp4" else oracle.round_bf16(E)
 
     def run(self, i):
         import oracle
@@ -531,21 +541,22 @@ class OracleDecode:
                                    keys_mx8=self.keys_mx8)
 
 
-def cpu_baseline(wl, samples=None, keys="bf16"):
+def cpu_baseline(wl, samples=None, keys="bf16", kv="bf16"):
     """The oracle on a bounded sample of the workload: one decode query per host core (at least 4) on
     one prepared sequence, in parallel threads (the oracle's C code releases the GIL)."""
     from concurrent.futures import ThreadPoolExecutor
     host = os.cpu_count() or 1
     samples = samples or max(4, host)
     threads = min(samples, host)
-    od = OracleDecode(wl, 0, rows=tuple(range(samples)), keys=keys)
+    od = OracleDecode(wl, 0, rows=tuple(range(samples)), keys=keys, kv=kv)
     t0 = time.perf_counter()
     with ThreadPoolExecutor(threads) as ex:
         list(ex.map(od.run, range(samples)))
     dt = time.perf_counter() - t0
     return {"value": samples / dt, "unit": "queries/s", "cores": threads, "host_cores": host, "kind": "oracle",
             "sample": f"{samples} decode queries of one sequence at L={od.L} (the workload's geometry, {keys} "
-                      f"indexer keys), caches prepared untimed, one query per thread"}
+                      f"indexer keys, {kv} entries), caches prepared untimed (FP4 entries dequantized), one query "
+                      f"per thread"}
 
 
 def run_reference(args, rank, world):
@@ -557,7 +568,7 @@ def run_reference(args, rank, world):
     wl = workload(args.config)
     B = wl.B
     K, W = args.steps, args.warmup
-    od = OracleDecode(wl, 0, rows=tuple(range(B)))
+    od = OracleDecode(wl, 0, rows=tuple(range(B)), keys=args.keys, kv=args.kv)
     threads = min(B, os.cpu_count() or 1)
     with ThreadPoolExecutor(threads) as ex:
         for _ in range(W):
@@ -570,7 +581,8 @@ def run_reference(args, rank, world):
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "queries/s", "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": dt * 1e3 / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded counter-based generator)",
-            "config": {"workload": wl.name, "B": B},
+            "config": {"workload": wl.name + ("_mx8keys" if args.keys == "mx8" else "") +
+                                   ("_fp4kv" if args.kv == "fp4" else ""), "B": B},
             "cpu_baseline": {"value": v, "unit": "queries/s", "cores": threads, "kind": "oracle",
                              "sample": f"each step: {B} decode queries at L={od.L} on one prepared sequence"},
             "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

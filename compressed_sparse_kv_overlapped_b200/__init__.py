@@ -31,7 +31,7 @@ CSA_OP_PREFILL = 5
 EXPORTS = ("csa_compress", "csa_compress_all", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
            "hybrid_attn_prefill", "csa_workspace_size", "csa_last_error", "csa_sync_status", "csa_version",
            "csa_set_stage_events", "csa_index_topk_noalloc", "csa_debug_inject", "csa_quantize_keys",
-           "csa_index_topk_mx8")
+           "csa_index_topk_mx8", "csa_quantize_entries", "csa_sparse_attn_fp4", "hca_dense_attn_fp4")
 CSA_DECODE_MARKS = 5
 
 _i32, _i64, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
@@ -57,7 +57,8 @@ class csa_decode_args(ctypes.Structure):
                 ("bias_c", _vp), ("bias_h", _vp), ("entries", _vp), ("entry_keys", _vp), ("hca_entries", _vp),
                 ("q", _vp), ("q_idx", _vp), ("w", _vp), ("out", _vp), ("lse", _vp), ("idx_out", _vp),
                 ("new_rows", _vp), ("keys_q", _vp), ("key_scales", _vp), ("idx_in", _vp),
-                ("norms", ctypes.POINTER(csa_norms))]
+                ("norms", ctypes.POINTER(csa_norms)), ("entries_q", _vp), ("entry_scales", _vp), ("hca_q", _vp),
+                ("hca_scales", _vp)]
 
 
 class csa_prefill_args(ctypes.Structure):
@@ -101,9 +102,16 @@ def lib() -> ctypes.CDLL:
         L.csa_index_topk_mx8.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                                          _vp, _sz, _vp]
         L.csa_index_topk_noalloc.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.csa_quantize_entries.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, ctypes.c_int, _vp, _vp, _vp,
+                                           _vp]
+        L.csa_sparse_attn_fp4.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _f32, _vp,
+                                          _vp, _vp, _sz, _vp]
+        L.hca_dense_attn_fp4.argtypes = [P(csa_dims), _vp, _vp, ctypes.c_int, _i64, _vp, _vp, _vp, _vp, ctypes.c_int,
+                                         _f32, _vp, _vp, _vp, _sz, _vp]
         for n in ("csa_compress", "csa_compress_all", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn", "hybrid_attn_decode",
                   "hybrid_attn_prefill", "csa_sync_status", "csa_version", "csa_set_stage_events",
-                  "csa_index_topk_noalloc", "csa_debug_inject", "csa_quantize_keys", "csa_index_topk_mx8"):
+                  "csa_index_topk_noalloc", "csa_debug_inject", "csa_quantize_keys", "csa_index_topk_mx8",
+                  "csa_quantize_entries", "csa_sparse_attn_fp4", "hca_dense_attn_fp4"):
             getattr(L, n).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -241,6 +249,29 @@ def hca_dense_attn(dims, seqs, queries, Q, max_len, q, hca_entries, x, W, scale,
                               _ptr(hca_entries), _ptr(x), W, scale, _ptr(out), _ptr(lse), _ptr(ws),
                               0 if ws is None else ws.numel() * ws.element_size(), _vp(_stream(stream)))
     _check(rc, "hca_dense_attn")
+
+
+def csa_quantize_entries(dims, seqs, ranges, B, max_entries, which, entries, entries_q, entry_scales,
+                         stream=None) -> None:
+    """FP4 copies of the stored bf16 entries of the CSA cache (which = 0) or the HCA cache (which = 1)."""
+    rc = lib().csa_quantize_entries(ctypes.byref(dims), _ptr(seqs), _ptr(ranges), B, max_entries, which,
+                                    _ptr(entries), _ptr(entries_q), _ptr(entry_scales), _vp(_stream(stream)))
+    _check(rc, "csa_quantize_entries")
+
+
+def csa_sparse_attn_fp4(dims, seqs, queries, Q, q, entries_q, entry_scales, idx, x, scale, out, lse, ws, stream=None):
+    rc = lib().csa_sparse_attn_fp4(ctypes.byref(dims), _ptr(seqs), _ptr(queries), Q, _ptr(q), _ptr(entries_q),
+                                   _ptr(entry_scales), _ptr(idx), _ptr(x), scale, _ptr(out), _ptr(lse), _ptr(ws),
+                                   0 if ws is None else ws.numel() * ws.element_size(), _vp(_stream(stream)))
+    _check(rc, "csa_sparse_attn_fp4")
+
+
+def hca_dense_attn_fp4(dims, seqs, queries, Q, max_len, q, hca_q, hca_scales, x, W, scale, out, lse, ws,
+                       stream=None):
+    rc = lib().hca_dense_attn_fp4(ctypes.byref(dims), _ptr(seqs), _ptr(queries), Q, max_len, _ptr(q), _ptr(hca_q),
+                                  _ptr(hca_scales), _ptr(x), W, scale, _ptr(out), _ptr(lse), _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(), _vp(_stream(stream)))
+    _check(rc, "hca_dense_attn_fp4")
 
 
 def hybrid_attn_decode(args: csa_decode_args, ws, stream=None) -> None:

@@ -62,7 +62,8 @@ struct Smem {
     static constexpr int kBar = kP1 + kBlock;          // mbarriers
     static constexpr int kMisc = kBar + 32 * 8;        // tmem base, abort flag, masks
     static constexpr int kRowPtr = kMisc + 64;         // per loader warp: 16 row pointers
-    static constexpr int kTotal = kRowPtr + 4 * 16 * 8;
+    static constexpr int kRowScl = kRowPtr + 4 * 16 * 8;  // and their FP4 scale rows (null: a bf16 row)
+    static constexpr int kTotal = kRowScl + 4 * 16 * 8;
     static constexpr int kAlloc = kTotal + 1024;       // slack for 1024-byte alignment
     // cluster merge: the CTA's [64 x D] fp32 result in the freed key stages, rows padded by 16 bytes
     // so that the eight rows a warp's quads store hit different banks
@@ -99,7 +100,11 @@ struct KeyList {
 };
 
 // Row pointer of slot `s` (nullptr = masked slot).
-__device__ __forceinline__ const uint16_t* key_row(const AttnParams& p, int D, const KeyList& kl, int64_t s) {
+// The source of key s: a bf16 row (returned, *scl = nullptr) or, for an entry of a cache held in FP4,
+// its code row (returned) with its scale row in *scl; nullptr for an empty or invalid slot.
+__device__ __forceinline__ const void* key_src(const AttnParams& p, int D, const KeyList& kl, int64_t s,
+                                               const uint8_t** scl) {
+    *scl = nullptr;
     if (s < p.k_slots) {
         const int32_t j = kl.idx[s];
         if (j < 0) return nullptr;
@@ -107,12 +112,23 @@ __device__ __forceinline__ const uint16_t* key_row(const AttnParams& p, int D, c
             report(p.status, CSA_ERR_INDEX);
             return nullptr;
         }
-        return p.entries + (kl.csa_row0 + j) * D;
+        const int64_t r = kl.csa_row0 + j;
+        if (p.entries_q) {
+            *scl = p.entries_s + r * (D / 32);
+            return p.entries_q + r * (D / 2);
+        }
+        return p.entries + r * D;
     }
     s -= p.k_slots;
     if (s < p.W) return s < kl.nw ? p.raw + (kl.win_row0 + s) * D : nullptr;
     s -= p.W;
-    return s < kl.n_hca ? p.hca + (kl.hca_row0 + s) * D : nullptr;
+    if (s >= kl.n_hca) return nullptr;
+    const int64_t r = kl.hca_row0 + s;
+    if (p.hca_q) {
+        *scl = p.hca_s + r * (D / 32);
+        return p.hca_q + r * (D / 2);
+    }
+    return p.hca + r * D;
 }
 
 template <int D>
@@ -212,6 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const int lw = warp - 4;
         const uint64_t* rowptr = reinterpret_cast<const uint64_t*>(sm + L::kRowPtr) + lw * 16;
         uint64_t* rowptr_w = reinterpret_cast<uint64_t*>(sm + L::kRowPtr) + lw * 16;
+        const uint64_t* rowscl = reinterpret_cast<const uint64_t*>(sm + L::kRowScl) + lw * 16;
+        uint64_t* rowscl_w = reinterpret_cast<uint64_t*>(sm + L::kRowScl) + lw * 16;
         constexpr int CPR = D / 8;  // 16-byte chunks per row
         // Lane l copies 16-byte chunks l, l+32, ... of each 64-chunk (1 KiB) row: chunk c lands in
         // block c/8 at swizzled position (c%8) ^ (row%8), and c%8 = l%8 for every chunk of a lane.
@@ -262,18 +280,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 }
                 continue;
             }
-            bool valid = false;
+            bool valid = false, fp4 = false;
             if (lane < 16) {
                 const int64_t s = tb + lw * 16 + lane;
-                const uint16_t* r = s < s1 ? key_row(p, D, kl, s) : nullptr;
+                const uint8_t* scl = nullptr;
+                const void* r = s < s1 ? key_src(p, D, kl, s, &scl) : nullptr;
                 rowptr_w[lane] = reinterpret_cast<uint64_t>(r);
+                rowscl_w[lane] = reinterpret_cast<uint64_t>(scl);
                 valid = r != nullptr;
+                fp4 = scl != nullptr;
             }
             const uint32_t vm = __ballot_sync(0xffffffffu, valid) & 0xFFFFu;
+            const bool tile_fp4 = __ballot_sync(0xffffffffu, fp4) != 0u;
             __syncwarp();
             const uint32_t kbase = sbase + L::kK + (uint32_t)st * L::kStage + lane_blk;
-#pragma unroll 4
-            for (int r = 0; r < 16; ++r) {
+            // a bf16 row (or an empty one: zeros) by cp.async, this lane's 16-byte chunks
+            auto copy_row = [&](int r) {
                 const uint16_t* row = reinterpret_cast<const uint16_t*>(rowptr[r]);
                 const int key = lw * 16 + r;
                 const uint32_t dst = kbase + (uint32_t)key * 128u + ((lane_c7 ^ (key & 7)) << 4);
@@ -284,6 +306,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                     for (int u = 0; u < CPL; ++u) cp_async16(dst + u * 4 * L::kBlock, src + (lane + 32 * u) * 8, nb);
                 } else if (lane < CPR) {
                     cp_async16(dst, src + lane * 8, nb);
+                }
+            };
+            if (!tile_fp4) {
+#pragma unroll 4
+                for (int r = 0; r < 16; ++r) copy_row(r);
+            } else {
+                // FP4 entries: chunk c of a row (channels 8c .. 8c+7) is the 4 code bytes at 4c and the
+                // scale byte c/4; dequantized in registers and stored into the tile's swizzled slot.
+                // Four rows at a time, their loads issued unconditionally (a row that is not FP4 loads
+                // from the query instead and goes by cp.async), then converted.
+#pragma unroll 1
+                for (int r0 = 0; r0 < 16; r0 += 4) {
+                    uint32_t cw[4][CPL], sb[4][CPL];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint8_t* sc = reinterpret_cast<const uint8_t*>(rowscl[r0 + i]);
+                        const uint8_t* cr = sc ? reinterpret_cast<const uint8_t*>(rowptr[r0 + i])
+                                               : reinterpret_cast<const uint8_t*>(p.q);
+                        const uint8_t* sr = sc ? sc : reinterpret_cast<const uint8_t*>(p.q);
+#pragma unroll
+                        for (int u = 0; u < CPL; ++u) {
+                            const int c = (lane + 32 * u) < CPR ? lane + 32 * u : 0;
+                            cw[i][u] = __ldg(reinterpret_cast<const unsigned int*>(cr + 4 * c));
+                            sb[i][u] = __ldg(sr + (c >> 2));
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = r0 + i;
+                        if (rowscl[r] == 0) {
+                            copy_row(r);
+                            continue;
+                        }
+                        const int key = lw * 16 + r;
+                        const uint32_t dst = kbase + (uint32_t)key * 128u + ((lane_c7 ^ (key & 7)) << 4);
+#pragma unroll
+                        for (int u = 0; u < CPL; ++u)
+                            if (lane + 32 * u < CPR) st_shared_v4(dst + u * 4 * L::kBlock, mx4_to_bf16x8(cw[i][u], sb[i][u]));
+                    }
                 }
             }
             cp_async_wait_all();
@@ -788,7 +849,7 @@ cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, 
     // inside one sequence's valid rows, so the row extent is left open
     AttnMaps maps;
     AttnParams q = p;
-    q.tma_hca = p.use_hca && p.hca &&
+    q.tma_hca = p.use_hca && p.hca && !p.hca_q &&
                 tensor_map_2d_bf16(&maps.hca, p.hca, D, 0x7FFFFFFFull, (uint64_t)D * 2, 64, kTileKeys) == cudaSuccess;
     q.tma_x = p.raw && p.W >= kTileKeys &&
               tensor_map_2d_bf16(&maps.x, p.raw, D, 0x7FFFFFFFull, (uint64_t)D * 2, 64, kTileKeys) == cudaSuccess;

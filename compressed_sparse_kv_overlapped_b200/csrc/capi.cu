@@ -300,13 +300,29 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
         }
     }
     if (tid < 8) {
+        // the entries (and their FP4 copies: four lanes per 32-channel block)
         const int c0 = c0s + 8 * tid;
-        if (c_do && csa_block_shape(p.m))
-            *reinterpret_cast<uint4*>(p.entries + (sq.csa_off + j) * d + c0) =
-                entry_bf16(cv, p.norm_c ? p.norm_c + c0 : nullptr, inv_c);
-        if (h_do && hca_block_shape(p.m_hca))
-            *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) =
-                entry_bf16(hv, p.norm_h ? p.norm_h + c0 : nullptr, inv_h);
+        const unsigned qmask = 0xFu << (tid & ~3);
+        if (c_do && csa_block_shape(p.m)) {
+            const int64_t row = sq.csa_off + j;
+            const uint4 e = entry_bf16(cv, p.norm_c ? p.norm_c + c0 : nullptr, inv_c);
+            *reinterpret_cast<uint4*>(p.entries + row * d + c0) = e;
+            if (p.entries_q) {
+                uint32_t sb;
+                *reinterpret_cast<uint32_t*>(p.entries_q + row * (d / 2) + c0 / 2) = quant_mx4(e, qmask, &sb);
+                if ((tid & 3) == 0) p.entries_s[row * (d / 32) + c0 / 32] = (uint8_t)sb;
+            }
+        }
+        if (h_do && hca_block_shape(p.m_hca)) {
+            const int64_t row = sq.hca_off + h;
+            const uint4 e = entry_bf16(hv, p.norm_h ? p.norm_h + c0 : nullptr, inv_h);
+            *reinterpret_cast<uint4*>(p.hca_entries + row * d + c0) = e;
+            if (p.hca_q) {
+                uint32_t sb;
+                *reinterpret_cast<uint32_t*>(p.hca_q + row * (d / 2) + c0 / 2) = quant_mx4(e, qmask, &sb);
+                if ((tid & 3) == 0) p.hca_s[row * (d / 32) + c0 / 32] = (uint8_t)sb;
+            }
+        }
     }
     // every CTA of the sequence has read seqs[b].len: CTA 0 may now write the new length
     cluster_barrier();
@@ -400,8 +416,8 @@ int status_ptr(int** out) {
 int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_e,
               int64_t e_stride, const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
               float* score_out, void* ws_index, bool zero_ws, int* status, cudaStream_t stream,
-              cudaEvent_t mid = nullptr, bool pdl = false, const csa_bf16* prefetch_entries = nullptr,
-              const uint8_t* keys_q = nullptr, const uint8_t* key_scales = nullptr) {
+              cudaEvent_t mid = nullptr, bool pdl = false, const void* prefetch_entries = nullptr,
+              int64_t prefetch_row_bytes = 0, const uint8_t* keys_q = nullptr, const uint8_t* key_scales = nullptr) {
     IndexParams ip{};
     ip.seqs = seqs;
     ip.queries = queries;
@@ -420,7 +436,7 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
     ip.keys_q = keys_q;
     ip.key_scales = key_scales;
     ip.prefetch_rows = reinterpret_cast<const unsigned char*>(prefetch_entries);
-    ip.prefetch_row_bytes = (int64_t)d.d * 2;
+    ip.prefetch_row_bytes = prefetch_row_bytes;
     index_ws_carve(ip, ws_index, Q, e_stride);
     cudaError_t e = launch_index_topk(ip, max_e, stream, zero_ws, mid, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "index_topk launch");
@@ -734,13 +750,21 @@ int csa_index_topk_mx8(const csa_dims* dims, const csa_seq* seqs, const csa_quer
     int64_t es = ((max_e + 3) / 4) * 4;
     if (es < 4) es = 4;
     return run_index(*dims, seqs, queries, Q, max_e, es, q_idx, w, nullptr, idx_out, score_out, ws, true, st, stream,
-                     nullptr, false, nullptr, keys_q, key_scales);
+                     nullptr, false, nullptr, 0, keys_q, key_scales);
 }
+
+// FP4 entry caches (codes and block scales) an attention call reads instead of the bf16 ones.
+struct Fp4Caches {
+    const uint8_t* entries_q = nullptr;
+    const uint8_t* entries_s = nullptr;
+    const uint8_t* hca_q = nullptr;
+    const uint8_t* hca_s = nullptr;
+};
 
 static int make_attn(AttnParams& p, const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q,
                      const csa_bf16* q, const csa_bf16* entries, const int32_t* idx, int k_slots, const csa_bf16* x,
                      int W, const csa_bf16* hca, float scale, float* out, float* lse, void* ws, const ItemPlan& ip,
-                     const csa_norms* norms = nullptr) {
+                     const csa_norms* norms = nullptr, const Fp4Caches& fp4 = Fp4Caches{}) {
     int* st = nullptr;
     int rc = status_ptr(&st);
     if (rc) return rc;
@@ -760,8 +784,12 @@ static int make_attn(AttnParams& p, const csa_dims* dims, const csa_seq* seqs, c
     p.raw = x;
     p.W = W;
     p.hca = hca;
+    p.entries_q = fp4.entries_q;
+    p.entries_s = fp4.entries_s;
+    p.hca_q = fp4.hca_q;
+    p.hca_s = fp4.hca_s;
     p.m_hca = dims->m_hca;
-    p.use_hca = hca != nullptr;
+    p.use_hca = hca != nullptr || fp4.hca_q != nullptr;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.n_items = ip.n_items;
     p.items_front = ip.items_front;
@@ -829,6 +857,71 @@ int hca_dense_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* q
     return run_attention_all(p, stream);
 }
 
+int csa_quantize_entries(const csa_dims* dims, const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries,
+                         int which, const csa_bf16* entries, uint8_t* entries_q, uint8_t* entry_scales,
+                         csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !ranges || !entries || !entries_q || !entry_scales) return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (which != 0 && which != 1) return fail(CSA_ERR_ARG, "which = %d (0 CSA, 1 HCA)", which);
+    if (B < 1 || max_entries < 0) return fail(CSA_ERR_ARG, "B = %d, max_entries = %lld", B, (long long)max_entries);
+    if (!aligned16(entries) || !aligned16(entries_q)) return fail(CSA_ERR_ARG, "entries / entries_q must be 16-byte aligned");
+    int* st = nullptr;
+    if ((rc = status_ptr(&st))) return rc;
+    cudaError_t e = launch_quantize_entries(seqs, ranges, B, max_entries, which, which ? dims->m_hca : dims->m,
+                                            dims->d, entries, entries_q, entry_scales, st, stream);
+    return e == cudaSuccess ? CSA_OK : cuda_fail(e, "quantize launch");
+}
+
+int csa_sparse_attn_fp4(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, const csa_bf16* q,
+                        const uint8_t* entries_q, const uint8_t* entry_scales, const int32_t* idx, const csa_bf16* x,
+                        float scale, float* out, float* lse, void* ws, size_t ws_bytes, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !queries || !q || !entries_q || !entry_scales || !idx || !x || !out)
+        return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (Q < 1) return fail(CSA_ERR_ARG, "Q = %d", Q);
+    if (!aligned16(q) || !aligned16(entries_q) || !aligned16(x) || !aligned16(out))
+        return fail(CSA_ERR_ARG, "q / entries_q / x / out must be 16-byte aligned");
+    csa_ws_query wq{*dims, Q, 0, 1};
+    const size_t need = csa_workspace_size(CSA_OP_SPARSE_ATTN, &wq);
+    if (need > 256 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+        return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", need);
+    Fp4Caches f4;
+    f4.entries_q = entries_q;
+    f4.entries_s = entry_scales;
+    AttnParams p;
+    int rc2 = make_attn(p, dims, seqs, queries, Q, q, nullptr, idx, dims->k, x, dims->W, nullptr, scale, out, lse, ws,
+                        plan_standalone((int64_t)dims->k + dims->W, 0, Q), nullptr, f4);
+    if (rc2) return rc2;
+    return run_attention_all(p, stream);
+}
+
+int hca_dense_attn_fp4(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
+                       const csa_bf16* q, const uint8_t* hca_q, const uint8_t* hca_scales, const csa_bf16* x, int W,
+                       float scale, float* out, float* lse, void* ws, size_t ws_bytes, csa_stream_t stream) {
+    int rc = check_dims(dims);
+    if (rc) return rc;
+    if (!seqs || !queries || !q || !hca_q || !hca_scales || !x || !out) return fail(CSA_ERR_ARG, "NULL pointer argument");
+    if (Q < 1 || max_len < 1 || W < 0 || W > 4096) return fail(CSA_ERR_ARG, "Q = %d, max_len, W = %d", Q, W);
+    if (!aligned16(q) || !aligned16(hca_q) || !aligned16(x) || !aligned16(out))
+        return fail(CSA_ERR_ARG, "q / hca_q / x / out must be 16-byte aligned");
+    csa_dims d2 = *dims;
+    d2.W = W;
+    csa_ws_query wq{d2, Q, 0, max_len};
+    const size_t need = csa_workspace_size(CSA_OP_HCA_ATTN, &wq);
+    if (need > 256 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)))
+        return fail(CSA_ERR_ARG, "workspace: need %zu bytes, 256-byte aligned", need);
+    Fp4Caches f4;
+    f4.hca_q = hca_q;
+    f4.hca_s = hca_scales;
+    AttnParams p;
+    int rc2 = make_attn(p, &d2, seqs, queries, Q, q, nullptr, nullptr, 0, x, W, nullptr, scale, out, lse, ws,
+                        plan_standalone(W, max_len / dims->m_hca, Q), nullptr, f4);
+    if (rc2) return rc2;
+    return run_attention_all(p, stream);
+}
+
 int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
     if (!a) return fail(CSA_ERR_ARG, "args is NULL");
     int rc = check_dims(&a->dims);
@@ -849,6 +942,13 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     if ((rc = check_norms(d, a->norms))) return rc;
     if (a->new_rows && !a->append) return fail(CSA_ERR_ARG, "new_rows without append");
     if ((a->keys_q == nullptr) != (a->key_scales == nullptr)) return fail(CSA_ERR_ARG, "keys_q and key_scales go together");
+    const bool fp4 = a->entries_q != nullptr;
+    if (fp4 != (a->entry_scales != nullptr) || fp4 != (a->hca_q != nullptr) || fp4 != (a->hca_scales != nullptr))
+        return fail(CSA_ERR_ARG, "entries_q, entry_scales, hca_q and hca_scales go together");
+    if (fp4 && (!aligned16(a->entries_q) || !aligned16(a->hca_q)))
+        return fail(CSA_ERR_ARG, "entries_q / hca_q must be 16-byte aligned");
+    if (fp4 && (!csa_block_shape(d.m) || !hca_block_shape(d.m_hca)))
+        return fail(CSA_ERR_UNSUPPORTED, "FP4 entry caches need m = 4 and m_hca a power of two from 4 to 128");
     if (a->keys_q && (!aligned16(a->keys_q) || (reinterpret_cast<uintptr_t>(a->key_scales) & 1u)))
         return fail(CSA_ERR_ARG, "keys_q must be 16-byte aligned, key_scales 2-byte aligned");
     const DecodePlan pl = plan_decode(d, a->B, a->max_len);
@@ -882,6 +982,10 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     ap.hca_entries = a->hca_entries;
     ap.keys_q = a->keys_q;
     ap.key_scales = a->key_scales;
+    ap.entries_q = a->entries_q;
+    ap.entries_s = a->entry_scales;
+    ap.hca_q = a->hca_q;
+    ap.hca_s = a->hca_scales;
     if (a->norms) {
         ap.norm_c = a->norms->entry_norm_c;
         ap.norm_h = a->norms->entry_norm_h;
@@ -898,8 +1002,13 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     if (e == cudaSuccess) e = mark(ev[1], stream);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
     AttnParams ap2;
+    Fp4Caches f4;
+    f4.entries_q = a->entries_q;
+    f4.entries_s = a->entry_scales;
+    f4.hca_q = a->hca_q;
+    f4.hca_s = a->hca_scales;
     rc = make_attn(ap2, &d, a->seqs, queries, a->B, a->q, a->entries, idx, d.k, a->x, d.W, a->hca_entries, a->scale,
-                   a->out, a->lse, w + pl.off_attn, pl.items, a->norms);
+                   a->out, a->lse, w + pl.off_attn, pl.items, a->norms, f4);
     if (rc) return rc;
     // programmatic dependent launch chains append -> scan -> select -> attention -> merge unless
     // stage events are being recorded between them
@@ -913,7 +1022,9 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     ap2.cluster = pl.cluster;
     if (!reuse) {
         rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
-                       ws_index, false, st, stream, ev[2], pdl, a->entries, a->keys_q, a->key_scales);
+                       ws_index, false, st, stream, ev[2], pdl,
+                       fp4 ? static_cast<const void*>(a->entries_q) : static_cast<const void*>(a->entries),
+                       fp4 ? (int64_t)d.d / 2 : (int64_t)d.d * 2, a->keys_q, a->key_scales);
         if (rc) return rc;
     } else if ((e = mark(ev[2], stream)) != cudaSuccess) {
         return cuda_fail(e, "event record");

@@ -143,6 +143,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// 16-byte store to shared memory (a shared-window address).
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy (tensor-core reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -348,6 +354,57 @@ __device__ __forceinline__ uint2 quant_mx8(const uint4& kb, unsigned mask, uint3
         w[i] = two;
     }
     return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// The 4-bit form for the FP4 entry cache: eight bf16 values (four lanes per 32-channel block, `mask`
+// those lanes) to E2M1 codes (sign, two exponent bits with bias 1, one mantissa bit; the hardware
+// conversion rounds to nearest, ties to even) with the block's scale 2^e, e the smallest integer
+// such that amax <= 6 * 2^e (e >= -127).  Returns the eight codes, the even channel in the low nibble
+// of each byte; *scale_byte = e + 127.
+__device__ __forceinline__ uint32_t quant_mx4(const uint4& kb, unsigned mask, uint32_t* scale_byte) {
+    float f[8];
+    unpack8(kb, f);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(mask, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(mask, amax, 2));
+    int e = -127;
+    if (amax > 0.f) {
+        int ex;
+        frexpf(amax, &ex);  // amax in [2^(ex-1), 2^ex)
+        e = ex - 3;
+        while (amax > ldexpf(6.f, e)) ++e;
+        while (e > -127 && amax <= ldexpf(6.f, e - 1)) --e;
+    }
+    *scale_byte = (uint32_t)(e + 127);
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t two;
+        // the first operand goes to the high nibble: element 2i + 1 high, 2i low
+        asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+            : "=r"(two) : "f"(ldexpf(f[2 * i + 1], -e)), "f"(ldexpf(f[2 * i], -e)));
+        w |= (two & 0xFFu) << (8 * i);
+    }
+    return w;
+}
+
+// Eight E2M1 codes (a word, the even channel in the low nibble of each byte) with the block scale
+// byte s to eight bf16 values: code value * 2^(s - 127), exact (two significant bits times a power of
+// two; the product is formed in fp32, subnormals included).
+__device__ __forceinline__ uint4 mx4_to_bf16x8(uint32_t w, uint32_t s) {
+    const float f = s ? __uint_as_float(s << 23) : __uint_as_float(0x00400000u);  // 2^(s - 127)
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h2;
+        asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "r"((w >> (8 * i)) & 0xFFu));
+        const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+        const __nv_bfloat162 b = __floats2bfloat162_rn(v.x * f, v.y * f);
+        o[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -918,6 +918,33 @@ __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexPara
         if (j >= 0) prefetch_l2(p.prefetch_rows + (sq.csa_off + j) * p.prefetch_row_bytes, p.prefetch_row_bytes);
     }
 }
+// FP4 copies (E2M1 codes, 32-channel power-of-two block scales; quant_mx4) of the stored bf16 entries
+// [ranges[b][0], ranges[b][1]) of every sequence's CSA cache (which = 0, ratio m) or HCA cache
+// (which = 1, ratio m_hca): d / 8 threads per entry, four lanes per block.
+__global__ void __launch_bounds__(256) quantize_entries_kernel(const csa_seq* seqs, const int64_t* ranges, int which,
+                                                               int ratio, int d, const uint16_t* entries,
+                                                               uint8_t* entries_q, uint8_t* scales, int* status) {
+    const int b = blockIdx.y;
+    const int tpe = d / 8;  // threads per entry (a multiple of 4)
+    const int64_t e0 = ranges[2 * b], e1 = ranges[2 * b + 1];
+    const csa_seq sq = seqs[b];
+    if (e0 < 0 || e1 < e0 || (int64_t)ratio * e1 > sq.len) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) report(status, CSA_ERR_INDEX);
+        return;
+    }
+    const int lane = threadIdx.x & 31, sub = threadIdx.x / tpe, g = threadIdx.x % tpe;
+    const unsigned mask = 0xFu << (lane & ~3);
+    const int64_t base = which ? sq.hca_off : sq.csa_off;
+    for (int64_t j = e0 + (int64_t)blockIdx.x * (256 / tpe) + sub; j < e1; j += (int64_t)gridDim.x * (256 / tpe)) {
+        const int64_t row = base + j;
+        const uint4 v = *reinterpret_cast<const uint4*>(entries + row * d + 8 * g);
+        uint32_t sb;
+        const uint32_t q = quant_mx4(v, mask, &sb);
+        *reinterpret_cast<uint32_t*>(entries_q + row * (d / 2) + 4 * g) = q;
+        if ((g & 3) == 0) scales[row * (d / 32) + g / 4] = (uint8_t)sb;
+    }
+}
+
 constexpr size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 }  // namespace
@@ -1029,6 +1056,18 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
     // the exact selection: one cluster of kFinalF CTAs per query
     return launch_kernel_cluster(index_final_kernel, dim3(kFinalF, (unsigned)p.Q), dim3(kFinalThreads), kFinalDynSmem,
                                  stream, pdl, dim3(kFinalF, 1, 1), p);
+}
+
+cudaError_t launch_quantize_entries(const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries, int which,
+                                    int ratio, int d, const uint16_t* entries, uint8_t* entries_q, uint8_t* scales,
+                                    int* status, cudaStream_t stream) {
+    if (max_entries <= 0) return cudaSuccess;
+    const int per_cta = 256 / (d / 8);
+    int64_t gx = (max_entries + per_cta - 1) / per_cta;
+    if (gx > 8192) gx = 8192;
+    quantize_entries_kernel<<<dim3((unsigned)gx, (unsigned)B), 256, 0, stream>>>(seqs, ranges, which, ratio, d, entries,
+                                                                                entries_q, scales, status);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_keys(const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries, int m,

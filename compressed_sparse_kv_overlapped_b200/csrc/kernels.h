@@ -100,6 +100,11 @@ size_t index_zero_bytes(int Q);  // leading bytes of the index workspace that mu
 // Points the workspace arrays of `p` into `ws` and sets the scan chunking (chunk, max_chunks,
 // cand_cap), all derived from (Q, e_stride) exactly as index_ws_bytes sizes them.
 void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride);
+// FP4 copies (codes [*, d / 2], scales [*, d / 32]) of the stored bf16 entries [ranges[b][0],
+// ranges[b][1]) of the CSA cache (which = 0, ratio m) or the HCA cache (which = 1, ratio m_hca).
+cudaError_t launch_quantize_entries(const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries, int which,
+                                    int ratio, int d, const uint16_t* entries, uint8_t* entries_q, uint8_t* scales,
+                                    int* status, cudaStream_t stream);
 // 8-bit block-scaled copies (keys_q [*, d_I] E4M3, scales [*, d_I / 32]) of the stored bf16 indexer
 // keys of entries [ranges[b][0], ranges[b][1]) of every sequence.
 cudaError_t launch_quantize_keys(const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries, int m,
@@ -143,6 +148,12 @@ struct AttnParams {
     const uint16_t* raw;        // raw latents (window)
     int W;
     const uint16_t* hca;        // HCA cache (nullable when use_hca == 0)
+    // FP4 entry caches (E2M1 codes [*, d / 2] and power-of-two block scales [*, d / 32]); when set, the
+    // CSA entries / HCA entries are read from these and dequantized into the key tiles
+    const uint8_t* entries_q;
+    const uint8_t* entries_s;
+    const uint8_t* hca_q;
+    const uint8_t* hca_s;
     int m_hca;
     int use_hca;
     float scale_log2;           // scale * log2(e)
@@ -216,6 +227,10 @@ struct AppendParams {
     uint16_t* hca_entries;
     uint8_t* keys_q;         // nullable: 8-bit block-scaled copy of each new indexer key
     uint8_t* key_scales;
+    uint8_t* entries_q;      // nullable: FP4 copies of each new CSA / HCA entry (codes, block scales)
+    uint8_t* entries_s;
+    uint8_t* hca_q;
+    uint8_t* hca_s;
     const float* norm_c;     // [d] RMS-normalization gains of new CSA / HCA entries (nullable)
     const float* norm_h;
     float eps;

@@ -7,6 +7,9 @@ Memory layout in HBM (row-major, every tensor 256-byte aligned by the allocator)
   CSA cache    entries             : [sum_b cap_b // m, d]   bf16   (rows csa_off[b]..)
                entry_keys          : [sum_b cap_b // m, d_I] bf16
   HCA cache    hca_entries         : [sum_b cap_b // m', d]  bf16   (rows hca_off[b]..)
+  optional     keys_q / key_scales  (key_format "mx8"): 8-bit indexer keys [*, d_I] + [*, d_I / 32]
+               entries_q / entry_scales, hca_q / hca_scales (kv_format "fp4"): FP4 entries
+               [*, d / 2] + [*, d / 32] beside the bf16 caches
   parameters   bias_c [2m, d], bias_h [m', d] fp32
   table        seqs                : [B, 4] int64 = (tok_off, csa_off, hca_off, len) = csa_seq
 
@@ -18,14 +21,17 @@ from __future__ import annotations
 import ctypes
 
 from . import (CSA_OP_DECODE, CSA_OP_PREFILL, csa_compress, csa_compress_all, csa_decode_args, csa_norms,
-               csa_prefill_args, csa_quantize_keys, csa_workspace_size, hybrid_attn_decode, hybrid_attn_prefill)
+               csa_prefill_args, csa_quantize_entries, csa_quantize_keys, csa_workspace_size, hybrid_attn_decode,
+               hybrid_attn_prefill)
 
 
 class HybridLayer:
     """key_format "mx8" adds 8-bit block-scaled copies of the indexer keys (keys_q [*, d_I] E4M3,
-    key_scales [*, d_I / 32]) that the decode's indexer scores instead of the bf16 keys."""
+    key_scales [*, d_I / 32]) that the decode's indexer scores instead of the bf16 keys.  kv_format
+    "fp4" adds FP4 copies of the CSA and HCA entries (E2M1 codes [*, d / 2], scales [*, d / 32]) that
+    the decode's attention reads instead of the bf16 entries."""
 
-    def __init__(self, dims, capacity, device="cuda", key_format="bf16"):
+    def __init__(self, dims, capacity, device="cuda", key_format="bf16", kv_format="bf16"):
         import torch
 
         self.dims = dims
@@ -57,6 +63,16 @@ class HybridLayer:
         if key_format == "mx8":
             self.keys_q = torch.zeros(max(c, 1), dI, dtype=torch.uint8, device=device)
             self.key_scales = torch.zeros(max(c, 1), dI // 32, dtype=torch.uint8, device=device)
+        if kv_format not in ("bf16", "fp4"):
+            raise ValueError(f"kv_format {kv_format!r}")
+        self.kv_format = kv_format
+        self.entries_q = self.entry_scales = self.hca_q = self.hca_scales = None
+        if kv_format == "fp4":
+            u8 = torch.uint8
+            self.entries_q = torch.zeros(max(c, 1), d // 2, dtype=u8, device=device)
+            self.entry_scales = torch.zeros(max(c, 1), d // 32, dtype=u8, device=device)
+            self.hca_q = torch.zeros(max(h, 1), d // 2, dtype=u8, device=device)
+            self.hca_scales = torch.zeros(max(h, 1), d // 32, dtype=u8, device=device)
         self.bias_c = torch.zeros(2 * m, d, dtype=torch.float32, device=device)
         self.bias_h = torch.zeros(mh, d, dtype=torch.float32, device=device)
         self.seqs = torch.tensor([[tok[b], csa[b], hca[b], 0] for b in range(self.B)], dtype=torch.int64,
@@ -92,7 +108,25 @@ class HybridLayer:
                              self.hca_entries, stream, norms=self.norms)
         if self.keys_q is not None:
             self.quantize_keys(stream)
+        if self.entries_q is not None:
+            self.quantize_entries(stream)
         self._keep = rt  # the kernels read the range table asynchronously
+
+    def quantize_entries(self, stream=None) -> None:
+        """The FP4 copies of every complete CSA and HCA entry (kv_format "fp4")."""
+        import torch
+        d = self.dims
+        ec = [n // d.m for n in self.lens]
+        eh = [n // d.m_hca for n in self.lens]
+        rc = torch.tensor([[0, n] for n in ec], dtype=torch.int64, device=self.device)
+        rh = torch.tensor([[0, n] for n in eh], dtype=torch.int64, device=self.device)
+        if max(ec) > 0:
+            csa_quantize_entries(d, self.seqs, rc, self.B, max(ec), 0, self.entries, self.entries_q, self.entry_scales,
+                                 stream)
+        if max(eh) > 0:
+            csa_quantize_entries(d, self.seqs, rh, self.B, max(eh), 1, self.hca_entries, self.hca_q, self.hca_scales,
+                                 stream)
+        self._keep_e = (rc, rh)
 
     def quantize_keys(self, stream=None) -> None:
         """The 8-bit copies of every complete entry's indexer key (key_format "mx8")."""
@@ -135,7 +169,8 @@ class HybridLayer:
                         ("entries", self.entries), ("entry_keys", self.entry_keys),
                         ("hca_entries", self.hca_entries), ("q", q), ("q_idx", q_idx), ("w", w), ("out", out),
                         ("lse", lse), ("idx_out", idx_out), ("new_rows", new_rows), ("keys_q", self.keys_q),
-                        ("key_scales", self.key_scales), ("idx_in", idx_in)):
+                        ("key_scales", self.key_scales), ("idx_in", idx_in), ("entries_q", self.entries_q),
+                        ("entry_scales", self.entry_scales), ("hca_q", self.hca_q), ("hca_scales", self.hca_scales)):
             setattr(a, name, None if t is None else t.data_ptr())
         if self.norms is not None:
             a.norms = ctypes.pointer(self.norms)

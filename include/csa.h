@@ -189,6 +189,32 @@ int csa_sparse_attn(const csa_dims* dims, const csa_seq* seqs, const csa_query* 
                     const csa_bf16* entries, const int32_t* idx, const csa_bf16* x, float scale, float* out,
                     float* lse, void* ws, size_t ws_bytes, csa_stream_t stream);
 
+/* f4 -- FP4 compressed entries with block scales ("Compressed attention · CSA / HCA", section 3: the
+ * FP4 KV cache of V4.1 carries block scales and a packing overhead).  Each 32-channel block of an
+ * entry row shares one power-of-two scale 2^e, stored as the byte e + 127, where 2^e is the smallest
+ * power of two with amax <= 6 * 2^e (a zero block: e = -127); the elements are E2M1 codes (sign, two
+ * exponent bits with bias 1, one mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) of x / 2^e
+ * rounded to nearest even, two per byte, the even channel in the low nibble.  Row r of an FP4 cache
+ * mirrors row r of its bf16 cache (CSA: csa_off + j, HCA: hca_off + j): d / 2 code bytes
+ * (entries_q, 16-byte aligned) and d / 32 scale bytes (entry_scales).  Per 512-wide entry 256 + 16
+ * bytes instead of 1,024.  The attention uses the dequantized entries (code * 2^e, every one a bf16
+ * value) as keys and values; the raw window stays bf16.
+ *
+ * csa_quantize_entries: the FP4 copies of the stored bf16 entries [ranges[b][0], ranges[b][1]) of
+ * every sequence's CSA cache (which = 0) or HCA cache (which = 1); ranges and max_entries as in
+ * csa_compress (the entries must exist, else CSA_ERR_INDEX on the device).
+ * csa_sparse_attn_fp4 / hca_dense_attn_fp4: csa_sparse_attn / hca_dense_attn reading the entries
+ * from the FP4 caches; same outputs and workspace sizes. */
+int csa_quantize_entries(const csa_dims* dims, const csa_seq* seqs, const int64_t* ranges, int B, int64_t max_entries,
+                         int which, const csa_bf16* entries, uint8_t* entries_q, uint8_t* entry_scales,
+                         csa_stream_t stream);
+int csa_sparse_attn_fp4(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, const csa_bf16* q,
+                        const uint8_t* entries_q, const uint8_t* entry_scales, const int32_t* idx, const csa_bf16* x,
+                        float scale, float* out, float* lse, void* ws, size_t ws_bytes, csa_stream_t stream);
+int hca_dense_attn_fp4(const csa_dims* dims, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_len,
+                       const csa_bf16* q, const uint8_t* hca_q, const uint8_t* hca_scales, const csa_bf16* x, int W,
+                       float scale, float* out, float* lse, void* ws, size_t ws_bytes, csa_stream_t stream);
+
 /* a6 -- dense MQA attention over every visible HCA entry ("Frontier Techniques", 2.2; "DeepSeek V4
  * comprimeix el context", "HCA: un resum global 128 vegades mes curt").  Keys: hca_entries[hca_off
  * + j] for j < floor(L/m_hca), then (when W > 0) the raw window [max(0, L-W), L).  An empty key set
@@ -242,6 +268,14 @@ typedef struct csa_decode_args {
                                  every layer of a sequence */
     const csa_norms* norms;   /* optional (host struct, see csa_norms): query / entry normalization
                                  and sink logits; NULL: none */
+    uint8_t* entries_q;       /* optional FP4 copy of the CSA entry cache [*, d / 2] (see
+                                 csa_quantize_entries; 16-byte aligned), with entry_scales [*, d / 32],
+                                 hca_q and hca_scales (all four or none; m = 4 and m_hca a power of two
+                                 from 4 to 128).  When given, the attention reads the FP4 caches and
+                                 the append also writes the FP4 copy of every entry it completes */
+    uint8_t* entry_scales;
+    uint8_t* hca_q;           /* optional FP4 copy of the HCA entry cache [*, d / 2] (16-byte aligned) */
+    uint8_t* hca_scales;      /* [*, d / 32] */
 } csa_decode_args;
 
 /* a8 + a3..a7 -- one decode step: optional append (and the compressor updates it triggers), then

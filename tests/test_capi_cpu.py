@@ -42,11 +42,11 @@ def test_struct_layouts_match_header(tmp_path):
     prog = tmp_path / "sizes.c"
     prog.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "csa.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(csa_dims), sizeof(csa_seq),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(csa_dims), sizeof(csa_seq),"
         " sizeof(csa_query), sizeof(csa_ws_query), sizeof(csa_decode_args), sizeof(csa_prefill_args),"
         " offsetof(csa_decode_args, out), offsetof(csa_prefill_args, idx_out),"
         " offsetof(csa_decode_args, new_rows), offsetof(csa_decode_args, norms), offsetof(csa_prefill_args, norms),"
-        " sizeof(csa_norms));return 0;}\n")
+        " sizeof(csa_norms), offsetof(csa_decode_args, entries_q), offsetof(csa_decode_args, hca_scales));return 0;}\n")
     exe = tmp_path / "sizes"
     subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
@@ -54,7 +54,8 @@ def test_struct_layouts_match_header(tmp_path):
                    ctypes.sizeof(csa.csa_decode_args), ctypes.sizeof(csa.csa_prefill_args),
                    csa.csa_decode_args.out.offset, csa.csa_prefill_args.idx_out.offset,
                    csa.csa_decode_args.new_rows.offset, csa.csa_decode_args.norms.offset,
-                   csa.csa_prefill_args.norms.offset, ctypes.sizeof(csa.csa_norms)]
+                   csa.csa_prefill_args.norms.offset, ctypes.sizeof(csa.csa_norms),
+                   csa.csa_decode_args.entries_q.offset, csa.csa_decode_args.hca_scales.offset]
 
 
 def test_version_and_error_string(lib):
@@ -98,6 +99,30 @@ def test_host_validation_rejects_bad_arguments(lib):
     rc = lib.hybrid_attn_decode(ctypes.byref(a), 256, 1 << 30, None)
     assert rc == csa.CSA_ERR_ARG and "aligned" in csa.csa_last_error()
     a.new_rows = None
+    # decode: the FP4 entry caches come as a set of four, 16-byte aligned, for the block shapes
+    a.entries_q = 256
+    rc = lib.hybrid_attn_decode(ctypes.byref(a), 256, 1 << 30, None)
+    assert rc == csa.CSA_ERR_ARG and "go together" in csa.csa_last_error()
+    a.entry_scales, a.hca_q, a.hca_scales = 256, 264, 256
+    rc = lib.hybrid_attn_decode(ctypes.byref(a), 256, 1 << 30, None)
+    assert rc == csa.CSA_ERR_ARG and "aligned" in csa.csa_last_error()
+    a.hca_q = 256
+    a.dims = csa.make_dims(m=2)
+    rc = lib.hybrid_attn_decode(ctypes.byref(a), 256, 1 << 30, None)
+    assert rc == csa.CSA_ERR_UNSUPPORTED and "FP4" in csa.csa_last_error()
+    a.dims = dims
+    a.entries_q = a.entry_scales = a.hca_q = a.hca_scales = None
+    # FP4 quantization and attention calls
+    rc = lib.csa_quantize_entries(ctypes.byref(dims), 16, 16, 1, 10, 2, 16, 16, 16, None)
+    assert rc == csa.CSA_ERR_ARG and "which" in csa.csa_last_error()
+    rc = lib.csa_quantize_entries(ctypes.byref(dims), 16, 16, 1, 10, 0, 16, 24, 16, None)
+    assert rc == csa.CSA_ERR_ARG and "aligned" in csa.csa_last_error()
+    rc = lib.csa_quantize_entries(ctypes.byref(dims), 16, None, 1, 10, 0, 16, 16, 16, None)
+    assert rc == csa.CSA_ERR_ARG and "NULL" in csa.csa_last_error()
+    rc = lib.csa_sparse_attn_fp4(ctypes.byref(dims), 16, 16, 1, 16, 16, None, 16, 16, 0.1, 16, None, None, 0, None)
+    assert rc == csa.CSA_ERR_ARG and "NULL" in csa.csa_last_error()
+    rc = lib.hca_dense_attn_fp4(ctypes.byref(dims), 16, 16, 1, 100, 16, 24, 16, 16, 0, 0.1, 16, None, None, 0, None)
+    assert rc == csa.CSA_ERR_ARG and "aligned" in csa.csa_last_error()
     # prefill: bad query range
     pa = csa.csa_prefill_args()
     pa.dims = dims

@@ -392,6 +392,159 @@ def test_decode_with_8bit_keys(wl, steps):
             gh.check_close(out[b].cpu().numpy(), O, f"8-bit keys: step {s} seq {b}")
 
 
+# --------------------------------------------------------------------------------- f4: FP4 entries
+
+def _mx4_codes_match(got, want):
+    """Packed E2M1 code bytes equal, except that a zero element (magnitude bits 0) may carry either
+    sign (both are the value 0)."""
+    def canon(b):
+        lo, hi = b & 15, b >> 4
+        lo = np.where((lo & 7) == 0, 0, lo)
+        hi = np.where((hi & 7) == 0, 0, hi)
+        return lo | (hi << 4)
+    return np.array_equal(canon(got), canon(want))
+
+
+def _check_mx4(eq, es, E_rows, what):
+    """The FP4 copies (codes eq, scales es) of bf16 rows E_rows are the oracle's quantization."""
+    rq, rs = oracle.quantize_entries_mx4(E_rows)
+    np.testing.assert_array_equal(es, rs, err_msg=f"{what}: scale bytes")
+    assert _mx4_codes_match(eq, rq), f"{what}: codes"
+    np.testing.assert_array_equal(oracle.dequantize_entries_mx4(eq, es), oracle.dequantize_entries_mx4(rq, rs))
+
+
+@pytest.mark.parametrize("E_list,d,scale", [([700, 33], 512, 1.0), ([257], 128, 2.0 ** -60), ([100, 5], 512, 7.0e4)])
+@pytest.mark.parametrize("which", [0, 1])
+def test_quantize_entries_matches_oracle(E_list, d, scale, which):
+    """csa_quantize_entries writes the oracle's scale bytes and E2M1 codes for stored CSA / HCA entries
+    (an all-zero row and extreme magnitudes included)."""
+    dims = csa.make_dims(d=d, H=8, d_I=32, H_I=4, m=4, m_hca=16, k=32, W=16)
+    ratio = 4 if which == 0 else 16
+    Es = [oracle.round_bf16(synth.bf16_to_f64(synth.bf16_normal(3301, synth.X, i, d, 0, E)) * scale)
+          for i, E in enumerate(E_list)]
+    Es[0][3] = 0
+    offs = np.cumsum([0] + list(E_list))
+    ent = gh.to_dev_bf16(np.concatenate(Es))
+    rows = [[0, offs[i], 0, ratio * E] if which == 0 else [0, 0, offs[i], ratio * E] for i, E in enumerate(E_list)]
+    seqs = torch.tensor(rows, dtype=torch.int64, device="cuda")
+    ranges = torch.tensor([[0, E] for E in E_list], dtype=torch.int64, device="cuda")
+    eq = torch.full((offs[-1], d // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    es = torch.full((offs[-1], d // 32), 0xAA, dtype=torch.uint8, device="cuda")
+    csa.csa_quantize_entries(dims, seqs, ranges, len(E_list), max(E_list), which, ent, eq, es)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    _check_mx4(eq.cpu().numpy(), es.cpu().numpy(), np.concatenate(Es), f"which={which}")
+
+
+@pytest.mark.parametrize("wl,lens", [(workloads.tiny(), [1023, 17, 5]),
+                                     (wl_small(5000, B=1), [5000, 4096, 130, 1]),
+                                     (wl_small([3000, 1300], B=2), [3000, 1299])],
+                         ids=["tiny", "prod", "prod_ragged"])
+def test_fp4_attention_stage(wl, lens):
+    """Sparse and HCA attention reading FP4 entry caches (the oracle's quantization of its own entries,
+    the same bytes on both sides) against the oracle's attention over the dequantized entries."""
+    layer, refs = _stage_layer(wl)
+    d = wl.dims
+    sh = gh.oshape(d)
+    n_rows_c, n_rows_h = layer.entries.shape[0], layer.hca_entries.shape[0]
+    eq = torch.zeros(n_rows_c, d.d // 2, dtype=torch.uint8, device="cuda")
+    es = torch.zeros(n_rows_c, d.d // 32, dtype=torch.uint8, device="cuda")
+    hq = torch.zeros(n_rows_h, d.d // 2, dtype=torch.uint8, device="cuda")
+    hs = torch.zeros(n_rows_h, d.d // 32, dtype=torch.uint8, device="cuda")
+    deq_c, deq_h = [], []
+    for b in range(wl.B):
+        n_c, n_h = len(refs[b].E), wl.n0[b] // d.m_hca
+        q_, s_ = oracle.quantize_entries_mx4(refs[b].E)
+        eq[layer.csa_off[b]:layer.csa_off[b] + n_c] = torch.from_numpy(q_).cuda()
+        es[layer.csa_off[b]:layer.csa_off[b] + n_c] = torch.from_numpy(s_).cuda()
+        deq_c.append(oracle.mx4_entries_as_bf16(refs[b].E))
+        if n_h:
+            q_, s_ = oracle.quantize_entries_mx4(refs[b].H[:n_h])
+            hq[layer.hca_off[b]:layer.hca_off[b] + n_h] = torch.from_numpy(q_).cuda()
+            hs[layer.hca_off[b]:layer.hca_off[b] + n_h] = torch.from_numpy(s_).cuda()
+            deq_h.append(oracle.mx4_entries_as_bf16(refs[b].H[:n_h]))
+        else:
+            deq_h.append(refs[b].H[:1])
+    pairs = [(i % wl.B, L) for i, L in enumerate(lens)]
+    pairs = [(b, min(L, wl.n0[b])) for b, L in pairs]
+    Q = len(pairs)
+    qs = np.stack([workloads.queries(wl, b, i, i + 1)[0][0] for i, (b, _) in enumerate(pairs)])
+    idxs = []
+    for i, (b, L) in enumerate(pairs):
+        _, qi_, w_ = workloads.queries(wl, b, i, i + 1)
+        idxs.append(oracle.topk(oracle.index_scores(qi_[0], w_[0], refs[b].KI[:L // d.m]), d.k))
+    qt = gh.query_table(pairs)
+    q_d = gh.to_dev_bf16(qs)
+    idx_d = torch.from_numpy(np.stack(idxs)).cuda()
+    out = torch.empty(Q, d.H, d.d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(Q, d.H, dtype=torch.float32, device="cuda")
+    dims = gh.dims_of(d)
+    wq = csa.csa_ws_query()
+    wq.dims, wq.Q, wq.max_len = dims, Q, max(wl.n0)
+    ws = torch.empty(max(csa.csa_workspace_size(csa.CSA_OP_SPARSE_ATTN, wq),
+                         csa.csa_workspace_size(csa.CSA_OP_HCA_ATTN, wq)) + 256, dtype=torch.uint8, device="cuda")
+    csa.csa_sparse_attn_fp4(dims, layer.seqs, qt, Q, q_d, eq, es, idx_d, layer.x, sh.scale, out, lse, ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    for i, (b, L) in enumerate(pairs):
+        O, l = oracle.csa_attn(qs[i], deq_c[b], idxs[i], d.m, refs[b].x, L, d.W, sh.scale)
+        gh.check_close(out[i].cpu().numpy(), O, f"fp4 csa q{i} L={L}")
+        gh.check_close(lse[i].cpu().numpy(), l, f"fp4 csa lse q{i}")
+    for W in (0, d.W):
+        out.fill_(float("nan"))
+        csa.hca_dense_attn_fp4(dims, layer.seqs, qt, Q, max(wl.n0), q_d, hq, hs, layer.x, W, sh.scale, out, lse, ws)
+        assert csa.csa_sync_status() == csa.CSA_OK
+        for i, (b, L) in enumerate(pairs):
+            O, l = oracle.hca_attn(qs[i], deq_h[b], d.m_hca, refs[b].x, L, W, sh.scale)
+            if np.isneginf(l).all():
+                assert np.isneginf(lse[i].cpu().numpy()).all() and (out[i] == 0).all()
+                continue
+            gh.check_close(out[i].cpu().numpy(), O, f"fp4 hca q{i} L={L} W={W}")
+            gh.check_close(lse[i].cpu().numpy(), l, f"fp4 hca lse q{i}")
+
+
+@pytest.mark.parametrize("wl,steps", [(workloads.tiny(), 3), (wl_small([3000, 9001], B=2), 5)], ids=["tiny", "prod"])
+def test_decode_with_fp4_entries(wl, steps):
+    """Decode reading FP4 entry caches: the FP4 copies (from the full pass, and from the append for the
+    entries it completes) are the oracle's quantization of the stored bf16 entries, the selection is
+    the oracle's top-k, and the output is the oracle's attention over the dequantized entries."""
+    wl = dataclasses.replace(wl, steps=max(wl.steps, steps))
+    d = wl.dims
+    layer = csa.HybridLayer(gh.dims_of(d), [wl.capacity(b) for b in range(wl.B)], kv_format="fp4")
+    sdev.fill_layer_inputs(layer, wl)
+    layer.set_lengths(list(wl.n0))
+    layer.compress()
+    B = wl.B
+    q = torch.empty(B, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(B, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(B, d.H_I, dtype=torch.float32, device="cuda")
+    out = torch.empty(B, d.H, d.d, dtype=torch.float32, device="cuda")
+    idx = torch.empty(B, d.k, dtype=torch.int32, device="cuda")
+    ws = layer.decode_workspace()
+    sh = gh.oshape(d)
+    for s in range(steps):
+        for b in range(B):
+            sdev.fill_queries(wl, b, s, s + 1, q[b:b + 1], qi[b:b + 1], w[b:b + 1])
+        layer.decode(layer.decode_args(q, qi, w, out, idx_out=idx), ws)
+        assert csa.csa_sync_status() == csa.CSA_OK
+        ent, hca, x, keys = gh.u16(layer.entries), gh.u16(layer.hca_entries), gh.u16(layer.x), gh.u16(layer.entry_keys)
+        eq, es = layer.entries_q.cpu().numpy(), layer.entry_scales.cpu().numpy()
+        hq, hs = layer.hca_q.cpu().numpy(), layer.hca_scales.cpu().numpy()
+        for b in range(B):
+            L = wl.n0[b] + s + 1
+            c0, n_c, h0, n_h, t0 = layer.csa_off[b], L // d.m, layer.hca_off[b], L // d.m_hca, layer.tok_off[b]
+            _check_mx4(eq[c0:c0 + n_c], es[c0:c0 + n_c], ent[c0:c0 + n_c], f"CSA step {s} seq {b}")
+            if n_h:
+                _check_mx4(hq[h0:h0 + n_h], hs[h0:h0 + n_h], hca[h0:h0 + n_h], f"HCA step {s} seq {b}")
+            qh, qih, wh = workloads.queries(wl, b, s, s + 1)
+            sc = oracle.index_scores(qih[0], wh[0], keys[c0:c0 + n_c])
+            gh.sets_match(idx[b].cpu().numpy(), oracle.topk(sc, d.k), sc, d.k)
+            dc = oracle.mx4_entries_as_bf16(ent[c0:c0 + max(n_c, 1)])
+            dh = oracle.mx4_entries_as_bf16(hca[h0:h0 + n_h]) if n_h else hca[h0:h0 + 1]
+            O_c, l_c = oracle.csa_attn(qh[0], dc, idx[b].cpu().numpy(), d.m, x[t0:t0 + L], L, d.W, sh.scale)
+            O_h, l_h = oracle.hca_attn(qh[0], dh, d.m_hca, x[t0:t0 + L], L, 0, sh.scale)
+            O, _ = oracle.lse_merge(O_c, l_c, O_h, l_h)
+            gh.check_close(out[b].cpu().numpy(), O, f"fp4 decode step {s} seq {b}")
+
+
 # --------------------------------------------------------------------------------- f2: index reuse
 
 def _oracle_on_gpu_caches(layer, b, L, qh, idx_b, d):
