@@ -314,13 +314,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             } else {
                 // FP4 entries: chunk c of a row (channels 8c .. 8c+7) is the 4 code bytes at 4c and the
                 // scale byte c/4; dequantized in registers and stored into the tile's swizzled slot.
-                // Four rows at a time, their loads issued unconditionally (a row that is not FP4 loads
-                // from the query instead and goes by cp.async), then converted.
+                // The loads of all 16 rows are issued first, unconditionally (a row that is not FP4
+                // loads from the query instead and goes by cp.async), so the tile costs one memory
+                // latency; then the rows are converted.
+                constexpr int kFp4Rows = 16;
 #pragma unroll 1
-                for (int r0 = 0; r0 < 16; r0 += 4) {
-                    uint32_t cw[4][CPL], sb[4][CPL];
+                for (int r0 = 0; r0 < 16; r0 += kFp4Rows) {
+                    uint32_t cw[kFp4Rows][CPL], sb[kFp4Rows][CPL];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < kFp4Rows; ++i) {
                         const uint8_t* sc = reinterpret_cast<const uint8_t*>(rowscl[r0 + i]);
                         const uint8_t* cr = sc ? reinterpret_cast<const uint8_t*>(rowptr[r0 + i])
                                                : reinterpret_cast<const uint8_t*>(p.q);
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                         }
                     }
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < kFp4Rows; ++i) {
                         const int r = r0 + i;
                         if (rowscl[r] == 0) {
                             copy_row(r);

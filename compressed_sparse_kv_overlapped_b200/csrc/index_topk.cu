@@ -106,6 +106,12 @@ __device__ __forceinline__ uint2 ld_stream8(const void* p, uint64_t pol) {
     return v;
 }
 
+// x * 2^e, correctly rounded (the same value as ldexpf): a multiply by the power of two built from
+// its exponent bits when 2^e is a normal float, else ldexpf itself.
+__device__ __forceinline__ float scale_pow2(float x, int e) {
+    return (e >= -126 && e <= 127) ? __fmul_rn(x, __uint_as_float((uint32_t)(e + 127) << 23)) : ldexpf(x, e);
+}
+
 // Two E4M3 values (low byte first) to two f16 values (exact: every E4M3 value is an f16 value).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
     uint32_t r;
@@ -147,10 +153,10 @@ __device__ __forceinline__ void score16_mx8(const uint8_t* keys, const uint8_t* 
         mma_f16_16816(acc, a0, bq[2 * b]);
         mma_f16_16816(acc, a1, bq[2 * b + 1]);
         const int el = (int)((sl >> (8 * b)) & 0xFFu) - 127, eh = (int)((sh >> (8 * b)) & 0xFFu) - 127;
-        tot[0] = __fadd_rn(tot[0], ldexpf(acc[0], el - qsh[0]));
-        tot[1] = __fadd_rn(tot[1], ldexpf(acc[1], el - qsh[1]));
-        tot[2] = __fadd_rn(tot[2], ldexpf(acc[2], eh - qsh[0]));
-        tot[3] = __fadd_rn(tot[3], ldexpf(acc[3], eh - qsh[1]));
+        tot[0] = __fadd_rn(tot[0], scale_pow2(acc[0], el - qsh[0]));
+        tot[1] = __fadd_rn(tot[1], scale_pow2(acc[1], el - qsh[1]));
+        tot[2] = __fadd_rn(tot[2], scale_pow2(acc[2], eh - qsh[0]));
+        tot[3] = __fadd_rn(tot[3], scale_pow2(acc[3], eh - qsh[1]));
     }
     float pl = wv[0] * fmaxf(tot[0], 0.f) + wv[1] * fmaxf(tot[1], 0.f);
     float ph = wv[0] * fmaxf(tot[2], 0.f) + wv[1] * fmaxf(tot[3], 0.f);
