@@ -263,8 +263,31 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
         }
     }
     float hv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (h_do) {  // uniform over the CTA (the block form has barriers)
-        if (hca_block_shape(p.m_hca)) {
+    // m' >= 16: the 16-tokens-per-warp form (warp 0 ends with the entry, two channels per lane);
+    // m' = 4, 8: the 4-token block form (threads 0..7 end with it, eight channels each)
+    const bool h16 = p.m_hca >= 16 && hca_block_shape(p.m_hca);
+    if (h_do) {  // uniform over the CTA (both forms have barriers)
+        if (h16) {
+            const int w16 = tid >> 5, lane = tid & 31, wpe = p.m_hca / 16;
+            const int cp = c0s + 2 * lane;
+            Part2 H2;
+            if (w16 < wpe) {
+                const int64_t row0 = sq.tok_off + (int64_t)p.m_hca * h + 16 * w16;
+                auto fetch = [&](int tensor, int t) -> uint32_t {
+                    const uint16_t* base = tensor == 0 ? p.logit_h : p.x;
+                    return __ldcg(reinterpret_cast<const unsigned int*>(base + (row0 + t) * d + cp));
+                };
+                auto bias2 = [&](int t) -> float2 {
+                    return __ldg(reinterpret_cast<const float2*>(p.bias_h + (int64_t)(16 * w16 + t) * d + cp));
+                };
+                hca_part16(fetch, bias2, H2);
+            } else {
+                H2 = Part2{{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+            }
+            hca_merge_warps(H2, wpe, xs);
+            hv[0] = entry_div(H2.acc[0], H2.den[0]);
+            hv[1] = entry_div(H2.acc[1], H2.den[1]);
+        } else if (hca_block_shape(p.m_hca)) {
             const int nb = p.m_hca / 4, u = tid >> 3, g = tid & 7, ub = u & (nb - 1);
             const int c0 = c0s + 8 * g;
             const int64_t row0 = sq.tok_off + (int64_t)p.m_hca * h + 4 * ub;
@@ -290,20 +313,23 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
         // entry normalization (block forms only): partial sums of squares of this CTA's 64 channels,
         // then the totals over the cluster's slices, in the same order as the full pass
         if (tid < 32) {
-            const float sc = sum_lane8(sumsq8(cv)), sh = sum_lane8(sumsq8(hv));
+            const float sc = sum_lane8(sumsq8(cv));
+            const float sh = h16 ? warp_sum(__fmaf_rn(hv[1], hv[1], __fmaf_rn(hv[0], hv[0], 0.f)))
+                                 : sum_lane8(sumsq8(hv));
             if (tid == 0) { ss[0] = sc; ss[1] = sh; }
         }
         cluster_barrier();
-        if (tid < 8) {
+        if (tid < 32) {
             if (c_do && p.norm_c) inv_c = rms_inv(cluster_sum(&ss[0], ns), d, p.eps);
             if (h_do && p.norm_h) inv_h = rms_inv(cluster_sum(&ss[1], ns), d, p.eps);
         }
     }
-    if (tid < 8) {
-        // the entries (and their FP4 copies: four lanes per 32-channel block)
-        const int c0 = c0s + 8 * tid;
-        const unsigned qmask = 0xFu << (tid & ~3);
-        if (c_do && csa_block_shape(p.m)) {
+    if (tid < 32) {
+        // the entries (and their FP4 copies: threads 0..7 with eight channels each, four lanes per
+        // 32-channel block)
+        const int c0 = c0s + 8 * (tid & 7);
+        const unsigned qmask = 0xFu << (tid & 4);
+        if (c_do && csa_block_shape(p.m) && tid < 8) {
             const int64_t row = sq.csa_off + j;
             const uint4 e = entry_bf16(cv, p.norm_c ? p.norm_c + c0 : nullptr, inv_c);
             *reinterpret_cast<uint4*>(p.entries + row * d + c0) = e;
@@ -315,9 +341,19 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
         }
         if (h_do && hca_block_shape(p.m_hca)) {
             const int64_t row = sq.hca_off + h;
-            const uint4 e = entry_bf16(hv, p.norm_h ? p.norm_h + c0 : nullptr, inv_h);
-            *reinterpret_cast<uint4*>(p.hca_entries + row * d + c0) = e;
-            if (p.hca_q) {
+            uint4 e;
+            if (h16) {
+                const int cp = c0s + 2 * tid;
+                const uint32_t hw = entry_bf16x2(hv[0], hv[1], p.norm_h ? p.norm_h + cp : nullptr, inv_h);
+                *reinterpret_cast<uint32_t*>(p.hca_entries + row * d + cp) = hw;
+                const int src = 4 * (tid & 7);  // the eight channels of thread t are lanes 4t .. 4t+3
+                e = make_uint4(__shfl_sync(0xffffffffu, hw, src), __shfl_sync(0xffffffffu, hw, src + 1),
+                               __shfl_sync(0xffffffffu, hw, src + 2), __shfl_sync(0xffffffffu, hw, src + 3));
+            } else {
+                e = entry_bf16(hv, p.norm_h ? p.norm_h + c0 : nullptr, inv_h);
+                if (tid < 8) *reinterpret_cast<uint4*>(p.hca_entries + row * d + c0) = e;
+            }
+            if (p.hca_q && tid < 8) {
                 uint32_t sb;
                 *reinterpret_cast<uint32_t*>(p.hca_q + row * (d / 2) + c0 / 2) = quant_mx4(e, qmask, &sb);
                 if ((tid & 3) == 0) p.hca_s[row * (d / 32) + c0 / 32] = (uint8_t)sb;

@@ -72,7 +72,7 @@ struct TileSmem {
     static constexpr int kAlloc = kTotal + 128;       // slack for 128-byte alignment
 };
 
-__global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_constant__ TileMaps maps,
+__global__ void __launch_bounds__(256, 3) compress_tile_kernel(const __grid_constant__ TileMaps maps,
                                                                 TileCompressParams p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
@@ -169,10 +169,33 @@ __global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_cons
             csa_entry_block4<false>(j, d, p.bias_c + c0, fetch, cv, nullptr);
         }
     }
+    // HCA: m' >= 16 in the 16-tokens-per-warp form (lane = channel pair); m' = 4, 8 in the 4-token
+    // block form (the block tree)
+    const bool h16 = mh >= 16;
     float hv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    Part2 H2;
     bool h_mine = false;
     int64_t h = 0;
-    if (hca) {
+    if (hca && h16) {
+        const int w16 = tid >> 5;
+        int r = (int)(tt0 + 16 * w16 - box0);  // smem row of the warp's first token
+        if (r < 0 || r + 16 > kBoxRows) r = 0;  // tokens past the loaded rows belong to no entry written here
+        const int cp = slice * kSlice + 2 * lane;
+        auto fetch = [&](int tensor, int t) -> uint32_t {
+            const uint16_t* base = tensor == 0 ? slh : sx;
+            return *reinterpret_cast<const uint32_t*>(base + (r + t) * kSlice + 2 * lane);
+        };
+        const int brow0 = (16 * w16) & (mh - 1);
+        auto bias2 = [&](int t) -> float2 {
+            return __ldg(reinterpret_cast<const float2*>(p.bias_h + (int64_t)(brow0 + t) * d + cp));
+        };
+        hca_part16(fetch, bias2, H2);
+        hca_merge_warps(H2, mh / 16, xs);
+        h = (tt0 + 16 * w16) / mh;
+        h_mine = loaded && (w16 % (mh / 16)) == 0 && h >= h_lo && h < h_hi;
+        hv[0] = entry_div(H2.acc[0], H2.den[0]);
+        hv[1] = entry_div(H2.acc[1], H2.den[1]);
+    } else if (hca) {
         const int nb = mh / 4;  // blocks per HCA entry
         // block u's 4 tokens; blocks past the loaded rows belong to no entry this tile writes
         int r = (int)(tt0 + 4 * u - box0);
@@ -198,11 +221,9 @@ __global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_cons
         // partial sums of squares over this CTA's 64 channels, one per entry of the tile, then the
         // totals over the cluster's slices
         const float sc = sum_lane8(sumsq8(cv));
-        const float sh = sum_lane8(sumsq8(hv));
-        if (g == 0) {
-            ss_c[u] = sc;
-            if (h_mine) ss_h[h - tt0 / mh] = sh;
-        }
+        const float sh = h16 ? warp_sum(__fmaf_rn(hv[1], hv[1], __fmaf_rn(hv[0], hv[0], 0.f))) : sum_lane8(sumsq8(hv));
+        if (g == 0) ss_c[u] = sc;
+        if (h_mine && (h16 ? lane == 0 : g == 0)) ss_h[h - tt0 / mh] = sh;
         cluster_barrier();
         const int ns = (int)gridDim.z;
         if (c_mine && p.norm_c) inv_c = rms_inv(cluster_sum(ss_c + u, ns), d, p.eps);
@@ -211,8 +232,16 @@ __global__ void __launch_bounds__(256, 2) compress_tile_kernel(const __grid_cons
     }
     if (c_mine)
         *reinterpret_cast<uint4*>(p.entries + (sq.csa_off + j) * d + c0) = entry_bf16(cv, p.norm_c ? p.norm_c + c0 : nullptr, inv_c);
-    if (h_mine)
-        *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) = entry_bf16(hv, p.norm_h ? p.norm_h + c0 : nullptr, inv_h);
+    if (h_mine) {
+        if (h16) {
+            const int cp = slice * kSlice + 2 * lane;
+            *reinterpret_cast<uint32_t*>(p.hca_entries + (sq.hca_off + h) * d + cp) =
+                entry_bf16x2(hv[0], hv[1], p.norm_h ? p.norm_h + cp : nullptr, inv_h);
+        } else {
+            *reinterpret_cast<uint4*>(p.hca_entries + (sq.hca_off + h) * d + c0) =
+                entry_bf16(hv, p.norm_h ? p.norm_h + c0 : nullptr, inv_h);
+        }
+    }
 }
 
 }  // namespace

@@ -317,4 +317,112 @@ __device__ __forceinline__ void hca_tree(Part8& P, int nb, float* xs) {
     }
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// HCA entries for m' a power of two from 16 to 128: warp w of the 256-thread CTA takes 16
+// consecutive tokens of the entry (tokens 16w .. 16w+15 of a tile, or of the entry at decode), lane l
+// the channel pair (2l, 2l+1) of the CTA's 64-channel slice.  Each lane forms the 16-token partial of
+// its two channels; the m'/16 partials of an entry are merged in shared memory in a fixed balanced
+// tree (warp order), with the same explicitly rounded steps as the 4-token form, so the full pass and
+// the decode append produce identical entries.
+// ---------------------------------------------------------------------------------------------
+struct Part2 {
+    float M[2], den[2], acc[2];
+};
+
+// Partial of 16 tokens: fetch(0, t) / fetch(1, t) give token t's logit / latent pair (two bf16 in a
+// word, the even channel low), bias2(t) its bias row's pair.
+template <typename Fetch, typename Bias>
+__device__ __forceinline__ void hca_part16(Fetch fetch, Bias bias2, Part2& P) {
+    float z[16][2];
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const uint32_t l = fetch(0, t);
+        const float2 b = bias2(t);
+        z[t][0] = __fadd_rn(bf16lo(l), b.x);
+        z[t][1] = __fadd_rn(bf16hi(l), b.y);
+        mx0 = fmaxf(mx0, z[t][0]);
+        mx1 = fmaxf(mx1, z[t][1]);
+    }
+    P.M[0] = __fmul_rn(mx0, kLog2e);
+    P.M[1] = __fmul_rn(mx1, kLog2e);
+    const float n0 = -P.M[0], n1 = -P.M[1];
+    float d0 = 0.f, d1 = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const uint32_t x = fetch(1, t);
+        const float e0 = fast_exp2(__fmaf_rn(z[t][0], kLog2e, n0));
+        const float e1 = fast_exp2(__fmaf_rn(z[t][1], kLog2e, n1));
+        d0 = __fadd_rn(d0, e0);
+        d1 = __fadd_rn(d1, e1);
+        a0 = __fmaf_rn(e0, bf16lo(x), a0);
+        a1 = __fmaf_rn(e1, bf16hi(x), a1);
+    }
+    P.den[0] = d0;
+    P.den[1] = d1;
+    P.acc[0] = a0;
+    P.acc[1] = a1;
+}
+
+// A <- merge(A, B); symmetric in A and B bit for bit (as merge8).
+__device__ __forceinline__ void merge2(Part2& A, const Part2& B) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float M = fmaxf(A.M[i], B.M[i]);
+        const float fa = fast_exp2(__fsub_rn(A.M[i], M));
+        const float fb = fast_exp2(__fsub_rn(B.M[i], M));
+        A.den[i] = __fadd_rn(__fmul_rn(fa, A.den[i]), __fmul_rn(fb, B.den[i]));
+        A.acc[i] = __fadd_rn(__fmul_rn(fa, A.acc[i]), __fmul_rn(fb, B.acc[i]));
+        A.M[i] = M;
+    }
+}
+
+// Merge the partials of the wpe (1, 2, 4 or 8) consecutive warps of each entry: every warp stores
+// its partial in xs ([8 warps][32 lanes][6 floats]), one barrier, then the first warp of each entry
+// merges them pairwise by levels (warps 2i and 2i+1, then the pairs, ...).  Every thread of the CTA
+// must call it when wpe > 1.  On return the first warp of each entry holds the merged partial in P.
+__device__ __forceinline__ void hca_merge_warps(Part2& P, int wpe, float* xs) {
+    if (wpe <= 1) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float* mine = xs + (warp * 32 + lane) * 6;
+    mine[0] = P.M[0]; mine[1] = P.M[1]; mine[2] = P.den[0]; mine[3] = P.den[1]; mine[4] = P.acc[0]; mine[5] = P.acc[1];
+    __syncthreads();
+    if (warp % wpe == 0) {
+        Part2 L[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k < wpe) {
+                const float* o = xs + ((warp + k) * 32 + lane) * 6;
+                L[k].M[0] = o[0]; L[k].M[1] = o[1]; L[k].den[0] = o[2]; L[k].den[1] = o[3];
+                L[k].acc[0] = o[4]; L[k].acc[1] = o[5];
+            }
+        }
+#pragma unroll
+        for (int step = 1; step < 8; step *= 2)
+#pragma unroll
+            for (int k = 0; k < 8; k += 2 * step)
+                if (step < wpe && k + step < wpe) merge2(L[k], L[k + step]);
+        P = L[0];
+    }
+}
+
+// Sum over the 32 lanes of a warp (every lane ends with the same bits).
+__device__ __forceinline__ float warp_sum(float s) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+    return s;
+}
+
+// Two entry values to a bf16 pair, normalized by inv * gain[c], gain[c + 1] when gain is given (the
+// same rounding steps as entry_bf16).
+__device__ __forceinline__ uint32_t entry_bf16x2(float v0, float v1, const float* gain_c, float inv) {
+    if (gain_c) {
+        const float2 g = __ldg(reinterpret_cast<const float2*>(gain_c));
+        v0 = __fmul_rn(__fmul_rn(v0, inv), g.x);
+        v1 = __fmul_rn(__fmul_rn(v1, inv), g.y);
+    }
+    return pack_bf16x2(v0, v1);
+}
+
 }  // namespace csa
