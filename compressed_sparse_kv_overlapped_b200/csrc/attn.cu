@@ -462,28 +462,44 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 inv0 = rsqrtf(ss0 / D + p.norm_eps);
                 inv1 = rsqrtf(ss1 / D + p.norm_eps);
             }
-            // dims 2col .. 2col + 3 of a row, normalized and rounded back to bf16 when a gain is given
-            auto qload = [&](const uint2* row, bool valid, float inv, int col) -> uint2 {
-                uint2 v = valid ? row[col / 2] : make_uint2(0, 0);
-                if (p.q_norm && valid) {
-                    const float4 gn = *reinterpret_cast<const float4*>(p.q_norm + 2 * col);
-                    v.x = pack_bf16x2(bf16lo(v.x) * inv * gn.x, bf16hi(v.x) * inv * gn.y);
-                    v.y = pack_bf16x2(bf16lo(v.y) * inv * gn.z, bf16hi(v.y) * inv * gn.w);
-                }
-                return v;
+            const bool ok0 = h0 < p.H, ok1 = h1 < p.H;
+            // dims 2col .. 2col + 3 of a row, normalized and rounded back to bf16 (gain p.q_norm)
+            auto qnorm = [&](uint32_t& x, uint32_t& y, float inv, int col) {
+                const float4 gn = *reinterpret_cast<const float4*>(p.q_norm + 2 * col);
+                x = pack_bf16x2(bf16lo(x) * inv * gn.x, bf16hi(x) * inv * gn.y);
+                y = pack_bf16x2(bf16lo(y) * inv * gn.z, bf16hi(y) * inv * gn.w);
             };
 #pragma unroll 1
             for (int cb = 0; cb < D / 2; cb += 128) {
                 uint32_t r[2][32];
+                // every load of the pass first, unconditionally (a column past the row reads column
+                // qc), so they are all in flight together; then the optional normalization and the
+                // zeros of heads past H by selects on the loaded registers
 #pragma unroll
                 for (int g = 0; g < 2; ++g) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
-                        const int col = cb + g * 64 + 8 * k + qc;  // a column holds 2 dims: uint2 index col / 2
                         const bool in = cb + g * 64 < D / 2;
-                        const uint2 v0 = qload(q0, in && h0 < p.H, inv0, col);
-                        const uint2 v1 = qload(q1, in && h1 < p.H, inv1, col);
+                        const int col = in ? cb + g * 64 + 8 * k + qc : qc;  // a column holds 2 dims
+                        const uint2 v0 = q0[col / 2], v1 = q1[col / 2];
                         r[g][4 * k] = v0.x; r[g][4 * k + 1] = v0.y; r[g][4 * k + 2] = v1.x; r[g][4 * k + 3] = v1.y;
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const bool in = cb + g * 64 < D / 2;
+                        const int col = in ? cb + g * 64 + 8 * k + qc : qc;
+                        if (p.q_norm) {
+                            qnorm(r[g][4 * k], r[g][4 * k + 1], inv0, col);
+                            qnorm(r[g][4 * k + 2], r[g][4 * k + 3], inv1, col);
+                        }
+                        const bool u0 = in && ok0, u1 = in && ok1;
+                        r[g][4 * k] = u0 ? r[g][4 * k] : 0u;
+                        r[g][4 * k + 1] = u0 ? r[g][4 * k + 1] : 0u;
+                        r[g][4 * k + 2] = u1 ? r[g][4 * k + 2] : 0u;
+                        r[g][4 * k + 3] = u1 ? r[g][4 * k + 3] : 0u;
                     }
                 }
 #pragma unroll
