@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const bool direct = n_items == 1;
     const bool clustered = !direct && p.cluster > 1;
     const bool dep_wait = !(p.hca_nowait && !direct && item >= p.items_front);
+    // front items with a ready word: the loaders poll it, nobody waits for the select grid up front
+    const bool ready_wait = dep_wait && p.ready != nullptr && !direct;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -236,7 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         constexpr int CPL = CPR / 32 > 0 ? CPR / 32 : 1;  // chunks per lane per row (2 at D = 512)
         const uint32_t lane_blk = (uint32_t)(lane >> 3) * L::kBlock;  // block of chunk `lane`
         const uint32_t lane_c7 = (uint32_t)(lane & 7);
-        if (dep_wait) grid_dep_wait();  // the selected indices come from the previous kernel
+        // the selected indices come from the previous kernel: its ready word for this query, or the
+        // end of its grid
+        bool go = true;
+        if (ready_wait) {
+            if (lane == 0) go = count_wait(p.ready + qi, 1u, p.status, abort_flag, p.wait_ns);
+            __syncwarp();  // orders the other lanes' reads after lane 0's acquire
+            go = __shfl_sync(0xffffffffu, go ? 1 : 0, 0) != 0;
+        } else if (dep_wait) {
+            grid_dep_wait();
+        }
         if (lw == 0 && lane == 0) {
             if (p.tma_hca) tma_prefetch_map(&maps.hca);
             if (p.tma_x) tma_prefetch_map(&maps.x);
@@ -244,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // per stage, the full-barrier parity of the last tile this thread loaded by TMA (bit 2 set:
         // one is pending), so that a CTA that gives up waits for its own copies before it exits
         uint32_t tma_pend = 0;
-        for (int t = 0; t < T; ++t) {
+        for (int t = 0; go && t < T; ++t) {
             const int st = t % kStages;
             if (t >= kStages && !mbar_wait(&bars->empty[st], ((t / kStages) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
             const int64_t tb = s0 + (int64_t)t * kTileKeys;
@@ -311,6 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             if (!tile_fp4) {
 #pragma unroll 4
                 for (int r = 0; r < 16; ++r) copy_row(r);
+                // the copies complete the tile's barrier phase themselves: no wait here, so the next
+                // tile's loads go out while these are still in flight
+                if (!skip) cp_async_mbar_arrive(&bars->full[st]);
             } else {
                 // FP4 entries: chunk c of a row (channels 8c .. 8c+7) is the 4 code bytes at 4c and the
                 // scale byte c/4; dequantized in registers and stored into the tile's swizzled slot.
@@ -348,9 +362,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                             if (lane + 32 * u < CPR) st_shared_v4(dst + u * 4 * L::kBlock, mx4_to_bf16x8(cw[i][u], sb[i][u]));
                     }
                 }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
             }
-            cp_async_wait_all();
-            fence_proxy_async_smem();
             if (lane == 0) mask16[st * 4 + lw] = (uint16_t)vm;
             __syncwarp();
             if (!skip) mbar_arrive(&bars->full[st]);
@@ -370,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // tile read MN-major as V): the two products of neighbouring tiles reach the tensor pipe
         // independently, so a P.V never waits behind the issue of the next Q.K^T.  Each warp runs
         // its loop with all lanes (warp-uniform waits and operands; one elected lane issues).
-        if (dep_wait) grid_dep_wait();
+        if (dep_wait && !ready_wait) grid_dep_wait();
         if (T > 0) {
             if (warp == 8) {
                 constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
@@ -381,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                     if (w && g1 >= 2) w = mbar_wait(&bars->s_free[g1 & 1], ((g1 >> 1) - 1) & 1, p.status, abort_flag, p.wait_ns);
                     if (!__all_sync(0xffffffffu, w)) break;
                     tc_fence_after();
+                    fence_proxy_async_smem();  // the tile's cp.async writes, observed through the barrier
                     const uint64_t kd = sdesc_kmajor(sbase + L::kK + (uint32_t)st * L::kStage);
                     const uint32_t tS = tmem + kColS + (uint32_t)(g1 & 1) * 64u;
 #pragma unroll
@@ -510,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             tc_fence_before();
             mbar_arrive(&bars->q_full);
         }
-        if (dep_wait) grid_dep_wait();
+        if (dep_wait && !ready_wait) grid_dep_wait();
         grid_dep_launch();
         const int i = lane;
         // S and O are read with the 16x256b shape, so all 32 lanes work: lane i holds rows ra = i/4
@@ -711,6 +726,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                     if (hr[rr] >= p.H) reinterpret_cast<float*>(sm + L::kP0)[hr[rr]] = -INFINITY;
         }
     }
+    // the select grid is complete before this one is (the merge that waits for this grid relies on it)
+    if (ready_wait) grid_dep_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == 8 && T > 0) {
@@ -778,6 +795,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 p.part_lse[((int64_t)qi * n_parts + part) * kHeadsPad + h] = mlse[h];
         cluster_barrier();  // no CTA leaves while another still reads its shared memory
     }
+    if (p.items_done && !direct) {
+        __syncthreads();  // every partial store of the CTA precedes the count
+        if (threadIdx.x == 0) {
+            __threadfence();
+            atomicAdd(p.items_done + qi, 1u);
+        }
+    }
 }
 
 // out[q][h] = sum_items exp(lse_i - lse) * O_i,  lse = logsumexp_i lse_i  (items with lse = -inf
@@ -786,14 +810,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 // partials with batched loads.
 template <int D, int SPLIT>
 __global__ void combine_kernel(AttnParams p) {
-    constexpr int kMaxBatch = 24;  // partial rows held in registers per pass
-    grid_dep_wait();  // the partials come from the attention grid
+    constexpr int kMaxBatch = 32;  // partial rows held in registers per pass
     const int h = blockIdx.x, qi = blockIdx.y;
     const int n_items = p.cluster > 1 ? p.n_items / p.cluster : p.n_items;  // partials per query
     const int lane = threadIdx.x & 31;
     __shared__ float s_lse[256];
     __shared__ float s_w[256];
     __shared__ float s_res[2];
+    __shared__ int s_go;
+    // the partials come from the attention grid: this query's item counter, or the end of the grid
+    if (p.items_done) {
+        if (threadIdx.x == 0) s_go = count_wait(p.items_done + qi, (uint32_t)p.n_items, p.status, nullptr, p.wait_ns);
+        __syncthreads();  // orders every thread's reads after thread 0's acquire
+        if (!s_go) {
+            grid_dep_wait();
+            return;
+        }
+    } else {
+        grid_dep_wait();
+    }
     // every thread owns one float4 column of the output row (D / 4 / SPLIT threads)
     const int c = (int)blockIdx.z * (D / SPLIT) + threadIdx.x * 4;
     const float* base = p.part_o + ((int64_t)qi * n_items * kHeadsPad + h) * D + c;

@@ -453,7 +453,8 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
               int64_t e_stride, const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
               float* score_out, void* ws_index, bool zero_ws, int* status, cudaStream_t stream,
               cudaEvent_t mid = nullptr, bool pdl = false, const void* prefetch_entries = nullptr,
-              int64_t prefetch_row_bytes = 0, const uint8_t* keys_q = nullptr, const uint8_t* key_scales = nullptr) {
+              int64_t prefetch_row_bytes = 0, const uint8_t* keys_q = nullptr, const uint8_t* key_scales = nullptr,
+              uint32_t* ready = nullptr) {
     IndexParams ip{};
     ip.seqs = seqs;
     ip.queries = queries;
@@ -474,6 +475,7 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
     ip.prefetch_rows = reinterpret_cast<const unsigned char*>(prefetch_entries);
     ip.prefetch_row_bytes = prefetch_row_bytes;
     index_ws_carve(ip, ws_index, Q, e_stride);
+    ip.ready = ready;
     cudaError_t e = launch_index_topk(ip, max_e, stream, zero_ws, mid, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "index_topk launch");
     return CSA_OK;
@@ -1028,7 +1030,7 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
         ap.eps = a->norms->eps;
     }
     ap.queries = queries;
-    ap.zero_words = static_cast<uint32_t*>(ws_index);  // histograms + counters of the index scratch
+    ap.zero_words = static_cast<uint32_t*>(ws_index);  // histograms + ready words of the index scratch
     ap.n_zero_words = (int64_t)(index_zero_bytes(a->B) / 4);
     ap.status = st;
     cudaEvent_t ev[CSA_DECODE_MARKS] = {};
@@ -1056,11 +1058,17 @@ int hybrid_attn_decode(const csa_decode_args* a, void* ws, size_t ws_bytes, csa_
     ap2.queries_early = reuse ? 0 : 1;  // the append is two launches back only with the indexer between
     ap2.hca_first = (pl.items.n_items > 1 && pl.items.items_front > 0) ? 1 : 0;
     ap2.cluster = pl.cluster;
+    // per-step words cleared by the append: the front items start on their query's ready word from
+    // the select, and the merge of a query on its item counter, not on the end of the previous grid
+    uint32_t* step_words = index_ready_words(ws_index, a->B);
+    uint32_t* ready = reuse ? nullptr : step_words;
+    ap2.ready = pl.items.n_items > 1 ? ready : nullptr;
+    ap2.items_done = pl.items.n_items > 1 ? step_words + a->B : nullptr;
     if (!reuse) {
         rc = run_index(d, a->seqs, queries, a->B, pl.max_e, pl.e_stride, a->q_idx, a->w, a->entry_keys, idx, nullptr,
                        ws_index, false, st, stream, ev[2], pdl,
                        fp4 ? static_cast<const void*>(a->entries_q) : static_cast<const void*>(a->entries),
-                       fp4 ? (int64_t)d.d / 2 : (int64_t)d.d * 2, a->keys_q, a->key_scales);
+                       fp4 ? (int64_t)d.d / 2 : (int64_t)d.d * 2, a->keys_q, a->key_scales, ready);
         if (rc) return rc;
     } else if ((e = mark(ev[2], stream)) != cudaSuccess) {
         return cuda_fail(e, "event record");

@@ -143,6 +143,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// One more pending arrival on `bar`, resolved when every cp.async this thread has issued so far has
+// completed; it does not count toward the expected arrivals, so the thread still arrives itself.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // 16-byte store to shared memory (a shared-window address).
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
@@ -302,6 +308,37 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 // allow the next grid to start its prologue.  Both are no-ops for a normally launched grid.
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// A flag word between two grids that run at the same time (a producer and the grid it launched
+// early): the producer publishes with a release store after its results, the consumer polls with
+// acquire loads, after which the producer's results are visible to it.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait for *word >= target, same contract as mbar_wait.  Polls with a short sleep between
+// reads, so that many waiting warps leave the memory system to the grid they wait for.
+__device__ __forceinline__ bool count_wait(const uint32_t* word, uint32_t target, int* status, volatile int* abort,
+                                           uint64_t limit_ns = kWaitLimitNs) {
+    if (ld_acquire_gpu(word) >= target) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(32);
+        if (ld_acquire_gpu(word) >= target) return true;
+        if ((it & 15u) == 0u) {
+            if (abort && *abort) return false;
+            if (globaltimer() - t0 > limit_ns) {
+                report(status, CSA_ERR_TIMEOUT);
+                if (abort) *abort = 1;
+                return false;
+            }
+        }
+    }
+}
 
 // 2^x with the hardware approximation (relative error about 2^-22; subnormal results flush to 0).
 __device__ __forceinline__ float fast_exp2(float x) {

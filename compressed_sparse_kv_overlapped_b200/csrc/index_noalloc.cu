@@ -25,7 +25,7 @@ constexpr int64_t kNoAllocMaxSlots = int64_t(1) << 20;  // Q * score-row stride
 // row plus 128 entries); two words per scan chunk (chunks of at least 256 entries, nine more per
 // query: a partial chunk and the ends of the final select's per-CTA prefixes); candidate keys (a
 // quarter of the entries plus 256 per query).
-constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * kHistBins * 4 + 256 +         // histograms
+constexpr size_t kScratchBytes = size_t(kNoAllocMaxQ) * kKeyBins * 4 + 256 +          // histograms, step words
                                  size_t(kNoAllocMaxSlots) * 4 + 256 +                  // scores
                                  size_t(kNoAllocMaxSlots + kNoAllocMaxQ * kSegPad) * 8 + 256 +
                                  2 * (size_t(kNoAllocMaxSlots / 256 + 9 * kNoAllocMaxQ) * 4 + 256) +

@@ -14,8 +14,8 @@
 //            indexer-key cache with coalesced 16-byte loads and computes the [16 entries x d_I] .
 //            [d_I x H_I] products on the tensor cores (mma.sync m16n8k16, K permuted so that every
 //            thread's operand is one contiguous 16-byte load), applies relu / head weights in
-//            registers, and counts the scores into the query's histogram of the top 11 key bits.
-//            Each chunk keeps its local candidates.
+//            registers, and counts the scores into the query's histogram of the top kKeyBits key
+//            bits.  Each chunk keeps its local candidates.
 //  index_final_kernel  -- one thread-block cluster per query after the scan: the exact top-k from
 //            the chunks' candidates (see the kernel).
 //  index_select_kernel -- one CTA per query, the prefill path: the top-k of a score row that the
@@ -204,14 +204,14 @@ __device__ __forceinline__ uint32_t excl_scan(uint32_t v, uint32_t* wsum, uint32
     return before + incl - v;
 }
 
-// Over kHistBins bins: the unique bin b with suffix(b) >= target > suffix(b + 1), where suffix(b) =
+// Over BINS bins: the unique bin b with suffix(b) >= target > suffix(b + 1), where suffix(b) =
 // sum of hist[b' >= b] (target >= 1).  out[0] = b (0xFFFFFFFF if the total is below target),
-// out[1] = suffix(b + 1), out[2] = suffix(b).  Thread t owns kHistBins/NT consecutive bins counted
+// out[1] = suffix(b + 1), out[2] = suffix(b).  Thread t owns BINS/NT consecutive bins counted
 // from the top, so a forward scan over threads is a suffix scan over bins; it reads them with
 // 16-byte loads (hist 16-byte aligned; a quarter-warp's loads cover all banks once).
-template <int NT>
+template <int NT, int BINS = kHistBins>
 __device__ void find_bin(const uint32_t* hist, uint32_t target, uint32_t* wsum, uint32_t* out) {
-    constexpr int PER = kHistBins / NT;
+    constexpr int PER = BINS / NT;
     static_assert(PER % 4 == 0, "find_bin reads its bins as 16-byte vectors");
     const int t = threadIdx.x;
     const int b0 = PER * (NT - 1 - t);  // bins [b0, b0 + PER)
@@ -245,27 +245,28 @@ struct KeyList {
     }
 };
 
-// The key T with exactly `need` of the list's members of bin top11 (top 11 bits) at or above it:
-// radix passes of 11 bits below the top 11, counted with shared-memory atomics in cnt[kHistBins];
-// stops as soon as the chosen digit holds exactly the remaining count.
-template <int NT>
-__device__ uint64_t radix_select(const KeyList& L, uint32_t n, uint32_t need, uint32_t top11, uint32_t* cnt,
+// The key T with exactly `need` of the list's members of bin `top` (their top BITS bits) at or above
+// it: radix passes of BITS bits below the top BITS, counted with shared-memory atomics in
+// cnt[1 << BITS]; stops as soon as the chosen digit holds exactly the remaining count.
+template <int NT, int BITS>
+__device__ uint64_t radix_select(const KeyList& L, uint32_t n, uint32_t need, uint32_t top, uint32_t* cnt,
                                  uint32_t* wsum, uint32_t* res) {
-    uint64_t prefix = (uint64_t)top11 << 53;
-    uint64_t mask = (uint64_t)0x7FF << 53;
+    constexpr int kBins = 1 << BITS;
+    uint64_t prefix = (uint64_t)top << (64 - BITS);
+    uint64_t mask = (uint64_t)(kBins - 1) << (64 - BITS);
     uint32_t remaining = need;
-    for (int shift = 42;; shift -= 11) {
+    for (int shift = 64 - 2 * BITS;; shift -= BITS) {
         const int sh = shift < 0 ? 0 : shift;
-        const int bits = shift < 0 ? 11 + shift : 11;
+        const int bits = shift < 0 ? BITS + shift : BITS;
         const uint32_t dmask = (1u << bits) - 1u;
-        for (int i = threadIdx.x; i < kHistBins; i += NT) cnt[i] = 0;
+        for (int i = threadIdx.x; i < kBins; i += NT) cnt[i] = 0;
         __syncthreads();
         for (uint32_t i = threadIdx.x; i < n; i += NT) {
             const uint64_t v = L.get(i);
             if ((v & mask) == prefix) atomicAdd(&cnt[(uint32_t)(v >> sh) & dmask], 1u);
         }
         __syncthreads();
-        find_bin<NT>(cnt, remaining, wsum, res);
+        find_bin<NT, kBins>(cnt, remaining, wsum, res);
         const uint32_t dg = res[0], above = res[1], in_digit = res[2] - res[1];
         __syncthreads();
         remaining -= above;
@@ -325,7 +326,6 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(const void* p, uint32_t rank)
 constexpr int kListKeys = 4096;                  // keys of the final list held in shared memory
 constexpr int kTailPer = 8;                      // items per thread and round of an ordered compaction
 constexpr int kScanDynSmem = kListKeys * 8;      // dynamic shared memory: chunk scores, then the list
-static_assert(kScanDynSmem <= 48 * 1024, "no opt-in needed for the scan's dynamic shared memory");
 constexpr int64_t kScanChunkMax = kScanDynSmem / 4;
 static_assert(kScanChunkMax >= 512, "a chunk holds at least one pass of the scan");
 
@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     }
     const uint32_t need = (uint32_t)p.k - above;
     const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53)
-                                     : radix_select<kSelectThreads>(KL, n_cand, need, b1, hist, s_wsum, s_res);
+                                     : radix_select<kSelectThreads, 11>(KL, n_cand, need, b1, hist, s_wsum, s_res);
     // 5. compaction in index order
     const uint32_t per_t = (n_cand + kSelectThreads - 1) / kSelectThreads;
     const uint32_t j0 = tid * per_t, j1 = min(n_cand, j0 + per_t);
@@ -520,14 +520,15 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
 //
 // Scan CTA (chunk c, query qi): the scores of entries [c*chunk, min(E, (c+1)*chunk)) on the tensor
 // cores, written to the score row and kept in shared memory, counted into the query's histogram of
-// the top 11 bits of the order-preserving score key; then the chunk's candidates -- its entries of
-// bin >= b_c, b_c the highest bin that still leaves at least kloc entries (kloc about twice the
-// chunk's expected share of the top-k) -- go to the candidate buffer in index order, with b_c.
+// the top kKeyBits bits of the order-preserving score key; then the chunk's candidates -- its
+// entries of bin >= b_c, b_c the highest bin that still leaves at least kloc entries (kloc about
+// twice the chunk's expected share of the top-k) -- go to the candidate buffer in index order, with
+// b_c.
 // index_final_kernel selects the exact top-k from them.
 template <int KV, bool MX8>
 __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams p) {
     extern __shared__ __align__(16) unsigned char dsm[];
-    __shared__ __align__(16) uint32_t hist[kHistBins];
+    __shared__ __align__(16) uint32_t hist[kKeyBins];
     __shared__ float sc[kScanThreads / 32][4][16];
     __shared__ uint32_t s_wsum[kScanThreads / 32];
     __shared__ uint32_t s_res[4];
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
     if (cidx >= nch) return;
     const int64_t c0 = (int64_t)cidx * chunk;
     const int64_t c1 = min(E, c0 + chunk);
-    for (int i = tid; i < kHistBins; i += kScanThreads) hist[i] = 0u;
+    for (int i = tid; i < kKeyBins; i += kScanThreads) hist[i] = 0u;
 
     const int lane = tid & 31, warp = tid >> 5;
     {
@@ -651,7 +652,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
                         const float v = sc[warp][u][lane];
                         srow[r] = v;
                         ssc[r - c0] = v;
-                        atomicAdd(&hist[float_key(v) >> 21], 1u);
+                        atomicAdd(&hist[float_key(v) >> (32 - kKeyBits)], 1u);
                     }
                 }
             }
@@ -660,8 +661,8 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
     }
     __syncthreads();
     {
-        uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
-        for (int i = tid; i < kHistBins; i += kScanThreads)
+        uint32_t* gh = p.hist + (int64_t)qi * kKeyBins;
+        for (int i = tid; i < kKeyBins; i += kScanThreads)
             if (hist[i]) atomicAdd(&gh[i], hist[i]);
     }
     // ---- the chunk's candidates
@@ -669,7 +670,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
     const int cap = p.cand_cap;
     const int64_t kloc64 = (2 * (int64_t)p.k * n + E - 1) / E + 16;
     const uint32_t kloc = (uint32_t)min((int64_t)cap, min((int64_t)n, kloc64));
-    find_bin<kScanThreads>(hist, kloc, s_wsum, s_res);
+    find_bin<kScanThreads, kKeyBins>(hist, kloc, s_wsum, s_res);
     uint32_t bc = s_res[0] == 0xFFFFFFFFu ? 0u : s_res[0];
     if (s_res[0] != 0xFFFFFFFFu && s_res[2] > (uint32_t)cap) bc += 1;  // suffix(bc + 1) < kloc <= cap
     {
@@ -683,7 +684,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
             for (int u = 0; u < kTailPer; ++u) {
                 const int i = first + u * 32;
                 const uint32_t key = i < n ? float_key(ssc[i]) : 0u;
-                keep[u] = i < n && (key >> 21) >= bc;
+                keep[u] = i < n && (key >> (32 - kKeyBits)) >= bc;
                 v[u] = composite(key, c0 + i);
             }
             n_cand += compact_round<kScanThreads, kTailPer>(
@@ -708,11 +709,19 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
 constexpr int kFinalF = 8;           // CTAs per query
 constexpr int kFinalThreads = 256;
 constexpr int kFinalDynSmem = kListKeys * 8;  // the members list (also this CTA's chunk words)
-constexpr int kFinalChunks = (kHistBins - 2) / 2;  // chunks per CTA whose words fit the histogram's space
+constexpr int kFinalChunks = (kKeyBins - 2) / 2;  // chunks per CTA whose words fit the histogram's space
+
+// Query qi's indices are out: publish its ready word (one thread, after the stores it covers are
+// ordered before it: by a CTA barrier, or by the grid dependency for the scan's own results).
+__device__ __forceinline__ void signal_ready(const IndexParams& p, int qi) {
+    if (!p.ready) return;
+    __threadfence();
+    st_release_gpu(p.ready + qi, 1u);
+}
 
 __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexParams p) {
     extern __shared__ __align__(16) unsigned char dsm[];
-    __shared__ __align__(16) uint32_t hist[kHistBins];
+    __shared__ __align__(16) uint32_t hist[kKeyBins];
     __shared__ uint32_t s_wsum[kFinalThreads / 32];
     __shared__ uint32_t s_res[4];
     __shared__ uint32_t s_cnt[kFinalF];  // the leader's: members per rank
@@ -727,7 +736,10 @@ __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexPara
     const bool valid = seq_ok && qr.len >= 1 && qr.len <= sq.len;
     const int64_t E = valid ? qr.len / p.m : 0;
     // the scan handled (and reported) these; the outcome is uniform over the cluster
-    if (!valid || E > p.max_entries || E <= p.k) return;
+    if (!valid || E > p.max_entries || E <= p.k) {
+        if (rank == 0 && tid == 0) signal_ready(p, qi);
+        return;
+    }
     const int64_t chunk = p.chunk;
     const int nch = (int)((E + chunk - 1) / chunk);
     const int cap = p.cand_cap;
@@ -738,20 +750,23 @@ __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexPara
     // 1. the threshold bin; the histogram and this CTA's chunk words are loaded together
     uint32_t* mw = reinterpret_cast<uint32_t*>(dsm);
     {
-        const uint32_t* gh = p.hist + (int64_t)qi * kHistBins;
-        uint32_t hv[kHistBins / kFinalThreads];
+        const uint32_t* gh = p.hist + (int64_t)qi * kKeyBins;
+        uint32_t hv[kKeyBins / kFinalThreads];
 #pragma unroll
-        for (int i = 0; i < kHistBins / kFinalThreads; ++i) hv[i] = __ldcg(gh + tid + i * kFinalThreads);
+        for (int i = 0; i < kKeyBins / kFinalThreads; ++i) hv[i] = __ldcg(gh + tid + i * kFinalThreads);
         if (words_smem)
             for (int c = tid; c < nmine; c += kFinalThreads) mw[c] = __ldcg(meta + c);
 #pragma unroll
-        for (int i = 0; i < kHistBins / kFinalThreads; ++i) hist[tid + i * kFinalThreads] = hv[i];
+        for (int i = 0; i < kKeyBins / kFinalThreads; ++i) hist[tid + i * kFinalThreads] = hv[i];
     }
     __syncthreads();
-    find_bin<kFinalThreads>(hist, (uint32_t)p.k, s_wsum, s_res);
+    find_bin<kFinalThreads, kKeyBins>(hist, (uint32_t)p.k, s_wsum, s_res);
     const uint32_t b1 = s_res[0], above = s_res[1], at = s_res[2];
     if (b1 == 0xFFFFFFFFu) {  // the histogram holds fewer than k scores: cannot happen for E > k
-        if (tid == 0 && rank == 0) report(p.status, CSA_ERR_INDEX);
+        if (tid == 0 && rank == 0) {
+            report(p.status, CSA_ERR_INDEX);
+            signal_ready(p, qi);
+        }
         return;
     }
     const uint32_t n_bin = at - above, need = (uint32_t)p.k - above, n_tot = at;
@@ -852,7 +867,7 @@ __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexPara
                     const uint32_t w = (jk[u] & 0x40000000u) ? (uint32_t)(v[u] >> 32) : (uint32_t)v[u];
                     v[u] = composite(float_key(__uint_as_float(w)), jk[u] & 0x3FFFFFFFu);
                 }
-                keep[u] = first + u * 32 < S && (uint32_t)(v[u] >> 53) >= b1;
+                keep[u] = first + u * 32 < S && (uint32_t)(v[u] >> (64 - kKeyBits)) >= b1;
             }
             written += compact_round<kFinalThreads, kTailPer>(v, keep, written, sink, s_wsum);
         }
@@ -877,7 +892,10 @@ __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexPara
         }
     }
     if (total != n_tot) {  // the members must be exactly the histogram's count of bins >= b1
-        if (tid == 0 && rank == 0) report(p.status, CSA_ERR_INDEX);
+        if (tid == 0 && rank == 0) {
+            report(p.status, CSA_ERR_INDEX);
+            signal_ready(p, qi);
+        }
         cluster_barrier();  // every CTA takes the same barriers
         return;
     }
@@ -892,7 +910,7 @@ __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexPara
     if (rank == 0) {
         // 4. the exact threshold inside bin b1, then compaction in index order
         const KeyList L{in_smem ? lst : nullptr, in_smem ? nullptr : gseg};
-        const uint64_t T = need == n_bin ? ((uint64_t)b1 << 53) : radix_select<kFinalThreads>(L, n_tot, need, b1, hist,
+        const uint64_t T = need == n_bin ? ((uint64_t)b1 << (64 - kKeyBits)) : radix_select<kFinalThreads, kKeyBits>(L, n_tot, need, b1, hist,
                                                                                                s_wsum, s_res);
         float* sout = p.score_out ? p.score_out + (int64_t)qi * p.k : nullptr;
         uint32_t kept = 0;
@@ -914,6 +932,10 @@ __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexPara
             }, s_wsum);
         }
         if (tid == 0 && kept != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
+        if (p.ready) {
+            __syncthreads();  // every index store of the CTA precedes the release
+            if (tid == 0) signal_ready(p, qi);
+        }
     }
     if (!p.prefetch_rows) return;  // (uniform over the cluster)
     cluster_barrier();  // the indices are out (the barrier orders global memory at cluster scope)
@@ -991,7 +1013,9 @@ size_t cand_keys(int Q, int64_t e_stride) { return (size_t)Q * (size_t)(e_stride
 
 }  // namespace
 
-size_t index_zero_bytes(int Q) { return align256((size_t)Q * kHistBins * 4); }
+size_t index_zero_bytes(int Q) { return align256((size_t)Q * (kKeyBins + 2) * 4); }
+
+uint32_t* index_ready_words(void* ws, int Q) { return static_cast<uint32_t*>(ws) + (size_t)Q * kKeyBins; }
 
 size_t index_ws_bytes(int Q, int64_t e_stride) {
     size_t s = index_zero_bytes(Q);
@@ -1016,6 +1040,7 @@ void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
     p.coff = reinterpret_cast<uint32_t*>(b);
     b += align256(chunk_words(Q, e_stride) * 4);
     p.cand = reinterpret_cast<uint64_t*>(b);
+    p.ready = nullptr;
     p.e_stride = e_stride;
     p.e_seg = e_stride + kSegPad;
     p.chunk = sp.chunk;
@@ -1051,6 +1076,18 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
     if (gx > p.max_chunks) return cudaErrorInvalidValue;  // the workspace was carved for fewer entries
     const dim3 grid((unsigned)gx, (unsigned)p.Q);
     const bool dep = pdl && !zero_ws;
+    // with the key histogram in static shared memory, the dynamic part needs the opt-in (per device)
+    static PerDeviceOnce attr_scan;
+    e = attr_scan.run([] {
+        cudaError_t r = cudaSuccess;
+        for (auto f : {index_scan_kernel<1, false>, index_scan_kernel<2, false>, index_scan_kernel<1, true>,
+                       index_scan_kernel<2, true>})
+            if (r == cudaSuccess) r = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanDynSmem);
+        if (r == cudaSuccess)
+            r = cudaFuncSetAttribute(index_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFinalDynSmem);
+        return r;
+    });
+    if (e != cudaSuccess) return e;
     if (p.keys_q)
         e = p.d_I == 64 ? launch_kernel(index_scan_kernel<2, true>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p)
                         : launch_kernel(index_scan_kernel<1, true>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p);

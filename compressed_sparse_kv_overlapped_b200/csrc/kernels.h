@@ -60,7 +60,13 @@ struct TileCompressParams {
 cudaError_t launch_compress_tiles(const TileCompressParams& p, int64_t max_span, cudaStream_t stream);
 
 // Indexer score scan + top-k select.
-constexpr int kHistBins = 2048;  // coarse histogram over the top 11 bits of the score key
+constexpr int kHistBins = 2048;  // sampled histogram of the prefill select: the top 11 bits of the score key
+// histogram of the decode scan and final select: the top kKeyBits bits of the score key (sign,
+// exponent and two mantissa bits: bins a quarter of an octave wide).  13 bits were measured slower at
+// 1M tokens: the lists get shorter, but the per-bin work of the scan's merge, the threshold search
+// and the radix passes grows more than that saves.
+constexpr int kKeyBits = 11;
+constexpr int kKeyBins = 1 << kKeyBits;
 constexpr int kMaxK = 2048;
 constexpr int kSegPad = 128;  // keys of slack past each score row in the segment buffer
 
@@ -81,11 +87,14 @@ struct IndexParams {
     int cand_cap;             // candidate keys a scan chunk may keep
     // workspace
     float* scores;            // [Q, e_stride]
-    uint32_t* hist;           // [Q, kHistBins]; zero before the scan
+    uint32_t* hist;           // [Q, kKeyBins]; zero before the scan
     uint64_t* seg;            // [Q, e_seg] kept entries (64-bit keys) when they exceed shared memory
     uint32_t* meta;           // [Q, max_chunks] per scan chunk: (threshold bin << 16) | candidate count
     uint32_t* coff;           // [Q, max_chunks + 8] the final select's per-CTA prefixes over chunks (many chunks)
     uint64_t* cand;           // [Q, max_chunks, cand_cap] candidate keys of each chunk, in index order
+    // nullable: [Q] words, zero before the scan; the final select sets word q (release) once query
+    // q's indices are out, for an attention grid that starts before the select grid ends
+    uint32_t* ready;
     // optional: rows of this cache (row stride prefetch_row_bytes, a multiple of 16) at the selected
     // entries are prefetched into L2 as soon as the selection is known (the attention's gather)
     const unsigned char* prefetch_rows;
@@ -97,6 +106,9 @@ struct IndexParams {
 };
 size_t index_ws_bytes(int Q, int64_t e_stride);
 size_t index_zero_bytes(int Q);  // leading bytes of the index workspace that must start at zero
+// Per-step words of `ws` inside its leading zero bytes, after the histograms: Q ready words (see
+// IndexParams::ready), then Q item counters (see AttnParams::items_done).
+uint32_t* index_ready_words(void* ws, int Q);
 // Points the workspace arrays of `p` into `ws` and sets the scan chunking (chunk, max_chunks,
 // cand_cap), all derived from (Q, e_stride) exactly as index_ws_bytes sizes them.
 void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride);
@@ -180,6 +192,12 @@ struct AttnParams {
     // they take the free SMs before the front items (which wait for the top-k) do.  Launches all
     // items of all queries.
     int hca_first;
+    // nullable (multi-item launches): [Q] words the top-k select sets once query q's indices are out;
+    // the front items of query q poll theirs instead of waiting for the whole previous grid
+    const uint32_t* ready;
+    // nullable (multi-item launches): [Q] counters, zero before the launch; every item CTA of query q
+    // adds 1 once its partial is stored, and the merge of query q starts when all n_items have
+    uint32_t* items_done;
     // > 1: the launch forms thread-block clusters of `cluster` consecutive items of one query (the
     // item counts of both parts are multiples of it); the CTAs of a cluster merge their results
     // through distributed shared memory and store one partial per cluster, so part_o holds
