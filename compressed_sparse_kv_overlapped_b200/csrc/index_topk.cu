@@ -53,22 +53,28 @@ __device__ __forceinline__ uint4 ld_stream(const void* p, uint64_t pol) {
     return v;
 }
 
-// Scores of 16 consecutive entries (rows r0 .. r0+15 of the key cache) for one warp.
+// Scores of 16 consecutive entries (rows r0 .. r0+15 of the key cache) for one warp, in two halves:
+// load16 issues the loads, score16 forms the scores from them.  A pass issues the loads of all its
+// groups before it scores any: an mma waits for its operands, and the loads of the next group must
+// not wait behind it.
 // KV = number of 16-byte vectors per key row (d_I / 8 / 4 per thread group): d_I = 64 -> 2, 32 -> 1.
 template <int KV>
-__device__ __forceinline__ void score16(const uint16_t* keys, int64_t r0, int64_t nrows, int g, int c,
-                                        const uint32_t (&bq)[2 * KV][2], const float (&wv)[2], uint64_t pol,
-                                        float& s_lo, float& s_hi) {
+__device__ __forceinline__ void load16(const uint16_t* keys, int64_t r0, int64_t nrows, int g, int c, uint64_t pol,
+                                       uint4 (&lo)[KV], uint4 (&hi)[KV]) {
     // thread (g, c) loads rows g and g+8, vectors [32*v + 8c, 32*v + 8c + 8) for v < KV.  Rows past
     // the end (scores the caller drops) load the last row instead: the loads stay unconditional,
     // so none waits at a branch join before the next is issued.
-    uint4 lo[KV], hi[KV];
     const int64_t rl = min(r0 + g, nrows - 1), rh = min(r0 + g + 8, nrows - 1);
 #pragma unroll
     for (int v = 0; v < KV; ++v) {
         lo[v] = ld_stream(keys + rl * (KV * 32) + v * 32 + c * 8, pol);
         hi[v] = ld_stream(keys + rh * (KV * 32) + v * 32 + c * 8, pol);
     }
+}
+
+template <int KV>
+__device__ __forceinline__ void score16(const uint4 (&lo)[KV], const uint4 (&hi)[KV], const uint32_t (&bq)[2 * KV][2],
+                                        const float (&wv)[2], float& s_lo, float& s_hi) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int v = 0; v < KV; ++v) {
@@ -121,38 +127,47 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
 
 // Scores of 16 consecutive entries with 8-bit block-scaled keys (blocks of 32 channels, E4M3
 // elements, one power-of-two scale byte per block): thread (g, c) loads 8 bytes of each block for
-// rows g and g + 8, converts them to f16 (exact), and the products with the f16 query (each head
-// pre-scaled by a power of two 2^qsh[.], so it is exact in f16) accumulate per block in fp32; the
-// block scales and the query scale are applied exactly (powers of two) before relu.
+// rows g and g + 8 (load16_mx8), converts them to f16 (exact), and the products with the f16 query
+// (each head pre-scaled by a power of two 2^qsh[.], so it is exact in f16) accumulate per block in
+// fp32; the block scales and the query scale are applied exactly (powers of two) before relu
+// (score16_mx8).
 template <int NB>
-__device__ __forceinline__ void score16_mx8(const uint8_t* keys, const uint8_t* scales, int64_t r0, int64_t nrows,
-                                            int g, int c, const uint32_t (&bq)[2 * NB][2], const float (&wv)[2],
-                                            const int (&qsh)[2], uint64_t pol, float& s_lo, float& s_hi) {
-    constexpr int DI = 32 * NB;
-    // rows past the end (scores the caller drops) load the last row: unconditional loads (see score16)
+struct Keys8 {
     uint2 lo[NB], hi[NB];
+    uint32_t sl, sh;  // scale bytes of rows g and g + 8
+};
+
+template <int NB>
+__device__ __forceinline__ void load16_mx8(const uint8_t* keys, const uint8_t* scales, int64_t r0, int64_t nrows,
+                                           int g, int c, uint64_t pol, Keys8<NB>& k) {
+    constexpr int DI = 32 * NB;
+    // rows past the end (scores the caller drops) load the last row: unconditional loads (see load16)
     const int64_t rl = min(r0 + g, nrows - 1), rh = min(r0 + g + 8, nrows - 1);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-        lo[b] = ld_stream8(keys + rl * DI + b * 32 + c * 8, pol);
-        hi[b] = ld_stream8(keys + rh * DI + b * 32 + c * 8, pol);
+        k.lo[b] = ld_stream8(keys + rl * DI + b * 32 + c * 8, pol);
+        k.hi[b] = ld_stream8(keys + rh * DI + b * 32 + c * 8, pol);
     }
-    // scale bytes of rows g and g + 8
-    const uint32_t sl = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rl * NB) : scales[rl];
-    const uint32_t sh = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rh * NB) : scales[rh];
+    k.sl = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rl * NB) : scales[rl];
+    k.sh = NB == 2 ? (uint32_t)*reinterpret_cast<const uint16_t*>(scales + rh * NB) : scales[rh];
+}
+
+template <int NB>
+__device__ __forceinline__ void score16_mx8(const Keys8<NB>& k, const uint32_t (&bq)[2 * NB][2], const float (&wv)[2],
+                                            const int (&qsh)[2], float& s_lo, float& s_hi) {
     float tot[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-        const uint32_t l0 = e4m3x2_to_f16x2(lo[b].x), l1 = e4m3x2_to_f16x2(lo[b].x >> 16);
-        const uint32_t l2 = e4m3x2_to_f16x2(lo[b].y), l3 = e4m3x2_to_f16x2(lo[b].y >> 16);
-        const uint32_t h0 = e4m3x2_to_f16x2(hi[b].x), h1 = e4m3x2_to_f16x2(hi[b].x >> 16);
-        const uint32_t h2 = e4m3x2_to_f16x2(hi[b].y), h3 = e4m3x2_to_f16x2(hi[b].y >> 16);
+        const uint32_t l0 = e4m3x2_to_f16x2(k.lo[b].x), l1 = e4m3x2_to_f16x2(k.lo[b].x >> 16);
+        const uint32_t l2 = e4m3x2_to_f16x2(k.lo[b].y), l3 = e4m3x2_to_f16x2(k.lo[b].y >> 16);
+        const uint32_t h0 = e4m3x2_to_f16x2(k.hi[b].x), h1 = e4m3x2_to_f16x2(k.hi[b].x >> 16);
+        const uint32_t h2 = e4m3x2_to_f16x2(k.hi[b].y), h3 = e4m3x2_to_f16x2(k.hi[b].y >> 16);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         const uint32_t a0[4] = {l0, h0, l1, h1};
         const uint32_t a1[4] = {l2, h2, l3, h3};
         mma_f16_16816(acc, a0, bq[2 * b]);
         mma_f16_16816(acc, a1, bq[2 * b + 1]);
-        const int el = (int)((sl >> (8 * b)) & 0xFFu) - 127, eh = (int)((sh >> (8 * b)) & 0xFFu) - 127;
+        const int el = (int)((k.sl >> (8 * b)) & 0xFFu) - 127, eh = (int)((k.sh >> (8 * b)) & 0xFFu) - 127;
         tot[0] = __fadd_rn(tot[0], scale_pow2(acc[0], el - qsh[0]));
         tot[1] = __fadd_rn(tot[1], scale_pow2(acc[1], el - qsh[1]));
         tot[2] = __fadd_rn(tot[2], scale_pow2(acc[2], eh - qsh[0]));
@@ -629,14 +644,23 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
         constexpr int kRowsPerPass = kScanThreads / 32 * 16 * 4;  // 512 entries: 4 groups of 16 per warp
         for (int64_t base = c0; base < c1; base += kRowsPerPass) {
             float s[4][2];
+            // every load of the pass first, then the scores
+            if (MX8) {
+                Keys8<KV> k8[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t r0 = base + (int64_t)(u * (kScanThreads / 32) + warp) * 16;
-                if (MX8)
-                    score16_mx8<KV>(p.keys_q + sq.csa_off * p.d_I, p.key_scales + sq.csa_off * KV, r0, c1, g, c, bq,
-                                    wv, qsh, pol, s[u][0], s[u][1]);
-                else
-                    score16<KV>(keys, r0, c1, g, c, bq, wv, pol, s[u][0], s[u][1]);
+                for (int u = 0; u < 4; ++u)
+                    load16_mx8<KV>(p.keys_q + sq.csa_off * p.d_I, p.key_scales + sq.csa_off * KV,
+                                   base + (int64_t)(u * (kScanThreads / 32) + warp) * 16, c1, g, c, pol, k8[u]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) score16_mx8<KV>(k8[u], bq, wv, qsh, s[u][0], s[u][1]);
+            } else {
+                uint4 klo[4][KV], khi[4][KV];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    load16<KV>(keys, base + (int64_t)(u * (kScanThreads / 32) + warp) * 16, c1, g, c, pol, klo[u],
+                               khi[u]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) score16<KV>(klo[u], khi[u], bq, wv, s[u][0], s[u][1]);
             }
             // stage in shared memory, then coalesced store + histogram
             if (c == 0) {
