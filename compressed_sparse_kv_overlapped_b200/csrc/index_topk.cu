@@ -641,36 +641,18 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
         const uint16_t* keys = p.entry_keys + sq.csa_off * p.d_I;
         float* srow = p.scores + (int64_t)qi * p.e_stride;
         const uint64_t pol = policy_evict_first();
-        constexpr int kRowsPerPass = kScanThreads / 32 * 16 * 4;  // 512 entries: 4 groups of 16 per warp
-        for (int64_t base = c0; base < c1; base += kRowsPerPass) {
-            float s[4][2];
-            // every load of the pass first, then the scores
-            if (MX8) {
-                Keys8<KV> k8[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    load16_mx8<KV>(p.keys_q + sq.csa_off * p.d_I, p.key_scales + sq.csa_off * KV,
-                                   base + (int64_t)(u * (kScanThreads / 32) + warp) * 16, c1, g, c, pol, k8[u]);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) score16_mx8<KV>(k8[u], bq, wv, qsh, s[u][0], s[u][1]);
-            } else {
-                uint4 klo[4][KV], khi[4][KV];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    load16<KV>(keys, base + (int64_t)(u * (kScanThreads / 32) + warp) * 16, c1, g, c, pol, klo[u],
-                               khi[u]);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) score16<KV>(klo[u], khi[u], bq, wv, s[u][0], s[u][1]);
-            }
-            // stage in shared memory, then coalesced store + histogram
+        // a pass's scores: staged in shared memory, then stored coalesced and counted (groups u of
+        // 16 rows at base + (u * 8 + warp) * 16)
+        auto finish = [&](int64_t base, const float (&s)[4][2], int groups) {
             if (c == 0) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) { sc[warp][u][g] = s[u][0]; sc[warp][u][g + 8] = s[u][1]; }
+                for (int u = 0; u < 4; ++u)
+                    if (u < groups) { sc[warp][u][g] = s[u][0]; sc[warp][u][g + 8] = s[u][1]; }
             }
             __syncwarp();
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                if (lane < 16) {
+                if (u < groups && lane < 16) {
                     const int64_t r = base + (int64_t)(u * (kScanThreads / 32) + warp) * 16 + lane;
                     if (r < c1) {
                         const float v = sc[warp][u][lane];
@@ -681,6 +663,46 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
                 }
             }
             __syncwarp();
+        };
+        if (MX8) {
+            constexpr int kRowsPerPass = kScanThreads / 32 * 16 * 4;  // 512 entries: 4 groups of 16 per warp
+            for (int64_t base = c0; base < c1; base += kRowsPerPass) {
+                float s[4][2];
+                // every load of the pass first, then the scores
+                Keys8<KV> k8[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    load16_mx8<KV>(p.keys_q + sq.csa_off * p.d_I, p.key_scales + sq.csa_off * KV,
+                                   base + (int64_t)(u * (kScanThreads / 32) + warp) * 16, c1, g, c, pol, k8[u]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) score16_mx8<KV>(k8[u], bq, wv, qsh, s[u][0], s[u][1]);
+                finish(base, s, 4);
+            }
+        } else {
+            // software pipeline over passes of two 16-row groups per warp, in two register buffers:
+            // the next pass's loads are in flight while this pass is scored (a warp never waits with
+            // no loads outstanding).  Loads past the chunk read its last row; their scores are dropped.
+            constexpr int kG = 2;
+            constexpr int64_t kRows = kScanThreads / 32 * 16 * kG;  // 256 entries per pass
+            uint4 alo[kG][KV], ahi[kG][KV], blo[kG][KV], bhi[kG][KV];
+            auto load_pass = [&](int64_t base, uint4 (&lo)[kG][KV], uint4 (&hi)[kG][KV]) {
+#pragma unroll
+                for (int u = 0; u < kG; ++u)
+                    load16<KV>(keys, base + (int64_t)(u * (kScanThreads / 32) + warp) * 16, c1, g, c, pol, lo[u], hi[u]);
+            };
+            auto score_pass = [&](int64_t base, const uint4 (&lo)[kG][KV], const uint4 (&hi)[kG][KV]) {
+                float s[4][2];
+#pragma unroll
+                for (int u = 0; u < kG; ++u) score16<KV>(lo[u], hi[u], bq, wv, s[u][0], s[u][1]);
+                finish(base, s, kG);
+            };
+            load_pass(c0, alo, ahi);
+            for (int64_t base = c0; base < c1; base += 2 * kRows) {
+                load_pass(base + kRows, blo, bhi);
+                score_pass(base, alo, ahi);
+                load_pass(base + 2 * kRows, alo, ahi);
+                score_pass(base + kRows, blo, bhi);
+            }
         }
     }
     __syncthreads();
