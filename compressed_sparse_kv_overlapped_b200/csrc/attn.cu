@@ -103,10 +103,10 @@ struct KeyList {
 // The source of key s: a bf16 row (returned, *scl = nullptr) or, for an entry of a cache held in FP4,
 // its code row (returned) with its scale row in *scl; nullptr for an empty or invalid slot.
 __device__ __forceinline__ const void* key_src(const AttnParams& p, int D, const KeyList& kl, int64_t s,
-                                               const uint8_t** scl) {
+                                               const uint8_t** scl, bool have_j = false, int32_t jpre = 0) {
     *scl = nullptr;
     if (s < p.k_slots) {
-        const int32_t j = kl.idx[s];
+        const int32_t j = have_j ? jpre : kl.idx[s];  // the slot's index, unless the caller read it already
         if (j < 0) return nullptr;
         if ((int64_t)j >= kl.n_causal) {
             report(p.status, CSA_ERR_INDEX);
@@ -252,6 +252,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             if (p.tma_hca) tma_prefetch_map(&maps.hca);
             if (p.tma_x) tma_prefetch_map(&maps.x);
         }
+        // the selected indices of this lane's rows in the first two tiles, read together (one memory
+        // latency, not one per tile); an address past the slots reads the last slot, unused
+        int32_t pre_j0 = -1, pre_j1 = -1;
+        const bool pre = go && kl.idx && s0 < p.k_slots && lane < 16;
+        if (pre) {
+            const int64_t sa = s0 + lw * 16 + lane, sb = sa + kTileKeys;
+            pre_j0 = kl.idx[sa < p.k_slots ? sa : p.k_slots - 1];
+            pre_j1 = kl.idx[sb < p.k_slots ? sb : p.k_slots - 1];
+        }
         // per stage, the full-barrier parity of the last tile this thread loaded by TMA (bit 2 set:
         // one is pending), so that a CTA that gives up waits for its own copies before it exits
         uint32_t tma_pend = 0;
@@ -295,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             if (lane < 16) {
                 const int64_t s = tb + lw * 16 + lane;
                 const uint8_t* scl = nullptr;
-                const void* r = s < s1 ? key_src(p, D, kl, s, &scl) : nullptr;
+                const void* r = s < s1 ? key_src(p, D, kl, s, &scl, pre && t < 2, t == 0 ? pre_j0 : pre_j1) : nullptr;
                 rowptr_w[lane] = reinterpret_cast<uint64_t>(r);
                 rowscl_w[lane] = reinterpret_cast<uint64_t>(scl);
                 valid = r != nullptr;
