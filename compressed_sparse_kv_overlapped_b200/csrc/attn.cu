@@ -131,7 +131,9 @@ __device__ __forceinline__ const void* key_src(const AttnParams& p, int D, const
     return p.hca + r * D;
 }
 
-template <int D>
+// FP4: the instantiation for FP4 entry caches (its loaders dequantize FP4 rows); the other holds no
+// FP4 code at all, which keeps the bf16 kernel's hot loops compact.
+template <int D, bool FP4>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnMaps maps, AttnParams p,
                                                            int p_item_base) {
     using L = Smem<D>;
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 rowptr_w[lane] = reinterpret_cast<uint64_t>(r);
                 rowscl_w[lane] = reinterpret_cast<uint64_t>(scl);
                 valid = r != nullptr;
-                fp4 = scl != nullptr;
+                fp4 = FP4 && scl != nullptr;
             }
             const uint32_t vm = __ballot_sync(0xffffffffu, valid) & 0xFFFFu;
             const bool tile_fp4 = __ballot_sync(0xffffffffu, fp4) != 0u;
@@ -328,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                     cp_async16(dst, src + lane * 8, nb);
                 }
             };
-            if (!tile_fp4) {
+            if (!FP4 || !tile_fp4) {
 #pragma unroll 4
                 for (int r = 0; r < 16; ++r) copy_row(r);
                 // the copies complete the tile's barrier phase themselves: no wait here, so the next
@@ -903,9 +905,14 @@ template <int D>
 cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, cudaStream_t stream, bool pdl) {
     using L = Smem<D>;
     static PerDeviceOnce attr;
-    cudaError_t ea = attr.run(
-        [] { return cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc); });
+    cudaError_t ea = attr.run([] {
+        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(attn_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+        return e;
+    });
     if (ea != cudaSuccess) return ea;
+    auto kernel = (p.entries_q || p.hca_q) ? attn_kernel<D, true> : attn_kernel<D, false>;
     const dim3 grid = p.hca_first ? dim3((unsigned)(p.n_items * p.Q)) : dim3((unsigned)item_count, (unsigned)p.Q);
     // tensor maps over the HCA cache and the raw latents; the kernel only issues boxes that lie
     // inside one sequence's valid rows, so the row extent is left open
@@ -918,9 +925,9 @@ cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, 
     if (!q.tma_hca) std::memset(&maps.hca, 0, sizeof(maps.hca));
     if (!q.tma_x) std::memset(&maps.x, 0, sizeof(maps.x));
     if (q.cluster > 1 && q.n_items > 1)
-        return launch_kernel_cluster(attn_kernel<D>, grid, dim3(kThreads), L::kAlloc, stream, pdl,
+        return launch_kernel_cluster(kernel, grid, dim3(kThreads), L::kAlloc, stream, pdl,
                                      dim3((unsigned)q.cluster, 1, 1), maps, q, item_begin);
-    return launch_kernel(attn_kernel<D>, grid, dim3(kThreads), L::kAlloc, stream, pdl, maps, q, item_begin);
+    return launch_kernel(kernel, grid, dim3(kThreads), L::kAlloc, stream, pdl, maps, q, item_begin);
 }
 
 }  // namespace
