@@ -105,13 +105,15 @@ def parse():
 
 
 def peaks(sustained=False):
+    """(copy GB/s, bf16 TFLOP/s, source): the measured figures of MEASURED_PEAKS.json, else the
+    fallback measurement on this hardware (6,650 GB/s; 1,590 TFLOP/s burst, 1,400 sustained)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
         tf = p.get("bf16_tflops_sustained" if sustained else "bf16_tflops", 1590.0)
-        return float(p["hbm_gbs"]), float(tf), "measured"
+        return float(p["hbm_gbs"]), float(tf), "measured (MEASURED_PEAKS.json)"
     except Exception:
-        return 6650.0, 1400.0 if sustained else 1590.0, "fallback"
+        return 6650.0, 1400.0 if sustained else 1590.0, "fallback (MEASURED_PEAKS.json absent)"
 
 
 # ------------------------------------------------------------------------------------ clocks
@@ -374,7 +376,7 @@ def run_ours(args, rank, world):
                      "traffic": scan_traffic() if wl.name.startswith("ctx1m") and args.keys == "bf16" else None,
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch, "
                                        "taken on the current scan source (null otherwise)",
-                     "bytes_per_launch": int(scan_bytes), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
+                     "bytes_per_launch": int(scan_bytes), "peak_source": f"{peak_src}: copy bandwidth"},
         "clocks": clocks.summary(t0, t1),
     }
     # kernel nodes of the timed graph (all of them this library's kernels)
@@ -795,7 +797,7 @@ def run_prefill(args, rank, world):
         "flops": {"index": f_index, "attention": f_attn, "total": f_index + f_attn},
         "roofline": {"kernel": "whole prefill (index + select + attention)", "bound": "tensor", "achieved": tflops,
                      "peak": tf_peak, "unit": "TFLOP/s", "frac": tflops / tf_peak, "traffic": None,
-                     "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops_sustained)"},
+                     "peak_source": f"{src}: sustained bf16 tensor throughput"},
         "compress": {"ms": ms_comp, "bytes": comp_bytes, "achieved_gbs": comp_bytes / (ms_comp * 1e-3) / 1e9,
                      "peak_gbs": hbm, "frac": comp_bytes / (ms_comp * 1e-3) / 1e9 / hbm,
                      "note": "csa_compress_all: CSA entries, indexer keys and HCA entries over all N tokens, one pass"},
