@@ -476,6 +476,10 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
     ip.prefetch_row_bytes = prefetch_row_bytes;
     index_ws_carve(ip, ws_index, Q, e_stride);
     ip.ready = ready;
+    if (ready) {
+        uint64_t unused;
+        debug_fault_state(&ip.debug_fault, &unused);
+    }
     cudaError_t e = launch_index_topk(ip, max_e, stream, zero_ws, mid, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "index_topk launch");
     return CSA_OK;
@@ -517,7 +521,8 @@ extern "C" {
 int csa_version(void) { return 200; }
 
 int csa_debug_inject(int fault, int64_t wait_limit_ns) {
-    if (fault < 0 || fault > 1) return fail(CSA_ERR_ARG, "fault = %d (0 none, 1 attention tile never full)", fault);
+    if (fault < 0 || fault > 2)
+        return fail(CSA_ERR_ARG, "fault = %d (0 none, 1 attention tile never full, 2 no ready word)", fault);
     if (wait_limit_ns < 0) return fail(CSA_ERR_ARG, "wait_limit_ns = %lld", (long long)wait_limit_ns);
     g_debug_fault.store(fault, std::memory_order_relaxed);
     g_debug_wait_ns.store((uint64_t)wait_limit_ns, std::memory_order_relaxed);

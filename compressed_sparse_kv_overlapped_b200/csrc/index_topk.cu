@@ -760,7 +760,7 @@ constexpr int kFinalChunks = (kKeyBins - 2) / 2;  // chunks per CTA whose words 
 // Query qi's indices are out: publish its ready word (one thread, after the stores it covers are
 // ordered before it: by a CTA barrier, or by the grid dependency for the scan's own results).
 __device__ __forceinline__ void signal_ready(const IndexParams& p, int qi) {
-    if (!p.ready) return;
+    if (!p.ready || p.debug_fault == 2) return;  // fault injection: the waits on the word run out
     __threadfence();
     st_release_gpu(p.ready + qi, 1u);
 }
@@ -1087,6 +1087,7 @@ void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
     b += align256(chunk_words(Q, e_stride) * 4);
     p.cand = reinterpret_cast<uint64_t*>(b);
     p.ready = nullptr;
+    p.debug_fault = 0;
     p.e_stride = e_stride;
     p.e_seg = e_stride + kSegPad;
     p.chunk = sp.chunk;

@@ -95,6 +95,7 @@ struct IndexParams {
     // nullable: [Q] words, zero before the scan; the final select sets word q (release) once query
     // q's indices are out, for an attention grid that starts before the select grid ends
     uint32_t* ready;
+    int debug_fault;          // 2 (tests of the bounded waits): the select publishes no ready word
     // optional: rows of this cache (row stride prefetch_row_bytes, a multiple of 16) at the selected
     // entries are prefetched into L2 as soon as the selection is known (the attention's gather)
     const unsigned char* prefetch_rows;

@@ -378,9 +378,11 @@ int csa_index_topk_noalloc(const csa_dims* dims, const csa_seq* seqs, const csa_
  * device status word and lets the kernel wind down (the CTA waits for its own copies in flight,
  * frees its tensor memory and exits), so a fault never hangs the device.  fault = 1 makes the
  * attention kernel's first loader warp skip its arrival on the first key tile of every CTA, so that
- * tile never becomes full and the waits on it run out; fault = 0 turns injection off.
+ * tile never becomes full and the waits on it run out; fault = 2 makes the top-k select of
+ * hybrid_attn_decode publish no per-query ready word, so the front attention items' waits on those
+ * words run out; fault = 0 turns injection off.
  * wait_limit_ns > 0 sets the limit of the attention kernel's waits (0 restores the default of 2 s).
- * Process-wide; applies to attention launches issued after the call.  Returns CSA_OK or
+ * Process-wide; applies to launches issued after the call.  Returns CSA_OK or
  * CSA_ERR_ARG. */
 int csa_debug_inject(int fault, int64_t wait_limit_ns);
 

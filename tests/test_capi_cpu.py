@@ -155,7 +155,8 @@ def test_compress_all_and_fault_injection_validation(lib):
     n.entry_norm_c, n.entry_norm_h = None, 16
     rc = lib.csa_compress_all(ctypes.byref(csa.make_dims(m_hca=256)), 16, 16, 1, 10, *P[:9], ctypes.byref(n), None)
     assert rc == csa.CSA_ERR_UNSUPPORTED
-    assert lib.csa_debug_inject(2, 0) == csa.CSA_ERR_ARG
+    assert lib.csa_debug_inject(3, 0) == csa.CSA_ERR_ARG
+    assert lib.csa_debug_inject(2, 0) == csa.CSA_OK
     assert lib.csa_debug_inject(1, -5) == csa.CSA_ERR_ARG
     assert lib.csa_debug_inject(0, 0) == csa.CSA_OK
 

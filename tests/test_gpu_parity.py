@@ -920,6 +920,38 @@ def _decode_e2e(wl, steps, check_every=1, via_new_rows=False):
     return n_diff
 
 
+def test_ready_word_wait_runs_out_and_the_device_recovers():
+    """The front attention items of a decode step wait for their query's ready word from the top-k
+    select with a bounded poll: with fault injection 2 the select publishes no word, the wait runs
+    out after the short limit and is reported as CSA_ERR_TIMEOUT, and the next step on the same
+    context matches the oracle."""
+    wl = wl_small(6000)
+    layer = gh.new_layer(wl)
+    d = wl.dims
+    q = torch.empty(1, d.H, d.d, dtype=torch.bfloat16, device="cuda")
+    qi = torch.empty(1, d.H_I, d.d_I, dtype=torch.bfloat16, device="cuda")
+    w = torch.empty(1, d.H_I, dtype=torch.float32, device="cuda")
+    out = torch.empty(1, d.H, d.d, dtype=torch.float32, device="cuda")
+    lse = torch.empty(1, d.H, dtype=torch.float32, device="cuda")
+    ws = layer.decode_workspace()
+    ref = gh.OracleSeq(wl, 0, wl.n0[0] + 2)
+    try:
+        csa.csa_debug_inject(2, 1_000_000)  # 1 ms limit
+        sdev.fill_queries(wl, 0, 0, 1, q, qi, w)
+        layer.decode(layer.decode_args(q, qi, w, out, lse=lse), ws)
+        assert csa.csa_sync_status() == csa.CSA_ERR_TIMEOUT
+    finally:
+        csa.csa_debug_inject(0, 0)
+    assert csa.csa_sync_status() == csa.CSA_OK  # reading the status cleared it
+    sdev.fill_queries(wl, 0, 1, 2, q, qi, w)
+    layer.decode(layer.decode_args(q, qi, w, out, lse=lse), ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    L = wl.n0[0] + 2
+    qh, qih, wh = workloads.queries(wl, 0, 1, 2)
+    r = ref.query(L, qh[0], qih[0], wh[0])
+    gh.check_close(out[0].cpu().numpy(), r["O"], "decode step after the timeout")
+
+
 @pytest.mark.parametrize("wl,steps", [(workloads.tiny(), 1), (wl_small(6000), 3),
                                       (wl_small([700, 3000, 9001], B=3), 2)],
                          ids=["tiny", "prod6000", "ragged3"])
