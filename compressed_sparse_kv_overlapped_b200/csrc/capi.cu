@@ -449,6 +449,23 @@ int status_ptr(int** out) {
     return CSA_OK;
 }
 
+// Multiprocessor count of the current device, looked up once per device.
+int sm_count(int* out) {
+    static std::mutex mu;
+    static int counts[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(CSA_ERR_CUDA, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!counts[dev]) {
+        e = cudaDeviceGetAttribute(&counts[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    }
+    *out = counts[dev];
+    return CSA_OK;
+}
+
 int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, int Q, int64_t max_e,
               int64_t e_stride, const csa_bf16* q_idx, const float* w, const csa_bf16* entry_keys, int32_t* idx_out,
               float* score_out, void* ws_index, bool zero_ws, int* status, cudaStream_t stream,
@@ -476,6 +493,17 @@ int run_index(const csa_dims& d, const csa_seq* seqs, const csa_query* queries, 
     ip.prefetch_row_bytes = prefetch_row_bytes;
     index_ws_carve(ip, ws_index, Q, e_stride);
     ip.ready = ready;
+    // with the per-step words the scan grid can select itself (when it fits the SMs): off by default.
+    // At four 1M-token sequences it is slower (62.2 against 60.8 µs per step): the scan CTAs stay
+    // resident through the selection, so the HCA attention items lose the SMs they otherwise take
+    // while the select kernel runs on 32 of them
+    if (ready && env_int("CSA_SCAN_SELECT", 0) != 0) {
+        int sms = 0;
+        if (sm_count(&sms) == CSA_OK) {
+            ip.qsync = ready + 2 * Q;
+            ip.sms = sms;
+        }
+    }
     if (ready) {
         uint64_t unused;
         debug_fault_state(&ip.debug_fault, &unused);

@@ -194,6 +194,15 @@ __device__ __forceinline__ uint64_t composite(uint32_t key, int64_t j) {
     return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
 }
 
+// Query qi's indices are out: publish its ready word (one thread, after the stores it covers are
+// ordered before it: by a CTA barrier, or by the grid dependency for the scan's own results).
+__device__ __forceinline__ void signal_ready(const IndexParams& p, int qi) {
+    if (!p.ready || p.debug_fault == 2) return;  // fault injection: the waits on the word run out
+    __threadfence();
+    st_release_gpu(p.ready + qi, 1u);
+}
+
+
 // Exclusive prefix of one value per thread; *total gets the block's sum.  wsum: NT/32 words.
 // Two barriers: the warps' totals are published, then every warp sums the ones before it.
 template <int NT>
@@ -531,6 +540,135 @@ __global__ void __launch_bounds__(kSelectThreads) index_select_kernel(IndexParam
     if (tid == 0 && kept_total != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
 }
 
+// ---- exact top-k inside the scan grid -------------------------------------------------------------
+//
+// When every scan CTA is resident at once (the grid fits the SMs), the CTAs of query qi finish the
+// selection themselves, meeting on the query's counters qs[0..2]:
+//   A. each CTA adds its histogram to the query's and counts itself in qs[0]; once all nch chunks
+//      have, every CTA reads the complete histogram and finds the threshold bin b1;
+//   B. each CTA counts its members (its scores of bin >= b1, still in shared memory), publishes the
+//      count and counts itself in qs[1]; once all counts are out, it stores its members in index
+//      order at its place (the counts of the chunks before it) of the query's list;
+//   C. the last CTA to count itself in qs[2] radix-selects the exact threshold inside bin b1 among
+//      the list's members, writes the k indices in ascending order and publishes the ready word.
+// Every wait is bounded (a wait that runs out records CSA_ERR_TIMEOUT; the CTA gives up).
+__device__ void scan_select(const IndexParams& p, int qi, int cidx, int nch, int64_t c0, int n, const float* ssc,
+                            uint64_t* slist, uint32_t* hist, uint32_t* s_wsum, uint32_t* s_res, int32_t* out,
+                            float* sout, int64_t csa_off) {
+    __shared__ int s_ok;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t* qs = p.qsync + (int64_t)qi * 4;
+    // A. the query's complete histogram and its threshold bin
+    __syncthreads();  // this CTA's histogram atomics are issued
+    if (tid == 0) {
+        __threadfence();
+        atomicAdd(qs + 0, 1u);
+        s_ok = count_wait(qs + 0, (uint32_t)nch, p.status, nullptr) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    {
+        const uint32_t* gh = p.hist + (int64_t)qi * kKeyBins;
+        uint32_t hv[kKeyBins / kScanThreads];
+#pragma unroll
+        for (int i = 0; i < kKeyBins / kScanThreads; ++i) hv[i] = __ldcg(gh + tid + i * kScanThreads);
+#pragma unroll
+        for (int i = 0; i < kKeyBins / kScanThreads; ++i) hist[tid + i * kScanThreads] = hv[i];
+    }
+    __syncthreads();
+    find_bin<kScanThreads, kKeyBins>(hist, (uint32_t)p.k, s_wsum, s_res);
+    const uint32_t b1 = s_res[0], above = s_res[1], at = s_res[2];
+    const bool bad = b1 == 0xFFFFFFFFu;  // fewer than k scores: cannot happen for E > k
+    // B. this chunk's members: count, publish, wait for every chunk's count, then store them
+    uint32_t mine = 0;
+    for (int i = tid; i < n; i += kScanThreads) mine += (!bad && (float_key(ssc[i]) >> (32 - kKeyBits)) >= b1) ? 1u : 0u;
+    uint32_t cnt;
+    (void)excl_scan<kScanThreads>(mine, s_wsum, &cnt);
+    uint32_t* counts = p.meta + (int64_t)qi * p.max_chunks;
+    if (tid == 0) {
+        counts[cidx] = cnt;
+        __threadfence();
+        atomicAdd(qs + 1, 1u);
+        s_ok = count_wait(qs + 1, (uint32_t)nch, p.status, nullptr) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    uint32_t before = 0;
+    for (int j = tid; j < cidx; j += kScanThreads) before += __ldcg(counts + j);
+    uint32_t off;
+    (void)excl_scan<kScanThreads>(before, s_wsum, &off);
+    uint64_t* lst = p.seg + (int64_t)qi * p.e_seg;
+    {
+        uint32_t written = 0;
+        for (int base = 0; base < n; base += kScanThreads * kTailPer) {
+            const int first = base + warp * 32 * kTailPer + lane;
+            uint64_t v[kTailPer];
+            bool keep[kTailPer];
+#pragma unroll
+            for (int u = 0; u < kTailPer; ++u) {
+                const int i = first + u * 32;
+                const uint32_t key = i < n ? float_key(ssc[i]) : 0u;
+                keep[u] = !bad && i < n && (key >> (32 - kKeyBits)) >= b1;
+                v[u] = composite(key, c0 + i);
+            }
+            written += compact_round<kScanThreads, kTailPer>(
+                v, keep, written, [&](uint32_t pos, uint64_t x) { lst[off + pos] = x; }, s_wsum);
+        }
+    }
+    // C. the last chunk of the query selects
+    __syncthreads();  // every member store of the CTA precedes the count
+    if (tid == 0) {
+        __threadfence();
+        s_ok = atomicAdd(qs + 2, 1u) == (uint32_t)nch - 1 ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    __threadfence();  // the other chunks' members, stored before their counts, are visible
+    if (bad) {
+        if (tid == 0) {
+            report(p.status, CSA_ERR_INDEX);
+            signal_ready(p, qi);
+        }
+        return;
+    }
+    const uint32_t n_tot = at, need = (uint32_t)p.k - above, n_bin = at - above;
+    const bool in_smem = n_tot <= (uint32_t)kListKeys;
+    if (in_smem) {
+        for (uint32_t i = tid; i < n_tot; i += kScanThreads) slist[i] = __ldcg(reinterpret_cast<const unsigned long long*>(lst) + i);
+        __syncthreads();
+    }
+    const KeyList L{in_smem ? slist : nullptr, in_smem ? nullptr : lst};
+    const uint64_t T = need == n_bin ? ((uint64_t)b1 << (64 - kKeyBits))
+                                     : radix_select<kScanThreads, kKeyBits>(L, n_tot, need, b1, hist, s_wsum, s_res);
+    uint32_t kept = 0;
+    for (uint32_t base = 0; base < n_tot; base += kScanThreads * kTailPer) {
+        const uint32_t first = base + (uint32_t)(warp * 32 * kTailPer + lane);
+        uint64_t v[kTailPer];
+        bool keep[kTailPer];
+#pragma unroll
+        for (int u = 0; u < kTailPer; ++u) {
+            const uint32_t i = first + u * 32;
+            v[u] = i < n_tot ? L.get(i) : 0ull;
+            keep[u] = i < n_tot && v[u] >= T;
+        }
+        kept += compact_round<kScanThreads, kTailPer>(v, keep, kept, [&](uint32_t o, uint64_t x) {
+            if (o < (uint32_t)p.k) {
+                out[o] = (int32_t)(0xFFFFFFFFu - (uint32_t)(x & 0xFFFFFFFFull));
+                if (sout) sout[o] = key_float((uint32_t)(x >> 32));
+            }
+        }, s_wsum);
+    }
+    if (tid == 0 && kept != (uint32_t)p.k) report(p.status, CSA_ERR_INDEX);
+    __syncthreads();  // every index store of the CTA precedes the release
+    if (tid == 0) signal_ready(p, qi);
+    // the attention that follows gathers the selected rows: start bringing them into L2
+    if (p.prefetch_rows)
+        for (int o = tid; o < p.k; o += kScanThreads) {
+            const int32_t j = __ldcg(out + o);
+            if (j >= 0) prefetch_l2(p.prefetch_rows + (csa_off + j) * p.prefetch_row_bytes, p.prefetch_row_bytes);
+        }
+}
+
 // ---- decode scan ------------------------------------------------------------------------------------
 //
 // Scan CTA (chunk c, query qi): the scores of entries [c*chunk, min(E, (c+1)*chunk)) on the tensor
@@ -572,6 +710,10 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
         if (sout && n > 0) {
             __syncthreads();
             scores_of_all(p, qi, sq.csa_off, n, sout);
+        }
+        if (p.qsync) {  // no final select follows: publish the ready word here
+            __syncthreads();
+            if (tid == 0) signal_ready(p, qi);
         }
         return;
     }
@@ -711,6 +853,11 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
         for (int i = tid; i < kKeyBins; i += kScanThreads)
             if (hist[i]) atomicAdd(&gh[i], hist[i]);
     }
+    if (p.qsync) {  // the scan grid selects (see scan_select)
+        scan_select(p, qi, cidx, nch, c0, (int)(c1 - c0), ssc, reinterpret_cast<uint64_t*>(dsm), hist, s_wsum, s_res,
+                    out, sout, sq.csa_off);
+        return;
+    }
     // ---- the chunk's candidates
     const int n = (int)(c1 - c0);
     const int cap = p.cand_cap;
@@ -756,14 +903,6 @@ constexpr int kFinalF = 8;           // CTAs per query
 constexpr int kFinalThreads = 256;
 constexpr int kFinalDynSmem = kListKeys * 8;  // the members list (also this CTA's chunk words)
 constexpr int kFinalChunks = (kKeyBins - 2) / 2;  // chunks per CTA whose words fit the histogram's space
-
-// Query qi's indices are out: publish its ready word (one thread, after the stores it covers are
-// ordered before it: by a CTA barrier, or by the grid dependency for the scan's own results).
-__device__ __forceinline__ void signal_ready(const IndexParams& p, int qi) {
-    if (!p.ready || p.debug_fault == 2) return;  // fault injection: the waits on the word run out
-    __threadfence();
-    st_release_gpu(p.ready + qi, 1u);
-}
 
 __global__ void __launch_bounds__(kFinalThreads, 1) index_final_kernel(IndexParams p) {
     extern __shared__ __align__(16) unsigned char dsm[];
@@ -1059,7 +1198,7 @@ size_t cand_keys(int Q, int64_t e_stride) { return (size_t)Q * (size_t)(e_stride
 
 }  // namespace
 
-size_t index_zero_bytes(int Q) { return align256((size_t)Q * (kKeyBins + 2) * 4); }
+size_t index_zero_bytes(int Q) { return align256((size_t)Q * (kKeyBins + 6) * 4); }
 
 uint32_t* index_ready_words(void* ws, int Q) { return static_cast<uint32_t*>(ws) + (size_t)Q * kKeyBins; }
 
@@ -1088,6 +1227,8 @@ void index_ws_carve(IndexParams& p, void* ws, int Q, int64_t e_stride) {
     p.cand = reinterpret_cast<uint64_t*>(b);
     p.ready = nullptr;
     p.debug_fault = 0;
+    p.qsync = nullptr;
+    p.sms = 0;
     p.e_stride = e_stride;
     p.e_seg = e_stride + kSegPad;
     p.chunk = sp.chunk;
@@ -1123,6 +1264,9 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
     if (gx > p.max_chunks) return cudaErrorInvalidValue;  // the workspace was carved for fewer entries
     const dim3 grid((unsigned)gx, (unsigned)p.Q);
     const bool dep = pdl && !zero_ws;
+    // the scan grid selects itself when all of its CTAs fit the SMs at once (two per SM)
+    const bool fused = p.qsync && p.sms > 0 && gx * (int64_t)p.Q <= 2 * (int64_t)p.sms;
+    if (!fused) p.qsync = nullptr;
     // with the key histogram in static shared memory, the dynamic part needs the opt-in (per device)
     static PerDeviceOnce attr_scan;
     e = attr_scan.run([] {
@@ -1143,6 +1287,7 @@ cudaError_t launch_index_topk(IndexParams& p, int64_t max_entries, cudaStream_t 
                         : launch_kernel(index_scan_kernel<1, false>, grid, dim3(kScanThreads), kScanDynSmem, stream, dep, p);
     if (e != cudaSuccess) return e;
     if (mid && (e = cudaEventRecordWithFlags(mid, stream, cudaEventRecordExternal)) != cudaSuccess) return e;
+    if (fused) return cudaSuccess;
     // the exact selection: one cluster of kFinalF CTAs per query
     return launch_kernel_cluster(index_final_kernel, dim3(kFinalF, (unsigned)p.Q), dim3(kFinalThreads), kFinalDynSmem,
                                  stream, pdl, dim3(kFinalF, 1, 1), p);

@@ -96,6 +96,11 @@ struct IndexParams {
     // q's indices are out, for an attention grid that starts before the select grid ends
     uint32_t* ready;
     int debug_fault;          // 2 (tests of the bounded waits): the select publishes no ready word
+    // nullable: [Q, 4] words, zero before the scan.  When set and the scan grid fits the SMs at
+    // once (sms: the device's multiprocessor count), the scan grid selects the top-k itself (no
+    // final-select launch): its CTAs meet on these per-query counters
+    uint32_t* qsync;
+    int sms;
     // optional: rows of this cache (row stride prefetch_row_bytes, a multiple of 16) at the selected
     // entries are prefetched into L2 as soon as the selection is known (the attention's gather)
     const unsigned char* prefetch_rows;
@@ -108,7 +113,8 @@ struct IndexParams {
 size_t index_ws_bytes(int Q, int64_t e_stride);
 size_t index_zero_bytes(int Q);  // leading bytes of the index workspace that must start at zero
 // Per-step words of `ws` inside its leading zero bytes, after the histograms: Q ready words (see
-// IndexParams::ready), then Q item counters (see AttnParams::items_done).
+// IndexParams::ready), Q item counters (see AttnParams::items_done), then 4 Q scan counters (see
+// IndexParams::qsync).
 uint32_t* index_ready_words(void* ws, int Q);
 // Points the workspace arrays of `p` into `ws` and sets the scan chunking (chunk, max_chunks,
 // cand_cap), all derived from (Q, e_stride) exactly as index_ws_bytes sizes them.

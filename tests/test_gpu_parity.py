@@ -984,6 +984,23 @@ def test_decode_cluster_merge(cluster):
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
 
 
+def test_decode_with_the_selection_in_the_scan_grid():
+    """The optional exact top-k inside the scan grid (CSA_SCAN_SELECT=1, read once per process, so the
+    decode end-to-end cases rerun in a child process with it set): the chunks meet on per-query
+    counters, the last one selects, and the results equal the oracle's as in the two-kernel path."""
+    import os
+    import pathlib
+    import subprocess
+    import sys
+    here = pathlib.Path(__file__).resolve()
+    env = dict(os.environ, CSA_SCAN_SELECT="1")
+    cases = [f"{here}::test_decode_end_to_end", f"{here}::test_decode_with_norms_and_sinks",
+             f"{here}::test_decode_with_8bit_keys", f"{here}::test_ready_word_wait_runs_out_and_the_device_recovers"]
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider", *cases],
+                       cwd=here.parents[1], env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
+
+
 @pytest.mark.parametrize("N,rows,dims", [
     (1024, list(range(0, 1024, 7)) + [1023], workloads.TINY_DIMS),
     (3000, [0, 1, 2, 3, 4, 5, 127, 128, 129, 1023, 1024, 2047, 2048, 2999], SMALL_PROD)],
