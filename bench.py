@@ -31,7 +31,7 @@ METRIC = "CSA+HCA decode queries/s at 1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel source it
 # was taken on: the key is the SHA-256 prefix of csrc/index_topk.cu at that capture.  Any other
 # source reports null traffic until it is captured again.
-SCAN_TRAFFIC = {"source_sha256": "7aa945c5db1bbe37", "bytes": 134275328 + 5008128}
+SCAN_TRAFFIC = {"source_sha256": "0c71bf725604b67a", "bytes": 134291712 + 5024512}
 
 
 def _source_sha(name):
