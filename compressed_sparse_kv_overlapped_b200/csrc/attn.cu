@@ -26,6 +26,7 @@
 // loaders (cp.async for gathered rows with manual swizzle and zero-fill of masked slots; TMA for
 // full tiles of consecutive cache rows), warp 8 TMEM allocator + Q.K^T issuer, warp 9 P.V issuer.
 // Three key stages; every wait is bounded (kWaitLimitNs) and winds the CTA down on timeout.
+#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -79,7 +80,8 @@ struct Bars {
     uint64_t s_free[2];       // softmax finished reading S buffer t&1
     uint64_t p_full[2];       // softmax wrote P buffer t&1 (and rescaled O if needed)
     uint64_t o_done[2];       // MMA commit after the P.V that read P buffer t&1
-    uint64_t q_full;          // softmax warps stored Q in TMEM
+    uint64_t q_full;          // softmax warps stored Q in TMEM (once per query)
+    uint64_t q_empty;         // MMA commit after the last Q.K^T of a query: the Q region is free
     uint64_t fin;             // both MMA issuers committed before teardown
 };
 
@@ -146,57 +148,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     const uint32_t sbase = smem_u32(sm);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int qi = blockIdx.y, item = blockIdx.x + p_item_base;
+    int qi0 = blockIdx.y, item = blockIdx.x + p_item_base;
     if (p.hca_first) {
         const int n_hca = p.n_items - p.items_front;
         const int lin = blockIdx.x;
         if (lin < p.Q * n_hca) {
-            qi = lin / n_hca;
+            qi0 = lin / n_hca;
             item = p.items_front + lin % n_hca;
         } else {
-            qi = (lin - p.Q * n_hca) / p.items_front;
+            qi0 = (lin - p.Q * n_hca) / p.items_front;
             item = (lin - p.Q * n_hca) % p.items_front;
         }
     }
-    // The query table and sequence lengths: in the decode chain with an indexer they come from the
-    // append two launches back, complete once this grid runs (every kernel of the chain waits before
-    // it lets the next start); otherwise the previous launch may still be writing them.
-    if (!p.queries_early) grid_dep_wait();
-    const csa_query qr = p.queries[qi];
-    const bool seq_ok = qr.seq >= 0 && qr.reserved == 0;
-    const csa_seq sq = seq_ok ? p.seqs[qr.seq] : csa_seq{0, 0, 0, 0};
-    const bool qvalid = seq_ok && qr.len >= 1 && qr.len <= sq.len;
-    KeyList kl;
-    kl.idx = p.idx ? p.idx + (int64_t)qi * p.k_slots : nullptr;
-    kl.n_causal = qr.len / p.m;
-    kl.n_hca = (p.use_hca && qvalid) ? qr.len / p.m_hca : 0;
-    kl.nw = qr.len < p.W ? qr.len : p.W;
-    kl.win_row0 = sq.tok_off + qr.len - kl.nw;
-    kl.csa_row0 = sq.csa_off;
-    kl.hca_row0 = sq.hca_off;
-    const int64_t front = (int64_t)p.k_slots + p.W;
-    const int64_t n_keys = front + kl.n_hca;
-    int64_t s0, s1;
-    if (p.n_items == 1) {
-        s0 = 0;
-        s1 = n_keys;
-    } else if (item < p.items_front) {
-        s0 = (int64_t)item * p.kpi_front;
-        s1 = min(front, s0 + p.kpi_front);
-    } else {
-        s0 = front + (int64_t)(item - p.items_front) * p.kpi_hca;
-        s1 = min(n_keys, s0 + p.kpi_hca);
-    }
-    if (s1 < s0) s1 = s0;
-    if (!qvalid) {
-        if (threadIdx.x == 0 && item == 0) report(p.status, CSA_ERR_INDEX);
-        s1 = s0;
-    }
-    // once any CTA has given up on a wait, later CTAs do no work (bounded total time on a fault)
-    if (p.status && *reinterpret_cast<volatile int*>(p.status) == CSA_ERR_TIMEOUT) s1 = s0;
-    const int T = s1 > s0 ? (int)((s1 - s0 + kTileKeys - 1) / kTileKeys) : 0;
     const int n_items = p.n_items;
     const bool direct = n_items == 1;
+    // A direct launch with q_step > 0 is persistent: the CTA takes queries qi0, qi0 + q_step, ... and
+    // its pipeline (key stages, S and P buffers, barrier phases) runs on from one query to the next,
+    // so that the next query's key loads and Q.K^T products overlap this query's epilogue.
+    const int q_step = direct ? p.q_step : 0;
+    const int n_q = q_step > 0 ? (qi0 < p.Q ? (p.Q - 1 - qi0) / q_step + 1 : 0) : 1;
     const bool clustered = !direct && p.cluster > 1;
     const bool dep_wait = !(p.hca_nowait && !direct && item >= p.items_front);
     // front items with a ready word: the loaders poll it, nobody waits for the select grid up front
@@ -214,11 +184,60 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             mbar_init(&bars->o_done[i], 1);
         }
         mbar_init(&bars->q_full, 128);
+        mbar_init(&bars->q_empty, 1);
         mbar_init(&bars->fin, 2);
         misc[1] = 0;
+        // once any CTA has given up on a wait, later CTAs do no work (bounded total time on a fault);
+        // read once, so that every role of the CTA cuts the same key lists
+        misc[8] = (p.status && *reinterpret_cast<volatile int*>(p.status) == CSA_ERR_TIMEOUT) ? 1u : 0u;
         fence_mbar_init();
     }
-    if (warp == 8 && T > 0) {
+    __syncthreads();
+    const bool timed_out = misc[8] != 0u;
+    // The query table and sequence lengths: in the decode chain with an indexer they come from the
+    // append two launches back, complete once this grid runs (every kernel of the chain waits before
+    // it lets the next start); otherwise the previous launch may still be writing them.
+    if (!p.queries_early) grid_dep_wait();
+    // The key list of query qi and the slice [s0, s1) of it that this CTA attends; returns its number
+    // of key tiles.  Every role evaluates it for every query of the CTA.
+    const int64_t front = (int64_t)p.k_slots + p.W;
+    auto work = [&](int qi, KeyList& kl, int64_t& s0, int64_t& s1) -> int {
+        const csa_query qr = p.queries[qi];
+        const bool seq_ok = qr.seq >= 0 && qr.reserved == 0;
+        const csa_seq sq = seq_ok ? p.seqs[qr.seq] : csa_seq{0, 0, 0, 0};
+        const bool qvalid = seq_ok && qr.len >= 1 && qr.len <= sq.len;
+        kl.idx = p.idx ? p.idx + (int64_t)qi * p.k_slots : nullptr;
+        kl.n_causal = qr.len / p.m;
+        kl.n_hca = (p.use_hca && qvalid) ? qr.len / p.m_hca : 0;
+        kl.nw = qr.len < p.W ? qr.len : p.W;
+        kl.win_row0 = sq.tok_off + qr.len - kl.nw;
+        kl.csa_row0 = sq.csa_off;
+        kl.hca_row0 = sq.hca_off;
+        const int64_t n_keys = front + kl.n_hca;
+        if (direct) {
+            s0 = 0;
+            s1 = n_keys;
+        } else if (item < p.items_front) {
+            s0 = (int64_t)item * p.kpi_front;
+            s1 = min(front, s0 + p.kpi_front);
+        } else {
+            s0 = front + (int64_t)(item - p.items_front) * p.kpi_hca;
+            s1 = min(n_keys, s0 + p.kpi_hca);
+        }
+        if (s1 < s0) s1 = s0;
+        if (!qvalid) {
+            if (threadIdx.x == 0 && item == 0) report(p.status, CSA_ERR_INDEX);
+            s1 = s0;
+        }
+        if (timed_out) s1 = s0;
+        return s1 > s0 ? (int)((s1 - s0 + kTileKeys - 1) / kTileKeys) : 0;
+    };
+    KeyList kl0{};
+    int64_t s00 = 0, s10 = 0;
+    const int T0 = n_q > 0 ? work(qi0, kl0, s00, s10) : 0;
+    // tensor memory for a CTA with work (any query of a persistent CTA may have key tiles)
+    const bool use_tc = q_step > 0 ? n_q > 0 : T0 > 0;
+    if (warp == 8 && use_tc) {
         tmem_alloc(misc, kTmemCols);
         tmem_relinquish();
     }
@@ -244,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // end of its grid
         bool go = true;
         if (ready_wait) {
-            if (lane == 0) go = count_wait(p.ready + qi, 1u, p.status, abort_flag, p.wait_ns);
+            if (lane == 0) go = count_wait(p.ready + qi0, 1u, p.status, abort_flag, p.wait_ns);
             __syncwarp();  // orders the other lanes' reads after lane 0's acquire
             go = __shfl_sync(0xffffffffu, go ? 1 : 0, 0) != 0;
         } else if (dep_wait) {
@@ -254,131 +273,146 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             if (p.tma_hca) tma_prefetch_map(&maps.hca);
             if (p.tma_x) tma_prefetch_map(&maps.x);
         }
-        // the selected indices of this lane's rows in the first two tiles, read together (one memory
-        // latency, not one per tile); an address past the slots reads the last slot, unused
-        int32_t pre_j0 = -1, pre_j1 = -1;
-        const bool pre = go && kl.idx && s0 < p.k_slots && lane < 16;
-        if (pre) {
-            const int64_t sa = s0 + lw * 16 + lane, sb = sa + kTileKeys;
-            pre_j0 = kl.idx[sa < p.k_slots ? sa : p.k_slots - 1];
-            pre_j1 = kl.idx[sb < p.k_slots ? sb : p.k_slots - 1];
-        }
         // per stage, the full-barrier parity of the last tile this thread loaded by TMA (bit 2 set:
         // one is pending), so that a CTA that gives up waits for its own copies before it exits
         uint32_t tma_pend = 0;
-        for (int t = 0; go && t < T; ++t) {
-            const int st = t % kStages;
-            if (t >= kStages && !mbar_wait(&bars->empty[st], ((t / kStages) - 1) & 1, p.status, abort_flag, p.wait_ns)) break;
-            const int64_t tb = s0 + (int64_t)t * kTileKeys;
-            // A full tile of consecutive cache rows (HCA entries, or raw window tokens) goes by TMA:
-            // one thread issues the boxes, the tile's bytes complete the full barrier, and the
-            // loaders move on without waiting for the data.
-            const CUtensorMap* map = nullptr;
-            int64_t row = 0;
-            if (tb + kTileKeys <= s1) {
-                if (p.tma_hca && tb >= front && tb - front + kTileKeys <= kl.n_hca) {
-                    map = &maps.hca;
-                    row = kl.hca_row0 + (tb - front);
-                } else if (p.tma_x && tb >= p.k_slots && tb - p.k_slots + kTileKeys <= kl.nw) {
-                    map = &maps.x;
-                    row = kl.win_row0 + (tb - p.k_slots);
-                }
-                if (row < 0 || row > 0x7FFFFFFF - kTileKeys) map = nullptr;
+        uint32_t g = 0;  // key tiles of the CTA's earlier queries (the stage ring runs on)
+        for (int j = 0; go && j < n_q; ++j) {
+            KeyList kl = kl0;
+            int64_t s0 = s00, s1 = s10;
+            const int T = j == 0 ? T0 : work(qi0 + j * q_step, kl, s0, s1);
+            // the selected indices of this lane's rows in the query's first two tiles, read together
+            // (one memory latency, not one per tile); an address past the slots reads the last slot
+            int32_t pre_j0 = -1, pre_j1 = -1;
+            const bool pre = kl.idx && s0 < p.k_slots && lane < 16;
+            if (pre) {
+                const int64_t sa = s0 + lw * 16 + lane, sb = sa + kTileKeys;
+                pre_j0 = kl.idx[sa < p.k_slots ? sa : p.k_slots - 1];
+                pre_j1 = kl.idx[sb < p.k_slots ? sb : p.k_slots - 1];
             }
-            // fault injection (tests of the bounded waits): the first loader warp skips its arrival
-            // on the first tile, which therefore never becomes full
-            const bool skip = p.debug_fault == 1 && t == 0 && lw == 0;
-            if (map) {
-                if (lw == 0 && lane == 0) {
-                    for (int w4 = 0; w4 < 4; ++w4) mask16[st * 4 + w4] = 0xFFFFu;
-                    mbar_arrive_expect_tx(&bars->full[st], (uint32_t)(kTileKeys * D * 2));
-                    const uint32_t kdst = sbase + L::kK + (uint32_t)st * L::kStage;
-#pragma unroll
-                    for (int kb = 0; kb < L::NKB; ++kb)
-                        tma_load_2d(kdst + (uint32_t)kb * L::kBlock, map, kb * 64, (int)row, &bars->full[st]);
-                    tma_pend = (tma_pend & ~(7u << (3 * st))) | ((4u | (uint32_t)((t / kStages) & 1)) << (3 * st));
-                } else if (!skip) {
-                    mbar_arrive(&bars->full[st]);
+            for (int t = 0; t < T; ++t) {
+                const uint32_t gt = g + (uint32_t)t;
+                const int st = (int)(gt % kStages);
+                if (gt >= kStages &&
+                    !mbar_wait(&bars->empty[st], ((gt / kStages) - 1) & 1, p.status, abort_flag, p.wait_ns)) {
+                    go = false;
+                    break;
                 }
-                continue;
-            }
-            bool valid = false, fp4 = false;
-            if (lane < 16) {
-                const int64_t s = tb + lw * 16 + lane;
-                const uint8_t* scl = nullptr;
-                const void* r = s < s1 ? key_src(p, D, kl, s, &scl, pre && t < 2, t == 0 ? pre_j0 : pre_j1) : nullptr;
-                rowptr_w[lane] = reinterpret_cast<uint64_t>(r);
-                rowscl_w[lane] = reinterpret_cast<uint64_t>(scl);
-                valid = r != nullptr;
-                fp4 = FP4 && scl != nullptr;
-            }
-            const uint32_t vm = __ballot_sync(0xffffffffu, valid) & 0xFFFFu;
-            const bool tile_fp4 = __ballot_sync(0xffffffffu, fp4) != 0u;
-            __syncwarp();
-            const uint32_t kbase = sbase + L::kK + (uint32_t)st * L::kStage + lane_blk;
-            // a bf16 row (or an empty one: zeros) by cp.async, this lane's 16-byte chunks
-            auto copy_row = [&](int r) {
-                const uint16_t* row = reinterpret_cast<const uint16_t*>(rowptr[r]);
-                const int key = lw * 16 + r;
-                const uint32_t dst = kbase + (uint32_t)key * 128u + ((lane_c7 ^ (key & 7)) << 4);
-                const uint32_t nb = row ? 16u : 0u;
-                const uint16_t* src = row ? row : p.q;
-                if (CPR >= 32) {
-#pragma unroll
-                    for (int u = 0; u < CPL; ++u) cp_async16(dst + u * 4 * L::kBlock, src + (lane + 32 * u) * 8, nb);
-                } else if (lane < CPR) {
-                    cp_async16(dst, src + lane * 8, nb);
-                }
-            };
-            if (!FP4 || !tile_fp4) {
-#pragma unroll 4
-                for (int r = 0; r < 16; ++r) copy_row(r);
-                // the copies complete the tile's barrier phase themselves: no wait here, so the next
-                // tile's loads go out while these are still in flight
-                if (!skip) cp_async_mbar_arrive(&bars->full[st]);
-            } else {
-                // FP4 entries: chunk c of a row (channels 8c .. 8c+7) is the 4 code bytes at 4c and the
-                // scale byte c/4; dequantized in registers and stored into the tile's swizzled slot.
-                // The loads of all 16 rows are issued first, unconditionally (a row that is not FP4
-                // loads from the query instead and goes by cp.async), so the tile costs one memory
-                // latency; then the rows are converted.
-                constexpr int kFp4Rows = 16;
-#pragma unroll 1
-                for (int r0 = 0; r0 < 16; r0 += kFp4Rows) {
-                    uint32_t cw[kFp4Rows][CPL], sb[kFp4Rows][CPL];
-#pragma unroll
-                    for (int i = 0; i < kFp4Rows; ++i) {
-                        const uint8_t* sc = reinterpret_cast<const uint8_t*>(rowscl[r0 + i]);
-                        const uint8_t* cr = sc ? reinterpret_cast<const uint8_t*>(rowptr[r0 + i])
-                                               : reinterpret_cast<const uint8_t*>(p.q);
-                        const uint8_t* sr = sc ? sc : reinterpret_cast<const uint8_t*>(p.q);
-#pragma unroll
-                        for (int u = 0; u < CPL; ++u) {
-                            const int c = (lane + 32 * u) < CPR ? lane + 32 * u : 0;
-                            cw[i][u] = __ldg(reinterpret_cast<const unsigned int*>(cr + 4 * c));
-                            sb[i][u] = __ldg(sr + (c >> 2));
-                        }
+                const int64_t tb = s0 + (int64_t)t * kTileKeys;
+                // A full tile of consecutive cache rows (HCA entries, or raw window tokens) goes by TMA:
+                // one thread issues the boxes, the tile's bytes complete the full barrier, and the
+                // loaders move on without waiting for the data.
+                const CUtensorMap* map = nullptr;
+                int64_t row = 0;
+                if (tb + kTileKeys <= s1) {
+                    if (p.tma_hca && tb >= front && tb - front + kTileKeys <= kl.n_hca) {
+                        map = &maps.hca;
+                        row = kl.hca_row0 + (tb - front);
+                    } else if (p.tma_x && tb >= p.k_slots && tb - p.k_slots + kTileKeys <= kl.nw) {
+                        map = &maps.x;
+                        row = kl.win_row0 + (tb - p.k_slots);
                     }
+                    if (row < 0 || row > 0x7FFFFFFF - kTileKeys) map = nullptr;
+                }
+                // fault injection (tests of the bounded waits): the first loader warp skips its arrival
+                // on the first tile, which therefore never becomes full
+                const bool skip = p.debug_fault == 1 && gt == 0 && lw == 0;
+                if (map) {
+                    if (lw == 0 && lane == 0) {
+                        for (int w4 = 0; w4 < 4; ++w4) mask16[st * 4 + w4] = 0xFFFFu;
+                        mbar_arrive_expect_tx(&bars->full[st], (uint32_t)(kTileKeys * D * 2));
+                        const uint32_t kdst = sbase + L::kK + (uint32_t)st * L::kStage;
 #pragma unroll
-                    for (int i = 0; i < kFp4Rows; ++i) {
-                        const int r = r0 + i;
-                        if (rowscl[r] == 0) {
-                            copy_row(r);
-                            continue;
-                        }
-                        const int key = lw * 16 + r;
-                        const uint32_t dst = kbase + (uint32_t)key * 128u + ((lane_c7 ^ (key & 7)) << 4);
+                        for (int kb = 0; kb < L::NKB; ++kb)
+                            tma_load_2d(kdst + (uint32_t)kb * L::kBlock, map, kb * 64, (int)row, &bars->full[st]);
+                        tma_pend = (tma_pend & ~(7u << (3 * st))) | ((4u | ((gt / kStages) & 1u)) << (3 * st));
+                    } else if (!skip) {
+                        mbar_arrive(&bars->full[st]);
+                    }
+                    continue;
+                }
+                bool valid = false, fp4 = false;
+                if (lane < 16) {
+                    const int64_t s = tb + lw * 16 + lane;
+                    const uint8_t* scl = nullptr;
+                    const void* r =
+                        s < s1 ? key_src(p, D, kl, s, &scl, pre && t < 2, t == 0 ? pre_j0 : pre_j1) : nullptr;
+                    rowptr_w[lane] = reinterpret_cast<uint64_t>(r);
+                    rowscl_w[lane] = reinterpret_cast<uint64_t>(scl);
+                    valid = r != nullptr;
+                    fp4 = FP4 && scl != nullptr;
+                }
+                const uint32_t vm = __ballot_sync(0xffffffffu, valid) & 0xFFFFu;
+                const bool tile_fp4 = __ballot_sync(0xffffffffu, fp4) != 0u;
+                __syncwarp();
+                const uint32_t kbase = sbase + L::kK + (uint32_t)st * L::kStage + lane_blk;
+                // a bf16 row (or an empty one: zeros) by cp.async, this lane's 16-byte chunks
+                auto copy_row = [&](int r) {
+                    const uint16_t* row = reinterpret_cast<const uint16_t*>(rowptr[r]);
+                    const int key = lw * 16 + r;
+                    const uint32_t dst = kbase + (uint32_t)key * 128u + ((lane_c7 ^ (key & 7)) << 4);
+                    const uint32_t nb = row ? 16u : 0u;
+                    const uint16_t* src = row ? row : p.q;
+                    if (CPR >= 32) {
 #pragma unroll
                         for (int u = 0; u < CPL; ++u)
-                            if (lane + 32 * u < CPR) st_shared_v4(dst + u * 4 * L::kBlock, mx4_to_bf16x8(cw[i][u], sb[i][u]));
+                            cp_async16(dst + u * 4 * L::kBlock, src + (lane + 32 * u) * 8, nb);
+                    } else if (lane < CPR) {
+                        cp_async16(dst, src + lane * 8, nb);
                     }
+                };
+                if (!FP4 || !tile_fp4) {
+#pragma unroll 4
+                    for (int r = 0; r < 16; ++r) copy_row(r);
+                    // the copies complete the tile's barrier phase themselves: no wait here, so the next
+                    // tile's loads go out while these are still in flight
+                    if (!skip) cp_async_mbar_arrive(&bars->full[st]);
+                } else {
+                    // FP4 entries: chunk c of a row (channels 8c .. 8c+7) is the 4 code bytes at 4c and the
+                    // scale byte c/4; dequantized in registers and stored into the tile's swizzled slot.
+                    // The loads of all 16 rows are issued first, unconditionally (a row that is not FP4
+                    // loads from the query instead and goes by cp.async), so the tile costs one memory
+                    // latency; then the rows are converted.
+                    constexpr int kFp4Rows = 16;
+#pragma unroll 1
+                    for (int r0 = 0; r0 < 16; r0 += kFp4Rows) {
+                        uint32_t cw[kFp4Rows][CPL], sb[kFp4Rows][CPL];
+#pragma unroll
+                        for (int i = 0; i < kFp4Rows; ++i) {
+                            const uint8_t* sc = reinterpret_cast<const uint8_t*>(rowscl[r0 + i]);
+                            const uint8_t* cr = sc ? reinterpret_cast<const uint8_t*>(rowptr[r0 + i])
+                                                   : reinterpret_cast<const uint8_t*>(p.q);
+                            const uint8_t* sr = sc ? sc : reinterpret_cast<const uint8_t*>(p.q);
+#pragma unroll
+                            for (int u = 0; u < CPL; ++u) {
+                                const int c = (lane + 32 * u) < CPR ? lane + 32 * u : 0;
+                                cw[i][u] = __ldg(reinterpret_cast<const unsigned int*>(cr + 4 * c));
+                                sb[i][u] = __ldg(sr + (c >> 2));
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < kFp4Rows; ++i) {
+                            const int r = r0 + i;
+                            if (rowscl[r] == 0) {
+                                copy_row(r);
+                                continue;
+                            }
+                            const int key = lw * 16 + r;
+                            const uint32_t dst = kbase + (uint32_t)key * 128u + ((lane_c7 ^ (key & 7)) << 4);
+#pragma unroll
+                            for (int u = 0; u < CPL; ++u)
+                                if (lane + 32 * u < CPR)
+                                    st_shared_v4(dst + u * 4 * L::kBlock, mx4_to_bf16x8(cw[i][u], sb[i][u]));
+                        }
+                    }
+                    cp_async_wait_all();
+                    fence_proxy_async_smem();
                 }
-                cp_async_wait_all();
-                fence_proxy_async_smem();
+                if (lane == 0) mask16[st * 4 + lw] = (uint16_t)vm;
+                __syncwarp();
+                if (!skip) mbar_arrive(&bars->full[st]);
             }
-            if (lane == 0) mask16[st * 4 + lw] = (uint16_t)vm;
-            __syncwarp();
-            if (!skip) mbar_arrive(&bars->full[st]);
+            g += (uint32_t)T;
         }
         cp_async_wait_all();
         if (*abort_flag && tma_pend) {
@@ -396,53 +430,81 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // independently, so a P.V never waits behind the issue of the next Q.K^T.  Each warp runs
         // its loop with all lanes (warp-uniform waits and operands; one elected lane issues).
         if (dep_wait && !ready_wait) grid_dep_wait();
-        if (T > 0) {
+        if (use_tc) {
+            // g: key tiles of the CTA's earlier queries (stage, S and P buffer phases run on)
+            uint32_t g = 0;
+            bool ok = true;
             if (warp == 8) {
                 constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
-                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_full, 0, p.status, abort_flag, p.wait_ns));
-                for (int g1 = 0; ok && g1 < T; ++g1) {
-                    const int st = g1 % kStages;
-                    bool w = mbar_wait(&bars->full[st], (g1 / kStages) & 1, p.status, abort_flag, p.wait_ns);
-                    if (w && g1 >= 2) w = mbar_wait(&bars->s_free[g1 & 1], ((g1 >> 1) - 1) & 1, p.status, abort_flag, p.wait_ns);
-                    if (!__all_sync(0xffffffffu, w)) break;
-                    tc_fence_after();
-                    fence_proxy_async_smem();  // the tile's cp.async writes, observed through the barrier
-                    const uint64_t kd = sdesc_kmajor(sbase + L::kK + (uint32_t)st * L::kStage);
-                    const uint32_t tS = tmem + kColS + (uint32_t)(g1 & 1) * 64u;
-#pragma unroll
-                    for (int kb = 0; kb < L::NKB; ++kb) {
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) {
-                            // K elements [64 kb + 16 ks, +16): columns 32 kb + 8 ks of Q, bytes of the tile block
-                            umma_bf16_ts(tS, tmem + (uint32_t)(kb * 32 + ks * 8),
-                                         kd + (uint64_t)((kb * L::kBlock + ks * 32) >> 4), id1, (kb | ks) != 0);
+                for (int j = 0; ok && j < n_q; ++j) {
+                    KeyList kl = kl0;
+                    int64_t s0 = s00, s1 = s10;
+                    const int T = j == 0 ? T0 : work(qi0 + j * q_step, kl, s0, s1);
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&bars->q_full, (uint32_t)j & 1u, p.status, abort_flag, p.wait_ns));
+                    for (int t = 0; ok && t < T; ++t) {
+                        const uint32_t gt = g + (uint32_t)t;
+                        const int st = (int)(gt % kStages);
+                        bool w = mbar_wait(&bars->full[st], (gt / kStages) & 1, p.status, abort_flag, p.wait_ns);
+                        if (w && gt >= 2)
+                            w = mbar_wait(&bars->s_free[gt & 1], ((gt >> 1) - 1) & 1, p.status, abort_flag, p.wait_ns);
+                        if (!__all_sync(0xffffffffu, w)) {
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after();
+                        fence_proxy_async_smem();  // the tile's cp.async writes, observed through the barrier
+                        const uint64_t kd = sdesc_kmajor(sbase + L::kK + (uint32_t)st * L::kStage);
+                        const uint32_t tS = tmem + kColS + (gt & 1u) * 64u;
+#pragma unroll
+                        for (int kb = 0; kb < L::NKB; ++kb) {
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks) {
+                                // K elements [64 kb + 16 ks, +16): columns 32 kb + 8 ks of Q, bytes of the tile block
+                                umma_bf16_ts(tS, tmem + (uint32_t)(kb * 32 + ks * 8),
+                                             kd + (uint64_t)((kb * L::kBlock + ks * 32) >> 4), id1, (kb | ks) != 0);
+                            }
+                        }
+                        umma_commit(&bars->s_full[gt & 1]);
                     }
-                    umma_commit(&bars->s_full[g1 & 1]);
+                    // the query's products have read Q once this completes: the next Q may be stored
+                    umma_commit(&bars->q_empty);
+                    g += (uint32_t)T;
                 }
             } else {
                 constexpr int N2 = D >= 256 ? 256 : D;
                 constexpr int HALVES = D >= 256 ? D / 256 : 1;
                 constexpr uint32_t id2 = idesc_bf16(64, N2, false, true);
-                for (int g2 = 0; g2 < T; ++g2) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bars->p_full[g2 & 1], (g2 >> 1) & 1, p.status, abort_flag, p.wait_ns)))
-                        break;
-                    tc_fence_after();
-                    const int st = g2 % kStages;
-                    const uint64_t vd = sdesc_mnmajor(sbase + L::kK + (uint32_t)st * L::kStage, L::kBlock);
-                    const uint64_t pd = sdesc_kmajor(sbase + ((g2 & 1) ? L::kP1 : L::kP0));
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-                        for (int half = 0; half < HALVES; ++half) {
-                            // V rows ks*16 .. ks*16+15 of the key tile, dims [half*256, half*256 + N2)
-                            const uint64_t b = vd + (uint64_t)((half * 4 * L::kBlock + ks * 16 * 128) >> 4);
-                            const uint32_t tO = tmem + (kLaneO << 16) + (uint32_t)(half * 256);
-                            umma_bf16(tO, pd + (uint64_t)((ks * 32) >> 4), b, id2, (g2 > 0 || ks > 0) ? 1u : 0u);
+                for (int j = 0; ok && j < n_q; ++j) {
+                    KeyList kl = kl0;
+                    int64_t s0 = s00, s1 = s10;
+                    const int T = j == 0 ? T0 : work(qi0 + j * q_step, kl, s0, s1);
+                    for (int t = 0; t < T; ++t) {
+                        const uint32_t gt = g + (uint32_t)t;
+                        const bool w = mbar_wait(&bars->p_full[gt & 1], (gt >> 1) & 1, p.status, abort_flag, p.wait_ns);
+                        if (!__all_sync(0xffffffffu, w)) {
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after();
+                        const int st = (int)(gt % kStages);
+                        const uint64_t vd = sdesc_mnmajor(sbase + L::kK + (uint32_t)st * L::kStage, L::kBlock);
+                        const uint64_t pd = sdesc_kmajor(sbase + ((gt & 1u) ? L::kP1 : L::kP0));
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+                            for (int half = 0; half < HALVES; ++half) {
+                                // V rows ks*16 .. ks*16+15 of the key tile, dims [half*256, half*256 + N2);
+                                // the query's first product overwrites O
+                                const uint64_t b = vd + (uint64_t)((half * 4 * L::kBlock + ks * 16 * 128) >> 4);
+                                const uint32_t tO = tmem + (kLaneO << 16) + (uint32_t)(half * 256);
+                                umma_bf16(tO, pd + (uint64_t)((ks * 32) >> 4), b, id2, (t > 0 || ks > 0) ? 1u : 0u);
+                            }
+                        }
+                        umma_commit(&bars->empty[st]);
+                        umma_commit(&bars->o_done[gt & 1]);
                     }
-                    umma_commit(&bars->empty[st]);
-                    umma_commit(&bars->o_done[g2 & 1]);
+                    g += (uint32_t)T;
                 }
             }
             umma_commit(&bars->fin);
@@ -453,11 +515,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // ------------------------------------------------------------------ softmax + epilogue
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const uint32_t o_base = tmem + lane_base + (kLaneO << 16);
-        if (T > 0) {
-            // Q (an input, so before the wait) in the A layout of Q.K^T: head row 16w + r in lane r
-            // of warp w's sub-partition, dims 2c and 2c + 1 in column c.  Written with the 16x256b
-            // shape, so every lane takes part: lane i writes rows i/4 and i/4 + 8 at columns
-            // 8k + 2(i%4) and 8k + 2(i%4) + 1, i.e. 8 bytes of each of those rows per 8 columns.
+        // Q of query qi (an input, so the first one before the wait) in the A layout of Q.K^T: head
+        // row 16w + r in lane r of warp w's sub-partition, dims 2c and 2c + 1 in column c.  Written
+        // with the 16x256b shape, so every lane takes part: lane i writes rows i/4 and i/4 + 8 at
+        // columns 8k + 2(i%4) and 8k + 2(i%4) + 1, i.e. 8 bytes of each of those rows per 8 columns.
+        // The j-th query of the CTA (j > 0) stores its Q once the products of query j - 1 are done
+        // with the region (q_empty); its loads are issued before that wait.
+        auto load_q = [&](int qi, int j) -> bool {
             const int qa = lane >> 2, qc = (lane & 3) * 2;
             const int h0 = warp * 16 + qa, h1 = h0 + 8;
             const uint2* q0 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h0 < p.H ? h0 : 0)) * D);
@@ -528,6 +592,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                         r[g][4 * k + 3] = u1 ? r[g][4 * k + 3] : 0u;
                     }
                 }
+                if (cb == 0 && j > 0) {
+                    if (!mbar_wait(&bars->q_empty, (uint32_t)(j - 1) & 1u, p.status, abort_flag, p.wait_ns))
+                        return false;
+                    tc_fence_after();
+                }
 #pragma unroll
                 for (int g = 0; g < 2; ++g)
                     if (cb + g * 64 < D / 2) tmem_st_16x256_x8(tmem + lane_base + (uint32_t)(cb + g * 64), r[g]);
@@ -535,7 +604,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars->q_full);
-        }
+            return true;
+        };
+        bool ok = true;
+        if (use_tc) ok = load_q(qi0, 0);
         if (dep_wait && !ready_wait) grid_dep_wait();
         grid_dep_launch();
         const int i = lane;
@@ -544,204 +616,224 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // the four lanes of a quad share a row and combine their partial max / sum by shuffles.
         const int ra = i >> 2, cq = (i & 3) * 2;
         const int hr[2] = {warp * 16 + ra, warp * 16 + ra + 8};
-        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-        bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int sb = t & 1, st = t % kStages;
-            ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, p.status, abort_flag, p.wait_ns) &&
-                 mbar_wait(&bars->full[st], (t / kStages) & 1, p.status, abort_flag, p.wait_ns);
-            if (!ok) break;
-            tc_fence_after();
-            float s[2][16];  // [row ra / ra+8][2k + e] = column 8k + cq + e
-            {
-                uint32_t r[32];
-                tmem_ld_16x256_x8(tmem + lane_base + kColS + (uint32_t)sb * 64u, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    s[0][2 * k] = __uint_as_float(r[4 * k]);
-                    s[0][2 * k + 1] = __uint_as_float(r[4 * k + 1]);
-                    s[1][2 * k] = __uint_as_float(r[4 * k + 2]);
-                    s[1][2 * k + 1] = __uint_as_float(r[4 * k + 3]);
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&bars->s_free[sb]);
-            const uint64_t vmask = (uint64_t)mask16[st * 4 + 0] | ((uint64_t)mask16[st * 4 + 1] << 16) |
-                                   ((uint64_t)mask16[st * 4 + 2] << 32) | ((uint64_t)mask16[st * 4 + 3] << 48);
-            const float sc = p.scale_log2;
-            float mx[2] = {-INFINITY, -INFINITY};
-            const uint64_t lm = vmask >> cq;  // bit 8k + e: column 8k + cq + e valid
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const bool v = (lm >> (8 * k + e)) & 1ull;
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        s[rr][2 * k + e] = v ? s[rr][2 * k + e] * sc : -INFINITY;
-                        mx[rr] = fmaxf(mx[rr], s[rr][2 * k + e]);
-                    }
-                }
-            }
-            float alpha[2] = {1.f, 1.f};
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
-                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
-                // lazy rescaling: move the reference max only when it grows by more than 2^8
-                if (mx[rr] > m_run[rr] + 8.f) {
-                    alpha[rr] = (m_run[rr] == -INFINITY) ? 0.f : exp2f(m_run[rr] - mx[rr]);
-                    m_run[rr] = mx[rr];
-                    l_run[rr] *= alpha[rr];
-                }
-            }
-            // O must hold every earlier P.V before it is rescaled (rare); O lives in lanes 16-31,
-            // in the same row / column layout as S
-            const bool any = __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f);
-            if (t > 0 && any) {
-                ok = mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, p.status, abort_flag, p.wait_ns);
+        uint32_t g = 0;  // key tiles of the CTA's earlier queries
+        KeyList kl = kl0;
+        int64_t s0 = s00, s1 = s10;
+        int T = T0;
+        for (int j = 0; j < n_q; ++j) {
+            const int qi = qi0 + j * q_step;
+            float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+            for (int t = 0; ok && t < T; ++t) {
+                const uint32_t gt = g + (uint32_t)t;
+                const int sb = (int)(gt & 1u), st = (int)(gt % kStages);
+                ok = mbar_wait(&bars->s_full[sb], (gt >> 1) & 1, p.status, abort_flag, p.wait_ns) &&
+                     mbar_wait(&bars->full[st], (gt / kStages) & 1, p.status, abort_flag, p.wait_ns);
                 if (!ok) break;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < D; c += 64) {
+                float s[2][16];  // [row ra / ra+8][2k + e] = column 8k + cq + e
+                {
                     uint32_t r[32];
-                    tmem_ld_16x256_x8(o_base + (uint32_t)c, r);
+                    tmem_ld_16x256_x8(tmem + lane_base + kColS + (uint32_t)sb * 64u, r);
                     tmem_ld_wait();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
-                        r[4 * k] = __float_as_uint(__uint_as_float(r[4 * k]) * alpha[0]);
-                        r[4 * k + 1] = __float_as_uint(__uint_as_float(r[4 * k + 1]) * alpha[0]);
-                        r[4 * k + 2] = __float_as_uint(__uint_as_float(r[4 * k + 2]) * alpha[1]);
-                        r[4 * k + 3] = __float_as_uint(__uint_as_float(r[4 * k + 3]) * alpha[1]);
+                        s[0][2 * k] = __uint_as_float(r[4 * k]);
+                        s[0][2 * k + 1] = __uint_as_float(r[4 * k + 1]);
+                        s[1][2 * k] = __uint_as_float(r[4 * k + 2]);
+                        s[1][2 * k + 1] = __uint_as_float(r[4 * k + 3]);
                     }
-                    tmem_st_16x256_x8(o_base + (uint32_t)c, r);
                 }
-                tmem_st_wait();
-            }
-            // P buffer t&1 is free once the P.V of tile t-2 finished
-            if (t >= 2) {
-                ok = mbar_wait(&bars->o_done[sb], ((t >> 1) - 1) & 1, p.status, abort_flag, p.wait_ns);
-                if (!ok) break;
-            }
-            {
-                // masked slots hold -inf: 2^(-inf - m) = 0; while a row has seen no key, m_use = 0
-                const uint32_t prow = sbase + (sb ? L::kP1 : L::kP0) + (uint32_t)(i & 3) * 4u;
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const float m_use = m_run[rr] == -INFINITY ? 0.f : m_run[rr];
-                    float lsum = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float p0 = fast_exp2(s[rr][2 * k] - m_use);
-                        const float p1 = fast_exp2(s[rr][2 * k + 1] - m_use);
-                        lsum += p0 + p1;
-                        asm volatile("st.shared.b32 [%0], %1;" ::"r"(prow + sw128_offset(hr[rr], k)),
-                                     "r"(pack_bf16x2(p0, p1))
-                                     : "memory");
-                    }
-                    l_run[rr] += lsum;  // this lane's part of the row sum; the quad adds them up at the end
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars->p_full[sb]);
-        }
-        // ---- epilogue: TMEM -> registers -> global memory
-        if (ok && T > 0) ok = mbar_wait(&bars->o_done[(T - 1) & 1], ((T - 1) >> 1) & 1, p.status, abort_flag, p.wait_ns);
-        float inv[2], lse2[2];  // lse2: log-sum-exp in log2 units
-        bool has[2];
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-            l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
-            l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
-            has[rr] = ok && T > 0 && l_run[rr] > 0.f;
-            inv[rr] = has[rr] ? 1.f / l_run[rr] : 0.f;
-            lse2[rr] = has[rr] ? m_run[rr] + log2f(l_run[rr]) : -INFINITY;
-            // a single item holds the query's whole softmax: its sink logit (one more term with a zero
-            // value) joins here; with several items it joins in the merge
-            const float z = (direct && p.sink && hr[rr] < p.H) ? p.sink[hr[rr]] * 1.4426950408889634f : -INFINITY;
-            if (z > -INFINITY && (ok || T == 0)) {
-                const float m_eff = has[rr] ? fmaxf(m_run[rr], z) : z;
-                const float a = has[rr] ? exp2f(m_run[rr] - m_eff) : 0.f;
-                const float l_eff = fmaf(l_run[rr], a, exp2f(z - m_eff));
-                inv[rr] = a / l_eff;
-                lse2[rr] = m_eff + log2f(l_eff);
-            }
-        }
-        const bool write_o = ok && T > 0;
-        const int rows = p.H < kHeadsPad ? p.H : kHeadsPad;
-        const bool to_smem = clustered;  // the cluster merges its CTAs' results in shared memory
-        float* o_smem = reinterpret_cast<float*>(sm + L::kK);
-        if (write_o) {
-            // straight from the registers: per row, the four lanes of a quad write 32 consecutive
-            // bytes (one full sector) per instruction
-            float* dst[2];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr)
-                dst[rr] = to_smem ? o_smem + hr[rr] * L::kOStride
-                          : direct ? p.out + ((int64_t)qi * p.H + hr[rr]) * D
-                                   : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + hr[rr]) * D;
-            tc_fence_after();
-            // two register buffers: the TMEM load of the next 64 columns is in flight while the
-            // current ones are stored
-            auto store64 = [&](const uint32_t (&r)[32], int c) {
+                tc_fence_before();
+                mbar_arrive(&bars->s_free[sb]);
+                const uint64_t vmask = (uint64_t)mask16[st * 4 + 0] | ((uint64_t)mask16[st * 4 + 1] << 16) |
+                                       ((uint64_t)mask16[st * 4 + 2] << 32) | ((uint64_t)mask16[st * 4 + 3] << 48);
+                const float sc = p.scale_log2;
+                float mx[2] = {-INFINITY, -INFINITY};
+                const uint64_t lm = vmask >> cq;  // bit 8k + e: column 8k + cq + e valid
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const int col = c + 8 * k + cq;
-                    if (hr[0] < rows)
-                        *reinterpret_cast<float2*>(dst[0] + col) =
-                            make_float2(__uint_as_float(r[4 * k]) * inv[0], __uint_as_float(r[4 * k + 1]) * inv[0]);
-                    if (hr[1] < rows)
-                        *reinterpret_cast<float2*>(dst[1] + col) = make_float2(__uint_as_float(r[4 * k + 2]) * inv[1],
-                                                                             __uint_as_float(r[4 * k + 3]) * inv[1]);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool v = (lm >> (8 * k + e)) & 1ull;
+#pragma unroll
+                        for (int rr = 0; rr < 2; ++rr) {
+                            s[rr][2 * k + e] = v ? s[rr][2 * k + e] * sc : -INFINITY;
+                            mx[rr] = fmaxf(mx[rr], s[rr][2 * k + e]);
+                        }
+                    }
                 }
-            };
-            static_assert(D % 128 == 0, "column chunks come in pairs");
-            uint32_t ra[32], rb[32];
-            tmem_ld_16x256_x8(o_base, ra);
-            tmem_ld_wait();
+                float alpha[2] = {1.f, 1.f};
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+                    mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+                    // lazy rescaling: move the reference max only when it grows by more than 2^8
+                    if (mx[rr] > m_run[rr] + 8.f) {
+                        alpha[rr] = (m_run[rr] == -INFINITY) ? 0.f : exp2f(m_run[rr] - mx[rr]);
+                        m_run[rr] = mx[rr];
+                        l_run[rr] *= alpha[rr];
+                    }
+                }
+                // O must hold every earlier P.V before it is rescaled (rare); O lives in lanes 16-31,
+                // in the same row / column layout as S
+                const bool any = __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f);
+                if (t > 0 && any) {
+                    ok = mbar_wait(&bars->o_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, p.status, abort_flag, p.wait_ns);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < D; c += 128) {
-                tmem_ld_16x256_x8(o_base + (uint32_t)(c + 64), rb);
-                store64(ra, c);
-                tmem_ld_wait();
-                if (c + 128 < D) tmem_ld_16x256_x8(o_base + (uint32_t)(c + 128), ra);
-                store64(rb, c + 64);
-                tmem_ld_wait();
+                    for (int c = 0; c < D; c += 64) {
+                        uint32_t r[32];
+                        tmem_ld_16x256_x8(o_base + (uint32_t)c, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            r[4 * k] = __float_as_uint(__uint_as_float(r[4 * k]) * alpha[0]);
+                            r[4 * k + 1] = __float_as_uint(__uint_as_float(r[4 * k + 1]) * alpha[0]);
+                            r[4 * k + 2] = __float_as_uint(__uint_as_float(r[4 * k + 2]) * alpha[1]);
+                            r[4 * k + 3] = __float_as_uint(__uint_as_float(r[4 * k + 3]) * alpha[1]);
+                        }
+                        tmem_st_16x256_x8(o_base + (uint32_t)c, r);
+                    }
+                    tmem_st_wait();
+                }
+                // P buffer t&1 is free once the P.V of tile t-2 finished
+                if (gt >= 2) {
+                    ok = mbar_wait(&bars->o_done[sb], ((gt >> 1) - 1) & 1, p.status, abort_flag, p.wait_ns);
+                    if (!ok) break;
+                }
+                {
+                    // masked slots hold -inf: 2^(-inf - m) = 0; while a row has seen no key, m_use = 0
+                    const uint32_t prow = sbase + (sb ? L::kP1 : L::kP0) + (uint32_t)(i & 3) * 4u;
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const float m_use = m_run[rr] == -INFINITY ? 0.f : m_run[rr];
+                        float lsum = 0.f;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const float p0 = fast_exp2(s[rr][2 * k] - m_use);
+                            const float p1 = fast_exp2(s[rr][2 * k + 1] - m_use);
+                            lsum += p0 + p1;
+                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(prow + sw128_offset(hr[rr], k)),
+                                         "r"(pack_bf16x2(p0, p1))
+                                         : "memory");
+                        }
+                        l_run[rr] += lsum;  // this lane's part of the row sum; the quad adds them up at the end
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bars->p_full[sb]);
             }
-        } else if (direct) {
-            const int tid = threadIdx.x;  // 0..127
-            for (int e = tid; e < rows * (D / 4); e += 128) {
-                const int hh = e / (D / 4), c4 = e % (D / 4);
-                *reinterpret_cast<float4*>(p.out + ((int64_t)qi * p.H + hh) * D + c4 * 4) =
-                    make_float4(0.f, 0.f, 0.f, 0.f);
+            const int Tq = T;
+            const uint32_t gq = g;
+            g += (uint32_t)T;
+            // the next query of a persistent CTA: its key list, and its Q stored as soon as this query's
+            // products are done with Q, ahead of this query's epilogue, so that the next products start
+            // while this query's output is stored
+            if (j + 1 < n_q) {
+                T = work(qi + q_step, kl, s0, s1);
+                if (ok) ok = load_q(qi + q_step, j + 1);
             }
-        }
-        if ((i & 3) == 0) {
+            // ---- epilogue: TMEM -> registers -> global memory
+            if (ok && Tq > 0) {
+                const uint32_t gl = gq + (uint32_t)Tq - 1u;
+                ok = mbar_wait(&bars->o_done[gl & 1], (gl >> 1) & 1, p.status, abort_flag, p.wait_ns);
+            }
+            float inv[2], lse2[2];  // lse2: log-sum-exp in log2 units
+            bool has[2];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
-                const int h = hr[rr];
-                if (h >= p.H) continue;
-                const float lse_v = lse2[rr] * 0.69314718055994531f;
-                if (direct) {
-                    if (p.lse) p.lse[(int64_t)qi * p.H + h] = lse_v;
-                } else if (to_smem) {
-                    reinterpret_cast<float*>(sm + L::kP0)[h] = lse_v;
-                } else {
-                    p.part_lse[((int64_t)qi * n_items + item) * kHeadsPad + h] = lse_v;
+                l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
+                l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
+                has[rr] = ok && Tq > 0 && l_run[rr] > 0.f;
+                inv[rr] = has[rr] ? 1.f / l_run[rr] : 0.f;
+                lse2[rr] = has[rr] ? m_run[rr] + log2f(l_run[rr]) : -INFINITY;
+                // a single item holds the query's whole softmax: its sink logit (one more term with a zero
+                // value) joins here; with several items it joins in the merge
+                const float z = (direct && p.sink && hr[rr] < p.H) ? p.sink[hr[rr]] * 1.4426950408889634f : -INFINITY;
+                if (z > -INFINITY && (ok || Tq == 0)) {
+                    const float m_eff = has[rr] ? fmaxf(m_run[rr], z) : z;
+                    const float a = has[rr] ? exp2f(m_run[rr] - m_eff) : 0.f;
+                    const float l_eff = fmaf(l_run[rr], a, exp2f(z - m_eff));
+                    inv[rr] = a / l_eff;
+                    lse2[rr] = m_eff + log2f(l_eff);
                 }
             }
-            if (to_smem && (i & 3) == 0)  // rows of heads past H: no contribution
+            const bool write_o = ok && Tq > 0;
+            const int rows = p.H < kHeadsPad ? p.H : kHeadsPad;
+            const bool to_smem = clustered;  // the cluster merges its CTAs' results in shared memory
+            float* o_smem = reinterpret_cast<float*>(sm + L::kK);
+            if (write_o) {
+                // straight from the registers: per row, the four lanes of a quad write 32 consecutive
+                // bytes (one full sector) per instruction
+                float* dst[2];
+#pragma unroll
                 for (int rr = 0; rr < 2; ++rr)
-                    if (hr[rr] >= p.H) reinterpret_cast<float*>(sm + L::kP0)[hr[rr]] = -INFINITY;
-        }
+                    dst[rr] = to_smem ? o_smem + hr[rr] * L::kOStride
+                              : direct ? p.out + ((int64_t)qi * p.H + hr[rr]) * D
+                                       : p.part_o + (((int64_t)qi * n_items + item) * kHeadsPad + hr[rr]) * D;
+                tc_fence_after();
+                // two register buffers: the TMEM load of the next 64 columns is in flight while the
+                // current ones are stored
+                auto store64 = [&](const uint32_t (&r)[32], int c) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int col = c + 8 * k + cq;
+                        if (hr[0] < rows)
+                            *reinterpret_cast<float2*>(dst[0] + col) =
+                                make_float2(__uint_as_float(r[4 * k]) * inv[0], __uint_as_float(r[4 * k + 1]) * inv[0]);
+                        if (hr[1] < rows)
+                            *reinterpret_cast<float2*>(dst[1] + col) = make_float2(__uint_as_float(r[4 * k + 2]) * inv[1],
+                                                                                 __uint_as_float(r[4 * k + 3]) * inv[1]);
+                    }
+                };
+                static_assert(D % 128 == 0, "column chunks come in pairs");
+                uint32_t ra[32], rb[32];
+                tmem_ld_16x256_x8(o_base, ra);
+                tmem_ld_wait();
+#pragma unroll 1
+                for (int c = 0; c < D; c += 128) {
+                    tmem_ld_16x256_x8(o_base + (uint32_t)(c + 64), rb);
+                    store64(ra, c);
+                    tmem_ld_wait();
+                    if (c + 128 < D) tmem_ld_16x256_x8(o_base + (uint32_t)(c + 128), ra);
+                    store64(rb, c + 64);
+                    tmem_ld_wait();
+                }
+            } else if (direct) {
+                const int tid = threadIdx.x;  // 0..127
+                for (int e = tid; e < rows * (D / 4); e += 128) {
+                    const int hh = e / (D / 4), c4 = e % (D / 4);
+                    *reinterpret_cast<float4*>(p.out + ((int64_t)qi * p.H + hh) * D + c4 * 4) =
+                        make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            if ((i & 3) == 0) {
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int h = hr[rr];
+                    if (h >= p.H) continue;
+                    const float lse_v = lse2[rr] * 0.69314718055994531f;
+                    if (direct) {
+                        if (p.lse) p.lse[(int64_t)qi * p.H + h] = lse_v;
+                    } else if (to_smem) {
+                        reinterpret_cast<float*>(sm + L::kP0)[h] = lse_v;
+                    } else {
+                        p.part_lse[((int64_t)qi * n_items + item) * kHeadsPad + h] = lse_v;
+                    }
+                }
+                if (to_smem && (i & 3) == 0)  // rows of heads past H: no contribution
+                    for (int rr = 0; rr < 2; ++rr)
+                        if (hr[rr] >= p.H) reinterpret_cast<float*>(sm + L::kP0)[hr[rr]] = -INFINITY;
+            }
+        }  // queries of the CTA
     }
     // the select grid is complete before this one is (the merge that waits for this grid relies on it)
     if (ready_wait) grid_dep_wait();
     tc_fence_before();
     __syncthreads();
-    if (warp == 8 && T > 0) {
+    if (warp == 8 && use_tc) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -799,18 +891,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 acc.w = fmaf(w[c], v[c].w, acc.w);
             }
             if (h < p.H)
-                *reinterpret_cast<float4*>(p.part_o + (((int64_t)qi * n_parts + part) * kHeadsPad + h) * D + col) = acc;
+                *reinterpret_cast<float4*>(p.part_o + (((int64_t)qi0 * n_parts + part) * kHeadsPad + h) * D + col) =
+                    acc;
         }
         if (rank == 0)
             for (int h = threadIdx.x; h < kHeadsPad; h += kThreads)
-                p.part_lse[((int64_t)qi * n_parts + part) * kHeadsPad + h] = mlse[h];
+                p.part_lse[((int64_t)qi0 * n_parts + part) * kHeadsPad + h] = mlse[h];
         cluster_barrier();  // no CTA leaves while another still reads its shared memory
     }
     if (p.items_done && !direct) {
         __syncthreads();  // every partial store of the CTA precedes the count
         if (threadIdx.x == 0) {
             __threadfence();
-            atomicAdd(p.items_done + qi, 1u);
+            atomicAdd(p.items_done + qi0, 1u);
         }
     }
 }
@@ -901,6 +994,19 @@ __global__ void combine_kernel(AttnParams p) {
     *reinterpret_cast<float4*>(p.out + ((int64_t)qi * p.H + h) * D + c) = acc;
 }
 
+// Multiprocessors of the current device (0 if unknown), cached per device.
+int device_sms() {
+    static std::atomic<int> counts[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    int v = counts[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        counts[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
 template <int D>
 cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, cudaStream_t stream, bool pdl) {
     using L = Smem<D>;
@@ -913,7 +1019,7 @@ cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, 
     });
     if (ea != cudaSuccess) return ea;
     auto kernel = (p.entries_q || p.hca_q) ? attn_kernel<D, true> : attn_kernel<D, false>;
-    const dim3 grid = p.hca_first ? dim3((unsigned)(p.n_items * p.Q)) : dim3((unsigned)item_count, (unsigned)p.Q);
+    dim3 grid = p.hca_first ? dim3((unsigned)(p.n_items * p.Q)) : dim3((unsigned)item_count, (unsigned)p.Q);
     // tensor maps over the HCA cache and the raw latents; the kernel only issues boxes that lie
     // inside one sequence's valid rows, so the row extent is left open
     AttnMaps maps;
@@ -924,6 +1030,16 @@ cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, 
               tensor_map_2d_bf16(&maps.x, p.raw, D, 0x7FFFFFFFull, (uint64_t)D * 2, 64, kTileKeys) == cudaSuccess;
     if (!q.tma_hca) std::memset(&maps.hca, 0, sizeof(maps.hca));
     if (!q.tma_x) std::memset(&maps.x, 0, sizeof(maps.x));
+    // direct outputs: one persistent CTA per SM (one fits, by its shared and tensor memory), each
+    // taking every G-th query, so that a query's epilogue overlaps the next one's first products
+    q.q_step = 0;
+    if (p.persist && p.n_items == 1 && !p.hca_first && p.cluster <= 1 && item_count == 1) {
+        const int sms = device_sms();
+        if (sms > 0 && p.Q > sms) {
+            q.q_step = sms;
+            grid = dim3(1u, (unsigned)sms);
+        }
+    }
     if (q.cluster > 1 && q.n_items > 1)
         return launch_kernel_cluster(kernel, grid, dim3(kThreads), L::kAlloc, stream, pdl,
                                      dim3((unsigned)q.cluster, 1, 1), maps, q, item_begin);

@@ -875,6 +875,7 @@ static int make_attn(AttnParams& p, const csa_dims* dims, const csa_seq* seqs, c
     }
     p.status = st;
     debug_fault_state(&p.debug_fault, &p.wait_ns);
+    p.persist = env_int("CSA_ATTN_PERSIST", 1) != 0;
     attn_ws_carve(p, ws);
     return CSA_OK;
 }

@@ -218,6 +218,10 @@ struct AttnParams {
     // the limit of every wait in the kernel
     int debug_fault;
     uint64_t wait_ns;
+    // 1: a launch with one item per query (direct outputs) runs one persistent CTA per SM over the
+    // queries; q_step is set by the launcher (the grid's CTA count; 0 = one CTA per query)
+    int persist;
+    int q_step;
     // outputs
     float* out;                 // [Q, H, d]
     float* lse;                 // [Q, H] nullable
