@@ -52,7 +52,28 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256;
 constexpr uint32_t kLaneO = 16;
 
-template <int D>
+// Per-CTA constants of the key list [CSA slots | raw window | HCA entries] of one query.
+struct KeyList {
+    const int32_t* idx;      // this query's k slots
+    int64_t n_causal;        // floor(L / m)
+    int64_t n_hca;           // floor(L / m') (0 without HCA)
+    int64_t win_row0;        // raw row of the first window token
+    int64_t nw;              // window tokens present
+    int64_t csa_row0, hca_row0;
+};
+
+// One query of a CTA: its key list, the slice [s0, s1) of it the CTA attends and its key tiles.
+struct QWork {
+    KeyList kl;
+    int64_t s0, s1;
+    int T;
+    int qi;
+};
+constexpr int kMaxQ = 64;  // queries of one persistent CTA (the launcher sizes the grid for it)
+
+// NQ: queries a persistent CTA holds in shared memory (kMaxQ; 0 for the single-query kernel, which
+// keeps its one query in registers)
+template <int D, int NQ>
 struct Smem {
     static constexpr int NKB = D / 64;                 // 64-wide blocks along d
     static constexpr int kBlock = 64 * 128;            // one block: 64 rows x 128 bytes
@@ -64,7 +85,8 @@ struct Smem {
     static constexpr int kMisc = kBar + 32 * 8;        // tmem base, abort flag, masks
     static constexpr int kRowPtr = kMisc + 64;         // per loader warp: 16 row pointers
     static constexpr int kRowScl = kRowPtr + 4 * 16 * 8;  // and their FP4 scale rows (null: a bf16 row)
-    static constexpr int kTotal = kRowScl + 4 * 16 * 8;
+    static constexpr int kQTab = kRowScl + 4 * 16 * 8;  // the CTA's queries (QWork)
+    static constexpr int kTotal = kQTab + NQ * (int)sizeof(QWork);
     static constexpr int kAlloc = kTotal + 1024;       // slack for 1024-byte alignment
     // cluster merge: the CTA's [64 x D] fp32 result in the freed key stages, rows padded by 16 bytes
     // so that the eight rows a warp's quads store hit different banks
@@ -91,15 +113,6 @@ struct AttnMaps {
     CUtensorMap x;
 };
 
-// Per-CTA constants of the key list [CSA slots | raw window | HCA entries] of one query.
-struct KeyList {
-    const int32_t* idx;      // this query's k slots
-    int64_t n_causal;        // floor(L / m)
-    int64_t n_hca;           // floor(L / m') (0 without HCA)
-    int64_t win_row0;        // raw row of the first window token
-    int64_t nw;              // window tokens present
-    int64_t csa_row0, hca_row0;
-};
 
 // Row pointer of slot `s` (nullptr = masked slot).
 // The source of key s: a bf16 row (returned, *scl = nullptr) or, for an entry of a cache held in FP4,
@@ -134,11 +147,12 @@ __device__ __forceinline__ const void* key_src(const AttnParams& p, int D, const
 }
 
 // FP4: the instantiation for FP4 entry caches (its loaders dequantize FP4 rows); the other holds no
-// FP4 code at all, which keeps the bf16 kernel's hot loops compact.
-template <int D, bool FP4>
+// FP4 code at all, which keeps the bf16 kernel's hot loops compact.  PERSIST: the instantiation for
+// persistent CTAs over many queries (direct outputs); the other serves one (query, item) per CTA.
+template <int D, bool FP4, bool PERSIST>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnMaps maps, AttnParams p,
                                                            int p_item_base) {
-    using L = Smem<D>;
+    using L = Smem<D, PERSIST ? kMaxQ : 0>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     Bars* bars = reinterpret_cast<Bars*>(sm + L::kBar);
@@ -165,8 +179,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // A direct launch with q_step > 0 is persistent: the CTA takes queries qi0, qi0 + q_step, ... and
     // its pipeline (key stages, S and P buffers, barrier phases) runs on from one query to the next,
     // so that the next query's key loads and Q.K^T products overlap this query's epilogue.
-    const int q_step = direct ? p.q_step : 0;
-    const int n_q = q_step > 0 ? (qi0 < p.Q ? (p.Q - 1 - qi0) / q_step + 1 : 0) : 1;
+    const int q_step = (PERSIST && direct) ? p.q_step : 0;
+    // (the launcher sizes the grid so that no CTA holds more than kMaxQ queries)
+    const int n_q = q_step > 0 ? (qi0 < p.Q ? min((p.Q - 1 - qi0) / q_step + 1, kMaxQ) : 0) : 1;
     const bool clustered = !direct && p.cluster > 1;
     const bool dep_wait = !(p.hca_nowait && !direct && item >= p.items_front);
     // front items with a ready word: the loaders poll it, nobody waits for the select grid up front
@@ -187,19 +202,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         mbar_init(&bars->q_empty, 1);
         mbar_init(&bars->fin, 2);
         misc[1] = 0;
-        // once any CTA has given up on a wait, later CTAs do no work (bounded total time on a fault);
-        // read once, so that every role of the CTA cuts the same key lists
-        misc[8] = (p.status && *reinterpret_cast<volatile int*>(p.status) == CSA_ERR_TIMEOUT) ? 1u : 0u;
         fence_mbar_init();
     }
-    __syncthreads();
-    const bool timed_out = misc[8] != 0u;
     // The query table and sequence lengths: in the decode chain with an indexer they come from the
     // append two launches back, complete once this grid runs (every kernel of the chain waits before
     // it lets the next start); otherwise the previous launch may still be writing them.
     if (!p.queries_early) grid_dep_wait();
     // The key list of query qi and the slice [s0, s1) of it that this CTA attends; returns its number
-    // of key tiles.  Every role evaluates it for every query of the CTA.
+    // of key tiles.
     const int64_t front = (int64_t)p.k_slots + p.W;
     auto work = [&](int qi, KeyList& kl, int64_t& s0, int64_t& s1) -> int {
         const csa_query qr = p.queries[qi];
@@ -226,18 +236,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         if (s1 < s0) s1 = s0;
         if (!qvalid) {
-            if (threadIdx.x == 0 && item == 0) report(p.status, CSA_ERR_INDEX);
+            if (item == 0 && (PERSIST || threadIdx.x == 0)) report(p.status, CSA_ERR_INDEX);
             s1 = s0;
         }
-        if (timed_out) s1 = s0;
+        // once any CTA has given up on a wait, later queries get no work (bounded total time on a fault)
+        if (p.status && *reinterpret_cast<volatile int*>(p.status) == CSA_ERR_TIMEOUT) s1 = s0;
         return s1 > s0 ? (int)((s1 - s0 + kTileKeys - 1) / kTileKeys) : 0;
     };
-    KeyList kl0{};
-    int64_t s00 = 0, s10 = 0;
-    const int T0 = n_q > 0 ? work(qi0, kl0, s00, s10) : 0;
-    // tensor memory for a CTA with work (any query of a persistent CTA may have key tiles)
-    const bool use_tc = q_step > 0 ? n_q > 0 : T0 > 0;
-    if (warp == 8 && use_tc) {
+    // The queries of a persistent CTA, evaluated once (one thread per query) into shared memory, so
+    // that all roles cut the same key lists; a single query is evaluated by every thread (registers).
+    QWork* qtab = reinterpret_cast<QWork*>(sm + L::kQTab);
+    QWork w0{};
+    if constexpr (PERSIST) {
+        for (int jj = threadIdx.x; jj < n_q; jj += kThreads) {
+            QWork w;
+            w.qi = qi0 + jj * q_step;
+            w.T = work(w.qi, w.kl, w.s0, w.s1);
+            qtab[jj] = w;
+        }
+    } else {
+        w0.qi = qi0;
+        w0.T = work(qi0, w0.kl, w0.s0, w0.s1);
+    }
+    auto query = [&](int j) -> const QWork& {
+        if constexpr (PERSIST) return qtab[j];
+        return w0;
+    };
+    if (warp == 8 && n_q > 0) {
         tmem_alloc(misc, kTmemCols);
         tmem_relinquish();
     }
@@ -245,6 +270,104 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    const int T0 = n_q > 0 ? query(0).T : 0;
+    // tensor-core work: any query of a persistent CTA may have key tiles
+    const bool use_tc = q_step > 0 ? n_q > 0 : T0 > 0;
+
+    // Q of query qi into TMEM, by the four warps of one role (warp w writes lane quarter w % 4), in
+    // the A layout of Q.K^T: head row 16w + r in lane r of sub-partition w, dims 2c and 2c + 1 in
+    // column c.  Written with the 16x256b shape, so every lane takes part: lane i writes rows i/4 and
+    // i/4 + 8 at columns 8k + 2(i%4) and 8k + 2(i%4) + 1, i.e. 8 bytes of each of those rows per 8
+    // columns.  The softmax warps store the first query's Q (an input, so before the wait on the
+    // previous launch); the loaders store the j-th one (j > 0) of a persistent CTA once the products
+    // of query j - 1 are done with the region (q_empty), its loads issued before that wait.
+    auto load_q = [&](int qi, int j) -> bool {
+        const int qw = warp & 3;
+        const uint32_t q_lanes = (uint32_t)(qw * 32) << 16;
+        const int qa = lane >> 2, qc = (lane & 3) * 2;
+        const int h0 = qw * 16 + qa, h1 = h0 + 8;
+        const uint2* q0 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h0 < p.H ? h0 : 0)) * D);
+        const uint2* q1 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h1 < p.H ? h1 : 0)) * D);
+        // optional RMS normalization of each head's query (gain p.q_norm): the four lanes of a quad
+        // hold a quarter of the row each; a first pass sums the squares, the second scales
+        float inv0 = 1.f, inv1 = 1.f;
+        if (p.q_norm) {
+            float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 4
+            for (int cb = 0; cb < D / 2; cb += 64) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int col = cb + 8 * k + qc;
+                    float f[4];
+                    const uint2 v0 = h0 < p.H ? q0[col / 2] : make_uint2(0, 0);
+                    const uint2 v1 = h1 < p.H ? q1[col / 2] : make_uint2(0, 0);
+                    f[0] = bf16lo(v0.x); f[1] = bf16hi(v0.x); f[2] = bf16lo(v0.y); f[3] = bf16hi(v0.y);
+                    ss0 = fmaf(f[0], f[0], fmaf(f[1], f[1], fmaf(f[2], f[2], fmaf(f[3], f[3], ss0))));
+                    f[0] = bf16lo(v1.x); f[1] = bf16hi(v1.x); f[2] = bf16lo(v1.y); f[3] = bf16hi(v1.y);
+                    ss1 = fmaf(f[0], f[0], fmaf(f[1], f[1], fmaf(f[2], f[2], fmaf(f[3], f[3], ss1))));
+                }
+            }
+            ss0 += __shfl_xor_sync(0xffffffffu, ss0, 1);
+            ss0 += __shfl_xor_sync(0xffffffffu, ss0, 2);
+            ss1 += __shfl_xor_sync(0xffffffffu, ss1, 1);
+            ss1 += __shfl_xor_sync(0xffffffffu, ss1, 2);
+            inv0 = rsqrtf(ss0 / D + p.norm_eps);
+            inv1 = rsqrtf(ss1 / D + p.norm_eps);
+        }
+        const bool ok0 = h0 < p.H, ok1 = h1 < p.H;
+        // dims 2col .. 2col + 3 of a row, normalized and rounded back to bf16 (gain p.q_norm)
+        auto qnorm = [&](uint32_t& x, uint32_t& y, float inv, int col) {
+            const float4 gn = *reinterpret_cast<const float4*>(p.q_norm + 2 * col);
+            x = pack_bf16x2(bf16lo(x) * inv * gn.x, bf16hi(x) * inv * gn.y);
+            y = pack_bf16x2(bf16lo(y) * inv * gn.z, bf16hi(y) * inv * gn.w);
+        };
+#pragma unroll 1
+        for (int cb = 0; cb < D / 2; cb += 128) {
+            uint32_t r[2][32];
+            // every load of the pass first, unconditionally (a column past the row reads column
+            // qc), so they are all in flight together; then the optional normalization and the
+            // zeros of heads past H by selects on the loaded registers
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const bool in = cb + g * 64 < D / 2;
+                    const int col = in ? cb + g * 64 + 8 * k + qc : qc;  // a column holds 2 dims
+                    const uint2 v0 = q0[col / 2], v1 = q1[col / 2];
+                    r[g][4 * k] = v0.x; r[g][4 * k + 1] = v0.y; r[g][4 * k + 2] = v1.x; r[g][4 * k + 3] = v1.y;
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const bool in = cb + g * 64 < D / 2;
+                    const int col = in ? cb + g * 64 + 8 * k + qc : qc;
+                    if (p.q_norm) {
+                        qnorm(r[g][4 * k], r[g][4 * k + 1], inv0, col);
+                        qnorm(r[g][4 * k + 2], r[g][4 * k + 3], inv1, col);
+                    }
+                    const bool u0 = in && ok0, u1 = in && ok1;
+                    r[g][4 * k] = u0 ? r[g][4 * k] : 0u;
+                    r[g][4 * k + 1] = u0 ? r[g][4 * k + 1] : 0u;
+                    r[g][4 * k + 2] = u1 ? r[g][4 * k + 2] : 0u;
+                    r[g][4 * k + 3] = u1 ? r[g][4 * k + 3] : 0u;
+                }
+            }
+            if (cb == 0 && j > 0) {
+                const bool w = mbar_wait(&bars->q_empty, (uint32_t)(j - 1) & 1u, p.status, abort_flag, p.wait_ns);
+                if (!__all_sync(0xffffffffu, w)) return false;  // (the stores below are warp-collective)
+                tc_fence_after();
+            }
+#pragma unroll
+            for (int g = 0; g < 2; ++g)
+                if (cb + g * 64 < D / 2) tmem_st_16x256_x8(tmem + q_lanes + (uint32_t)(cb + g * 64), r[g]);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->q_full);
+        return true;
+    };
 
     if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------------ loaders
@@ -278,19 +401,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         uint32_t tma_pend = 0;
         uint32_t g = 0;  // key tiles of the CTA's earlier queries (the stage ring runs on)
         for (int j = 0; go && j < n_q; ++j) {
-            KeyList kl = kl0;
-            int64_t s0 = s00, s1 = s10;
-            const int T = j == 0 ? T0 : work(qi0 + j * q_step, kl, s0, s1);
-            // the selected indices of this lane's rows in the query's first two tiles, read together
-            // (one memory latency, not one per tile); an address past the slots reads the last slot
-            int32_t pre_j0 = -1, pre_j1 = -1;
-            const bool pre = kl.idx && s0 < p.k_slots && lane < 16;
-            if (pre) {
-                const int64_t sa = s0 + lw * 16 + lane, sb = sa + kTileKeys;
-                pre_j0 = kl.idx[sa < p.k_slots ? sa : p.k_slots - 1];
-                pre_j1 = kl.idx[sb < p.k_slots ? sb : p.k_slots - 1];
-            }
+            const KeyList kl = query(j).kl;
+            const int64_t s0 = query(j).s0, s1 = query(j).s1;
+            const int T = query(j).T;
+            // the selected index of this lane's row in tile t, read ahead: the first two tiles' together
+            // (one memory latency, not one per tile), and in a persistent CTA, whose queries span many
+            // tiles of slots, tile t + 2's while tile t is loaded, so that no tile waits on its indices
+            // (a single-query CTA reads later tiles' indices as it loads them); an address past the
+            // slots reads the last slot, unused
+            const bool pre = kl.idx && lane < 16;
+            auto read_j = [&](int t) -> int32_t {
+                const int64_t tb = s0 + (int64_t)t * kTileKeys;
+                if (!PERSIST && t >= 2) return -1;
+                if (!pre || t >= T || tb >= p.k_slots) return -1;
+                const int64_t sa = tb + lw * 16 + lane;
+                return kl.idx[sa < p.k_slots ? sa : p.k_slots - 1];
+            };
+            int32_t j_next = read_j(0), j_after = read_j(1);
             for (int t = 0; t < T; ++t) {
+                const int32_t j_t = j_next;
+                j_next = j_after;
+                j_after = read_j(t + 2);
+                // a persistent CTA's next query: its Q goes into TMEM after the query's first tile is
+                // issued (the products of the previous query still read the region until then)
+                if (PERSIST && j > 0 && t == 1 && !load_q(query(j).qi, j)) {
+                    go = false;
+                    break;
+                }
                 const uint32_t gt = g + (uint32_t)t;
                 const int st = (int)(gt % kStages);
                 if (gt >= kStages &&
@@ -335,8 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 if (lane < 16) {
                     const int64_t s = tb + lw * 16 + lane;
                     const uint8_t* scl = nullptr;
-                    const void* r =
-                        s < s1 ? key_src(p, D, kl, s, &scl, pre && t < 2, t == 0 ? pre_j0 : pre_j1) : nullptr;
+                    const void* r = s < s1 ? key_src(p, D, kl, s, &scl, pre && (PERSIST || t < 2), j_t) : nullptr;
                     rowptr_w[lane] = reinterpret_cast<uint64_t>(r);
                     rowscl_w[lane] = reinterpret_cast<uint64_t>(scl);
                     valid = r != nullptr;
@@ -412,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 __syncwarp();
                 if (!skip) mbar_arrive(&bars->full[st]);
             }
+            if (PERSIST && go && j > 0 && T <= 1 && !load_q(query(j).qi, j)) go = false;
             g += (uint32_t)T;
         }
         cp_async_wait_all();
@@ -437,9 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             if (warp == 8) {
                 constexpr uint32_t id1 = idesc_bf16(64, 64, false, false);
                 for (int j = 0; ok && j < n_q; ++j) {
-                    KeyList kl = kl0;
-                    int64_t s0 = s00, s1 = s10;
-                    const int T = j == 0 ? T0 : work(qi0 + j * q_step, kl, s0, s1);
+                    const int T = query(j).T;
                     ok = __all_sync(0xffffffffu,
                                     mbar_wait(&bars->q_full, (uint32_t)j & 1u, p.status, abort_flag, p.wait_ns));
                     for (int t = 0; ok && t < T; ++t) {
@@ -468,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                         umma_commit(&bars->s_full[gt & 1]);
                     }
                     // the query's products have read Q once this completes: the next Q may be stored
-                    umma_commit(&bars->q_empty);
+                    if (PERSIST) umma_commit(&bars->q_empty);
                     g += (uint32_t)T;
                 }
             } else {
@@ -476,9 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 constexpr int HALVES = D >= 256 ? D / 256 : 1;
                 constexpr uint32_t id2 = idesc_bf16(64, N2, false, true);
                 for (int j = 0; ok && j < n_q; ++j) {
-                    KeyList kl = kl0;
-                    int64_t s0 = s00, s1 = s10;
-                    const int T = j == 0 ? T0 : work(qi0 + j * q_step, kl, s0, s1);
+                    const int T = query(j).T;
                     for (int t = 0; t < T; ++t) {
                         const uint32_t gt = g + (uint32_t)t;
                         const bool w = mbar_wait(&bars->p_full[gt & 1], (gt >> 1) & 1, p.status, abort_flag, p.wait_ns);
@@ -515,97 +648,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         // ------------------------------------------------------------------ softmax + epilogue
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const uint32_t o_base = tmem + lane_base + (kLaneO << 16);
-        // Q of query qi (an input, so the first one before the wait) in the A layout of Q.K^T: head
-        // row 16w + r in lane r of warp w's sub-partition, dims 2c and 2c + 1 in column c.  Written
-        // with the 16x256b shape, so every lane takes part: lane i writes rows i/4 and i/4 + 8 at
-        // columns 8k + 2(i%4) and 8k + 2(i%4) + 1, i.e. 8 bytes of each of those rows per 8 columns.
-        // The j-th query of the CTA (j > 0) stores its Q once the products of query j - 1 are done
-        // with the region (q_empty); its loads are issued before that wait.
-        auto load_q = [&](int qi, int j) -> bool {
-            const int qa = lane >> 2, qc = (lane & 3) * 2;
-            const int h0 = warp * 16 + qa, h1 = h0 + 8;
-            const uint2* q0 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h0 < p.H ? h0 : 0)) * D);
-            const uint2* q1 = reinterpret_cast<const uint2*>(p.q + ((int64_t)qi * p.H + (h1 < p.H ? h1 : 0)) * D);
-            // optional RMS normalization of each head's query (gain p.q_norm): the four lanes of a quad
-            // hold a quarter of the row each; a first pass sums the squares, the second scales
-            float inv0 = 1.f, inv1 = 1.f;
-            if (p.q_norm) {
-                float ss0 = 0.f, ss1 = 0.f;
-#pragma unroll 4
-                for (int cb = 0; cb < D / 2; cb += 64) {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int col = cb + 8 * k + qc;
-                        float f[4];
-                        const uint2 v0 = h0 < p.H ? q0[col / 2] : make_uint2(0, 0);
-                        const uint2 v1 = h1 < p.H ? q1[col / 2] : make_uint2(0, 0);
-                        f[0] = bf16lo(v0.x); f[1] = bf16hi(v0.x); f[2] = bf16lo(v0.y); f[3] = bf16hi(v0.y);
-                        ss0 = fmaf(f[0], f[0], fmaf(f[1], f[1], fmaf(f[2], f[2], fmaf(f[3], f[3], ss0))));
-                        f[0] = bf16lo(v1.x); f[1] = bf16hi(v1.x); f[2] = bf16lo(v1.y); f[3] = bf16hi(v1.y);
-                        ss1 = fmaf(f[0], f[0], fmaf(f[1], f[1], fmaf(f[2], f[2], fmaf(f[3], f[3], ss1))));
-                    }
-                }
-                ss0 += __shfl_xor_sync(0xffffffffu, ss0, 1);
-                ss0 += __shfl_xor_sync(0xffffffffu, ss0, 2);
-                ss1 += __shfl_xor_sync(0xffffffffu, ss1, 1);
-                ss1 += __shfl_xor_sync(0xffffffffu, ss1, 2);
-                inv0 = rsqrtf(ss0 / D + p.norm_eps);
-                inv1 = rsqrtf(ss1 / D + p.norm_eps);
-            }
-            const bool ok0 = h0 < p.H, ok1 = h1 < p.H;
-            // dims 2col .. 2col + 3 of a row, normalized and rounded back to bf16 (gain p.q_norm)
-            auto qnorm = [&](uint32_t& x, uint32_t& y, float inv, int col) {
-                const float4 gn = *reinterpret_cast<const float4*>(p.q_norm + 2 * col);
-                x = pack_bf16x2(bf16lo(x) * inv * gn.x, bf16hi(x) * inv * gn.y);
-                y = pack_bf16x2(bf16lo(y) * inv * gn.z, bf16hi(y) * inv * gn.w);
-            };
-#pragma unroll 1
-            for (int cb = 0; cb < D / 2; cb += 128) {
-                uint32_t r[2][32];
-                // every load of the pass first, unconditionally (a column past the row reads column
-                // qc), so they are all in flight together; then the optional normalization and the
-                // zeros of heads past H by selects on the loaded registers
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const bool in = cb + g * 64 < D / 2;
-                        const int col = in ? cb + g * 64 + 8 * k + qc : qc;  // a column holds 2 dims
-                        const uint2 v0 = q0[col / 2], v1 = q1[col / 2];
-                        r[g][4 * k] = v0.x; r[g][4 * k + 1] = v0.y; r[g][4 * k + 2] = v1.x; r[g][4 * k + 3] = v1.y;
-                    }
-                }
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const bool in = cb + g * 64 < D / 2;
-                        const int col = in ? cb + g * 64 + 8 * k + qc : qc;
-                        if (p.q_norm) {
-                            qnorm(r[g][4 * k], r[g][4 * k + 1], inv0, col);
-                            qnorm(r[g][4 * k + 2], r[g][4 * k + 3], inv1, col);
-                        }
-                        const bool u0 = in && ok0, u1 = in && ok1;
-                        r[g][4 * k] = u0 ? r[g][4 * k] : 0u;
-                        r[g][4 * k + 1] = u0 ? r[g][4 * k + 1] : 0u;
-                        r[g][4 * k + 2] = u1 ? r[g][4 * k + 2] : 0u;
-                        r[g][4 * k + 3] = u1 ? r[g][4 * k + 3] : 0u;
-                    }
-                }
-                if (cb == 0 && j > 0) {
-                    if (!mbar_wait(&bars->q_empty, (uint32_t)(j - 1) & 1u, p.status, abort_flag, p.wait_ns))
-                        return false;
-                    tc_fence_after();
-                }
-#pragma unroll
-                for (int g = 0; g < 2; ++g)
-                    if (cb + g * 64 < D / 2) tmem_st_16x256_x8(tmem + lane_base + (uint32_t)(cb + g * 64), r[g]);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars->q_full);
-            return true;
-        };
         bool ok = true;
         if (use_tc) ok = load_q(qi0, 0);
         if (dep_wait && !ready_wait) grid_dep_wait();
@@ -617,11 +659,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const int ra = i >> 2, cq = (i & 3) * 2;
         const int hr[2] = {warp * 16 + ra, warp * 16 + ra + 8};
         uint32_t g = 0;  // key tiles of the CTA's earlier queries
-        KeyList kl = kl0;
-        int64_t s0 = s00, s1 = s10;
-        int T = T0;
         for (int j = 0; j < n_q; ++j) {
-            const int qi = qi0 + j * q_step;
+            const int qi = query(j).qi;
+            const int T = query(j).T;
             float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
             for (int t = 0; ok && t < T; ++t) {
                 const uint32_t gt = g + (uint32_t)t;
@@ -728,13 +768,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             const int Tq = T;
             const uint32_t gq = g;
             g += (uint32_t)T;
-            // the next query of a persistent CTA: its key list, and its Q stored as soon as this query's
-            // products are done with Q, ahead of this query's epilogue, so that the next products start
-            // while this query's output is stored
-            if (j + 1 < n_q) {
-                T = work(qi + q_step, kl, s0, s1);
-                if (ok) ok = load_q(qi + q_step, j + 1);
-            }
             // ---- epilogue: TMEM -> registers -> global memory
             if (ok && Tq > 0) {
                 const uint32_t gl = gq + (uint32_t)Tq - 1u;
@@ -833,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     if (ready_wait) grid_dep_wait();
     tc_fence_before();
     __syncthreads();
-    if (warp == 8 && use_tc) {
+    if (warp == 8 && n_q > 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -1009,16 +1042,20 @@ int device_sms() {
 
 template <int D>
 cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, cudaStream_t stream, bool pdl) {
-    using L = Smem<D>;
+    using L = Smem<D, 0>;
+    using LP = Smem<D, kMaxQ>;
     static PerDeviceOnce attr;
     cudaError_t ea = attr.run([] {
-        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(attn_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+        constexpr auto a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, false, false>, a, L::kAlloc);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_kernel<D, true, false>, a, L::kAlloc);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_kernel<D, false, true>, a, LP::kAlloc);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_kernel<D, true, true>, a, LP::kAlloc);
         return e;
     });
     if (ea != cudaSuccess) return ea;
-    auto kernel = (p.entries_q || p.hca_q) ? attn_kernel<D, true> : attn_kernel<D, false>;
+    const bool fp4 = p.entries_q || p.hca_q;
+    auto kernel = fp4 ? attn_kernel<D, true, false> : attn_kernel<D, false, false>;
     dim3 grid = p.hca_first ? dim3((unsigned)(p.n_items * p.Q)) : dim3((unsigned)item_count, (unsigned)p.Q);
     // tensor maps over the HCA cache and the raw latents; the kernel only issues boxes that lie
     // inside one sequence's valid rows, so the row extent is left open
@@ -1030,20 +1067,25 @@ cudaError_t launch_items_d(const AttnParams& p, int item_begin, int item_count, 
               tensor_map_2d_bf16(&maps.x, p.raw, D, 0x7FFFFFFFull, (uint64_t)D * 2, 64, kTileKeys) == cudaSuccess;
     if (!q.tma_hca) std::memset(&maps.hca, 0, sizeof(maps.hca));
     if (!q.tma_x) std::memset(&maps.x, 0, sizeof(maps.x));
-    // direct outputs: one persistent CTA per SM (one fits, by its shared and tensor memory), each
-    // taking every G-th query, so that a query's epilogue overlaps the next one's first products
+    // direct outputs: persistent CTAs, one per SM (one fits, by its shared and tensor memory) or
+    // more when a CTA would otherwise hold over kMaxQ queries, each taking every G-th query, so that
+    // a query's epilogue overlaps the next one's first products
     q.q_step = 0;
+    int smem = L::kAlloc;
     if (p.persist && p.n_items == 1 && !p.hca_first && p.cluster <= 1 && item_count == 1) {
         const int sms = device_sms();
-        if (sms > 0 && p.Q > sms) {
-            q.q_step = sms;
-            grid = dim3(1u, (unsigned)sms);
+        const int G = sms > (p.Q + kMaxQ - 1) / kMaxQ ? sms : (p.Q + kMaxQ - 1) / kMaxQ;
+        if (sms > 0 && p.Q > G) {
+            q.q_step = G;
+            grid = dim3(1u, (unsigned)G);
+            kernel = fp4 ? attn_kernel<D, true, true> : attn_kernel<D, false, true>;
+            smem = LP::kAlloc;
         }
     }
     if (q.cluster > 1 && q.n_items > 1)
-        return launch_kernel_cluster(kernel, grid, dim3(kThreads), L::kAlloc, stream, pdl,
+        return launch_kernel_cluster(kernel, grid, dim3(kThreads), smem, stream, pdl,
                                      dim3((unsigned)q.cluster, 1, 1), maps, q, item_begin);
-    return launch_kernel(kernel, grid, dim3(kThreads), L::kAlloc, stream, pdl, maps, q, item_begin);
+    return launch_kernel(kernel, grid, dim3(kThreads), smem, stream, pdl, maps, q, item_begin);
 }
 
 }  // namespace
