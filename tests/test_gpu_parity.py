@@ -819,6 +819,43 @@ def test_sparse_and_hca_attention_stage(wl, lens):
             gh.check_close(lse[i].cpu().numpy(), l, f"hca lse q{i}")
 
 
+def test_sparse_attention_persistent_ctas():
+    """More queries than SMs in one direct launch: persistent CTAs take every G-th query, the loader
+    warps store each later query's Q and read its slot indices ahead.  Rows that CTAs run first,
+    second and third are checked against the oracle."""
+    wl = wl_small(5000, B=1)
+    layer, refs = _stage_layer(wl)
+    d = wl.dims
+    sh = gh.oshape(d)
+    Q = 300
+    lens = [1 + (i * 2711) % 5000 for i in range(Q)]
+    lens[5], lens[160], lens[299] = 5000, 1, 4
+    pairs = [(0, L) for L in lens]
+    qs = np.stack([workloads.queries(wl, 0, i % 64, i % 64 + 1)[0][0] for i in range(Q)])
+    idxs = []
+    for i, L in enumerate(lens):
+        _, qi_, w_ = workloads.queries(wl, 0, i % 64, i % 64 + 1)
+        s = oracle.index_scores(qi_[0], w_[0], refs[0].KI[:L // d.m])
+        idxs.append(oracle.topk(s, d.k))
+    qt = gh.query_table(pairs)
+    q_d = gh.to_dev_bf16(qs)
+    idx_d = torch.from_numpy(np.stack(idxs)).cuda()
+    out = torch.full((Q, d.H, d.d), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.empty(Q, d.H, dtype=torch.float32, device="cuda")
+    dims = gh.dims_of(d)
+    wq = csa.csa_ws_query()
+    wq.dims, wq.Q, wq.max_len = dims, Q, max(wl.n0)
+    ws = torch.empty(csa.csa_workspace_size(csa.CSA_OP_SPARSE_ATTN, wq) + 256, dtype=torch.uint8, device="cuda")
+    csa.csa_sparse_attn(dims, layer.seqs, qt, Q, q_d, layer.entries, idx_d, layer.x, sh.scale, out, lse, ws)
+    assert csa.csa_sync_status() == csa.CSA_OK
+    assert torch.isfinite(out).all()
+    for i in (0, 5, 7, 147, 148, 150, 160, 220, 295, 296, 299):
+        L = lens[i]
+        O, l = oracle.csa_attn(qs[i], refs[0].E, idxs[i], d.m, refs[0].x, L, d.W, sh.scale)
+        gh.check_close(out[i].cpu().numpy(), O, f"csa q{i} L={L}")
+        gh.check_close(lse[i].cpu().numpy(), l, f"csa lse q{i}")
+
+
 def test_bad_index_is_reported_not_read():
     wl = workloads.tiny()
     layer, refs = _stage_layer(wl)
