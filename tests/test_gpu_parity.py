@@ -819,17 +819,21 @@ def test_sparse_and_hca_attention_stage(wl, lens):
             gh.check_close(lse[i].cpu().numpy(), l, f"hca lse q{i}")
 
 
-def test_sparse_attention_persistent_ctas():
+@pytest.mark.parametrize("fp4", [False, True], ids=["bf16", "fp4"])
+def test_sparse_attention_persistent_ctas(fp4):
     """More queries than SMs in one direct launch: persistent CTAs take every G-th query, the loader
     warps store each later query's Q and read its slot indices ahead.  Rows that CTAs run first,
-    second and third are checked against the oracle."""
+    second and third are checked against the oracle (bf16 entries, or the FP4 cache against the
+    oracle's dequantized entries); one query with no visible token (length 0) is reported, gets zeros
+    and lse = -inf, and leaves the others intact."""
     wl = wl_small(5000, B=1)
     layer, refs = _stage_layer(wl)
     d = wl.dims
     sh = gh.oshape(d)
-    Q = 300
+    Q = 301
     lens = [1 + (i * 2711) % 5000 for i in range(Q)]
     lens[5], lens[160], lens[299] = 5000, 1, 4
+    lens[200] = 0  # invalid: reported, zeros
     pairs = [(0, L) for L in lens]
     qs = np.stack([workloads.queries(wl, 0, i % 64, i % 64 + 1)[0][0] for i in range(Q)])
     idxs = []
@@ -837,6 +841,7 @@ def test_sparse_attention_persistent_ctas():
         _, qi_, w_ = workloads.queries(wl, 0, i % 64, i % 64 + 1)
         s = oracle.index_scores(qi_[0], w_[0], refs[0].KI[:L // d.m])
         idxs.append(oracle.topk(s, d.k))
+    ent = refs[0].E
     qt = gh.query_table(pairs)
     q_d = gh.to_dev_bf16(qs)
     idx_d = torch.from_numpy(np.stack(idxs)).cuda()
@@ -846,12 +851,26 @@ def test_sparse_attention_persistent_ctas():
     wq = csa.csa_ws_query()
     wq.dims, wq.Q, wq.max_len = dims, Q, max(wl.n0)
     ws = torch.empty(csa.csa_workspace_size(csa.CSA_OP_SPARSE_ATTN, wq) + 256, dtype=torch.uint8, device="cuda")
-    csa.csa_sparse_attn(dims, layer.seqs, qt, Q, q_d, layer.entries, idx_d, layer.x, sh.scale, out, lse, ws)
-    assert csa.csa_sync_status() == csa.CSA_OK
-    assert torch.isfinite(out).all()
-    for i in (0, 5, 7, 147, 148, 150, 160, 220, 295, 296, 299):
+    if fp4:
+        n_c = len(refs[0].E)
+        eq = torch.zeros(layer.entries.shape[0], d.d // 2, dtype=torch.uint8, device="cuda")
+        es = torch.zeros(layer.entries.shape[0], d.d // 32, dtype=torch.uint8, device="cuda")
+        q_, s_ = oracle.quantize_entries_mx4(refs[0].E)
+        eq[layer.csa_off[0]:layer.csa_off[0] + n_c] = torch.from_numpy(q_).cuda()
+        es[layer.csa_off[0]:layer.csa_off[0] + n_c] = torch.from_numpy(s_).cuda()
+        ent = oracle.mx4_entries_as_bf16(refs[0].E)
+        csa.csa_sparse_attn_fp4(dims, layer.seqs, qt, Q, q_d, eq, es, idx_d, layer.x, sh.scale, out, lse, ws)
+    else:
+        csa.csa_sparse_attn(dims, layer.seqs, qt, Q, q_d, layer.entries, idx_d, layer.x, sh.scale, out, lse, ws)
+    assert csa.csa_sync_status() == csa.CSA_ERR_INDEX
+    assert csa.csa_sync_status() == csa.CSA_OK  # cleared
+    assert (out[200] == 0).all() and torch.isneginf(lse[200]).all()
+    keep = torch.ones(Q, dtype=torch.bool)
+    keep[200] = False
+    assert torch.isfinite(out[keep.cuda()]).all()
+    for i in (0, 5, 7, 147, 148, 150, 160, 199, 201, 295, 296, 299, 300):
         L = lens[i]
-        O, l = oracle.csa_attn(qs[i], refs[0].E, idxs[i], d.m, refs[0].x, L, d.W, sh.scale)
+        O, l = oracle.csa_attn(qs[i], ent, idxs[i], d.m, refs[0].x, L, d.W, sh.scale)
         gh.check_close(out[i].cpu().numpy(), O, f"csa q{i} L={L}")
         gh.check_close(lse[i].cpu().numpy(), l, f"csa lse q{i}")
 
