@@ -1189,8 +1189,13 @@ int hybrid_attn_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, cs
                 sp.m_shift = d.m == 1 ? 0 : d.m == 2 ? 1 : d.m == 4 ? 2 : 3;  // m is 1, 2, 4 or 8
                 sp.Qn = (int)n;
                 sp.pos0 = p0;
+                // entry ranges for two waves of one CTA per SM: at most 2 x SMs CTAs in all (ranges
+                // rounded up to whole tiles, so that a few leftover CTAs never form a third wave)
                 const int64_t gy = (n + 127) / 128;
-                int64_t ent = (max_e_chunk * gy + 2 * 148 - 1) / (2 * 148);
+                int sms = 148;
+                if (sm_count(&sms) != CSA_OK) sms = 148;
+                const int64_t gx_max = 2 * (int64_t)sms / gy > 0 ? 2 * (int64_t)sms / gy : 1;
+                int64_t ent = (max_e_chunk + gx_max - 1) / gx_max;
                 ent = ((ent + 63) / 64) * 64;
                 sp.ent_per_cta = ent < 64 ? 64 : ent;
                 sp.scores = ip.scores;
