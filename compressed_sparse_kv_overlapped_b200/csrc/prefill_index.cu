@@ -11,8 +11,9 @@
 // threshold from a sample of the scores (see index_topk.cu).
 //
 // Warp roles: warp 0 cp.async loader (the CTA's q^I once, then key tiles through a 4-stage ring),
-// warp 1 TMEM allocator + MMA issuer, warps 2-9 epilogue, two per TMEM lane quarter, each over half
-// of a tile's 64 entries (TMEM -> relu / weights -> shared-memory staging -> coalesced row stores).  TMEM holds two accumulator sets (4 heads x 64 columns each)
+// warp 1 TMEM allocator + MMA issuer, the other warps epilogue, kPsSplit per TMEM lane quarter, each
+// over a part of a tile's 64 entries (TMEM -> relu / weights -> shared-memory staging -> coalesced
+// row stores).  TMEM holds two accumulator sets (4 heads x 64 columns each)
 // so the products of tile t+1 overlap the epilogue of tile t.  Every wait is bounded.
 #include "common.cuh"
 #include "kernels.h"
@@ -25,15 +26,18 @@ constexpr int kPsRows = 128;    // queries per CTA (MMA M)
 constexpr int kPsTile = 64;     // entries per tile (MMA N)
 constexpr int kPsStages = 4;
 constexpr int kPsHeads = 4;     // accumulators per tile (H_I <= 4; missing heads get zero rows / weight)
-constexpr int kPsThreads = 320;        // loader, MMA issuer, 8 epilogue warps (two per TMEM lane quarter)
-constexpr int kPsHalf = kPsTile / 2;   // entries of a tile one epilogue warp handles
-constexpr int kPsStride = kPsHalf + 4;  // staging row stride (floats)
+constexpr int kPsSplit = 4;                 // epilogue warps per TMEM lane quarter
+constexpr int kPsEpi = 4 * kPsSplit;         // epilogue warps
+constexpr int kPsThreads = 64 + 32 * kPsEpi;  // loader, MMA issuer, the epilogue warps
+constexpr int kPsPart = kPsTile / kPsSplit;   // entries of a tile one epilogue warp handles
+constexpr int kPsStride = kPsPart + 4;        // staging row stride (floats)
+static_assert(kPsPart % 16 == 0, "whole 16-column TMEM loads");
 
 struct PsSmem {
     static constexpr int kA = 0;                                    // 4 heads x [128 rows x 128 B]
     static constexpr int kB = kA + kPsHeads * kPsRows * 128;        // stages x [64 rows x 128 B]
-    static constexpr int kStg = kB + kPsStages * kPsTile * 128;     // 8 warps x 32 rows x kPsStride floats
-    static constexpr int kBar = kStg + 8 * 32 * kPsStride * 4;
+    static constexpr int kStg = kB + kPsStages * kPsTile * 128;     // epilogue warps x 32 rows x kPsStride floats
+    static constexpr int kBar = kStg + kPsEpi * 32 * kPsStride * 4;
     static constexpr int kMisc = kBar + 16 * 8;
     static constexpr int kTotal = kMisc + 64;
     static constexpr int kAlloc = kTotal + 1024;
@@ -73,7 +77,7 @@ __global__ void __launch_bounds__(kPsThreads, 1) prefill_score_kernel(PrefillSco
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->acc_full[i], 1);
-            mbar_init(&bars->acc_empty[i], 256);
+            mbar_init(&bars->acc_empty[i], 32 * kPsEpi);
         }
         mbar_init(&bars->a_full, 32);
         mbar_init(&bars->fin, 1);
@@ -147,9 +151,9 @@ __global__ void __launch_bounds__(kPsThreads, 1) prefill_score_kernel(PrefillSco
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ epilogue
-        const int ew = warp - 2;                 // 0..7
+        const int ew = warp - 2;                 // 0 .. kPsEpi - 1
         const int sp = warp & 3;                 // TMEM sub-partition of this warp: rows 32 sp .. 32 sp + 31
-        const int ch = ew >> 2;                  // this warp's half of each tile: entries 32 ch .. 32 ch + 31
+        const int ch = ew >> 2;                  // this warp's part of each tile: entries kPsPart ch .. + kPsPart - 1
         const int r = sp * 32 + lane;            // this lane's query row in the block
         const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
         float wv[kPsHeads];
@@ -158,17 +162,19 @@ __global__ void __launch_bounds__(kPsThreads, 1) prefill_score_kernel(PrefillSco
         float* stg = reinterpret_cast<float*>(sm + PsSmem::kStg) + ew * 32 * kPsStride;
         // causal entries of this lane's row (the store loop below broadcasts them row by row)
         const int e_mine = (int)((p.pos0 + row0 + r + 1) >> p.m_shift);
-        const int hl = lane >> 4, l16 = lane & 15;  // store loop: half-warp hl takes row rr + hl
+        // store loop: kPsPart / 2 lanes per row (two entries each), 64 / kPsPart rows per instruction
+        constexpr int kLpr = kPsPart / 2, kRpi = 32 / kLpr;
+        const int hl = lane / kLpr, l16 = lane % kLpr;
         for (int t = 0; t < T; ++t) {
             const int ab = t & 1;
             if (!mbar_wait(&bars->acc_full[ab], (t >> 1) & 1, p.status, abort_flag)) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < kPsHalf; c += 16) {
+            for (int c = 0; c < kPsPart; c += 16) {
                 uint32_t v[kPsHeads][16];
 #pragma unroll
                 for (int h = 0; h < kPsHeads; ++h)
-                    tmem_ld16(tmem + lane_base + (uint32_t)(ab * 256 + h * 64 + ch * kPsHalf + c), v[h]);
+                    tmem_ld16(tmem + lane_base + (uint32_t)(ab * 256 + h * 64 + ch * kPsPart + c), v[h]);
                 tmem_ld_wait();
 #pragma unroll
                 for (int j4 = 0; j4 < 16; j4 += 4) {
@@ -186,9 +192,9 @@ __global__ void __launch_bounds__(kPsThreads, 1) prefill_score_kernel(PrefillSco
             tc_fence_before();
             mbar_arrive(&bars->acc_empty[ab]);
             __syncwarp();
-            // the warp's 32 rows, two 128-byte row halves per instruction (lane: two entries)
-            const int64_t tb = e0 + (int64_t)t * kPsTile + ch * kPsHalf + 2 * l16;
-            for (int rr = 0; rr < 32; rr += 2) {
+            // the warp's 32 rows, kRpi row parts per instruction (lane: two entries)
+            const int64_t tb = e0 + (int64_t)t * kPsTile + ch * kPsPart + 2 * l16;
+            for (int rr = 0; rr < 32; rr += kRpi) {
                 const int row = sp * 32 + rr + hl;
                 const int64_t e_row = __shfl_sync(0xffffffffu, e_mine, rr + hl);  // causal entries of this query
                 if (row < rows) {
