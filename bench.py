@@ -792,7 +792,7 @@ def run_prefill(args, rank, world):
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded counter-based generator)",
         "config": {"workload": wl.name, "N": N, "d": wd.d, "heads": wd.H, "d_I": wd.d_I, "H_I": wd.H_I, "k": wd.k,
-                   "W": wd.W, "m": wd.m, "m_hca": wd.m_hca, "prefill_chunk": int(os.environ.get("CSA_PREFILL_CHUNK", 2048)),
+                   "W": wd.W, "m": wd.m, "m_hca": wd.m_hca, "prefill_chunk": int(os.environ.get("CSA_PREFILL_CHUNK", 0)) or 64 * torch.cuda.get_device_properties(dev).multi_processor_count,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "flops": {"index": f_index, "attention": f_attn, "total": f_index + f_attn},
         "roofline": {"kernel": "whole prefill (index + select + attention)", "bound": "tensor", "achieved": tflops,

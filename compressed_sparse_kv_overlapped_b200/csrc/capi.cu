@@ -411,13 +411,22 @@ struct PrefillPlan {
     size_t off_queries, off_idx, off_index, total;
 };
 
+int sm_count(int* out);  // multiprocessors of the current device (below)
+
 PrefillPlan plan_prefill(const csa_dims& d, int64_t q_end) {
     PrefillPlan pl{};
     const int64_t max_e = q_end / d.m;
     pl.e_stride = ((max_e + 3) / 4) * 4;
     if (pl.e_stride < 4) pl.e_stride = 4;
-    pl.qc = env_int("CSA_PREFILL_CHUNK", 2048);
-    if (pl.qc < 1) pl.qc = 1;
+    // queries per chunk: by default 64 per SM, whole rounds of the persistent attention CTAs (one
+    // per SM, 64 queries each, the most one holds); longer chunks also make longer score GEMMs and
+    // fewer launches (measured at N = 131,072: 2,048 per chunk 56.9 ms, 4,736 = 32 x 148 53.9 ms,
+    // 9,472 = 64 x 148 52.9 ms; the score rows of a chunk take 4 B x 9,472 x N/m of workspace)
+    pl.qc = env_int("CSA_PREFILL_CHUNK", 0);
+    if (pl.qc < 1) {
+        int sms = 0;
+        pl.qc = sm_count(&sms) == CSA_OK && sms > 0 ? 64 * (int64_t)sms : 9472;
+    }
     size_t off = 0;
     pl.off_queries = off;
     off += align256((size_t)pl.qc * sizeof(csa_query));
