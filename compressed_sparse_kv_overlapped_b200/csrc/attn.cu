@@ -26,6 +26,12 @@
 // loaders (cp.async for gathered rows with manual swizzle and zero-fill of masked slots; TMA for
 // full tiles of consecutive cache rows), warp 8 TMEM allocator + Q.K^T issuer, warp 9 P.V issuer.
 // Three key stages; every wait is bounded (kWaitLimitNs) and winds the CTA down on timeout.
+//
+// Persistent CTAs (direct outputs of more queries than SMs, the PERSIST instantiation): one CTA per
+// SM takes every G-th query of the launch; the key-stage ring, the S and P buffers and all barrier
+// phases run on from one query to the next (a running tile count), the CTA's queries are set up
+// once in shared memory, and the loader warps store each later query's Q (they own the same TMEM
+// lane quarters as the softmax warps) once the previous query's last Q.K^T is done (q_empty).
 #include <atomic>
 #include <cstring>
 
