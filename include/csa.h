@@ -314,7 +314,11 @@ typedef struct csa_prefill_args {
                                 normalization applies to the compress step (compress = 1) */
 } csa_prefill_args;
 
-/* a1, a2 full pass + a3..a7 for every query position in [q_begin, q_end) of one sequence. */
+/* a1, a2 full pass + a3..a7 for every query position in [q_begin, q_end) of one sequence.
+ * The positions run in chunks of 64 queries per multiprocessor of the current device (environment
+ * CSA_PREFILL_CHUNK overrides it); the workspace holds one chunk's score rows, about
+ * 4 B x chunk x floor(q_end / m), so query its size (CSA_OP_PREFILL) on the device that runs the call:
+ * a workspace smaller than the call's plan is rejected with CSA_ERR_ARG. */
 int hybrid_attn_prefill(const csa_prefill_args* args, void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* Workspace sizes.  `op` selects the call and `args` points to the arguments it describes:
